@@ -1,0 +1,283 @@
+/*
+ * Flint MoE block oracle, fp64 CPU.  TEST INFRASTRUCTURE ONLY (tests, smoke
+ * check, benchmark CPU baseline); see oracle.h for the definitions followed and
+ * the readings taken where the pages are silent.  Every sum is a plain
+ * left-to-right fp64 loop; threads only split independent output rows.
+ */
+#include "oracle.h"
+
+#include <math.h>
+#include <pthread.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------ threading */
+static int g_threads = 1;
+void oracle_set_threads(int n) { g_threads = n < 1 ? 1 : n; }
+int oracle_get_threads(void) { return g_threads; }
+
+typedef void (*range_fn)(void *ctx, int64_t i);
+typedef struct {
+  range_fn fn;
+  void *ctx;
+  int64_t lo, hi;
+} chunk;
+
+static void *run_chunk(void *p) {
+  chunk *c = (chunk *)p;
+  for (int64_t i = c->lo; i < c->hi; ++i) c->fn(c->ctx, i);
+  return NULL;
+}
+
+/* fn(ctx, i) for i in [0, n): contiguous chunks, one per thread. */
+static void par_for(int64_t n, range_fn fn, void *ctx) {
+  int t = g_threads;
+  if (t > n) t = (int)n;
+  if (t <= 1) {
+    for (int64_t i = 0; i < n; ++i) fn(ctx, i);
+    return;
+  }
+  pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * t);
+  chunk *ch = (chunk *)malloc(sizeof(chunk) * t);
+  for (int i = 0; i < t; ++i) {
+    ch[i].fn = fn;
+    ch[i].ctx = ctx;
+    ch[i].lo = n * i / t;
+    ch[i].hi = n * (i + 1) / t;
+    pthread_create(&th[i], NULL, run_chunk, &ch[i]);
+  }
+  for (int i = 0; i < t; ++i) pthread_join(th[i], NULL);
+  free(th);
+  free(ch);
+}
+
+/* ------------------------------------------------------------ numbers */
+double oracle_bf16_to_double(uint16_t v) {
+  uint32_t u = (uint32_t)v << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return (double)f;
+}
+
+uint16_t oracle_double_to_bf16(double v) {
+  /* v = m * 2^e with 0.5 <= |m| < 1; keep 8 significant bits of m, rounding
+   * to nearest with ties to even (nearbyint under the default mode). */
+  int e;
+  double m = frexp(v, &e);
+  double r = ldexp(nearbyint(m * 256.0), e - 8);
+  float f = (float)r; /* exact: r has at most 8 significant bits */
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  return (uint16_t)(u >> 16);
+}
+
+static float round_to_float(double v) { return (float)v; } /* IEEE nearest-even */
+
+/* The int4 code of element k of a packed row (low nibble = even element). */
+static int code_of(const uint8_t *row, int64_t k) {
+  uint8_t byte = row[k / 2];
+  int nib = (k % 2 == 0) ? (byte & 0x0F) : (byte >> 4);
+  return nib >= 8 ? nib - 16 : nib;
+}
+
+void oracle_unpack_int4(const uint8_t *q, int64_t n, int8_t *codes) {
+  for (int64_t k = 0; k < n; ++k) codes[k] = (int8_t)code_of(q, k);
+}
+
+/* Weight element (n, k) of a packed [N, K] matrix: code * its group's scale. */
+static double weight(const uint8_t *q, const uint16_t *s, int64_t K, int64_t n, int64_t k) {
+  const uint8_t *row = q + n * (K / 2);
+  double scale = oracle_bf16_to_double(s[n * (K / 128) + k / 128]);
+  return (double)code_of(row, k) * scale;
+}
+
+void oracle_dequant(const uint8_t *q, const uint16_t *s, int64_t N, int64_t K, double *W) {
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k) W[n * K + k] = weight(q, s, K, n, k);
+}
+
+/* sum_k W[n][k] x[k], left to right */
+static double row_dot(const uint8_t *q, const uint16_t *s, int64_t K, int64_t n, const double *x) {
+  double acc = 0.0;
+  for (int64_t k = 0; k < K; ++k) acc += weight(q, s, K, n, k) * x[k];
+  return acc;
+}
+
+static double sigmoid(double z) { return 1.0 / (1.0 + exp(-z)); }
+
+/* ------------------------------------------------------------ int4 GEMV */
+typedef struct {
+  const uint8_t *q;
+  const uint16_t *s;
+  int64_t N, K;
+  const double *x; /* [K] */
+  double *y;       /* [N] */
+} gemv_ctx;
+
+static void gemv_row(void *p, int64_t n) {
+  gemv_ctx *c = (gemv_ctx *)p;
+  c->y[n] = row_dot(c->q, c->s, c->K, n, c->x);
+}
+
+static void to_double(const uint16_t *x, int64_t n, double *out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = oracle_bf16_to_double(x[i]);
+}
+
+void oracle_int4_gemv(const uint8_t *q, const uint16_t *s, int64_t N, int64_t K,
+                      const uint16_t *x, int B, double *y, int32_t *argmax, double *gap) {
+  double *xd = (double *)malloc(sizeof(double) * K);
+  for (int b = 0; b < B; ++b) {
+    to_double(x + (int64_t)b * K, K, xd);
+    gemv_ctx c = {q, s, N, K, xd, y + (int64_t)b * N};
+    par_for(N, gemv_row, &c);
+    /* argmax, lowest index on ties; gap = best minus second best value */
+    const double *yb = y + (int64_t)b * N;
+    int64_t best = 0;
+    for (int64_t n = 1; n < N; ++n)
+      if (yb[n] > yb[best]) best = n;
+    double second = -INFINITY;
+    for (int64_t n = 0; n < N; ++n)
+      if (n != best && yb[n] > second) second = yb[n];
+    if (argmax) argmax[b] = (int32_t)best;
+    if (gap) gap[b] = yb[best] - second;
+  }
+  free(xd);
+}
+
+/* ------------------------------------------------------------ router */
+/* Selection order: larger biased score first, lower expert index on ties. */
+static int ranks_before(double bi, int i, double bj, int j) { return bi > bj || (bi == bj && i < j); }
+
+static void route_row(const oracle_layer *L, const double *x, double *z, double *sig,
+                      double *biased, int32_t *idx, double *w, double *gap) {
+  const int E = L->n_experts, H = L->hidden, k = L->top_k;
+  for (int e = 0; e < E; ++e) {
+    double acc = 0.0;
+    for (int h = 0; h < H; ++h)
+      acc += oracle_bf16_to_double(L->router_w[(int64_t)e * H + h]) * x[h];
+    z[e] = acc;
+    sig[e] = sigmoid(acc);
+    biased[e] = sig[e] + (double)L->router_b[e];
+  }
+  /* k picks by repeated scan (selection sort), then the (k+1)-th for the gap */
+  char *taken = (char *)calloc(E, 1);
+  int order[64];
+  int npick = k + 1 <= E ? k + 1 : E;
+  for (int p = 0; p < npick; ++p) {
+    int best = -1;
+    for (int e = 0; e < E; ++e) {
+      if (taken[e]) continue;
+      if (best < 0 || ranks_before(biased[e], e, biased[best], best)) best = e;
+    }
+    taken[best] = 1;
+    order[p] = best;
+  }
+  free(taken);
+  double ssum = 0.0;
+  for (int j = 0; j < k; ++j) ssum += sig[order[j]];
+  for (int j = 0; j < k; ++j) {
+    idx[j] = order[j];
+    w[j] = sig[order[j]] / ssum;
+  }
+  *gap = (k < E) ? biased[order[k - 1]] - biased[order[k]] : INFINITY;
+}
+
+void oracle_route(const oracle_layer *L, const uint16_t *x, int B, double *z, double *sig,
+                  double *biased, int32_t *idx, double *w, double *gap) {
+  const int E = L->n_experts, H = L->hidden, k = L->top_k;
+  double *xd = (double *)malloc(sizeof(double) * H);
+  double *zz = (double *)malloc(sizeof(double) * E * 3);
+  for (int b = 0; b < B; ++b) {
+    to_double(x + (int64_t)b * H, H, xd);
+    double g;
+    route_row(L, xd, zz, zz + E, zz + 2 * E, idx + b * k, w + b * k, &g);
+    if (z) memcpy(z + (int64_t)b * E, zz, sizeof(double) * E);
+    if (sig) memcpy(sig + (int64_t)b * E, zz + E, sizeof(double) * E);
+    if (biased) memcpy(biased + (int64_t)b * E, zz + 2 * E, sizeof(double) * E);
+    if (gap) gap[b] = g;
+  }
+  free(xd);
+  free(zz);
+}
+
+/* ------------------------------------------------------------ experts */
+void oracle_swiglu_expert(const uint8_t *q13, const uint16_t *s13, const uint8_t *q2,
+                          const uint16_t *s2, int hidden, int inter, const double *x, double *y) {
+  double *hmid = (double *)malloc(sizeof(double) * inter);
+  for (int r = 0; r < inter; ++r) {
+    double gate = row_dot(q13, s13, hidden, r, x);
+    double up = row_dot(q13, s13, hidden, inter + r, x);
+    hmid[r] = gate * sigmoid(gate) * up; /* silu(gate) * up */
+  }
+  for (int n = 0; n < hidden; ++n) y[n] = row_dot(q2, s2, inter, n, hmid);
+  free(hmid);
+}
+
+typedef struct {
+  const oracle_layer *L;
+  const uint16_t *x;
+  double *out;
+  int32_t *idx;
+  double *w, *gap;
+} moe_ctx;
+
+static void moe_row(void *p, int64_t b) {
+  moe_ctx *c = (moe_ctx *)p;
+  const oracle_layer *L = c->L;
+  const int E = L->n_experts, H = L->hidden, k = L->top_k, I = L->expert_i, Is = L->shared_i;
+  double *xd = (double *)malloc(sizeof(double) * H);
+  double *scr = (double *)malloc(sizeof(double) * 3 * E);
+  double *y = (double *)malloc(sizeof(double) * H);
+  int32_t idx[64];
+  double w[64], gap;
+  to_double(c->x + b * H, H, xd);
+  route_row(L, xd, scr, scr + E, scr + 2 * E, idx, w, &gap);
+  double *out = c->out + b * H;
+  for (int n = 0; n < H; ++n) out[n] = 0.0;
+  for (int j = 0; j < k; ++j) {
+    const int64_t e = idx[j];
+    oracle_swiglu_expert(L->w13_q + e * (2 * I) * (H / 2), L->w13_s + e * (2 * I) * (H / 128),
+                         L->w2_q + e * H * (I / 2), L->w2_s + e * H * (I / 128), H, I, xd, y);
+    for (int n = 0; n < H; ++n) out[n] += w[j] * y[n];
+  }
+  oracle_swiglu_expert(L->sh13_q, L->sh13_s, L->sh2_q, L->sh2_s, H, Is, xd, y);
+  for (int n = 0; n < H; ++n) out[n] += y[n];
+  if (c->idx) memcpy(c->idx + b * k, idx, sizeof(int32_t) * k);
+  if (c->w) memcpy(c->w + b * k, w, sizeof(double) * k);
+  if (c->gap) c->gap[b] = gap;
+  free(xd);
+  free(scr);
+  free(y);
+}
+
+void oracle_moe_layer(const oracle_layer *L, const uint16_t *x, int B, double *out,
+                      int32_t *idx, double *w, double *gap) {
+  moe_ctx c = {L, x, out, idx, w, gap};
+  par_for(B, moe_row, &c);
+}
+
+/* ------------------------------------------------------------ stack layer */
+void oracle_rmsnorm_bf16(const float *h, int B, int H, double eps, uint16_t *x) {
+  for (int b = 0; b < B; ++b) {
+    const float *hb = h + (int64_t)b * H;
+    double ss = 0.0;
+    for (int i = 0; i < H; ++i) ss += (double)hb[i] * (double)hb[i];
+    double inv = 1.0 / sqrt(ss / H + eps);
+    for (int i = 0; i < H; ++i) x[(int64_t)b * H + i] = oracle_double_to_bf16((double)hb[i] * inv);
+  }
+}
+
+void oracle_stack_layer(const oracle_layer *L, float *h, int B, double eps, int32_t *idx,
+                        double *w, double *gap) {
+  const int H = L->hidden;
+  uint16_t *x = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)B * H);
+  double *out = (double *)malloc(sizeof(double) * (size_t)B * H);
+  oracle_rmsnorm_bf16(h, B, H, eps, x);
+  oracle_moe_layer(L, x, B, out, idx, w, gap);
+  for (int64_t i = 0; i < (int64_t)B * H; ++i) {
+    double o = oracle_bf16_to_double(oracle_double_to_bf16(out[i])); /* block output is bf16 */
+    h[i] = round_to_float((double)h[i] + o);                         /* residual add in fp32 */
+  }
+  free(x);
+  free(out);
+}

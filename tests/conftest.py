@@ -1,0 +1,19 @@
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a B200 and the built CUDA library")
+    config.addinivalue_line("markers", "slow: large CPU oracle work")
+
+
+def pytest_collection_modifyitems(config, items):
+    # a GPU test on a box without a GPU is an error, not a skip, unless the run
+    # deselected GPU tests with -m "not gpu"
+    pass

@@ -1,0 +1,383 @@
+"""Pins of the fp64 oracle to facts fixed by the pages and by mathematics.
+
+Every test here runs on the CPU.  Each checks the oracle against something
+other than itself: values the pages print, hand-computed cases, brute force on
+tiny inputs, numpy's fp64 matmul, and invariants of the definition (routing
+weights sum to one, selection is invariant to a common bias shift, the block is
+linear in the down-projection scales).
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ------------------------------------------------------------------ helpers
+def pack_codes(codes: np.ndarray) -> np.ndarray:
+    """Independent packer: even element -> low nibble, two's complement."""
+    c = np.asarray(codes, np.int64).reshape(-1, 2)
+    lo = c[:, 0] & 0xF
+    hi = c[:, 1] & 0xF
+    return (lo | (hi << 4)).astype(np.uint8)
+
+
+def unpack_codes(q: np.ndarray) -> np.ndarray:
+    """Independent unpacker by arithmetic: ((nibble ^ 8) - 8)."""
+    q = np.asarray(q, np.int64)
+    lo = ((q & 0xF) ^ 8) - 8
+    hi = (((q >> 4) & 0xF) ^ 8) - 8
+    return np.stack([lo, hi], axis=-1).reshape(*q.shape[:-1], 2 * q.shape[-1])
+
+
+def dequant_np(q, s):
+    codes = unpack_codes(q).astype(np.float64)
+    sc = synth.bf16_to_f64(s)
+    return codes * np.repeat(sc, 128, axis=-1)
+
+
+def bf16(v):
+    return synth.bf16_bits(np.asarray(v, np.float64))
+
+
+def silu(v):
+    return v / (1.0 + math.exp(-v))
+
+
+def sigm(v):
+    return 1.0 / (1.0 + math.exp(-v))
+
+
+def tiny_layer(E=8, H=128, I=128, Is=128, seed=7, k=6):
+    dims = synth.Dims(hidden=H, n_experts=E, top_k=k, expert_i=I, shared_i=Is)
+    return synth.layer_host(seed, dims), dims
+
+
+# ------------------------------------------------------------------ format
+def test_unpack_every_byte_value():
+    q = np.arange(256, dtype=np.uint8)
+    codes = oracle.unpack_int4(q).reshape(256, 2)
+    for b in range(256):
+        lo, hi = b & 15, b >> 4
+        assert codes[b, 0] == (lo - 16 if lo >= 8 else lo)
+        assert codes[b, 1] == (hi - 16 if hi >= 8 else hi)
+
+
+def test_pack_unpack_round_trip_all_codes_both_positions():
+    codes = np.array([[a, b] for a in range(-8, 8) for b in range(-8, 8)], np.int8).reshape(-1)
+    q = pack_codes(codes)
+    assert np.array_equal(oracle.unpack_int4(q), codes)
+    assert np.array_equal(pack_codes(oracle.unpack_int4(q)), q)
+
+
+def test_dequant_is_code_times_group_scale_exactly():
+    rng = np.random.default_rng(0)
+    q = rng.integers(0, 256, size=(5, 192), dtype=np.uint8)  # K = 384: three groups
+    s = bf16(rng.uniform(1e-3, 5e-3, size=(5, 3)))
+    W = oracle.dequant(q, s)
+    assert np.array_equal(W, dequant_np(q, s))
+    # group boundary: element 127 uses scale 0, element 128 uses scale 1
+    c = unpack_codes(q)
+    sc = synth.bf16_to_f64(s)
+    assert W[2, 127] == c[2, 127] * sc[2, 0]
+    assert W[2, 128] == c[2, 128] * sc[2, 1]
+
+
+def test_bf16_rounding_ties_to_even():
+    f = oracle.bf16_from_double
+    assert f(1.0) == 0x3F80
+    assert f(1.0 + 2 ** -8) == 0x3F80            # tie -> even (mantissa 0)
+    assert f(1.0 + 3 * 2 ** -8) == 0x3F82        # tie -> even (mantissa 2)
+    assert f(1.0 + 2 ** -8 + 2 ** -30) == 0x3F81  # just above the tie
+    assert f(-2.0) == 0xC000
+    assert f(0.0) == 0x0000
+    rng = np.random.default_rng(1)
+    v = rng.normal(size=2000) * np.exp(rng.uniform(-20, 20, size=2000))
+    assert all(f(x) == int(b) for x, b in zip(v, synth.bf16_bits(v)))
+
+
+# ------------------------------------------------------------------ GEMV
+def test_int4_gemv_matches_numpy_fp64_matmul():
+    rng = np.random.default_rng(2)
+    N, K, B = 37, 384, 3
+    q = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    s = bf16(rng.uniform(1e-3, 5e-3, size=(N, K // 128)))
+    x = bf16(rng.normal(size=(B, K)))
+    y, am, gap = oracle.int4_gemv(q, s, x)
+    ref = synth.bf16_to_f64(x) @ dequant_np(q, s).T
+    np.testing.assert_allclose(y, ref, rtol=1e-13, atol=1e-15)
+    assert np.array_equal(am, ref.argmax(axis=1))
+    srt = np.sort(ref, axis=1)
+    np.testing.assert_allclose(gap, srt[:, -1] - srt[:, -2], rtol=1e-9, atol=1e-15)
+
+
+def test_int4_gemv_argmax_ties_go_to_lowest_index():
+    K = 128
+    q = np.zeros((6, K // 2), np.uint8)
+    # rows 1 and 4 identical and largest
+    q[1, 0] = q[4, 0] = 0x07   # code 7 at element 0
+    q[2, 0] = 0x03
+    s = np.full((6, 1), bf16(0.5), np.uint16)
+    x = np.zeros((1, K), np.uint16)
+    x[0, 0] = bf16(1.0)
+    y, am, gap = oracle.int4_gemv(q, s, x)
+    assert am[0] == 1 and gap[0] == 0.0
+    assert y[0, 1] == 3.5 and y[0, 2] == 1.5
+
+
+# ------------------------------------------------------------------ routing
+def brute_force_topk(b, k):
+    """The unique k-subset whose members all rank above every non-member
+    (rank: larger score, then lower index)."""
+    E = len(b)
+    found = []
+    for S in itertools.combinations(range(E), k):
+        inside = set(S)
+        ok = all((b[i] > b[j]) or (b[i] == b[j] and i < j)
+                 for i in inside for j in range(E) if j not in inside)
+        if ok:
+            found.append(S)
+    assert len(found) == 1
+    return set(found[0])
+
+
+@pytest.mark.parametrize("E", [8, 10, 12])
+def test_route_top6_matches_brute_force(E):
+    rng = np.random.default_rng(E)
+    H = 128
+    for trial in range(6):
+        t, dims = tiny_layer(E=E, H=H, seed=100 + trial)
+        if trial >= 3:   # plant exact ties in the biased score
+            t["router_w"][:] = 0
+            t["router_b"][:] = np.float32(0.0)
+            t["router_b"][[1, 3, 5, 7]] = np.float32(0.25)
+        L = oracle.Layer(t)
+        x = bf16(rng.normal(size=(3, H)))
+        r = oracle.route(L, x)
+        for row in range(3):
+            sel = brute_force_topk(list(r["biased"][row]), 6)
+            assert set(r["idx"][row]) == sel
+            # selection order: biased score descending, index ascending on ties
+            key = sorted(range(E), key=lambda e: (-r["biased"][row][e], e))
+            assert list(r["idx"][row]) == key[:6]
+            assert r["gap"][row] == r["biased"][row][key[5]] - r["biased"][row][key[6]]
+
+
+def test_route_scores_closed_form():
+    t, _ = tiny_layer()
+    L = oracle.Layer(t)
+    x = bf16(np.random.default_rng(3).normal(size=(2, 128)))
+    r = oracle.route(L, x)
+    Wr = synth.bf16_to_f64(t["router_w"])
+    z = synth.bf16_to_f64(x) @ Wr.T
+    np.testing.assert_allclose(r["z"], z, rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(r["sig"], 1 / (1 + np.exp(-z)), rtol=1e-14)
+    np.testing.assert_allclose(r["biased"], r["sig"] + t["router_b"].astype(np.float64), rtol=1e-14)
+
+
+def test_route_weights_positive_and_sum_to_one_full_size():
+    L = oracle.Layer(synth.layer_host(0, with_codes=False) | {
+        k: np.zeros(1, np.uint8) for k in ("w13_q", "w2_q", "sh13_q", "sh2_q")})
+    x = synth.decode_x([0, 1, 2, 3, 4])
+    r = oracle.route(L, x)
+    assert np.all(r["w"] > 0)
+    np.testing.assert_allclose(r["w"].sum(axis=1), 1.0, rtol=0, atol=1e-15)
+    # weights are the unbiased scores of the chosen experts, renormalized
+    for row in range(5):
+        s = r["sig"][row][r["idx"][row]]
+        np.testing.assert_allclose(r["w"][row], s / s.sum(), rtol=1e-15)
+
+
+def test_route_invariant_to_common_bias_shift_and_bias_zero_is_top_z():
+    t, _ = tiny_layer(E=12, seed=9)
+    x = bf16(np.random.default_rng(4).normal(size=(4, 128)))
+    r0 = oracle.route(oracle.Layer(t), x)
+    t2 = dict(t)
+    t2["router_b"] = (t["router_b"] + np.float32(0.5)).astype(np.float32)  # exact in fp32 here
+    r1 = oracle.route(oracle.Layer(t2), x)
+    assert np.array_equal(r0["idx"], r1["idx"])
+    np.testing.assert_array_equal(r0["w"], r1["w"])
+    t3 = dict(t)
+    t3["router_b"] = np.zeros_like(t["router_b"])
+    r3 = oracle.route(oracle.Layer(t3), x)
+    for row in range(4):   # sigmoid is monotone: top-6 of sigmoid(z) is top-6 of z
+        assert list(r3["idx"][row]) == list(np.argsort(-r3["z"][row], kind="stable")[:6])
+
+
+# ------------------------------------------------------------------ hand case
+def test_hand_computed_one_token_eight_experts():
+    """1 token, 8 experts, H = I = Is = 128.  Every weight is a small integer
+    code times a power-of-two scale; the expected output is written out below
+    from the definition: z = W_r x, s = sigmoid(z), selection by s + bias,
+    w = s / sum(s) over the chosen six, expert = W2 (silu(W1 x) * W3 x),
+    out = sum_j w_j y_j + y_shared."""
+    E, H, I = 8, 128, 128
+    t, _ = tiny_layer(E=E, H=H, I=I, Is=I)
+    for k in ("w13_q", "w2_q", "sh13_q", "sh2_q"):
+        t[k] = np.zeros_like(t[k])
+    for k in ("w13_s", "w2_s", "sh13_s", "sh2_s"):
+        t[k] = np.full_like(t[k], bf16(1.0))
+    # router: z_e = Wr[e,0]*1 + Wr[e,1]*0.5
+    wr0 = [0.0, 0.5, -0.5, 1.0, -1.0, 0.25, 2.0, -2.0]
+    wr1 = [0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 1.0]   # z_7 = -2 + 0.5 = -1.5
+    t["router_w"] = np.zeros((E, H), np.uint16)
+    t["router_w"][:, 0] = bf16(wr0)
+    t["router_w"][:, 1] = bf16(wr1)
+    t["router_w"][:, 5] = bf16(3.0)   # multiplies x[5] = 0
+    t["router_b"] = np.array([0, 0, 0, -1.0, 0, 0, 0, 1.0], np.float32)
+    x = np.zeros((1, H), np.uint16)
+    x[0, 0] = bf16(1.0)
+    x[0, 1] = bf16(0.5)
+
+    g0 = [1, 2, -1, 3, 0, -2, 1, 2]
+    g1 = [2, 0, 1, -1, 1, 2, -2, 2]
+    u0 = [3, -1, 2, 1, 1, 1, -3, 2]
+    d = [[1, -2, 3], [2, 1, 0], [-1, -1, 1], [4, 0, -4], [1, 1, 1], [0, 2, -2], [3, -3, 1], [-2, 1, 2]]
+
+    def set_expert(q13, s13, q2, s2, gg0, gg1, uu0, dd):
+        q13[0, 0] = pack_codes([gg0, gg1])[0]     # gate row 0, elements 0, 1
+        s13[0, 0] = bf16(0.25)
+        q13[I, 0] = pack_codes([uu0, 0])[0]        # up row 0 (row I), element 0
+        s13[I, 0] = bf16(0.5)
+        for n in range(3):                          # down rows 0..2, column 0
+            q2[n, 0] = pack_codes([dd[n], 0])[0]
+            s2[n, 0] = bf16(0.125)
+        q2[0, 0] |= pack_codes([0, 5])[0]           # W2[0,1]: multiplies h_1 = 0
+        q2[0, 1] = pack_codes([-3, 0])[0]           # W2[0,2]: multiplies h_2 = 0
+
+    for e in range(E):
+        set_expert(t["w13_q"][e], t["w13_s"][e], t["w2_q"][e], t["w2_s"][e], g0[e], g1[e], u0[e], d[e])
+    set_expert(t["sh13_q"], t["sh13_s"], t["sh2_q"], t["sh2_s"], 2, -1, 1, [1, 0, -1])
+
+    out, idx, w, gap = oracle.moe_layer(oracle.Layer(t), x)
+
+    z = [wr0[e] + 0.5 * wr1[e] for e in range(E)]
+    s = [sigm(v) for v in z]
+    b = [s[e] + [0, 0, 0, -1.0, 0, 0, 0, 1.0][e] for e in range(E)]
+    # by hand: b = [.5, .6225, .3775, -.2689, .2689, .5622, .8808, 1.1824]
+    assert list(idx[0]) == [7, 6, 1, 5, 0, 2]
+    assert gap[0] == pytest.approx(b[2] - b[4], abs=1e-15)
+    ssum = sum(s[e] for e in (7, 6, 1, 5, 0, 2))
+    expect = np.zeros(H)
+    for e in (7, 6, 1, 5, 0, 2):
+        g = (g0[e] * 1.0 + g1[e] * 0.5) * 0.25
+        u = u0[e] * 0.5
+        h0 = silu(g) * u
+        for n in range(3):
+            expect[n] += (s[e] / ssum) * d[e][n] * 0.125 * h0
+    hs = silu((2 * 1.0 - 1 * 0.5) * 0.25) * (1 * 0.5)
+    expect[0] += 1 * 0.125 * hs
+    expect[2] += -1 * 0.125 * hs
+    np.testing.assert_allclose(out[0], expect, rtol=1e-14, atol=1e-17)
+    np.testing.assert_allclose(w[0], [s[e] / ssum for e in (7, 6, 1, 5, 0, 2)], rtol=1e-15)
+
+
+# ------------------------------------------------------------------ layer invariants
+def numpy_expert(q13, s13, q2, s2, x):
+    W13 = dequant_np(q13, s13)
+    I = W13.shape[0] // 2
+    g, u = W13[:I] @ x, W13[I:] @ x
+    return dequant_np(q2, s2) @ (g / (1 + np.exp(-g)) * u)
+
+
+def test_expert_matches_numpy_definition():
+    t, _ = tiny_layer(E=4, H=256, I=128, Is=256, seed=11)
+    x = synth.bf16_to_f64(bf16(np.random.default_rng(5).normal(size=256)))
+    for e in range(4):
+        y = oracle.swiglu_expert(t["w13_q"][e], t["w13_s"][e], t["w2_q"][e], t["w2_s"][e], x)
+        np.testing.assert_allclose(y, numpy_expert(t["w13_q"][e], t["w13_s"][e], t["w2_q"][e],
+                                                   t["w2_s"][e], x), rtol=1e-11, atol=1e-14)
+
+
+def test_identical_experts_make_routing_irrelevant():
+    t, _ = tiny_layer(E=10, H=256, I=128, Is=128, seed=12)
+    for k in ("w13_q", "w13_s", "w2_q", "w2_s"):
+        t[k] = np.ascontiguousarray(np.broadcast_to(t[k][3], t[k].shape))
+    x = bf16(np.random.default_rng(6).normal(size=(3, 256)))
+    out, idx, w, gap = oracle.moe_layer(oracle.Layer(t), x)
+    for row in range(3):
+        xd = synth.bf16_to_f64(x[row])
+        expect = numpy_expert(t["w13_q"][3], t["w13_s"][3], t["w2_q"][3], t["w2_s"][3], xd) + \
+            numpy_expert(t["sh13_q"], t["sh13_s"], t["sh2_q"], t["sh2_s"], xd)
+        np.testing.assert_allclose(out[row], expect, rtol=1e-11, atol=1e-13)
+
+
+def test_doubling_down_scales_doubles_output_exactly():
+    t, _ = tiny_layer(E=10, H=256, I=128, Is=256, seed=13)
+    x = bf16(np.random.default_rng(7).normal(size=(2, 256)))
+    out0, idx0, _, _ = oracle.moe_layer(oracle.Layer(t), x)
+    t2 = dict(t)
+    for k in ("w2_s", "sh2_s"):
+        t2[k] = (t[k].astype(np.uint32) + 0x80).astype(np.uint16)   # exponent + 1
+    out1, idx1, _, _ = oracle.moe_layer(oracle.Layer(t2), x)
+    assert np.array_equal(idx0, idx1)
+    assert np.array_equal(out1, 2 * out0)
+
+
+def test_layer_matches_numpy_definition_random():
+    t, _ = tiny_layer(E=16, H=256, I=128, Is=256, seed=14)
+    x = bf16(np.random.default_rng(8).normal(size=(3, 256)))
+    out, idx, w, gap = oracle.moe_layer(oracle.Layer(t), x)
+    Wr = synth.bf16_to_f64(t["router_w"])
+    for row in range(3):
+        xd = synth.bf16_to_f64(x[row])
+        z = Wr @ xd
+        s = 1 / (1 + np.exp(-z))
+        b = s + t["router_b"].astype(np.float64)
+        sel = np.lexsort((np.arange(16), -b))[:6]
+        assert list(sel) == list(idx[row])
+        expect = sum(s[e] / s[sel].sum() * numpy_expert(t["w13_q"][e], t["w13_s"][e], t["w2_q"][e],
+                                                         t["w2_s"][e], xd) for e in sel)
+        expect = expect + numpy_expert(t["sh13_q"], t["sh13_s"], t["sh2_q"], t["sh2_s"], xd)
+        np.testing.assert_allclose(out[row], expect, rtol=1e-10, atol=1e-13)
+
+
+# ------------------------------------------------------------------ stack
+def test_rmsnorm_closed_forms():
+    h = np.zeros((2, 4), np.float32)
+    h[0] = [3.0, 4.0, 0.0, 0.0]           # mean square 25/4
+    h[1] = [-2.0, -2.0, -2.0, -2.0]       # mean square 4
+    x = synth.bf16_to_f64(oracle.rmsnorm_bf16(h, eps=1e-6))
+    r0 = 1 / math.sqrt(25 / 4 + 1e-6)
+    assert x[0, 0] == synth.bf16_to_f64(bf16(3 * r0)) and x[0, 2] == 0.0
+    assert x[0, 1] == synth.bf16_to_f64(bf16(4 * r0))
+    assert np.all(x[1] == -1.0)           # -2/sqrt(4 + 1e-6) rounds to -1 in bf16
+
+
+def test_stack_layer_is_norm_then_block_then_fp32_residual():
+    t, _ = tiny_layer(E=12, H=256, I=128, Is=128, seed=15)
+    L = oracle.Layer(t)
+    h = (np.random.default_rng(9).normal(size=(2, 256)) * 3).astype(np.float32)
+    hn, idx, w, gap = oracle.stack_layer(L, h, eps=1e-6)
+    x = oracle.rmsnorm_bf16(h, 1e-6)
+    out, idx2, _, _ = oracle.moe_layer(L, x)
+    assert np.array_equal(idx, idx2)
+    expect = (h.astype(np.float64) + synth.bf16_to_f64(bf16(out))).astype(np.float32)
+    assert np.array_equal(hn, expect)
+
+
+# ------------------------------------------------------------------ the pages' counts
+def test_parameter_counts_match_the_pages():
+    d = synth.FLINT
+    golden = {}
+    for line in open(os.path.join(GOLDEN, "flint_param_counts.txt")):
+        if line.strip() and not line.startswith("#"):
+            name, value = line.split()[:2]
+            golden[name] = int(value)
+    expert = 3 * d.hidden * d.expert_i
+    # shapes of the packed tensors, in elements (two per byte)
+    assert 2 * np.prod(d.w13_q()[1:]) + 2 * np.prod(d.w2_q()[1:]) == expert
+    assert round(6 * expert * 47 / 1e5) * 1e5 == golden["routed_active_47_layers"]
+    assert round(3 * d.hidden * d.shared_i * 47 / 1e5) * 1e5 == golden["shared_47_layers"]
+    assert 2 * np.prod(d.sh13_q()) + 2 * np.prod(d.sh2_q()) == 3 * d.hidden * d.shared_i
+    assert round(d.n_experts * d.hidden * 47 / 1e5) * 1e5 == golden["routers_47_layers"]
+    assert synth.VOCAB * synth.HIDDEN == golden["lm_head"]
+    assert round(expert / 1e5) * 1e5 == golden["routed_expert"]
+    assert round(256 * expert / 1e6) * 1e6 == golden["routed_layer"]
+    assert round(47 * 256 * expert / 1e8) * 1e8 == golden["routed_all_layers"]
