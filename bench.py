@@ -1,0 +1,425 @@
+"""Benchmark of the Flint int4 MoE block decode on B200.
+
+Step: one decode token-step of a batch of B rows through the stack of 47
+Flint MoE layers (RMSNorm -> MoE block -> fp32 residual add per layer), each
+layer with its own seeded int4 weights (19.7 GB resident, so no layer's
+weights stay in the 126 MB L2 between its uses), fresh seeded input rows per
+step.  The reported value is device time per MoE layer (us/layer, lower is
+better); the MoE-stack tokens/s, the batch-1 figure and the 150,144 x 2,048
+int4 head GEMV are reported beside it.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--batch B] [--impl flint|reference]
+
+N > 1 runs N independent replicas (the path is not sharded), one process per
+GPU under torchrun; the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+N_LAYERS = synth.N_MOE_LAYERS
+H = synth.HIDDEN
+LAYER_FIXED_BYTES = 256 * 2048 * 2 + 256 * 4 + 2048 * (1024 + 32) + 2048 * (512 + 16)
+EXPERT_BYTES = 1024 * (1024 + 32) + 2048 * (256 + 8)
+HEAD_BYTES = synth.VOCAB * (1024 + 32)
+METRIC = "us per MoE-layer decode (B=4), fraction of HBM roofline"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--batch", type=int, default=4)
+    p.add_argument("--impl", default="flint", choices=["flint", "reference"])
+    p.add_argument("--layers", type=int, default=N_LAYERS)
+    p.add_argument("--no-head", action="store_true")
+    p.add_argument("--no-cpu", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    Q = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap,utilization.gpu")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "20"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = []
+        for ts, line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                rows.append((ts, float(parts[0]), float(parts[1]), parts[2:6], float(parts[6])))
+            except ValueError:
+                continue
+        inside = [r for r in rows if t0 <= r[0] <= t1] or rows
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in inside for i, v in enumerate(r[3]) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[1] for r in inside),
+                "sm_max_mhz": max(r[2] for r in inside), "reasons": reasons,
+                "samples": len(inside)}
+
+
+# ------------------------------------------------------------------ workload
+def step_inputs(steps: int, B: int) -> np.ndarray:
+    """Fresh residual rows for each step: seed 10000 + 4*step + row."""
+    return np.stack([synth.residual_h([10000 + 4 * s + r for r in range(B)]) for s in range(steps)])
+
+
+def build_layers(n: int, device):
+    import int4_expert_routing_b200 as F
+    layers, structs = [], []
+    for l in range(n):
+        d = synth.layer_device(l, device)
+        layers.append(d)
+        structs.append(F.make_layer(d))
+    return layers, structs
+
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, v: float) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_baseline(B: int, n_samples: int = 6):
+    """The fp64 oracle on the host cores: n_samples stack-layer calls at batch
+    B (layer l, rows of step l), timed; reported as us per MoE layer."""
+    import oracle
+    threads = os.cpu_count() or 1
+    oracle.set_threads(threads)
+    hs = step_inputs(n_samples, B)
+    t = 0.0
+    for i in range(n_samples):
+        L = oracle.Layer(synth.layer_host(i % N_LAYERS))
+        t0 = time.perf_counter()
+        oracle.stack_layer(L, hs[i])
+        t += time.perf_counter() - t0
+    return {"value": t / n_samples * 1e6, "unit": "us/layer", "cores": min(threads, B),
+            "kind": "oracle",
+            "sample": f"{n_samples} stack-layer calls at batch {B} (layers 0..{n_samples - 1}, "
+                      f"fp64 oracle threaded over the {B} rows)"}
+
+
+def run_reference(args):
+    """Reference arm: the fp64 CPU oracle, each step one stack-layer call for
+    ONE row (layer = step mod 47); value scaled to us per layer at batch B."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1 and rank != 0:
+        return
+    import oracle
+    oracle.set_threads(1)
+    B = args.batch
+    hs = step_inputs(args.steps + args.warmup, 1)
+    cache = {}
+
+    def layer(l):
+        if l not in cache:
+            cache.clear()
+            cache[l] = oracle.Layer(synth.layer_host(l))
+        return cache[l]
+
+    for s in range(args.warmup):
+        oracle.stack_layer(layer(s % args.layers), hs[s])
+    t = 0.0
+    for s in range(args.warmup, args.warmup + args.steps):
+        L = layer(s % args.layers)
+        t0 = time.perf_counter()
+        oracle.stack_layer(L, hs[s])
+        t += time.perf_counter() - t0
+    per_layer_us = t / args.steps * 1e6 * B
+    line = {"impl": "reference", "metric": METRIC, "value": per_layer_us, "unit": "us/layer",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": per_layer_us * args.layers / 1e3, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"flint moe decode, 47-layer stack, batch {B}",
+                       "batch": B, "layers": args.layers},
+            "cpu_baseline": {"value": per_layer_us, "unit": "us/layer", "cores": 1,
+                             "kind": "oracle",
+                             "sample": f"{args.steps} stack-layer calls of one row each, "
+                                       f"scaled x{B} to a batch-{B} layer"},
+            "e2e": {"value": per_layer_us, "unit": "us/layer", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    import torch
+    import int4_expert_routing_b200 as F
+    F.build()
+    world, rank, local = dist_setup(args)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    B, nl = args.batch, args.layers
+    hbm, peak_kind = peaks()
+
+    layers, structs = build_layers(nl, dev)
+    total = args.steps + args.warmup
+    h_host = torch.from_numpy(step_inputs(total, B)).pin_memory()          # [S][B][H]
+    h_dev = h_host.to(dev)
+    h_work = torch.empty((B, H), dtype=torch.float32, device=dev)
+    nb = F.flint_workspace_bytes(F.FLINT_OP_DECODE, B)
+    ws = torch.zeros(nb, dtype=torch.uint8, device=dev)
+    F.flint_workspace_init(ws, nb)
+    stream = torch.cuda.Stream(dev)
+
+    def one_step(s, st):
+        h_work.copy_(h_dev[s], non_blocking=True)
+        for l in range(nl):
+            F.flint_moe_decode_residual(structs[l], h_work, B, None, None, ws, nb, stream=st)
+
+    # routing of every (step, layer), outside the timed region, for the bytes count
+    idx = torch.empty((nl, B, 6), dtype=torch.int32, device=dev)
+    distinct = []
+    with torch.cuda.stream(stream):
+        for s in range(args.warmup, total):
+            h_work.copy_(h_dev[s])
+            for l in range(nl):
+                F.flint_moe_decode_residual(structs[l], h_work, B, idx[l], None, ws, nb,
+                                            stream=stream)
+            distinct.append(idx.cpu().numpy())
+    stream.synchronize()
+    U = float(np.mean([len(set(a[l].ravel().tolist())) for a in distinct for l in range(nl)]))
+    bytes_per_layer = LAYER_FIXED_BYTES + U * EXPERT_BYTES + 2 * B * H * 4
+
+    # capture the K timed steps (and warmup steps) as CUDA graphs
+    with torch.cuda.stream(stream):
+        for s in range(args.warmup):
+            one_step(s, stream)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for s in range(args.warmup, total):
+            one_step(s, stream)
+    gw = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gw, stream=stream):
+        for s in range(min(args.warmup, total)):
+            one_step(s, stream)
+    for _ in range(3):
+        gw.replay()
+    stream.synchronize()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    # soak: replay the timed graph for ~1 s so the clock record covers a loaded GPU
+    t_soak = time.time()
+    while time.time() - t_soak < 1.0:
+        g.replay()
+        stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    tw0 = time.time()
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    e1.synchronize()
+    tw1 = time.time()
+    barrier(world)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(world, e0.elapsed_time(e1))
+    clocks = sampler.summary(tw0 - 0.5, tw1 + 0.5)
+
+    layers_done = args.steps * nl * world
+    us_per_layer = ms * 1e3 / (args.steps * nl) / world
+    achieved = bytes_per_layer / (ms * 1e-3 / (args.steps * nl)) / 1e9
+
+    # ---- batch 1, same stack (context figure)
+    extra = {}
+    if B != 1:
+        h1 = torch.empty((1, H), dtype=torch.float32, device=dev)
+        nb1 = F.flint_workspace_bytes(F.FLINT_OP_DECODE, 1)
+        ws1 = torch.zeros(nb1, dtype=torch.uint8, device=dev)
+        F.flint_workspace_init(ws1, nb1)
+        g1 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g1, stream=stream):
+            for s in range(args.warmup, total):
+                h1.copy_(h_dev[s, :1], non_blocking=True)
+                for l in range(nl):
+                    F.flint_moe_decode_residual(structs[l], h1, 1, None, None, ws1, nb1,
+                                                stream=stream)
+        g1.replay()
+        stream.synchronize()
+        e0.record(stream)
+        g1.replay()
+        e1.record(stream)
+        e1.synchronize()
+        ms1 = e0.elapsed_time(e1)
+        us1 = ms1 * 1e3 / (args.steps * nl)
+        b1_bytes = LAYER_FIXED_BYTES + 6 * EXPERT_BYTES + 2 * H * 4
+        extra["batch1"] = {"us_per_layer": us1, "stack_tokens_per_s": 1e6 / (us1 * nl),
+                           "roofline_frac": b1_bytes / (us1 * 1e-6) / 1e9 / hbm,
+                           "bytes_per_layer": b1_bytes}
+
+    # ---- e2e through the C ABI with host buffers: H2D of the step's rows,
+    # 47 layer calls, D2H of the result rows, every step
+    out_host = torch.empty((args.steps, B, H), dtype=torch.float32).pin_memory()
+    ge = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(ge, stream=stream):
+        for i, s in enumerate(range(args.warmup, total)):
+            h_work.copy_(h_host[s], non_blocking=True)
+            for l in range(nl):
+                F.flint_moe_decode_residual(structs[l], h_work, B, None, None, ws, nb,
+                                            stream=stream)
+            out_host[i].copy_(h_work, non_blocking=True)
+    ge.replay()
+    stream.synchronize()
+    barrier(world)
+    e0.record(stream)
+    ge.replay()
+    e1.record(stream)
+    e1.synchronize()
+    barrier(world)
+    mse = max_over_ranks(world, e0.elapsed_time(e1))
+    e2e_us = mse * 1e3 / (args.steps * nl) / world
+
+    # ---- output head int4 GEMV (B = 1 and the bench batch), context
+    if not args.no_head and rank == 0:
+        hq = synth.random_bytes_torch(0, synth.T_HEAD_Q, synth.VOCAB * H // 2, dev).view(
+            synth.VOCAB, H // 2)
+        hs_ = synth.to_device({"s": synth.head_host(with_codes=False)["s"]}, dev)["s"]
+        for hb in sorted({1, min(B, 8)}):
+            xh = synth.to_device({"x": synth.head_x(list(range(hb)))}, dev)["x"]
+            y = torch.empty((hb, synth.VOCAB), dtype=torch.float32, device=dev)
+            am = torch.empty(hb, dtype=torch.int32, device=dev)
+            nbh = F.flint_gemv_workspace_bytes(synth.VOCAB, hb)
+            wsh = torch.zeros(nbh, dtype=torch.uint8, device=dev)
+            F.flint_workspace_init(wsh, nbh)
+            flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+            times = []
+            for it in range(23):
+                flush.zero_()                  # evict the head from L2 between launches
+                e0.record(stream)
+                F.flint_int4_gemv(hq, hs_, synth.VOCAB, H, xh, hb, y, am, wsh, nbh,
+                                  stream=stream)
+                e1.record(stream)
+                e1.synchronize()
+                if it >= 3:
+                    times.append(e0.elapsed_time(e1) * 1e3)
+            us = statistics.median(times)
+            extra[f"head_gemv_b{hb}"] = {"us": us, "GBps": HEAD_BYTES / (us * 1e-6) / 1e9,
+                                        "roofline_frac": HEAD_BYTES / (us * 1e-6) / 1e9 / hbm}
+    sampler.stop()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(B)
+
+    line = {
+        "metric": METRIC, "value": us_per_layer, "unit": "us/layer", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms / args.steps, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 activations x int4 weights, fp32 accumulate",
+        "data": "synthetic (seeded; weights as the workload recipe)",
+        "config": {"workload": f"flint moe decode, 47-layer stack (RMSNorm->MoE->residual), "
+                               f"batch {B}, fresh rows per step",
+                   "batch": B, "layers": nl, "hidden": H, "experts": 256, "top_k": 6,
+                   "l2": "inputs larger than L2: 47 layers x 420 MB of int4 weights rotate",
+                   "stack_tokens_per_s": B * 1e6 / (us_per_layer * nl * world) * world,
+                   "mean_distinct_experts": U},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None,
+                     "kernel": "decode layer (3 PDL-chained kernels)",
+                     "peak_kind": peak_kind, "bytes_per_layer": bytes_per_layer},
+        "e2e": {"value": e2e_us, "unit": "us/layer", "h2d_bytes_per_step": B * H * 4,
+                "d2h_bytes_per_step": B * H * 4},
+        "gpu_launches": 3 * nl * args.steps,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+        "extra": extra,
+    }
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        del g, gw, ge
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,181 @@
+/*
+ * flint.h: C ABI of the Flint int4 MoE block library for NVIDIA B200 (sm_100a).
+ *
+ * The block is the per-token mixture-of-experts layer of Flint, as described
+ * on "How to Run Flint Locally", section "The architecture, from config.json"
+ * (hidden 2,048; 256 routed experts of size 512 with 6 chosen per token by a
+ * sigmoid router with normalized top-k; one shared expert of size 1,024 that
+ * runs for every token) and on TandemLLM "21 Flint", section 21.1 "The model"
+ * (experts routed by sigmoid score with a bias, SwiGLU experts).  The same
+ * int4 GEMV serves the 150,144 x 2,048 output head ("How to Run Flint
+ * Locally", section "One decode step in bytes": the head is read in full for
+ * every token and was quantized to 4 bits).
+ *
+ * Conventions for every entry point:
+ *  - All tensor arguments are DEVICE pointers to memory the caller owns; the
+ *    library never allocates, frees or keeps them past the call.  Every
+ *    pointer must be 16-byte aligned.  Layouts are dense, row-major.
+ *  - bf16 values are passed as their 16-bit patterns (uint16_t).
+ *  - Packed int4 matrix [N, K]: q is N rows of K/2 bytes; byte j of a row
+ *    holds element 2j in its low nibble and element 2j+1 in its high nibble,
+ *    each a two's-complement code in [-8, 7].  s is [N, K/128] bf16: the scale
+ *    of elements 128g .. 128g+127 of the row.  Weight = code * scale.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
+ *    asynchronous; errors in arguments are reported before anything is
+ *    launched, by the return code.  Device-side errors are recorded in the
+ *    workspace's status word and read with flint_read_status.
+ *  - Workspace: `ws` is caller-owned device scratch of at least
+ *    flint_workspace_bytes(op, n) bytes.  Calls that share a workspace must
+ *    be ordered on one stream.  The first use of a workspace must be preceded
+ *    by flint_workspace_init (which zeroes its counters and status word).
+ *  - Return value: FLINT_OK or a FLINT_E* code; never aborts the process.
+ */
+#ifndef FLINT_H
+#define FLINT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FLINT_API __attribute__((visibility("default")))
+#else
+#define FLINT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FLINT_HIDDEN 2048
+#define FLINT_EXPERTS 256
+#define FLINT_TOPK 6
+#define FLINT_EXPERT_I 512
+#define FLINT_SHARED_I 1024
+#define FLINT_GROUP 128
+#define FLINT_MAX_DECODE_B 8
+#define FLINT_RMS_EPS 1e-6
+
+enum {
+  FLINT_OK = 0,
+  FLINT_EINVAL = 1,   /* bad pointer, alignment, size or workspace */
+  FLINT_ECUDA = 2,    /* a CUDA runtime call or launch failed */
+  FLINT_ETIMEOUT = 3, /* a bounded device-side wait gave up (status word) */
+  FLINT_EDEVICE = 4   /* a device-side check failed (status word) */
+};
+
+/* Workspace kinds for flint_workspace_bytes. */
+enum { FLINT_OP_ROUTE = 0, FLINT_OP_DECODE = 1, FLINT_OP_PREFILL = 2, FLINT_OP_GEMV = 3 };
+
+/*
+ * One MoE layer's weights (all device pointers, read only).
+ *  router_w  bf16 [256][2048]        z = router_w . x
+ *  router_b  fp32 [256]              selection bias
+ *  w13_q/s   packed [256][1024][2048]: per expert, rows 0..511 are the gate
+ *            projection W1, rows 512..1023 the up projection W3
+ *  w2_q/s    packed [256][2048][512]: per expert, the down projection W2
+ *  sh13_q/s  packed [2048][2048]: shared expert, rows 0..1023 gate, 1024..2047 up
+ *  sh2_q/s   packed [2048][1024]: shared expert down projection
+ * Expert e's block starts at e * rows * row_bytes; the struct holds only base
+ * pointers.
+ */
+typedef struct {
+  const uint16_t *router_w;
+  const float *router_b;
+  const uint8_t *w13_q;
+  const uint16_t *w13_s;
+  const uint8_t *w2_q;
+  const uint16_t *w2_s;
+  const uint8_t *sh13_q;
+  const uint16_t *sh13_s;
+  const uint8_t *sh2_q;
+  const uint16_t *sh2_s;
+} flint_moe_layer;
+
+/* Library version (major*10000 + minor*100 + patch). */
+FLINT_API int flint_version(void);
+
+/* Human-readable name of a FLINT_* code (static string). */
+FLINT_API const char *flint_strerror(int code);
+
+/* Bytes of workspace `op` needs for n rows (B for decode and gemv, T for
+ * route and prefill); for FLINT_OP_GEMV, n = B and the size also depends on
+ * N via flint_gemv_workspace_bytes.  Returns 0 for an unsupported n. */
+FLINT_API size_t flint_workspace_bytes(int op, int n);
+FLINT_API size_t flint_gemv_workspace_bytes(int N, int B);
+
+/* Zero a workspace's counters and status word (async on `stream`). */
+FLINT_API int flint_workspace_init(void *ws, size_t ws_bytes, void *stream);
+
+/* Copy the workspace's device status word to *status (synchronizes `stream`).
+ * *status is FLINT_OK unless a device-side check or bounded wait failed. */
+FLINT_API int flint_read_status(const void *ws, int *status, void *stream);
+
+/*
+ * Router for B rows ("How to Run Flint Locally", section "The architecture,
+ * from config.json": sigmoid router over 256 experts, top 6 kept, weights
+ * normalized; TandemLLM "21 Flint" section 21.1: selection by sigmoid score
+ * with a bias).
+ *   z = router_w . x  (bf16 products, accumulated in fp64, rounded to fp32)
+ *   s = sigmoid(z) (fp32);  b = s + router_b (fp32)
+ *   idx[r][0..5] = the 6 largest b, largest first; equal b -> lower index
+ *   w[r][j] = s[idx[r][j]] / sum_j s[idx[r][j]]   (fp32)
+ *   x    bf16 [B][2048];  idx int32 [B][6];  w fp32 [B][6];  B >= 1
+ *   ws   workspace of flint_workspace_bytes(FLINT_OP_ROUTE, B)
+ */
+FLINT_API int flint_moe_route(const flint_moe_layer *layer, const uint16_t *x, int B, int32_t *idx,
+                    float *w, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Decode step of the MoE block for B in [1, 8] rows:
+ *   out[r] = sum_j w[r][j] * W2_e (silu(W1_e x) * (W3_e x))  (j over the 6
+ *            chosen experts e, in ascending expert order)
+ *          + W2_sh (silu(W1_sh x) * (W3_sh x))               (shared expert)
+ * with routing as in flint_moe_route.  fp32 accumulation throughout, fp32
+ * SwiGLU intermediates (they can exceed the fp16 range: TandemLLM "21 Flint",
+ * section 21.2 "The packs"), bf16 output.  Each output row is bit-identical
+ * to running that row alone (batch invariance, as the Strix Halo engine
+ * states in "Flint preview", section "What is in it").
+ *   x   bf16 [B][2048];  out bf16 [B][2048] (may not alias x)
+ *   ws  workspace of flint_workspace_bytes(FLINT_OP_DECODE, B)
+ */
+FLINT_API int flint_moe_decode(const flint_moe_layer *layer, const uint16_t *x, int B, uint16_t *out,
+                     void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * One stacked decode layer on an fp32 residual stream h [B][2048], B in [1, 8]:
+ *   x = bf16(h / sqrt(mean(h^2) + 1e-6))   (RMSNorm, unit weight, fp64 inside)
+ *   h = h + bf16(moe(x))                   (residual add in fp32, in place)
+ * Optional outputs (NULL to skip): idx int32 [B][6], w fp32 [B][6] in
+ * selection order, as flint_moe_route returns them.
+ */
+FLINT_API int flint_moe_decode_residual(const flint_moe_layer *layer, float *h, int B, int32_t *idx,
+                              float *w, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Prefill of the MoE block for T >= 1 tokens: the same function as
+ * flint_moe_decode row by row, computed as routing for T tokens, a stable
+ * token-by-expert sort, grouped GEMMs on the tensor cores (weights
+ * dequantized to bf16 tiles in shared memory; bf16 SwiGLU intermediate) and a
+ * fixed-order combine.
+ *   x bf16 [T][2048];  out bf16 [T][2048]
+ *   ws workspace of flint_workspace_bytes(FLINT_OP_PREFILL, T)
+ */
+FLINT_API int flint_moe_prefill(const flint_moe_layer *layer, const uint16_t *x, int T, uint16_t *out,
+                      void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Int4 GEMV for B in [1, 8] rows (the output head: N = 150,144, K = 2,048):
+ *   y[r][n] = sum_k W[n][k] x[r][k]  (fp32 accumulation)
+ *   argmax[r] = the lowest n with the largest y[r][n]   (argmax may be NULL)
+ *   q, s  packed int4 [N][K], K a multiple of 128 and at most 8192
+ *   x bf16 [B][K];  y fp32 [B][N]
+ *   ws workspace of flint_gemv_workspace_bytes(N, B)
+ * Rows are batch-invariant like flint_moe_decode.
+ */
+FLINT_API int flint_int4_gemv(const uint8_t *q, const uint16_t *s, int N, int K, const uint16_t *x, int B,
+                    float *y, int32_t *argmax, void *ws, size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FLINT_H */

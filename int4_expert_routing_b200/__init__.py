@@ -1,0 +1,151 @@
+"""Python binding of libflint (the Flint int4 MoE block for B200).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``libflint.so``.  Each function has the name and argument order of
+its C entry point (see ``include/flint.h``); device buffers are torch CUDA
+tensors (their data pointers are passed), and ``stream`` defaults to torch's
+current stream.  A missing or unloadable library raises: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libflint.so")
+
+FLINT_OK, FLINT_EINVAL, FLINT_ECUDA, FLINT_ETIMEOUT, FLINT_EDEVICE = range(5)
+FLINT_OP_ROUTE, FLINT_OP_DECODE, FLINT_OP_PREFILL, FLINT_OP_GEMV = range(4)
+HIDDEN, EXPERTS, TOP_K, EXPERT_I, SHARED_I, GROUP, MAX_DECODE_B = 2048, 256, 6, 512, 1024, 128, 8
+
+EXPORTS = ("flint_version", "flint_strerror", "flint_workspace_bytes",
+           "flint_gemv_workspace_bytes", "flint_workspace_init", "flint_read_status",
+           "flint_moe_route", "flint_moe_decode", "flint_moe_decode_residual",
+           "flint_moe_prefill", "flint_int4_gemv")
+
+_lib = None
+
+
+class FlintError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {strerror(code)} ({code})")
+
+
+class flint_moe_layer(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in (
+        "router_w", "router_b", "w13_q", "w13_s", "w2_q", "w2_s",
+        "sh13_q", "sh13_s", "sh2_q", "sh2_s")]
+
+
+def build(force: bool = False) -> str:
+    from . import buildlib
+    return buildlib.build(force=force)
+
+
+def lib() -> C.CDLL:
+    """Load libflint.so (raises if it is not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built: run int4_expert_routing_b200.build()")
+        L = C.CDLL(LIB_PATH)
+        vp, i, sz = C.c_void_p, C.c_int, C.c_size_t
+        L.flint_version.restype = i
+        L.flint_strerror.restype = C.c_char_p
+        L.flint_strerror.argtypes = [i]
+        L.flint_workspace_bytes.restype = sz
+        L.flint_workspace_bytes.argtypes = [i, i]
+        L.flint_gemv_workspace_bytes.restype = sz
+        L.flint_gemv_workspace_bytes.argtypes = [i, i]
+        L.flint_workspace_init.argtypes = [vp, sz, vp]
+        L.flint_read_status.argtypes = [vp, C.POINTER(C.c_int), vp]
+        lp = C.POINTER(flint_moe_layer)
+        L.flint_moe_route.argtypes = [lp, vp, i, vp, vp, vp, sz, vp]
+        L.flint_moe_decode.argtypes = [lp, vp, i, vp, vp, sz, vp]
+        L.flint_moe_decode_residual.argtypes = [lp, vp, i, vp, vp, vp, sz, vp]
+        L.flint_moe_prefill.argtypes = [lp, vp, i, vp, vp, sz, vp]
+        L.flint_int4_gemv.argtypes = [vp, vp, i, i, vp, i, vp, vp, vp, sz, vp]
+        for name in EXPORTS:
+            getattr(L, name).restype = getattr(L, name).restype or i
+        _lib = L
+    return _lib
+
+
+def strerror(code: int) -> str:
+    return lib().flint_strerror(int(code)).decode()
+
+
+def version() -> int:
+    return lib().flint_version()
+
+
+# ------------------------------------------------------------- marshalling
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def _check(code: int, where: str):
+    if code != FLINT_OK:
+        raise FlintError(code, where)
+
+
+def make_layer(t: dict) -> flint_moe_layer:
+    """The C layer struct from a dict of device tensors (keys as in flint.h)."""
+    return flint_moe_layer(*[_ptr(t[n]) for n, _ in flint_moe_layer._fields_])
+
+
+def flint_workspace_bytes(op: int, n: int) -> int:
+    return lib().flint_workspace_bytes(op, n)
+
+
+def flint_gemv_workspace_bytes(N: int, B: int) -> int:
+    return lib().flint_gemv_workspace_bytes(N, B)
+
+
+def flint_workspace_init(ws, ws_bytes: int, stream=None):
+    _check(lib().flint_workspace_init(_ptr(ws), ws_bytes, _stream(stream)), "flint_workspace_init")
+
+
+def flint_read_status(ws, stream=None) -> int:
+    st = C.c_int(0)
+    _check(lib().flint_read_status(_ptr(ws), C.byref(st), _stream(stream)), "flint_read_status")
+    return st.value
+
+
+def flint_moe_route(layer: flint_moe_layer, x, B: int, idx, w, ws, ws_bytes: int, stream=None):
+    _check(lib().flint_moe_route(C.byref(layer), _ptr(x), B, _ptr(idx), _ptr(w), _ptr(ws),
+                                 ws_bytes, _stream(stream)), "flint_moe_route")
+
+
+def flint_moe_decode(layer: flint_moe_layer, x, B: int, out, ws, ws_bytes: int, stream=None):
+    _check(lib().flint_moe_decode(C.byref(layer), _ptr(x), B, _ptr(out), _ptr(ws), ws_bytes,
+                                  _stream(stream)), "flint_moe_decode")
+
+
+def flint_moe_decode_residual(layer: flint_moe_layer, h, B: int, idx, w, ws, ws_bytes: int,
+                              stream=None):
+    _check(lib().flint_moe_decode_residual(C.byref(layer), _ptr(h), B, _ptr(idx), _ptr(w),
+                                           _ptr(ws), ws_bytes, _stream(stream)),
+           "flint_moe_decode_residual")
+
+
+def flint_moe_prefill(layer: flint_moe_layer, x, T: int, out, ws, ws_bytes: int, stream=None):
+    _check(lib().flint_moe_prefill(C.byref(layer), _ptr(x), T, _ptr(out), _ptr(ws), ws_bytes,
+                                   _stream(stream)), "flint_moe_prefill")
+
+
+def flint_int4_gemv(q, s, N: int, K: int, x, B: int, y, argmax, ws, ws_bytes: int, stream=None):
+    _check(lib().flint_int4_gemv(_ptr(q), _ptr(s), N, K, _ptr(x), B, _ptr(y), _ptr(argmax),
+                                 _ptr(ws), ws_bytes, _stream(stream)), "flint_int4_gemv")

@@ -1,0 +1,123 @@
+// C ABI entry points: argument checks (before anything is launched), workspace
+// sizing, status read-back.  All compute is in the kernels of decode.cu,
+// gemv.cu and prefill.cu.
+#include <cuda_runtime.h>
+
+#include "../../include/flint.h"
+#include "internal.h"
+
+using namespace flint;
+
+namespace {
+
+bool aligned16(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool layer_ok(const flint_moe_layer *l) {
+  return l && aligned16(l->router_w) && aligned16(l->router_b) && aligned16(l->w13_q) &&
+         aligned16(l->w13_s) && aligned16(l->w2_q) && aligned16(l->w2_s) && aligned16(l->sh13_q) &&
+         aligned16(l->sh13_s) && aligned16(l->sh2_q) && aligned16(l->sh2_s);
+}
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? FLINT_OK : FLINT_ECUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int flint_version(void) { return 100; }
+
+const char *flint_strerror(int code) {
+  switch (code) {
+    case FLINT_OK: return "ok";
+    case FLINT_EINVAL: return "invalid argument (pointer, alignment, size or workspace)";
+    case FLINT_ECUDA: return "CUDA runtime or launch error";
+    case FLINT_ETIMEOUT: return "a bounded device-side wait gave up";
+    case FLINT_EDEVICE: return "a device-side check failed";
+    default: return "unknown flint status";
+  }
+}
+
+size_t flint_workspace_bytes(int op, int n) {
+  if (n < 1) return 0;
+  switch (op) {
+    case FLINT_OP_ROUTE:
+    case FLINT_OP_DECODE:
+      return n <= FLINT_MAX_DECODE_B ? decode_layout(n).total : 0;
+    case FLINT_OP_GEMV:
+      return 0;  // depends on N: flint_gemv_workspace_bytes
+    default:
+      return 0;
+  }
+}
+
+size_t flint_gemv_workspace_bytes(int N, int B) {
+  if (N < 1 || B < 1 || B > FLINT_MAX_DECODE_B) return 0;
+  return gemv_ws_bytes(N, B);
+}
+
+int flint_workspace_init(void *ws, size_t ws_bytes, void *stream) {
+  if (!aligned16(ws) || ws_bytes < 256) return FLINT_EINVAL;
+  return from_cuda(cudaMemsetAsync(ws, 0, 256, static_cast<cudaStream_t>(stream)));
+}
+
+int flint_read_status(const void *ws, int *status, void *stream) {
+  if (!aligned16(ws) || !status) return FLINT_EINVAL;
+  uint32_t ctrl[2] = {0, 0};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(ctrl, ws, sizeof(ctrl), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return FLINT_ECUDA;
+  *status = static_cast<int>(ctrl[1]);
+  return FLINT_OK;
+}
+
+int flint_moe_route(const flint_moe_layer *layer, const uint16_t *x, int B, int32_t *idx,
+                    float *w, void *ws, size_t ws_bytes, void *stream) {
+  if (!layer_ok(layer) || !aligned16(x) || !idx || !w || B < 1 || B > FLINT_MAX_DECODE_B ||
+      !aligned16(ws) || ws_bytes < flint_workspace_bytes(FLINT_OP_ROUTE, B))
+    return FLINT_EINVAL;
+  return from_cuda(launch_decode(layer_args(layer), x, nullptr, nullptr, B, nullptr, idx, w,
+                                 static_cast<char *>(ws), static_cast<cudaStream_t>(stream),
+                                 true));
+}
+
+int flint_moe_decode(const flint_moe_layer *layer, const uint16_t *x, int B, uint16_t *out,
+                     void *ws, size_t ws_bytes, void *stream) {
+  if (!layer_ok(layer) || !aligned16(x) || !aligned16(out) || B < 1 || B > FLINT_MAX_DECODE_B ||
+      !aligned16(ws) || ws_bytes < flint_workspace_bytes(FLINT_OP_DECODE, B) ||
+      static_cast<const void *>(x) == static_cast<const void *>(out))
+    return FLINT_EINVAL;
+  return from_cuda(launch_decode(layer_args(layer), x, nullptr, nullptr, B, out, nullptr, nullptr,
+                                 static_cast<char *>(ws), static_cast<cudaStream_t>(stream),
+                                 false));
+}
+
+int flint_moe_decode_residual(const flint_moe_layer *layer, float *h, int B, int32_t *idx,
+                              float *w, void *ws, size_t ws_bytes, void *stream) {
+  if (!layer_ok(layer) || !aligned16(h) || B < 1 || B > FLINT_MAX_DECODE_B || !aligned16(ws) ||
+      ws_bytes < flint_workspace_bytes(FLINT_OP_DECODE, B))
+    return FLINT_EINVAL;
+  return from_cuda(launch_decode(layer_args(layer), nullptr, h, h, B, nullptr, idx, w,
+                                 static_cast<char *>(ws), static_cast<cudaStream_t>(stream),
+                                 false));
+}
+
+int flint_int4_gemv(const uint8_t *q, const uint16_t *s, int N, int K, const uint16_t *x, int B,
+                    float *y, int32_t *argmax, void *ws, size_t ws_bytes, void *stream) {
+  if (!aligned16(q) || !aligned16(s) || !aligned16(x) || !aligned16(y) || N < 1 || K < 128 ||
+      K % 128 || K > 8192 || B < 1 || B > FLINT_MAX_DECODE_B || !aligned16(ws) ||
+      ws_bytes < flint_gemv_workspace_bytes(N, B))
+    return FLINT_EINVAL;
+  // rows of scales are K/128 bf16 = K/64 bytes; 16-byte alignment of each
+  // row's start is not needed (scales are read one at a time)
+  return from_cuda(launch_gemv(q, s, N, K, x, B, y, argmax, static_cast<char *>(ws),
+                               static_cast<cudaStream_t>(stream)));
+}
+
+int flint_moe_prefill(const flint_moe_layer *layer, const uint16_t *x, int T, uint16_t *out,
+                      void *ws, size_t ws_bytes, void *stream) {
+  (void)layer, (void)x, (void)T, (void)out, (void)ws, (void)ws_bytes, (void)stream;
+  return FLINT_EINVAL;  // prefill path: not built yet
+}
+
+}  // extern "C"

@@ -320,3 +320,27 @@ def layer_codes_torch(seed: int, device, dims: Dims = FLINT) -> dict:
         "sh13_q": random_bytes_torch(seed, T_SH13_Q, _n(dims.sh13_q()), device).view(dims.sh13_q()),
         "sh2_q": random_bytes_torch(seed, T_SH2_Q, _n(dims.sh2_q()), device).view(dims.sh2_q()),
     }
+
+
+def to_device(arrays: dict, device) -> dict:
+    """Upload a dict of host arrays to ``device`` as torch tensors holding the
+    same bytes (uint16 travels as int16, uint8 as uint8)."""
+    import torch
+    out = {}
+    for k, v in arrays.items():
+        a = np.ascontiguousarray(v)
+        if a.dtype == np.uint16:
+            a = a.view(np.int16)
+        out[k] = torch.from_numpy(a).to(device)
+    return out
+
+
+def layer_device(seed: int, device, dims: Dims = FLINT, host: dict | None = None) -> dict:
+    """A layer's tensors on ``device``.  With ``host`` (from layer_host with
+    codes) the bytes are uploaded; otherwise the codes are drawn on the device
+    and only the floating tensors are drawn on the host."""
+    if host is not None:
+        return to_device(host, device)
+    d = to_device(layer_host(seed, dims, with_codes=False), device)
+    d.update(layer_codes_torch(seed, device, dims))
+    return d

@@ -1,0 +1,73 @@
+"""The C ABI library without a GPU: it loads, exports every entry point the
+header declares, and rejects bad arguments before touching the device."""
+import os
+import re
+
+import pytest
+
+import int4_expert_routing_b200 as F
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    F.build()
+    return F.lib()
+
+
+def declared_entry_points():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"FLINT_API\s+[\w\s\*]*?\b(flint_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_entry_points()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(F.EXPORTS)
+
+
+def test_version_and_strerror(lib):
+    assert F.version() >= 100
+    assert "invalid" in F.strerror(F.FLINT_EINVAL)
+    assert F.strerror(99) == "unknown flint status"
+
+
+def test_workspace_sizes(lib):
+    assert F.flint_workspace_bytes(F.FLINT_OP_DECODE, 0) == 0
+    assert F.flint_workspace_bytes(F.FLINT_OP_DECODE, 9) == 0
+    s1 = F.flint_workspace_bytes(F.FLINT_OP_DECODE, 1)
+    s8 = F.flint_workspace_bytes(F.FLINT_OP_DECODE, 8)
+    assert 0 < s1 < s8 and s8 % 256 == 0
+    assert F.flint_gemv_workspace_bytes(150144, 4) > 256
+    assert F.flint_gemv_workspace_bytes(150144, 9) == 0
+
+
+def test_bad_arguments_rejected_before_launch(lib):
+    layer = F.flint_moe_layer()                      # all NULL
+    fake = 1 << 20                                   # aligned, never dereferenced
+    with pytest.raises(F.FlintError) as e:
+        F.flint_moe_decode(layer, fake, 1, fake, fake, 1 << 20, stream=0)
+    assert e.value.code == F.FLINT_EINVAL
+    good = F.flint_moe_layer(*([fake] * 10))
+    for B in (0, 9):
+        with pytest.raises(F.FlintError):
+            F.flint_moe_decode(good, fake, B, fake + 4096, fake, 1 << 20, stream=0)
+    with pytest.raises(F.FlintError):                # misaligned x
+        F.flint_moe_decode(good, fake + 2, 1, fake + 4096, fake, 1 << 20, stream=0)
+    with pytest.raises(F.FlintError):                # workspace too small
+        F.flint_moe_decode(good, fake, 1, fake + 4096, fake, 64, stream=0)
+    with pytest.raises(F.FlintError):                # x aliases out
+        F.flint_moe_decode(good, fake, 1, fake, fake + 8192, 1 << 20, stream=0)
+    with pytest.raises(F.FlintError):                # K not a multiple of 128
+        F.flint_int4_gemv(fake, fake, 16, 100, fake, 1, fake, None, fake, 1 << 20, stream=0)
+    with pytest.raises(F.FlintError):
+        F.flint_moe_route(good, fake, 1, None, fake, fake, 1 << 20, stream=0)
+    with pytest.raises(F.FlintError):
+        F.flint_workspace_init(fake + 8, 16, stream=0)

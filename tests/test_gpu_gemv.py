@@ -1,0 +1,86 @@
+"""Int4 GEMV + argmax on the GPU (the 150,144 x 2,048 output head and ragged
+shapes), through the C ABI, against the fp64 oracle."""
+import numpy as np
+import pytest
+
+import int4_expert_routing_b200 as F
+import oracle
+import synth
+from gpu_util import check_close, dev_bf16, torch
+
+pytestmark = pytest.mark.gpu
+
+# Rows whose oracle top-1/top-2 gap is below this are excluded from the exact
+# argmax check (fp32 accumulation error of a 2,048-term sum at these
+# magnitudes is ~1e-6).
+ARGMAX_GAP = 1e-5
+
+
+def gemv(q, s, xbits, N, K):
+    B = xbits.shape[0]
+    qd = torch().from_numpy(np.ascontiguousarray(q)).cuda()
+    sd = torch().from_numpy(np.ascontiguousarray(s).view(np.int16)).cuda()
+    x = dev_bf16(xbits)
+    y = torch().empty((B, N), dtype=torch().float32, device="cuda")
+    am = torch().empty(B, dtype=torch().int32, device="cuda")
+    nb = F.flint_gemv_workspace_bytes(N, B)
+    ws = torch().zeros(nb, dtype=torch().uint8, device="cuda")
+    F.flint_workspace_init(ws, nb)
+    F.flint_int4_gemv(qd, sd, N, K, x, B, y, am, ws, nb)
+    torch().cuda.synchronize()
+    return y.cpu().numpy(), am.cpu().numpy()
+
+
+@pytest.fixture(scope="module")
+def head():
+    F.build()
+    return synth.head_host()
+
+
+@pytest.mark.parametrize("rows", [[0], [0, 1, 2, 3]])
+def test_head_gemv_matches_oracle(head, rows):
+    x = synth.head_x(rows)
+    y, am = gemv(head["q"], head["s"], x, synth.VOCAB, synth.HIDDEN)
+    ref, ram, gap = oracle.int4_gemv(head["q"], head["s"], x)
+    check_close(y, ref, what="logits")
+    for b in range(len(rows)):
+        if gap[b] < ARGMAX_GAP:
+            print(f"row {b}: top-1/top-2 gap {gap[b]:.3e}: argmax excluded")
+            continue
+        assert am[b] == ram[b]
+    print("max |y - oracle|:", float(np.max(np.abs(y - ref))))
+
+
+def test_head_batch_invariance(head):
+    x = synth.head_x([0, 1, 2, 3])
+    y4, a4 = gemv(head["q"], head["s"], x, synth.VOCAB, synth.HIDDEN)
+    for b in range(4):
+        y1, a1 = gemv(head["q"], head["s"], x[b:b + 1], synth.VOCAB, synth.HIDDEN)
+        assert np.array_equal(y4[b], y1[0]) and a4[b] == a1[0]
+
+
+@pytest.mark.parametrize("N,K,B", [(1007, 384, 3), (16, 128, 8), (5, 2048, 1), (4099, 8192, 2)])
+def test_ragged_shapes(N, K, B):
+    q = synth.random_bytes(N, 77, N * K // 2).reshape(N, K // 2)
+    s = synth.scale_bits(N, 78, N * K // 128).reshape(N, K // 128)
+    x = np.stack([synth.bf16_bits(synth.normals(r, 79, K)) for r in range(B)])
+    y, am = gemv(q, s, x, N, K)
+    ref, ram, gap = oracle.int4_gemv(q, s, x)
+    check_close(y, ref, what="y")
+    for b in range(B):
+        if gap[b] >= ARGMAX_GAP:
+            assert am[b] == ram[b]
+
+
+def test_argmax_ties_go_to_lowest_row():
+    N, K = 4000, 256
+    q = np.zeros((N, K // 2), np.uint8)
+    s = np.full((N, K // 128), synth.bf16_bits(np.array([0.5]))[0], np.uint16)
+    for r in (3001, 17, 2500):          # three identical maxima
+        q[r, 0] = 0x07
+    q[100, 0] = 0x05
+    x = np.zeros((2, K), np.uint16)
+    x[:, 0] = synth.bf16_bits(np.array([1.0]))[0]
+    y, am = gemv(q, s, x, N, K)
+    assert list(am) == [17, 17]
+    assert y[0, 17] == 3.5 and y[0, 100] == 2.5
