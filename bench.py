@@ -279,8 +279,9 @@ def main():
     with torch.cuda.graph(gw, stream=stream):
         for s in range(min(args.warmup, total)):
             one_step(s, stream)
-    for _ in range(3):
-        gw.replay()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            gw.replay()
     stream.synchronize()
 
     sampler = ClockSampler(local)
@@ -289,15 +290,17 @@ def main():
     # soak: replay the timed graph for ~1 s so the clock record covers a loaded GPU
     t_soak = time.time()
     while time.time() - t_soak < 1.0:
-        g.replay()
+        with torch.cuda.stream(stream):
+            g.replay()
         stream.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
     tw0 = time.time()
-    e0.record(stream)
-    g.replay()
-    e1.record(stream)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
     e1.synchronize()
     tw1 = time.time()
     barrier(world)
@@ -323,11 +326,12 @@ def main():
                 for l in range(nl):
                     F.flint_moe_decode_residual(structs[l], h1, 1, None, None, ws1, nb1,
                                                 stream=stream)
-        g1.replay()
-        stream.synchronize()
-        e0.record(stream)
-        g1.replay()
-        e1.record(stream)
+        with torch.cuda.stream(stream):
+            g1.replay()
+            stream.synchronize()
+            e0.record(stream)
+            g1.replay()
+            e1.record(stream)
         e1.synchronize()
         ms1 = e0.elapsed_time(e1)
         us1 = ms1 * 1e3 / (args.steps * nl)
@@ -347,12 +351,14 @@ def main():
                 F.flint_moe_decode_residual(structs[l], h_work, B, None, None, ws, nb,
                                             stream=stream)
             out_host[i].copy_(h_work, non_blocking=True)
-    ge.replay()
+    with torch.cuda.stream(stream):
+        ge.replay()
     stream.synchronize()
     barrier(world)
-    e0.record(stream)
-    ge.replay()
-    e1.record(stream)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        ge.replay()
+        e1.record(stream)
     e1.synchronize()
     barrier(world)
     mse = max_over_ranks(world, e0.elapsed_time(e1))
@@ -373,7 +379,8 @@ def main():
             flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
             times = []
             for it in range(23):
-                flush.zero_()                  # evict the head from L2 between launches
+                with torch.cuda.stream(stream):
+                    flush.zero_()              # evict the head from L2 between launches
                 e0.record(stream)
                 F.flint_int4_gemv(hq, hs_, synth.VOCAB, H, xh, hb, y, am, wsh, nbh,
                                   stream=stream)

@@ -94,6 +94,10 @@ typedef struct {
 /* Library version (major*10000 + minor*100 + patch). */
 FLINT_API int flint_version(void);
 
+/* Name of the CUDA error behind the calling thread's last FLINT_ECUDA
+ * ("none" if there was none); static string. */
+FLINT_API const char *flint_last_cuda_error(void);
+
 /* Human-readable name of a FLINT_* code (static string). */
 FLINT_API const char *flint_strerror(int code);
 

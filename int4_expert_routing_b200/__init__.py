@@ -18,7 +18,7 @@ FLINT_OK, FLINT_EINVAL, FLINT_ECUDA, FLINT_ETIMEOUT, FLINT_EDEVICE = range(5)
 FLINT_OP_ROUTE, FLINT_OP_DECODE, FLINT_OP_PREFILL, FLINT_OP_GEMV = range(4)
 HIDDEN, EXPERTS, TOP_K, EXPERT_I, SHARED_I, GROUP, MAX_DECODE_B = 2048, 256, 6, 512, 1024, 128, 8
 
-EXPORTS = ("flint_version", "flint_strerror", "flint_workspace_bytes",
+EXPORTS = ("flint_version", "flint_strerror", "flint_last_cuda_error", "flint_workspace_bytes",
            "flint_gemv_workspace_bytes", "flint_workspace_init", "flint_read_status",
            "flint_moe_route", "flint_moe_decode", "flint_moe_decode_residual",
            "flint_moe_prefill", "flint_int4_gemv")
@@ -29,7 +29,8 @@ _lib = None
 class FlintError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
-        super().__init__(f"{where}: {strerror(code)} ({code})")
+        detail = f" [{lib().flint_last_cuda_error().decode()}]" if code == FLINT_ECUDA else ""
+        super().__init__(f"{where}: {strerror(code)} ({code}){detail}")
 
 
 class flint_moe_layer(C.Structure):
@@ -54,6 +55,7 @@ def lib() -> C.CDLL:
         L.flint_version.restype = i
         L.flint_strerror.restype = C.c_char_p
         L.flint_strerror.argtypes = [i]
+        L.flint_last_cuda_error.restype = C.c_char_p
         L.flint_workspace_bytes.restype = sz
         L.flint_workspace_bytes.argtypes = [i, i]
         L.flint_gemv_workspace_bytes.restype = sz
@@ -102,8 +104,12 @@ def _check(code: int, where: str):
 
 
 def make_layer(t: dict) -> flint_moe_layer:
-    """The C layer struct from a dict of device tensors (keys as in flint.h)."""
-    return flint_moe_layer(*[_ptr(t[n]) for n, _ in flint_moe_layer._fields_])
+    """The C layer struct from a dict of device tensors (keys as in flint.h).
+    The struct keeps a reference to the tensors, so their memory stays
+    allocated while the struct is alive."""
+    layer = flint_moe_layer(*[_ptr(t[n]) for n, _ in flint_moe_layer._fields_])
+    layer._tensors = t
+    return layer
 
 
 def flint_workspace_bytes(op: int, n: int) -> int:

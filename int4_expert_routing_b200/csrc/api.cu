@@ -2,6 +2,7 @@
 // sizing, status read-back.  All compute is in the kernels of decode.cu,
 // gemv.cu and prefill.cu.
 #include <cuda_runtime.h>
+#include <stdio.h>
 
 #include "../../include/flint.h"
 #include "internal.h"
@@ -18,13 +19,37 @@ bool layer_ok(const flint_moe_layer *l) {
          aligned16(l->sh13_s) && aligned16(l->sh2_q) && aligned16(l->sh2_s);
 }
 
-int from_cuda(cudaError_t e) { return e == cudaSuccess ? FLINT_OK : FLINT_ECUDA; }
+thread_local cudaError_t g_last_cuda = cudaSuccess;
+thread_local const char *g_last_where = "";
+thread_local const char *g_step = "";
+thread_local char g_msg[160];
+
+int from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return FLINT_OK;
+  g_last_cuda = e;
+  g_last_where = g_step;
+  return FLINT_ECUDA;
+}
 
 }  // namespace
+
+namespace flint {
+void note_step(const char *where) { g_step = where; }
+cudaError_t noted(cudaError_t e, const char *where) {
+  g_step = where;
+  return e;
+}
+}  // namespace flint
 
 extern "C" {
 
 int flint_version(void) { return 100; }
+
+const char *flint_last_cuda_error(void) {
+  if (g_last_cuda == cudaSuccess) return "none";
+  snprintf(g_msg, sizeof(g_msg), "%s at %s", cudaGetErrorName(g_last_cuda), g_last_where);
+  return g_msg;
+}
 
 const char *flint_strerror(int code) {
   switch (code) {
@@ -66,7 +91,7 @@ int flint_read_status(const void *ws, int *status, void *stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemcpyAsync(ctrl, ws, sizeof(ctrl), cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-  if (e != cudaSuccess) return FLINT_ECUDA;
+  if (e != cudaSuccess) return from_cuda(e);
   *status = static_cast<int>(ctrl[1]);
   return FLINT_OK;
 }

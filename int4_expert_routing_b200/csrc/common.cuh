@@ -55,20 +55,19 @@ FLINT_DEV uint32_t ld_nc_u16(const void *p) {
   asm("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
   return v;
 }
-// Data written by an earlier kernel of the same chain: read at L2.
-FLINT_DEV uint4 ld_cg_v4(const void *p) {
-  uint4 v;
-  asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
+// Data written by an earlier kernel of the chain (or by other CTAs of this
+// one before a fence + counter): read at L2, never from a possibly stale L1
+// line.  Plain (non-volatile) loads, so independent ones overlap.
+FLINT_DEV uint4 ld_cg_v4(const void *p) { return __ldcg(reinterpret_cast<const uint4 *>(p)); }
 FLINT_DEV uint32_t ld_cg_u32(const void *p) {
-  uint32_t v;
-  asm volatile("ld.global.cg.u32 %0, [%1];" : "=r"(v) : "l"(p));
-  return v;
+  return __ldcg(reinterpret_cast<const unsigned int *>(p));
 }
-FLINT_DEV float ld_cg_f32(const void *p) { return __uint_as_float(ld_cg_u32(p)); }
+FLINT_DEV float ld_cg_f32(const void *p) { return __ldcg(reinterpret_cast<const float *>(p)); }
+FLINT_DEV double ld_cg_f64(const void *p) { return __ldcg(reinterpret_cast<const double *>(p)); }
+
+FLINT_DEV uint32_t smem_addr_(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
 
 // ------------------------------------------------------------------ PDL
 FLINT_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -183,6 +182,13 @@ FLINT_DEV int frag_slot(int k) {
   return (((G * 4 + t) * 16) + 4 * q + p) * 2 + half;
 }
 
+// ------------------------------------------------------------------ cp.async (16 B, L2 only)
+FLINT_DEV void cp_async16(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr_(dst)), "l"(src)
+               : "memory");
+}
+FLINT_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // ------------------------------------------------------------------ mbarrier / bulk copy
 FLINT_DEV uint32_t smem_addr(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -190,6 +196,15 @@ FLINT_DEV uint32_t smem_addr(const void *p) {
 FLINT_DEV void mbar_init(uint64_t *bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count));
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+// Raise the expected transaction bytes of the current phase without arriving.
+FLINT_DEV void mbar_add_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+FLINT_DEV void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 FLINT_DEV void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
@@ -204,6 +219,10 @@ FLINT_DEV void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *ba
       "l"(src), "r"(bytes), "r"(smem_addr(bar))
       : "memory");
 }
+// Order this thread's earlier generic-proxy shared-memory accesses before
+// later async-proxy (bulk copy / tensor core) accesses of the same memory.
+FLINT_DEV void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 // Bounded wait for phase `parity` of `bar`; false if it did not complete.
 FLINT_DEV bool mbar_wait(uint64_t *bar, uint32_t parity) {
   for (uint32_t i = 0; i < kWaitPolls; ++i) {

@@ -1,29 +1,33 @@
 // Decode step of the Flint MoE block: three kernels chained with programmatic
-// dependent launch (PDL), each loading the weights it can before waiting on
-// its predecessor.
+// dependent launch (PDL).  Each kernel issues every load that does not depend
+// on its predecessor before it waits on it.
 //
-//   K1  router (bf16 W_r, fp64 sum of fp32 group partials, fp32 sigmoid,
-//       + bias, top-6 with the lower index winning ties, normalized weights)
-//       and, in other CTAs, the shared expert's gate/up GEMV + SwiGLU, which
-//       does not depend on routing.  The last router CTA to finish picks the
-//       experts and builds the slot table (the union of chosen experts, in
-//       ascending expert order).
-//   K2  gate/up int4 GEMV + SwiGLU for every slot, weighted by the routing
-//       weight of each row that chose it; writes the fp32 intermediate as an
-//       exact-enough hi/lo bf16 pair image for K3's tensor-core fragments.
-//   K3  down-projection GEMV of every slot and of the shared expert, with the
-//       weights staged in shared memory by bulk copies issued before the PDL
-//       wait; combine per row in a fixed order (the row's experts in
-//       ascending index, then the shared expert).
+//   K1  router: bf16 W_r against the input, one 128-wide k-group per warp on
+//       mma.sync, group partials summed in fp64 in a fixed order; the last
+//       CTA to finish takes sigmoid (fp32), adds the bias, picks the top 6
+//       (lower index wins ties), normalizes the weights and builds the slot
+//       table (the union of chosen experts, ascending).
+//   K2  gate/up int4 GEMV + SwiGLU.  Shared-expert items need no routing and
+//       run before the PDL wait, overlapping K1; routed items run after it,
+//       for every slot, scaled by the routing weight of each row that chose
+//       the expert, and leave the fp32 intermediate as a hi/lo bf16 pair image
+//       shaped for K3's tensor-core fragments.
+//   K3  down projection of every slot and of the shared expert: the weights
+//       are bulk-copied into shared memory before the PDL wait; after it the
+//       intermediates are staged in one round trip and each row is combined
+//       in a fixed order (its experts in ascending index, then the shared
+//       expert).
 //
 // Model structure: "How to Run Flint Locally", section "The architecture,
 // from config.json" (256 routed experts, 6 per token, expert size 512,
 // sigmoid router with normalized top-k, shared expert of size 1,024 for every
 // token); TandemLLM "21 Flint" section 21.1 (routing by sigmoid score with a
-// bias) and section 21.2 (fp32 intermediates: routed SwiGLU activations reach
-// 2.6e5, past fp16).  The kernel structure follows the low-latency decode
-// path described under "What vLLM changed" (routing and combine folded into
-// the neighbouring GEMVs, every kernel launched as a programmatic dependent).
+// bias) and section 21.2 (routed SwiGLU activations reach 2.6e5, past fp16:
+// intermediates stay fp32).  The kernel structure follows the low-latency
+// decode path under "What vLLM changed" (routing and combine folded into the
+// neighbouring GEMVs, every kernel a programmatic dependent that loads its
+// weights while the previous one runs) and TandemLLM section 21.4 (the
+// shared expert overlapped with the routed path, same bits either way).
 //
 // Batch invariance: every output element of row b is computed by the same
 // lanes, in the same order, from row b's data alone, whatever B is; the
@@ -33,13 +37,10 @@
 
 namespace flint {
 
-constexpr int kRouterCtas = 64;  // 256 router items: 16 expert tiles x 16 k-groups
-constexpr int kSharedCtas = 32;  // 128 shared gate/up items of 8 intermediate rows
-constexpr int kK1Threads = 128;
-constexpr int kK2Threads = 128;
+constexpr int kRouterCtas = 32;   // 16 expert tiles x 2 k-halves
+constexpr int kK1Threads = 256;   // 8 warps: one 128-wide k-group each
 constexpr int kK3Threads = 256;
-constexpr int kXFragBytes = 16 * 128 * 16;  // 16 groups, 128 uint4 each
-constexpr int kNPre = 4;                    // groups of weights in flight per warp
+constexpr int kXFragBytes = 16 * 128 * 16;  // 16 groups x 128 uint4
 
 FLINT_DEV float silu_f(float v) { return v / (1.f + expf(-v)); }
 
@@ -51,79 +52,59 @@ FLINT_DEV void write_hilo(uint16_t *img_hi, uint16_t *img_lo, int k, float v) {
   img_lo[s] = __bfloat16_as_ushort(lo);
 }
 
-// Gate/up GEMV of one 8-row item: tile rows g = gate row, g + 8 = up row.
-// Returns acc[0..1] = gate (cols 2t, 2t+1), acc[2..3] = up.
-struct GateUpPtrs {
-  const uint8_t *gate;
-  const uint8_t *up;
-  const uint16_t *gate_s;
-  const uint16_t *up_s;
-};
-
-FLINT_DEV void gateup_prefetch(const GateUpPtrs &p, uint4 (&pg)[kNPre], uint4 (&pu)[kNPre],
-                               uint32_t (&sg)[kNPre], uint32_t (&su)[kNPre]) {
+// ---------------------------------------------------------------- input
+// RMSNorm scale 1/sqrt(mean(h^2) + eps) per row, fp64, in one fixed order
+// whatever the block size: threads 0..127 each sum a strided slice, then an
+// xor tree per warp and the four warps in order.  K1 and K2 both call this,
+// so they normalize to the same bits.
+constexpr int kRmsThreads = 128;
+FLINT_DEV void rms_inv(const float *h, int B, double *s_red /*[4 * kMaxB]*/, double *inv,
+                       int tid) {
+  const int warp = tid >> 5, lane = tid & 31;
+  if (tid < kRmsThreads) {
+    for (int b = 0; b < B; ++b) {
+      double ss = 0.0;
+      for (int i = tid; i < kH; i += kRmsThreads) {
+        const double v = (double)ld_cg_f32(h + (size_t)b * kH + i);
+        ss = fma(v, v, ss);
+      }
 #pragma unroll
-  for (int G = 0; G < kNPre; ++G) {
-    pg[G] = ld_stream(p.gate + 64 * G);
-    pu[G] = ld_stream(p.up + 64 * G);
-    sg[G] = ld_nc_u16(p.gate_s + G);
-    su[G] = ld_nc_u16(p.up_s + G);
-  }
-}
-
-FLINT_DEV void gateup_compute(const GateUpPtrs &p, uint4 (&pg)[kNPre], uint4 (&pu)[kNPre],
-                              uint32_t (&sg)[kNPre], uint32_t (&su)[kNPre], const uint4 *xfrag,
-                              int lane, float (&acc)[4]) {
-  acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
-#pragma unroll
-  for (int G = 0; G < kH / kG; ++G) {
-    const int sl = G % kNPre;
-    const uint4 wg = pg[sl], wu = pu[sl];
-    const float sgf = bf16_bits_to_f32(sg[sl]), suf = bf16_bits_to_f32(su[sl]);
-    if (G + kNPre < kH / kG) {
-      pg[sl] = ld_stream(p.gate + 64 * (G + kNPre));
-      pu[sl] = ld_stream(p.up + 64 * (G + kNPre));
-      sg[sl] = ld_nc_u16(p.gate_s + G + kNPre);
-      su[sl] = ld_nc_u16(p.up_s + G + kNPre);
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if (lane == 0) s_red[warp * kMaxB + b] = ss;
     }
-    uint32_t ra[16], rb[16], xb[16];
-    int4x32_to_bf16x2(wg, ra);
-    int4x32_to_bf16x2(wu, rb);
-    load_frag(xfrag + (G * 32 + lane) * 4, xb);
-    float d[4];
-    group_mma(ra, rb, xb, d);
-    acc[0] = fmaf(d[0], sgf, acc[0]);
-    acc[1] = fmaf(d[1], sgf, acc[1]);
-    acc[2] = fmaf(d[2], suf, acc[2]);
-    acc[3] = fmaf(d[3], suf, acc[3]);
   }
+  __syncthreads();
+  if (tid < B) {
+    double ss = 0.0;
+    for (int w = 0; w < kRmsThreads / 32; ++w) ss += s_red[w * kMaxB + tid];
+    inv[tid] = 1.0 / sqrt(ss / kH + FLINT_RMS_EPS);
+  }
+  __syncthreads();
 }
 
-// x fragment of the block's input rows into shared memory.  Plain decode
-// reads the bf16 input; the residual form computes RMSNorm of the fp32
-// residual (fp64 inside) and rounds to bf16, and CTA `writer` also stores the
-// normalized rows for the next kernel.
+// Activation fragment of groups G0 .. G0+nG-1 of the block's input rows into
+// shared memory (local group index G - G0).  Plain decode reads the bf16
+// input; the residual form rounds RMSNorm(h) to bf16 (fp64 product, one
+// rounding).
 template <bool kResidual>
-FLINT_DEV void stage_input(uint4 *xfrag, const uint16_t *x_in, const float *h, int B,
-                           const double *inv, uint16_t *xn_out, bool writer, int tid,
-                           int nthreads) {
-  for (int task = tid; task < 16 * 128; task += nthreads) {
-    const int G = task >> 7, ln = (task >> 2) & 31, q = task & 3;
+FLINT_DEV void stage_input(uint4 *xfrag, int G0, int nG, const uint16_t *x_in, const float *h,
+                           int B, const double *inv, int tid, int nthreads) {
+  for (int task = tid; task < nG * 128; task += nthreads) {
+    const int G = G0 + (task >> 7), ln = (task >> 2) & 31, q = task & 3;
     const int gg = ln >> 2, tt = ln & 3;
     const int k0 = 128 * G + 32 * tt + 8 * q;
     uint4 v = make_uint4(0, 0, 0, 0);
     if (gg < B) {
       if (kResidual) {
-        const uint4 a = ld_cg_v4(h + (size_t)gg * kH + k0);
-        const uint4 c = ld_cg_v4(h + (size_t)gg * kH + k0 + 4);
+        const float4 a = __ldcg(reinterpret_cast<const float4 *>(h + (size_t)gg * kH + k0));
+        const float4 c = __ldcg(reinterpret_cast<const float4 *>(h + (size_t)gg * kH + k0 + 4));
         const double s = inv[gg];
-        const uint32_t f[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+        const float f[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
         uint32_t bits[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) bits[i] = f64_to_bf16_bits((double)__uint_as_float(f[i]) * s);
+        for (int i = 0; i < 8; ++i) bits[i] = f64_to_bf16_bits((double)f[i] * s);
         v = make_uint4(bits[0] | (bits[1] << 16), bits[2] | (bits[3] << 16),
                        bits[4] | (bits[5] << 16), bits[6] | (bits[7] << 16));
-        if (writer) *reinterpret_cast<uint4 *>(xn_out + (size_t)gg * kH + k0) = v;
       } else {
         v = ld_cg_v4(x_in + (size_t)gg * kH + k0);
       }
@@ -132,147 +113,124 @@ FLINT_DEV void stage_input(uint4 *xfrag, const uint16_t *x_in, const float *h, i
   }
 }
 
-// RMSNorm scale 1/sqrt(mean(h^2) + eps) per row, fp64, fixed reduction order.
-FLINT_DEV void rms_inv(const float *h, int B, double *s_red /*[nwarps][kMaxB]*/, double *inv,
-                       int tid, int nthreads) {
-  const int warp = tid >> 5, lane = tid & 31, nw = nthreads >> 5;
-  for (int b = 0; b < B; ++b) {
-    double ss = 0.0;
-    for (int i = tid; i < kH; i += nthreads) {
-      const double v = (double)ld_cg_f32(h + (size_t)b * kH + i);
-      ss = fma(v, v, ss);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (lane == 0) s_red[warp * kMaxB + b] = ss;
+// ============================================================== K1: router
+constexpr uint32_t kSlotInvalid = 0xffffffffu;
+FLINT_DEV uint32_t slot_expert(uint32_t w) { return w & 0xffu; }
+FLINT_DEV uint32_t slot_mask(uint32_t w) { return (w >> 8) & 0xffu; }
+FLINT_DEV int slot_count(uint32_t w) { return (int)((w >> 16) & 0x1ffu); }
+
+// Release-publish this CTA's results and tell whether it is the last of
+// `nctas` to do so; one fence per CTA on each side of the counter.
+FLINT_DEV bool last_cta(uint32_t *counter, uint32_t nctas, int *s_flag) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const uint32_t prev = atomicAdd(counter, 1u);
+    const bool last = prev == nctas - 1;
+    if (last) __threadfence();
+    *s_flag = last;
   }
   __syncthreads();
-  if (tid < B) {
-    double ss = 0.0;
-    for (int w = 0; w < nw; ++w) ss += s_red[w * kMaxB + tid];
-    inv[tid] = 1.0 / sqrt(ss / kH + FLINT_RMS_EPS);
-  }
-  __syncthreads();
+  return *s_flag != 0;
 }
 
-// ============================================================== K1
 template <bool kResidual>
 __global__ void __launch_bounds__(kK1Threads)
-    k1_route_shared(LayerArgs L, const uint16_t *__restrict__ x_in, const float *__restrict__ h,
-                    int B, char *__restrict__ ws, DecodeLayout lay, int32_t *__restrict__ idx_out,
-                    float *__restrict__ w_out) {
-  extern __shared__ uint4 xfrag[];
+    k1_router(LayerArgs L, const uint16_t *__restrict__ x_in, const float *__restrict__ h, int B,
+              char *__restrict__ ws, DecodeLayout lay, int32_t *__restrict__ idx_out,
+              float *__restrict__ w_out) {
+  extern __shared__ __align__(128) unsigned char sm[];  // [16 rows][2048 B] | x fragment
+  uint4 *xfrag = reinterpret_cast<uint4 *>(sm + 16 * 2048);
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ double s_part[8][kMaxB][16];
   __shared__ double s_red[4 * kMaxB];
   __shared__ double s_inv[kMaxB];
   __shared__ int s_last;
   __shared__ int s_asc_e[kMaxB][kTopK];
   __shared__ float s_asc_w[kMaxB][kTopK];
   __shared__ int s_slot_of[kE];
-  __shared__ uint32_t s_mask[kE];
-  __shared__ int s_wcount[4];
+  __shared__ int s_slot_e[kE];
+  __shared__ uint32_t s_slot_m[kE];
+  __shared__ int s_wcount[8];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   uint32_t *ctrl = reinterpret_cast<uint32_t *>(ws + lay.ctrl);
-  const bool router = blockIdx.x < kRouterCtas;
-  const int item = (router ? (int)blockIdx.x : (int)blockIdx.x - kRouterCtas) * 4 + warp;
+  const int et = blockIdx.x >> 1, kh = blockIdx.x & 1;
 
-  // ---- weights first: nothing here depends on the previous kernel
-  uint4 wa[4], wb[4];
-  uint4 pg[kNPre], pu[kNPre];
-  uint32_t sg[kNPre], su[kNPre];
-  GateUpPtrs gp{};
-  if (router) {
-    const int et = item >> 4, G = item & 15;
-    const uint16_t *ra = L.router_w + (size_t)(16 * et + g) * kH + 128 * G + 32 * t;
-    const uint16_t *rb = ra + 8 * kH;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      wa[q] = ld_stream(ra + 8 * q);
-      wb[q] = ld_stream(rb + 8 * q);
-    }
-  } else {
-    const int r = 8 * item + g;
-    gp.gate = L.sh13_q + (size_t)r * (kH / 2) + 16 * t;
-    gp.up = L.sh13_q + (size_t)(kIs + r) * (kH / 2) + 16 * t;
-    gp.gate_s = L.sh13_s + (size_t)r * (kH / kG);
-    gp.up_s = L.sh13_s + (size_t)(kIs + r) * (kH / kG);
-    gateup_prefetch(gp, pg, pu, sg, su);
+  // this CTA's router block: 16 experts x one k-half (2 KB per row), fetched
+  // before the wait (the weights do not depend on the previous kernel)
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    mbar_expect_tx(&bar, 16 * 2048);
   }
-
+  __syncthreads();
+  if (tid < 16)
+    bulk_g2s(sm + tid * 2048, L.router_w + (size_t)(16 * et + tid) * kH + kh * (kH / 2), 2048, &bar);
   pdl_wait();
   pdl_trigger();
 
-  // ---- input rows -> activation fragment
-  if (kResidual) rms_inv(h, B, s_red, s_inv, tid, kK1Threads);
-  stage_input<kResidual>(xfrag, x_in, h, B, s_inv, reinterpret_cast<uint16_t *>(ws + lay.xn),
-                         blockIdx.x == 0, tid, kK1Threads);
-  __syncthreads();
-
-  if (!router) {
-    float acc[4];
-    gateup_compute(gp, pg, pu, sg, su, xfrag, lane, acc);
-    uint16_t *hfs = reinterpret_cast<uint16_t *>(ws + lay.hfs);
-    const int r = 8 * item + g;
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const int b = 2 * t + c;
-      if (b < B) {
-        const float v = silu_f(acc[c]) * acc[2 + c];
-        write_hilo(hfs + (size_t)(2 * b) * kIs, hfs + (size_t)(2 * b + 1) * kIs, r, v);
-      }
-    }
+  if (kResidual) rms_inv(h, B, s_red, s_inv, tid);
+  stage_input<kResidual>(xfrag, 8 * kh, 8, x_in, h, B, s_inv, tid, kK1Threads);
+  const bool ok = mbar_wait(&bar, 0);
+  if (__syncthreads_or(!ok)) {
+    if (tid == 0) set_status(ctrl + 1, kStatusTimeout);
+    if (!ok) mbar_wait(&bar, 0);
     return;
   }
-
-  // ---- router item: 16 experts x one 128-wide group, fp32 group partials
   {
-    const int et = item >> 4, G = item & 15;
     uint32_t ra[16], rb[16], xb[16];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const uint4 a = bf16x8_to_pairs(wa[q]), c = bf16x8_to_pairs(wb[q]);
+      const uint4 a = bf16x8_to_pairs(
+          *reinterpret_cast<const uint4 *>(sm + g * 2048 + 256 * warp + 64 * t + 16 * q));
+      const uint4 c = bf16x8_to_pairs(
+          *reinterpret_cast<const uint4 *>(sm + (g + 8) * 2048 + 256 * warp + 64 * t + 16 * q));
       ra[4 * q] = a.x, ra[4 * q + 1] = a.y, ra[4 * q + 2] = a.z, ra[4 * q + 3] = a.w;
       rb[4 * q] = c.x, rb[4 * q + 1] = c.y, rb[4 * q + 2] = c.z, rb[4 * q + 3] = c.w;
     }
-    load_frag(xfrag + (G * 32 + lane) * 4, xb);
+    load_frag(xfrag + (warp * 32 + lane) * 4, xb);
     float d[4];
     group_mma(ra, rb, xb, d);
-    float *zp = reinterpret_cast<float *>(ws + lay.zpart);
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       const int b = 2 * t + c;
       if (b < B) {
-        zp[((size_t)G * B + b) * kE + 16 * et + g] = d[c];
-        zp[((size_t)G * B + b) * kE + 16 * et + g + 8] = d[2 + c];
+        s_part[warp][b][g] = (double)d[c];
+        s_part[warp][b][g + 8] = (double)d[2 + c];
       }
     }
   }
   __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    const uint32_t prev = atomicAdd(&ctrl[0], 1u);
-    s_last = (prev == (uint32_t)(kRouterCtas - 1));
+  double *zp = reinterpret_cast<double *>(ws + lay.zpart);
+  if (tid < B * 16) {
+    const int b = tid >> 4, r = tid & 15;
+    double p = 0.0;
+    for (int w = 0; w < 8; ++w) p += s_part[w][b][r];
+    zp[((size_t)kh * B + b) * kE + 16 * et + r] = p;
   }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
+  if (!last_cta(&ctrl[0], kRouterCtas, &s_last)) return;
 
-  // ---- last router CTA: scores, top-6, weights, slot table
-  const float *zp = reinterpret_cast<const float *>(ws + lay.zpart);
+  // ---- last CTA: scores, top-6, weights, slot table (one warp per row)
   int32_t *sel_idx = reinterpret_cast<int32_t *>(ws + lay.sel_idx);
   float *sel_w = reinterpret_cast<float *>(ws + lay.sel_w);
-  for (int b = warp; b < B; b += 4) {
+  if (warp < B) {
+    const int b = warp;
+    double z0[8], z1[8];
+    float bias[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      z0[i] = ld_cg_f64(zp + (size_t)b * kE + lane + 32 * i);
+      z1[i] = ld_cg_f64(zp + ((size_t)B + b) * kE + lane + 32 * i);
+      bias[i] = L.router_b[lane + 32 * i];
+    }
     float sv[8];
     uint32_t key[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const int e = lane + 32 * i;
-      double z = 0.0;
-      for (int G = 0; G < 16; ++G) z += (double)ld_cg_f32(zp + ((size_t)G * B + b) * kE + e);
-      const float zf = (float)z;
+      const float zf = (float)(z0[i] + z1[i]);
       const float s = 1.f / (1.f + expf(-zf));
       sv[i] = s;
-      key[i] = float_key(s + L.router_b[e]);
+      key[i] = float_key(s + bias[i]);
     }
     uint32_t taken = 0;
     int sel_e[kTopK];
@@ -298,64 +256,50 @@ __global__ void __launch_bounds__(kK1Threads)
     float ssum = 0.f;
 #pragma unroll
     for (int j = 0; j < kTopK; ++j) ssum += sel_s[j];
-    if (lane == 0) {
-      float wj[kTopK];
+    // lane j < 6 writes entry j; ascending order by counting smaller experts
+    if (lane < kTopK) {
+      int e_me = sel_e[0];
+      float s_me = sel_s[0];
 #pragma unroll
-      for (int j = 0; j < kTopK; ++j) {
-        wj[j] = sel_s[j] / ssum;
-        sel_idx[b * kTopK + j] = sel_e[j];
-        sel_w[b * kTopK + j] = wj[j];
-        if (idx_out) idx_out[b * kTopK + j] = sel_e[j];
-        if (w_out) w_out[b * kTopK + j] = wj[j];
-      }
-      // ascending expert order for the combine
-      int ae[kTopK];
-      float aw[kTopK];
-      for (int j = 0; j < kTopK; ++j) {
-        int p = j;
-        while (p > 0 && ae[p - 1] > sel_e[j]) {
-          ae[p] = ae[p - 1];
-          aw[p] = aw[p - 1];
-          --p;
-        }
-        ae[p] = sel_e[j];
-        aw[p] = wj[j];
-      }
-      for (int j = 0; j < kTopK; ++j) s_asc_e[b][j] = ae[j], s_asc_w[b][j] = aw[j];
+      for (int j = 1; j < kTopK; ++j)
+        if (lane == j) e_me = sel_e[j], s_me = sel_s[j];
+      const float w_me = s_me / ssum;
+      sel_idx[b * kTopK + lane] = e_me;
+      sel_w[b * kTopK + lane] = w_me;
+      if (idx_out) idx_out[b * kTopK + lane] = e_me;
+      if (w_out) w_out[b * kTopK + lane] = w_me;
+      int rank = 0;
+#pragma unroll
+      for (int j = 0; j < kTopK; ++j) rank += sel_e[j] < e_me;
+      s_asc_e[b][rank] = e_me;
+      s_asc_w[b][rank] = w_me;
     }
   }
   __syncthreads();
-  for (int e = tid; e < kE; e += kK1Threads) {
-    uint32_t m = 0;
-    for (int b = 0; b < B; ++b)
-      for (int j = 0; j < kTopK; ++j)
-        if (s_asc_e[b][j] == e) m |= 1u << b;
-    s_mask[e] = m;
+  // slot table: experts used by any row, ascending; one expert per thread
+  const int e = tid;
+  uint32_t m = 0;
+  for (int b = 0; b < B; ++b)
+    for (int j = 0; j < kTopK; ++j)
+      if (s_asc_e[b][j] == e) m |= 1u << b;
+  const uint32_t bal = __ballot_sync(0xffffffffu, m != 0);
+  if (lane == 0) s_wcount[warp] = __popc(bal);
+  __syncthreads();
+  int off = 0, total = 0;
+  for (int w = 0; w < 8; ++w) {
+    if (w < warp) off += s_wcount[w];
+    total += s_wcount[w];
+  }
+  if (m) {
+    const int slot = off + __popc(bal & ((1u << lane) - 1u));
+    s_slot_of[e] = slot;
+    s_slot_e[slot] = e;
+    s_slot_m[slot] = m;
   }
   __syncthreads();
-  int32_t *slot_e = reinterpret_cast<int32_t *>(ws + lay.slot_e);
-  uint32_t *slot_rows = reinterpret_cast<uint32_t *>(ws + lay.slot_rows);
-  int base = 0;
-  for (int round = 0; round < kE / kK1Threads; ++round) {
-    const int e = round * kK1Threads + tid;
-    const bool used = s_mask[e] != 0;
-    const uint32_t bal = __ballot_sync(0xffffffffu, used);
-    if (lane == 0) s_wcount[warp] = __popc(bal);
-    __syncthreads();
-    int off = base, total = 0;
-    for (int w = 0; w < 4; ++w) {
-      if (w < warp) off += s_wcount[w];
-      total += s_wcount[w];
-    }
-    if (used) {
-      const int slot = off + __popc(bal & ((1u << lane) - 1u));
-      s_slot_of[e] = slot;
-      slot_e[slot] = e;
-      slot_rows[slot] = s_mask[e];
-    }
-    base += total;
-    __syncthreads();
-  }
+  uint32_t *slot_word = reinterpret_cast<uint32_t *>(ws + lay.slot_word);
+  slot_word[tid] = tid < total ? ((uint32_t)s_slot_e[tid] | (s_slot_m[tid] << 8) | ((uint32_t)total << 16))
+                               : kSlotInvalid;
   int32_t *asc_slot = reinterpret_cast<int32_t *>(ws + lay.asc_slot);
   float *asc_w = reinterpret_cast<float *>(ws + lay.asc_w);
   if (tid < B * kTopK) {
@@ -364,144 +308,341 @@ __global__ void __launch_bounds__(kK1Threads)
     asc_w[tid] = s_asc_w[b][j];
   }
   if (tid == 0) {
-    ctrl[2] = (uint32_t)base;
+    ctrl[2] = (uint32_t)total;
     ctrl[0] = 0;  // ready for the next call on this workspace
   }
 }
 
-// ============================================================== K2
+// ============================================================== K2: gate/up + SwiGLU
+// One CTA per work item: 8 intermediate rows of one expert (shared expert:
+// items 0..127; routed: item 128 + 64u + r/8 for slot u).  The item's bytes
+// (8 gate rows, 8 up rows, their scales; 16.5 KB) arrive in shared memory by
+// four bulk copies; the 4 warps split the 16 k-groups and their partial sums
+// are added in warp order.
+constexpr int kK2Warps = 4;
+constexpr int kItemBytes = 16384 + 512;
+constexpr int kSharedItems = kIs / 8;
+
+struct ItemSrc {
+  const uint8_t *gate;
+  const uint8_t *up;
+  const uint16_t *gate_s;
+  const uint16_t *up_s;
+};
+
+FLINT_DEV ItemSrc shared_item(const LayerArgs &L, int it) {
+  const int r = 8 * it;
+  return ItemSrc{L.sh13_q + (size_t)r * (kH / 2), L.sh13_q + (size_t)(kIs + r) * (kH / 2),
+                 L.sh13_s + (size_t)r * (kH / kG), L.sh13_s + (size_t)(kIs + r) * (kH / kG)};
+}
+FLINT_DEV ItemSrc routed_item(const LayerArgs &L, int e, int r0) {
+  const size_t row = (size_t)e * (2 * kI) + r0;
+  return ItemSrc{L.w13_q + row * (kH / 2), L.w13_q + (row + kI) * (kH / 2),
+                 L.w13_s + row * (kH / kG), L.w13_s + (row + kI) * (kH / kG)};
+}
+// one thread
+FLINT_DEV void issue_item(const ItemSrc &src, unsigned char *buf, uint64_t *bar) {
+  mbar_expect_tx(bar, kItemBytes);
+  bulk_g2s(buf, src.gate, 8192, bar);
+  bulk_g2s(buf + 8192, src.up, 8192, bar);
+  bulk_g2s(buf + 16384, src.gate_s, 256, bar);
+  bulk_g2s(buf + 16640, src.up_s, 256, bar);
+}
+
+// Compact activation fragment (only the B live columns, lanes g < B):
+// frag[(G * 4B + g * 4 + t) * 4 + q]; other lanes read zeros.
 template <bool kResidual>
-__global__ void __launch_bounds__(kK2Threads)
-    k2_routed_gateup(LayerArgs L, const uint16_t *__restrict__ x_in, int B,
-                     char *__restrict__ ws, DecodeLayout lay) {
-  extern __shared__ uint4 xfrag[];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-  pdl_wait();
-  pdl_trigger();
-  const uint32_t *ctrl = reinterpret_cast<const uint32_t *>(ws + lay.ctrl);
-  const int n_slots = (int)ld_cg_u32(ctrl + 2);
-  const int item0 = blockIdx.x * 4;
-  if (item0 >= n_slots * 64) return;
-
-  const uint16_t *src = kResidual ? reinterpret_cast<const uint16_t *>(ws + lay.xn) : x_in;
-  stage_input<false>(xfrag, src, nullptr, B, nullptr, nullptr, false, tid, kK2Threads);
-  __syncthreads();
-
-  const int item = item0 + warp;
-  if (item >= n_slots * 64) return;
-  const int u = item >> 6, r0 = 8 * (item & 63);
-  const int e = (int)ld_cg_u32(reinterpret_cast<const uint32_t *>(ws + lay.slot_e) + u);
-  const size_t row = (size_t)e * (2 * kI) + r0 + g;
-  GateUpPtrs gp;
-  gp.gate = L.w13_q + row * (kH / 2) + 16 * t;
-  gp.up = L.w13_q + (row + kI) * (kH / 2) + 16 * t;
-  gp.gate_s = L.w13_s + row * (kH / kG);
-  gp.up_s = L.w13_s + (row + kI) * (kH / kG);
-  uint4 pg[kNPre], pu[kNPre];
-  uint32_t sg[kNPre], su[kNPre];
-  gateup_prefetch(gp, pg, pu, sg, su);
-  float acc[4];
-  gateup_compute(gp, pg, pu, sg, su, xfrag, lane, acc);
-
-  const uint32_t mask = ld_cg_u32(reinterpret_cast<const uint32_t *>(ws + lay.slot_rows) + u);
-  const int32_t *asc_slot = reinterpret_cast<const int32_t *>(ws + lay.asc_slot);
-  const float *asc_w = reinterpret_cast<const float *>(ws + lay.asc_w);
-  uint16_t *hfr = reinterpret_cast<uint16_t *>(ws + lay.hfr);
+FLINT_DEV void stage_input_compact(uint4 *frag, const uint16_t *x_in, const float *h, int B,
+                                   const double *inv, int tid, int nthreads) {
+  const int n = 16 * 4 * B * 4;
+  for (int task = tid; task < n; task += nthreads) {
+    const int q = task & 3, gt = (task >> 2) % (4 * B), G = (task >> 2) / (4 * B);
+    const int gg = gt >> 2, tt = gt & 3;
+    const int k0 = 128 * G + 32 * tt + 8 * q;
+    uint4 v;
+    if (kResidual) {
+      const float4 a = __ldcg(reinterpret_cast<const float4 *>(h + (size_t)gg * kH + k0));
+      const float4 c = __ldcg(reinterpret_cast<const float4 *>(h + (size_t)gg * kH + k0 + 4));
+      const double s = inv[gg];
+      const float f[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+      uint32_t bits[8];
 #pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    const int b = 2 * t + c;
-    if (b < B && ((mask >> b) & 1u)) {
-      int j = 0;
-      for (int jj = 0; jj < kTopK; ++jj)
-        if ((int)ld_cg_u32(asc_slot + b * kTopK + jj) == u) j = jj;
-      const float w = ld_cg_f32(asc_w + b * kTopK + j);
-      const float v = w * (silu_f(acc[c]) * acc[2 + c]);
-      uint16_t *img = hfr + (size_t)((b * kTopK + j) * 2) * kI;
-      write_hilo(img, img + kI, r0 + g, v);
+      for (int i = 0; i < 8; ++i) bits[i] = f64_to_bf16_bits((double)f[i] * s);
+      v = make_uint4(bits[0] | (bits[1] << 16), bits[2] | (bits[3] << 16),
+                     bits[4] | (bits[5] << 16), bits[6] | (bits[7] << 16));
+    } else {
+      v = ld_cg_v4(x_in + (size_t)gg * kH + k0);
     }
+    frag[task] = bf16x8_to_pairs(v);
   }
 }
 
-// ============================================================== K3
+FLINT_DEV void load_frag_compact(const uint4 *frag, int G, int B, int lane, uint32_t (&x)[16]) {
+  const int g = lane >> 2, t = lane & 3;
+  if (g < B) {
+    const uint4 *p = frag + (size_t)(G * 4 * B + g * 4 + t) * 4;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 v = p[i];
+      x[4 * i] = v.x, x[4 * i + 1] = v.y, x[4 * i + 2] = v.z, x[4 * i + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) x[i] = 0u;
+  }
+}
+
+// This warp's 4 k-groups of the item: acc[0..1] gate, [2..3] up partials for
+// columns 2t, 2t+1 of row r0 + g.
+FLINT_DEV void item_part(const unsigned char *buf, const uint4 *frag, int B, int warp, int lane,
+                         float (&acc)[4]) {
+  const int g = lane >> 2, t = lane & 3;
+  acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+  const uint16_t *sg = reinterpret_cast<const uint16_t *>(buf + 16384 + g * 32);
+  const uint16_t *su = reinterpret_cast<const uint16_t *>(buf + 16640 + g * 32);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int G = 4 * warp + k;
+    const uint4 wg = *reinterpret_cast<const uint4 *>(buf + g * 1024 + 64 * G + 16 * t);
+    const uint4 wu = *reinterpret_cast<const uint4 *>(buf + 8192 + g * 1024 + 64 * G + 16 * t);
+    uint32_t ra[16], rb[16], xb[16];
+    int4x32_to_bf16x2(wg, ra);
+    int4x32_to_bf16x2(wu, rb);
+    load_frag_compact(frag, G, B, lane, xb);
+    float d[4];
+    group_mma(ra, rb, xb, d);
+    const float sgf = bf16_bits_to_f32(sg[G]), suf = bf16_bits_to_f32(su[G]);
+    acc[0] = fmaf(d[0], sgf, acc[0]);
+    acc[1] = fmaf(d[1], sgf, acc[1]);
+    acc[2] = fmaf(d[2], suf, acc[2]);
+    acc[3] = fmaf(d[3], suf, acc[3]);
+  }
+}
+
 template <bool kResidual>
+__global__ void __launch_bounds__(kK2Warps * 32)
+    k2_gateup(LayerArgs L, const uint16_t *__restrict__ x_in, const float *__restrict__ h, int B,
+              char *__restrict__ ws, DecodeLayout lay) {
+  extern __shared__ __align__(128) unsigned char sm[];  // item | x fragment (compact)
+  unsigned char *buf = sm;
+  uint4 *frag = reinterpret_cast<uint4 *>(sm + kItemBytes);
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ float s_acc[kK2Warps][32][4];
+  __shared__ double s_red[4 * kMaxB];
+  __shared__ double s_inv[kMaxB];
+  __shared__ uint32_t s_word;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const int it = blockIdx.x;
+  const bool shared_item_cta = it < kSharedItems;
+  uint32_t *ctrl = reinterpret_cast<uint32_t *>(ws + lay.ctrl);
+
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    if (shared_item_cta) issue_item(shared_item(L, it), buf, &bar);
+  }
+  // The input is final here: this grid was launched after K1 passed its wait.
+  if (kResidual) rms_inv(h, B, s_red, s_inv, tid);
+  stage_input_compact<kResidual>(frag, x_in, h, B, s_inv, tid, kK2Warps * 32);
+  if (!shared_item_cta) {
+    pdl_wait();
+    pdl_trigger();
+    if (tid == 0) {
+      const uint32_t w =
+          ld_cg_u32(reinterpret_cast<const uint32_t *>(ws + lay.slot_word) + ((it - kSharedItems) >> 6));
+      s_word = w;
+      if (w != kSlotInvalid)
+        issue_item(routed_item(L, (int)slot_expert(w), 8 * ((it - kSharedItems) & 63)), buf, &bar);
+    }
+  }
+  __syncthreads();
+  const uint32_t word = shared_item_cta ? 0u : s_word;
+  if (word == kSlotInvalid) return;  // a slot past the routed experts of this call
+  const bool ok = mbar_wait(&bar, 0);
+  if (__syncthreads_or(!ok)) {
+    if (tid == 0) set_status(ctrl + 1, kStatusTimeout);
+    if (!ok) mbar_wait(&bar, 0);
+    if (shared_item_cta) {
+      pdl_wait();
+      pdl_trigger();
+    }
+    return;
+  }
+  float acc[4];
+  item_part(buf, frag, B, warp, lane, acc);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) s_acc[warp][lane][i] = acc[i];
+  __syncthreads();
+  if (warp == 0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      acc[i] = ((s_acc[0][lane][i] + s_acc[1][lane][i]) + s_acc[2][lane][i]) + s_acc[3][lane][i];
+    if (shared_item_cta) {
+      uint16_t *hfs = reinterpret_cast<uint16_t *>(ws + lay.hfs);
+      const int r = 8 * it + g;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int b = 2 * t + c;
+        if (b < B)
+          write_hilo(hfs + (size_t)(2 * b) * kIs, hfs + (size_t)(2 * b + 1) * kIs, r,
+                     silu_f(acc[c]) * acc[2 + c]);
+      }
+    } else {
+      const int u = (it - kSharedItems) >> 6, r0 = 8 * ((it - kSharedItems) & 63);
+      const uint32_t mask = slot_mask(word);
+      const int32_t *asc_slot = reinterpret_cast<const int32_t *>(ws + lay.asc_slot);
+      const float *asc_w = reinterpret_cast<const float *>(ws + lay.asc_w);
+      uint16_t *hfr = reinterpret_cast<uint16_t *>(ws + lay.hfr);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int b = 2 * t + c;
+        if (b < B && ((mask >> b) & 1u)) {
+          int j = 0;
+#pragma unroll
+          for (int jj = 0; jj < kTopK; ++jj)
+            if (ld_cg_u32(asc_slot + b * kTopK + jj) == (uint32_t)u) j = jj;
+          const float w = ld_cg_f32(asc_w + b * kTopK + j);
+          uint16_t *img = hfr + (size_t)((b * kTopK + j) * 2) * kI;
+          write_hilo(img, img + kI, r0 + g, w * (silu_f(acc[c]) * acc[2 + c]));
+        }
+      }
+    }
+  }
+  if (shared_item_cta) {
+    pdl_wait();
+    pdl_trigger();
+  }
+}
+
+// ============================================================== K3: down + combine
+// Shared-memory plan (bytes): weights [umax][16 rows][256] | scales
+// [umax][16][4] bf16 | shared down [16][512] | shared scales [16][8] |
+// intermediates (kStage) routed [B][6][2][512] bf16, shared [B][2][1024] |
+// per-row results [8][8][16] fp32.
+struct K3Smem {
+  int umax, B;
+  __host__ __device__ size_t w() const { return 0; }
+  __host__ __device__ size_t s() const { return (size_t)umax * 4096; }
+  __host__ __device__ size_t shw() const { return s() + (size_t)umax * 128; }
+  __host__ __device__ size_t shs() const { return shw() + 8192; }
+  __host__ __device__ size_t hr() const { return shs() + 256; }
+  __host__ __device__ size_t hs() const { return hr() + (size_t)B * kTopK * 2 * kI * 2; }
+  __host__ __device__ size_t ysel(bool stage) const {
+    return stage ? hs() + (size_t)B * 2 * kIs * 2 : hr();
+  }
+  __host__ __device__ size_t total(bool stage) const { return ysel(stage) + 8 * 8 * 16 * 4; }
+};
+
+template <bool kResidual, bool kStage>
 __global__ void __launch_bounds__(kK3Threads)
     k3_down_combine(LayerArgs L, int B, uint16_t *__restrict__ out, float *__restrict__ h,
                     char *__restrict__ ws, DecodeLayout lay, int umax) {
   extern __shared__ __align__(128) unsigned char sm[];
-  unsigned char *wsm = sm;                   // [umax][16 rows][256 B]
-  unsigned char *ssm = wsm + umax * 4096;    // [umax][16 rows][4] bf16
-  unsigned char *shm = ssm + umax * 128;     // [16 rows][512 B]
-  unsigned char *shs = shm + 8192;           // [16 rows][8] bf16
-  float *ysel = reinterpret_cast<float *>(shs + 256);  // [8 rows b][7][16]
+  const K3Smem P{umax, B};
+  unsigned char *wsm = sm + P.w();
+  unsigned char *ssm = sm + P.s();
+  unsigned char *shm = sm + P.shw();
+  unsigned char *shs = sm + P.shs();
+  uint16_t *himg_r = reinterpret_cast<uint16_t *>(sm + P.hr());
+  uint16_t *himg_s = reinterpret_cast<uint16_t *>(sm + P.hs());
+  float *ysel = reinterpret_cast<float *>(sm + P.ysel(kStage));
   __shared__ __align__(8) uint64_t bar;
-  __shared__ int s_slots;
+  __shared__ int s_ns;
+  __shared__ uint32_t s_rows[kE];
+  __shared__ int s_asc[kMaxB * kTopK];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const int n0 = blockIdx.x * 16;
   uint32_t *ctrl = reinterpret_cast<uint32_t *>(ws + lay.ctrl);
 
   // Routing is final here (K2 triggered this launch after its own wait on
-  // K1), so the chosen experts' down rows can be fetched before the wait.
-  if (tid == 0) {
-    const int ns = (int)ld_cg_u32(ctrl + 2);
-    s_slots = ns;
-    mbar_init(&bar, 1);
-    mbar_expect_tx(&bar, (uint32_t)ns * (4096u + 128u) + 8192u + 256u);
-    const uint32_t *slot_e = reinterpret_cast<const uint32_t *>(ws + lay.slot_e);
-    for (int u = 0; u < ns; ++u) {
-      const size_t e = ld_cg_u32(slot_e + u);
-      bulk_g2s(wsm + u * 4096, L.w2_q + (e * kH + n0) * (kI / 2), 4096, &bar);
-      bulk_g2s(ssm + u * 128, L.w2_s + (e * kH + n0) * (kI / kG), 128, &bar);
+  // K1): fetch the chosen experts' down rows before waiting on K2.
+  if (tid == 0) mbar_init(&bar, 1);
+  __syncthreads();
+  {
+    const uint32_t word = ld_cg_u32(reinterpret_cast<const uint32_t *>(ws + lay.slot_word) + tid);
+    if (word != kSlotInvalid) {
+      const size_t e = slot_expert(word);
+      s_rows[tid] = slot_mask(word);
+      mbar_add_tx(&bar, 4096 + 128);
+      bulk_g2s(wsm + tid * 4096, L.w2_q + (e * kH + n0) * (kI / 2), 4096, &bar);
+      bulk_g2s(ssm + tid * 128, L.w2_s + (e * kH + n0) * (kI / kG), 128, &bar);
+      if (tid == 0) s_ns = slot_count(word);
     }
-    bulk_g2s(shm, L.sh2_q + (size_t)n0 * (kIs / 2), 8192, &bar);
-    bulk_g2s(shs, L.sh2_s + (size_t)n0 * (kIs / kG), 256, &bar);
+    if (tid == kK3Threads - 1) {
+      mbar_add_tx(&bar, 8192 + 256);
+      bulk_g2s(shm, L.sh2_q + (size_t)n0 * (kIs / 2), 8192, &bar);
+      bulk_g2s(shs, L.sh2_s + (size_t)n0 * (kIs / kG), 256, &bar);
+    }
+    if (tid < B * kTopK)
+      s_asc[tid] = (int)ld_cg_u32(reinterpret_cast<const uint32_t *>(ws + lay.asc_slot) + tid);
   }
+  __syncthreads();
+  if (tid == 0) mbar_arrive(&bar);
+
   pdl_wait();
   pdl_trigger();
-  __syncthreads();
-  const int ns = s_slots;
+  if (kStage) {
+    const unsigned char *src_r = reinterpret_cast<const unsigned char *>(ws + lay.hfr);
+    const unsigned char *src_s = reinterpret_cast<const unsigned char *>(ws + lay.hfs);
+    const int nr = B * kTopK * 2 * kI * 2 / 16, nsh = B * 2 * kIs * 2 / 16;
+    for (int i = tid; i < nr; i += kK3Threads)
+      cp_async16(reinterpret_cast<unsigned char *>(himg_r) + 16 * i, src_r + 16 * i);
+    for (int i = tid; i < nsh; i += kK3Threads)
+      cp_async16(reinterpret_cast<unsigned char *>(himg_s) + 16 * i, src_s + 16 * i);
+    cp_async_wait_all();
+  }
   const bool arrived = mbar_wait(&bar, 0);
   if (__syncthreads_or(!arrived)) {
     if (tid == 0) set_status(ctrl + 1, kStatusTimeout);
     if (!arrived) mbar_wait(&bar, 0);  // copies still in flight get one more bounded wait
     return;
   }
+  const int ns = s_ns;
 
-  const int32_t *asc_slot = reinterpret_cast<const int32_t *>(ws + lay.asc_slot);
-  const uint32_t *slot_rows = reinterpret_cast<const uint32_t *>(ws + lay.slot_rows);
-  const uint16_t *hfr = reinterpret_cast<const uint16_t *>(ws + lay.hfr);
-  const uint16_t *hfs = reinterpret_cast<const uint16_t *>(ws + lay.hfs);
-
-  for (int task = warp; task <= ns; task += kK3Threads / 32) {
-    const bool sh = (task == ns);
-    const int ngroups = sh ? kIs / kG : kI / kG;
+  const uint16_t *gr = kStage ? himg_r : reinterpret_cast<const uint16_t *>(ws + lay.hfr);
+  const uint16_t *gs = kStage ? himg_s : reinterpret_cast<const uint16_t *>(ws + lay.hfs);
+  // tasks: routed slots 0..ns-1, then the shared expert's two k-halves
+  for (int task = warp; task < ns + 2; task += kK3Threads / 32) {
+    const bool sh = task >= ns;
+    const int half = task - ns;
     const int rowbytes = sh ? kIs / 2 : kI / 2;
+    const int gbase = sh ? 4 * half : 0;  // first k-group of this task
     const unsigned char *wbase = sh ? shm : wsm + task * 4096;
-    const unsigned char *sbase = sh ? shs : ssm + task * 128;
-    const uint32_t mask = sh ? ((1u << B) - 1u) : ld_cg_u32(slot_rows + task);
+    const uint16_t *sc = reinterpret_cast<const uint16_t *>(sh ? shs : ssm + task * 128);
+    const int spr = sh ? kIs / kG : kI / kG;
+    const uint32_t mask = sh ? ((1u << B) - 1u) : s_rows[task];
     // this lane supplies activation column g
     const uint16_t *img = nullptr;
-    int imgstride = 0;
+    int stride = 0;
     if (g < B && ((mask >> g) & 1u)) {
       if (sh) {
-        img = hfs + (size_t)(2 * g) * kIs;
-        imgstride = kIs;
+        img = gs + (size_t)(2 * g) * kIs;
+        stride = kIs;
       } else {
         int j = 0;
         for (int jj = 0; jj < kTopK; ++jj)
-          if (ld_cg_u32(asc_slot + g * kTopK + jj) == (uint32_t)task) j = jj;
-        img = hfr + (size_t)((g * kTopK + j) * 2) * kI;
-        imgstride = kI;
+          if (s_asc[g * kTopK + jj] == task) j = jj;
+        img = gr + (size_t)((g * kTopK + j) * 2) * kI;
+        stride = kI;
       }
     }
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int G = 0; G < ngroups; ++G) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int G = gbase + k;
       uint32_t xh[16], xl[16];
       if (img) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const uint4 a = ld_cg_v4(img + ((G * 4 + t) * 16 + 4 * i) * 2);
-          const uint4 b = ld_cg_v4(img + imgstride + ((G * 4 + t) * 16 + 4 * i) * 2);
+          const int off = ((G * 4 + t) * 16 + 4 * i) * 2;
+          uint4 a, b;
+          if (kStage) {
+            a = *reinterpret_cast<const uint4 *>(img + off);
+            b = *reinterpret_cast<const uint4 *>(img + stride + off);
+          } else {
+            a = ld_cg_v4(img + off);
+            b = ld_cg_v4(img + stride + off);
+          }
           xh[4 * i] = a.x, xh[4 * i + 1] = a.y, xh[4 * i + 2] = a.z, xh[4 * i + 3] = a.w;
           xl[4 * i] = b.x, xl[4 * i + 1] = b.y, xl[4 * i + 2] = b.z, xl[4 * i + 3] = b.w;
         }
@@ -518,9 +659,8 @@ __global__ void __launch_bounds__(kK3Threads)
       float d[4] = {0.f, 0.f, 0.f, 0.f};
       group_mma_acc(ra, rb, xh, d);
       group_mma_acc(ra, rb, xl, d);
-      const uint16_t *sc = reinterpret_cast<const uint16_t *>(sbase);
-      const float s0 = bf16_bits_to_f32(sc[g * ngroups + G]);
-      const float s1 = bf16_bits_to_f32(sc[(g + 8) * ngroups + G]);
+      const float s0 = bf16_bits_to_f32(sc[g * spr + G]);
+      const float s1 = bf16_bits_to_f32(sc[(g + 8) * spr + G]);
       acc[0] = fmaf(d[0], s0, acc[0]);
       acc[1] = fmaf(d[1], s0, acc[1]);
       acc[2] = fmaf(d[2], s1, acc[2]);
@@ -530,12 +670,12 @@ __global__ void __launch_bounds__(kK3Threads)
     for (int c = 0; c < 2; ++c) {
       const int b = 2 * t + c;
       if (b < B && ((mask >> b) & 1u)) {
-        int j = kTopK;
+        int j = kTopK + half;  // shared halves: 6, 7
         if (!sh)
           for (int jj = 0; jj < kTopK; ++jj)
-            if (ld_cg_u32(asc_slot + b * kTopK + jj) == (uint32_t)task) j = jj;
-        ysel[(b * 7 + j) * 16 + g] = acc[c];
-        ysel[(b * 7 + j) * 16 + g + 8] = acc[2 + c];
+            if (s_asc[b * kTopK + jj] == task) j = jj;
+        ysel[(b * 8 + j) * 16 + g] = acc[c];
+        ysel[(b * 8 + j) * 16 + g + 8] = acc[2 + c];
       }
     }
   }
@@ -544,7 +684,7 @@ __global__ void __launch_bounds__(kK3Threads)
     const int n = tid & 15, b = tid >> 4;
     float y = 0.f;
 #pragma unroll
-    for (int j = 0; j < 7; ++j) y += ysel[(b * 7 + j) * 16 + n];
+    for (int j = 0; j < 8; ++j) y += ysel[(b * 8 + j) * 16 + n];
     const size_t o = (size_t)b * kH + n0 + n;
     if (kResidual) {
       const float yb = __bfloat162float(__float2bfloat16_rn(y));
@@ -556,8 +696,6 @@ __global__ void __launch_bounds__(kK3Threads)
 }
 
 // ============================================================== host
-static size_t k3_smem_bytes(int umax) { return (size_t)umax * (4096 + 128) + 8192 + 256 + 8 * 7 * 16 * 4; }
-
 template <typename... KArgs, typename... Args>
 static cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, size_t smem,
                               cudaStream_t st, Args... args) {
@@ -574,41 +712,64 @@ static cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, siz
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
+static int current_device() {
+  int d = 0;
+  cudaGetDevice(&d);
+  return d;
+}
+
+// dynamic shared memory cap: the 227 KB opt-in limit minus K3's static arrays
+constexpr size_t kK3MaxSmem = 224 * 1024;
+constexpr int kK1Smem = 16 * 2048 + kXFragBytes / 2;
+constexpr int kK2Smem = kItemBytes + kXFragBytes;  // item + compact fragment for B <= 8
+
 template <bool kResidual>
-static cudaError_t set_attrs_once() {
-  static bool done = false;  // per process; the attribute is per device function
-  static cudaError_t err = cudaSuccess;
-  if (!done) {
-    err = cudaFuncSetAttribute(k3_down_combine<kResidual>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)k3_smem_bytes(kTopK * kMaxB));
-    if (err == cudaSuccess)
-      err = cudaFuncSetAttribute(k1_route_shared<kResidual>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kXFragBytes);
-    if (err == cudaSuccess)
-      err = cudaFuncSetAttribute(k2_routed_gateup<kResidual>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kXFragBytes);
-    done = true;
-  }
-  return err;
+static cudaError_t set_attrs(int dev) {
+  static uint64_t done = 0;  // one bit per device
+  if (dev < 64 && ((done >> dev) & 1u)) return cudaSuccess;
+  note_step("k1_router smem attribute");
+  cudaError_t e = cudaFuncSetAttribute(k1_router<kResidual>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kK1Smem);
+  if (e == cudaSuccess)
+    e = noted(cudaFuncSetAttribute(k2_gateup<kResidual>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kK2Smem),
+              "k2_gateup smem attribute");
+  if (e == cudaSuccess)
+    e = noted(cudaFuncSetAttribute(k3_down_combine<kResidual, true>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kK3MaxSmem),
+              "k3 smem attribute");
+  if (e == cudaSuccess)
+    e = noted(cudaFuncSetAttribute(k3_down_combine<kResidual, false>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kK3MaxSmem),
+              "k3 (unstaged) smem attribute");
+  if (e == cudaSuccess && dev < 64) done |= uint64_t(1) << dev;
+  return e;
 }
 
 template <bool kResidual>
 static cudaError_t launch_decode_t(const LayerArgs &L, const uint16_t *x, float *h, int B,
                                    uint16_t *out, int32_t *idx_out, float *w_out, char *ws,
                                    cudaStream_t st, bool route_only) {
-  cudaError_t err = set_attrs_once<kResidual>();
+  cudaError_t err = set_attrs<kResidual>(current_device());
   if (err != cudaSuccess) return err;
   const DecodeLayout lay = decode_layout(B);
-  const int k1_grid = route_only ? kRouterCtas : kRouterCtas + kSharedCtas;
-  err = launch_pdl(k1_route_shared<kResidual>, k1_grid, kK1Threads, kXFragBytes, st, L, x,
+  note_step("k1_router launch");
+  err = launch_pdl(k1_router<kResidual>, kRouterCtas, kK1Threads, kK1Smem, st, L, x,
                    (const float *)h, B, ws, lay, idx_out, w_out);
   if (err != cudaSuccess || route_only) return err;
   const int umax = kTopK * B < kE ? kTopK * B : kE;
-  err = launch_pdl(k2_routed_gateup<kResidual>, umax * 16, kK2Threads, kXFragBytes, st, L, x, B,
-                   ws, lay);
+  const int n_items = kSharedItems + 64 * umax;
+  note_step("k2_gateup launch");
+  err = launch_pdl(k2_gateup<kResidual>, n_items, kK2Warps * 32,
+                   (size_t)kItemBytes + (size_t)16 * 4 * B * 64, st, L, x, (const float *)h, B, ws,
+                   lay);
   if (err != cudaSuccess) return err;
-  return launch_pdl(k3_down_combine<kResidual>, kH / 16, kK3Threads, k3_smem_bytes(umax), st, L,
+  const K3Smem P{umax, B};
+  note_step("k3_down_combine launch");
+  if (P.total(true) <= kK3MaxSmem)
+    return launch_pdl(k3_down_combine<kResidual, true>, kH / 16, kK3Threads, P.total(true), st,
+                      L, B, out, h, ws, lay, umax);
+  return launch_pdl(k3_down_combine<kResidual, false>, kH / 16, kK3Threads, P.total(false), st, L,
                     B, out, h, ws, lay, umax);
 }
 

@@ -1,20 +1,27 @@
 // Int4 GEMV with fused argmax for the output head ("How to Run Flint
-// Locally", section "One decode step in bytes": lm_head is 150,144 x 2,048
-// and is read in full for every token; Recursive quantized it to 4 bits).
+// Locally", section "One decode step in bytes": lm_head is 150,144 x 2,048,
+// read in full for every token; Recursive quantized it to 4 bits).
 //
-// One warp computes a 16-row tile against up to 8 activation columns with
-// mma.sync (see common.cuh); weights stream through registers with a few
-// groups in flight; the activation fragment sits in shared memory.  Each
-// warp keeps its best (value, row) per column; CTAs publish partials and the
-// last CTA to finish reduces them (lowest row on ties), so the whole call is
-// one launch.
+// Persistent kernel, one CTA per SM.  A producer warp streams whole 16-row
+// tiles (16 x K/2 bytes of codes plus their 16 x K/64 bytes of scales, both
+// contiguous) into a ring of shared-memory stages with 1-D bulk copies;
+// consumer warps take ring slots strictly in order from a shared counter and
+// run each tile against up to 8 activation columns on mma.sync (see
+// common.cuh).  There are never more consumers than stages, so a consumer
+// waits at most one phase ahead on a stage barrier (parity waits cannot
+// alias).  A final partial tile
+// (N % 16 rows) is read straight from global memory.  Each warp keeps its best
+// (value, row) per column; CTAs publish partials and the last CTA to finish
+// reduces them (lowest row on ties), so the call is one launch.
 #include "common.cuh"
 #include "internal.h"
 
 namespace flint {
 
-constexpr int kGemvThreads = 256;
-constexpr int kGemvNPre = 4;
+constexpr int kMaxConsumers = 16;
+constexpr int kGemvWarps = kMaxConsumers + 1;  // producer = the last warp launched
+constexpr size_t kGemvSmemCap = 200 * 1024;
+constexpr int kMaxGemvCtas = 1024;
 
 struct ArgPartial {
   float v;
@@ -27,102 +34,204 @@ FLINT_DEV bool better(float v, int i, float bv, int bi) {
   return bi < 0 ? (v == v) : (v > bv || (v == bv && i < bi));
 }
 
-size_t gemv_ws_bytes(int N, int B) {
-  const int tiles = (N + 15) / 16;
-  int grid = (tiles + 7) / 8;
-  if (grid > 148 * 4) grid = 148 * 4;
-  return align256(256) + align256(sizeof(ArgPartial) * (size_t)grid * B);
-}
-
 static int gemv_grid(int N) {
   const int tiles = (N + 15) / 16;
-  int grid = (tiles + 7) / 8;
-  return grid > 148 * 4 ? 148 * 4 : grid;
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (sms > kMaxGemvCtas) sms = kMaxGemvCtas;
+  return tiles < sms ? tiles : sms;
 }
 
-__global__ void __launch_bounds__(kGemvThreads)
-    k_int4_gemv(const uint8_t *__restrict__ q, const uint16_t *__restrict__ s, int N, int K,
-                const uint16_t *__restrict__ x, int B, float *__restrict__ y,
-                int32_t *__restrict__ argmax, char *__restrict__ ws) {
-  extern __shared__ uint4 xfrag[];
-  __shared__ ArgPartial s_part[kGemvThreads / 32][kMaxB];
-  __shared__ int s_last;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-  const int ngroups = K / kG;
-  uint32_t *ctrl = reinterpret_cast<uint32_t *>(ws);
-  ArgPartial *parts = reinterpret_cast<ArgPartial *>(ws + align256(256));
+size_t gemv_ws_bytes(int N, int B) {
+  (void)N;
+  return align256(256) + align256(sizeof(ArgPartial) * (size_t)kMaxGemvCtas * B);
+}
 
-  pdl_wait();
-  pdl_trigger();
-  build_x_frag(xfrag, ngroups, B, [&](int r) { return x + (size_t)r * K; }, tid, kGemvThreads);
-  __syncthreads();
+struct GemvPlan {
+  size_t stage_bytes, frag_bytes, smem;
+  int stages;
+};
 
-  float best_v[2] = {0.f, 0.f};
-  int best_i[2] = {-1, -1};
-  const int tiles = (N + 15) / 16;
-  const size_t rb = (size_t)K / 2;
-  for (int tile = blockIdx.x * 8 + warp; tile < tiles; tile += gridDim.x * 8) {
-    const int n_a = tile * 16 + g, n_b = n_a + 8;
-    const bool va = n_a < N, vb = n_b < N;
-    const uint8_t *pa = q + (size_t)(va ? n_a : 0) * rb + 16 * t;
-    const uint8_t *pb = q + (size_t)(vb ? n_b : 0) * rb + 16 * t;
-    const uint16_t *sa = s + (size_t)(va ? n_a : 0) * ngroups;
-    const uint16_t *sb = s + (size_t)(vb ? n_b : 0) * ngroups;
-    uint4 wa[kGemvNPre], wb[kGemvNPre];
-    uint32_t sva[kGemvNPre], svb[kGemvNPre];
+static GemvPlan gemv_plan(int K, int B) {
+  GemvPlan p;
+  p.stage_bytes = align256((size_t)8 * K + (size_t)K / 4);
+  p.frag_bytes = align256((size_t)(K / kG) * 4 * B * 64);
+  p.stages = (int)((kGemvSmemCap - p.frag_bytes) / p.stage_bytes);
+  if (p.stages > 16) p.stages = 16;
+  p.smem = p.frag_bytes + (size_t)p.stages * p.stage_bytes;
+  return p;
+}
+
+// Compact activation fragment: only the B live columns (lanes g < B) are
+// stored, frag[(G * 4B + g * 4 + t) * 4 + q] (uint4); other lanes read zeros.
+FLINT_DEV void load_frag_compact(const uint4 *frag, int G, int B, int lane, uint32_t (&x)[16]) {
+  const int g = lane >> 2, t = lane & 3;
+  if (g < B) {
+    const uint4 *p = frag + (size_t)(G * 4 * B + g * 4 + t) * 4;
 #pragma unroll
-    for (int G = 0; G < kGemvNPre; ++G) {
-      if (G < ngroups) {
-        wa[G] = ld_stream(pa + 64 * G);
-        wb[G] = ld_stream(pb + 64 * G);
-        sva[G] = ld_nc_u16(sa + G);
-        svb[G] = ld_nc_u16(sb + G);
-      }
+    for (int i = 0; i < 4; ++i) {
+      const uint4 v = p[i];
+      x[4 * i] = v.x, x[4 * i + 1] = v.y, x[4 * i + 2] = v.z, x[4 * i + 3] = v.w;
     }
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int G0 = 0; G0 < ngroups; G0 += kGemvNPre) {
+  } else {
 #pragma unroll
-      for (int k = 0; k < kGemvNPre; ++k) {
-        const int G = G0 + k;
-        if (G < ngroups) {
-          const uint4 w0 = wa[k], w1 = wb[k];
-          const float s0 = bf16_bits_to_f32(sva[k]), s1 = bf16_bits_to_f32(svb[k]);
-          if (G + kGemvNPre < ngroups) {
-            wa[k] = ld_stream(pa + 64 * (G + kGemvNPre));
-            wb[k] = ld_stream(pb + 64 * (G + kGemvNPre));
-            sva[k] = ld_nc_u16(sa + G + kGemvNPre);
-            svb[k] = ld_nc_u16(sb + G + kGemvNPre);
-          }
-          uint32_t ra[16], rbv[16], xb[16];
-          int4x32_to_bf16x2(w0, ra);
-          int4x32_to_bf16x2(w1, rbv);
-          load_frag(xfrag + (G * 32 + lane) * 4, xb);
-          float d[4];
-          group_mma(ra, rbv, xb, d);
-          acc[0] = fmaf(d[0], s0, acc[0]);
-          acc[1] = fmaf(d[1], s0, acc[1]);
-          acc[2] = fmaf(d[2], s1, acc[2]);
-          acc[3] = fmaf(d[3], s1, acc[3]);
-        }
-      }
+    for (int i = 0; i < 16; ++i) x[i] = 0u;
+  }
+}
+
+// Rows ra, rb (codes at row stride K/2 bytes, scales at row stride K/128)
+// against the fragment: acc[0..1] row ra, acc[2..3] row rb, columns 2t, 2t+1.
+template <bool kGlobal>
+FLINT_DEV void rows_dot(const uint8_t *qa, const uint8_t *qb, const uint16_t *sa,
+                        const uint16_t *sb, int K, int B, const uint4 *frag, int lane,
+                        float (&acc)[4]) {
+  const int t = lane & 3;
+  const int ng = K / kG;
+  acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+#pragma unroll 2
+  for (int G = 0; G < ng; ++G) {
+    uint4 w0, w1;
+    uint32_t s0b, s1b;
+    if (kGlobal) {
+      w0 = ld_stream(qa + 64 * G + 16 * t);
+      w1 = ld_stream(qb + 64 * G + 16 * t);
+      s0b = ld_nc_u16(sa + G);
+      s1b = ld_nc_u16(sb + G);
+    } else {
+      w0 = *reinterpret_cast<const uint4 *>(qa + 64 * G + 16 * t);
+      w1 = *reinterpret_cast<const uint4 *>(qb + 64 * G + 16 * t);
+      s0b = sa[G];
+      s1b = sb[G];
     }
+    uint32_t ra[16], rbv[16], xb[16];
+    int4x32_to_bf16x2(w0, ra);
+    int4x32_to_bf16x2(w1, rbv);
+    load_frag_compact(frag, G, B, lane, xb);
+    float d[4];
+    group_mma(ra, rbv, xb, d);
+    const float s0 = bf16_bits_to_f32(s0b), s1 = bf16_bits_to_f32(s1b);
+    acc[0] = fmaf(d[0], s0, acc[0]);
+    acc[1] = fmaf(d[1], s0, acc[1]);
+    acc[2] = fmaf(d[2], s1, acc[2]);
+    acc[3] = fmaf(d[3], s1, acc[3]);
+  }
+}
+
+FLINT_DEV void rows_store(const float (&acc)[4], int n_a, int n_b, int N, int B, float *y, int t,
+                          float (&best_v)[2], int (&best_i)[2]) {
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const int b = 2 * t + c;
-      if (b < B) {
-        if (va) {
-          y[(size_t)b * N + n_a] = acc[c];
-          if (better(acc[c], n_a, best_v[c], best_i[c])) best_v[c] = acc[c], best_i[c] = n_a;
-        }
-        if (vb) {
-          y[(size_t)b * N + n_b] = acc[2 + c];
-          if (better(acc[2 + c], n_b, best_v[c], best_i[c])) best_v[c] = acc[2 + c], best_i[c] = n_b;
-        }
+  for (int c = 0; c < 2; ++c) {
+    const int b = 2 * t + c;
+    if (b < B) {
+      if (n_a < N) {
+        y[(size_t)b * N + n_a] = acc[c];
+        if (better(acc[c], n_a, best_v[c], best_i[c])) best_v[c] = acc[c], best_i[c] = n_a;
+      }
+      if (n_b < N) {
+        y[(size_t)b * N + n_b] = acc[2 + c];
+        if (better(acc[2 + c], n_b, best_v[c], best_i[c])) best_v[c] = acc[2 + c], best_i[c] = n_b;
       }
     }
   }
-  if (!argmax) return;
+}
 
+__global__ void __launch_bounds__(kGemvWarps * 32, 1)
+    k_int4_gemv(const uint8_t *__restrict__ q, const uint16_t *__restrict__ s, int N, int K,
+                const uint16_t *__restrict__ x, int B, float *__restrict__ y,
+                int32_t *__restrict__ argmax, char *__restrict__ ws, int stages,
+                uint32_t stage_bytes, uint32_t frag_bytes) {
+  extern __shared__ __align__(128) unsigned char sm[];
+  uint4 *frag = reinterpret_cast<uint4 *>(sm);
+  unsigned char *ring = sm + frag_bytes;
+  __shared__ __align__(8) uint64_t full[16], empty[16];
+  __shared__ ArgPartial s_part[kGemvWarps][kMaxB];
+  __shared__ int s_last;
+  __shared__ int s_next;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const int ncons = (int)(blockDim.x >> 5) - 1, nthreads = (int)blockDim.x;
+  uint32_t *ctrl = reinterpret_cast<uint32_t *>(ws);
+  ArgPartial *parts = reinterpret_cast<ArgPartial *>(ws + align256(256));
+  const int full_tiles = N / 16;
+  const size_t rbytes = (size_t)K / 2;
+  const int ng = K / kG;
+  const uint32_t wbytes = (uint32_t)(8 * K), sbytes = (uint32_t)(K / 4);
+
+  if (tid == 0) {
+    s_next = 0;
+    for (int i = 0; i < stages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);  // each stage is released by the one warp that consumed it
+    }
+  }
+  __syncthreads();
+  bool failed = false;
+  float best_v[2] = {0.f, 0.f};
+  int best_i[2] = {-1, -1};
+
+  if (warp == ncons) {
+    // ---- producer: the weights do not depend on the previous kernel
+    if (lane == 0) {
+      int k = 0;
+      for (int tile = blockIdx.x; tile < full_tiles; tile += gridDim.x, ++k) {
+        const int st = k % stages;
+        if (k >= stages && !mbar_wait(&empty[st], ((k / stages) - 1) & 1)) {
+          failed = true;
+          break;
+        }
+        unsigned char *dst = ring + (size_t)st * stage_bytes;
+        mbar_expect_tx(&full[st], wbytes + sbytes);
+        bulk_g2s(dst, q + (size_t)tile * wbytes, wbytes, &full[st]);
+        bulk_g2s(dst + wbytes, reinterpret_cast<const unsigned char *>(s) + (size_t)tile * sbytes,
+                 sbytes, &full[st]);
+      }
+    }
+    pdl_wait();
+    pdl_trigger();
+  } else {
+    // ---- consumers
+    pdl_wait();
+    pdl_trigger();
+    const int nfrag = ng * 4 * B * 4;
+    for (int task = tid; task < nfrag; task += ncons * 32) {
+      const int q4 = task & 3, gt = (task >> 2) % (4 * B), G = (task >> 2) / (4 * B);
+      const int gg = gt >> 2, tt = gt & 3;
+      frag[task] = bf16x8_to_pairs(ld_cg_v4(x + (size_t)gg * K + 128 * G + 32 * tt + 8 * q4));
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(ncons * 32) : "memory");  // consumers only
+    const int my_tiles = full_tiles > (int)blockIdx.x
+                             ? (full_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
+                             : 0;
+    for (;;) {
+      int k = 0;
+      if (lane == 0) k = atomicAdd(&s_next, 1);
+      k = __shfl_sync(0xffffffffu, k, 0);
+      if (k >= my_tiles) break;
+      const int tile = (int)blockIdx.x + k * (int)gridDim.x;
+      const int st = k % stages;
+      if (!mbar_wait(&full[st], (k / stages) & 1)) {
+        failed = true;
+        break;
+      }
+      const unsigned char *src = ring + (size_t)st * stage_bytes;
+      const uint16_t *sc = reinterpret_cast<const uint16_t *>(src + wbytes);
+      float acc[4];
+      rows_dot<false>(src + g * rbytes, src + (g + 8) * rbytes, sc + g * ng, sc + (g + 8) * ng,
+                      K, B, frag, lane, acc);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+      rows_store(acc, tile * 16 + g, tile * 16 + g + 8, N, B, y, t, best_v, best_i);
+    }
+    // the partial last tile (N % 16 rows), straight from global memory
+    if (!failed && (N % 16) && warp == 0 && (int)blockIdx.x == full_tiles % (int)gridDim.x) {
+      const int n_a = full_tiles * 16 + g, n_b = n_a + 8;
+      const size_t ra = n_a < N ? (size_t)n_a : 0, rb = n_b < N ? (size_t)n_b : 0;
+      float acc[4];
+      rows_dot<true>(q + ra * rbytes, q + rb * rbytes, s + ra * ng, s + rb * ng, K, B, frag, lane,
+                     acc);
+      rows_store(acc, n_a, n_b, N, B, y, t, best_v, best_i);
+    }
+  }
   // lanes sharing t hold the same columns: reduce over g (xor 4, 8, 16)
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
@@ -130,16 +239,19 @@ __global__ void __launch_bounds__(kGemvThreads)
     for (int o = 4; o < 32; o <<= 1) {
       const float ov = __shfl_xor_sync(0xffffffffu, best_v[c], o);
       const int oi = __shfl_xor_sync(0xffffffffu, best_i[c], o);
-      if (oi >= 0 && better(ov, oi, best_v[c], best_i[c]))
-        best_v[c] = ov, best_i[c] = oi;
+      if (oi >= 0 && better(ov, oi, best_v[c], best_i[c])) best_v[c] = ov, best_i[c] = oi;
     }
     const int b = 2 * t + c;
     if (g == 0 && b < B) s_part[warp][b] = ArgPartial{best_v[c], best_i[c]};
   }
-  __syncthreads();
+  if (__syncthreads_or(failed)) {
+    if (tid == 0) set_status(ctrl + 1, kStatusTimeout);
+    return;
+  }
+  if (!argmax) return;
   if (tid < B) {
     ArgPartial p{0.f, -1};
-    for (int w = 0; w < kGemvThreads / 32; ++w) {
+    for (int w = 0; w <= ncons; ++w) {
       const ArgPartial o = s_part[w][tid];
       if (o.i >= 0 && better(o.v, o.i, p.v, p.i)) p = o;
     }
@@ -149,17 +261,35 @@ __global__ void __launch_bounds__(kGemvThreads)
   if (tid == 0) {
     __threadfence();
     const uint32_t prev = atomicAdd(&ctrl[0], 1u);
-    s_last = (prev == gridDim.x - 1);
+    const bool last = prev == gridDim.x - 1;
+    if (last) __threadfence();
+    s_last = last;
   }
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
+  // last CTA: every thread scans a strided share of the CTA partials, then
+  // warps and the CTA reduce (order-free: lowest row wins ties).
+  for (int b = 0; b < B; ++b) {
+    ArgPartial p{0.f, -1};
+    for (int cta = tid; cta < (int)gridDim.x; cta += nthreads) {
+      const float ov = ld_cg_f32(&parts[(size_t)cta * B + b].v);
+      const int oi = (int)ld_cg_u32(&parts[(size_t)cta * B + b].i);
+      if (oi >= 0 && better(ov, oi, p.v, p.i)) p = ArgPartial{ov, oi};
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, p.v, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, p.i, o);
+      if (oi >= 0 && better(ov, oi, p.v, p.i)) p = ArgPartial{ov, oi};
+    }
+    if (lane == 0) s_part[warp][b] = p;
+  }
+  __syncthreads();
   if (tid < B) {
     ArgPartial p{0.f, -1};
-    for (int cta = 0; cta < (int)gridDim.x; ++cta) {
-      const float ov = ld_cg_f32(&parts[(size_t)cta * B + tid].v);
-      const int oi = (int)ld_cg_u32(&parts[(size_t)cta * B + tid].i);
-      if (oi >= 0 && better(ov, oi, p.v, p.i)) p = ArgPartial{ov, oi};
+    for (int w = 0; w <= ncons; ++w) {
+      const ArgPartial o = s_part[w][tid];
+      if (o.i >= 0 && better(o.v, o.i, p.v, p.i)) p = o;
     }
     argmax[tid] = p.i;
   }
@@ -168,25 +298,27 @@ __global__ void __launch_bounds__(kGemvThreads)
 
 cudaError_t launch_gemv(const uint8_t *q, const uint16_t *s, int N, int K, const uint16_t *x,
                         int B, float *y, int32_t *argmax, char *ws, cudaStream_t st) {
-  const size_t smem = (size_t)(K / kG) * 128 * 16;
-  static int configured = 0;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(k_int4_gemv, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (8192 / kG) * 128 * 16);
-    if (e != cudaSuccess) return e;
-    configured = 1;
-  }
+  const GemvPlan p = gemv_plan(K, B);
+  note_step("k_int4_gemv plan");
+  if (p.stages < 2) return cudaErrorInvalidValue;
+  note_step("k_int4_gemv smem attribute");
+  cudaError_t e = cudaFuncSetAttribute(k_int4_gemv, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kGemvSmemCap);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(gemv_grid(N));
-  cfg.blockDim = dim3(kGemvThreads);
-  cfg.dynamicSmemBytes = smem;
+  const int ncons = p.stages < kMaxConsumers ? p.stages : kMaxConsumers;
+  cfg.blockDim = dim3((ncons + 1) * 32);
+  cfg.dynamicSmemBytes = p.smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_int4_gemv, q, s, N, K, x, B, y, argmax, ws);
+  note_step("k_int4_gemv launch");
+  return cudaLaunchKernelEx(&cfg, k_int4_gemv, q, s, N, K, x, B, y, argmax, ws, p.stages,
+                            (uint32_t)p.stage_bytes, (uint32_t)p.frag_bytes);
 }
 
 }  // namespace flint
