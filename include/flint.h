@@ -179,6 +179,31 @@ FLINT_API int flint_moe_prefill(const flint_moe_layer *layer, const uint16_t *x,
 FLINT_API int flint_int4_gemv(const uint8_t *q, const uint16_t *s, int N, int K, const uint16_t *x, int B,
                     float *y, int32_t *argmax, void *ws, size_t ws_bytes, void *stream);
 
+/*
+ * flint_int4_gemv without a workspace, for callers that cannot allocate
+ * device memory themselves: code embedded in a host program that owns every
+ * device allocation (and forbids cudaMalloc from libraries), or a hot path
+ * whose memory budget is fixed up front and that must not fail or stall on an
+ * allocation.  The pages have no counterpart: this entry point is an
+ * integration convenience, not part of the method.
+ *
+ * Same arguments, results and errors as flint_int4_gemv, minus `ws`.  The
+ * scratch (a counter, a status word and per-CTA argmax partials) is a
+ * 65,792-byte array inside the library, one per GPU that loads it, kept until
+ * the process exits; calls whose scratch would not fit are rejected with
+ * FLINT_EINVAL (none with B <= 8 do).  Nothing is allocated: the call clears
+ * the counter and status word with an asynchronous memset on `stream`, then
+ * launches.  The first call on a device looks the array's device address up
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * first call before any stream capture.  All calls on a device share the one
+ * array and it keeps the last call's contents, so calls that may overlap on
+ * the GPU (different streams without ordering between them) race and must
+ * not be issued; order them on one stream.
+ */
+FLINT_API int flint_int4_gemv_noalloc(const uint8_t *q, const uint16_t *s, int N, int K,
+                                      const uint16_t *x, int B, float *y, int32_t *argmax,
+                                      void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -21,7 +21,7 @@ HIDDEN, EXPERTS, TOP_K, EXPERT_I, SHARED_I, GROUP, MAX_DECODE_B = 2048, 256, 6, 
 EXPORTS = ("flint_version", "flint_strerror", "flint_last_cuda_error", "flint_workspace_bytes",
            "flint_gemv_workspace_bytes", "flint_workspace_init", "flint_read_status",
            "flint_moe_route", "flint_moe_decode", "flint_moe_decode_residual",
-           "flint_moe_prefill", "flint_int4_gemv")
+           "flint_moe_prefill", "flint_int4_gemv", "flint_int4_gemv_noalloc")
 
 _lib = None
 
@@ -68,6 +68,7 @@ def lib() -> C.CDLL:
         L.flint_moe_decode_residual.argtypes = [lp, vp, i, vp, vp, vp, sz, vp]
         L.flint_moe_prefill.argtypes = [lp, vp, i, vp, vp, sz, vp]
         L.flint_int4_gemv.argtypes = [vp, vp, i, i, vp, i, vp, vp, vp, sz, vp]
+        L.flint_int4_gemv_noalloc.argtypes = [vp, vp, i, i, vp, i, vp, vp, vp]
         for name in EXPORTS:
             getattr(L, name).restype = getattr(L, name).restype or i
         _lib = L
@@ -155,3 +156,9 @@ def flint_moe_prefill(layer: flint_moe_layer, x, T: int, out, ws, ws_bytes: int,
 def flint_int4_gemv(q, s, N: int, K: int, x, B: int, y, argmax, ws, ws_bytes: int, stream=None):
     _check(lib().flint_int4_gemv(_ptr(q), _ptr(s), N, K, _ptr(x), B, _ptr(y), _ptr(argmax),
                                  _ptr(ws), ws_bytes, _stream(stream)), "flint_int4_gemv")
+
+
+def flint_int4_gemv_noalloc(q, s, N: int, K: int, x, B: int, y, argmax, stream=None):
+    """flint_int4_gemv with the library's own static scratch (no workspace)."""
+    _check(lib().flint_int4_gemv_noalloc(_ptr(q), _ptr(s), N, K, _ptr(x), B, _ptr(y),
+                                         _ptr(argmax), _stream(stream)), "flint_int4_gemv_noalloc")

@@ -33,6 +33,8 @@ int from_cuda(cudaError_t e) {
 
 }  // namespace
 
+int flint_from_cuda(cudaError_t e) { return from_cuda(e); }
+
 namespace flint {
 void note_step(const char *where) { g_step = where; }
 cudaError_t noted(cudaError_t e, const char *where) {

@@ -13,6 +13,8 @@
 // (N % 16 rows) is read straight from global memory.  Each warp keeps its best
 // (value, row) per column; CTAs publish partials and the last CTA to finish
 // reduces them (lowest row on ties), so the call is one launch.
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -322,3 +324,58 @@ cudaError_t launch_gemv(const uint8_t *q, const uint16_t *s, int N, int K, const
 }
 
 }  // namespace flint
+
+// ------------------------------------------------------------------------
+// Allocation-free variant.  The scratch the GEMV needs (completion counter,
+// status word, one argmax partial per CTA and row) lives in this file-scope
+// device array instead of a caller workspace.  Every GPU that loads the
+// library holds it until the process exits.  In host code the array's name is
+// only a host-side stand-in, so its device address is looked up once per
+// device (cudaGetSymbolAddress, on the first call made with that device
+// current) and cached.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 256 + 8 * 1024 * 8;  // counter/status + 1024 CTAs x 8 rows
+static __device__ __align__(256) unsigned char g_gemv_scratch[kNoAllocScratchBytes];
+
+std::mutex g_scratch_mu;
+void *g_scratch_ptr[64] = {};
+
+// Device address of g_gemv_scratch on the current device (looked up once).
+cudaError_t scratch_address(void **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void *ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_gemv_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = ptr;
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" FLINT_API int flint_int4_gemv_noalloc(const uint8_t *q, const uint16_t *s, int N,
+                                                  int K, const uint16_t *x, int B, float *y,
+                                                  int32_t *argmax, void *stream) {
+  auto aligned16 = [](const void *p) {
+    return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+  };
+  if (!aligned16(q) || !aligned16(s) || !aligned16(x) || !aligned16(y) || N < 1 || K < 128 ||
+      K % 128 || K > 8192 || B < 1 || B > FLINT_MAX_DECODE_B)
+    return FLINT_EINVAL;
+  if (flint::gemv_ws_bytes(N, B) > kNoAllocScratchBytes) return FLINT_EINVAL;  // cannot happen for B <= 8
+  void *scratch = nullptr;
+  cudaError_t e = flint::noted(scratch_address(&scratch), "no-alloc scratch address");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the counter and status word must start at zero; the partials need not
+  if (e == cudaSuccess) e = flint::noted(cudaMemsetAsync(scratch, 0, 256, st), "no-alloc scratch clear");
+  if (e == cudaSuccess)
+    e = flint::launch_gemv(q, s, N, K, x, B, y, argmax, static_cast<char *>(scratch), st);
+  return flint_from_cuda(e);
+}

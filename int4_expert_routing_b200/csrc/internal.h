@@ -62,6 +62,13 @@ inline LayerArgs layer_args(const flint_moe_layer *l) {
 void note_step(const char *where);
 cudaError_t noted(cudaError_t e, const char *where);
 
+}  // namespace flint
+
+// FLINT_OK, or FLINT_ECUDA after recording e for flint_last_cuda_error.
+int flint_from_cuda(cudaError_t e);
+
+namespace flint {
+
 // Launchers (return a cudaError_t from the launches).
 cudaError_t launch_decode(const LayerArgs &L, const uint16_t *x, const float *h_in, float *h_out,
                           int B, uint16_t *out, int32_t *idx_out, float *w_out, char *ws,
