@@ -53,6 +53,7 @@ extern "C" {
 #define FLINT_SHARED_I 1024
 #define FLINT_GROUP 128
 #define FLINT_MAX_DECODE_B 8
+#define FLINT_MAX_PREFILL_T (1 << 20)
 #define FLINT_RMS_EPS 1e-6
 
 enum {
@@ -123,8 +124,11 @@ FLINT_API int flint_read_status(const void *ws, int *status, void *stream);
  *   s = sigmoid(z) (fp32);  b = s + router_b (fp32)
  *   idx[r][0..5] = the 6 largest b, largest first; equal b -> lower index
  *   w[r][j] = s[idx[r][j]] / sum_j s[idx[r][j]]   (fp32)
- *   x    bf16 [B][2048];  idx int32 [B][6];  w fp32 [B][6];  B >= 1
+ *   x    bf16 [B][2048];  idx int32 [B][6];  w fp32 [B][6];  1 <= B <= 2^20
  *   ws   workspace of flint_workspace_bytes(FLINT_OP_ROUTE, B)
+ * B <= 8 uses the decode router; larger B the prefill router (tensor-core
+ * tiles over tokens); both sum bf16 products in fp32 per 128-wide k-group and
+ * the groups in fp64, so they select the same experts up to near-ties.
  */
 FLINT_API int flint_moe_route(const flint_moe_layer *layer, const uint16_t *x, int B, int32_t *idx,
                     float *w, void *ws, size_t ws_bytes, void *stream);
@@ -161,8 +165,10 @@ FLINT_API int flint_moe_decode_residual(const flint_moe_layer *layer, float *h, 
  * token-by-expert sort, grouped GEMMs on the tensor cores (weights
  * dequantized to bf16 tiles in shared memory; bf16 SwiGLU intermediate) and a
  * fixed-order combine.
- *   x bf16 [T][2048];  out bf16 [T][2048]
- *   ws workspace of flint_workspace_bytes(FLINT_OP_PREFILL, T)
+ *   x bf16 [T][2048];  out bf16 [T][2048] (may not alias x);  1 <= T <= 2^20
+ *   ws workspace of flint_workspace_bytes(FLINT_OP_PREFILL, T) (about 70 KB
+ *      per token: routing tables, the gathered rows, the SwiGLU and expert
+ *      outputs)
  */
 FLINT_API int flint_moe_prefill(const flint_moe_layer *layer, const uint16_t *x, int T, uint16_t *out,
                       void *ws, size_t ws_bytes, void *stream);

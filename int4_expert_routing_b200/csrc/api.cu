@@ -68,8 +68,11 @@ size_t flint_workspace_bytes(int op, int n) {
   if (n < 1) return 0;
   switch (op) {
     case FLINT_OP_ROUTE:
+      return n <= FLINT_MAX_DECODE_B ? decode_layout(n).total : prefill_layout(n).route_total;
     case FLINT_OP_DECODE:
       return n <= FLINT_MAX_DECODE_B ? decode_layout(n).total : 0;
+    case FLINT_OP_PREFILL:
+      return n <= FLINT_MAX_PREFILL_T ? prefill_layout(n).total : 0;
     case FLINT_OP_GEMV:
       return 0;  // depends on N: flint_gemv_workspace_bytes
     default:
@@ -100,9 +103,12 @@ int flint_read_status(const void *ws, int *status, void *stream) {
 
 int flint_moe_route(const flint_moe_layer *layer, const uint16_t *x, int B, int32_t *idx,
                     float *w, void *ws, size_t ws_bytes, void *stream) {
-  if (!layer_ok(layer) || !aligned16(x) || !idx || !w || B < 1 || B > FLINT_MAX_DECODE_B ||
+  if (!layer_ok(layer) || !aligned16(x) || !idx || !w || B < 1 || B > FLINT_MAX_PREFILL_T ||
       !aligned16(ws) || ws_bytes < flint_workspace_bytes(FLINT_OP_ROUTE, B))
     return FLINT_EINVAL;
+  if (B > FLINT_MAX_DECODE_B)
+    return from_cuda(launch_route_many(layer_args(layer), x, B, idx, w, static_cast<char *>(ws),
+                                       static_cast<cudaStream_t>(stream)));
   return from_cuda(launch_decode(layer_args(layer), x, nullptr, nullptr, B, nullptr, idx, w,
                                  static_cast<char *>(ws), static_cast<cudaStream_t>(stream),
                                  true));
@@ -143,8 +149,12 @@ int flint_int4_gemv(const uint8_t *q, const uint16_t *s, int N, int K, const uin
 
 int flint_moe_prefill(const flint_moe_layer *layer, const uint16_t *x, int T, uint16_t *out,
                       void *ws, size_t ws_bytes, void *stream) {
-  (void)layer, (void)x, (void)T, (void)out, (void)ws, (void)ws_bytes, (void)stream;
-  return FLINT_EINVAL;  // prefill path: not built yet
+  if (!layer_ok(layer) || !aligned16(x) || !aligned16(out) || T < 1 || T > FLINT_MAX_PREFILL_T ||
+      !aligned16(ws) || ws_bytes < flint_workspace_bytes(FLINT_OP_PREFILL, T) ||
+      static_cast<const void *>(x) == static_cast<const void *>(out))
+    return FLINT_EINVAL;
+  return from_cuda(launch_prefill(layer_args(layer), x, T, out, static_cast<char *>(ws),
+                                  static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

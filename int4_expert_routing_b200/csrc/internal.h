@@ -39,6 +39,59 @@ inline DecodeLayout decode_layout(int B) {
   return L;
 }
 
+// Prefill workspace for T tokens (token tile of 128 per expert group).
+// ctrl words: [1] status, [3] GEMM1 tile count, [4] GEMM2 tile count,
+// [5] routed rows (padded).
+constexpr int kPfTile = 128;
+constexpr int kPfChunk = 256;
+struct PrefillLayout {
+  size_t ctrl, z, sel_idx, sel_w, asc_e, asc_w, route_total;
+  size_t pos, chunk_cnt, chunk_off, ebase, ecount, perm, pw, tiles1, tiles2, xp, hr, hs, yw, ys,
+      total;
+  int mr_max, max_tiles1, max_tiles2, nchunks;
+};
+
+inline PrefillLayout prefill_layout(int T) {
+  PrefillLayout L{};
+  L.nchunks = (T + kPfChunk - 1) / kPfChunk;
+  // at most min(256, 6T) experts hold tokens; each group is padded to the tile
+  const int busy = 6 * T < 256 ? 6 * T : 256;
+  L.mr_max = 6 * T + busy * (kPfTile - 1);
+  const int nsh = (T + kPfTile - 1) / kPfTile;
+  const int nrt = (6 * T) / kPfTile + busy;  // routed 128-token tiles, upper bound
+  L.max_tiles1 = 8 * nrt + 16 * nsh;
+  L.max_tiles2 = 16 * nrt + 16 * nsh;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = o;
+    o = align256(o + bytes);
+    return at;
+  };
+  L.ctrl = take(256);
+  L.z = take(sizeof(float) * (size_t)T * 256);
+  L.sel_idx = take(sizeof(int32_t) * (size_t)T * 6);
+  L.sel_w = take(sizeof(float) * (size_t)T * 6);
+  L.asc_e = take(sizeof(int32_t) * (size_t)T * 6);
+  L.asc_w = take(sizeof(float) * (size_t)T * 6);
+  L.route_total = o;
+  L.pos = take(sizeof(int32_t) * (size_t)T * 6);
+  L.chunk_cnt = take(sizeof(int32_t) * (size_t)L.nchunks * 256);
+  L.chunk_off = take(sizeof(int32_t) * (size_t)L.nchunks * 256);
+  L.ebase = take(sizeof(int32_t) * 257);
+  L.ecount = take(sizeof(int32_t) * 256);
+  L.perm = take(sizeof(int32_t) * (size_t)L.mr_max);
+  L.pw = take(sizeof(float) * (size_t)L.mr_max);
+  L.tiles1 = take(sizeof(int32_t) * (size_t)L.max_tiles1);
+  L.tiles2 = take(sizeof(int32_t) * (size_t)L.max_tiles2);
+  L.xp = take(sizeof(uint16_t) * (size_t)L.mr_max * 2048);
+  L.hr = take(sizeof(uint16_t) * (size_t)L.mr_max * 512 * 2);  // SwiGLU hi, lo
+  L.hs = take(sizeof(uint16_t) * (size_t)T * 1024 * 2);
+  L.yw = take(sizeof(uint16_t) * (size_t)L.mr_max * 2048);
+  L.ys = take(sizeof(uint16_t) * (size_t)T * 2048);
+  L.total = o;
+  return L;
+}
+
 struct LayerArgs {
   const uint16_t *router_w;
   const float *router_b;
@@ -76,5 +129,9 @@ cudaError_t launch_decode(const LayerArgs &L, const uint16_t *x, const float *h_
 cudaError_t launch_gemv(const uint8_t *q, const uint16_t *s, int N, int K, const uint16_t *x,
                         int B, float *y, int32_t *argmax, char *ws, cudaStream_t st);
 size_t gemv_ws_bytes(int N, int B);
+cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_t *out, char *ws,
+                           cudaStream_t st);
+cudaError_t launch_route_many(const LayerArgs &L, const uint16_t *x, int T, int32_t *idx, float *w,
+                              char *ws, cudaStream_t st);
 
 }  // namespace flint

@@ -1,0 +1,778 @@
+// Prefill of the Flint MoE block for T tokens.
+//
+// The block is defined per token ("How to Run Flint Locally", section "The
+// architecture, from config.json"); for many tokens it is computed as
+//   1. router logits for all tokens (bf16 products on mma.sync, fp32
+//      partials of each 128-wide k-group summed in fp64) and a per-token
+//      top-6 with the same selection rule as decode;
+//   2. a stable token-by-expert counting sort: per-chunk bitmask counts, one
+//      scan over (expert, chunk), then positions in token order inside every
+//      expert; each expert's group is padded to the 128-token tile;
+//   3. a gather of the routed token rows;
+//   4. grouped GEMM 1 (gate/up + SwiGLU) and grouped GEMM 2 (down, scaled by
+//      the routing weight) on the tcgen05 tensor cores: the weights are the
+//      128-row A operand, their int4 codes land in shared memory by TMA and
+//      four warps dequantize them to bf16 tiles in the 128-byte-swizzled
+//      K-major layout the MMA reads; the tokens are the N operand, loaded by
+//      TMA; the fp32 accumulator lives in tensor memory.  The shared expert
+//      is one more group that covers every token;
+//   5. a fixed-order combine per token (its experts in ascending index, then
+//      the shared expert).
+// "What vLLM changed" on the same page: the small-batch MoE kernels that read
+// only the selected experts were also the largest prefill gain.  SwiGLU
+// intermediates are bf16 (their range: TandemLLM "21 Flint", section 21.2
+// reports routed activations up to 2.6e5, past fp16).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace flint {
+
+// ============================================================== router (T tokens)
+constexpr int kRtTok = 64;  // tokens per CTA (8 column blocks of 8)
+
+__global__ void __launch_bounds__(256)
+    k_pf_router(LayerArgs L, const uint16_t *__restrict__ x, int T, float *__restrict__ z) {
+  extern __shared__ __align__(128) unsigned char sm[];
+  uint4 *frag = reinterpret_cast<uint4 *>(sm);  // [8 groups][8 blocks][32 lanes][4]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const int t0 = blockIdx.x * kRtTok, e0 = 128 * blockIdx.y + 16 * warp;
+  double acc[8][4];
+#pragma unroll
+  for (int nb = 0; nb < 8; ++nb)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[nb][i] = 0.0;
+
+  for (int half = 0; half < 2; ++half) {
+    __syncthreads();
+    for (int task = tid; task < 8 * 8 * 32 * 4; task += 256) {
+      const int q = task & 3, ln = (task >> 2) & 31, nb = (task >> 7) & 7, Gl = task >> 10;
+      const int tok = t0 + 8 * nb + (ln >> 2);
+      const int k0 = 128 * (8 * half + Gl) + 32 * (ln & 3) + 8 * q;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (tok < T) v = ld_cg_v4(x + (size_t)tok * kH + k0);
+      frag[task] = bf16x8_to_pairs(v);
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int Gl = 0; Gl < 8; ++Gl) {
+      const int G = 8 * half + Gl;
+      const uint16_t *ra = L.router_w + (size_t)(e0 + g) * kH + 128 * G + 32 * t;
+      uint32_t a[16], b[16];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 p0 = bf16x8_to_pairs(ld_stream(ra + 8 * q));
+        const uint4 p1 = bf16x8_to_pairs(ld_stream(ra + 8 * kH + 8 * q));
+        a[4 * q] = p0.x, a[4 * q + 1] = p0.y, a[4 * q + 2] = p0.z, a[4 * q + 3] = p0.w;
+        b[4 * q] = p1.x, b[4 * q + 1] = p1.y, b[4 * q + 2] = p1.z, b[4 * q + 3] = p1.w;
+      }
+#pragma unroll
+      for (int nb = 0; nb < 8; ++nb) {
+        uint32_t xb[16];
+        load_frag(frag + ((Gl * 8 + nb) * 32 + lane) * 4, xb);
+        float d[4];
+        group_mma(a, b, xb, d);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[nb][i] += (double)d[i];
+      }
+    }
+  }
+#pragma unroll
+  for (int nb = 0; nb < 8; ++nb)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int tok = t0 + 8 * nb + 2 * t + c;
+      if (tok < T) {
+        z[(size_t)tok * kE + e0 + g] = (float)acc[nb][c];
+        z[(size_t)tok * kE + e0 + g + 8] = (float)acc[nb][2 + c];
+      }
+    }
+}
+
+// One warp per token: sigmoid, bias, top-6 (lower index wins ties), weights;
+// selection order to sel_*, ascending expert order to asc_*.
+__global__ void __launch_bounds__(256)
+    k_pf_topk(const float *__restrict__ router_b, const float *__restrict__ z, int T,
+              int32_t *__restrict__ sel_idx, float *__restrict__ sel_w, int32_t *__restrict__ asc_e,
+              float *__restrict__ asc_w) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tok = blockIdx.x * 8 + warp;
+  if (tok >= T) return;
+  float sv[8];
+  uint32_t key[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float zf = z[(size_t)tok * kE + lane + 32 * i];
+    const float s = 1.f / (1.f + expf(-zf));
+    sv[i] = s;
+    key[i] = float_key(s + router_b[lane + 32 * i]);
+  }
+  uint32_t taken = 0;
+  int sel_e[kTopK];
+  float sel_s[kTopK];
+#pragma unroll
+  for (int j = 0; j < kTopK; ++j) {
+    uint32_t best = 0;
+    int bi = -1;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (!((taken >> i) & 1u) && key[i] > best) best = key[i], bi = i;
+    const uint32_t m = __reduce_max_sync(0xffffffffu, best);
+    const uint32_t cand = (bi >= 0 && best == m) ? (uint32_t)(lane + 32 * bi) : 0xffffffffu;
+    const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
+    float mys = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (i == bi) mys = sv[i];
+    sel_s[j] = __shfl_sync(0xffffffffu, mys, (int)(win & 31));
+    sel_e[j] = (int)win;
+    if (lane == (int)(win & 31)) taken |= 1u << (win >> 5);
+  }
+  float ssum = 0.f;
+#pragma unroll
+  for (int j = 0; j < kTopK; ++j) ssum += sel_s[j];
+  if (lane < kTopK) {
+    int e_me = sel_e[0];
+    float s_me = sel_s[0];
+#pragma unroll
+    for (int j = 1; j < kTopK; ++j)
+      if (lane == j) e_me = sel_e[j], s_me = sel_s[j];
+    const float w_me = s_me / ssum;
+    sel_idx[(size_t)tok * kTopK + lane] = e_me;
+    sel_w[(size_t)tok * kTopK + lane] = w_me;
+    int rank = 0;
+#pragma unroll
+    for (int j = 0; j < kTopK; ++j) rank += sel_e[j] < e_me;
+    if (asc_e) {
+      asc_e[(size_t)tok * kTopK + rank] = e_me;
+      asc_w[(size_t)tok * kTopK + rank] = w_me;
+    }
+  }
+}
+
+// ============================================================== stable sort by expert
+// Per chunk of 256 tokens (one per thread), bits[e][w] has bit `lane` set when
+// token 32w + lane of the chunk chose expert e.
+FLINT_DEV void chunk_bits(const int32_t *asc_e, int T, int c, uint32_t (*bits)[8]) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < kE * 8; i += 256) bits[i >> 3][i & 7] = 0u;
+  __syncthreads();
+  const int tok = c * kPfChunk + tid;
+  if (tok < T)
+    for (int j = 0; j < kTopK; ++j) atomicOr(&bits[asc_e[(size_t)tok * kTopK + j]][warp], 1u << lane);
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(256)
+    k_pf_count(const int32_t *__restrict__ asc_e, int T, int32_t *__restrict__ chunk_cnt) {
+  __shared__ uint32_t bits[kE][8];
+  chunk_bits(asc_e, T, blockIdx.x, bits);
+  const int e = threadIdx.x;
+  int n = 0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) n += __popc(bits[e][w]);
+  chunk_cnt[(size_t)blockIdx.x * kE + e] = n;
+}
+
+// exclusive scan of one value per thread over a 256-thread block; returns the
+// prefix and writes the total to *total
+FLINT_DEV int block_scan(int v, int *s_warp, int *total) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  int off = 0, tot = 0;
+  for (int w = 0; w < 8; ++w) {
+    if (w < warp) off += s_warp[w];
+    tot += s_warp[w];
+  }
+  __syncthreads();
+  *total = tot;
+  return off + incl - v;
+}
+
+FLINT_DEV uint32_t pack_tile(int e, int mt, int nt) {
+  return (uint32_t)e | ((uint32_t)mt << 9) | ((uint32_t)nt << 14);
+}
+
+// One CTA of 256 threads (one per expert): chunk offsets, expert counts,
+// padded bases, padding rows of the permutation, and both GEMM tile lists
+// (the 16 or 8 row tiles of one token tile are adjacent, so the token tile is
+// reused from L2).
+__global__ void __launch_bounds__(256)
+    k_pf_scan(int T, int nchunks, const int32_t *__restrict__ chunk_cnt,
+              int32_t *__restrict__ chunk_off, int32_t *__restrict__ ebase,
+              int32_t *__restrict__ ecount, int32_t *__restrict__ perm,
+              uint32_t *__restrict__ tiles1, uint32_t *__restrict__ tiles2,
+              uint32_t *__restrict__ ctrl) {
+  __shared__ int s_warp[8];
+  const int e = threadIdx.x;
+  int off = 0;
+#pragma unroll 8
+  for (int c = 0; c < nchunks; ++c) {
+    chunk_off[(size_t)c * kE + e] = off;
+    off += chunk_cnt[(size_t)c * kE + e];
+  }
+  ecount[e] = off;
+  const int ntile = (off + kPfTile - 1) / kPfTile;
+  int total_rows, total1, total2;
+  const int base = block_scan(ntile * kPfTile, s_warp, &total_rows);
+  const int o1 = block_scan(8 * ntile, s_warp, &total1);
+  const int o2 = block_scan(16 * ntile, s_warp, &total2);
+  ebase[e] = base;
+  if (e == 0) ebase[kE] = total_rows;
+  for (int p = base + off; p < base + ntile * kPfTile; ++p) perm[p] = -1;
+  for (int nt = 0; nt < ntile; ++nt) {
+    for (int mt = 0; mt < 8; ++mt) tiles1[o1 + nt * 8 + mt] = pack_tile(e, mt, nt);
+    for (int mt = 0; mt < 16; ++mt) tiles2[o2 + nt * 16 + mt] = pack_tile(e, mt, nt);
+  }
+  // the shared expert: one group over all T tokens
+  const int nsh = (T + kPfTile - 1) / kPfTile;
+  for (int i = e; i < 16 * nsh; i += kE) {
+    tiles1[total1 + i] = pack_tile(kE, i & 15, i >> 4);
+    tiles2[total2 + i] = pack_tile(kE, i & 15, i >> 4);
+  }
+  if (e == 0) {
+    ctrl[3] = (uint32_t)(total1 + 16 * nsh);
+    ctrl[4] = (uint32_t)(total2 + 16 * nsh);
+    ctrl[5] = (uint32_t)total_rows;
+  }
+}
+
+__global__ void __launch_bounds__(256)
+    k_pf_place(const int32_t *__restrict__ asc_e, const float *__restrict__ asc_w, int T,
+               const int32_t *__restrict__ chunk_off, const int32_t *__restrict__ ebase,
+               int32_t *__restrict__ pos, int32_t *__restrict__ perm, float *__restrict__ pw) {
+  __shared__ uint32_t bits[kE][8];
+  const int c = blockIdx.x;
+  chunk_bits(asc_e, T, c, bits);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tok = c * kPfChunk + tid;
+  if (tok >= T) return;
+  for (int j = 0; j < kTopK; ++j) {
+    const int e = asc_e[(size_t)tok * kTopK + j];
+    int rank = __popc(bits[e][warp] & ((1u << lane) - 1u));
+    for (int w = 0; w < warp; ++w) rank += __popc(bits[e][w]);
+    const int p = ebase[e] + chunk_off[(size_t)c * kE + e] + rank;
+    pos[(size_t)tok * kTopK + j] = p;
+    perm[p] = tok;
+    pw[p] = asc_w[(size_t)tok * kTopK + j];
+  }
+}
+
+// Routed token rows in sorted order; padding rows are zero.
+__global__ void __launch_bounds__(256)
+    k_pf_gather(const uint16_t *__restrict__ x, const int32_t *__restrict__ perm,
+                const uint32_t *__restrict__ ctrl, uint16_t *__restrict__ xp) {
+  const size_t rows = __ldcg(ctrl + 5);
+  const size_t n = rows * (kH / 8);
+  for (size_t i = (size_t)blockIdx.x * 256 + threadIdx.x; i < n; i += (size_t)gridDim.x * 256) {
+    const size_t row = i / (kH / 8), c = i % (kH / 8);
+    const int tok = perm[row];
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (tok >= 0) v = ld_cg_v4(x + (size_t)tok * kH + 8 * c);
+    *reinterpret_cast<uint4 *>(xp + row * kH + 8 * c) = v;
+  }
+}
+
+// ============================================================== tcgen05 grouped GEMM
+// Tile: 128 weight rows (A) x 128 tokens (N), K in stages of 64.  A holds the
+// int4 codes as exact bf16 values; the bf16 scale of each (row, 128-wide
+// k-group) is applied in fp32 when the group's partial sum is read out of
+// tensor memory, so the weights enter the product exactly.  Two TMEM
+// accumulator buffers let the MMAs of group G+1 run while group G is read.
+// GEMM 2's token operand is the SwiGLU intermediate as a hi/lo bf16 pair (two
+// MMA passes over the same A tile), ~16 significant bits.
+constexpr int kABytes = 128 * 128;      // 128 weight rows x 64 bf16
+constexpr int kBBytes = kPfTile * 128;  // 128 token rows x 64 bf16
+constexpr int kRawBytes = 128 * 32;     // 128 weight rows x 64 int4
+constexpr int kGemmThreads = 320;       // producer, MMA, 4 dequant warps, 4 epilogue warps
+constexpr int kTmemCols = 256;          // two 128-column fp32 accumulators
+
+template <int kMode>
+struct GemmCfg {
+  static constexpr int kNB = kMode == 1 ? 1 : 2;  // token operands per stage (hi, lo)
+  static constexpr int kStageBytes = kABytes + kNB * kBBytes + kRawBytes;
+  static constexpr int kStages = kMode == 1 ? 5 : 4;
+  static constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024;
+};
+
+struct GemmArgs {
+  const uint32_t *tiles;
+  const uint32_t *ctrl;
+  int count_word;
+  const int32_t *ebase;
+  const int32_t *ecount;
+  int T;
+  const uint16_t *sc_r;  // scales of the routed weight tensor
+  const uint16_t *sc_s;  // scales of the shared expert's tensor
+  uint16_t *out_r;       // GEMM 1: H hi (lo follows at out_r_lo); GEMM 2: Yw
+  uint16_t *out_r_lo;
+  uint16_t *out_s;       // GEMM 1: Hs hi; GEMM 2: Ys
+  uint16_t *out_s_lo;
+  const float *pw;
+  uint32_t *status;
+};
+
+FLINT_DEV uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | (1ull << 16) | (64ull << 32) | (1ull << 46) |
+         (2ull << 61);
+}
+
+FLINT_DEV void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, "
+      "{%2, %3}], [%4];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+
+FLINT_DEV void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                         uint32_t accum) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, "
+      "%3, p;\n}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum));
+}
+
+FLINT_DEV void umma_commit(uint64_t *bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_addr(bar))
+      : "memory");
+}
+
+FLINT_DEV void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%"
+      "15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
+        "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
+        "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+FLINT_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+FLINT_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 32 int4 codes (one 16-byte chunk of a raw row) -> four 16-byte chunks of
+// exact bf16 codes in natural element order.
+FLINT_DEV void codes32(uint4 w, uint4 (&out)[4]) {
+  uint32_t r[16];
+  int4x32_to_bf16x2(w, r);
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    out[q] = make_uint4(__byte_perm(r[4 * q + 0], r[4 * q + 1], 0x5410),   // (c0, c1)
+                        __byte_perm(r[4 * q + 2], r[4 * q + 3], 0x5410),   // (c2, c3)
+                        __byte_perm(r[4 * q + 0], r[4 * q + 1], 0x7632),   // (c4, c5)
+                        __byte_perm(r[4 * q + 2], r[4 * q + 3], 0x7632));  // (c6, c7)
+}
+
+FLINT_DEV void split_hilo(float v, uint16_t &hi, uint16_t &lo) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(v);
+  hi = __bfloat16_as_ushort(h);
+  lo = __bfloat16_as_ushort(__float2bfloat16_rn(v - __bfloat162float(h)));
+}
+
+// kMode 1: gate/up + SwiGLU -> H hi/lo (routed [rows][512], shared [T][1024]).
+// kMode 2: down -> Yw (routed, weighted, [rows][2048]) / Ys (shared, [T][2048]).
+template <int kMode>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    k_pf_gemm(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
+              const __grid_constant__ CUtensorMap tmB_r, const __grid_constant__ CUtensorMap tmB_s,
+              const __grid_constant__ CUtensorMap tmB_r_lo,
+              const __grid_constant__ CUtensorMap tmB_s_lo, GemmArgs args) {
+  using Cfg = GemmCfg<kMode>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ unsigned char smraw[];
+  unsigned char *sm = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full[S], afull[S], empty[S], gfull[2], gempty[2];
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_fail;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t ntiles = __ldcg(args.ctrl + args.count_word);
+  if (blockIdx.x >= ntiles) return;
+  const uint32_t packed = __ldcg(args.tiles + blockIdx.x);
+  const int e = (int)(packed & 511u), mt = (int)((packed >> 9) & 31u), nt = (int)(packed >> 14);
+  const bool sh = e == kE;
+  const int n0 = nt * kPfTile;
+  const int n_valid = min(kPfTile, (sh ? args.T : __ldcg(args.ecount + e)) - n0);
+  if (n_valid <= 0) return;  // not produced by the scan; guards against an N = 0 MMA
+  const int b_row = sh ? n0 : __ldcg(args.ebase + e) + n0;
+  const int ks = kMode == 1 ? kH / 64 : (sh ? kIs / 64 : kI / 64);  // k stages
+  const int ng = ks / 2;                                              // 128-wide k-groups
+  const int n_mma = (n_valid + 15) & ~15;
+  int row0, row1;  // weight rows: GEMM 1 gate (tile rows 2i) / up (2i+1); GEMM 2 row0 + i
+  if (kMode == 1) {
+    row0 = sh ? 64 * mt : e * 2 * kI + 64 * mt;
+    row1 = sh ? kIs + 64 * mt : e * 2 * kI + kI + 64 * mt;
+  } else {
+    row0 = sh ? 128 * mt : e * kH + 128 * mt;
+    row1 = row0;
+  }
+  const CUtensorMap *tA = sh ? &tmA_s : &tmA_r;
+  const CUtensorMap *tB = sh ? &tmB_s : &tmB_r;
+  const CUtensorMap *tBl = sh ? &tmB_s_lo : &tmB_r_lo;
+
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&afull[s], 128);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&gfull[b], 1);
+      mbar_init(&gempty[b], 128);
+    }
+    s_fail = 0;
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(&s_tmem)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  if (warp == 0) {
+    // ---- producer: int4 codes of the weight tile and the token tile(s), by TMA
+    if (lane == 0) {
+      for (int kb = 0; kb < ks; ++kb) {
+        const int s = kb % S;
+        if (kb >= S && !mbar_wait(&empty[s], ((kb / S) - 1) & 1)) {
+          s_fail = 1;
+          break;
+        }
+        unsigned char *st = sm + (size_t)s * Cfg::kStageBytes;
+        unsigned char *raw = st + kABytes + Cfg::kNB * kBBytes;
+        mbar_expect_tx(&full[s], kRawBytes + Cfg::kNB * kBBytes);
+        if (kMode == 1) {
+          tma_load_2d(raw, tA, kb * 32, row0, &full[s]);
+          tma_load_2d(raw + 64 * 32, tA, kb * 32, row1, &full[s]);
+        } else {
+          tma_load_2d(raw, tA, kb * 32, row0, &full[s]);
+          tma_load_2d(st + kABytes + kBBytes, tBl, kb * 64, b_row, &full[s]);
+        }
+        tma_load_2d(st + kABytes, tB, kb * 64, b_row, &full[s]);
+      }
+    }
+  } else if (warp == 1) {
+    // ---- MMA issuer: group G accumulates into TMEM buffer G & 1
+    if (lane == 0) {
+      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n_mma >> 3) << 17) |
+                             ((uint32_t)(128 >> 4) << 24);
+      for (int G = 0; G < ng && !s_fail; ++G) {
+        const int b = G & 1;
+        if (G >= 2 && !mbar_wait(&gempty[b], ((G >> 1) - 1) & 1)) {
+          s_fail = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(128 * b);
+        for (int h = 0; h < 2; ++h) {
+          const int kb = 2 * G + h, s = kb % S;
+          const uint32_t ph = (kb / S) & 1;
+          if (!mbar_wait(&full[s], ph) || !mbar_wait(&afull[s], ph)) {
+            s_fail = 1;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_addr(sm + (size_t)s * Cfg::kStageBytes);
+          const uint32_t b_addr = a_addr + kABytes;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            umma_bf16(d, sw128_desc(a_addr + 32 * k), sw128_desc(b_addr + 32 * k), idesc,
+                      (h | k) != 0);
+            if (kMode == 2)
+              umma_bf16(d, sw128_desc(a_addr + 32 * k), sw128_desc(b_addr + kBBytes + 32 * k),
+                        idesc, 1u);
+          }
+          umma_commit(&empty[s]);
+        }
+        umma_commit(&gfull[b]);
+      }
+    }
+  } else if (warp < 6) {
+    // ---- dequant: thread i owns weight row i of the tile (exact codes)
+    const int i = tid - 64;
+    const int raw_row = kMode == 1 ? ((i & 1) ? 64 + (i >> 1) : (i >> 1)) : i;
+    for (int kb = 0; kb < ks; ++kb) {
+      const int s = kb % S;
+      if (!mbar_wait(&full[s], (kb / S) & 1)) {
+        s_fail = 1;
+        break;
+      }
+      unsigned char *st = sm + (size_t)s * Cfg::kStageBytes;
+      const unsigned char *raw = st + kABytes + Cfg::kNB * kBBytes + raw_row * 32;
+      const uint4 w0 = *reinterpret_cast<const uint4 *>(raw);
+      const uint4 w1 = *reinterpret_cast<const uint4 *>(raw + 16);
+      uint4 c[4];
+      unsigned char *arow = st + i * 128;
+      codes32(w0, c);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4 *>(arow + ((q ^ (i & 7)) * 16)) = c[q];
+      codes32(w1, c);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4 *>(arow + (((4 + q) ^ (i & 7)) * 16)) = c[q];
+      fence_proxy_async();
+      mbar_arrive(&afull[s]);
+    }
+  } else {
+    // ---- epilogue warps 6..9: TMEM lane quarter (warp % 4) -> tile rows
+    const int q4 = warp & 3;
+    const int r = 32 * q4 + lane;
+    const int wrow = kMode == 1 ? ((r & 1) ? row1 : row0) + (r >> 1) : row0 + r;
+    const int gpr = kMode == 1 ? kH / kG : (sh ? kIs / kG : kI / kG);
+    const uint16_t *srow = (sh ? args.sc_s : args.sc_r) + (size_t)wrow * gpr;
+    float acc[kPfTile];
+#pragma unroll
+    for (int j = 0; j < kPfTile; ++j) acc[j] = 0.f;
+    bool ok = true;
+    for (int G = 0; G < ng; ++G) {
+      const int b = G & 1;
+      const float sc = bf16_bits_to_f32(ld_nc_u16(srow + G));
+      if (!mbar_wait(&gfull[b], (G >> 1) & 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t base = tmem + (uint32_t)(128 * b) + ((uint32_t)(32 * q4) << 16);
+#pragma unroll
+      for (int c0 = 0; c0 < kPfTile; c0 += 32) {
+        if (c0 < n_mma) {
+          uint32_t v[32];
+          tmem_ld32(base + (uint32_t)c0, v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) acc[c0 + j] = fmaf(__uint_as_float(v[j]), sc, acc[c0 + j]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&gempty[b]);
+    }
+    if (!ok) {
+      s_fail = 1;
+    } else if (kMode == 1) {
+      const int col = 64 * mt + (r >> 1);
+      const size_t ld = sh ? kIs : kI;
+      uint16_t *hi = sh ? args.out_s + (size_t)n0 * kIs + col : args.out_r + (size_t)b_row * kI + col;
+      uint16_t *lo = sh ? args.out_s_lo + (size_t)n0 * kIs + col
+                        : args.out_r_lo + (size_t)b_row * kI + col;
+#pragma unroll
+      for (int j = 0; j < kPfTile; ++j) {
+        const float other = __shfl_xor_sync(0xffffffffu, acc[j], 1);
+        if (!(r & 1) && j < n_valid) {
+          const float hv = acc[j] / (1.f + expf(-acc[j])) * other;  // silu(gate) * up
+          uint16_t h16, l16;
+          split_hilo(hv, h16, l16);
+          hi[(size_t)j * ld] = h16;
+          lo[(size_t)j * ld] = l16;
+        }
+      }
+    } else {
+      const int col = 128 * mt + r;
+#pragma unroll
+      for (int j = 0; j < kPfTile; ++j) {
+        if (j < n_valid) {
+          if (sh) {
+            args.out_s[(size_t)(n0 + j) * kH + col] = f32_to_bf16_bits(acc[j]);
+          } else {
+            args.out_r[(size_t)(b_row + j) * kH + col] =
+                f32_to_bf16_bits(acc[j] * args.pw[b_row + j]);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (s_fail && tid == 0) set_status(args.status, kStatusTimeout);
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols));
+  }
+}
+
+// ============================================================== combine
+__global__ void __launch_bounds__(256)
+    k_pf_combine(const int32_t *__restrict__ pos, const uint16_t *__restrict__ yw,
+                 const uint16_t *__restrict__ ys, int T, uint16_t *__restrict__ out) {
+  const size_t n = (size_t)T * (kH / 8);
+  for (size_t i = (size_t)blockIdx.x * 256 + threadIdx.x; i < n; i += (size_t)gridDim.x * 256) {
+    const size_t tok = i / (kH / 8), c = i % (kH / 8);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j <= kTopK; ++j) {
+      const uint16_t *src = j < kTopK ? yw + (size_t)pos[tok * kTopK + j] * kH : ys + tok * kH;
+      const uint4 v = ld_cg_v4(src + 8 * c);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        acc[2 * k] += __uint_as_float(w[k] << 16);
+        acc[2 * k + 1] += __uint_as_float(w[k] & 0xffff0000u);
+      }
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      o[k] = (uint32_t)f32_to_bf16_bits(acc[2 * k]) | ((uint32_t)f32_to_bf16_bits(acc[2 * k + 1]) << 16);
+    *reinterpret_cast<uint4 *>(out + tok * kH + 8 * c) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// ============================================================== host
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::mutex g_encode_mu;
+
+cudaError_t get_encode() {
+  std::lock_guard<std::mutex> lock(g_encode_mu);
+  if (g_encode) return cudaSuccess;
+  void *fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+  if (e != cudaSuccess) return e;
+  if (q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return cudaSuccess;
+}
+
+// 2-D tile map: rows x cols (inner), row pitch in bytes.
+cudaError_t make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint64_t cols,
+                     uint64_t rows, uint64_t pitch, uint32_t box_cols, uint32_t box_rows,
+                     CUtensorMapSwizzle sw) {
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {pitch};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t elem[2] = {1, 1};
+  const CUresult r = g_encode(m, dt, 2, const_cast<void *>(base), dims, strides, box, elem,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_route_many(const LayerArgs &L, const uint16_t *x, int T, int32_t *idx, float *w,
+                              char *ws, cudaStream_t st) {
+  const PrefillLayout P = prefill_layout(T);
+  float *z = reinterpret_cast<float *>(ws + P.z);
+  note_step("prefill router attribute");
+  cudaError_t e = cudaFuncSetAttribute(k_pf_router, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       8 * 8 * 32 * 64);
+  if (e != cudaSuccess) return e;
+  note_step("prefill router launch");
+  k_pf_router<<<dim3((T + kRtTok - 1) / kRtTok, 2), 256, 8 * 8 * 32 * 64, st>>>(L, x, T, z);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  note_step("prefill top-6 launch");
+  k_pf_topk<<<(T + 7) / 8, 256, 0, st>>>(L.router_b, z, T, idx, w,
+                                          reinterpret_cast<int32_t *>(ws + P.asc_e),
+                                          reinterpret_cast<float *>(ws + P.asc_w));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_t *out, char *ws,
+                           cudaStream_t st) {
+  const PrefillLayout P = prefill_layout(T);
+  cudaError_t e = noted(get_encode(), "cuTensorMapEncodeTiled entry point");
+  if (e != cudaSuccess) return e;
+  uint32_t *ctrl = reinterpret_cast<uint32_t *>(ws + P.ctrl);
+  int32_t *asc_e = reinterpret_cast<int32_t *>(ws + P.asc_e);
+  float *asc_w = reinterpret_cast<float *>(ws + P.asc_w);
+  int32_t *pos = reinterpret_cast<int32_t *>(ws + P.pos);
+  int32_t *cc = reinterpret_cast<int32_t *>(ws + P.chunk_cnt);
+  int32_t *co = reinterpret_cast<int32_t *>(ws + P.chunk_off);
+  int32_t *ebase = reinterpret_cast<int32_t *>(ws + P.ebase);
+  int32_t *ecount = reinterpret_cast<int32_t *>(ws + P.ecount);
+  int32_t *perm = reinterpret_cast<int32_t *>(ws + P.perm);
+  float *pw = reinterpret_cast<float *>(ws + P.pw);
+  uint32_t *tiles1 = reinterpret_cast<uint32_t *>(ws + P.tiles1);
+  uint32_t *tiles2 = reinterpret_cast<uint32_t *>(ws + P.tiles2);
+  uint16_t *xp = reinterpret_cast<uint16_t *>(ws + P.xp);
+  uint16_t *hr = reinterpret_cast<uint16_t *>(ws + P.hr);          // hi
+  uint16_t *hr_lo = hr + (size_t)P.mr_max * kI;                     // lo
+  uint16_t *hs = reinterpret_cast<uint16_t *>(ws + P.hs);
+  uint16_t *hs_lo = hs + (size_t)T * kIs;
+  uint16_t *yw = reinterpret_cast<uint16_t *>(ws + P.yw);
+  uint16_t *ys = reinterpret_cast<uint16_t *>(ws + P.ys);
+
+  // 1. routing
+  e = launch_route_many(L, x, T, reinterpret_cast<int32_t *>(ws + P.sel_idx),
+                        reinterpret_cast<float *>(ws + P.sel_w), ws, st);
+  if (e != cudaSuccess) return e;
+  // 2. stable sort by expert
+  note_step("prefill sort launches");
+  k_pf_count<<<P.nchunks, 256, 0, st>>>(asc_e, T, cc);
+  k_pf_scan<<<1, 256, 0, st>>>(T, P.nchunks, cc, co, ebase, ecount, perm, tiles1, tiles2, ctrl);
+  k_pf_place<<<P.nchunks, 256, 0, st>>>(asc_e, asc_w, T, co, ebase, pos, perm, pw);
+  // 3. gather
+  {
+    int blocks = (int)(((size_t)P.mr_max * (kH / 8) + 255) / 256);
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    k_pf_gather<<<blocks, 256, 0, st>>>(x, perm, ctrl, xp);
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // 4. tensor maps and the two grouped GEMMs
+  CUtensorMap mA1r, mA1s, mB1r, mB1s, mA2r, mA2s, mB2r, mB2s, mB2rl, mB2sl;
+  note_step("prefill tensor maps");
+  const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const auto SW = CU_TENSOR_MAP_SWIZZLE_128B, NS = CU_TENSOR_MAP_SWIZZLE_NONE;
+  if ((e = make_map(&mA1r, L.w13_q, U8, kH / 2, (uint64_t)kE * 2 * kI, kH / 2, 32, 64, NS)) ||
+      (e = make_map(&mA1s, L.sh13_q, U8, kH / 2, 2 * kIs, kH / 2, 32, 64, NS)) ||
+      (e = make_map(&mB1r, xp, BF, kH, (uint64_t)P.mr_max, kH * 2, 64, kPfTile, SW)) ||
+      (e = make_map(&mB1s, x, BF, kH, (uint64_t)T, kH * 2, 64, kPfTile, SW)) ||
+      (e = make_map(&mA2r, L.w2_q, U8, kI / 2, (uint64_t)kE * kH, kI / 2, 32, 128, NS)) ||
+      (e = make_map(&mA2s, L.sh2_q, U8, kIs / 2, kH, kIs / 2, 32, 128, NS)) ||
+      (e = make_map(&mB2r, hr, BF, kI, (uint64_t)P.mr_max, kI * 2, 64, kPfTile, SW)) ||
+      (e = make_map(&mB2rl, hr_lo, BF, kI, (uint64_t)P.mr_max, kI * 2, 64, kPfTile, SW)) ||
+      (e = make_map(&mB2s, hs, BF, kIs, (uint64_t)T, kIs * 2, 64, kPfTile, SW)) ||
+      (e = make_map(&mB2sl, hs_lo, BF, kIs, (uint64_t)T, kIs * 2, 64, kPfTile, SW)))
+    return e;
+  note_step("prefill GEMM attributes");
+  if ((e = cudaFuncSetAttribute(k_pf_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)GemmCfg<1>::kSmem)) != cudaSuccess ||
+      (e = cudaFuncSetAttribute(k_pf_gemm<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)GemmCfg<2>::kSmem)) != cudaSuccess)
+    return e;
+  GemmArgs a1{tiles1, ctrl, 3,  ebase, ecount, T,       L.w13_s, L.sh13_s,
+              hr,     hr_lo, hs, hs_lo, nullptr, ctrl + 1};
+  note_step("prefill GEMM 1 launch");
+  k_pf_gemm<1><<<P.max_tiles1, kGemmThreads, GemmCfg<1>::kSmem, st>>>(mA1r, mA1s, mB1r, mB1s,
+                                                                        mB1r, mB1s, a1);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  GemmArgs a2{tiles2, ctrl, 4, ebase, ecount, T, L.w2_s, L.sh2_s, yw, nullptr, ys, nullptr, pw,
+              ctrl + 1};
+  note_step("prefill GEMM 2 launch");
+  k_pf_gemm<2><<<P.max_tiles2, kGemmThreads, GemmCfg<2>::kSmem, st>>>(mA2r, mA2s, mB2r, mB2s,
+                                                                        mB2rl, mB2sl, a2);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // 5. combine
+  note_step("prefill combine launch");
+  {
+    int blocks = (int)(((size_t)T * (kH / 8) + 255) / 256);
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    k_pf_combine<<<blocks, 256, 0, st>>>(pos, yw, ys, T, out);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace flint
