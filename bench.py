@@ -49,7 +49,20 @@ def parse():
     p.add_argument("--layers", type=int, default=N_LAYERS)
     p.add_argument("--no-head", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
+    p.add_argument("--no-prefill", action="store_true")
     return p.parse_args()
+
+
+# router 2*256*2048 + routed 6 * 3 * 2 * 2048 * 512 + shared 3 * 2 * 2048 * 1024
+PREFILL_FLOP_PER_TOKEN = 2 * 256 * 2048 + 6 * 6 * 2048 * 512 + 6 * 2048 * 1024
+
+
+def tensor_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
 
 
 def peaks():
@@ -365,6 +378,7 @@ def main():
     e2e_us = mse * 1e3 / (args.steps * nl) / world
 
     # ---- output head int4 GEMV (B = 1 and the bench batch), context
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     if not args.no_head and rank == 0:
         hq = synth.random_bytes_torch(0, synth.T_HEAD_Q, synth.VOCAB * H // 2, dev).view(
             synth.VOCAB, H // 2)
@@ -376,7 +390,6 @@ def main():
             nbh = F.flint_gemv_workspace_bytes(synth.VOCAB, hb)
             wsh = torch.zeros(nbh, dtype=torch.uint8, device=dev)
             F.flint_workspace_init(wsh, nbh)
-            flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
             times = []
             for it in range(23):
                 with torch.cuda.stream(stream):
@@ -391,6 +404,31 @@ def main():
             us = statistics.median(times)
             extra[f"head_gemv_b{hb}"] = {"us": us, "GBps": HEAD_BYTES / (us * 1e-6) / 1e9,
                                         "roofline_frac": HEAD_BYTES / (us * 1e-6) / 1e9 / hbm}
+    # ---- prefill of one MoE layer (layer 0): tokens/s and tensor-pipe roofline
+    if not args.no_prefill and rank == 0:
+        peak_tf, peak_kind_tf = tensor_peak()
+        for T in (2048, 4096, 32768):
+            xt = synth.to_device({"x": synth.prefill_x(T, T)}, dev)["x"]
+            out_t = torch.empty((T, H), dtype=torch.int16, device=dev)
+            nbp = F.flint_workspace_bytes(F.FLINT_OP_PREFILL, T)
+            wsp = torch.zeros(nbp, dtype=torch.uint8, device=dev)
+            F.flint_workspace_init(wsp, nbp)
+            times = []
+            for it in range(7):
+                with torch.cuda.stream(stream):
+                    flush.zero_()  # evict L2 between runs
+                    e0.record(stream)
+                    F.flint_moe_prefill(structs[0], xt, T, out_t, wsp, nbp, stream=stream)
+                    e1.record(stream)
+                e1.synchronize()
+                if it >= 2:
+                    times.append(e0.elapsed_time(e1) * 1e3)
+            us = statistics.median(times)
+            tflops = T * PREFILL_FLOP_PER_TOKEN / (us * 1e-6) / 1e12
+            extra[f"prefill_T{T}"] = {"us": us, "tokens_per_s": T / (us * 1e-6),
+                                      "TFLOPs": tflops, "tensor_frac": tflops / peak_tf,
+                                      "peak_kind": peak_kind_tf}
+            del wsp, out_t, xt
     sampler.stop()
 
     cpu = None

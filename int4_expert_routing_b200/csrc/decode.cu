@@ -113,6 +113,49 @@ FLINT_DEV void stage_input(uint4 *xfrag, int G0, int nG, const uint16_t *x_in, c
   }
 }
 
+// Compact activation fragment (only the B live columns, lanes g < B):
+// frag[(G * 4B + g * 4 + t) * 4 + q]; other lanes read zeros.
+template <bool kResidual>
+FLINT_DEV void stage_input_compact(uint4 *frag, const uint16_t *x_in, const float *h, int B,
+                                   const double *inv, int tid, int nthreads) {
+  const int n = 16 * 4 * B * 4;
+  for (int task = tid; task < n; task += nthreads) {
+    const int q = task & 3, gt = (task >> 2) % (4 * B), G = (task >> 2) / (4 * B);
+    const int gg = gt >> 2, tt = gt & 3;
+    const int k0 = 128 * G + 32 * tt + 8 * q;
+    uint4 v;
+    if (kResidual) {
+      const float4 a = __ldcg(reinterpret_cast<const float4 *>(h + (size_t)gg * kH + k0));
+      const float4 c = __ldcg(reinterpret_cast<const float4 *>(h + (size_t)gg * kH + k0 + 4));
+      const double s = inv[gg];
+      const float f[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+      uint32_t bits[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) bits[i] = f64_to_bf16_bits((double)f[i] * s);
+      v = make_uint4(bits[0] | (bits[1] << 16), bits[2] | (bits[3] << 16),
+                     bits[4] | (bits[5] << 16), bits[6] | (bits[7] << 16));
+    } else {
+      v = ld_cg_v4(x_in + (size_t)gg * kH + k0);
+    }
+    frag[task] = bf16x8_to_pairs(v);
+  }
+}
+
+FLINT_DEV void load_frag_compact(const uint4 *frag, int G, int B, int lane, uint32_t (&x)[16]) {
+  const int g = lane >> 2, t = lane & 3;
+  if (g < B) {
+    const uint4 *p = frag + (size_t)(G * 4 * B + g * 4 + t) * 4;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 v = p[i];
+      x[4 * i] = v.x, x[4 * i + 1] = v.y, x[4 * i + 2] = v.z, x[4 * i + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) x[i] = 0u;
+  }
+}
+
 // ============================================================== K1: router
 constexpr uint32_t kSlotInvalid = 0xffffffffu;
 FLINT_DEV uint32_t slot_expert(uint32_t w) { return w & 0xffu; }
@@ -171,6 +214,9 @@ __global__ void __launch_bounds__(kK1Threads)
 
   if (kResidual) rms_inv(h, B, s_red, s_inv, tid);
   stage_input<kResidual>(xfrag, 8 * kh, 8, x_in, h, B, s_inv, tid, kK1Threads);
+  if (blockIdx.x == 0)  // the routed gate/up CTAs bulk-copy this image
+    stage_input_compact<kResidual>(reinterpret_cast<uint4 *>(ws + lay.xfrag), x_in, h, B, s_inv,
+                                   tid, kK1Threads);
   const bool ok = mbar_wait(&bar, 0);
   if (__syncthreads_or(!ok)) {
     if (tid == 0) set_status(ctrl + 1, kStatusTimeout);
@@ -349,49 +395,6 @@ FLINT_DEV void issue_item(const ItemSrc &src, unsigned char *buf, uint64_t *bar)
   bulk_g2s(buf + 16640, src.up_s, 256, bar);
 }
 
-// Compact activation fragment (only the B live columns, lanes g < B):
-// frag[(G * 4B + g * 4 + t) * 4 + q]; other lanes read zeros.
-template <bool kResidual>
-FLINT_DEV void stage_input_compact(uint4 *frag, const uint16_t *x_in, const float *h, int B,
-                                   const double *inv, int tid, int nthreads) {
-  const int n = 16 * 4 * B * 4;
-  for (int task = tid; task < n; task += nthreads) {
-    const int q = task & 3, gt = (task >> 2) % (4 * B), G = (task >> 2) / (4 * B);
-    const int gg = gt >> 2, tt = gt & 3;
-    const int k0 = 128 * G + 32 * tt + 8 * q;
-    uint4 v;
-    if (kResidual) {
-      const float4 a = __ldcg(reinterpret_cast<const float4 *>(h + (size_t)gg * kH + k0));
-      const float4 c = __ldcg(reinterpret_cast<const float4 *>(h + (size_t)gg * kH + k0 + 4));
-      const double s = inv[gg];
-      const float f[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
-      uint32_t bits[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) bits[i] = f64_to_bf16_bits((double)f[i] * s);
-      v = make_uint4(bits[0] | (bits[1] << 16), bits[2] | (bits[3] << 16),
-                     bits[4] | (bits[5] << 16), bits[6] | (bits[7] << 16));
-    } else {
-      v = ld_cg_v4(x_in + (size_t)gg * kH + k0);
-    }
-    frag[task] = bf16x8_to_pairs(v);
-  }
-}
-
-FLINT_DEV void load_frag_compact(const uint4 *frag, int G, int B, int lane, uint32_t (&x)[16]) {
-  const int g = lane >> 2, t = lane & 3;
-  if (g < B) {
-    const uint4 *p = frag + (size_t)(G * 4 * B + g * 4 + t) * 4;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 v = p[i];
-      x[4 * i] = v.x, x[4 * i + 1] = v.y, x[4 * i + 2] = v.z, x[4 * i + 3] = v.w;
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) x[i] = 0u;
-  }
-}
-
 // This warp's 4 k-groups of the item: acc[0..1] gate, [2..3] up partials for
 // columns 2t, 2t+1 of row r0 + g.
 FLINT_DEV void item_part(const unsigned char *buf, const uint4 *frag, int B, int warp, int lane,
@@ -440,18 +443,24 @@ __global__ void __launch_bounds__(kK2Warps * 32)
     mbar_init(&bar, 1);
     if (shared_item_cta) issue_item(shared_item(L, it), buf, &bar);
   }
-  // The input is final here: this grid was launched after K1 passed its wait.
-  if (kResidual) rms_inv(h, B, s_red, s_inv, tid);
-  stage_input_compact<kResidual>(frag, x_in, h, B, s_inv, tid, kK2Warps * 32);
-  if (!shared_item_cta) {
+  if (shared_item_cta) {
+    // The input is final here: this grid was launched after K1 passed its wait.
+    if (kResidual) rms_inv(h, B, s_red, s_inv, tid);
+    stage_input_compact<kResidual>(frag, x_in, h, B, s_inv, tid, kK2Warps * 32);
+  } else {
     pdl_wait();
     pdl_trigger();
     if (tid == 0) {
       const uint32_t w =
           ld_cg_u32(reinterpret_cast<const uint32_t *>(ws + lay.slot_word) + ((it - kSharedItems) >> 6));
       s_word = w;
-      if (w != kSlotInvalid)
+      if (w != kSlotInvalid) {
+        // the block input as K1 staged it, and this item's weights
+        const uint32_t fbytes = 16u * 4u * (uint32_t)B * 64u;
+        mbar_add_tx(&bar, fbytes);  // issue_item makes the phase's single arrival
+        bulk_g2s(frag, ws + lay.xfrag, fbytes, &bar);
         issue_item(routed_item(L, (int)slot_expert(w), 8 * ((it - kSharedItems) & 63)), buf, &bar);
+      }
     }
   }
   __syncthreads();

@@ -13,7 +13,7 @@ namespace flint {
 // Slot word u: expert (bits 0-7) | row mask (bits 8-15) | number of slots
 // (bits 16-24) for u < number of slots, else all ones.
 struct DecodeLayout {
-  size_t ctrl, zpart, sel_idx, sel_w, asc_slot, asc_w, slot_word, hfr, hfs, total;
+  size_t ctrl, zpart, sel_idx, sel_w, asc_slot, asc_w, slot_word, hfr, hfs, xfrag, total;
 };
 
 __host__ __device__ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -35,6 +35,7 @@ inline DecodeLayout decode_layout(int B) {
   L.slot_word = take(sizeof(uint32_t) * 256);          // slot table, see kSlotInvalid
   L.hfr = take(sizeof(uint16_t) * B * 6 * 2 * 512);    // routed SwiGLU hi/lo images
   L.hfs = take(sizeof(uint16_t) * B * 2 * 1024);       // shared SwiGLU hi/lo images
+  L.xfrag = take((size_t)16 * 4 * B * 64);             // block input as a compact fragment image
   L.total = o;
   return L;
 }
