@@ -37,9 +37,35 @@
 
 namespace flint {
 
+// Optional timeline trace (build with -DFLINT_TRACE): thread 0 of every CTA
+// records %globaltimer at marked points, read back with flint_trace_dump.
+#ifdef FLINT_TRACE
+constexpr unsigned kTraceCap = 1u << 18;
+static __device__ unsigned long long g_trace_time[kTraceCap];
+static __device__ unsigned int g_trace_tag[kTraceCap];
+static __device__ unsigned int g_trace_n;
+// Event 0 (kernel start) reserves the CTA's eight records with one atomic,
+// before any wait; later events are plain stores.
+FLINT_DEV void trace_point(uint32_t kernel, uint32_t event) {
+  __shared__ unsigned s_base;
+  if (threadIdx.x == 0) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    if (event == 0) s_base = atomicAdd(&g_trace_n, 8u);
+    const unsigned i = s_base + event;
+    if (i < kTraceCap) {
+      g_trace_time[i] = t;
+      g_trace_tag[i] = (kernel << 28) | (event << 24) | blockIdx.x;
+    }
+  }
+}
+#else
+FLINT_DEV void trace_point(uint32_t, uint32_t) {}
+#endif
+
 constexpr int kRouterCtas = 32;   // 16 expert tiles x 2 k-halves
 constexpr int kK1Threads = 256;   // 8 warps: one 128-wide k-group each
-constexpr int kK3Threads = 256;
+constexpr int kK3Threads = 512;
 constexpr int kXFragBytes = 16 * 128 * 16;  // 16 groups x 128 uint4
 
 FLINT_DEV float silu_f(float v) { return v / (1.f + expf(-v)); }
@@ -54,91 +80,91 @@ FLINT_DEV void write_hilo(uint16_t *img_hi, uint16_t *img_lo, int k, float v) {
 
 // ---------------------------------------------------------------- input
 // RMSNorm scale 1/sqrt(mean(h^2) + eps) per row, fp64, in one fixed order
-// whatever the block size: threads 0..127 each sum a strided slice, then an
-// xor tree per warp and the four warps in order.  K1 and K2 both call this,
-// so they normalize to the same bits.
-constexpr int kRmsThreads = 128;
-FLINT_DEV void rms_inv(const float *h, int B, double *s_red /*[4 * kMaxB]*/, double *inv,
-                       int tid) {
-  const int warp = tid >> 5, lane = tid & 31;
-  if (tid < kRmsThreads) {
-    for (int b = 0; b < B; ++b) {
+// whatever the block size: 128 "lanes" t each sum the squares of elements
+// t, t+128, ..., t+1920 in that order, then an xor tree inside each warp of
+// 32 consecutive t, then the four warps in order.  K1 and K2 both call
+// rms_stage, so they normalize to the same bits.
+//
+// The normalized row, rounded to bf16 (fp64 product, one rounding), goes
+// straight into the compact mma fragment: for element k of row b the slot is
+// 8 * ((G * 4B + 4b + tt) * 4 + q) + 2 * (e & 3) + (e >> 2) with G = k/128,
+// tt = k/32 mod 4, q = k/8 mod 4, e = k mod 8 (the pair order that
+// bf16x8_to_pairs produces).  Other lanes of the fragment read zeros.
+FLINT_DEV int compact_slot(int b, int k, int B) {
+  const int G = k >> 7, tt = (k >> 5) & 3, q = (k >> 3) & 3, e = k & 7;
+  return 8 * ((G * 4 * B + 4 * b + tt) * 4 + q) + 2 * (e & 3) + (e >> 2);
+}
+
+// All kThreads threads; rows are taken kThreads/128 at a time, each thread
+// holding up to kRowsPerPass rows' 16 elements in registers so that every
+// load of a pass is in flight at once.
+template <int kThreads, int kRowsPerPass>
+FLINT_DEV void rms_stage(const float *h, int B, double *s_red /*[4 * kMaxB]*/, double *s_inv,
+                         uint16_t *frag16, int tid) {
+  constexpr int kPar = kThreads / 128;
+  const int t = tid & 127, hv = tid >> 7, lane = tid & 31, tw = t >> 5;
+  for (int p0 = 0; p0 < B; p0 += kPar * kRowsPerPass) {
+    float v[kRowsPerPass][16];
+#pragma unroll
+    for (int r = 0; r < kRowsPerPass; ++r) {
+      const int b = p0 + hv + kPar * r;
+      if (b < B) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[r][j] = __ldcg(h + (size_t)b * kH + t + 128 * j);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kRowsPerPass; ++r) {
+      const int b = p0 + hv + kPar * r;
+      if (b < B) {  // the same b for all lanes of a warp
+        double ss = 0.0;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) ss = fma((double)v[r][j], (double)v[r][j], ss);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (lane == 0) s_red[tw * kMaxB + b] = ss;
+      }
+    }
+    __syncthreads();
+    if (tid < B && tid >= p0 && tid < p0 + kPar * kRowsPerPass) {
       double ss = 0.0;
-      for (int i = tid; i < kH; i += kRmsThreads) {
-        const double v = (double)ld_cg_f32(h + (size_t)b * kH + i);
-        ss = fma(v, v, ss);
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      if (lane == 0) s_red[warp * kMaxB + b] = ss;
+      for (int w = 0; w < 4; ++w) ss += s_red[w * kMaxB + tid];
+      s_inv[tid] = 1.0 / sqrt(ss / kH + FLINT_RMS_EPS);
     }
-  }
-  __syncthreads();
-  if (tid < B) {
-    double ss = 0.0;
-    for (int w = 0; w < kRmsThreads / 32; ++w) ss += s_red[w * kMaxB + tid];
-    inv[tid] = 1.0 / sqrt(ss / kH + FLINT_RMS_EPS);
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < kRowsPerPass; ++r) {
+      const int b = p0 + hv + kPar * r;
+      if (b < B) {
+        const double sc = s_inv[b];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          frag16[compact_slot(b, t + 128 * j, B)] =
+              (uint16_t)f64_to_bf16_bits((double)v[r][j] * sc);
+      }
+    }
   }
   __syncthreads();
 }
 
-// Activation fragment of groups G0 .. G0+nG-1 of the block's input rows into
-// shared memory (local group index G - G0).  Plain decode reads the bf16
-// input; the residual form rounds RMSNorm(h) to bf16 (fp64 product, one
-// rounding).
-template <bool kResidual>
-FLINT_DEV void stage_input(uint4 *xfrag, int G0, int nG, const uint16_t *x_in, const float *h,
-                           int B, const double *inv, int tid, int nthreads) {
-  for (int task = tid; task < nG * 128; task += nthreads) {
-    const int G = G0 + (task >> 7), ln = (task >> 2) & 31, q = task & 3;
-    const int gg = ln >> 2, tt = ln & 3;
-    const int k0 = 128 * G + 32 * tt + 8 * q;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (gg < B) {
-      if (kResidual) {
-        const float4 a = __ldcg(reinterpret_cast<const float4 *>(h + (size_t)gg * kH + k0));
-        const float4 c = __ldcg(reinterpret_cast<const float4 *>(h + (size_t)gg * kH + k0 + 4));
-        const double s = inv[gg];
-        const float f[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
-        uint32_t bits[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) bits[i] = f64_to_bf16_bits((double)f[i] * s);
-        v = make_uint4(bits[0] | (bits[1] << 16), bits[2] | (bits[3] << 16),
-                       bits[4] | (bits[5] << 16), bits[6] | (bits[7] << 16));
-      } else {
-        v = ld_cg_v4(x_in + (size_t)gg * kH + k0);
-      }
-    }
-    xfrag[task] = bf16x8_to_pairs(v);
-  }
-}
-
-// Compact activation fragment (only the B live columns, lanes g < B):
-// frag[(G * 4B + g * 4 + t) * 4 + q]; other lanes read zeros.
-template <bool kResidual>
-FLINT_DEV void stage_input_compact(uint4 *frag, const uint16_t *x_in, const float *h, int B,
-                                   const double *inv, int tid, int nthreads) {
+// Compact fragment of a bf16 input (plain decode): frag[(G * 4B + 4g + t) * 4 + q].
+FLINT_DEV void stage_x_compact(uint4 *frag, const uint16_t *x_in, int B, int tid, int nthreads) {
   const int n = 16 * 4 * B * 4;
   for (int task = tid; task < n; task += nthreads) {
     const int q = task & 3, gt = (task >> 2) % (4 * B), G = (task >> 2) / (4 * B);
     const int gg = gt >> 2, tt = gt & 3;
-    const int k0 = 128 * G + 32 * tt + 8 * q;
-    uint4 v;
-    if (kResidual) {
-      const float4 a = __ldcg(reinterpret_cast<const float4 *>(h + (size_t)gg * kH + k0));
-      const float4 c = __ldcg(reinterpret_cast<const float4 *>(h + (size_t)gg * kH + k0 + 4));
-      const double s = inv[gg];
-      const float f[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
-      uint32_t bits[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) bits[i] = f64_to_bf16_bits((double)f[i] * s);
-      v = make_uint4(bits[0] | (bits[1] << 16), bits[2] | (bits[3] << 16),
-                     bits[4] | (bits[5] << 16), bits[6] | (bits[7] << 16));
-    } else {
-      v = ld_cg_v4(x_in + (size_t)gg * kH + k0);
-    }
-    frag[task] = bf16x8_to_pairs(v);
+    frag[task] = bf16x8_to_pairs(ld_cg_v4(x_in + (size_t)gg * kH + 128 * G + 32 * tt + 8 * q));
   }
+  __syncthreads();
+}
+
+template <bool kResidual, int kThreads, int kRowsPerPass>
+FLINT_DEV void stage_input(uint4 *frag, const uint16_t *x_in, const float *h, int B,
+                           double *s_red, double *s_inv, int tid) {
+  if (kResidual)
+    rms_stage<kThreads, kRowsPerPass>(h, B, s_red, s_inv, reinterpret_cast<uint16_t *>(frag), tid);
+  else
+    stage_x_compact(frag, x_in, B, tid, kThreads);
 }
 
 FLINT_DEV void load_frag_compact(const uint4 *frag, int G, int B, int lane, uint32_t (&x)[16]) {
@@ -165,15 +191,13 @@ FLINT_DEV int slot_count(uint32_t w) { return (int)((w >> 16) & 0x1ffu); }
 // Release-publish this CTA's results and tell whether it is the last of
 // `nctas` to do so; one fence per CTA on each side of the counter.
 FLINT_DEV bool last_cta(uint32_t *counter, uint32_t nctas, int *s_flag) {
-  __syncthreads();
+  __syncthreads();  // the CTA's writes happen before thread 0's release
   if (threadIdx.x == 0) {
-    __threadfence();
-    const uint32_t prev = atomicAdd(counter, 1u);
-    const bool last = prev == nctas - 1;
-    if (last) __threadfence();
-    *s_flag = last;
+    uint32_t prev;
+    asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(prev) : "l"(counter) : "memory");
+    *s_flag = prev == nctas - 1;
   }
-  __syncthreads();
+  __syncthreads();  // ... and the acquire happens before the CTA's reads
   return *s_flag != 0;
 }
 
@@ -182,8 +206,8 @@ __global__ void __launch_bounds__(kK1Threads)
     k1_router(LayerArgs L, const uint16_t *__restrict__ x_in, const float *__restrict__ h, int B,
               char *__restrict__ ws, DecodeLayout lay, int32_t *__restrict__ idx_out,
               float *__restrict__ w_out) {
-  extern __shared__ __align__(128) unsigned char sm[];  // [16 rows][2048 B] | x fragment
-  uint4 *xfrag = reinterpret_cast<uint4 *>(sm + 16 * 2048);
+  extern __shared__ __align__(128) unsigned char sm[];  // [16 rows][2048 B] | compact x fragment
+  uint4 *frag = reinterpret_cast<uint4 *>(sm + 16 * 2048);
   __shared__ __align__(8) uint64_t bar;
   __shared__ double s_part[8][kMaxB][16];
   __shared__ double s_red[4 * kMaxB];
@@ -199,6 +223,7 @@ __global__ void __launch_bounds__(kK1Threads)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   uint32_t *ctrl = reinterpret_cast<uint32_t *>(ws + lay.ctrl);
   const int et = blockIdx.x >> 1, kh = blockIdx.x & 1;
+  trace_point(1, 0);
 
   // this CTA's router block: 16 experts x one k-half (2 KB per row), fetched
   // before the wait (the weights do not depend on the previous kernel)
@@ -209,20 +234,31 @@ __global__ void __launch_bounds__(kK1Threads)
   __syncthreads();
   if (tid < 16)
     bulk_g2s(sm + tid * 2048, L.router_w + (size_t)(16 * et + tid) * kH + kh * (kH / 2), 2048, &bar);
+  // selection bias for the last CTA's top-6 (lane + 32 i), also a weight
+  float bias[8];
+  if (warp < B) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) bias[i] = __ldg(L.router_b + lane + 32 * i);
+  }
   pdl_wait();
   pdl_trigger();
+  trace_point(1, 1);
 
-  if (kResidual) rms_inv(h, B, s_red, s_inv, tid);
-  stage_input<kResidual>(xfrag, 8 * kh, 8, x_in, h, B, s_inv, tid, kK1Threads);
-  if (blockIdx.x == 0)  // the routed gate/up CTAs bulk-copy this image
-    stage_input_compact<kResidual>(reinterpret_cast<uint4 *>(ws + lay.xfrag), x_in, h, B, s_inv,
-                                   tid, kK1Threads);
+  stage_input<kResidual, kK1Threads, 4>(frag, x_in, h, B, s_red, s_inv, tid);
+  trace_point(1, 4);
+  {  // publish the fragment (each CTA a share) for the routed gate/up CTAs
+    const int n = 256 * B;  // uint4 per call: 4096 B per row
+    uint4 *dst = reinterpret_cast<uint4 *>(ws + lay.xfrag);
+    for (int i = blockIdx.x * kK1Threads + tid; i < n; i += kRouterCtas * kK1Threads)
+      dst[i] = frag[i];
+  }
   const bool ok = mbar_wait(&bar, 0);
   if (__syncthreads_or(!ok)) {
     if (tid == 0) set_status(ctrl + 1, kStatusTimeout);
     if (!ok) mbar_wait(&bar, 0);
     return;
   }
+  trace_point(1, 5);
   {
     uint32_t ra[16], rb[16], xb[16];
 #pragma unroll
@@ -234,7 +270,7 @@ __global__ void __launch_bounds__(kK1Threads)
       ra[4 * q] = a.x, ra[4 * q + 1] = a.y, ra[4 * q + 2] = a.z, ra[4 * q + 3] = a.w;
       rb[4 * q] = c.x, rb[4 * q + 1] = c.y, rb[4 * q + 2] = c.z, rb[4 * q + 3] = c.w;
     }
-    load_frag(xfrag + (warp * 32 + lane) * 4, xb);
+    load_frag_compact(frag, 8 * kh + warp, B, lane, xb);
     float d[4];
     group_mma(ra, rb, xb, d);
 #pragma unroll
@@ -254,7 +290,9 @@ __global__ void __launch_bounds__(kK1Threads)
     for (int w = 0; w < 8; ++w) p += s_part[w][b][r];
     zp[((size_t)kh * B + b) * kE + 16 * et + r] = p;
   }
+  trace_point(1, 2);
   if (!last_cta(&ctrl[0], kRouterCtas, &s_last)) return;
+  trace_point(1, 6);
 
   // ---- last CTA: scores, top-6, weights, slot table (one warp per row)
   int32_t *sel_idx = reinterpret_cast<int32_t *>(ws + lay.sel_idx);
@@ -262,12 +300,10 @@ __global__ void __launch_bounds__(kK1Threads)
   if (warp < B) {
     const int b = warp;
     double z0[8], z1[8];
-    float bias[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       z0[i] = ld_cg_f64(zp + (size_t)b * kE + lane + 32 * i);
       z1[i] = ld_cg_f64(zp + ((size_t)B + b) * kE + lane + 32 * i);
-      bias[i] = L.router_b[lane + 32 * i];
     }
     float sv[8];
     uint32_t key[8];
@@ -322,6 +358,7 @@ __global__ void __launch_bounds__(kK1Threads)
     }
   }
   __syncthreads();
+  trace_point(1, 7);
   // slot table: experts used by any row, ascending; one expert per thread
   const int e = tid;
   uint32_t m = 0;
@@ -357,6 +394,7 @@ __global__ void __launch_bounds__(kK1Threads)
     ctrl[2] = (uint32_t)total;
     ctrl[0] = 0;  // ready for the next call on this workspace
   }
+  trace_point(1, 3);
 }
 
 // ============================================================== K2: gate/up + SwiGLU
@@ -434,10 +472,13 @@ __global__ void __launch_bounds__(kK2Warps * 32)
   __shared__ double s_red[4 * kMaxB];
   __shared__ double s_inv[kMaxB];
   __shared__ uint32_t s_word;
+  __shared__ int s_aslot[kMaxB * kTopK];
+  __shared__ float s_aw[kMaxB * kTopK];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const int it = blockIdx.x;
   const bool shared_item_cta = it < kSharedItems;
   uint32_t *ctrl = reinterpret_cast<uint32_t *>(ws + lay.ctrl);
+  trace_point(2, 0);
 
   if (tid == 0) {
     mbar_init(&bar, 1);
@@ -445,11 +486,11 @@ __global__ void __launch_bounds__(kK2Warps * 32)
   }
   if (shared_item_cta) {
     // The input is final here: this grid was launched after K1 passed its wait.
-    if (kResidual) rms_inv(h, B, s_red, s_inv, tid);
-    stage_input_compact<kResidual>(frag, x_in, h, B, s_inv, tid, kK2Warps * 32);
+    stage_input<kResidual, kK2Warps * 32, 4>(frag, x_in, h, B, s_red, s_inv, tid);
   } else {
     pdl_wait();
     pdl_trigger();
+    trace_point(2, 1);
     if (tid == 0) {
       const uint32_t w =
           ld_cg_u32(reinterpret_cast<const uint32_t *>(ws + lay.slot_word) + ((it - kSharedItems) >> 6));
@@ -461,12 +502,16 @@ __global__ void __launch_bounds__(kK2Warps * 32)
         bulk_g2s(frag, ws + lay.xfrag, fbytes, &bar);
         issue_item(routed_item(L, (int)slot_expert(w), 8 * ((it - kSharedItems) & 63)), buf, &bar);
       }
+    } else if (tid >= 32 && tid < 32 + B * kTopK) {  // the rows' slots and weights, meanwhile
+      s_aslot[tid - 32] = (int)ld_cg_u32(reinterpret_cast<const uint32_t *>(ws + lay.asc_slot) + tid - 32);
+      s_aw[tid - 32] = ld_cg_f32(reinterpret_cast<const float *>(ws + lay.asc_w) + tid - 32);
     }
   }
   __syncthreads();
   const uint32_t word = shared_item_cta ? 0u : s_word;
   if (word == kSlotInvalid) return;  // a slot past the routed experts of this call
   const bool ok = mbar_wait(&bar, 0);
+  trace_point(2, 2);
   if (__syncthreads_or(!ok)) {
     if (tid == 0) set_status(ctrl + 1, kStatusTimeout);
     if (!ok) mbar_wait(&bar, 0);
@@ -478,9 +523,11 @@ __global__ void __launch_bounds__(kK2Warps * 32)
   }
   float acc[4];
   item_part(buf, frag, B, warp, lane, acc);
+  trace_point(2, 4);
 #pragma unroll
   for (int i = 0; i < 4; ++i) s_acc[warp][lane][i] = acc[i];
   __syncthreads();
+  trace_point(2, 5);
   if (warp == 0) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -498,8 +545,6 @@ __global__ void __launch_bounds__(kK2Warps * 32)
     } else {
       const int u = (it - kSharedItems) >> 6, r0 = 8 * ((it - kSharedItems) & 63);
       const uint32_t mask = slot_mask(word);
-      const int32_t *asc_slot = reinterpret_cast<const int32_t *>(ws + lay.asc_slot);
-      const float *asc_w = reinterpret_cast<const float *>(ws + lay.asc_w);
       uint16_t *hfr = reinterpret_cast<uint16_t *>(ws + lay.hfr);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
@@ -508,8 +553,8 @@ __global__ void __launch_bounds__(kK2Warps * 32)
           int j = 0;
 #pragma unroll
           for (int jj = 0; jj < kTopK; ++jj)
-            if (ld_cg_u32(asc_slot + b * kTopK + jj) == (uint32_t)u) j = jj;
-          const float w = ld_cg_f32(asc_w + b * kTopK + j);
+            if (s_aslot[b * kTopK + jj] == u) j = jj;
+          const float w = s_aw[b * kTopK + j];
           uint16_t *img = hfr + (size_t)((b * kTopK + j) * 2) * kI;
           write_hilo(img, img + kI, r0 + g, w * (silu_f(acc[c]) * acc[2 + c]));
         }
@@ -520,13 +565,14 @@ __global__ void __launch_bounds__(kK2Warps * 32)
     pdl_wait();
     pdl_trigger();
   }
+  trace_point(2, 3);
 }
 
 // ============================================================== K3: down + combine
 // Shared-memory plan (bytes): weights [umax][16 rows][256] | scales
 // [umax][16][4] bf16 | shared down [16][512] | shared scales [16][8] |
 // intermediates (kStage) routed [B][6][2][512] bf16, shared [B][2][1024] |
-// per-row results [8][8][16] fp32.
+// per-row partial results [8 rows][16 parts][16 columns] fp32.
 struct K3Smem {
   int umax, B;
   __host__ __device__ size_t w() const { return 0; }
@@ -538,7 +584,7 @@ struct K3Smem {
   __host__ __device__ size_t ysel(bool stage) const {
     return stage ? hs() + (size_t)B * 2 * kIs * 2 : hr();
   }
-  __host__ __device__ size_t total(bool stage) const { return ysel(stage) + 8 * 8 * 16 * 4; }
+  __host__ __device__ size_t total(bool stage) const { return ysel(stage) + 8 * 16 * 16 * 4; }
 };
 
 template <bool kResidual, bool kStage>
@@ -562,12 +608,15 @@ __global__ void __launch_bounds__(kK3Threads)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const int n0 = blockIdx.x * 16;
   uint32_t *ctrl = reinterpret_cast<uint32_t *>(ws + lay.ctrl);
+  trace_point(3, 0);
 
   // Routing is final here (K2 triggered this launch after its own wait on
   // K1): fetch the chosen experts' down rows before waiting on K2.
   if (tid == 0) mbar_init(&bar, 1);
   __syncthreads();
-  {
+  float h_old = 0.f;  // this thread's residual element (final: K1 waited for it)
+  if (kResidual && tid < 16 * B) h_old = ld_cg_f32(h + (size_t)(tid >> 4) * kH + n0 + (tid & 15));
+  if (tid < kE) {
     const uint32_t word = ld_cg_u32(reinterpret_cast<const uint32_t *>(ws + lay.slot_word) + tid);
     if (word != kSlotInvalid) {
       const size_t e = slot_expert(word);
@@ -577,19 +626,20 @@ __global__ void __launch_bounds__(kK3Threads)
       bulk_g2s(ssm + tid * 128, L.w2_s + (e * kH + n0) * (kI / kG), 128, &bar);
       if (tid == 0) s_ns = slot_count(word);
     }
-    if (tid == kK3Threads - 1) {
-      mbar_add_tx(&bar, 8192 + 256);
-      bulk_g2s(shm, L.sh2_q + (size_t)n0 * (kIs / 2), 8192, &bar);
-      bulk_g2s(shs, L.sh2_s + (size_t)n0 * (kIs / kG), 256, &bar);
-    }
-    if (tid < B * kTopK)
-      s_asc[tid] = (int)ld_cg_u32(reinterpret_cast<const uint32_t *>(ws + lay.asc_slot) + tid);
+  } else if (tid == kE) {
+    mbar_add_tx(&bar, 8192 + 256);
+    bulk_g2s(shm, L.sh2_q + (size_t)n0 * (kIs / 2), 8192, &bar);
+    bulk_g2s(shs, L.sh2_s + (size_t)n0 * (kIs / kG), 256, &bar);
+  } else if (tid >= kE + 32 && tid < kE + 32 + B * kTopK) {
+    const int i = tid - kE - 32;
+    s_asc[i] = (int)ld_cg_u32(reinterpret_cast<const uint32_t *>(ws + lay.asc_slot) + i);
   }
   __syncthreads();
   if (tid == 0) mbar_arrive(&bar);
 
   pdl_wait();
   pdl_trigger();
+  trace_point(3, 1);
   if (kStage) {
     const unsigned char *src_r = reinterpret_cast<const unsigned char *>(ws + lay.hfr);
     const unsigned char *src_s = reinterpret_cast<const unsigned char *>(ws + lay.hfs);
@@ -607,19 +657,22 @@ __global__ void __launch_bounds__(kK3Threads)
     return;
   }
   const int ns = s_ns;
+  trace_point(3, 2);
 
   const uint16_t *gr = kStage ? himg_r : reinterpret_cast<const uint16_t *>(ws + lay.hfr);
   const uint16_t *gs = kStage ? himg_s : reinterpret_cast<const uint16_t *>(ws + lay.hfs);
-  // tasks: routed slots 0..ns-1, then the shared expert's two k-halves
-  for (int task = warp; task < ns + 2; task += kK3Threads / 32) {
-    const bool sh = task >= ns;
-    const int half = task - ns;
+  // tasks: two k-parts (2 groups each) of routed slots 0..ns-1, then four
+  // k-parts of the shared expert; partial sums land in ysel[b][m] with
+  // m = 2j + part for the row's j-th expert (ascending), 12 + part shared.
+  for (int task = warp; task < 2 * ns + 4; task += kK3Threads / 32) {
+    const bool sh = task >= 2 * ns;
+    const int slot = task >> 1;
+    const int part = sh ? task - 2 * ns : task & 1;
     const int rowbytes = sh ? kIs / 2 : kI / 2;
-    const int gbase = sh ? 4 * half : 0;  // first k-group of this task
-    const unsigned char *wbase = sh ? shm : wsm + task * 4096;
-    const uint16_t *sc = reinterpret_cast<const uint16_t *>(sh ? shs : ssm + task * 128);
+    const unsigned char *wbase = sh ? shm : wsm + slot * 4096;
+    const uint16_t *sc = reinterpret_cast<const uint16_t *>(sh ? shs : ssm + slot * 128);
     const int spr = sh ? kIs / kG : kI / kG;
-    const uint32_t mask = sh ? ((1u << B) - 1u) : s_rows[task];
+    const uint32_t mask = sh ? ((1u << B) - 1u) : s_rows[slot];
     // this lane supplies activation column g
     const uint16_t *img = nullptr;
     int stride = 0;
@@ -630,15 +683,15 @@ __global__ void __launch_bounds__(kK3Threads)
       } else {
         int j = 0;
         for (int jj = 0; jj < kTopK; ++jj)
-          if (s_asc[g * kTopK + jj] == task) j = jj;
+          if (s_asc[g * kTopK + jj] == slot) j = jj;
         img = gr + (size_t)((g * kTopK + j) * 2) * kI;
         stride = kI;
       }
     }
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int G = gbase + k;
+    for (int k = 0; k < 2; ++k) {
+      const int G = 2 * part + k;
       uint32_t xh[16], xl[16];
       if (img) {
 #pragma unroll
@@ -679,29 +732,32 @@ __global__ void __launch_bounds__(kK3Threads)
     for (int c = 0; c < 2; ++c) {
       const int b = 2 * t + c;
       if (b < B && ((mask >> b) & 1u)) {
-        int j = kTopK + half;  // shared halves: 6, 7
+        int m = 12 + part;
         if (!sh)
           for (int jj = 0; jj < kTopK; ++jj)
-            if (s_asc[b * kTopK + jj] == task) j = jj;
-        ysel[(b * 8 + j) * 16 + g] = acc[c];
-        ysel[(b * 8 + j) * 16 + g + 8] = acc[2 + c];
+            if (s_asc[b * kTopK + jj] == slot) m = 2 * jj + part;
+        ysel[(b * 16 + m) * 16 + g] = acc[c];
+        ysel[(b * 16 + m) * 16 + g + 8] = acc[2 + c];
       }
     }
   }
+  trace_point(3, 4);
   __syncthreads();
+  trace_point(3, 5);
   if (tid < 16 * B) {
     const int n = tid & 15, b = tid >> 4;
     float y = 0.f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) y += ysel[(b * 8 + j) * 16 + n];
+    for (int m = 0; m < 16; ++m) y += ysel[(b * 16 + m) * 16 + n];
     const size_t o = (size_t)b * kH + n0 + n;
     if (kResidual) {
       const float yb = __bfloat162float(__float2bfloat16_rn(y));
-      h[o] = ld_cg_f32(h + o) + yb;
+      h[o] = h_old + yb;
     } else {
       out[o] = f32_to_bf16_bits(y);
     }
   }
+  trace_point(3, 3);
 }
 
 // ============================================================== host
@@ -729,7 +785,7 @@ static int current_device() {
 
 // dynamic shared memory cap: the 227 KB opt-in limit minus K3's static arrays
 constexpr size_t kK3MaxSmem = 224 * 1024;
-constexpr int kK1Smem = 16 * 2048 + kXFragBytes / 2;
+constexpr int kK1Smem = 16 * 2048 + kXFragBytes;
 constexpr int kK2Smem = kItemBytes + kXFragBytes;  // item + compact fragment for B <= 8
 
 template <bool kResidual>
@@ -781,6 +837,23 @@ static cudaError_t launch_decode_t(const LayerArgs &L, const uint16_t *x, float 
   return launch_pdl(k3_down_combine<kResidual, false>, kH / 16, kK3Threads, P.total(false), st, L,
                     B, out, h, ws, lay, umax);
 }
+
+#ifdef FLINT_TRACE
+extern "C" FLINT_API int flint_trace_dump(unsigned long long *t, unsigned int *tag, int cap) {
+  unsigned int n = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  cudaMemcpyFromSymbol(&n, g_trace_n, sizeof(n));
+  if (n > kTraceCap) n = kTraceCap;
+  if ((int)n > cap) n = (unsigned)cap;  // unwritten records (events not reached) keep tag 0
+  cudaMemcpyFromSymbol(t, g_trace_time, sizeof(unsigned long long) * n);
+  cudaMemcpyFromSymbol(tag, g_trace_tag, sizeof(unsigned int) * n);
+  const unsigned int zero = 0;
+  cudaMemcpyToSymbol(g_trace_n, &zero, sizeof(zero));
+  static unsigned int zeros[kTraceCap];
+  cudaMemcpyToSymbol(g_trace_tag, zeros, sizeof(zeros));
+  return (int)n;
+}
+#endif
 
 cudaError_t launch_decode(const LayerArgs &L, const uint16_t *x, const float *h_in, float *h_out,
                           int B, uint16_t *out, int32_t *idx_out, float *w_out, char *ws,
