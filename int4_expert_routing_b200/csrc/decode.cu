@@ -44,14 +44,14 @@ constexpr unsigned kTraceCap = 1u << 18;
 static __device__ unsigned long long g_trace_time[kTraceCap];
 static __device__ unsigned int g_trace_tag[kTraceCap];
 static __device__ unsigned int g_trace_n;
-// Event 0 (kernel start) reserves the CTA's eight records with one atomic,
+// Event 0 (kernel start) reserves the CTA's 16 records with one atomic,
 // before any wait; later events are plain stores.
-FLINT_DEV void trace_point(uint32_t kernel, uint32_t event) {
+FLINT_DEV void trace_point(uint32_t kernel, uint32_t event, uint32_t dep = 0) {
   __shared__ unsigned s_base;
   if (threadIdx.x == 0) {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    if (event == 0) s_base = atomicAdd(&g_trace_n, 8u);
+    unsigned long long t;  // dep: a value the mark must wait for
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t) : "r"(dep));
+    if (event == 0) s_base = atomicAdd(&g_trace_n, 16u);
     const unsigned i = s_base + event;
     if (i < kTraceCap) {
       g_trace_time[i] = t;
@@ -60,13 +60,17 @@ FLINT_DEV void trace_point(uint32_t kernel, uint32_t event) {
   }
 }
 #else
-FLINT_DEV void trace_point(uint32_t, uint32_t) {}
+FLINT_DEV void trace_point(uint32_t, uint32_t, uint32_t = 0) {}
 #endif
 
 constexpr int kRouterCtas = 32;   // 16 expert tiles x 2 k-halves
 constexpr int kK1Threads = 256;   // 8 warps: one 128-wide k-group each
+static_assert(kK1Threads == kE, "the last router CTA scores one expert per thread");
 constexpr int kK3Threads = 512;
 constexpr int kXFragBytes = 16 * 128 * 16;  // 16 groups x 128 uint4
+// Router rows sit 2064 B apart in shared memory (16 B of padding) so that the
+// eight rows a fragment load touches fall in different banks.
+constexpr int kRouterRowStride = 2048 + 16;
 
 FLINT_DEV float silu_f(float v) { return v / (1.f + expf(-v)); }
 
@@ -82,8 +86,8 @@ FLINT_DEV void write_hilo(uint16_t *img_hi, uint16_t *img_lo, int k, float v) {
 // RMSNorm scale 1/sqrt(mean(h^2) + eps) per row, fp64, in one fixed order
 // whatever the block size: 128 "lanes" t each sum the squares of elements
 // t, t+128, ..., t+1920 in that order, then an xor tree inside each warp of
-// 32 consecutive t, then the four warps in order.  K1 and K2 both call
-// rms_stage, so they normalize to the same bits.
+// 32 consecutive t, then the four warps in order.  Every K1 CTA runs the
+// same code on the same row, so all of them normalize to the same bits.
 //
 // The normalized row, rounded to bf16 (fp64 product, one rounding), goes
 // straight into the compact mma fragment: for element k of row b the slot is
@@ -97,10 +101,11 @@ FLINT_DEV int compact_slot(int b, int k, int B) {
 
 // All kThreads threads; rows are taken kThreads/128 at a time, each thread
 // holding up to kRowsPerPass rows' 16 elements in registers so that every
-// load of a pass is in flight at once.
-template <int kThreads, int kRowsPerPass>
-FLINT_DEV void rms_stage(const float *h, int B, double *s_red /*[4 * kMaxB]*/, double *s_inv,
-                         uint16_t *frag16, int tid) {
+// load of a pass is in flight at once.  The scale needs the whole row; only
+// k-groups g_lo .. g_lo+7 are converted into the fragment.
+template <int kThreads, int kRowsPerPass, int kTraceK = 0>
+FLINT_DEV void rms_stage(const float *h, int B, int g_lo, double *s_red /*[4 * kMaxB]*/,
+                         double *s_inv, uint16_t *frag16, int tid) {
   constexpr int kPar = kThreads / 128;
   const int t = tid & 127, hv = tid >> 7, lane = tid & 31, tw = t >> 5;
   for (int p0 = 0; p0 < B; p0 += kPar * kRowsPerPass) {
@@ -113,6 +118,7 @@ FLINT_DEV void rms_stage(const float *h, int B, double *s_red /*[4 * kMaxB]*/, d
         for (int j = 0; j < 16; ++j) v[r][j] = __ldcg(h + (size_t)b * kH + t + 128 * j);
       }
     }
+    if (kTraceK && p0 == 0) trace_point(kTraceK, 13, __float_as_uint(v[0][15]));
 #pragma unroll
     for (int r = 0; r < kRowsPerPass; ++r) {
       const int b = p0 + hv + kPar * r;
@@ -132,6 +138,7 @@ FLINT_DEV void rms_stage(const float *h, int B, double *s_red /*[4 * kMaxB]*/, d
       s_inv[tid] = 1.0 / sqrt(ss / kH + FLINT_RMS_EPS);
     }
     __syncthreads();
+    if (kTraceK && p0 == 0) trace_point(kTraceK, 14);
 #pragma unroll
     for (int r = 0; r < kRowsPerPass; ++r) {
       const int b = p0 + hv + kPar * r;
@@ -139,18 +146,22 @@ FLINT_DEV void rms_stage(const float *h, int B, double *s_red /*[4 * kMaxB]*/, d
         const double sc = s_inv[b];
 #pragma unroll
         for (int j = 0; j < 16; ++j)
-          frag16[compact_slot(b, t + 128 * j, B)] =
-              (uint16_t)f64_to_bf16_bits((double)v[r][j] * sc);
+          if ((unsigned)(j - g_lo) < 8u)
+            frag16[compact_slot(b, t + 128 * j, B)] =
+                (uint16_t)f64_to_bf16_bits((double)v[r][j] * sc);
       }
     }
   }
   __syncthreads();
 }
 
-// Compact fragment of a bf16 input (plain decode): frag[(G * 4B + 4g + t) * 4 + q].
-FLINT_DEV void stage_x_compact(uint4 *frag, const uint16_t *x_in, int B, int tid, int nthreads) {
-  const int n = 16 * 4 * B * 4;
-  for (int task = tid; task < n; task += nthreads) {
+// Compact fragment of a bf16 input (plain decode), k-groups g_lo .. g_lo+7:
+// frag[(G * 4B + 4g + t) * 4 + q].
+FLINT_DEV void stage_x_compact(uint4 *frag, const uint16_t *x_in, int B, int g_lo, int tid,
+                               int nthreads) {
+  const int n = 8 * 4 * B * 4, base = g_lo * 4 * B * 4;
+  for (int i = tid; i < n; i += nthreads) {
+    const int task = base + i;
     const int q = task & 3, gt = (task >> 2) % (4 * B), G = (task >> 2) / (4 * B);
     const int gg = gt >> 2, tt = gt & 3;
     frag[task] = bf16x8_to_pairs(ld_cg_v4(x_in + (size_t)gg * kH + 128 * G + 32 * tt + 8 * q));
@@ -158,13 +169,14 @@ FLINT_DEV void stage_x_compact(uint4 *frag, const uint16_t *x_in, int B, int tid
   __syncthreads();
 }
 
-template <bool kResidual, int kThreads, int kRowsPerPass>
-FLINT_DEV void stage_input(uint4 *frag, const uint16_t *x_in, const float *h, int B,
+template <bool kResidual, int kThreads, int kRowsPerPass, int kTraceK = 0>
+FLINT_DEV void stage_input(uint4 *frag, const uint16_t *x_in, const float *h, int B, int g_lo,
                            double *s_red, double *s_inv, int tid) {
   if (kResidual)
-    rms_stage<kThreads, kRowsPerPass>(h, B, s_red, s_inv, reinterpret_cast<uint16_t *>(frag), tid);
+    rms_stage<kThreads, kRowsPerPass, kTraceK>(h, B, g_lo, s_red, s_inv,
+                                               reinterpret_cast<uint16_t *>(frag), tid);
   else
-    stage_x_compact(frag, x_in, B, tid, kThreads);
+    stage_x_compact(frag, x_in, B, g_lo, tid, kThreads);
 }
 
 FLINT_DEV void load_frag_compact(const uint4 *frag, int G, int B, int lane, uint32_t (&x)[16]) {
@@ -187,6 +199,11 @@ constexpr uint32_t kSlotInvalid = 0xffffffffu;
 FLINT_DEV uint32_t slot_expert(uint32_t w) { return w & 0xffu; }
 FLINT_DEV uint32_t slot_mask(uint32_t w) { return (w >> 8) & 0xffu; }
 FLINT_DEV int slot_count(uint32_t w) { return (int)((w >> 16) & 0x1ffu); }
+// Index of the i-th set bit (i from 0) of m; m has more than i bits set.
+FLINT_DEV int nth_bit(uint32_t m, int i) {
+  for (int r = 0; r < i; ++r) m &= m - 1u;
+  return __ffs(m) - 1;
+}
 
 // Release-publish this CTA's results and tell whether it is the last of
 // `nctas` to do so; one fence per CTA on each side of the counter.
@@ -206,8 +223,8 @@ __global__ void __launch_bounds__(kK1Threads)
     k1_router(LayerArgs L, const uint16_t *__restrict__ x_in, const float *__restrict__ h, int B,
               char *__restrict__ ws, DecodeLayout lay, int32_t *__restrict__ idx_out,
               float *__restrict__ w_out) {
-  extern __shared__ __align__(128) unsigned char sm[];  // [16 rows][2048 B] | compact x fragment
-  uint4 *frag = reinterpret_cast<uint4 *>(sm + 16 * 2048);
+  extern __shared__ __align__(128) unsigned char sm[];  // [16 rows][2064 B] | compact x fragment
+  uint4 *frag = reinterpret_cast<uint4 *>(sm + 16 * kRouterRowStride);
   __shared__ __align__(8) uint64_t bar;
   __shared__ double s_part[8][kMaxB][16];
   __shared__ double s_red[4 * kMaxB];
@@ -219,6 +236,10 @@ __global__ void __launch_bounds__(kK1Threads)
   __shared__ int s_slot_e[kE];
   __shared__ uint32_t s_slot_m[kE];
   __shared__ int s_wcount[8];
+  __shared__ __align__(16) uint32_t s_key[kMaxB][kE];  // selection keys, one row per warp
+  __shared__ float s_sv[kMaxB][kE];
+  __shared__ int s_sel_e[kMaxB][kTopK];
+  __shared__ float s_sel_s[kMaxB][kTopK];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   uint32_t *ctrl = reinterpret_cast<uint32_t *>(ws + lay.ctrl);
@@ -233,24 +254,19 @@ __global__ void __launch_bounds__(kK1Threads)
   }
   __syncthreads();
   if (tid < 16)
-    bulk_g2s(sm + tid * 2048, L.router_w + (size_t)(16 * et + tid) * kH + kh * (kH / 2), 2048, &bar);
-  // selection bias for the last CTA's top-6 (lane + 32 i), also a weight
-  float bias[8];
-  if (warp < B) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) bias[i] = __ldg(L.router_b + lane + 32 * i);
-  }
+    bulk_g2s(sm + tid * kRouterRowStride, L.router_w + (size_t)(16 * et + tid) * kH + kh * (kH / 2), 2048, &bar);
+  // selection bias of expert tid for the last CTA's top-6, also a weight
+  const float bias = __ldg(L.router_b + tid);
   pdl_wait();
   pdl_trigger();
   trace_point(1, 1);
 
-  stage_input<kResidual, kK1Threads, 4>(frag, x_in, h, B, s_red, s_inv, tid);
+  stage_input<kResidual, kK1Threads, 4, 1>(frag, x_in, h, B, 8 * kh, s_red, s_inv, tid);
   trace_point(1, 4);
-  {  // publish the fragment (each CTA a share) for the routed gate/up CTAs
-    const int n = 256 * B;  // uint4 per call: 4096 B per row
-    uint4 *dst = reinterpret_cast<uint4 *>(ws + lay.xfrag);
-    for (int i = blockIdx.x * kK1Threads + tid; i < n; i += kRouterCtas * kK1Threads)
-      dst[i] = frag[i];
+  {  // publish this k-half of the fragment (the 16 CTAs of the half a share each)
+    const int per = 8 * B;  // uint4: the half is 128 B uint4, split 16 ways
+    const int i = (8 * kh) * 4 * B * 4 + et * per + tid;
+    if (tid < per) reinterpret_cast<uint4 *>(ws + lay.xfrag)[i] = frag[i];
   }
   const bool ok = mbar_wait(&bar, 0);
   if (__syncthreads_or(!ok)) {
@@ -264,9 +280,9 @@ __global__ void __launch_bounds__(kK1Threads)
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const uint4 a = bf16x8_to_pairs(
-          *reinterpret_cast<const uint4 *>(sm + g * 2048 + 256 * warp + 64 * t + 16 * q));
+          *reinterpret_cast<const uint4 *>(sm + g * kRouterRowStride + 256 * warp + 64 * t + 16 * q));
       const uint4 c = bf16x8_to_pairs(
-          *reinterpret_cast<const uint4 *>(sm + (g + 8) * 2048 + 256 * warp + 64 * t + 16 * q));
+          *reinterpret_cast<const uint4 *>(sm + (g + 8) * kRouterRowStride + 256 * warp + 64 * t + 16 * q));
       ra[4 * q] = a.x, ra[4 * q + 1] = a.y, ra[4 * q + 2] = a.z, ra[4 * q + 3] = a.w;
       rb[4 * q] = c.x, rb[4 * q + 1] = c.y, rb[4 * q + 2] = c.z, rb[4 * q + 3] = c.w;
     }
@@ -294,65 +310,65 @@ __global__ void __launch_bounds__(kK1Threads)
   if (!last_cta(&ctrl[0], kRouterCtas, &s_last)) return;
   trace_point(1, 6);
 
-  // ---- last CTA: scores, top-6, weights, slot table (one warp per row)
+  // ---- last CTA: scores, top-6, weights, slot table.  Thread e scores
+  // expert e of every row into shared memory; warp b then picks row b's 6
+  // best in 6 rounds, lane l holding experts 8l .. 8l+7: the lane's best live
+  // key (ties to the lower expert), the warp's largest key, the lowest lane
+  // holding it (= the lowest expert).  Rounds 0..5 give the selection order.
   int32_t *sel_idx = reinterpret_cast<int32_t *>(ws + lay.sel_idx);
   float *sel_w = reinterpret_cast<float *>(ws + lay.sel_w);
+  {
+    double zz[kMaxB];
+#pragma unroll
+    for (int b = 0; b < kMaxB; ++b)
+      if (b < B) zz[b] = ld_cg_f64(zp + (size_t)b * kE + tid) + ld_cg_f64(zp + ((size_t)B + b) * kE + tid);
+#pragma unroll
+    for (int b = 0; b < kMaxB; ++b) {
+      if (b < B) {
+        const float sv = 1.f / (1.f + expf(-(float)zz[b]));
+        s_key[b][tid] = float_key(sv + bias);
+        s_sv[b][tid] = sv;
+      }
+    }
+  }
+  trace_point(1, 10);
+  __syncthreads();
   if (warp < B) {
     const int b = warp;
-    double z0[8], z1[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      z0[i] = ld_cg_f64(zp + (size_t)b * kE + lane + 32 * i);
-      z1[i] = ld_cg_f64(zp + ((size_t)B + b) * kE + lane + 32 * i);
-    }
-    float sv[8];
-    uint32_t key[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float zf = (float)(z0[i] + z1[i]);
-      const float s = 1.f / (1.f + expf(-zf));
-      sv[i] = s;
-      key[i] = float_key(s + bias[i]);
-    }
-    uint32_t taken = 0;
-    int sel_e[kTopK];
-    float sel_s[kTopK];
+    const uint4 ka = *reinterpret_cast<const uint4 *>(&s_key[b][8 * lane]);
+    const uint4 kb = *reinterpret_cast<const uint4 *>(&s_key[b][8 * lane + 4]);
+    const uint32_t key[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
+    uint32_t live = 0xffu;
 #pragma unroll
     for (int j = 0; j < kTopK; ++j) {
       uint32_t best = 0;
-      int bi = -1;
+      int bi = 0;
 #pragma unroll
       for (int i = 0; i < 8; ++i)
-        if (!((taken >> i) & 1u) && key[i] > best) best = key[i], bi = i;
+        if (((live >> i) & 1u) && key[i] > best) best = key[i], bi = i;
       const uint32_t m = __reduce_max_sync(0xffffffffu, best);
-      const uint32_t cand = (bi >= 0 && best == m) ? (uint32_t)(lane + 32 * bi) : 0xffffffffu;
-      const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
-      float mys = 0.f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if (i == bi) mys = sv[i];
-      sel_s[j] = __shfl_sync(0xffffffffu, mys, (int)(win & 31));
-      sel_e[j] = (int)win;
-      if (lane == (int)(win & 31)) taken |= 1u << (win >> 5);
+      const uint32_t win = __ballot_sync(0xffffffffu, live != 0u && best == m);
+      if (lane == __ffs(win) - 1) {
+        live &= ~(1u << bi);
+        s_sel_e[b][j] = 8 * lane + bi;
+        s_sel_s[b][j] = s_sv[b][8 * lane + bi];
+      }
     }
-    float ssum = 0.f;
-#pragma unroll
-    for (int j = 0; j < kTopK; ++j) ssum += sel_s[j];
-    // lane j < 6 writes entry j; ascending order by counting smaller experts
+    __syncwarp();
+    trace_point(1, 11);
     if (lane < kTopK) {
-      int e_me = sel_e[0];
-      float s_me = sel_s[0];
+      float ssum = 0.f;
 #pragma unroll
-      for (int j = 1; j < kTopK; ++j)
-        if (lane == j) e_me = sel_e[j], s_me = sel_s[j];
-      const float w_me = s_me / ssum;
+      for (int j = 0; j < kTopK; ++j) ssum += s_sel_s[b][j];
+      const int e_me = s_sel_e[b][lane];
+      const float w_me = s_sel_s[b][lane] / ssum;
       sel_idx[b * kTopK + lane] = e_me;
       sel_w[b * kTopK + lane] = w_me;
       if (idx_out) idx_out[b * kTopK + lane] = e_me;
       if (w_out) w_out[b * kTopK + lane] = w_me;
-      int rank = 0;
+      int rank = 0;  // ascending expert order
 #pragma unroll
-      for (int j = 0; j < kTopK; ++j) rank += sel_e[j] < e_me;
+      for (int j = 0; j < kTopK; ++j) rank += s_sel_e[b][j] < e_me;
       s_asc_e[b][rank] = e_me;
       s_asc_w[b][rank] = w_me;
     }
@@ -390,6 +406,7 @@ __global__ void __launch_bounds__(kK1Threads)
     asc_slot[tid] = s_slot_of[s_asc_e[b][j]];
     asc_w[tid] = s_asc_w[b][j];
   }
+  trace_point(1, 12);
   if (tid == 0) {
     ctrl[2] = (uint32_t)total;
     ctrl[0] = 0;  // ready for the next call on this workspace
@@ -401,8 +418,9 @@ __global__ void __launch_bounds__(kK1Threads)
 // One CTA per work item: 8 intermediate rows of one expert (shared expert:
 // items 0..127; routed: item 128 + 64u + r/8 for slot u).  The item's bytes
 // (8 gate rows, 8 up rows, their scales; 16.5 KB) arrive in shared memory by
-// four bulk copies; the 4 warps split the 16 k-groups and their partial sums
-// are added in warp order.
+// four bulk copies (the shared expert's before the wait on K1), the block
+// input fragment K1 published by one more after it; the 4 warps split the 16
+// k-groups and their partial sums are added in warp order.
 constexpr int kK2Warps = 4;
 constexpr int kItemBytes = 16384 + 512;
 constexpr int kSharedItems = kIs / 8;
@@ -424,9 +442,8 @@ FLINT_DEV ItemSrc routed_item(const LayerArgs &L, int e, int r0) {
   return ItemSrc{L.w13_q + row * (kH / 2), L.w13_q + (row + kI) * (kH / 2),
                  L.w13_s + row * (kH / kG), L.w13_s + (row + kI) * (kH / kG)};
 }
-// one thread
+// one thread; the caller accounts the bytes on the barrier (mbar_add_tx)
 FLINT_DEV void issue_item(const ItemSrc &src, unsigned char *buf, uint64_t *bar) {
-  mbar_expect_tx(bar, kItemBytes);
   bulk_g2s(buf, src.gate, 8192, bar);
   bulk_g2s(buf + 8192, src.up, 8192, bar);
   bulk_g2s(buf + 16384, src.gate_s, 256, bar);
@@ -460,17 +477,13 @@ FLINT_DEV void item_part(const unsigned char *buf, const uint4 *frag, int B, int
   }
 }
 
-template <bool kResidual>
 __global__ void __launch_bounds__(kK2Warps * 32)
-    k2_gateup(LayerArgs L, const uint16_t *__restrict__ x_in, const float *__restrict__ h, int B,
-              char *__restrict__ ws, DecodeLayout lay) {
+    k2_gateup(LayerArgs L, int B, char *__restrict__ ws, DecodeLayout lay) {
   extern __shared__ __align__(128) unsigned char sm[];  // item | x fragment (compact)
   unsigned char *buf = sm;
   uint4 *frag = reinterpret_cast<uint4 *>(sm + kItemBytes);
   __shared__ __align__(8) uint64_t bar;
   __shared__ float s_acc[kK2Warps][32][4];
-  __shared__ double s_red[4 * kMaxB];
-  __shared__ double s_inv[kMaxB];
   __shared__ uint32_t s_word;
   __shared__ int s_aslot[kMaxB * kTopK];
   __shared__ float s_aw[kMaxB * kTopK];
@@ -480,45 +493,48 @@ __global__ void __launch_bounds__(kK2Warps * 32)
   uint32_t *ctrl = reinterpret_cast<uint32_t *>(ws + lay.ctrl);
   trace_point(2, 0);
 
+  // The shared expert's rows do not depend on K1: fetch them before the wait.
+  // One arrival (thread 0, after the wait) closes the phase; every copy adds
+  // its bytes first, so the phase cannot complete early.
   if (tid == 0) {
     mbar_init(&bar, 1);
-    if (shared_item_cta) issue_item(shared_item(L, it), buf, &bar);
-  }
-  if (shared_item_cta) {
-    // The input is final here: this grid was launched after K1 passed its wait.
-    stage_input<kResidual, kK2Warps * 32, 4>(frag, x_in, h, B, s_red, s_inv, tid);
-  } else {
-    pdl_wait();
-    pdl_trigger();
-    trace_point(2, 1);
-    if (tid == 0) {
-      const uint32_t w =
-          ld_cg_u32(reinterpret_cast<const uint32_t *>(ws + lay.slot_word) + ((it - kSharedItems) >> 6));
-      s_word = w;
-      if (w != kSlotInvalid) {
-        // the block input as K1 staged it, and this item's weights
-        const uint32_t fbytes = 16u * 4u * (uint32_t)B * 64u;
-        mbar_add_tx(&bar, fbytes);  // issue_item makes the phase's single arrival
-        bulk_g2s(frag, ws + lay.xfrag, fbytes, &bar);
-        issue_item(routed_item(L, (int)slot_expert(w), 8 * ((it - kSharedItems) & 63)), buf, &bar);
-      }
-    } else if (tid >= 32 && tid < 32 + B * kTopK) {  // the rows' slots and weights, meanwhile
-      s_aslot[tid - 32] = (int)ld_cg_u32(reinterpret_cast<const uint32_t *>(ws + lay.asc_slot) + tid - 32);
-      s_aw[tid - 32] = ld_cg_f32(reinterpret_cast<const float *>(ws + lay.asc_w) + tid - 32);
+    if (shared_item_cta) {
+      mbar_add_tx(&bar, kItemBytes);
+      issue_item(shared_item(L, it), buf, &bar);
     }
   }
+  pdl_wait();  // K1 is complete: routing and the block input fragment are final
+  pdl_trigger();
+  trace_point(2, 1);
+  if (tid == 0) {
+    uint32_t w = 0;
+    if (!shared_item_cta) {
+      w = ld_cg_u32(reinterpret_cast<const uint32_t *>(ws + lay.slot_word) + ((it - kSharedItems) >> 6));
+      if (w != kSlotInvalid) {
+        mbar_add_tx(&bar, kItemBytes);
+        issue_item(routed_item(L, (int)slot_expert(w), 8 * ((it - kSharedItems) & 63)), buf, &bar);
+      }
+    }
+    s_word = w;
+    if (w != kSlotInvalid) {
+      const uint32_t fbytes = 16u * 4u * (uint32_t)B * 64u;
+      mbar_add_tx(&bar, fbytes);
+      bulk_g2s(frag, ws + lay.xfrag, fbytes, &bar);
+      mbar_arrive(&bar);
+    }
+  } else if (!shared_item_cta && tid >= 32 && tid < 32 + B * kTopK) {
+    // the rows' slots and weights, while the slot word is in flight
+    s_aslot[tid - 32] = (int)ld_cg_u32(reinterpret_cast<const uint32_t *>(ws + lay.asc_slot) + tid - 32);
+    s_aw[tid - 32] = ld_cg_f32(reinterpret_cast<const float *>(ws + lay.asc_w) + tid - 32);
+  }
   __syncthreads();
-  const uint32_t word = shared_item_cta ? 0u : s_word;
+  const uint32_t word = s_word;
   if (word == kSlotInvalid) return;  // a slot past the routed experts of this call
   const bool ok = mbar_wait(&bar, 0);
   trace_point(2, 2);
   if (__syncthreads_or(!ok)) {
     if (tid == 0) set_status(ctrl + 1, kStatusTimeout);
     if (!ok) mbar_wait(&bar, 0);
-    if (shared_item_cta) {
-      pdl_wait();
-      pdl_trigger();
-    }
     return;
   }
   float acc[4];
@@ -560,10 +576,6 @@ __global__ void __launch_bounds__(kK2Warps * 32)
         }
       }
     }
-  }
-  if (shared_item_cta) {
-    pdl_wait();
-    pdl_trigger();
   }
   trace_point(2, 3);
 }
@@ -664,6 +676,9 @@ __global__ void __launch_bounds__(kK3Threads)
   // tasks: two k-parts (2 groups each) of routed slots 0..ns-1, then four
   // k-parts of the shared expert; partial sums land in ysel[b][m] with
   // m = 2j + part for the row's j-th expert (ascending), 12 + part shared.
+  // The MMA's columns carry the task's rows R (those that chose the expert,
+  // every row for the shared one) as pairs: column 2i the hi image of row
+  // R[4p + i], column 2i+1 its lo image; one pass p per 4 rows.
   for (int task = warp; task < 2 * ns + 4; task += kK3Threads / 32) {
     const bool sh = task >= 2 * ns;
     const int slot = task >> 1;
@@ -673,71 +688,73 @@ __global__ void __launch_bounds__(kK3Threads)
     const uint16_t *sc = reinterpret_cast<const uint16_t *>(sh ? shs : ssm + slot * 128);
     const int spr = sh ? kIs / kG : kI / kG;
     const uint32_t mask = sh ? ((1u << B) - 1u) : s_rows[slot];
-    // this lane supplies activation column g
-    const uint16_t *img = nullptr;
-    int stride = 0;
-    if (g < B && ((mask >> g) & 1u)) {
-      if (sh) {
-        img = gs + (size_t)(2 * g) * kIs;
-        stride = kIs;
-      } else {
-        int j = 0;
-        for (int jj = 0; jj < kTopK; ++jj)
-          if (s_asc[g * kTopK + jj] == slot) j = jj;
-        img = gr + (size_t)((g * kTopK + j) * 2) * kI;
-        stride = kI;
+    const int nr = __popc(mask);
+    // this lane's column (g) in each pass, and its output row (t)
+    const uint16_t *img[2] = {nullptr, nullptr};
+    int orow[2] = {-1, -1}, om[2] = {0, 0};
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+      const int ic = 4 * p + (g >> 1), io = 4 * p + t;
+      if (ic < nr) {
+        const int b = nth_bit(mask, ic), hl = g & 1;
+        if (sh) {
+          img[p] = gs + (size_t)(2 * b + hl) * kIs;
+        } else {
+          int j = 0;
+          for (int jj = 0; jj < kTopK; ++jj)
+            if (s_asc[b * kTopK + jj] == slot) j = jj;
+          img[p] = gr + (size_t)((b * kTopK + j) * 2 + hl) * kI;
+        }
+      }
+      if (io < nr) {
+        const int b = nth_bit(mask, io);
+        orow[p] = b;
+        om[p] = 12 + part;
+        if (!sh)
+          for (int jj = 0; jj < kTopK; ++jj)
+            if (s_asc[b * kTopK + jj] == slot) om[p] = 2 * jj + part;
       }
     }
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const int G = 2 * part + k;
-      uint32_t xh[16], xl[16];
-      if (img) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int off = ((G * 4 + t) * 16 + 4 * i) * 2;
-          uint4 a, b;
-          if (kStage) {
-            a = *reinterpret_cast<const uint4 *>(img + off);
-            b = *reinterpret_cast<const uint4 *>(img + stride + off);
-          } else {
-            a = ld_cg_v4(img + off);
-            b = ld_cg_v4(img + stride + off);
-          }
-          xh[4 * i] = a.x, xh[4 * i + 1] = a.y, xh[4 * i + 2] = a.z, xh[4 * i + 3] = a.w;
-          xl[4 * i] = b.x, xl[4 * i + 1] = b.y, xl[4 * i + 2] = b.z, xl[4 * i + 3] = b.w;
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) xh[i] = xl[i] = 0u;
-      }
       const uint4 w0 = *reinterpret_cast<const uint4 *>(wbase + g * rowbytes + 64 * G + 16 * t);
       const uint4 w1 =
           *reinterpret_cast<const uint4 *>(wbase + (g + 8) * rowbytes + 64 * G + 16 * t);
       uint32_t ra[16], rb[16];
       int4x32_to_bf16x2(w0, ra);
       int4x32_to_bf16x2(w1, rb);
-      float d[4] = {0.f, 0.f, 0.f, 0.f};
-      group_mma_acc(ra, rb, xh, d);
-      group_mma_acc(ra, rb, xl, d);
       const float s0 = bf16_bits_to_f32(sc[g * spr + G]);
       const float s1 = bf16_bits_to_f32(sc[(g + 8) * spr + G]);
-      acc[0] = fmaf(d[0], s0, acc[0]);
-      acc[1] = fmaf(d[1], s0, acc[1]);
-      acc[2] = fmaf(d[2], s1, acc[2]);
-      acc[3] = fmaf(d[3], s1, acc[3]);
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {
+        if (4 * p < nr) {  // the same for the whole warp
+          uint32_t xb[16];
+          if (img[p]) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int off = ((G * 4 + t) * 16 + 4 * i) * 2;
+              const uint4 a = kStage ? *reinterpret_cast<const uint4 *>(img[p] + off)
+                                     : ld_cg_v4(img[p] + off);
+              xb[4 * i] = a.x, xb[4 * i + 1] = a.y, xb[4 * i + 2] = a.z, xb[4 * i + 3] = a.w;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) xb[i] = 0u;
+          }
+          float d[4] = {0.f, 0.f, 0.f, 0.f};
+          group_mma_acc(ra, rb, xb, d);
+          acc[p][0] = fmaf(d[0] + d[1], s0, acc[p][0]);
+          acc[p][1] = fmaf(d[2] + d[3], s1, acc[p][1]);
+        }
+      }
     }
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const int b = 2 * t + c;
-      if (b < B && ((mask >> b) & 1u)) {
-        int m = 12 + part;
-        if (!sh)
-          for (int jj = 0; jj < kTopK; ++jj)
-            if (s_asc[b * kTopK + jj] == slot) m = 2 * jj + part;
-        ysel[(b * 16 + m) * 16 + g] = acc[c];
-        ysel[(b * 16 + m) * 16 + g + 8] = acc[2 + c];
+    for (int p = 0; p < 2; ++p) {
+      if (orow[p] >= 0) {
+        ysel[(orow[p] * 16 + om[p]) * 16 + g] = acc[p][0];
+        ysel[(orow[p] * 16 + om[p]) * 16 + g + 8] = acc[p][1];
       }
     }
   }
@@ -785,7 +802,7 @@ static int current_device() {
 
 // dynamic shared memory cap: the 227 KB opt-in limit minus K3's static arrays
 constexpr size_t kK3MaxSmem = 224 * 1024;
-constexpr int kK1Smem = 16 * 2048 + kXFragBytes;
+constexpr int kK1Smem = 16 * kRouterRowStride + kXFragBytes;
 constexpr int kK2Smem = kItemBytes + kXFragBytes;  // item + compact fragment for B <= 8
 
 template <bool kResidual>
@@ -796,7 +813,7 @@ static cudaError_t set_attrs(int dev) {
   cudaError_t e = cudaFuncSetAttribute(k1_router<kResidual>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kK1Smem);
   if (e == cudaSuccess)
-    e = noted(cudaFuncSetAttribute(k2_gateup<kResidual>,
+    e = noted(cudaFuncSetAttribute(k2_gateup,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kK2Smem),
               "k2_gateup smem attribute");
   if (e == cudaSuccess)
@@ -825,9 +842,8 @@ static cudaError_t launch_decode_t(const LayerArgs &L, const uint16_t *x, float 
   const int umax = kTopK * B < kE ? kTopK * B : kE;
   const int n_items = kSharedItems + 64 * umax;
   note_step("k2_gateup launch");
-  err = launch_pdl(k2_gateup<kResidual>, n_items, kK2Warps * 32,
-                   (size_t)kItemBytes + (size_t)16 * 4 * B * 64, st, L, x, (const float *)h, B, ws,
-                   lay);
+  err = launch_pdl(k2_gateup, n_items, kK2Warps * 32,
+                   (size_t)kItemBytes + (size_t)16 * 4 * B * 64, st, L, B, ws, lay);
   if (err != cudaSuccess) return err;
   const K3Smem P{umax, B};
   note_step("k3_down_combine launch");
