@@ -20,8 +20,9 @@
 //      the shared expert).
 // "What vLLM changed" on the same page: the small-batch MoE kernels that read
 // only the selected experts were also the largest prefill gain.  SwiGLU
-// intermediates are bf16 (their range: TandemLLM "21 Flint", section 21.2
-// reports routed activations up to 2.6e5, past fp16).
+// intermediates travel as hi/lo bf16 pairs: bf16 range (TandemLLM "21 Flint",
+// section 21.2 reports routed activations up to 2.6e5, past fp16) with about
+// 16 significant bits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
