@@ -50,6 +50,8 @@ def parse():
     p.add_argument("--no-head", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
     p.add_argument("--no-prefill", action="store_true")
+    p.add_argument("--prefill-t", type=int, nargs="+", default=[2048, 4096, 32768],
+                   help="prefill token counts timed as extra lines")
     return p.parse_args()
 
 
@@ -407,7 +409,7 @@ def main():
     # ---- prefill of one MoE layer (layer 0): tokens/s and tensor-pipe roofline
     if not args.no_prefill and rank == 0:
         peak_tf, peak_kind_tf = tensor_peak()
-        for T in (2048, 4096, 32768):
+        for T in args.prefill_t:
             xt = synth.to_device({"x": synth.prefill_x(T, T)}, dev)["x"]
             out_t = torch.empty((T, H), dtype=torch.int16, device=dev)
             nbp = F.flint_workspace_bytes(F.FLINT_OP_PREFILL, T)
