@@ -477,105 +477,151 @@ FLINT_DEV void item_part(const unsigned char *buf, const uint4 *frag, int B, int
   }
 }
 
+constexpr int kK2Stages = 2;     // items in flight per CTA
+constexpr int kK2MaxItems = 16;  // items per CTA (the host sizes the grid to keep within it)
+
+// Item list of one call: shared items 0..127, then 64 items per routed slot.
+// CTA c takes items c, c + grid, c + 2 grid, ...; a CTA's first item is
+// fetched before the wait when it is a shared one.
 __global__ void __launch_bounds__(kK2Warps * 32)
-    k2_gateup(LayerArgs L, int B, char *__restrict__ ws, DecodeLayout lay) {
-  extern __shared__ __align__(128) unsigned char sm[];  // item | x fragment (compact)
-  unsigned char *buf = sm;
-  uint4 *frag = reinterpret_cast<uint4 *>(sm + kItemBytes);
-  __shared__ __align__(8) uint64_t bar;
+    k2_gateup(LayerArgs L, int B, int n_items, char *__restrict__ ws, DecodeLayout lay) {
+  extern __shared__ __align__(128) unsigned char sm[];  // stages | x fragment (compact)
+  uint4 *frag = reinterpret_cast<uint4 *>(sm + kK2Stages * kItemBytes);
+  __shared__ __align__(8) uint64_t bar[kK2Stages];
+  __shared__ __align__(8) uint64_t fbar;
   __shared__ float s_acc[kK2Warps][32][4];
-  __shared__ uint32_t s_word;
+  __shared__ uint32_t s_word[kK2MaxItems];
+  __shared__ int s_n;
   __shared__ int s_aslot[kMaxB * kTopK];
   __shared__ float s_aw[kMaxB * kTopK];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-  const int it = blockIdx.x;
-  const bool shared_item_cta = it < kSharedItems;
+  const int c0 = blockIdx.x, step = gridDim.x;
   uint32_t *ctrl = reinterpret_cast<uint32_t *>(ws + lay.ctrl);
+  const uint32_t *slot_word = reinterpret_cast<const uint32_t *>(ws + lay.slot_word);
   trace_point(2, 0);
 
-  // The shared expert's rows do not depend on K1: fetch them before the wait.
-  // One arrival (thread 0, after the wait) closes the phase; every copy adds
-  // its bytes first, so the phase cannot complete early.
+  // The shared expert's rows do not depend on K1.  Every copy adds its bytes
+  // before the phase's single arrival, so no phase can complete early.
   if (tid == 0) {
-    mbar_init(&bar, 1);
-    if (shared_item_cta) {
-      mbar_add_tx(&bar, kItemBytes);
-      issue_item(shared_item(L, it), buf, &bar);
+    for (int i = 0; i < kK2Stages; ++i) mbar_init(&bar[i], 1);
+    mbar_init(&fbar, 1);
+    if (c0 < kSharedItems) {
+      mbar_add_tx(&bar[0], kItemBytes);
+      issue_item(shared_item(L, c0), sm, &bar[0]);
     }
   }
   pdl_wait();  // K1 is complete: routing and the block input fragment are final
   pdl_trigger();
   trace_point(2, 1);
-  if (tid == 0) {
-    uint32_t w = 0;
-    if (!shared_item_cta) {
-      w = ld_cg_u32(reinterpret_cast<const uint32_t *>(ws + lay.slot_word) + ((it - kSharedItems) >> 6));
-      if (w != kSlotInvalid) {
-        mbar_add_tx(&bar, kItemBytes);
-        issue_item(routed_item(L, (int)slot_expert(w), 8 * ((it - kSharedItems) & 63)), buf, &bar);
-      }
-    }
-    s_word = w;
-    if (w != kSlotInvalid) {
-      const uint32_t fbytes = 16u * 4u * (uint32_t)B * 64u;
-      mbar_add_tx(&bar, fbytes);
-      bulk_g2s(frag, ws + lay.xfrag, fbytes, &bar);
-      mbar_arrive(&bar);
-    }
-  } else if (!shared_item_cta && tid >= 32 && tid < 32 + B * kTopK) {
-    // the rows' slots and weights, while the slot word is in flight
+  if (tid == 0) {  // every CTA takes the fragment (and waits for it, even with no item)
+    const uint32_t fbytes = 16u * 4u * (uint32_t)B * 64u;
+    mbar_add_tx(&fbar, fbytes);
+    bulk_g2s(frag, ws + lay.xfrag, fbytes, &fbar);
+    mbar_arrive(&fbar);
+  }
+  // this CTA's items: slot words read together (kSlotInvalid ends the list)
+  if (tid < kK2MaxItems) {
+    const int it = c0 + tid * step;
+    uint32_t w = kSlotInvalid;
+    if (it < kSharedItems) w = 0u;
+    else if (it < n_items) w = ld_cg_u32(slot_word + ((it - kSharedItems) >> 6));
+    s_word[tid] = w;
+  } else if (tid >= 32 && tid < 32 + B * kTopK) {
     s_aslot[tid - 32] = (int)ld_cg_u32(reinterpret_cast<const uint32_t *>(ws + lay.asc_slot) + tid - 32);
     s_aw[tid - 32] = ld_cg_f32(reinterpret_cast<const float *>(ws + lay.asc_w) + tid - 32);
   }
   __syncthreads();
-  const uint32_t word = s_word;
-  if (word == kSlotInvalid) return;  // a slot past the routed experts of this call
-  const bool ok = mbar_wait(&bar, 0);
-  trace_point(2, 2);
-  if (__syncthreads_or(!ok)) {
-    if (tid == 0) set_status(ctrl + 1, kStatusTimeout);
-    if (!ok) mbar_wait(&bar, 0);
-    return;
-  }
-  float acc[4];
-  item_part(buf, frag, B, warp, lane, acc);
-  trace_point(2, 4);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) s_acc[warp][lane][i] = acc[i];
-  __syncthreads();
-  trace_point(2, 5);
-  if (warp == 0) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      acc[i] = ((s_acc[0][lane][i] + s_acc[1][lane][i]) + s_acc[2][lane][i]) + s_acc[3][lane][i];
-    if (shared_item_cta) {
-      uint16_t *hfs = reinterpret_cast<uint16_t *>(ws + lay.hfs);
-      const int r = 8 * it + g;
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int b = 2 * t + c;
-        if (b < B)
-          write_hilo(hfs + (size_t)(2 * b) * kIs, hfs + (size_t)(2 * b + 1) * kIs, r,
-                     silu_f(acc[c]) * acc[2 + c]);
-      }
-    } else {
-      const int u = (it - kSharedItems) >> 6, r0 = 8 * ((it - kSharedItems) & 63);
-      const uint32_t mask = slot_mask(word);
-      uint16_t *hfr = reinterpret_cast<uint16_t *>(ws + lay.hfr);
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int b = 2 * t + c;
-        if (b < B && ((mask >> b) & 1u)) {
-          int j = 0;
-#pragma unroll
-          for (int jj = 0; jj < kTopK; ++jj)
-            if (s_aslot[b * kTopK + jj] == u) j = jj;
-          const float w = s_aw[b * kTopK + j];
-          uint16_t *img = hfr + (size_t)((b * kTopK + j) * 2) * kI;
-          write_hilo(img, img + kI, r0 + g, w * (silu_f(acc[c]) * acc[2 + c]));
+  if (tid == 0) {
+    int n = 0;
+    while (n < kK2MaxItems && s_word[n] != kSlotInvalid) ++n;
+    s_n = n;
+    if (n > 0) {
+      for (int j = 0; j < n && j < kK2Stages; ++j) {
+        const int it = c0 + j * step;
+        if (j == 0 && it < kSharedItems) {
+          mbar_arrive(&bar[0]);  // fetched before the wait
+        } else {
+          mbar_add_tx(&bar[j], kItemBytes);
+          issue_item(it < kSharedItems ? shared_item(L, it)
+                                       : routed_item(L, (int)slot_expert(s_word[j]),
+                                                     8 * ((it - kSharedItems) & 63)),
+                     sm + j * kItemBytes, &bar[j]);
+          mbar_arrive(&bar[j]);
         }
       }
     }
+  }
+  __syncthreads();
+  const int n = s_n;
+  bool ok = mbar_wait(&fbar, 0);
+  if (n == 0) {
+    if (!ok && tid == 0) set_status(ctrl + 1, kStatusTimeout);
+    return;
+  }
+  for (int j = 0; j < n; ++j) {
+    const int st = j % kK2Stages;
+    const int it = c0 + j * step;
+    const uint32_t word = s_word[j];
+    unsigned char *buf = sm + st * kItemBytes;
+    ok = mbar_wait(&bar[st], (uint32_t)((j / kK2Stages) & 1)) && ok;
+    trace_point(2, 2);
+    if (__syncthreads_or(!ok)) {
+      if (tid == 0) set_status(ctrl + 1, kStatusTimeout);
+      // copies still in flight get one more bounded wait each
+      for (int jj = j; jj < n && jj < j + kK2Stages; ++jj)
+        mbar_wait(&bar[jj % kK2Stages], (uint32_t)((jj / kK2Stages) & 1));
+      return;
+    }
+    float acc[4];
+    item_part(buf, frag, B, warp, lane, acc);
+    trace_point(2, 4);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s_acc[warp][lane][i] = acc[i];
+    __syncthreads();  // every warp is done with buf: refill it
+    trace_point(2, 5);
+    if (tid == 0 && j + kK2Stages < n) {
+      const int jn = j + kK2Stages, itn = c0 + jn * step;
+      mbar_add_tx(&bar[st], kItemBytes);
+      issue_item(itn < kSharedItems ? shared_item(L, itn)
+                                    : routed_item(L, (int)slot_expert(s_word[jn]),
+                                                  8 * ((itn - kSharedItems) & 63)),
+                 buf, &bar[st]);
+      mbar_arrive(&bar[st]);
+    }
+    if (warp == 0) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        acc[i] = ((s_acc[0][lane][i] + s_acc[1][lane][i]) + s_acc[2][lane][i]) + s_acc[3][lane][i];
+      if (it < kSharedItems) {
+        uint16_t *hfs = reinterpret_cast<uint16_t *>(ws + lay.hfs);
+        const int r = 8 * it + g;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int b = 2 * t + c;
+          if (b < B)
+            write_hilo(hfs + (size_t)(2 * b) * kIs, hfs + (size_t)(2 * b + 1) * kIs, r,
+                       silu_f(acc[c]) * acc[2 + c]);
+        }
+      } else {
+        const int u = (it - kSharedItems) >> 6, r0 = 8 * ((it - kSharedItems) & 63);
+        const uint32_t mask = slot_mask(word);
+        uint16_t *hfr = reinterpret_cast<uint16_t *>(ws + lay.hfr);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int b = 2 * t + c;
+          if (b < B && ((mask >> b) & 1u)) {
+            int jj = 0;
+#pragma unroll
+            for (int q = 0; q < kTopK; ++q)
+              if (s_aslot[b * kTopK + q] == u) jj = q;
+            const float w = s_aw[b * kTopK + jj];
+            uint16_t *img = hfr + (size_t)((b * kTopK + jj) * 2) * kI;
+            write_hilo(img, img + kI, r0 + g, w * (silu_f(acc[c]) * acc[2 + c]));
+          }
+        }
+      }
+    }
+    __syncthreads();  // s_acc is read before the next item writes it
   }
   trace_point(2, 3);
 }
@@ -803,7 +849,25 @@ static int current_device() {
 // dynamic shared memory cap: the 227 KB opt-in limit minus K3's static arrays
 constexpr size_t kK3MaxSmem = 224 * 1024;
 constexpr int kK1Smem = 16 * kRouterRowStride + kXFragBytes;
-constexpr int kK2Smem = kItemBytes + kXFragBytes;  // item + compact fragment for B <= 8
+constexpr int kK2Smem = kK2Stages * kItemBytes + kXFragBytes;  // ring + fragment for B <= 8
+static size_t k2_smem(int B) { return (size_t)kK2Stages * kItemBytes + (size_t)4096 * B; }
+
+// K2 grid: as many CTAs as fit on the device at once (at most one per item),
+// but never so few that a CTA would own more than kK2MaxItems items.
+static int k2_grid(int dev, int B, int n_items) {
+  static int cache[64][kMaxB + 1];  // 0 = not computed
+  int per_sm = dev < 64 ? cache[dev][B] : 0;
+  if (per_sm == 0) {
+    int sms = 0, occ = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k2_gateup, kK2Warps * 32, k2_smem(B));
+    per_sm = sms * (occ > 0 ? occ : 1);
+    if (dev < 64) cache[dev][B] = per_sm;
+  }
+  int grid = per_sm < n_items ? per_sm : n_items;
+  const int floor_grid = (n_items + kK2MaxItems - 1) / kK2MaxItems;
+  return grid > floor_grid ? grid : floor_grid;
+}
 
 template <bool kResidual>
 static cudaError_t set_attrs(int dev) {
@@ -842,8 +906,8 @@ static cudaError_t launch_decode_t(const LayerArgs &L, const uint16_t *x, float 
   const int umax = kTopK * B < kE ? kTopK * B : kE;
   const int n_items = kSharedItems + 64 * umax;
   note_step("k2_gateup launch");
-  err = launch_pdl(k2_gateup, n_items, kK2Warps * 32,
-                   (size_t)kItemBytes + (size_t)16 * 4 * B * 64, st, L, B, ws, lay);
+  err = launch_pdl(k2_gateup, k2_grid(current_device(), B, n_items), kK2Warps * 32, k2_smem(B),
+                   st, L, B, n_items, ws, lay);
   if (err != cudaSuccess) return err;
   const K3Smem P{umax, B};
   note_step("k3_down_combine launch");
