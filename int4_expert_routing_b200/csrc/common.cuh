@@ -237,4 +237,21 @@ FLINT_DEV bool mbar_wait(uint64_t *bar, uint32_t parity) {
   return false;
 }
 
+// The same wait for threads off the critical issue path: each poll may
+// suspend the thread (up to the hint, in ns) until the phase completes, so
+// waiting warps leave the issue slots to the warps that have work.
+constexpr uint32_t kSleepPolls = 1u << 22;
+FLINT_DEV bool mbar_wait_sleep(uint64_t *bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kSleepPolls; ++i) {
+    uint32_t done;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(20000u)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+
 }  // namespace flint

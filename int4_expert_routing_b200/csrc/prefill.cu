@@ -296,15 +296,32 @@ __global__ void __launch_bounds__(256)
 constexpr int kABytes = 128 * 128;      // 128 weight rows x 64 bf16
 constexpr int kBBytes = kPfTile * 128;  // 128 token rows x 64 bf16
 constexpr int kRawBytes = 128 * 32;     // 128 weight rows x 64 int4
-constexpr int kGemmThreads = 320;       // producer, MMA, 4 dequant warps, 4 epilogue warps
+// Four warpgroups: 0 = producer, MMA issuer and two idle warps; 1 = four
+// dequant warps (one weight row per thread); 2-3 = eight epilogue warps (two
+// per TMEM lane quarter, one per 64-token half of the tile).  The block is
+// launched at 128 registers per thread (65,536); setmaxnreg then moves them:
+// 128 x 40 + 128 x 64 + 256 x 200 = 64,512.
+constexpr int kGemmThreads = 512;
+constexpr int kDeqThreads = 128;
+constexpr int kEpiThreads = 256;
+constexpr int kRegCtl = 40, kRegDeq = 64, kRegEpi = 200;
+static_assert(128 * kRegCtl + 128 * kRegDeq + 256 * kRegEpi <= 65536, "register split");
 constexpr int kTmemCols = 256;          // two 128-column fp32 accumulators
 
 template <int kMode>
 struct GemmCfg {
-  static constexpr int kNB = kMode == 1 ? 1 : 2;  // token operands per stage (hi, lo)
-  static constexpr int kStageBytes = kABytes + kNB * kBBytes + kRawBytes;
-  static constexpr int kStages = kMode == 1 ? 5 : 4;
+  static constexpr int kNB = kMode == 1 ? 1 : 2;      // token operands per stage (hi, lo)
+  static constexpr int kAtoms = kMode == 1 ? 2 : 1;   // 64-wide k atoms per stage
+  static constexpr int kSPG = 2 / kAtoms;             // stages per 128-wide k-group
+  // stage: A atoms | token atoms (operand-major) | int4 codes of the atoms
+  static constexpr int kStageBytes = kAtoms * (kABytes + kNB * kBBytes + kRawBytes);
+  static constexpr int kStages = kMode == 1 ? 3 : 4;
   static constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024;
+  static constexpr uint32_t a_off(int atom) { return (uint32_t)(atom * kABytes); }
+  static constexpr uint32_t b_off(int nb, int atom) {
+    return (uint32_t)(kAtoms * kABytes + (nb * kAtoms + atom) * kBBytes);
+  }
+  static constexpr uint32_t raw_off() { return (uint32_t)(kAtoms * (kABytes + kNB * kBBytes)); }
 };
 
 struct GemmArgs {
@@ -352,7 +369,30 @@ FLINT_DEV void umma_commit(uint64_t *bar) {
       : "memory");
 }
 
-FLINT_DEV void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+// Optional GEMM timeline (build with -DFLINT_TRACE): for the first kPfTrTiles
+// CTAs of each GEMM, %globaltimer per k-stage for the producer (TMA issued),
+// the dequant warps (tile written), the MMA warp (MMAs issued), and per
+// k-group for the epilogue (group read out); read with flint_pf_trace_dump.
+#ifdef FLINT_TRACE
+constexpr int kPfTrTiles = 8;
+static __device__ unsigned long long g_pf_tr[2][kPfTrTiles][8][64];
+FLINT_DEV void pf_mark(int mode, int role, int idx) {
+  if (blockIdx.x < kPfTrTiles && idx < 64) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    g_pf_tr[mode - 1][blockIdx.x][role][idx] = t;
+  }
+}
+extern "C" FLINT_API int flint_pf_trace_dump(unsigned long long *out) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  return cudaMemcpyFromSymbol(out, g_pf_tr, sizeof(g_pf_tr)) == cudaSuccess ? 0 : -1;
+}
+#else
+FLINT_DEV void pf_mark(int, int, int) {}
+#endif
+
+// 32 consecutive TMEM columns of this warp's 32 lanes; completes at tmem_wait_ld().
+FLINT_DEV void tmem_ld32_async(uint32_t taddr, uint32_t (&v)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%"
       "15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
@@ -362,8 +402,8 @@ FLINT_DEV void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
         "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
         "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
       : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+FLINT_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 FLINT_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 FLINT_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -414,8 +454,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int n_valid = min(kPfTile, (sh ? args.T : __ldcg(args.ecount + e)) - n0);
   if (n_valid <= 0) return;  // not produced by the scan; guards against an N = 0 MMA
   const int b_row = sh ? n0 : __ldcg(args.ebase + e) + n0;
-  const int ks = kMode == 1 ? kH / 64 : (sh ? kIs / 64 : kI / 64);  // k stages
-  const int ng = ks / 2;                                              // 128-wide k-groups
+  const int ks = (kMode == 1 ? kH : (sh ? kIs : kI)) / (64 * Cfg::kAtoms);  // k stages
+  const int ng = ks / Cfg::kSPG;                                            // 128-wide k-groups
   const int n_mma = (n_valid + 15) & ~15;
   int row0, row1;  // weight rows: GEMM 1 gate (tile rows 2i) / up (2i+1); GEMM 2 row0 + i
   if (kMode == 1) {
@@ -432,12 +472,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&afull[s], 128);
+      mbar_init(&afull[s], kDeqThreads);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&gfull[b], 1);
-      mbar_init(&gempty[b], 128);
+      mbar_init(&gempty[b], kEpiThreads);
     }
     s_fail = 0;
   }
@@ -451,123 +491,153 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
+  if (tid == 0) pf_mark(kMode, 4, 0);
 
-  if (warp == 0) {
-    // ---- producer: int4 codes of the weight tile and the token tile(s), by TMA
-    if (lane == 0) {
-      for (int kb = 0; kb < ks; ++kb) {
-        const int s = kb % S;
-        if (kb >= S && !mbar_wait(&empty[s], ((kb / S) - 1) & 1)) {
-          s_fail = 1;
-          break;
-        }
-        unsigned char *st = sm + (size_t)s * Cfg::kStageBytes;
-        unsigned char *raw = st + kABytes + Cfg::kNB * kBBytes;
-        mbar_expect_tx(&full[s], kRawBytes + Cfg::kNB * kBBytes);
-        if (kMode == 1) {
-          tma_load_2d(raw, tA, kb * 32, row0, &full[s]);
-          tma_load_2d(raw + 64 * 32, tA, kb * 32, row1, &full[s]);
-        } else {
-          tma_load_2d(raw, tA, kb * 32, row0, &full[s]);
-          tma_load_2d(st + kABytes + kBBytes, tBl, kb * 64, b_row, &full[s]);
-        }
-        tma_load_2d(st + kABytes, tB, kb * 64, b_row, &full[s]);
-      }
-    }
-  } else if (warp == 1) {
-    // ---- MMA issuer: group G accumulates into TMEM buffer G & 1
-    if (lane == 0) {
-      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n_mma >> 3) << 17) |
-                             ((uint32_t)(128 >> 4) << 24);
-      for (int G = 0; G < ng && !s_fail; ++G) {
-        const int b = G & 1;
-        if (G >= 2 && !mbar_wait(&gempty[b], ((G >> 1) - 1) & 1)) {
-          s_fail = 1;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d = tmem + (uint32_t)(128 * b);
-        for (int h = 0; h < 2; ++h) {
-          const int kb = 2 * G + h, s = kb % S;
-          const uint32_t ph = (kb / S) & 1;
-          if (!mbar_wait(&full[s], ph) || !mbar_wait(&afull[s], ph)) {
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegCtl));
+    if (warp == 0) {
+      // ---- producer: int4 codes of the weight tile and the token tile(s), by TMA
+      if (lane == 0) {
+        for (int kb = 0; kb < ks; ++kb) {
+          const int s = kb % S;
+          if (kb >= S && !mbar_wait_sleep(&empty[s], ((kb / S) - 1) & 1)) {
             s_fail = 1;
             break;
           }
-          tc_fence_after();
-          const uint32_t a_addr = smem_addr(sm + (size_t)s * Cfg::kStageBytes);
-          const uint32_t b_addr = a_addr + kABytes;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            umma_bf16(d, sw128_desc(a_addr + 32 * k), sw128_desc(b_addr + 32 * k), idesc,
-                      (h | k) != 0);
-            if (kMode == 2)
-              umma_bf16(d, sw128_desc(a_addr + 32 * k), sw128_desc(b_addr + kBBytes + 32 * k),
-                        idesc, 1u);
+          unsigned char *st = sm + (size_t)s * Cfg::kStageBytes;
+          unsigned char *raw = st + Cfg::raw_off();
+          mbar_expect_tx(&full[s], Cfg::kAtoms * (kRawBytes + Cfg::kNB * kBBytes));
+          if (kMode == 1) {  // gate rows then up rows, 128 codes (64 B) each
+            tma_load_2d(raw, tA, kb * 64, row0, &full[s]);
+            tma_load_2d(raw + 64 * 64, tA, kb * 64, row1, &full[s]);
+            tma_load_2d(st + Cfg::b_off(0, 0), tB, kb * 128, b_row, &full[s]);
+            tma_load_2d(st + Cfg::b_off(0, 1), tB, kb * 128 + 64, b_row, &full[s]);
+          } else {
+            tma_load_2d(raw, tA, kb * 32, row0, &full[s]);
+            tma_load_2d(st + Cfg::b_off(0, 0), tB, kb * 64, b_row, &full[s]);
+            tma_load_2d(st + Cfg::b_off(1, 0), tBl, kb * 64, b_row, &full[s]);
           }
-          umma_commit(&empty[s]);
+          pf_mark(kMode, 0, kb);
         }
-        umma_commit(&gfull[b]);
       }
-    }
-  } else if (warp < 6) {
+    } else if (warp == 1) {
+      // ---- MMA issuer: group G accumulates into TMEM buffer G & 1
+      if (lane == 0) {
+        const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n_mma >> 3) << 17) |
+                               ((uint32_t)(128 >> 4) << 24);
+        for (int G = 0; G < ng && !s_fail; ++G) {
+          const int b = G & 1;
+          if (G >= 2 && !mbar_wait(&gempty[b], ((G >> 1) - 1) & 1)) {
+            s_fail = 1;
+            break;
+          }
+          pf_mark(kMode, 5, G);
+          tc_fence_after();
+          const uint32_t d = tmem + (uint32_t)(128 * b);
+          for (int h = 0; h < Cfg::kSPG; ++h) {
+            const int kb = Cfg::kSPG * G + h, s = kb % S;
+            const uint32_t ph = (kb / S) & 1;
+            if (!mbar_wait(&full[s], ph)) {
+              s_fail = 1;
+              break;
+            }
+            pf_mark(kMode, 6, kb);
+            if (!mbar_wait(&afull[s], ph)) {
+              s_fail = 1;
+              break;
+            }
+            pf_mark(kMode, 7, kb);
+            tc_fence_after();
+            const uint32_t st_addr = smem_addr(sm + (size_t)s * Cfg::kStageBytes);
+  #pragma unroll
+            for (int atom = 0; atom < Cfg::kAtoms; ++atom) {
+              const uint32_t a_addr = st_addr + Cfg::a_off(atom);
+              const uint32_t b_addr = st_addr + Cfg::b_off(0, atom);
+  #pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                umma_bf16(d, sw128_desc(a_addr + 32 * k), sw128_desc(b_addr + 32 * k), idesc,
+                          (h | atom | k) != 0);
+                if (kMode == 2)
+                  umma_bf16(d, sw128_desc(a_addr + 32 * k),
+                            sw128_desc(st_addr + Cfg::b_off(1, atom) + 32 * k), idesc, 1u);
+              }
+            }
+            umma_commit(&empty[s]);
+            pf_mark(kMode, 2, kb);
+          }
+          umma_commit(&gfull[b]);
+        }
+      }
+    }  // warps 2-3: idle (register donors)
+  } else if (warp < 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegDeq));
     // ---- dequant: thread i owns weight row i of the tile (exact codes)
-    const int i = tid - 64;
+    const int i = tid - 128;
     const int raw_row = kMode == 1 ? ((i & 1) ? 64 + (i >> 1) : (i >> 1)) : i;
     for (int kb = 0; kb < ks; ++kb) {
       const int s = kb % S;
-      if (!mbar_wait(&full[s], (kb / S) & 1)) {
+      if (!mbar_wait_sleep(&full[s], (kb / S) & 1)) {
         s_fail = 1;
         break;
       }
       unsigned char *st = sm + (size_t)s * Cfg::kStageBytes;
-      const unsigned char *raw = st + kABytes + Cfg::kNB * kBBytes + raw_row * 32;
-      const uint4 w0 = *reinterpret_cast<const uint4 *>(raw);
-      const uint4 w1 = *reinterpret_cast<const uint4 *>(raw + 16);
-      uint4 c[4];
-      unsigned char *arow = st + i * 128;
-      codes32(w0, c);
+      // the row's codes: 32 B per atom; chunk j (32 codes) -> atom j / 2, 16-byte
+      // slots 4 (j % 2) .. +3 of the row, XOR-swizzled by the row (SW128)
+      const unsigned char *raw = st + Cfg::raw_off() + raw_row * (32 * Cfg::kAtoms);
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<uint4 *>(arow + ((q ^ (i & 7)) * 16)) = c[q];
-      codes32(w1, c);
+      for (int j = 0; j < 2 * Cfg::kAtoms; ++j) {
+        const uint4 w = *reinterpret_cast<const uint4 *>(raw + 16 * j);
+        uint4 c[4];
+        codes32(w, c);
+        unsigned char *arow = st + Cfg::a_off(j >> 1) + i * 128;
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<uint4 *>(arow + (((4 + q) ^ (i & 7)) * 16)) = c[q];
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<uint4 *>(arow + ((((j & 1) * 4 + q) ^ (i & 7)) * 16)) = c[q];
+      }
       fence_proxy_async();
       mbar_arrive(&afull[s]);
+      if (tid == 128) pf_mark(kMode, 1, kb);
     }
   } else {
-    // ---- epilogue warps 6..9: TMEM lane quarter (warp % 4) -> tile rows
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegEpi));
+    // ---- epilogue warps 8..15: TMEM lane quarter (warp % 4) -> tile rows;
+    // token half (warp - 8) / 4 -> tile columns 64 h .. 64 h + 63
     const int q4 = warp & 3;
+    const int c_lo = 64 * ((warp - 8) >> 2);
     const int r = 32 * q4 + lane;
     const int wrow = kMode == 1 ? ((r & 1) ? row1 : row0) + (r >> 1) : row0 + r;
     const int gpr = kMode == 1 ? kH / kG : (sh ? kIs / kG : kI / kG);
     const uint16_t *srow = (sh ? args.sc_s : args.sc_r) + (size_t)wrow * gpr;
-    float acc[kPfTile];
+    float acc[64];
 #pragma unroll
-    for (int j = 0; j < kPfTile; ++j) acc[j] = 0.f;
+    for (int j = 0; j < 64; ++j) acc[j] = 0.f;
     bool ok = true;
     for (int G = 0; G < ng; ++G) {
       const int b = G & 1;
       const float sc = bf16_bits_to_f32(ld_nc_u16(srow + G));
-      if (!mbar_wait(&gfull[b], (G >> 1) & 1)) {
+      if (!mbar_wait_sleep(&gfull[b], (G >> 1) & 1)) {
         ok = false;
         break;
       }
+      if (tid == 256) pf_mark(kMode, 4, 2 + G);
       tc_fence_after();
-      const uint32_t base = tmem + (uint32_t)(128 * b) + ((uint32_t)(32 * q4) << 16);
+      const uint32_t base = tmem + (uint32_t)(128 * b + c_lo) + ((uint32_t)(32 * q4) << 16);
+      if (c_lo < n_mma) {  // the same for the whole warp
+        uint32_t v0[32], v1[32];
+        tmem_ld32_async(base, v0);
+        if (c_lo + 32 < n_mma) tmem_ld32_async(base + 32u, v1);
+        tmem_wait_ld();
 #pragma unroll
-      for (int c0 = 0; c0 < kPfTile; c0 += 32) {
-        if (c0 < n_mma) {
-          uint32_t v[32];
-          tmem_ld32(base + (uint32_t)c0, v);
+        for (int j = 0; j < 32; ++j) acc[j] = fmaf(__uint_as_float(v0[j]), sc, acc[j]);
+        if (c_lo + 32 < n_mma) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) acc[c0 + j] = fmaf(__uint_as_float(v[j]), sc, acc[c0 + j]);
+          for (int j = 0; j < 32; ++j) acc[32 + j] = fmaf(__uint_as_float(v1[j]), sc, acc[32 + j]);
         }
       }
       tc_fence_before();
       mbar_arrive(&gempty[b]);
+      if (tid == 256) pf_mark(kMode, 3, G);
+      if (tid == 480) pf_mark(kMode, 3, 20 + G);
     }
     if (!ok) {
       s_fail = 1;
@@ -578,10 +648,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint16_t *lo = sh ? args.out_s_lo + (size_t)n0 * kIs + col
                         : args.out_r_lo + (size_t)b_row * kI + col;
 #pragma unroll
-      for (int j = 0; j < kPfTile; ++j) {
-        const float other = __shfl_xor_sync(0xffffffffu, acc[j], 1);
+      for (int jj = 0; jj < 64; ++jj) {
+        const int j = c_lo + jj;
+        const float other = __shfl_xor_sync(0xffffffffu, acc[jj], 1);
         if (!(r & 1) && j < n_valid) {
-          const float hv = acc[j] / (1.f + expf(-acc[j])) * other;  // silu(gate) * up
+          const float hv = acc[jj] / (1.f + expf(-acc[jj])) * other;  // silu(gate) * up
           uint16_t h16, l16;
           split_hilo(hv, h16, l16);
           hi[(size_t)j * ld] = h16;
@@ -591,13 +662,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else {
       const int col = 128 * mt + r;
 #pragma unroll
-      for (int j = 0; j < kPfTile; ++j) {
+      for (int jj = 0; jj < 64; ++jj) {
+        const int j = c_lo + jj;
         if (j < n_valid) {
           if (sh) {
-            args.out_s[(size_t)(n0 + j) * kH + col] = f32_to_bf16_bits(acc[j]);
+            args.out_s[(size_t)(n0 + j) * kH + col] = f32_to_bf16_bits(acc[jj]);
           } else {
             args.out_r[(size_t)(b_row + j) * kH + col] =
-                f32_to_bf16_bits(acc[j] * args.pw[b_row + j]);
+                f32_to_bf16_bits(acc[jj] * args.pw[b_row + j]);
           }
         }
       }
@@ -605,6 +677,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if (tid == 0) pf_mark(kMode, 4, 1);
   if (s_fail && tid == 0) set_status(args.status, kStatusTimeout);
   if (warp == 1) {
     tc_fence_after();
@@ -737,8 +810,8 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
   note_step("prefill tensor maps");
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
   const auto SW = CU_TENSOR_MAP_SWIZZLE_128B, NS = CU_TENSOR_MAP_SWIZZLE_NONE;
-  if ((e = make_map(&mA1r, L.w13_q, U8, kH / 2, (uint64_t)kE * 2 * kI, kH / 2, 32, 64, NS)) ||
-      (e = make_map(&mA1s, L.sh13_q, U8, kH / 2, 2 * kIs, kH / 2, 32, 64, NS)) ||
+  if ((e = make_map(&mA1r, L.w13_q, U8, kH / 2, (uint64_t)kE * 2 * kI, kH / 2, 64, 64, NS)) ||
+      (e = make_map(&mA1s, L.sh13_q, U8, kH / 2, 2 * kIs, kH / 2, 64, 64, NS)) ||
       (e = make_map(&mB1r, xp, BF, kH, (uint64_t)P.mr_max, kH * 2, 64, kPfTile, SW)) ||
       (e = make_map(&mB1s, x, BF, kH, (uint64_t)T, kH * 2, 64, kPfTile, SW)) ||
       (e = make_map(&mA2r, L.w2_q, U8, kI / 2, (uint64_t)kE * kH, kI / 2, 32, 128, NS)) ||
