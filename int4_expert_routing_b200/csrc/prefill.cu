@@ -429,6 +429,41 @@ FLINT_DEV void split_hilo(float v, uint16_t &hi, uint16_t &lo) {
 
 // kMode 1: gate/up + SwiGLU -> H hi/lo (routed [rows][512], shared [T][1024]).
 // kMode 2: down -> Yw (routed, weighted, [rows][2048]) / Ys (shared, [T][2048]).
+// One tile of a grouped GEMM, as every role of the CTA derives it.
+template <int kMode>
+struct PfTile {
+  int e, mt, n0, n_valid, n_mma, b_row, row0, row1, ks, ng;
+  bool sh;
+};
+template <int kMode>
+FLINT_DEV bool pf_tile(const GemmArgs &args, uint32_t idx, PfTile<kMode> &t) {
+  using Cfg = GemmCfg<kMode>;
+  const uint32_t packed = __ldcg(args.tiles + idx);
+  t.e = (int)(packed & 511u);
+  t.mt = (int)((packed >> 9) & 31u);
+  const int nt = (int)(packed >> 14);
+  t.sh = t.e == kE;
+  t.n0 = nt * kPfTile;
+  t.n_valid = min(kPfTile, (t.sh ? args.T : __ldcg(args.ecount + t.e)) - t.n0);
+  if (t.n_valid <= 0) return false;  // not produced by the scan; guards against an N = 0 MMA
+  t.n_mma = (t.n_valid + 15) & ~15;
+  t.b_row = t.sh ? t.n0 : __ldcg(args.ebase + t.e) + t.n0;
+  t.ks = (kMode == 1 ? kH : (t.sh ? kIs : kI)) / (64 * Cfg::kAtoms);  // k stages
+  t.ng = t.ks / Cfg::kSPG;                                            // 128-wide k-groups
+  if (kMode == 1) {  // weight rows: gate (tile rows 2i) / up (2i+1)
+    t.row0 = t.sh ? 64 * t.mt : t.e * 2 * kI + 64 * t.mt;
+    t.row1 = t.sh ? kIs + 64 * t.mt : t.e * 2 * kI + kI + 64 * t.mt;
+  } else {  // tile row i is weight row row0 + i
+    t.row0 = t.sh ? 128 * t.mt : t.e * kH + 128 * t.mt;
+    t.row1 = t.row0;
+  }
+  return true;
+}
+
+// Persistent: CTA c takes tiles c, c + grid, ...  Every role walks the same
+// tile sequence; the stage ring and the two TMEM accumulator buffers carry
+// on across tiles (running counters it, gc), so one tile's epilogue and the
+// next tile's loads and MMAs overlap.
 template <int kMode>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     k_pf_gemm(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
@@ -442,32 +477,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   __shared__ __align__(8) uint64_t full[S], afull[S], empty[S], gfull[2], gempty[2];
   __shared__ uint32_t s_tmem;
-  __shared__ int s_fail;
+  __shared__ volatile int s_fail;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t ntiles = __ldcg(args.ctrl + args.count_word);
   if (blockIdx.x >= ntiles) return;
-  const uint32_t packed = __ldcg(args.tiles + blockIdx.x);
-  const int e = (int)(packed & 511u), mt = (int)((packed >> 9) & 31u), nt = (int)(packed >> 14);
-  const bool sh = e == kE;
-  const int n0 = nt * kPfTile;
-  const int n_valid = min(kPfTile, (sh ? args.T : __ldcg(args.ecount + e)) - n0);
-  if (n_valid <= 0) return;  // not produced by the scan; guards against an N = 0 MMA
-  const int b_row = sh ? n0 : __ldcg(args.ebase + e) + n0;
-  const int ks = (kMode == 1 ? kH : (sh ? kIs : kI)) / (64 * Cfg::kAtoms);  // k stages
-  const int ng = ks / Cfg::kSPG;                                            // 128-wide k-groups
-  const int n_mma = (n_valid + 15) & ~15;
-  int row0, row1;  // weight rows: GEMM 1 gate (tile rows 2i) / up (2i+1); GEMM 2 row0 + i
-  if (kMode == 1) {
-    row0 = sh ? 64 * mt : e * 2 * kI + 64 * mt;
-    row1 = sh ? kIs + 64 * mt : e * 2 * kI + kI + 64 * mt;
-  } else {
-    row0 = sh ? 128 * mt : e * kH + 128 * mt;
-    row1 = row0;
-  }
-  const CUtensorMap *tA = sh ? &tmA_s : &tmA_r;
-  const CUtensorMap *tB = sh ? &tmB_s : &tmB_r;
-  const CUtensorMap *tBl = sh ? &tmB_s_lo : &tmB_r_lo;
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
@@ -495,12 +509,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegCtl));
-    if (warp == 0) {
+    if (warp == 0 && lane == 0) {
       // ---- producer: int4 codes of the weight tile and the token tile(s), by TMA
-      if (lane == 0) {
-        for (int kb = 0; kb < ks; ++kb) {
-          const int s = kb % S;
-          if (kb >= S && !mbar_wait_sleep(&empty[s], ((kb / S) - 1) & 1)) {
+      uint32_t it = 0;
+      for (uint32_t ti = blockIdx.x; ti < ntiles && !s_fail; ti += gridDim.x) {
+        PfTile<kMode> t;
+        if (!pf_tile<kMode>(args, ti, t)) continue;
+        const CUtensorMap *tA = t.sh ? &tmA_s : &tmA_r;
+        const CUtensorMap *tB = t.sh ? &tmB_s : &tmB_r;
+        const CUtensorMap *tBl = t.sh ? &tmB_s_lo : &tmB_r_lo;
+        for (int kb = 0; kb < t.ks; ++kb, ++it) {
+          const int s = it % S;
+          if (it >= (uint32_t)S && !mbar_wait_sleep(&empty[s], ((it / S) - 1) & 1)) {
             s_fail = 1;
             break;
           }
@@ -508,52 +528,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           unsigned char *raw = st + Cfg::raw_off();
           mbar_expect_tx(&full[s], Cfg::kAtoms * (kRawBytes + Cfg::kNB * kBBytes));
           if (kMode == 1) {  // gate rows then up rows, 128 codes (64 B) each
-            tma_load_2d(raw, tA, kb * 64, row0, &full[s]);
-            tma_load_2d(raw + 64 * 64, tA, kb * 64, row1, &full[s]);
-            tma_load_2d(st + Cfg::b_off(0, 0), tB, kb * 128, b_row, &full[s]);
-            tma_load_2d(st + Cfg::b_off(0, 1), tB, kb * 128 + 64, b_row, &full[s]);
+            tma_load_2d(raw, tA, kb * 64, t.row0, &full[s]);
+            tma_load_2d(raw + 64 * 64, tA, kb * 64, t.row1, &full[s]);
+            tma_load_2d(st + Cfg::b_off(0, 0), tB, kb * 128, t.b_row, &full[s]);
+            tma_load_2d(st + Cfg::b_off(0, 1), tB, kb * 128 + 64, t.b_row, &full[s]);
           } else {
-            tma_load_2d(raw, tA, kb * 32, row0, &full[s]);
-            tma_load_2d(st + Cfg::b_off(0, 0), tB, kb * 64, b_row, &full[s]);
-            tma_load_2d(st + Cfg::b_off(1, 0), tBl, kb * 64, b_row, &full[s]);
+            tma_load_2d(raw, tA, kb * 32, t.row0, &full[s]);
+            tma_load_2d(st + Cfg::b_off(0, 0), tB, kb * 64, t.b_row, &full[s]);
+            tma_load_2d(st + Cfg::b_off(1, 0), tBl, kb * 64, t.b_row, &full[s]);
           }
-          pf_mark(kMode, 0, kb);
+          if (ti == blockIdx.x) pf_mark(kMode, 0, kb);
         }
       }
-    } else if (warp == 1) {
-      // ---- MMA issuer: group G accumulates into TMEM buffer G & 1
-      if (lane == 0) {
-        const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n_mma >> 3) << 17) |
-                               ((uint32_t)(128 >> 4) << 24);
-        for (int G = 0; G < ng && !s_fail; ++G) {
-          const int b = G & 1;
-          if (G >= 2 && !mbar_wait(&gempty[b], ((G >> 1) - 1) & 1)) {
+    } else if (warp == 1 && lane == 0) {
+      // ---- MMA issuer: group gc accumulates into TMEM buffer gc & 1
+      uint32_t it = 0, gc = 0;
+      for (uint32_t ti = blockIdx.x; ti < ntiles && !s_fail; ti += gridDim.x) {
+        PfTile<kMode> t;
+        if (!pf_tile<kMode>(args, ti, t)) continue;
+        const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                               ((uint32_t)(t.n_mma >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+        for (int G = 0; G < t.ng && !s_fail; ++G, ++gc) {
+          const int b = gc & 1;
+          if (gc >= 2 && !mbar_wait(&gempty[b], ((gc >> 1) - 1) & 1)) {
             s_fail = 1;
             break;
           }
-          pf_mark(kMode, 5, G);
+          if (ti == blockIdx.x) pf_mark(kMode, 5, G);
           tc_fence_after();
           const uint32_t d = tmem + (uint32_t)(128 * b);
-          for (int h = 0; h < Cfg::kSPG; ++h) {
-            const int kb = Cfg::kSPG * G + h, s = kb % S;
-            const uint32_t ph = (kb / S) & 1;
-            if (!mbar_wait(&full[s], ph)) {
+          for (int h = 0; h < Cfg::kSPG; ++h, ++it) {
+            const int s = it % S;
+            const uint32_t ph = (it / S) & 1;
+            if (!mbar_wait(&full[s], ph) || !mbar_wait(&afull[s], ph)) {
               s_fail = 1;
               break;
             }
-            pf_mark(kMode, 6, kb);
-            if (!mbar_wait(&afull[s], ph)) {
-              s_fail = 1;
-              break;
-            }
-            pf_mark(kMode, 7, kb);
             tc_fence_after();
             const uint32_t st_addr = smem_addr(sm + (size_t)s * Cfg::kStageBytes);
-  #pragma unroll
+#pragma unroll
             for (int atom = 0; atom < Cfg::kAtoms; ++atom) {
               const uint32_t a_addr = st_addr + Cfg::a_off(atom);
               const uint32_t b_addr = st_addr + Cfg::b_off(0, atom);
-  #pragma unroll
+#pragma unroll
               for (int k = 0; k < 4; ++k) {
                 umma_bf16(d, sw128_desc(a_addr + 32 * k), sw128_desc(b_addr + 32 * k), idesc,
                           (h | atom | k) != 0);
@@ -563,40 +580,45 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               }
             }
             umma_commit(&empty[s]);
-            pf_mark(kMode, 2, kb);
+            if (ti == blockIdx.x) pf_mark(kMode, 2, Cfg::kSPG * G + h);
           }
           umma_commit(&gfull[b]);
         }
       }
-    }  // warps 2-3: idle (register donors)
+    }  // other lanes and warps 2-3: idle (register donors)
   } else if (warp < 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegDeq));
-    // ---- dequant: thread i owns weight row i of the tile (exact codes)
+    // ---- dequant: thread i owns weight row i of every tile (exact codes)
     const int i = tid - 128;
     const int raw_row = kMode == 1 ? ((i & 1) ? 64 + (i >> 1) : (i >> 1)) : i;
-    for (int kb = 0; kb < ks; ++kb) {
-      const int s = kb % S;
-      if (!mbar_wait_sleep(&full[s], (kb / S) & 1)) {
-        s_fail = 1;
-        break;
-      }
-      unsigned char *st = sm + (size_t)s * Cfg::kStageBytes;
-      // the row's codes: 32 B per atom; chunk j (32 codes) -> atom j / 2, 16-byte
-      // slots 4 (j % 2) .. +3 of the row, XOR-swizzled by the row (SW128)
-      const unsigned char *raw = st + Cfg::raw_off() + raw_row * (32 * Cfg::kAtoms);
+    uint32_t it = 0;
+    for (uint32_t ti = blockIdx.x; ti < ntiles && !s_fail; ti += gridDim.x) {
+      PfTile<kMode> t;
+      if (!pf_tile<kMode>(args, ti, t)) continue;
+      for (int kb = 0; kb < t.ks; ++kb, ++it) {
+        const int s = it % S;
+        if (!mbar_wait_sleep(&full[s], (it / S) & 1)) {
+          s_fail = 1;
+          break;
+        }
+        unsigned char *st = sm + (size_t)s * Cfg::kStageBytes;
+        // the row's codes: 32 B per atom; chunk j (32 codes) -> atom j / 2, 16-byte
+        // slots 4 (j % 2) .. +3 of the row, XOR-swizzled by the row (SW128)
+        const unsigned char *raw = st + Cfg::raw_off() + raw_row * (32 * Cfg::kAtoms);
 #pragma unroll
-      for (int j = 0; j < 2 * Cfg::kAtoms; ++j) {
-        const uint4 w = *reinterpret_cast<const uint4 *>(raw + 16 * j);
-        uint4 c[4];
-        codes32(w, c);
-        unsigned char *arow = st + Cfg::a_off(j >> 1) + i * 128;
+        for (int j = 0; j < 2 * Cfg::kAtoms; ++j) {
+          const uint4 w = *reinterpret_cast<const uint4 *>(raw + 16 * j);
+          uint4 c[4];
+          codes32(w, c);
+          unsigned char *arow = st + Cfg::a_off(j >> 1) + i * 128;
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          *reinterpret_cast<uint4 *>(arow + ((((j & 1) * 4 + q) ^ (i & 7)) * 16)) = c[q];
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4 *>(arow + ((((j & 1) * 4 + q) ^ (i & 7)) * 16)) = c[q];
+        }
+        fence_proxy_async();
+        mbar_arrive(&afull[s]);
+        if (tid == 128 && ti == blockIdx.x) pf_mark(kMode, 1, kb);
       }
-      fence_proxy_async();
-      mbar_arrive(&afull[s]);
-      if (tid == 128) pf_mark(kMode, 1, kb);
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegEpi));
@@ -605,71 +627,80 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int q4 = warp & 3;
     const int c_lo = 64 * ((warp - 8) >> 2);
     const int r = 32 * q4 + lane;
-    const int wrow = kMode == 1 ? ((r & 1) ? row1 : row0) + (r >> 1) : row0 + r;
-    const int gpr = kMode == 1 ? kH / kG : (sh ? kIs / kG : kI / kG);
-    const uint16_t *srow = (sh ? args.sc_s : args.sc_r) + (size_t)wrow * gpr;
-    float acc[64];
+    uint32_t gc = 0;
+    for (uint32_t ti = blockIdx.x; ti < ntiles && !s_fail; ti += gridDim.x) {
+      PfTile<kMode> t;
+      if (!pf_tile<kMode>(args, ti, t)) continue;
+      const int wrow = kMode == 1 ? ((r & 1) ? t.row1 : t.row0) + (r >> 1) : t.row0 + r;
+      const int gpr = kMode == 1 ? kH / kG : (t.sh ? kIs / kG : kI / kG);
+      const uint16_t *srow = (t.sh ? args.sc_s : args.sc_r) + (size_t)wrow * gpr;
+      float acc[64];
 #pragma unroll
-    for (int j = 0; j < 64; ++j) acc[j] = 0.f;
-    bool ok = true;
-    for (int G = 0; G < ng; ++G) {
-      const int b = G & 1;
-      const float sc = bf16_bits_to_f32(ld_nc_u16(srow + G));
-      if (!mbar_wait_sleep(&gfull[b], (G >> 1) & 1)) {
-        ok = false;
+      for (int j = 0; j < 64; ++j) acc[j] = 0.f;
+      bool ok = true;
+      for (int G = 0; G < t.ng; ++G, ++gc) {
+        const int b = gc & 1;
+        const float sc = bf16_bits_to_f32(ld_nc_u16(srow + G));
+        if (!mbar_wait_sleep(&gfull[b], (gc >> 1) & 1)) {
+          ok = false;
+          break;
+        }
+        if (tid == 256 && ti == blockIdx.x) pf_mark(kMode, 4, 2 + G);
+        tc_fence_after();
+        const uint32_t base = tmem + (uint32_t)(128 * b + c_lo) + ((uint32_t)(32 * q4) << 16);
+        if (c_lo < t.n_mma) {  // the same for the whole warp
+          uint32_t v0[32], v1[32];
+          tmem_ld32_async(base, v0);
+          if (c_lo + 32 < t.n_mma) tmem_ld32_async(base + 32u, v1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) acc[j] = fmaf(__uint_as_float(v0[j]), sc, acc[j]);
+          if (c_lo + 32 < t.n_mma) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              acc[32 + j] = fmaf(__uint_as_float(v1[j]), sc, acc[32 + j]);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&gempty[b]);
+        if (tid == 256 && ti == blockIdx.x) pf_mark(kMode, 3, G);
+        if (tid == 480 && ti == blockIdx.x) pf_mark(kMode, 3, 20 + G);
+      }
+      if (!ok) {
+        s_fail = 1;
         break;
       }
-      if (tid == 256) pf_mark(kMode, 4, 2 + G);
-      tc_fence_after();
-      const uint32_t base = tmem + (uint32_t)(128 * b + c_lo) + ((uint32_t)(32 * q4) << 16);
-      if (c_lo < n_mma) {  // the same for the whole warp
-        uint32_t v0[32], v1[32];
-        tmem_ld32_async(base, v0);
-        if (c_lo + 32 < n_mma) tmem_ld32_async(base + 32u, v1);
-        tmem_wait_ld();
+      if (kMode == 1) {
+        const int col = 64 * t.mt + (r >> 1);
+        const size_t ld = t.sh ? kIs : kI;
+        uint16_t *hi = t.sh ? args.out_s + (size_t)t.n0 * kIs + col
+                            : args.out_r + (size_t)t.b_row * kI + col;
+        uint16_t *lo = t.sh ? args.out_s_lo + (size_t)t.n0 * kIs + col
+                            : args.out_r_lo + (size_t)t.b_row * kI + col;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) acc[j] = fmaf(__uint_as_float(v0[j]), sc, acc[j]);
-        if (c_lo + 32 < n_mma) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) acc[32 + j] = fmaf(__uint_as_float(v1[j]), sc, acc[32 + j]);
+        for (int jj = 0; jj < 64; ++jj) {
+          const int j = c_lo + jj;
+          const float other = __shfl_xor_sync(0xffffffffu, acc[jj], 1);
+          if (!(r & 1) && j < t.n_valid) {
+            const float hv = acc[jj] / (1.f + expf(-acc[jj])) * other;  // silu(gate) * up
+            uint16_t h16, l16;
+            split_hilo(hv, h16, l16);
+            hi[(size_t)j * ld] = h16;
+            lo[(size_t)j * ld] = l16;
+          }
         }
-      }
-      tc_fence_before();
-      mbar_arrive(&gempty[b]);
-      if (tid == 256) pf_mark(kMode, 3, G);
-      if (tid == 480) pf_mark(kMode, 3, 20 + G);
-    }
-    if (!ok) {
-      s_fail = 1;
-    } else if (kMode == 1) {
-      const int col = 64 * mt + (r >> 1);
-      const size_t ld = sh ? kIs : kI;
-      uint16_t *hi = sh ? args.out_s + (size_t)n0 * kIs + col : args.out_r + (size_t)b_row * kI + col;
-      uint16_t *lo = sh ? args.out_s_lo + (size_t)n0 * kIs + col
-                        : args.out_r_lo + (size_t)b_row * kI + col;
+      } else {
+        const int col = 128 * t.mt + r;
 #pragma unroll
-      for (int jj = 0; jj < 64; ++jj) {
-        const int j = c_lo + jj;
-        const float other = __shfl_xor_sync(0xffffffffu, acc[jj], 1);
-        if (!(r & 1) && j < n_valid) {
-          const float hv = acc[jj] / (1.f + expf(-acc[jj])) * other;  // silu(gate) * up
-          uint16_t h16, l16;
-          split_hilo(hv, h16, l16);
-          hi[(size_t)j * ld] = h16;
-          lo[(size_t)j * ld] = l16;
-        }
-      }
-    } else {
-      const int col = 128 * mt + r;
-#pragma unroll
-      for (int jj = 0; jj < 64; ++jj) {
-        const int j = c_lo + jj;
-        if (j < n_valid) {
-          if (sh) {
-            args.out_s[(size_t)(n0 + j) * kH + col] = f32_to_bf16_bits(acc[jj]);
-          } else {
-            args.out_r[(size_t)(b_row + j) * kH + col] =
-                f32_to_bf16_bits(acc[jj] * args.pw[b_row + j]);
+        for (int jj = 0; jj < 64; ++jj) {
+          const int j = c_lo + jj;
+          if (j < t.n_valid) {
+            if (t.sh) {
+              args.out_s[(size_t)(t.n0 + j) * kH + col] = f32_to_bf16_bits(acc[jj]);
+            } else {
+              args.out_r[(size_t)(t.b_row + j) * kH + col] =
+                  f32_to_bf16_bits(acc[jj] * args.pw[t.b_row + j]);
+            }
           }
         }
       }
@@ -827,17 +858,22 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
       (e = cudaFuncSetAttribute(k_pf_gemm<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)GemmCfg<2>::kSmem)) != cudaSuccess)
     return e;
+  // persistent GEMMs: one CTA per SM at most (the tile counts are on the device)
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (sms < 1) sms = 1;
   GemmArgs a1{tiles1, ctrl, 3,  ebase, ecount, T,       L.w13_s, L.sh13_s,
               hr,     hr_lo, hs, hs_lo, nullptr, ctrl + 1};
   note_step("prefill GEMM 1 launch");
-  k_pf_gemm<1><<<P.max_tiles1, kGemmThreads, GemmCfg<1>::kSmem, st>>>(mA1r, mA1s, mB1r, mB1s,
-                                                                        mB1r, mB1s, a1);
+  k_pf_gemm<1><<<min(P.max_tiles1, sms), kGemmThreads, GemmCfg<1>::kSmem, st>>>(
+      mA1r, mA1s, mB1r, mB1s, mB1r, mB1s, a1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   GemmArgs a2{tiles2, ctrl, 4, ebase, ecount, T, L.w2_s, L.sh2_s, yw, nullptr, ys, nullptr, pw,
               ctrl + 1};
   note_step("prefill GEMM 2 launch");
-  k_pf_gemm<2><<<P.max_tiles2, kGemmThreads, GemmCfg<2>::kSmem, st>>>(mA2r, mA2s, mB2r, mB2s,
-                                                                        mB2rl, mB2sl, a2);
+  k_pf_gemm<2><<<min(P.max_tiles2, sms), kGemmThreads, GemmCfg<2>::kSmem, st>>>(
+      mA2r, mA2s, mB2r, mB2s, mB2rl, mB2sl, a2);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // 5. combine
   note_step("prefill combine launch");
