@@ -310,12 +310,11 @@ constexpr int kTmemCols = 256;          // two 128-column fp32 accumulators
 
 template <int kMode>
 struct GemmCfg {
-  static constexpr int kNB = kMode == 1 ? 1 : 2;      // token operands per stage (hi, lo)
-  static constexpr int kAtoms = kMode == 1 ? 2 : 1;   // 64-wide k atoms per stage
-  static constexpr int kSPG = 2 / kAtoms;             // stages per 128-wide k-group
+  static constexpr int kNB = kMode == 1 ? 1 : 2;  // token operands per stage (hi, lo)
+  static constexpr int kAtoms = 2;                // 64-wide k atoms per stage: one k-group
   // stage: A atoms | token atoms (operand-major) | int4 codes of the atoms
   static constexpr int kStageBytes = kAtoms * (kABytes + kNB * kBBytes + kRawBytes);
-  static constexpr int kStages = kMode == 1 ? 3 : 4;
+  static constexpr int kStages = kMode == 1 ? 3 : 2;
   static constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024;
   static constexpr uint32_t a_off(int atom) { return (uint32_t)(atom * kABytes); }
   static constexpr uint32_t b_off(int nb, int atom) {
@@ -448,8 +447,8 @@ FLINT_DEV bool pf_tile(const GemmArgs &args, uint32_t idx, PfTile<kMode> &t) {
   if (t.n_valid <= 0) return false;  // not produced by the scan; guards against an N = 0 MMA
   t.n_mma = (t.n_valid + 15) & ~15;
   t.b_row = t.sh ? t.n0 : __ldcg(args.ebase + t.e) + t.n0;
-  t.ks = (kMode == 1 ? kH : (t.sh ? kIs : kI)) / (64 * Cfg::kAtoms);  // k stages
-  t.ng = t.ks / Cfg::kSPG;                                            // 128-wide k-groups
+  t.ks = (kMode == 1 ? kH : (t.sh ? kIs : kI)) / (64 * Cfg::kAtoms);  // k stages = k-groups
+  t.ng = t.ks;
   if (kMode == 1) {  // weight rows: gate (tile rows 2i) / up (2i+1)
     t.row0 = t.sh ? 64 * t.mt : t.e * 2 * kI + 64 * t.mt;
     t.row1 = t.sh ? kIs + 64 * t.mt : t.e * 2 * kI + kI + 64 * t.mt;
@@ -475,7 +474,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t full[S], afull[S], empty[S], gfull[2], gempty[2];
+  __shared__ __align__(8) uint64_t full[S], afull[S], empty[S], gempty[2];
+  static_assert(S >= 2, "the epilogue's wait on empty[] needs two stages");
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_fail;
 
@@ -489,10 +489,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&afull[s], kDeqThreads);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&gfull[b], 1);
-      mbar_init(&gempty[b], kEpiThreads);
-    }
+    for (int b = 0; b < 2; ++b) mbar_init(&gempty[b], kEpiThreads);
     s_fail = 0;
   }
   if (warp == 1) {
@@ -532,10 +529,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tma_load_2d(raw + 64 * 64, tA, kb * 64, t.row1, &full[s]);
             tma_load_2d(st + Cfg::b_off(0, 0), tB, kb * 128, t.b_row, &full[s]);
             tma_load_2d(st + Cfg::b_off(0, 1), tB, kb * 128 + 64, t.b_row, &full[s]);
-          } else {
-            tma_load_2d(raw, tA, kb * 32, t.row0, &full[s]);
-            tma_load_2d(st + Cfg::b_off(0, 0), tB, kb * 64, t.b_row, &full[s]);
-            tma_load_2d(st + Cfg::b_off(1, 0), tBl, kb * 64, t.b_row, &full[s]);
+          } else {  // 128 rows x 128 codes; hi and lo token atoms
+            tma_load_2d(raw, tA, kb * 64, t.row0, &full[s]);
+            for (int atom = 0; atom < 2; ++atom) {
+              tma_load_2d(st + Cfg::b_off(0, atom), tB, kb * 128 + 64 * atom, t.b_row, &full[s]);
+              tma_load_2d(st + Cfg::b_off(1, atom), tBl, kb * 128 + 64 * atom, t.b_row, &full[s]);
+            }
           }
           if (ti == blockIdx.x) pf_mark(kMode, 0, kb);
         }
@@ -557,10 +556,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (ti == blockIdx.x) pf_mark(kMode, 5, G);
           tc_fence_after();
           const uint32_t d = tmem + (uint32_t)(128 * b);
-          for (int h = 0; h < Cfg::kSPG; ++h, ++it) {
+          {  // the group's single stage
             const int s = it % S;
             const uint32_t ph = (it / S) & 1;
-            if (!mbar_wait(&full[s], ph) || !mbar_wait(&afull[s], ph)) {
+            // afull implies full: the dequant warps arrive on afull only after
+            // they have waited on full (the stage's TMA bytes) themselves
+            if (!mbar_wait(&afull[s], ph)) {
               s_fail = 1;
               break;
             }
@@ -573,16 +574,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
                 umma_bf16(d, sw128_desc(a_addr + 32 * k), sw128_desc(b_addr + 32 * k), idesc,
-                          (h | atom | k) != 0);
+                          (atom | k) != 0);
                 if (kMode == 2)
                   umma_bf16(d, sw128_desc(a_addr + 32 * k),
                             sw128_desc(st_addr + Cfg::b_off(1, atom) + 32 * k), idesc, 1u);
               }
             }
+            // one commit: frees the stage for the producer and tells the
+            // epilogue that group gc is in TMEM buffer b
             umma_commit(&empty[s]);
-            if (ti == blockIdx.x) pf_mark(kMode, 2, Cfg::kSPG * G + h);
+            if (ti == blockIdx.x) pf_mark(kMode, 2, G);
+            ++it;
           }
-          umma_commit(&gfull[b]);
         }
       }
     }  // other lanes and warps 2-3: idle (register donors)
@@ -641,7 +644,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int G = 0; G < t.ng; ++G, ++gc) {
         const int b = gc & 1;
         const float sc = bf16_bits_to_f32(ld_nc_u16(srow + G));
-        if (!mbar_wait_sleep(&gfull[b], (gc >> 1) & 1)) {
+        // group gc's MMAs are done when its stage's empty phase completes; the
+        // MMA warp cannot start group gc + 2 (stage gc + S, S >= 2) before this
+        // thread releases buffer b, so that phase is never two ahead
+        if (!mbar_wait_sleep(&empty[gc % S], (gc / S) & 1)) {
           ok = false;
           break;
         }
@@ -845,8 +851,8 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
       (e = make_map(&mA1s, L.sh13_q, U8, kH / 2, 2 * kIs, kH / 2, 64, 64, NS)) ||
       (e = make_map(&mB1r, xp, BF, kH, (uint64_t)P.mr_max, kH * 2, 64, kPfTile, SW)) ||
       (e = make_map(&mB1s, x, BF, kH, (uint64_t)T, kH * 2, 64, kPfTile, SW)) ||
-      (e = make_map(&mA2r, L.w2_q, U8, kI / 2, (uint64_t)kE * kH, kI / 2, 32, 128, NS)) ||
-      (e = make_map(&mA2s, L.sh2_q, U8, kIs / 2, kH, kIs / 2, 32, 128, NS)) ||
+      (e = make_map(&mA2r, L.w2_q, U8, kI / 2, (uint64_t)kE * kH, kI / 2, 64, 128, NS)) ||
+      (e = make_map(&mA2s, L.sh2_q, U8, kIs / 2, kH, kIs / 2, 64, 128, NS)) ||
       (e = make_map(&mB2r, hr, BF, kI, (uint64_t)P.mr_max, kI * 2, 64, kPfTile, SW)) ||
       (e = make_map(&mB2rl, hr_lo, BF, kI, (uint64_t)P.mr_max, kI * 2, 64, kPfTile, SW)) ||
       (e = make_map(&mB2s, hs, BF, kIs, (uint64_t)T, kIs * 2, 64, kPfTile, SW)) ||
