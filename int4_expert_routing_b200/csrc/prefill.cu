@@ -306,7 +306,8 @@ constexpr int kDeqThreads = 128;
 constexpr int kEpiThreads = 256;
 constexpr int kRegCtl = 40, kRegDeq = 64, kRegEpi = 200;
 static_assert(128 * kRegCtl + 128 * kRegDeq + 256 * kRegEpi <= 65536, "register split");
-constexpr int kTmemCols = 256;          // two 128-column fp32 accumulators
+constexpr int kTmemCols = 512;          // four 128-column fp32 accumulators (one CTA per SM)
+constexpr int kTmemBufs = kTmemCols / 128;
 
 template <int kMode>
 struct GemmCfg {
@@ -474,8 +475,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t full[S], afull[S], empty[S], gempty[2];
-  static_assert(S >= 2, "the epilogue's wait on empty[] needs two stages");
+  __shared__ __align__(8) uint64_t full[S], afull[S], empty[S], gfull[kTmemBufs],
+      gempty[kTmemBufs];
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_fail;
 
@@ -489,7 +490,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&afull[s], kDeqThreads);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) mbar_init(&gempty[b], kEpiThreads);
+    for (int b = 0; b < kTmemBufs; ++b) {
+      mbar_init(&gfull[b], 1);
+      mbar_init(&gempty[b], kEpiThreads);
+    }
     s_fail = 0;
   }
   if (warp == 1) {
@@ -540,7 +544,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
     } else if (warp == 1 && lane == 0) {
-      // ---- MMA issuer: group gc accumulates into TMEM buffer gc & 1
+      // ---- MMA issuer: group gc accumulates into TMEM buffer gc % kTmemBufs
       uint32_t it = 0, gc = 0;
       for (uint32_t ti = blockIdx.x; ti < ntiles && !s_fail; ti += gridDim.x) {
         PfTile<kMode> t;
@@ -548,8 +552,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) |
                                ((uint32_t)(t.n_mma >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
         for (int G = 0; G < t.ng && !s_fail; ++G, ++gc) {
-          const int b = gc & 1;
-          if (gc >= 2 && !mbar_wait(&gempty[b], ((gc >> 1) - 1) & 1)) {
+          const int b = gc % kTmemBufs;
+          if (gc >= kTmemBufs && !mbar_wait(&gempty[b], ((gc / kTmemBufs) - 1) & 1)) {
             s_fail = 1;
             break;
           }
@@ -580,9 +584,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             sw128_desc(st_addr + Cfg::b_off(1, atom) + 32 * k), idesc, 1u);
               }
             }
-            // one commit: frees the stage for the producer and tells the
-            // epilogue that group gc is in TMEM buffer b
-            umma_commit(&empty[s]);
+            umma_commit(&empty[s]);    // the stage is free for the producer
+            umma_commit(&gfull[b]);    // group gc is complete in TMEM buffer b
             if (ti == blockIdx.x) pf_mark(kMode, 2, G);
             ++it;
           }
@@ -642,12 +645,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int j = 0; j < 64; ++j) acc[j] = 0.f;
       bool ok = true;
       for (int G = 0; G < t.ng; ++G, ++gc) {
-        const int b = gc & 1;
+        const int b = gc % kTmemBufs;
         const float sc = bf16_bits_to_f32(ld_nc_u16(srow + G));
-        // group gc's MMAs are done when its stage's empty phase completes; the
-        // MMA warp cannot start group gc + 2 (stage gc + S, S >= 2) before this
-        // thread releases buffer b, so that phase is never two ahead
-        if (!mbar_wait_sleep(&empty[gc % S], (gc / S) & 1)) {
+        if (!mbar_wait_sleep(&gfull[b], (gc / kTmemBufs) & 1)) {
           ok = false;
           break;
         }
