@@ -96,3 +96,35 @@ def test_prefill_deterministic_and_consistent_with_decode(layer0):
         torch().cuda.synchronize()
         dec.append(host_bf16(o))
     check_close(bf16_to_f64(a), bf16_to_f64(np.concatenate(dec)), what="prefill vs decode")
+
+
+def test_prefill_large_activations(layer0):
+    """x scaled by 512 (exact in bf16): routed SwiGLU intermediates reach ~1e5
+    (past the fp16 range); the bf16 hi/lo intermediate keeps the bound."""
+    x = synth.prefill_x(40, 4040)
+    xs = synth.bf16_bits(synth.bf16_to_f64(x) * 512.0)
+    out = prefill(layer0, xs)
+    ref, idx, w, gap = oracle.moe_layer(layer0["O"], xs)
+    ridx, _ = route(layer0, xs)
+    rows = routing_rows(ridx, idx, gap)
+    assert np.all(np.isfinite(bf16_to_f64(out)))
+    worst = check_close(bf16_to_f64(out), ref, rows, what="prefill x*512")
+    print(f"prefill x*512: max |ref| {np.abs(ref).max():.3e}, worst |err|/bound {worst:.3e}")
+
+
+def test_prefill_one_row_repeated(layer0):
+    """1,000 copies of one token: its 6 experts get 1,000 tokens each (eight
+    128-token tiles per expert), the other 250 none; every output row equals
+    the single-row oracle result."""
+    T = 1000
+    x1 = synth.prefill_x(1, 9001)
+    x = np.repeat(x1, T, axis=0)
+    out = prefill(layer0, x)
+    ref, idx, w, gap = oracle.moe_layer(layer0["O"], x1)
+    ridx, _ = route(layer0, x)
+    assert (ridx == ridx[0]).all()
+    keep = routing_rows(ridx[:1], idx, gap)
+    if keep:
+        check_close(bf16_to_f64(out), np.repeat(ref, T, axis=0), list(range(T)),
+                    what="repeated row")
+    assert (out == out[0]).all()  # batch invariance across the repeats
