@@ -36,12 +36,15 @@ namespace flint {
 // ============================================================== router (T tokens)
 constexpr int kRtTok = 64;  // tokens per CTA (8 column blocks of 8)
 
-__global__ void __launch_bounds__(256)
+// 16 warps: warp w multiplies experts 16w .. 16w+15 against the CTA's 64 tokens.
+__global__ void __launch_bounds__(512)
     k_pf_router(LayerArgs L, const uint16_t *__restrict__ x, int T, float *__restrict__ z) {
+  // fragment of one k-half: [8 groups][8 blocks][4 words q][32 lanes] (uint4),
+  // so the 32 lanes of a load read 512 consecutive bytes
   extern __shared__ __align__(128) unsigned char sm[];
-  uint4 *frag = reinterpret_cast<uint4 *>(sm);  // [8 groups][8 blocks][32 lanes][4]
+  uint4 *frag = reinterpret_cast<uint4 *>(sm);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-  const int t0 = blockIdx.x * kRtTok, e0 = 128 * blockIdx.y + 16 * warp;
+  const int t0 = blockIdx.x * kRtTok, e0 = 16 * warp;
   double acc[8][4];
 #pragma unroll
   for (int nb = 0; nb < 8; ++nb)
@@ -50,8 +53,8 @@ __global__ void __launch_bounds__(256)
 
   for (int half = 0; half < 2; ++half) {
     __syncthreads();
-    for (int task = tid; task < 8 * 8 * 32 * 4; task += 256) {
-      const int q = task & 3, ln = (task >> 2) & 31, nb = (task >> 7) & 7, Gl = task >> 10;
+    for (int task = tid; task < 8 * 8 * 32 * 4; task += 512) {
+      const int ln = task & 31, q = (task >> 5) & 3, nb = (task >> 7) & 7, Gl = task >> 10;
       const int tok = t0 + 8 * nb + (ln >> 2);
       const int k0 = 128 * (8 * half + Gl) + 32 * (ln & 3) + 8 * q;
       uint4 v = make_uint4(0, 0, 0, 0);
@@ -74,7 +77,11 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
       for (int nb = 0; nb < 8; ++nb) {
         uint32_t xb[16];
-        load_frag(frag + ((Gl * 8 + nb) * 32 + lane) * 4, xb);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 v = frag[((Gl * 8 + nb) * 4 + q) * 32 + lane];
+          xb[4 * q] = v.x, xb[4 * q + 1] = v.y, xb[4 * q + 2] = v.z, xb[4 * q + 3] = v.w;
+        }
         float d[4];
         group_mma(a, b, xb, d);
 #pragma unroll
@@ -792,7 +799,7 @@ cudaError_t launch_route_many(const LayerArgs &L, const uint16_t *x, int T, int3
                                        8 * 8 * 32 * 64);
   if (e != cudaSuccess) return e;
   note_step("prefill router launch");
-  k_pf_router<<<dim3((T + kRtTok - 1) / kRtTok, 2), 256, 8 * 8 * 32 * 64, st>>>(L, x, T, z);
+  k_pf_router<<<(T + kRtTok - 1) / kRtTok, 512, 8 * 8 * 32 * 64, st>>>(L, x, T, z);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   note_step("prefill top-6 launch");
   k_pf_topk<<<(T + 7) / 8, 256, 0, st>>>(L.router_b, z, T, idx, w,
