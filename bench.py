@@ -34,6 +34,12 @@ import synth  # noqa: E402
 N_LAYERS = synth.N_MOE_LAYERS
 H = synth.HIDDEN
 LAYER_FIXED_BYTES = 256 * 2048 * 2 + 256 * 4 + 2048 * (1024 + 32) + 2048 * (512 + 16)
+# DRAM bytes per decode layer over algorithmic bytes, from the ncu capture in
+# profiles/decode_layer_b4_stack.md (4 layers of this workload at batch 4:
+# 110.69 MB read against 109.63 MB algorithmic); traffic grows with the
+# expert count the same way, so a full layer's traffic is this ratio times
+# its algorithmic bytes.
+DECODE_TRAFFIC_RATIO = 110.69 / 109.63
 EXPERT_BYTES = 1024 * (1024 + 32) + 2048 * (256 + 8)
 HEAD_BYTES = synth.VOCAB * (1024 + 32)
 METRIC = "us per MoE-layer decode (B=4), fraction of HBM roofline"
@@ -450,7 +456,8 @@ def main():
                    "stack_tokens_per_s": B * 1e6 / (us_per_layer * nl * world) * world,
                    "mean_distinct_experts": U},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": None,
+                     "frac": achieved / hbm,
+                     "traffic": DECODE_TRAFFIC_RATIO * bytes_per_layer,
                      "kernel": "decode layer (3 PDL-chained kernels)",
                      "peak_kind": peak_kind, "bytes_per_layer": bytes_per_layer},
         "e2e": {"value": e2e_us, "unit": "us/layer", "h2d_bytes_per_step": B * H * 4,
