@@ -115,6 +115,18 @@ FLINT_API int flint_workspace_init(void *ws, size_t ws_bytes, void *stream);
  * *status is FLINT_OK unless a device-side check or bounded wait failed. */
 FLINT_API int flint_read_status(const void *ws, int *status, void *stream);
 
+/* Test hook for the failure path: the poll bound of the decode kernels'
+ * (flint_moe_route, flint_moe_decode, flint_moe_decode_residual) first wait
+ * on each shared-memory barrier.  The default is 1 << 26 polls (seconds); a
+ * small value, 0 included, makes those waits give up at once, so the call
+ * records FLINT_ETIMEOUT in the workspace status word and returns without a
+ * result (the outputs are left as they were).  Every wait on that error path
+ * keeps the default bound, so copies already in flight land before a CTA
+ * exits.  polls = 0xFFFFFFFF restores the default.  Applies to the current
+ * device; synchronous.  Not for production use: a lowered bound turns
+ * ordinary latency into timeouts. */
+FLINT_API int flint_debug_set_wait_polls(uint32_t polls);
+
 /*
  * Router for B rows ("How to Run Flint Locally", section "The architecture,
  * from config.json": sigmoid router over 256 experts, top 6 kept, weights

@@ -21,7 +21,8 @@ HIDDEN, EXPERTS, TOP_K, EXPERT_I, SHARED_I, GROUP, MAX_DECODE_B = 2048, 256, 6, 
 EXPORTS = ("flint_version", "flint_strerror", "flint_last_cuda_error", "flint_workspace_bytes",
            "flint_gemv_workspace_bytes", "flint_workspace_init", "flint_read_status",
            "flint_moe_route", "flint_moe_decode", "flint_moe_decode_residual",
-           "flint_moe_prefill", "flint_int4_gemv", "flint_int4_gemv_noalloc")
+           "flint_moe_prefill", "flint_int4_gemv", "flint_int4_gemv_noalloc",
+           "flint_debug_set_wait_polls")
 
 _lib = None
 
@@ -62,6 +63,7 @@ def lib() -> C.CDLL:
         L.flint_gemv_workspace_bytes.argtypes = [i, i]
         L.flint_workspace_init.argtypes = [vp, sz, vp]
         L.flint_read_status.argtypes = [vp, C.POINTER(C.c_int), vp]
+        L.flint_debug_set_wait_polls.argtypes = [C.c_uint32]
         lp = C.POINTER(flint_moe_layer)
         L.flint_moe_route.argtypes = [lp, vp, i, vp, vp, vp, sz, vp]
         L.flint_moe_decode.argtypes = [lp, vp, i, vp, vp, sz, vp]
@@ -123,6 +125,12 @@ def flint_gemv_workspace_bytes(N: int, B: int) -> int:
 
 def flint_workspace_init(ws, ws_bytes: int, stream=None):
     _check(lib().flint_workspace_init(_ptr(ws), ws_bytes, _stream(stream)), "flint_workspace_init")
+
+
+def flint_debug_set_wait_polls(polls: int) -> None:
+    """Poll bound of the decode kernels' first barrier waits (test hook for
+    the timeout path); 0xFFFFFFFF restores the default."""
+    _check(lib().flint_debug_set_wait_polls(polls), "flint_debug_set_wait_polls")
 
 
 def flint_read_status(ws, stream=None) -> int:

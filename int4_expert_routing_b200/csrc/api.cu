@@ -101,6 +101,10 @@ int flint_read_status(const void *ws, int *status, void *stream) {
   return FLINT_OK;
 }
 
+int flint_debug_set_wait_polls(uint32_t polls) {
+  return from_cuda(noted(decode_set_wait_polls(polls), "debug wait bound"));
+}
+
 int flint_moe_route(const flint_moe_layer *layer, const uint16_t *x, int B, int32_t *idx,
                     float *w, void *ws, size_t ws_bytes, void *stream) {
   if (!layer_ok(layer) || !aligned16(x) || !idx || !w || B < 1 || B > FLINT_MAX_PREFILL_T ||

@@ -223,6 +223,17 @@ FLINT_DEV void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *ba
 // later async-proxy (bulk copy / tensor core) accesses of the same memory.
 FLINT_DEV void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
+// One poll of phase `parity` of `bar`.
+FLINT_DEV bool mbar_try(uint64_t *bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
 // Bounded wait for phase `parity` of `bar`; false if it did not complete.
 FLINT_DEV bool mbar_wait(uint64_t *bar, uint32_t parity) {
   for (uint32_t i = 0; i < kWaitPolls; ++i) {

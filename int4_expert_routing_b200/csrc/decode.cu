@@ -63,6 +63,18 @@ FLINT_DEV void trace_point(uint32_t kernel, uint32_t event, uint32_t dep = 0) {
 FLINT_DEV void trace_point(uint32_t, uint32_t, uint32_t = 0) {}
 #endif
 
+// Poll bound of the decode kernels' first wait on each barrier (the copies a
+// CTA issued).  flint_debug_set_wait_polls lowers it so that a test can drive
+// the timeout path; every wait on an error path uses the fixed kWaitPolls,
+// so copies still in flight land before the CTA exits.
+static __device__ uint32_t g_decode_polls = kWaitPolls;
+FLINT_DEV bool dwait(uint64_t *bar, uint32_t parity) {
+  const uint32_t n = *reinterpret_cast<volatile uint32_t *>(&g_decode_polls);
+  for (uint32_t i = 0; i < n; ++i)
+    if (mbar_try(bar, parity)) return true;
+  return false;
+}
+
 constexpr int kRouterCtas = 32;   // 16 expert tiles x 2 k-halves
 constexpr int kK1Threads = 256;   // 8 warps: one 128-wide k-group each
 static_assert(kK1Threads == kE, "the last router CTA scores one expert per thread");
@@ -268,10 +280,10 @@ __global__ void __launch_bounds__(kK1Threads)
     const int i = (8 * kh) * 4 * B * 4 + et * per + tid;
     if (tid < per) reinterpret_cast<uint4 *>(ws + lay.xfrag)[i] = frag[i];
   }
-  const bool ok = mbar_wait(&bar, 0);
+  const bool ok = dwait(&bar, 0);
   if (__syncthreads_or(!ok)) {
     if (tid == 0) set_status(ctrl + 1, kStatusTimeout);
-    if (!ok) mbar_wait(&bar, 0);
+    if (!ok) mbar_wait(&bar, 0);  // the router rows still in flight land first
     return;
   }
   trace_point(1, 5);
@@ -553,9 +565,13 @@ __global__ void __launch_bounds__(kK2Warps * 32)
   }
   __syncthreads();
   const int n = s_n;
-  bool ok = mbar_wait(&fbar, 0);
+  const bool fok = dwait(&fbar, 0);
+  bool ok = fok;
   if (n == 0) {
-    if (!ok && tid == 0) set_status(ctrl + 1, kStatusTimeout);
+    if (!fok) {
+      if (tid == 0) set_status(ctrl + 1, kStatusTimeout);
+      mbar_wait(&fbar, 0);  // the fragment copy still in flight lands first
+    }
     return;
   }
   for (int j = 0; j < n; ++j) {
@@ -563,11 +579,12 @@ __global__ void __launch_bounds__(kK2Warps * 32)
     const int it = c0 + j * step;
     const uint32_t word = s_word[j];
     unsigned char *buf = sm + st * kItemBytes;
-    ok = mbar_wait(&bar[st], (uint32_t)((j / kK2Stages) & 1)) && ok;
+    ok = dwait(&bar[st], (uint32_t)((j / kK2Stages) & 1)) && ok;
     trace_point(2, 2);
     if (__syncthreads_or(!ok)) {
       if (tid == 0) set_status(ctrl + 1, kStatusTimeout);
-      // copies still in flight get one more bounded wait each
+      // copies still in flight land before the CTA exits
+      if (!fok) mbar_wait(&fbar, 0);
       for (int jj = j; jj < n && jj < j + kK2Stages; ++jj)
         mbar_wait(&bar[jj % kK2Stages], (uint32_t)((jj / kK2Stages) & 1));
       return;
@@ -676,13 +693,15 @@ __global__ void __launch_bounds__(kK3Threads)
   if (kResidual && tid < 16 * B) h_old = ld_cg_f32(h + (size_t)(tid >> 4) * kH + n0 + (tid & 15));
   if (tid < kE) {
     const uint32_t word = ld_cg_u32(reinterpret_cast<const uint32_t *>(ws + lay.slot_word) + tid);
-    if (word != kSlotInvalid) {
+    // at most umax slots have room here; a routing left by a failed K1 may
+    // hold more, and none of it is used after the status is set
+    if (word != kSlotInvalid && tid < umax) {
       const size_t e = slot_expert(word);
       s_rows[tid] = slot_mask(word);
       mbar_add_tx(&bar, 4096 + 128);
       bulk_g2s(wsm + tid * 4096, L.w2_q + (e * kH + n0) * (kI / 2), 4096, &bar);
       bulk_g2s(ssm + tid * 128, L.w2_s + (e * kH + n0) * (kI / kG), 128, &bar);
-      if (tid == 0) s_ns = slot_count(word);
+      if (tid == 0) s_ns = min(slot_count(word), umax);
     }
   } else if (tid == kE) {
     mbar_add_tx(&bar, 8192 + 256);
@@ -708,10 +727,10 @@ __global__ void __launch_bounds__(kK3Threads)
       cp_async16(reinterpret_cast<unsigned char *>(himg_s) + 16 * i, src_s + 16 * i);
     cp_async_wait_all();
   }
-  const bool arrived = mbar_wait(&bar, 0);
+  const bool arrived = dwait(&bar, 0);
   if (__syncthreads_or(!arrived)) {
     if (tid == 0) set_status(ctrl + 1, kStatusTimeout);
-    if (!arrived) mbar_wait(&bar, 0);  // copies still in flight get one more bounded wait
+    if (!arrived) mbar_wait(&bar, 0);  // copies still in flight land before the CTA exits
     return;
   }
   const int ns = s_ns;
@@ -916,6 +935,11 @@ static cudaError_t launch_decode_t(const LayerArgs &L, const uint16_t *x, float 
                       L, B, out, h, ws, lay, umax);
   return launch_pdl(k3_down_combine<kResidual, false>, kH / 16, kK3Threads, P.total(false), st, L,
                     B, out, h, ws, lay, umax);
+}
+
+cudaError_t decode_set_wait_polls(uint32_t polls) {
+  if (polls == 0xFFFFFFFFu) polls = kWaitPolls;
+  return cudaMemcpyToSymbol(g_decode_polls, &polls, sizeof(polls));
 }
 
 #ifdef FLINT_TRACE
