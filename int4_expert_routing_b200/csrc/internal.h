@@ -40,28 +40,30 @@ inline DecodeLayout decode_layout(int B) {
   return L;
 }
 
-// Prefill workspace for T tokens (token tile of 128 per expert group).
+// Prefill workspace for T tokens.  The 6T routed rows are sorted by expert
+// with no padding; the token tiles of GEMM 1 (kPfN1 tokens) and GEMM 2
+// (kPfN2) read past a group's end into the next group or, at the end, the
+// zero fill of the TMA box, and those columns are never stored.
 // ctrl words: [1] status, [3] GEMM1 tile count, [4] GEMM2 tile count,
-// [5] routed rows (padded).
-constexpr int kPfTile = 128;
+// [5] routed rows.
+constexpr int kPfN1 = 256;
+constexpr int kPfN2 = 192;
 constexpr int kPfChunk = 256;
 struct PrefillLayout {
   size_t ctrl, z, sel_idx, sel_w, asc_e, asc_w, route_total;
-  size_t pos, chunk_cnt, chunk_off, ebase, ecount, perm, pw, tiles1, tiles2, xp, hr, hs, yw, ys,
-      total;
-  int mr_max, max_tiles1, max_tiles2, nchunks;
+  size_t pos, chunk_cnt, chunk_off, ebase, ecount, perm, pw, tiles1, tiles2, wst, wbound, xstat,
+      rsc, rm3, xp, hr, hs, yw, ys, total;
+  int mr, max_tiles1, max_tiles2, nchunks;
 };
 
 inline PrefillLayout prefill_layout(int T) {
   PrefillLayout L{};
   L.nchunks = (T + kPfChunk - 1) / kPfChunk;
-  // at most min(256, 6T) experts hold tokens; each group is padded to the tile
+  // at most min(256, 6T) experts hold tokens; each adds at most one partial tile
   const int busy = 6 * T < 256 ? 6 * T : 256;
-  L.mr_max = 6 * T + busy * (kPfTile - 1);
-  const int nsh = (T + kPfTile - 1) / kPfTile;
-  const int nrt = (6 * T) / kPfTile + busy;  // routed 128-token tiles, upper bound
-  L.max_tiles1 = 8 * nrt + 16 * nsh;
-  L.max_tiles2 = 16 * nrt + 16 * nsh;
+  L.mr = 6 * T;
+  L.max_tiles1 = 8 * ((6 * T) / kPfN1 + busy) + 16 * ((T + kPfN1 - 1) / kPfN1);
+  L.max_tiles2 = 16 * ((6 * T) / kPfN2 + busy) + 16 * ((T + kPfN2 - 1) / kPfN2);
   size_t o = 0;
   auto take = [&](size_t bytes) {
     size_t at = o;
@@ -80,14 +82,19 @@ inline PrefillLayout prefill_layout(int T) {
   L.chunk_off = take(sizeof(int32_t) * (size_t)L.nchunks * 256);
   L.ebase = take(sizeof(int32_t) * 257);
   L.ecount = take(sizeof(int32_t) * 256);
-  L.perm = take(sizeof(int32_t) * (size_t)L.mr_max);
-  L.pw = take(sizeof(float) * (size_t)L.mr_max);
+  L.perm = take(sizeof(int32_t) * (size_t)L.mr);
+  L.pw = take(sizeof(float) * (size_t)L.mr);
   L.tiles1 = take(sizeof(int32_t) * (size_t)L.max_tiles1);
   L.tiles2 = take(sizeof(int32_t) * (size_t)L.max_tiles2);
-  L.xp = take(sizeof(uint16_t) * (size_t)L.mr_max * 2048);
-  L.hr = take(sizeof(uint16_t) * (size_t)L.mr_max * 512 * 2);  // SwiGLU hi, lo
-  L.hs = take(sizeof(uint16_t) * (size_t)T * 1024 * 2);
-  L.yw = take(sizeof(uint16_t) * (size_t)L.mr_max * 2048);
+  L.wst = take(sizeof(float) * 4 * 257);   // per expert matrix pair: power-of-two shifts
+  L.wbound = take(sizeof(float) * 257);    // per expert: bound factor of the SwiGLU output
+  L.xstat = take(sizeof(float) * 2 * (size_t)T);     // per token: 2^-F, 2^E
+  L.rsc = take(sizeof(float) * 2 * (size_t)7 * T);   // per row: 2^F, 2^-E
+  L.rm3 = take(sizeof(float) * (size_t)7 * T);       // per row: 2^E x routing weight
+  L.xp = take(sizeof(uint16_t) * (size_t)7 * T * 2048);  // fp16 token rows: routed, then all T
+  L.hr = take(sizeof(uint16_t) * (size_t)L.mr * 512);    // fp16 SwiGLU intermediate, routed
+  L.hs = take(sizeof(uint16_t) * (size_t)T * 1024);      // fp16 SwiGLU intermediate, shared
+  L.yw = take(sizeof(uint16_t) * (size_t)L.mr * 2048);
   L.ys = take(sizeof(uint16_t) * (size_t)T * 2048);
   L.total = o;
   return L;

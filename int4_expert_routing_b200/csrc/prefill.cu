@@ -213,15 +213,13 @@ FLINT_DEV uint32_t pack_tile(int e, int mt, int nt) {
 }
 
 // One CTA of 256 threads (one per expert): chunk offsets, expert counts,
-// padded bases, padding rows of the permutation, and both GEMM tile lists
-// (the 16 or 8 row tiles of one token tile are adjacent, so the token tile is
-// reused from L2).
+// group bases (no padding) and both GEMM tile lists (the 8 or 16 row tiles of
+// one token tile are adjacent, so the token tile is reused from L2).
 __global__ void __launch_bounds__(256)
     k_pf_scan(int T, int nchunks, const int32_t *__restrict__ chunk_cnt,
               int32_t *__restrict__ chunk_off, int32_t *__restrict__ ebase,
-              int32_t *__restrict__ ecount, int32_t *__restrict__ perm,
-              uint32_t *__restrict__ tiles1, uint32_t *__restrict__ tiles2,
-              uint32_t *__restrict__ ctrl) {
+              int32_t *__restrict__ ecount, uint32_t *__restrict__ tiles1,
+              uint32_t *__restrict__ tiles2, uint32_t *__restrict__ ctrl) {
   __shared__ int s_warp[8];
   const int e = threadIdx.x;
   int off = 0;
@@ -231,27 +229,24 @@ __global__ void __launch_bounds__(256)
     off += chunk_cnt[(size_t)c * kE + e];
   }
   ecount[e] = off;
-  const int ntile = (off + kPfTile - 1) / kPfTile;
+  const int nt1 = (off + kPfN1 - 1) / kPfN1, nt2 = (off + kPfN2 - 1) / kPfN2;
   int total_rows, total1, total2;
-  const int base = block_scan(ntile * kPfTile, s_warp, &total_rows);
-  const int o1 = block_scan(8 * ntile, s_warp, &total1);
-  const int o2 = block_scan(16 * ntile, s_warp, &total2);
+  const int base = block_scan(off, s_warp, &total_rows);
+  const int o1 = block_scan(8 * nt1, s_warp, &total1);
+  const int o2 = block_scan(16 * nt2, s_warp, &total2);
   ebase[e] = base;
   if (e == 0) ebase[kE] = total_rows;
-  for (int p = base + off; p < base + ntile * kPfTile; ++p) perm[p] = -1;
-  for (int nt = 0; nt < ntile; ++nt) {
+  for (int nt = 0; nt < nt1; ++nt)
     for (int mt = 0; mt < 8; ++mt) tiles1[o1 + nt * 8 + mt] = pack_tile(e, mt, nt);
+  for (int nt = 0; nt < nt2; ++nt)
     for (int mt = 0; mt < 16; ++mt) tiles2[o2 + nt * 16 + mt] = pack_tile(e, mt, nt);
-  }
   // the shared expert: one group over all T tokens
-  const int nsh = (T + kPfTile - 1) / kPfTile;
-  for (int i = e; i < 16 * nsh; i += kE) {
-    tiles1[total1 + i] = pack_tile(kE, i & 15, i >> 4);
-    tiles2[total2 + i] = pack_tile(kE, i & 15, i >> 4);
-  }
+  const int nsh1 = (T + kPfN1 - 1) / kPfN1, nsh2 = (T + kPfN2 - 1) / kPfN2;
+  for (int i = e; i < 16 * nsh1; i += kE) tiles1[total1 + i] = pack_tile(kE, i & 15, i >> 4);
+  for (int i = e; i < 16 * nsh2; i += kE) tiles2[total2 + i] = pack_tile(kE, i & 15, i >> 4);
   if (e == 0) {
-    ctrl[3] = (uint32_t)(total1 + 16 * nsh);
-    ctrl[4] = (uint32_t)(total2 + 16 * nsh);
+    ctrl[3] = (uint32_t)(total1 + 16 * nsh1);
+    ctrl[4] = (uint32_t)(total2 + 16 * nsh2);
     ctrl[5] = (uint32_t)total_rows;
   }
 }
@@ -277,58 +272,201 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// Routed token rows in sorted order; padding rows are zero.
+// ---------------------------------------------------------- fp16 operand scaling
+// Both GEMM operands are fp16 holding exact values (see the GEMM below), made
+// so by power-of-two shifts: per expert matrix for the weights, per token for
+// the token rows and the SwiGLU intermediate.
+
+// 2^n as a float for n in the normal range
+FLINT_DEV float exp2i(int n) { return __int_as_float((n + 127) << 23); }
+// a shift n such that both 2^n and 2^-n are normal floats
+FLINT_DEV int clamp_shift(int n) { return min(max(n, -126), 126); }
+
+// One CTA per expert (expert 256 = the shared one).  For the gate/up matrix
+// and the down matrix the shift S puts the largest |code x scale| (|code| <= 8)
+// in [2^14, 2^15); wst[e] = (2^-S1, 2^S1, 2^-S2, 2^S2).  wbound[e] bounds the
+// SwiGLU output per unit of |x|^2: by Cauchy-Schwarz |W1 x| <= |x| |W1 row| and
+// |silu(g)| <= |g|, so |silu(W1 x) (W3 x)| <= |x|^2 max|W1 row| max|W3 row|,
+// with |row| <= 8 sqrt(128 sum_g scale_g^2) for 128-wide groups of codes in [-8, 7].
 __global__ void __launch_bounds__(256)
-    k_pf_gather(const uint16_t *__restrict__ x, const int32_t *__restrict__ perm,
-                const uint32_t *__restrict__ ctrl, uint16_t *__restrict__ xp) {
-  const size_t rows = __ldcg(ctrl + 5);
+    k_pf_wstats(const uint16_t *__restrict__ w13_s, const uint16_t *__restrict__ w2_s,
+                const uint16_t *__restrict__ sh13_s, const uint16_t *__restrict__ sh2_s,
+                float4 *__restrict__ wst, float *__restrict__ wbound) {
+  __shared__ float red[4][8];
+  const int e = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool sh = e == kE;
+  const int r13 = sh ? 2 * kIs : 2 * kI;  // gate rows, then as many up rows
+  const uint16_t *s13 = sh ? sh13_s : w13_s + (size_t)e * r13 * (kH / kG);
+  const int g2 = (sh ? kIs : kI) / kG;
+  const uint16_t *s2 = sh ? sh2_s : w2_s + (size_t)e * kH * g2;
+  float mx1 = 0.f, mx2 = 0.f, bg = 0.f, bu = 0.f;
+  for (int r = tid; r < r13; r += 256) {
+    const uint4 *p = reinterpret_cast<const uint4 *>(s13 + (size_t)r * (kH / kG));
+    float ss = 0.f;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint4 v = __ldg(p + h);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float a = fabsf(__uint_as_float(w[q] << 16)), b = fabsf(__uint_as_float(w[q] & 0xffff0000u));
+        mx1 = fmaxf(mx1, fmaxf(a, b));
+        ss = fmaf(a, a, fmaf(b, b, ss));
+      }
+    }
+    const float rb = 8.f * sqrtf(128.f * ss);
+    if (r < r13 / 2) bg = fmaxf(bg, rb);
+    else bu = fmaxf(bu, rb);
+  }
+  for (int i = tid; i < kH * g2 / 2; i += 256) {
+    const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(s2) + i);
+    mx2 = fmaxf(mx2, fmaxf(fabsf(__uint_as_float(w << 16)), fabsf(__uint_as_float(w & 0xffff0000u))));
+  }
+  float v[4] = {mx1, mx2, bg, bu};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v[k] = fmaxf(v[k], __shfl_xor_sync(0xffffffffu, v[k], o));
+    if (lane == 0) red[k][warp] = v[k];
+  }
+  __syncthreads();
+  if (tid == 0) {
+    float m[4];
+    for (int k = 0; k < 4; ++k) {
+      m[k] = red[k][0];
+      for (int w = 1; w < 8; ++w) m[k] = fmaxf(m[k], red[k][w]);
+    }
+    const int S1 = m[0] > 0.f ? clamp_shift(ilogbf(m[0]) + 3 - 14) : 0;
+    const int S2 = m[1] > 0.f ? clamp_shift(ilogbf(m[1]) + 3 - 14) : 0;
+    wst[e] = make_float4(exp2i(-S1), exp2i(S1), exp2i(-S2), exp2i(S2));
+    wbound[e] = m[2] * m[3];
+  }
+}
+
+// One warp per token: F puts max|x| in [2^14, 2^15); E puts the SwiGLU output
+// bound |x|^2 max_e wbound[e] below 2^15.  xstat[t] = (2^-F, 2^E).
+__global__ void __launch_bounds__(256)
+    k_pf_xstats(const uint16_t *__restrict__ x, int T, const float *__restrict__ wbound,
+                float2 *__restrict__ xstat) {
+  __shared__ float s_k;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (warp == 0) {
+    float k = 0.f;
+    for (int i = lane; i <= kE; i += 32) k = fmaxf(k, wbound[i]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) k = fmaxf(k, __shfl_xor_sync(0xffffffffu, k, o));
+    if (lane == 0) s_k = k;
+  }
+  __syncthreads();
+  const int t = blockIdx.x * 8 + warp;
+  if (t >= T) return;
+  const uint4 *row = reinterpret_cast<const uint4 *>(x + (size_t)t * kH);
+  float mx = 0.f;
+  double ss = 0.0;
+#pragma unroll
+  for (int c = 0; c < kH / 8 / 32; ++c) {
+    const uint4 v = ld_cg_v4(reinterpret_cast<const uint16_t *>(row + c * 32 + lane));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float a = __uint_as_float(w[q] << 16), b = __uint_as_float(w[q] & 0xffff0000u);
+      mx = fmaxf(mx, fmaxf(fabsf(a), fabsf(b)));
+      ss += (double)a * a + (double)b * b;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  }
+  if (lane == 0) {
+    const int F = mx > 0.f ? clamp_shift(ilogbf(mx) - 14) : 0;
+    const double bound = ss * (double)s_k * (1.0 + 1.0 / 1024);  // rounding margin
+    const int E = bound > 0.0 ? clamp_shift(ilogb(bound) + 1 - 15) : 0;
+    xstat[t] = make_float2(exp2i(-F), exp2i(E));
+  }
+}
+
+// Token rows as the fp16 operand of GEMM 1: rows [0, 6T) are the routed rows
+// in sorted order, rows [6T, 7T) every token for the shared expert.  Each
+// 8-element block is stored in the order 0,4,1,5,2,6,3,7.  Per row, rsc =
+// (2^F, 2^-E) for GEMM 1's read-out and rm3 = 2^E x routing weight for GEMM 2's.
+__global__ void __launch_bounds__(256)
+    k_pf_gather(const uint16_t *__restrict__ x, int T, const int32_t *__restrict__ perm,
+                const float *__restrict__ pw, const float2 *__restrict__ xstat,
+                uint16_t *__restrict__ xp, float2 *__restrict__ rsc, float *__restrict__ rm3) {
+  const size_t rows = (size_t)7 * T;
   const size_t n = rows * (kH / 8);
   for (size_t i = (size_t)blockIdx.x * 256 + threadIdx.x; i < n; i += (size_t)gridDim.x * 256) {
     const size_t row = i / (kH / 8), c = i % (kH / 8);
-    const int tok = perm[row];
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (tok >= 0) v = ld_cg_v4(x + (size_t)tok * kH + 8 * c);
-    *reinterpret_cast<uint4 *>(xp + row * kH + 8 * c) = v;
+    const bool routed = row < (size_t)6 * T;
+    const int tok = routed ? perm[row] : (int)(row - (size_t)6 * T);
+    const float2 st = xstat[tok];
+    const uint4 v = ld_cg_v4(x + (size_t)tok * kH + 8 * c);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t h[8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      h[2 * q] = __half_as_ushort(__float2half_rn(__uint_as_float(w[q] << 16) * st.x));
+      h[2 * q + 1] = __half_as_ushort(__float2half_rn(__uint_as_float(w[q] & 0xffff0000u) * st.x));
+    }
+    // natural h[0..7] -> pairs (0,4), (1,5), (2,6), (3,7)
+    *reinterpret_cast<uint4 *>(xp + row * kH + 8 * c) =
+        make_uint4(h[0] | (h[4] << 16), h[1] | (h[5] << 16), h[2] | (h[6] << 16), h[3] | (h[7] << 16));
+    if (c == 0) {
+      rsc[row] = make_float2(1.f / st.x, 1.f / st.y);
+      rm3[row] = routed ? st.y * pw[row] : st.y;
+    }
   }
 }
 
 // ============================================================== tcgen05 grouped GEMM
-// Tile: 128 weight rows (A) x 128 tokens (N), K in stages of 64.  A holds the
-// int4 codes as exact bf16 values; the bf16 scale of each (row, 128-wide
-// k-group) is applied in fp32 when the group's partial sum is read out of
-// tensor memory, so the weights enter the product exactly.  Two TMEM
-// accumulator buffers let the MMAs of group G+1 run while group G is read.
-// GEMM 2's token operand is the SwiGLU intermediate as a hi/lo bf16 pair (two
-// MMA passes over the same A tile), ~16 significant bits.
-constexpr int kABytes = 128 * 128;      // 128 weight rows x 64 bf16
-constexpr int kBBytes = kPfTile * 128;  // 128 token rows x 64 bf16
-constexpr int kRawBytes = 128 * 32;     // 128 weight rows x 64 int4
-// Four warpgroups: 0 = producer, MMA issuer and two idle warps; 1 = four
-// dequant warps (one weight row per thread); 2-3 = eight epilogue warps (two
-// per TMEM lane quarter, one per 64-token half of the tile).  The block is
-// launched at 128 registers per thread (65,536); setmaxnreg then moves them:
-// 128 x 40 + 128 x 64 + 256 x 200 = 64,512.
+// One tile is 128 weight rows (the MMA's M) by kN tokens (its N), with the
+// whole K summed in one fp32 accumulator in tensor memory.  Both operands are
+// fp16 holding exact values:
+//  - the weights as code x scale x 2^-S: a code in [-8, 7] has at most 3
+//    significant bits and a bf16 scale 8, so the product fits fp16's 11, and
+//    the per-matrix shift S keeps it in the normal range.  Four dequant warps
+//    write the tile straight into tensor memory (tcgen05.st), and the MMA
+//    takes A from there;
+//  - the tokens as x 2^-F (bf16 values, exact in fp16) for GEMM 1 and as the
+//    SwiGLU intermediate x 2^-E (rounded to fp16, 11 bits) for GEMM 2, loaded
+//    by TMA into 128-byte-swizzled shared memory.
+// The read-out multiplies by 2^(S+F) or 2^(S+E).  Inside every 8-wide k block
+// both operands hold the order 0,4,1,5,2,6,3,7 (the order int4 unpacking
+// yields two codes per 32-bit word); the dot products do not depend on it.
+constexpr int kRawBytes = 128 * 64;  // 128 weight rows x 128 int4 codes: one k-group
+// Four warpgroups: 0 = producer (warp 0), MMA issuer (warp 1) and two idle
+// warps; 1 = four dequant warps (one weight row per thread); 2-3 = eight
+// epilogue warps (two per TMEM lane quarter, one per half of the tile's
+// tokens).  The block is launched at 128 registers per thread (65,536);
+// setmaxnreg moves them: 128 x 40 + 128 x 88 + 256 x 184 = 63,488.
 constexpr int kGemmThreads = 512;
-constexpr int kDeqThreads = 128;
-constexpr int kEpiThreads = 256;
-constexpr int kRegCtl = 40, kRegDeq = 64, kRegEpi = 200;
+constexpr int kRegCtl = 40, kRegDeq = 88, kRegEpi = 184;
 static_assert(128 * kRegCtl + 128 * kRegDeq + 256 * kRegEpi <= 65536, "register split");
-constexpr int kTmemCols = 512;          // four 128-column fp32 accumulators (one CTA per SM)
-constexpr int kTmemBufs = kTmemCols / 128;
+constexpr int kTmemCols = 512;
 
+// kN tokens per tile, kAcc accumulators of kN columns, kNA weight tiles of 64
+// columns (128 fp16 k values per row), kS shared-memory stages (int4 codes and
+// the token tile of one 128-wide k-group each).
 template <int kMode>
 struct GemmCfg {
-  static constexpr int kNB = kMode == 1 ? 1 : 2;  // token operands per stage (hi, lo)
-  static constexpr int kAtoms = 2;                // 64-wide k atoms per stage: one k-group
-  // stage: A atoms | token atoms (operand-major) | int4 codes of the atoms
-  static constexpr int kStageBytes = kAtoms * (kABytes + kNB * kBBytes + kRawBytes);
-  static constexpr int kStages = kMode == 1 ? 3 : 2;
-  static constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024;
-  static constexpr uint32_t a_off(int atom) { return (uint32_t)(atom * kABytes); }
-  static constexpr uint32_t b_off(int nb, int atom) {
-    return (uint32_t)(kAtoms * kABytes + (nb * kAtoms + atom) * kBBytes);
+  static constexpr int kN = kMode == 1 ? kPfN1 : kPfN2;
+  static constexpr int kAcc = kMode == 1 ? 1 : 2;
+  static constexpr int kNA = kMode == 1 ? 4 : 2;
+  static constexpr int kS = 3;
+  static constexpr int kBAtom = kN * 128;  // kN token rows x 64 fp16
+  static constexpr int kStageBytes = kRawBytes + 2 * kBAtom;
+  static constexpr size_t kSmem = (size_t)kS * kStageBytes + 1024;
+  // TMEM columns: GEMM 1: accumulator 0..255, weight tiles 256, 320, 384, 448;
+  // GEMM 2: accumulators at 0 and 256 (192 columns each), weight tiles 192, 448
+  static constexpr uint32_t acc_col(int b) { return (uint32_t)(256 * b); }
+  static constexpr uint32_t a_col(int a) {
+    return kMode == 1 ? (uint32_t)(256 + 64 * a) : (uint32_t)(192 + 256 * a);
   }
-  static constexpr uint32_t raw_off() { return (uint32_t)(kAtoms * (kABytes + kNB * kBBytes)); }
+  static_assert(kMode == 1 ? (kN <= 256 && kAcc == 1 && kNA == 4)
+                           : (kN <= 192 && kAcc == 2 && kNA == 2), "tensor memory");
+  static_assert(kBAtom % 1024 == 0 && kN % 32 == 0, "tile shape");
 };
 
 struct GemmArgs {
@@ -340,11 +478,11 @@ struct GemmArgs {
   int T;
   const uint16_t *sc_r;  // scales of the routed weight tensor
   const uint16_t *sc_s;  // scales of the shared expert's tensor
-  uint16_t *out_r;       // GEMM 1: H hi (lo follows at out_r_lo); GEMM 2: Yw
-  uint16_t *out_r_lo;
-  uint16_t *out_s;       // GEMM 1: Hs hi; GEMM 2: Ys
-  uint16_t *out_s_lo;
-  const float *pw;
+  const float4 *wst;     // per expert: 2^-S1, 2^S1, 2^-S2, 2^S2
+  const float2 *rsc;     // per row: 2^F, 2^-E
+  const float *rm3;      // per row: 2^E x routing weight
+  uint16_t *out_r;       // GEMM 1: Hr fp16 [6T][512]; GEMM 2: Yw bf16 [6T][2048]
+  uint16_t *out_s;       // GEMM 1: Hs fp16 [T][1024]; GEMM 2: Ys bf16 [T][2048]
   uint32_t *status;
 };
 
@@ -361,12 +499,13 @@ FLINT_DEV void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint
       : "memory");
 }
 
-FLINT_DEV void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                         uint32_t accum) {
+// D (TMEM) += A (TMEM, 128 lanes x 8 columns of fp16 pairs) x B (shared memory)
+FLINT_DEV void umma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                           uint32_t accum) {
   asm volatile(
-      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, "
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, "
       "%3, p;\n}\n" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum));
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accum));
 }
 
 FLINT_DEV void umma_commit(uint64_t *bar) {
@@ -377,9 +516,10 @@ FLINT_DEV void umma_commit(uint64_t *bar) {
 }
 
 // Optional GEMM timeline (build with -DFLINT_TRACE): for the first kPfTrTiles
-// CTAs of each GEMM, %globaltimer per k-stage for the producer (TMA issued),
-// the dequant warps (tile written), the MMA warp (MMAs issued), and per
-// k-group for the epilogue (group read out); read with flint_pf_trace_dump.
+// CTAs of each GEMM, %globaltimer per k-group of the CTA's first tile for the
+// producer (TMA issued), the dequant warps (tile written), the MMA warp (MMAs
+// issued) and, per tile, the epilogue (accumulator read); read with
+// flint_pf_trace_dump.
 #ifdef FLINT_TRACE
 constexpr int kPfTrTiles = 8;
 static __device__ unsigned long long g_pf_tr[2][kPfTrTiles][8][64];
@@ -398,8 +538,9 @@ extern "C" FLINT_API int flint_pf_trace_dump(unsigned long long *out) {
 FLINT_DEV void pf_mark(int, int, int) {}
 #endif
 
-// 32 consecutive TMEM columns of this warp's 32 lanes; completes at tmem_wait_ld().
-FLINT_DEV void tmem_ld32_async(uint32_t taddr, uint32_t (&v)[32]) {
+// 32 consecutive TMEM columns of this warp's 32 lanes into v[0..31]; completes
+// at tmem_wait_ld().
+FLINT_DEV void tmem_ld32_async(uint32_t taddr, uint32_t *v) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%"
       "15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
@@ -412,51 +553,61 @@ FLINT_DEV void tmem_ld32_async(uint32_t taddr, uint32_t (&v)[32]) {
 }
 FLINT_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// v[0..31] into 32 consecutive TMEM columns of this warp's 32 lanes
+FLINT_DEV void tmem_st32(uint32_t taddr, const uint32_t *v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%"
+      "14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+      "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+      "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+FLINT_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 FLINT_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 FLINT_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// 32 int4 codes (one 16-byte chunk of a raw row) -> four 16-byte chunks of
-// exact bf16 codes in natural element order.
-FLINT_DEV void codes32(uint4 w, uint4 (&out)[4]) {
-  uint32_t r[16];
-  int4x32_to_bf16x2(w, r);
+// 8 int4 codes (one 32-bit word, code k in bits 4k..4k+3) times an fp16x2
+// scale: pairs (k, k+4) for k = 0..3, exact.
+FLINT_DEV void codes8_f16(uint32_t w, uint32_t sc2, uint32_t *out) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q)
-    out[q] = make_uint4(__byte_perm(r[4 * q + 0], r[4 * q + 1], 0x5410),   // (c0, c1)
-                        __byte_perm(r[4 * q + 2], r[4 * q + 3], 0x5410),   // (c2, c3)
-                        __byte_perm(r[4 * q + 0], r[4 * q + 1], 0x7632),   // (c4, c5)
-                        __byte_perm(r[4 * q + 2], r[4 * q + 3], 0x7632));  // (c6, c7)
+  for (int p = 0; p < 4; ++p) {
+    // (code ^ 8) + 1024 as fp16, exact; minus 1032 gives the signed code
+    const uint32_t t = ((w >> (4 * p)) & 0x000F000Fu) ^ 0x64086408u;
+    uint32_t c;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(c) : "r"(t), "r"(0x64086408u));
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(out[p]) : "r"(c), "r"(sc2));
+  }
 }
 
-FLINT_DEV void split_hilo(float v, uint16_t &hi, uint16_t &lo) {
-  const __nv_bfloat16 h = __float2bfloat16_rn(v);
-  hi = __bfloat16_as_ushort(h);
-  lo = __bfloat16_as_ushort(__float2bfloat16_rn(v - __bfloat162float(h)));
-}
+// position of natural column c inside its 8-wide block: 0,4,1,5,2,6,3,7 order
+FLINT_DEV int perm8(int c) { return (c & ~7) | ((c & 7) < 4 ? 2 * (c & 7) : 2 * (c & 7) - 7); }
 
-// kMode 1: gate/up + SwiGLU -> H hi/lo (routed [rows][512], shared [T][1024]).
-// kMode 2: down -> Yw (routed, weighted, [rows][2048]) / Ys (shared, [T][2048]).
+// kMode 1: gate/up + SwiGLU -> Hr (routed rows) / Hs (shared, [T][1024]), fp16.
+// kMode 2: down -> Yw (routed, weighted, [6T][2048]) / Ys ([T][2048]), bf16.
 // One tile of a grouped GEMM, as every role of the CTA derives it.
-template <int kMode>
 struct PfTile {
-  int e, mt, n0, n_valid, n_mma, b_row, row0, row1, ks, ng;
+  int e, mt, n0, n_valid, n_mma, b_row, row0, row1, ng;
   bool sh;
 };
 template <int kMode>
-FLINT_DEV bool pf_tile(const GemmArgs &args, uint32_t idx, PfTile<kMode> &t) {
-  using Cfg = GemmCfg<kMode>;
+FLINT_DEV bool pf_tile(const GemmArgs &args, uint32_t idx, PfTile &t) {
+  constexpr int kN = GemmCfg<kMode>::kN;
   const uint32_t packed = __ldcg(args.tiles + idx);
   t.e = (int)(packed & 511u);
   t.mt = (int)((packed >> 9) & 31u);
   const int nt = (int)(packed >> 14);
   t.sh = t.e == kE;
-  t.n0 = nt * kPfTile;
-  t.n_valid = min(kPfTile, (t.sh ? args.T : __ldcg(args.ecount + t.e)) - t.n0);
+  t.n0 = nt * kN;
+  t.n_valid = min(kN, (t.sh ? args.T : __ldcg(args.ecount + t.e)) - t.n0);
   if (t.n_valid <= 0) return false;  // not produced by the scan; guards against an N = 0 MMA
   t.n_mma = (t.n_valid + 15) & ~15;
-  t.b_row = t.sh ? t.n0 : __ldcg(args.ebase + t.e) + t.n0;
-  t.ks = (kMode == 1 ? kH : (t.sh ? kIs : kI)) / (64 * Cfg::kAtoms);  // k stages = k-groups
-  t.ng = t.ks;
+  // row of the per-row tables (and of the fp16 token rows): routed rows, then the T shared rows
+  t.b_row = t.sh ? 6 * args.T + t.n0 : __ldcg(args.ebase + t.e) + t.n0;
+  t.ng = (kMode == 1 ? kH : (t.sh ? kIs : kI)) / kG;  // 128-wide k-groups
   if (kMode == 1) {  // weight rows: gate (tile rows 2i) / up (2i+1)
     t.row0 = t.sh ? 64 * t.mt : t.e * 2 * kI + 64 * t.mt;
     t.row1 = t.sh ? kIs + 64 * t.mt : t.e * 2 * kI + kI + 64 * t.mt;
@@ -468,22 +619,21 @@ FLINT_DEV bool pf_tile(const GemmArgs &args, uint32_t idx, PfTile<kMode> &t) {
 }
 
 // Persistent: CTA c takes tiles c, c + grid, ...  Every role walks the same
-// tile sequence; the stage ring and the two TMEM accumulator buffers carry
-// on across tiles (running counters it, gc), so one tile's epilogue and the
-// next tile's loads and MMAs overlap.
+// tile sequence with running counters (it: k-groups, tc: tiles), so the
+// stage ring, the weight tiles in TMEM and the accumulators carry on across
+// tiles and one tile's epilogue overlaps the next tile's MMAs.
 template <int kMode>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     k_pf_gemm(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
               const __grid_constant__ CUtensorMap tmB_r, const __grid_constant__ CUtensorMap tmB_s,
-              const __grid_constant__ CUtensorMap tmB_r_lo,
-              const __grid_constant__ CUtensorMap tmB_s_lo, GemmArgs args) {
+              GemmArgs args) {
   using Cfg = GemmCfg<kMode>;
-  constexpr int S = Cfg::kStages;
+  constexpr int S = Cfg::kS, NA = Cfg::kNA, NACC = Cfg::kAcc, kN = Cfg::kN, kHalf = kN / 2;
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t full[S], afull[S], empty[S], gfull[kTmemBufs],
-      gempty[kTmemBufs];
+  __shared__ __align__(8) uint64_t full[S], empty[S], afull[NA], aempty[NA], accfull[NACC],
+      accempty[NACC], mma_done;
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_fail;
 
@@ -494,13 +644,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&afull[s], kDeqThreads);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < kTmemBufs; ++b) {
-      mbar_init(&gfull[b], 1);
-      mbar_init(&gempty[b], kEpiThreads);
+    for (int a = 0; a < NA; ++a) {
+      mbar_init(&afull[a], 4);  // one arrival per dequant warp
+      mbar_init(&aempty[a], 1);
     }
+    for (int b = 0; b < NACC; ++b) {
+      mbar_init(&accfull[b], 1);
+      mbar_init(&accempty[b], 8);  // one arrival per epilogue warp
+    }
+    mbar_init(&mma_done, 1);
     s_fail = 0;
   }
   if (warp == 1) {
@@ -518,203 +672,211 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegCtl));
     if (warp == 0 && lane == 0) {
-      // ---- producer: int4 codes of the weight tile and the token tile(s), by TMA
+      // ---- producer: int4 codes of the weight tile and the token tile, by TMA
       uint32_t it = 0;
       for (uint32_t ti = blockIdx.x; ti < ntiles && !s_fail; ti += gridDim.x) {
-        PfTile<kMode> t;
+        PfTile t;
         if (!pf_tile<kMode>(args, ti, t)) continue;
         const CUtensorMap *tA = t.sh ? &tmA_s : &tmA_r;
         const CUtensorMap *tB = t.sh ? &tmB_s : &tmB_r;
-        const CUtensorMap *tBl = t.sh ? &tmB_s_lo : &tmB_r_lo;
-        for (int kb = 0; kb < t.ks; ++kb, ++it) {
+        const int brow = (kMode == 2 && t.sh) ? t.n0 : t.b_row;  // GEMM 2's shared B is Hs
+        for (int G = 0; G < t.ng; ++G, ++it) {
           const int s = it % S;
           if (it >= (uint32_t)S && !mbar_wait_sleep(&empty[s], ((it / S) - 1) & 1)) {
             s_fail = 1;
             break;
           }
           unsigned char *st = sm + (size_t)s * Cfg::kStageBytes;
-          unsigned char *raw = st + Cfg::raw_off();
-          mbar_expect_tx(&full[s], Cfg::kAtoms * (kRawBytes + Cfg::kNB * kBBytes));
+          mbar_expect_tx(&full[s], kRawBytes + 2 * Cfg::kBAtom);
           if (kMode == 1) {  // gate rows then up rows, 128 codes (64 B) each
-            tma_load_2d(raw, tA, kb * 64, t.row0, &full[s]);
-            tma_load_2d(raw + 64 * 64, tA, kb * 64, t.row1, &full[s]);
-            tma_load_2d(st + Cfg::b_off(0, 0), tB, kb * 128, t.b_row, &full[s]);
-            tma_load_2d(st + Cfg::b_off(0, 1), tB, kb * 128 + 64, t.b_row, &full[s]);
-          } else {  // 128 rows x 128 codes; hi and lo token atoms
-            tma_load_2d(raw, tA, kb * 64, t.row0, &full[s]);
-            for (int atom = 0; atom < 2; ++atom) {
-              tma_load_2d(st + Cfg::b_off(0, atom), tB, kb * 128 + 64 * atom, t.b_row, &full[s]);
-              tma_load_2d(st + Cfg::b_off(1, atom), tBl, kb * 128 + 64 * atom, t.b_row, &full[s]);
-            }
+            tma_load_2d(st, tA, G * 64, t.row0, &full[s]);
+            tma_load_2d(st + 64 * 64, tA, G * 64, t.row1, &full[s]);
+          } else {  // 128 rows x 128 codes
+            tma_load_2d(st, tA, G * 64, t.row0, &full[s]);
           }
-          if (ti == blockIdx.x) pf_mark(kMode, 0, kb);
+          tma_load_2d(st + kRawBytes, tB, G * 128, brow, &full[s]);
+          tma_load_2d(st + kRawBytes + Cfg::kBAtom, tB, G * 128 + 64, brow, &full[s]);
+          if (ti == blockIdx.x) pf_mark(kMode, 0, G);
         }
       }
     } else if (warp == 1 && lane == 0) {
-      // ---- MMA issuer: group gc accumulates into TMEM buffer gc % kTmemBufs
-      uint32_t it = 0, gc = 0;
+      // ---- MMA issuer: tile tc accumulates into buffer tc % NACC
+      uint32_t it = 0, tc = 0;
       for (uint32_t ti = blockIdx.x; ti < ntiles && !s_fail; ti += gridDim.x) {
-        PfTile<kMode> t;
+        PfTile t;
         if (!pf_tile<kMode>(args, ti, t)) continue;
-        const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) |
-                               ((uint32_t)(t.n_mma >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
-        for (int G = 0; G < t.ng && !s_fail; ++G, ++gc) {
-          const int b = gc % kTmemBufs;
-          if (gc >= kTmemBufs && !mbar_wait(&gempty[b], ((gc / kTmemBufs) - 1) & 1)) {
-            s_fail = 1;
-            break;
-          }
-          if (ti == blockIdx.x) pf_mark(kMode, 5, G);
-          tc_fence_after();
-          const uint32_t d = tmem + (uint32_t)(128 * b);
-          {  // the group's single stage
-            const int s = it % S;
-            const uint32_t ph = (it / S) & 1;
-            // afull implies full: the dequant warps arrive on afull only after
-            // they have waited on full (the stage's TMA bytes) themselves
-            if (!mbar_wait(&afull[s], ph)) {
-              s_fail = 1;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t st_addr = smem_addr(sm + (size_t)s * Cfg::kStageBytes);
-#pragma unroll
-            for (int atom = 0; atom < Cfg::kAtoms; ++atom) {
-              const uint32_t a_addr = st_addr + Cfg::a_off(atom);
-              const uint32_t b_addr = st_addr + Cfg::b_off(0, atom);
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                umma_bf16(d, sw128_desc(a_addr + 32 * k), sw128_desc(b_addr + 32 * k), idesc,
-                          (atom | k) != 0);
-                if (kMode == 2)
-                  umma_bf16(d, sw128_desc(a_addr + 32 * k),
-                            sw128_desc(st_addr + Cfg::b_off(1, atom) + 32 * k), idesc, 1u);
-              }
-            }
-            umma_commit(&empty[s]);    // the stage is free for the producer
-            umma_commit(&gfull[b]);    // group gc is complete in TMEM buffer b
-            if (ti == blockIdx.x) pf_mark(kMode, 2, G);
-            ++it;
-          }
-        }
-      }
-    }  // other lanes and warps 2-3: idle (register donors)
-  } else if (warp < 8) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegDeq));
-    // ---- dequant: thread i owns weight row i of every tile (exact codes)
-    const int i = tid - 128;
-    const int raw_row = kMode == 1 ? ((i & 1) ? 64 + (i >> 1) : (i >> 1)) : i;
-    uint32_t it = 0;
-    for (uint32_t ti = blockIdx.x; ti < ntiles && !s_fail; ti += gridDim.x) {
-      PfTile<kMode> t;
-      if (!pf_tile<kMode>(args, ti, t)) continue;
-      for (int kb = 0; kb < t.ks; ++kb, ++it) {
-        const int s = it % S;
-        if (!mbar_wait_sleep(&full[s], (it / S) & 1)) {
+        const int b = tc % NACC;
+        if (tc >= (uint32_t)NACC && !mbar_wait(&accempty[b], ((tc / NACC) - 1) & 1)) {
           s_fail = 1;
           break;
         }
-        unsigned char *st = sm + (size_t)s * Cfg::kStageBytes;
-        // the row's codes: 32 B per atom; chunk j (32 codes) -> atom j / 2, 16-byte
-        // slots 4 (j % 2) .. +3 of the row, XOR-swizzled by the row (SW128)
-        const unsigned char *raw = st + Cfg::raw_off() + raw_row * (32 * Cfg::kAtoms);
+        tc_fence_after();
+        const uint32_t d = tmem + Cfg::acc_col(b);
+        // kind::f16, A = B = f16, D = f32, K-major, N = n_mma, M = 128
+        const uint32_t idesc =
+            (1u << 4) | ((uint32_t)(t.n_mma >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+        bool ok = true;
+        for (int G = 0; G < t.ng; ++G, ++it) {
+          const int s = it % S, a = it % NA;
+          // afull implies full: the dequant warps arrive only after waiting on full
+          if (!mbar_wait(&afull[a], (it / NA) & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t b_addr = smem_addr(sm + (size_t)s * Cfg::kStageBytes + kRawBytes);
+          const uint32_t a_tm = tmem + Cfg::a_col(a);
 #pragma unroll
-        for (int j = 0; j < 2 * Cfg::kAtoms; ++j) {
-          const uint4 w = *reinterpret_cast<const uint4 *>(raw + 16 * j);
-          uint4 c[4];
-          codes32(w, c);
-          unsigned char *arow = st + Cfg::a_off(j >> 1) + i * 128;
+          for (int atom = 0; atom < 2; ++atom) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            *reinterpret_cast<uint4 *>(arow + ((((j & 1) * 4 + q) ^ (i & 7)) * 16)) = c[q];
+            for (int k = 0; k < 4; ++k)
+              umma_f16_ts(d, a_tm + 8u * (4 * atom + k),
+                          sw128_desc(b_addr + atom * Cfg::kBAtom + 32 * k), idesc,
+                          (G | atom | k) != 0);
+          }
+          umma_commit(&empty[s]);   // the stage's shared memory is free for the producer
+          umma_commit(&aempty[a]);  // the weight tile's TMEM is free for the dequant warps
+          if (ti == blockIdx.x) pf_mark(kMode, 2, G);
         }
-        fence_proxy_async();
-        mbar_arrive(&afull[s]);
-        if (tid == 128 && ti == blockIdx.x) pf_mark(kMode, 1, kb);
+        if (!ok) {
+          s_fail = 1;
+          break;
+        }
+        umma_commit(&accfull[b]);  // the tile's sum is complete in accumulator b
+        ++tc;
       }
-    }
-  } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegEpi));
-    // ---- epilogue warps 8..15: TMEM lane quarter (warp % 4) -> tile rows;
-    // token half (warp - 8) / 4 -> tile columns 64 h .. 64 h + 63
-    const int q4 = warp & 3;
-    const int c_lo = 64 * ((warp - 8) >> 2);
-    const int r = 32 * q4 + lane;
-    uint32_t gc = 0;
+      // every MMA this thread issued completes before the CTA frees tensor memory
+      umma_commit(&mma_done);
+      if (!mbar_wait(&mma_done, 0)) s_fail = 1;
+    }  // other lanes and warps 2-3: idle (register donors)
+  } else if (warp < 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegDeq));
+    // ---- dequant: thread i owns weight row i of every tile, TMEM lane i
+    const int i = tid - 128, q = warp - 4;
+    const int raw_row = kMode == 1 ? ((i & 1) ? 64 + (i >> 1) : (i >> 1)) : i;
+    uint32_t it = 0;
     for (uint32_t ti = blockIdx.x; ti < ntiles && !s_fail; ti += gridDim.x) {
-      PfTile<kMode> t;
+      PfTile t;
       if (!pf_tile<kMode>(args, ti, t)) continue;
-      const int wrow = kMode == 1 ? ((r & 1) ? t.row1 : t.row0) + (r >> 1) : t.row0 + r;
-      const int gpr = kMode == 1 ? kH / kG : (t.sh ? kIs / kG : kI / kG);
-      const uint16_t *srow = (t.sh ? args.sc_s : args.sc_r) + (size_t)wrow * gpr;
-      float acc[64];
+      // the row's bf16 scales for the whole K (16, 8 or 4 groups) and the matrix shift
+      const int wrow = kMode == 1 ? ((i & 1) ? t.row1 : t.row0) + (i >> 1) : t.row0 + i;
+      const int gpr = t.ng;
+      const uint32_t *srow = reinterpret_cast<const uint32_t *>(
+          (t.sh ? args.sc_s : args.sc_r) + (size_t)wrow * gpr);
+      uint32_t scw[8];
 #pragma unroll
-      for (int j = 0; j < 64; ++j) acc[j] = 0.f;
+      for (int w = 0; w < 8; ++w) scw[w] = w < gpr / 2 ? __ldg(srow + w) : 0u;
+      const float4 ws = __ldg(args.wst + t.e);
+      const float smul = kMode == 1 ? ws.x : ws.z;
       bool ok = true;
-      for (int G = 0; G < t.ng; ++G, ++gc) {
-        const int b = gc % kTmemBufs;
-        const float sc = bf16_bits_to_f32(ld_nc_u16(srow + G));
-        if (!mbar_wait_sleep(&gfull[b], (gc / kTmemBufs) & 1)) {
+      for (int G = 0; G < t.ng; ++G, ++it) {
+        const int s = it % S, a = it % NA;
+        if (!mbar_wait_sleep(&full[s], (it / S) & 1) ||
+            (it >= (uint32_t)NA && !mbar_wait_sleep(&aempty[a], ((it / NA) - 1) & 1))) {
           ok = false;
           break;
         }
-        if (tid == 256 && ti == blockIdx.x) pf_mark(kMode, 4, 2 + G);
         tc_fence_after();
-        const uint32_t base = tmem + (uint32_t)(128 * b + c_lo) + ((uint32_t)(32 * q4) << 16);
-        if (c_lo < t.n_mma) {  // the same for the whole warp
-          uint32_t v0[32], v1[32];
-          tmem_ld32_async(base, v0);
-          if (c_lo + 32 < t.n_mma) tmem_ld32_async(base + 32u, v1);
-          tmem_wait_ld();
+        // the group's scale x 2^-S as fp16x2 (exact: 8 significant bits, normal range)
+        const uint32_t sw = scw[G >> 1] >> (16 * (G & 1));
+        const float sf = __uint_as_float(sw << 16) * smul;
+        const uint32_t hs = __half_as_ushort(__float2half_rn(sf));
+        const uint32_t sc2 = hs | (hs << 16);
+        const unsigned char *raw =
+            sm + (size_t)s * Cfg::kStageBytes + raw_row * 64;
+        const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + Cfg::a_col(a);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) acc[j] = fmaf(__uint_as_float(v0[j]), sc, acc[j]);
-          if (c_lo + 32 < t.n_mma) {
+        for (int hf = 0; hf < 2; ++hf) {  // TMEM columns 32 hf .. 32 hf + 31: chunks 2 hf, 2 hf + 1
+          uint32_t v[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              acc[32 + j] = fmaf(__uint_as_float(v1[j]), sc, acc[32 + j]);
+          for (int jj = 0; jj < 2; ++jj) {
+            // chunk j = codes 32 j .. 32 j + 31 of the group -> columns 16 j ..
+            const int j = 2 * hf + jj;
+            const uint4 w = *reinterpret_cast<const uint4 *>(raw + 16 * j);
+            codes8_f16(w.x, sc2, v + 16 * jj + 0);
+            codes8_f16(w.y, sc2, v + 16 * jj + 4);
+            codes8_f16(w.z, sc2, v + 16 * jj + 8);
+            codes8_f16(w.w, sc2, v + 16 * jj + 12);
           }
+          tmem_st32(tbase + 32u * hf, v);
         }
+        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&gempty[b]);
-        if (tid == 256 && ti == blockIdx.x) pf_mark(kMode, 3, G);
-        if (tid == 480 && ti == blockIdx.x) pf_mark(kMode, 3, 20 + G);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&afull[a]);
+        if (tid == 128 && ti == blockIdx.x) pf_mark(kMode, 1, G);
       }
       if (!ok) {
         s_fail = 1;
         break;
       }
-      if (kMode == 1) {
-        const int col = 64 * t.mt + (r >> 1);
-        const size_t ld = t.sh ? kIs : kI;
-        uint16_t *hi = t.sh ? args.out_s + (size_t)t.n0 * kIs + col
-                            : args.out_r + (size_t)t.b_row * kI + col;
-        uint16_t *lo = t.sh ? args.out_s_lo + (size_t)t.n0 * kIs + col
-                            : args.out_r_lo + (size_t)t.b_row * kI + col;
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegEpi));
+    // ---- epilogue warps 8..15: TMEM lane quarter (warp % 4) -> tile rows;
+    // token half (warp - 8) / 4 -> tile columns kHalf h .. kHalf h + kHalf - 1
+    const int q4 = warp & 3;
+    const int c_lo = kHalf * ((warp - 8) >> 2);
+    const int r = 32 * q4 + lane;
+    uint32_t tc = 0;
+    for (uint32_t ti = blockIdx.x; ti < ntiles && !s_fail; ti += gridDim.x) {
+      PfTile t;
+      if (!pf_tile<kMode>(args, ti, t)) continue;
+      const int b = tc % NACC;
+      const float4 ws = __ldg(args.wst + t.e);
+      if (!mbar_wait_sleep(&accfull[b], (tc / NACC) & 1)) {
+        s_fail = 1;
+        break;
+      }
+      tc_fence_after();
+      uint32_t acc[kHalf];
+      if (c_lo < t.n_mma) {  // the same for the whole warp
+        const uint32_t base = tmem + Cfg::acc_col(b) + (uint32_t)c_lo + ((uint32_t)(32 * q4) << 16);
 #pragma unroll
-        for (int jj = 0; jj < 64; ++jj) {
-          const int j = c_lo + jj;
-          const float other = __shfl_xor_sync(0xffffffffu, acc[jj], 1);
-          if (!(r & 1) && j < t.n_valid) {
-            const float hv = acc[jj] / (1.f + expf(-acc[jj])) * other;  // silu(gate) * up
-            uint16_t h16, l16;
-            split_hilo(hv, h16, l16);
-            hi[(size_t)j * ld] = h16;
-            lo[(size_t)j * ld] = l16;
-          }
+        for (int c = 0; c < kHalf / 32; ++c)
+          if (c_lo + 32 * c < t.n_mma) tmem_ld32_async(base + 32u * c, acc + 32 * c);
+        tmem_wait_ld();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&accempty[b]);  // the MMAs of tile tc + NACC may start
+      if (tid == 256 && ti == blockIdx.x) pf_mark(kMode, 3, 0);
+      ++tc;
+      const int nv = t.n_valid - c_lo;  // valid tokens in this half
+      if (nv <= 0) continue;            // the same for the whole warp
+      if (kMode == 1) {
+        // lanes r (gate row) and r + 1 (up row) hold the same column: the gate
+        // lane finishes the first half of the warp's tokens, the up lane the rest
+        const bool up_lane = r & 1;
+        const int col = perm8(64 * t.mt + (r >> 1));
+        uint16_t *hb = t.sh ? args.out_s + (size_t)t.n0 * kIs + col
+                            : args.out_r + (size_t)t.b_row * kI + col;
+        const size_t ld = t.sh ? kIs : kI;
+        const float mw = ws.y;  // 2^S1
+        constexpr int kQ = kHalf / 2;
+#pragma unroll
+        for (int jj = 0; jj < kQ; ++jj) {
+          const float mine = __uint_as_float(up_lane ? acc[kQ + jj] : acc[jj]);
+          const float theirs =
+              __shfl_xor_sync(0xffffffffu, __uint_as_float(up_lane ? acc[jj] : acc[kQ + jj]), 1);
+          const int j = jj + (up_lane ? kQ : 0);
+          const float2 rs = __ldg(args.rsc + t.b_row + c_lo + min(j, nv - 1));
+          const float m = mw * rs.x;
+          const float g = (up_lane ? theirs : mine) * m, uu = (up_lane ? mine : theirs) * m;
+          const float h = __fdividef(g, 1.f + __expf(-g)) * uu * rs.y;  // silu(gate) * up / 2^E
+          const uint16_t hv = __half_as_ushort(__float2half_rn(h));
+          if (j < nv) hb[(size_t)(c_lo + j) * ld] = hv;
         }
       } else {
         const int col = 128 * t.mt + r;
+        const float mw = ws.w;  // 2^S2
+        uint16_t *yb = t.sh ? args.out_s + (size_t)t.n0 * kH + col
+                            : args.out_r + (size_t)t.b_row * kH + col;
 #pragma unroll
-        for (int jj = 0; jj < 64; ++jj) {
-          const int j = c_lo + jj;
-          if (j < t.n_valid) {
-            if (t.sh) {
-              args.out_s[(size_t)(t.n0 + j) * kH + col] = f32_to_bf16_bits(acc[jj]);
-            } else {
-              args.out_r[(size_t)(t.b_row + j) * kH + col] =
-                  f32_to_bf16_bits(acc[jj] * args.pw[t.b_row + j]);
-            }
-          }
+        for (int j = 0; j < kHalf; ++j) {
+          const float m = mw * __ldg(args.rm3 + t.b_row + c_lo + min(j, nv - 1));
+          const uint16_t yv = f32_to_bf16_bits(__uint_as_float(acc[j]) * m);
+          if (j < nv) yb[(size_t)(c_lo + j) * kH] = yv;
         }
       }
     }
@@ -825,11 +987,14 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
   float *pw = reinterpret_cast<float *>(ws + P.pw);
   uint32_t *tiles1 = reinterpret_cast<uint32_t *>(ws + P.tiles1);
   uint32_t *tiles2 = reinterpret_cast<uint32_t *>(ws + P.tiles2);
+  float4 *wst = reinterpret_cast<float4 *>(ws + P.wst);
+  float *wbound = reinterpret_cast<float *>(ws + P.wbound);
+  float2 *xstat = reinterpret_cast<float2 *>(ws + P.xstat);
+  float2 *rsc = reinterpret_cast<float2 *>(ws + P.rsc);
+  float *rm3 = reinterpret_cast<float *>(ws + P.rm3);
   uint16_t *xp = reinterpret_cast<uint16_t *>(ws + P.xp);
-  uint16_t *hr = reinterpret_cast<uint16_t *>(ws + P.hr);          // hi
-  uint16_t *hr_lo = hr + (size_t)P.mr_max * kI;                     // lo
+  uint16_t *hr = reinterpret_cast<uint16_t *>(ws + P.hr);
   uint16_t *hs = reinterpret_cast<uint16_t *>(ws + P.hs);
-  uint16_t *hs_lo = hs + (size_t)T * kIs;
   uint16_t *yw = reinterpret_cast<uint16_t *>(ws + P.yw);
   uint16_t *ys = reinterpret_cast<uint16_t *>(ws + P.ys);
 
@@ -840,30 +1005,30 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
   // 2. stable sort by expert
   note_step("prefill sort launches");
   k_pf_count<<<P.nchunks, 256, 0, st>>>(asc_e, T, cc);
-  k_pf_scan<<<1, 256, 0, st>>>(T, P.nchunks, cc, co, ebase, ecount, perm, tiles1, tiles2, ctrl);
+  k_pf_scan<<<1, 256, 0, st>>>(T, P.nchunks, cc, co, ebase, ecount, tiles1, tiles2, ctrl);
   k_pf_place<<<P.nchunks, 256, 0, st>>>(asc_e, asc_w, T, co, ebase, pos, perm, pw);
-  // 3. gather
+  // 3. power-of-two shifts of the fp16 operands, and the fp16 token rows
+  note_step("prefill operand scaling launches");
+  k_pf_wstats<<<kE + 1, 256, 0, st>>>(L.w13_s, L.w2_s, L.sh13_s, L.sh2_s, wst, wbound);
+  k_pf_xstats<<<(T + 7) / 8, 256, 0, st>>>(x, T, wbound, xstat);
   {
-    int blocks = (int)(((size_t)P.mr_max * (kH / 8) + 255) / 256);
+    int blocks = (int)(((size_t)7 * T * (kH / 8) + 255) / 256);
     if (blocks > 148 * 16) blocks = 148 * 16;
-    k_pf_gather<<<blocks, 256, 0, st>>>(x, perm, ctrl, xp);
+    k_pf_gather<<<blocks, 256, 0, st>>>(x, T, perm, pw, xstat, xp, rsc, rm3);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // 4. tensor maps and the two grouped GEMMs
-  CUtensorMap mA1r, mA1s, mB1r, mB1s, mA2r, mA2s, mB2r, mB2s, mB2rl, mB2sl;
+  CUtensorMap mA1r, mA1s, mB1, mA2r, mA2s, mB2r, mB2s;
   note_step("prefill tensor maps");
-  const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const auto F16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16, U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
   const auto SW = CU_TENSOR_MAP_SWIZZLE_128B, NS = CU_TENSOR_MAP_SWIZZLE_NONE;
   if ((e = make_map(&mA1r, L.w13_q, U8, kH / 2, (uint64_t)kE * 2 * kI, kH / 2, 64, 64, NS)) ||
       (e = make_map(&mA1s, L.sh13_q, U8, kH / 2, 2 * kIs, kH / 2, 64, 64, NS)) ||
-      (e = make_map(&mB1r, xp, BF, kH, (uint64_t)P.mr_max, kH * 2, 64, kPfTile, SW)) ||
-      (e = make_map(&mB1s, x, BF, kH, (uint64_t)T, kH * 2, 64, kPfTile, SW)) ||
+      (e = make_map(&mB1, xp, F16, kH, (uint64_t)7 * T, kH * 2, 64, kPfN1, SW)) ||
       (e = make_map(&mA2r, L.w2_q, U8, kI / 2, (uint64_t)kE * kH, kI / 2, 64, 128, NS)) ||
       (e = make_map(&mA2s, L.sh2_q, U8, kIs / 2, kH, kIs / 2, 64, 128, NS)) ||
-      (e = make_map(&mB2r, hr, BF, kI, (uint64_t)P.mr_max, kI * 2, 64, kPfTile, SW)) ||
-      (e = make_map(&mB2rl, hr_lo, BF, kI, (uint64_t)P.mr_max, kI * 2, 64, kPfTile, SW)) ||
-      (e = make_map(&mB2s, hs, BF, kIs, (uint64_t)T, kIs * 2, 64, kPfTile, SW)) ||
-      (e = make_map(&mB2sl, hs_lo, BF, kIs, (uint64_t)T, kIs * 2, 64, kPfTile, SW)))
+      (e = make_map(&mB2r, hr, F16, kI, (uint64_t)P.mr, kI * 2, 64, kPfN2, SW)) ||
+      (e = make_map(&mB2s, hs, F16, kIs, (uint64_t)T, kIs * 2, 64, kPfN2, SW)))
     return e;
   note_step("prefill GEMM attributes");
   if ((e = cudaFuncSetAttribute(k_pf_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -876,17 +1041,15 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (sms < 1) sms = 1;
-  GemmArgs a1{tiles1, ctrl, 3,  ebase, ecount, T,       L.w13_s, L.sh13_s,
-              hr,     hr_lo, hs, hs_lo, nullptr, ctrl + 1};
+  GemmArgs a1{tiles1, ctrl, 3, ebase, ecount, T, L.w13_s, L.sh13_s, wst, rsc, rm3, hr, hs, ctrl + 1};
   note_step("prefill GEMM 1 launch");
-  k_pf_gemm<1><<<min(P.max_tiles1, sms), kGemmThreads, GemmCfg<1>::kSmem, st>>>(
-      mA1r, mA1s, mB1r, mB1s, mB1r, mB1s, a1);
+  k_pf_gemm<1><<<min(P.max_tiles1, sms), kGemmThreads, GemmCfg<1>::kSmem, st>>>(mA1r, mA1s, mB1,
+                                                                                mB1, a1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  GemmArgs a2{tiles2, ctrl, 4, ebase, ecount, T, L.w2_s, L.sh2_s, yw, nullptr, ys, nullptr, pw,
-              ctrl + 1};
+  GemmArgs a2{tiles2, ctrl, 4, ebase, ecount, T, L.w2_s, L.sh2_s, wst, rsc, rm3, yw, ys, ctrl + 1};
   note_step("prefill GEMM 2 launch");
-  k_pf_gemm<2><<<min(P.max_tiles2, sms), kGemmThreads, GemmCfg<2>::kSmem, st>>>(
-      mA2r, mA2s, mB2r, mB2s, mB2rl, mB2sl, a2);
+  k_pf_gemm<2><<<min(P.max_tiles2, sms), kGemmThreads, GemmCfg<2>::kSmem, st>>>(mA2r, mA2s, mB2r,
+                                                                                mB2s, a2);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // 5. combine
   note_step("prefill combine launch");
