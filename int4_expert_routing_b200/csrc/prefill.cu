@@ -436,28 +436,34 @@ __global__ void __launch_bounds__(256)
 // both operands hold the order 0,4,1,5,2,6,3,7 (the order int4 unpacking
 // yields two codes per 32-bit word); the dot products do not depend on it.
 constexpr int kRawBytes = 128 * 64;  // 128 weight rows x 128 int4 codes: one k-group
-// Four warpgroups: 0 = producer (warp 0), MMA issuer (warp 1) and two idle
-// warps; 1 = four dequant warps (one weight row per thread); 2-3 = eight
-// epilogue warps (two per TMEM lane quarter, one per half of the tile's
-// tokens).  The block is launched at 128 registers per thread (65,536);
+// Four warpgroups: 0 = token-tile producer (warp 0), MMA issuer (warp 1),
+// int4-code producer (warp 2) and an idle warp; 1 = four dequant warps (one
+// weight row per thread); 2-3 = eight epilogue warps (two per TMEM lane
+// quarter, one per half of the tile's tokens).  The block is launched at 128 registers per thread (65,536);
 // setmaxnreg moves them: 128 x 40 + 128 x 88 + 256 x 184 = 63,488.
 constexpr int kGemmThreads = 512;
+constexpr int kEpiThreads = 256;
 constexpr int kRegCtl = 40, kRegDeq = 88, kRegEpi = 184;
 static_assert(128 * kRegCtl + 128 * kRegDeq + 256 * kRegEpi <= 65536, "register split");
 constexpr int kTmemCols = 512;
 
 // kN tokens per tile, kAcc accumulators of kN columns, kNA weight tiles of 64
-// columns (128 fp16 k values per row), kS shared-memory stages (int4 codes and
-// the token tile of one 128-wide k-group each).
+// columns (128 fp16 k values per row) in TMEM; two rings in shared memory, one
+// 128-wide k-group per stage: kS token tiles (freed when the MMAs that read
+// them complete) and kR int4-code tiles (freed once the dequant warps have
+// read them, so the codes run ahead of the MMAs).
 template <int kMode>
 struct GemmCfg {
   static constexpr int kN = kMode == 1 ? kPfN1 : kPfN2;
   static constexpr int kAcc = kMode == 1 ? 1 : 2;
   static constexpr int kNA = kMode == 1 ? 4 : 2;
-  static constexpr int kS = 3;
+  static constexpr int kS = kMode == 1 ? 3 : 4;
+  static constexpr int kR = 3;
   static constexpr int kBAtom = kN * 128;  // kN token rows x 64 fp16
-  static constexpr int kStageBytes = kRawBytes + 2 * kBAtom;
-  static constexpr size_t kSmem = (size_t)kS * kStageBytes + 1024;
+  static constexpr int kBStage = 2 * kBAtom;
+  static constexpr size_t kSmem = (size_t)kS * kBStage + (size_t)kR * kRawBytes + 1024;
+  static constexpr size_t b_off(int s) { return (size_t)s * kBStage; }
+  static constexpr size_t raw_off(int r) { return (size_t)kS * kBStage + (size_t)r * kRawBytes; }
   // TMEM columns: GEMM 1: accumulator 0..255, weight tiles 256, 320, 384, 448;
   // GEMM 2: accumulators at 0 and 256 (192 columns each), weight tiles 192, 448
   static constexpr uint32_t acc_col(int b) { return (uint32_t)(256 * b); }
@@ -567,6 +573,11 @@ FLINT_DEV void tmem_st32(uint32_t taddr, const uint32_t *v) {
 }
 FLINT_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// barrier `id` over the first `n` threads that reach it (a subset of warps)
+FLINT_DEV void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 FLINT_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 FLINT_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -581,6 +592,12 @@ FLINT_DEV void codes8_f16(uint32_t w, uint32_t sc2, uint32_t *out) {
     asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(c) : "r"(t), "r"(0x64086408u));
     asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(out[p]) : "r"(c), "r"(sc2));
   }
+}
+
+// 16-bit global store, skipped when `pred` is false (no branch)
+FLINT_DEV void st_u16_if(uint16_t *p, uint32_t v, bool pred) {
+  asm volatile("{ .reg .pred q; setp.ne.b32 q, %2, 0; @q st.global.b16 [%0], %1; }" ::"l"(p),
+               "h"((unsigned short)v), "r"((int)pred));
 }
 
 // position of natural column c inside its 8-wide block: 0,4,1,5,2,6,3,7 order
@@ -628,14 +645,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               const __grid_constant__ CUtensorMap tmB_r, const __grid_constant__ CUtensorMap tmB_s,
               GemmArgs args) {
   using Cfg = GemmCfg<kMode>;
-  constexpr int S = Cfg::kS, NA = Cfg::kNA, NACC = Cfg::kAcc, kN = Cfg::kN, kHalf = kN / 2;
+  constexpr int S = Cfg::kS, R = Cfg::kR, NA = Cfg::kNA, NACC = Cfg::kAcc, kN = Cfg::kN;
+  constexpr int kHalf = kN / 2;
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t full[S], empty[S], afull[NA], aempty[NA], accfull[NACC],
-      accempty[NACC], mma_done;
+  __shared__ __align__(8) uint64_t full[S], empty[S], rfull[R], rempty[R], afull[NA], aempty[NA],
+      accfull[NACC], accempty[NACC], mma_done;
   __shared__ uint32_t s_tmem;
-  __shared__ volatile int s_fail;
+  __shared__ volatile int s_fail, s_epi_fail;
+  __shared__ float2 s_mul[kN];  // per token of the tile: (2^F, 2^-E) or (2^E x weight, -)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t ntiles = __ldcg(args.ctrl + args.count_word);
@@ -645,6 +664,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+    }
+    for (int r = 0; r < R; ++r) {
+      mbar_init(&rfull[r], 1);
+      mbar_init(&rempty[r], 4);  // one arrival per dequant warp
     }
     for (int a = 0; a < NA; ++a) {
       mbar_init(&afull[a], 4);  // one arrival per dequant warp
@@ -656,6 +679,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     mbar_init(&mma_done, 1);
     s_fail = 0;
+    s_epi_fail = 0;
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -672,12 +696,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegCtl));
     if (warp == 0 && lane == 0) {
-      // ---- producer: int4 codes of the weight tile and the token tile, by TMA
+      // ---- token-tile producer, by TMA
       uint32_t it = 0;
       for (uint32_t ti = blockIdx.x; ti < ntiles && !s_fail; ti += gridDim.x) {
         PfTile t;
         if (!pf_tile<kMode>(args, ti, t)) continue;
-        const CUtensorMap *tA = t.sh ? &tmA_s : &tmA_r;
         const CUtensorMap *tB = t.sh ? &tmB_s : &tmB_r;
         const int brow = (kMode == 2 && t.sh) ? t.n0 : t.b_row;  // GEMM 2's shared B is Hs
         for (int G = 0; G < t.ng; ++G, ++it) {
@@ -686,17 +709,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             s_fail = 1;
             break;
           }
-          unsigned char *st = sm + (size_t)s * Cfg::kStageBytes;
-          mbar_expect_tx(&full[s], kRawBytes + 2 * Cfg::kBAtom);
-          if (kMode == 1) {  // gate rows then up rows, 128 codes (64 B) each
-            tma_load_2d(st, tA, G * 64, t.row0, &full[s]);
-            tma_load_2d(st + 64 * 64, tA, G * 64, t.row1, &full[s]);
-          } else {  // 128 rows x 128 codes
-            tma_load_2d(st, tA, G * 64, t.row0, &full[s]);
-          }
-          tma_load_2d(st + kRawBytes, tB, G * 128, brow, &full[s]);
-          tma_load_2d(st + kRawBytes + Cfg::kBAtom, tB, G * 128 + 64, brow, &full[s]);
+          unsigned char *st = sm + Cfg::b_off(s);
+          mbar_expect_tx(&full[s], Cfg::kBStage);
+          tma_load_2d(st, tB, G * 128, brow, &full[s]);
+          tma_load_2d(st + Cfg::kBAtom, tB, G * 128 + 64, brow, &full[s]);
           if (ti == blockIdx.x) pf_mark(kMode, 0, G);
+        }
+      }
+    } else if (warp == 2 && lane == 0) {
+      // ---- int4-code producer, by TMA
+      uint32_t it = 0;
+      for (uint32_t ti = blockIdx.x; ti < ntiles && !s_fail; ti += gridDim.x) {
+        PfTile t;
+        if (!pf_tile<kMode>(args, ti, t)) continue;
+        const CUtensorMap *tA = t.sh ? &tmA_s : &tmA_r;
+        for (int G = 0; G < t.ng; ++G, ++it) {
+          const int r = it % R;
+          if (it >= (uint32_t)R && !mbar_wait_sleep(&rempty[r], ((it / R) - 1) & 1)) {
+            s_fail = 1;
+            break;
+          }
+          unsigned char *rw = sm + Cfg::raw_off(r);
+          mbar_expect_tx(&rfull[r], kRawBytes);
+          if (kMode == 1) {  // gate rows then up rows, 128 codes (64 B) each
+            tma_load_2d(rw, tA, G * 64, t.row0, &rfull[r]);
+            tma_load_2d(rw + 64 * 64, tA, G * 64, t.row1, &rfull[r]);
+          } else {  // 128 rows x 128 codes
+            tma_load_2d(rw, tA, G * 64, t.row0, &rfull[r]);
+          }
         }
       }
     } else if (warp == 1 && lane == 0) {
@@ -718,13 +758,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         bool ok = true;
         for (int G = 0; G < t.ng; ++G, ++it) {
           const int s = it % S, a = it % NA;
-          // afull implies full: the dequant warps arrive only after waiting on full
-          if (!mbar_wait(&afull[a], (it / NA) & 1)) {
+          if (!mbar_wait(&afull[a], (it / NA) & 1) || !mbar_wait(&full[s], (it / S) & 1)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t b_addr = smem_addr(sm + (size_t)s * Cfg::kStageBytes + kRawBytes);
+          const uint32_t b_addr = smem_addr(sm + Cfg::b_off(s));
           const uint32_t a_tm = tmem + Cfg::a_col(a);
 #pragma unroll
           for (int atom = 0; atom < 2; ++atom) {
@@ -748,7 +787,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // every MMA this thread issued completes before the CTA frees tensor memory
       umma_commit(&mma_done);
       if (!mbar_wait(&mma_done, 0)) s_fail = 1;
-    }  // other lanes and warps 2-3: idle (register donors)
+    }  // other lanes and warp 3: idle (register donors)
   } else if (warp < 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegDeq));
     // ---- dequant: thread i owns weight row i of every tile, TMEM lane i
@@ -770,8 +809,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const float smul = kMode == 1 ? ws.x : ws.z;
       bool ok = true;
       for (int G = 0; G < t.ng; ++G, ++it) {
-        const int s = it % S, a = it % NA;
-        if (!mbar_wait_sleep(&full[s], (it / S) & 1) ||
+        const int rr = it % R, a = it % NA;
+        if (!mbar_wait_sleep(&rfull[rr], (it / R) & 1) ||
             (it >= (uint32_t)NA && !mbar_wait_sleep(&aempty[a], ((it / NA) - 1) & 1))) {
           ok = false;
           break;
@@ -782,8 +821,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const float sf = __uint_as_float(sw << 16) * smul;
         const uint32_t hs = __half_as_ushort(__float2half_rn(sf));
         const uint32_t sc2 = hs | (hs << 16);
-        const unsigned char *raw =
-            sm + (size_t)s * Cfg::kStageBytes + raw_row * 64;
+        const unsigned char *raw = sm + Cfg::raw_off(rr) + raw_row * 64;
         const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + Cfg::a_col(a);
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {  // TMEM columns 32 hf .. 32 hf + 31: chunks 2 hf, 2 hf + 1
@@ -803,7 +841,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&afull[a]);
+        if (lane == 0) {
+          mbar_arrive(&rempty[rr]);  // the codes are in registers and TMEM
+          mbar_arrive(&afull[a]);
+        }
         if (tid == 128 && ti == blockIdx.x) pf_mark(kMode, 1, G);
       }
       if (!ok) {
@@ -818,19 +859,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int q4 = warp & 3;
     const int c_lo = kHalf * ((warp - 8) >> 2);
     const int r = 32 * q4 + lane;
+    // The tile's per-token multipliers pass through shared memory (thread
+    // tid - 256 fetches token tid - 256 before the accumulator is ready);
+    // two barriers of the 256 epilogue threads per tile guard the array, and
+    // the loop ends on a flag only these threads write before the second, so
+    // all eight warps leave in the same iteration.
+    const int et = tid - 256;
     uint32_t tc = 0;
-    for (uint32_t ti = blockIdx.x; ti < ntiles && !s_fail; ti += gridDim.x) {
+    for (uint32_t ti = blockIdx.x; ti < ntiles; ti += gridDim.x) {
       PfTile t;
       if (!pf_tile<kMode>(args, ti, t)) continue;
       const int b = tc % NACC;
       const float4 ws = __ldg(args.wst + t.e);
-      if (!mbar_wait_sleep(&accfull[b], (tc / NACC) & 1)) {
-        s_fail = 1;
-        break;
+      float2 pre = make_float2(0.f, 0.f);
+      if (et < t.n_valid) {
+        if (kMode == 1) pre = __ldg(args.rsc + t.b_row + et);
+        else pre.x = __ldg(args.rm3 + t.b_row + et);
       }
+      const bool ok = mbar_wait_sleep(&accfull[b], (tc / NACC) & 1);
       tc_fence_after();
       uint32_t acc[kHalf];
-      if (c_lo < t.n_mma) {  // the same for the whole warp
+      if (ok && c_lo < t.n_mma) {  // the same for the whole warp
         const uint32_t base = tmem + Cfg::acc_col(b) + (uint32_t)c_lo + ((uint32_t)(32 * q4) << 16);
 #pragma unroll
         for (int c = 0; c < kHalf / 32; ++c)
@@ -839,9 +888,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&accempty[b]);  // the MMAs of tile tc + NACC may start
+      if (lane == 0 && ok) mbar_arrive(&accempty[b]);  // the MMAs of tile tc + NACC may start
       if (tid == 256 && ti == blockIdx.x) pf_mark(kMode, 3, 0);
       ++tc;
+      named_bar_sync(1, kEpiThreads);  // every warp is done with the previous tile's multipliers
+      if (!ok) s_epi_fail = 1;
+      if (et < kN) s_mul[et] = pre;
+      named_bar_sync(1, kEpiThreads);
+      if (s_epi_fail) {
+        s_fail = 1;
+        break;
+      }
       const int nv = t.n_valid - c_lo;  // valid tokens in this half
       if (nv <= 0) continue;            // the same for the whole warp
       if (kMode == 1) {
@@ -854,18 +911,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const size_t ld = t.sh ? kIs : kI;
         const float mw = ws.y;  // 2^S1
         constexpr int kQ = kHalf / 2;
+        const int j0 = up_lane ? kQ : 0;
+        // branch-free arithmetic first (the tokens overlap), then predicated stores
+        constexpr int kC = 16;  // tokens per pass (bounds the live registers)
 #pragma unroll
-        for (int jj = 0; jj < kQ; ++jj) {
-          const float mine = __uint_as_float(up_lane ? acc[kQ + jj] : acc[jj]);
-          const float theirs =
-              __shfl_xor_sync(0xffffffffu, __uint_as_float(up_lane ? acc[jj] : acc[kQ + jj]), 1);
-          const int j = jj + (up_lane ? kQ : 0);
-          const float2 rs = __ldg(args.rsc + t.b_row + c_lo + min(j, nv - 1));
-          const float m = mw * rs.x;
-          const float g = (up_lane ? theirs : mine) * m, uu = (up_lane ? mine : theirs) * m;
-          const float h = __fdividef(g, 1.f + __expf(-g)) * uu * rs.y;  // silu(gate) * up / 2^E
-          const uint16_t hv = __half_as_ushort(__float2half_rn(h));
-          if (j < nv) hb[(size_t)(c_lo + j) * ld] = hv;
+        for (int c0 = 0; c0 < kQ; c0 += kC) {
+          uint32_t hp[kC / 2];
+#pragma unroll
+          for (int u = 0; u < kC; ++u) {
+            const int jj = c0 + u;
+            const float mine = __uint_as_float(up_lane ? acc[kQ + jj] : acc[jj]);
+            const float theirs =
+                __shfl_xor_sync(0xffffffffu, __uint_as_float(up_lane ? acc[jj] : acc[kQ + jj]), 1);
+            const float2 rs = s_mul[c_lo + j0 + jj];
+            const float m = mw * rs.x;
+            const float g = (up_lane ? theirs : mine) * m, uu = (up_lane ? mine : theirs) * m;
+            const float h = __fdividef(g, 1.f + __expf(-g)) * uu * rs.y;  // silu(gate) * up / 2^E
+            const uint32_t hv = __half_as_ushort(__float2half_rn(h));
+            hp[u >> 1] = (u & 1) ? (hp[u >> 1] | (hv << 16)) : hv;
+          }
+#pragma unroll
+          for (int u = 0; u < kC; ++u) {
+            const int jj = c0 + u;
+            st_u16_if(hb + (size_t)(c_lo + j0 + jj) * ld, hp[u >> 1] >> (16 * (u & 1)), j0 + jj < nv);
+          }
         }
       } else {
         const int col = 128 * t.mt + r;
@@ -874,9 +943,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             : args.out_r + (size_t)t.b_row * kH + col;
 #pragma unroll
         for (int j = 0; j < kHalf; ++j) {
-          const float m = mw * __ldg(args.rm3 + t.b_row + c_lo + min(j, nv - 1));
-          const uint16_t yv = f32_to_bf16_bits(__uint_as_float(acc[j]) * m);
-          if (j < nv) yb[(size_t)(c_lo + j) * kH] = yv;
+          const float m = mw * s_mul[c_lo + j].x;
+          st_u16_if(yb + (size_t)(c_lo + j) * kH, f32_to_bf16_bits(__uint_as_float(acc[j]) * m), j < nv);
         }
       }
     }
