@@ -62,8 +62,9 @@ inline PrefillLayout prefill_layout(int T) {
   // at most min(256, 6T) experts hold tokens; each adds at most one partial tile
   const int busy = 6 * T < 256 ? 6 * T : 256;
   L.mr = 6 * T;
-  L.max_tiles1 = 8 * ((6 * T) / kPfN1 + busy) + 16 * ((T + kPfN1 - 1) / kPfN1);
-  L.max_tiles2 = 16 * ((6 * T) / kPfN2 + busy) + 16 * ((T + kPfN2 - 1) / kPfN2);
+  // tiles of 256 weight rows (a CTA pair) by one token tile
+  L.max_tiles1 = 4 * ((6 * T) / kPfN1 + busy) + 8 * ((T + kPfN1 - 1) / kPfN1);
+  L.max_tiles2 = 8 * ((6 * T) / kPfN2 + busy) + 8 * ((T + kPfN2 - 1) / kPfN2);
   size_t o = 0;
   auto take = [&](size_t bytes) {
     size_t at = o;

@@ -213,8 +213,9 @@ FLINT_DEV uint32_t pack_tile(int e, int mt, int nt) {
 }
 
 // One CTA of 256 threads (one per expert): chunk offsets, expert counts,
-// group bases (no padding) and both GEMM tile lists (the 8 or 16 row tiles of
-// one token tile are adjacent, so the token tile is reused from L2).
+// group bases (no padding) and both GEMM tile lists.  A tile is 256 weight
+// rows (two 128-row tiles, one per CTA of a pair) by one token tile; the 4 or
+// 8 tiles of one token tile are adjacent, so the token tile is reused from L2.
 __global__ void __launch_bounds__(256)
     k_pf_scan(int T, int nchunks, const int32_t *__restrict__ chunk_cnt,
               int32_t *__restrict__ chunk_off, int32_t *__restrict__ ebase,
@@ -232,21 +233,21 @@ __global__ void __launch_bounds__(256)
   const int nt1 = (off + kPfN1 - 1) / kPfN1, nt2 = (off + kPfN2 - 1) / kPfN2;
   int total_rows, total1, total2;
   const int base = block_scan(off, s_warp, &total_rows);
-  const int o1 = block_scan(8 * nt1, s_warp, &total1);
-  const int o2 = block_scan(16 * nt2, s_warp, &total2);
+  const int o1 = block_scan(4 * nt1, s_warp, &total1);
+  const int o2 = block_scan(8 * nt2, s_warp, &total2);
   ebase[e] = base;
   if (e == 0) ebase[kE] = total_rows;
   for (int nt = 0; nt < nt1; ++nt)
-    for (int mt = 0; mt < 8; ++mt) tiles1[o1 + nt * 8 + mt] = pack_tile(e, mt, nt);
+    for (int mp = 0; mp < 4; ++mp) tiles1[o1 + nt * 4 + mp] = pack_tile(e, mp, nt);
   for (int nt = 0; nt < nt2; ++nt)
-    for (int mt = 0; mt < 16; ++mt) tiles2[o2 + nt * 16 + mt] = pack_tile(e, mt, nt);
+    for (int mp = 0; mp < 8; ++mp) tiles2[o2 + nt * 8 + mp] = pack_tile(e, mp, nt);
   // the shared expert: one group over all T tokens
   const int nsh1 = (T + kPfN1 - 1) / kPfN1, nsh2 = (T + kPfN2 - 1) / kPfN2;
-  for (int i = e; i < 16 * nsh1; i += kE) tiles1[total1 + i] = pack_tile(kE, i & 15, i >> 4);
-  for (int i = e; i < 16 * nsh2; i += kE) tiles2[total2 + i] = pack_tile(kE, i & 15, i >> 4);
+  for (int i = e; i < 8 * nsh1; i += kE) tiles1[total1 + i] = pack_tile(kE, i & 7, i >> 3);
+  for (int i = e; i < 8 * nsh2; i += kE) tiles2[total2 + i] = pack_tile(kE, i & 7, i >> 3);
   if (e == 0) {
-    ctrl[3] = (uint32_t)(total1 + 16 * nsh1);
-    ctrl[4] = (uint32_t)(total2 + 16 * nsh2);
+    ctrl[3] = (uint32_t)(total1 + 8 * nsh1);
+    ctrl[4] = (uint32_t)(total2 + 8 * nsh2);
     ctrl[5] = (uint32_t)total_rows;
   }
 }
@@ -436,10 +437,17 @@ __global__ void __launch_bounds__(256)
 // both operands hold the order 0,4,1,5,2,6,3,7 (the order int4 unpacking
 // yields two codes per 32-bit word); the dot products do not depend on it.
 constexpr int kRawBytes = 128 * 64;  // 128 weight rows x 128 int4 codes: one k-group
-// Four warpgroups: 0 = token-tile producer (warp 0), MMA issuer (warp 1),
-// int4-code producer (warp 2) and an idle warp; 1 = four dequant warps (one
-// weight row per thread); 2-3 = eight epilogue warps (two per TMEM lane
-// quarter, one per half of the tile's tokens).  The block is launched at 128 registers per thread (65,536);
+// A pair of CTAs (a cluster of two on neighbouring SMs) computes one tile of
+// 256 weight rows: each CTA dequantizes its 128 rows into its own tensor
+// memory and loads half of the token tile into its shared memory; one thread
+// of the first CTA issues tcgen05.mma.cta_group::2, which reads A from both
+// CTAs' tensor memory and B from both CTAs' shared memory, and writes each
+// CTA's 128 accumulator rows into that CTA's tensor memory.  Every token byte
+// thus crosses L2 -> SM once per 256 weight rows.
+// Four warpgroups per CTA: 0 = token-tile producer (warp 0), MMA issuer
+// (warp 1, first CTA), int4-code producer (warp 2) and an idle warp; 1 = four
+// dequant warps (one weight row per thread); 2-3 = eight epilogue warps (two
+// per TMEM lane quarter, one per half of the tile's tokens).  The block is launched at 128 registers per thread (65,536);
 // setmaxnreg moves them: 128 x 40 + 128 x 88 + 256 x 184 = 63,488.
 constexpr int kGemmThreads = 512;
 constexpr int kEpiThreads = 256;
@@ -449,17 +457,18 @@ constexpr int kTmemCols = 512;
 
 // kN tokens per tile, kAcc accumulators of kN columns, kNA weight tiles of 64
 // columns (128 fp16 k values per row) in TMEM; two rings in shared memory, one
-// 128-wide k-group per stage: kS token tiles (freed when the MMAs that read
-// them complete) and kR int4-code tiles (freed once the dequant warps have
-// read them, so the codes run ahead of the MMAs).
+// 128-wide k-group per stage: kS half token tiles (freed when the MMAs that
+// read them complete) and kR int4-code tiles (freed once the dequant warps
+// have read them, so the codes run ahead of the MMAs).
 template <int kMode>
 struct GemmCfg {
   static constexpr int kN = kMode == 1 ? kPfN1 : kPfN2;
   static constexpr int kAcc = kMode == 1 ? 1 : 2;
   static constexpr int kNA = kMode == 1 ? 4 : 2;
-  static constexpr int kS = kMode == 1 ? 3 : 4;
+  static constexpr int kS = kMode == 1 ? 6 : 8;
   static constexpr int kR = 3;
-  static constexpr int kBAtom = kN * 128;  // kN token rows x 64 fp16
+  static constexpr int kBRows = kN / 2;       // token rows per CTA (the TMA box height)
+  static constexpr int kBAtom = kBRows * 128;  // kN / 2 token rows x 64 fp16
   static constexpr int kBStage = 2 * kBAtom;
   static constexpr size_t kSmem = (size_t)kS * kBStage + (size_t)kR * kRawBytes + 1024;
   static constexpr size_t b_off(int s) { return (size_t)s * kBStage; }
@@ -505,19 +514,86 @@ FLINT_DEV void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint
       : "memory");
 }
 
-// D (TMEM) += A (TMEM, 128 lanes x 8 columns of fp16 pairs) x B (shared memory)
-FLINT_DEV void umma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
-                           uint32_t accum) {
+// D (TMEM) += A (TMEM, 128 lanes x 8 columns of fp16 pairs) x B (shared memory),
+// the same, issued for the CTA pair (M = 256: A rows 0..127 in the first
+// CTA's TMEM lanes, 128..255 in the second's; B rows split in halves between
+// the two CTAs' shared memory at the same offset)
+FLINT_DEV void umma_f16_ts_pair(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                uint32_t accum) {
   asm volatile(
-      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, "
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, "
       "%3, p;\n}\n" ::"r"(tmem_d),
       "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accum));
 }
 
-FLINT_DEV void umma_commit(uint64_t *bar) {
+// arrive on `bar` (same offset) in both CTAs of the pair once the pair's
+// earlier MMAs have completed
+FLINT_DEV void umma_commit_pair(uint64_t *bar) {
   asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          smem_addr(bar))
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
+      "[%0], %1;" ::"r"(smem_addr(bar)),
+      "h"((unsigned short)3)
+      : "memory");
+}
+
+FLINT_DEV uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of `p` (this CTA's shared memory) in CTA `rank`
+FLINT_DEV uint32_t cluster_addr(const void *p, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_addr(p)), "r"(rank));
+  return a;
+}
+FLINT_DEV void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" :::
+                   "memory");
+}
+// arrive on an mbarrier of either CTA of the pair (a shared::cluster address),
+// with the default CTA-scope release: what it orders for the other CTA is
+// tensor-memory or shared-memory state that this CTA's own tensor core or TMA
+// reads, completed before the arrival (tcgen05.wait + tcgen05.fence); a
+// cluster-scope release would also wait for this thread's global stores
+FLINT_DEV void mbar_arrive_cluster(uint32_t cl_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
+}
+// bounded waits with cluster-scope acquire (the arrivals come from the other
+// CTA of the pair or from its MMAs); the second form may suspend the thread
+FLINT_DEV bool cwait(uint64_t *bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kWaitPolls; ++i) {
+    uint32_t done;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2; "
+        "selp.u32 %0, 1, 0, p; }"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+FLINT_DEV bool cwait_sleep(uint64_t *bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kSleepPolls; ++i) {
+    uint32_t done;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3; "
+        "selp.u32 %0, 1, 0, p; }"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(20000u)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+// TMA tile load into this CTA's shared memory whose completion is counted on
+// an mbarrier of either CTA of the pair (`bar_cl`, a shared::cluster address)
+FLINT_DEV void tma_load_2d_pair(void *dst, const CUtensorMap *map, int x, int y, uint32_t bar_cl) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cl)
       : "memory");
 }
 
@@ -610,18 +686,19 @@ struct PfTile {
   int e, mt, n0, n_valid, n_mma, b_row, row0, row1, ng;
   bool sh;
 };
+// mt is this CTA's 128-row tile: 2 x (the pair's tile) + the CTA's rank
 template <int kMode>
-FLINT_DEV bool pf_tile(const GemmArgs &args, uint32_t idx, PfTile &t) {
+FLINT_DEV bool pf_tile(const GemmArgs &args, uint32_t idx, uint32_t rank, PfTile &t) {
   constexpr int kN = GemmCfg<kMode>::kN;
   const uint32_t packed = __ldcg(args.tiles + idx);
   t.e = (int)(packed & 511u);
-  t.mt = (int)((packed >> 9) & 31u);
+  t.mt = 2 * (int)((packed >> 9) & 31u) + (int)rank;
   const int nt = (int)(packed >> 14);
   t.sh = t.e == kE;
   t.n0 = nt * kN;
   t.n_valid = min(kN, (t.sh ? args.T : __ldcg(args.ecount + t.e)) - t.n0);
   if (t.n_valid <= 0) return false;  // not produced by the scan; guards against an N = 0 MMA
-  t.n_mma = (t.n_valid + 15) & ~15;
+  t.n_mma = (t.n_valid + 31) & ~31;  // the pair MMA takes N in steps of 32
   // row of the per-row tables (and of the fp16 token rows): routed rows, then the T shared rows
   t.b_row = t.sh ? 6 * args.T + t.n0 : __ldcg(args.ebase + t.e) + t.n0;
   t.ng = (kMode == 1 ? kH : (t.sh ? kIs : kI)) / kG;  // 128-wide k-groups
@@ -635,12 +712,14 @@ FLINT_DEV bool pf_tile(const GemmArgs &args, uint32_t idx, PfTile &t) {
   return true;
 }
 
-// Persistent: CTA c takes tiles c, c + grid, ...  Every role walks the same
-// tile sequence with running counters (it: k-groups, tc: tiles), so the
-// stage ring, the weight tiles in TMEM and the accumulators carry on across
-// tiles and one tile's epilogue overlaps the next tile's MMAs.
+// Persistent: pair c takes tiles c, c + pairs, ...  Every role of both CTAs
+// walks the same tile sequence with running counters (it: k-groups, tc:
+// tiles), so the stage rings, the weight tiles in TMEM and the accumulators
+// carry on across tiles and one tile's epilogue overlaps the next tile's MMAs.
+// Barriers that gather both CTAs (full, afull, accempty) live in the first
+// CTA; the MMA commits arrive on both CTAs' copies of empty, aempty, accfull.
 template <int kMode>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     k_pf_gemm(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
               const __grid_constant__ CUtensorMap tmB_r, const __grid_constant__ CUtensorMap tmB_s,
               GemmArgs args) {
@@ -657,8 +736,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __shared__ float2 s_mul[kN];  // per token of the tile: (2^F, 2^-E) or (2^E x weight, -)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_rank();
+  const uint32_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const uint32_t ntiles = __ldcg(args.ctrl + args.count_word);
-  if (blockIdx.x >= ntiles) return;
+  if (pair >= ntiles) return;  // the same for both CTAs of the pair
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
@@ -670,27 +751,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&rempty[r], 4);  // one arrival per dequant warp
     }
     for (int a = 0; a < NA; ++a) {
-      mbar_init(&afull[a], 4);  // one arrival per dequant warp
+      mbar_init(&afull[a], 8);  // one arrival per dequant warp of both CTAs
       mbar_init(&aempty[a], 1);
     }
     for (int b = 0; b < NACC; ++b) {
       mbar_init(&accfull[b], 1);
-      mbar_init(&accempty[b], 8);  // one arrival per epilogue warp
+      mbar_init(&accempty[b], 16);  // one arrival per epilogue warp of both CTAs
     }
     mbar_init(&mma_done, 1);
     s_fail = 0;
     s_epi_fail = 0;
   }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+  if (warp == 1) {  // the same warp in both CTAs, the same columns in both
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_addr(&s_tmem)),
                  "r"(kTmemCols));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers are initialised before any remote arrival
   tc_fence_after();
   const uint32_t tmem = s_tmem;
+  // the first CTA's gathering barriers, as shared::cluster addresses
+  const uint32_t full_cl = cluster_addr(&full[0], 0);
+  const uint32_t afull_cl = cluster_addr(&afull[0], 0);
+  const uint32_t accempty_cl = cluster_addr(&accempty[0], 0);
   if (tid == 0) pf_mark(kMode, 4, 0);
 
   if (warp < 4) {
@@ -698,30 +784,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (warp == 0 && lane == 0) {
       // ---- token-tile producer, by TMA
       uint32_t it = 0;
-      for (uint32_t ti = blockIdx.x; ti < ntiles && !s_fail; ti += gridDim.x) {
+      for (uint32_t ti = pair; ti < ntiles && !s_fail; ti += npairs) {
         PfTile t;
-        if (!pf_tile<kMode>(args, ti, t)) continue;
+        if (!pf_tile<kMode>(args, ti, rank, t)) continue;
         const CUtensorMap *tB = t.sh ? &tmB_s : &tmB_r;
-        const int brow = (kMode == 2 && t.sh) ? t.n0 : t.b_row;  // GEMM 2's shared B is Hs
+        // this CTA's half of the token rows (GEMM 2's shared B is Hs)
+        const int brow = ((kMode == 2 && t.sh) ? t.n0 : t.b_row) + (int)rank * (t.n_mma / 2);
         for (int G = 0; G < t.ng; ++G, ++it) {
           const int s = it % S;
-          if (it >= (uint32_t)S && !mbar_wait_sleep(&empty[s], ((it / S) - 1) & 1)) {
+          if (it >= (uint32_t)S && !cwait_sleep(&empty[s], ((it / S) - 1) & 1)) {
             s_fail = 1;
             break;
           }
           unsigned char *st = sm + Cfg::b_off(s);
-          mbar_expect_tx(&full[s], Cfg::kBStage);
-          tma_load_2d(st, tB, G * 128, brow, &full[s]);
-          tma_load_2d(st + Cfg::kBAtom, tB, G * 128 + 64, brow, &full[s]);
-          if (ti == blockIdx.x) pf_mark(kMode, 0, G);
+          if (rank == 0) mbar_expect_tx(&full[s], 2 * Cfg::kBStage);  // both halves
+          const uint32_t fb = full_cl + 8u * s;
+          tma_load_2d_pair(st, tB, G * 128, brow, fb);
+          tma_load_2d_pair(st + Cfg::kBAtom, tB, G * 128 + 64, brow, fb);
+          if (ti == pair) pf_mark(kMode, 0, G);
         }
       }
     } else if (warp == 2 && lane == 0) {
       // ---- int4-code producer, by TMA
       uint32_t it = 0;
-      for (uint32_t ti = blockIdx.x; ti < ntiles && !s_fail; ti += gridDim.x) {
+      for (uint32_t ti = pair; ti < ntiles && !s_fail; ti += npairs) {
         PfTile t;
-        if (!pf_tile<kMode>(args, ti, t)) continue;
+        if (!pf_tile<kMode>(args, ti, rank, t)) continue;
         const CUtensorMap *tA = t.sh ? &tmA_s : &tmA_r;
         for (int G = 0; G < t.ng; ++G, ++it) {
           const int r = it % R;
@@ -739,26 +827,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
+    } else if (warp == 1 && lane == 0 && rank == 1) {
+      // the pair's MMAs write this CTA's tensor memory: they complete before it is freed
+      if (!cwait_sleep(&mma_done, 0)) s_fail = 1;
     } else if (warp == 1 && lane == 0) {
-      // ---- MMA issuer: tile tc accumulates into buffer tc % NACC
+      // ---- MMA issuer (first CTA): tile tc accumulates into buffer tc % NACC of both CTAs
       uint32_t it = 0, tc = 0;
-      for (uint32_t ti = blockIdx.x; ti < ntiles && !s_fail; ti += gridDim.x) {
+      for (uint32_t ti = pair; ti < ntiles && !s_fail; ti += npairs) {
         PfTile t;
-        if (!pf_tile<kMode>(args, ti, t)) continue;
+        if (!pf_tile<kMode>(args, ti, rank, t)) continue;
         const int b = tc % NACC;
-        if (tc >= (uint32_t)NACC && !mbar_wait(&accempty[b], ((tc / NACC) - 1) & 1)) {
+        if (tc >= (uint32_t)NACC && !cwait_sleep(&accempty[b], ((tc / NACC) - 1) & 1)) {
           s_fail = 1;
           break;
         }
         tc_fence_after();
         const uint32_t d = tmem + Cfg::acc_col(b);
-        // kind::f16, A = B = f16, D = f32, K-major, N = n_mma, M = 128
+        // kind::f16, A = B = f16, D = f32, K-major, N = n_mma, M = 256 (the pair)
         const uint32_t idesc =
-            (1u << 4) | ((uint32_t)(t.n_mma >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+            (1u << 4) | ((uint32_t)(t.n_mma >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
         bool ok = true;
         for (int G = 0; G < t.ng; ++G, ++it) {
           const int s = it % S, a = it % NA;
-          if (!mbar_wait(&afull[a], (it / NA) & 1) || !mbar_wait(&full[s], (it / S) & 1)) {
+          if (!cwait_sleep(&afull[a], (it / NA) & 1) || !cwait_sleep(&full[s], (it / S) & 1)) {
             ok = false;
             break;
           }
@@ -769,24 +860,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int atom = 0; atom < 2; ++atom) {
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-              umma_f16_ts(d, a_tm + 8u * (4 * atom + k),
-                          sw128_desc(b_addr + atom * Cfg::kBAtom + 32 * k), idesc,
-                          (G | atom | k) != 0);
+              umma_f16_ts_pair(d, a_tm + 8u * (4 * atom + k),
+                               sw128_desc(b_addr + atom * Cfg::kBAtom + 32 * k), idesc,
+                               (G | atom | k) != 0);
           }
-          umma_commit(&empty[s]);   // the stage's shared memory is free for the producer
-          umma_commit(&aempty[a]);  // the weight tile's TMEM is free for the dequant warps
-          if (ti == blockIdx.x) pf_mark(kMode, 2, G);
+          umma_commit_pair(&empty[s]);   // both halves of the stage are free for the producers
+          umma_commit_pair(&aempty[a]);  // both weight tiles are free for the dequant warps
+          if (ti == pair) pf_mark(kMode, 2, G);
         }
         if (!ok) {
           s_fail = 1;
           break;
         }
-        umma_commit(&accfull[b]);  // the tile's sum is complete in accumulator b
+        umma_commit_pair(&accfull[b]);  // the tile's sums are complete in accumulator b
         ++tc;
       }
-      // every MMA this thread issued completes before the CTA frees tensor memory
-      umma_commit(&mma_done);
-      if (!mbar_wait(&mma_done, 0)) s_fail = 1;
+      // every MMA this thread issued completes before either CTA frees tensor memory
+      umma_commit_pair(&mma_done);
+      if (!cwait_sleep(&mma_done, 0)) s_fail = 1;
     }  // other lanes and warp 3: idle (register donors)
   } else if (warp < 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegDeq));
@@ -794,9 +885,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int i = tid - 128, q = warp - 4;
     const int raw_row = kMode == 1 ? ((i & 1) ? 64 + (i >> 1) : (i >> 1)) : i;
     uint32_t it = 0;
-    for (uint32_t ti = blockIdx.x; ti < ntiles && !s_fail; ti += gridDim.x) {
+    for (uint32_t ti = pair; ti < ntiles && !s_fail; ti += npairs) {
       PfTile t;
-      if (!pf_tile<kMode>(args, ti, t)) continue;
+      if (!pf_tile<kMode>(args, ti, rank, t)) continue;
       // the row's bf16 scales for the whole K (16, 8 or 4 groups) and the matrix shift
       const int wrow = kMode == 1 ? ((i & 1) ? t.row1 : t.row0) + (i >> 1) : t.row0 + i;
       const int gpr = t.ng;
@@ -811,7 +902,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int G = 0; G < t.ng; ++G, ++it) {
         const int rr = it % R, a = it % NA;
         if (!mbar_wait_sleep(&rfull[rr], (it / R) & 1) ||
-            (it >= (uint32_t)NA && !mbar_wait_sleep(&aempty[a], ((it / NA) - 1) & 1))) {
+            (it >= (uint32_t)NA && !cwait_sleep(&aempty[a], ((it / NA) - 1) & 1))) {
           ok = false;
           break;
         }
@@ -843,9 +934,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&rempty[rr]);  // the codes are in registers and TMEM
-          mbar_arrive(&afull[a]);
+          mbar_arrive_cluster(afull_cl + 8u * a);
         }
-        if (tid == 128 && ti == blockIdx.x) pf_mark(kMode, 1, G);
+        if (tid == 128 && ti == pair) pf_mark(kMode, 1, G);
       }
       if (!ok) {
         s_fail = 1;
@@ -866,9 +957,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // all eight warps leave in the same iteration.
     const int et = tid - 256;
     uint32_t tc = 0;
-    for (uint32_t ti = blockIdx.x; ti < ntiles; ti += gridDim.x) {
+    for (uint32_t ti = pair; ti < ntiles; ti += npairs) {
       PfTile t;
-      if (!pf_tile<kMode>(args, ti, t)) continue;
+      if (!pf_tile<kMode>(args, ti, rank, t)) continue;
       const int b = tc % NACC;
       const float4 ws = __ldg(args.wst + t.e);
       float2 pre = make_float2(0.f, 0.f);
@@ -876,7 +967,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (kMode == 1) pre = __ldg(args.rsc + t.b_row + et);
         else pre.x = __ldg(args.rm3 + t.b_row + et);
       }
-      const bool ok = mbar_wait_sleep(&accfull[b], (tc / NACC) & 1);
+      const bool ok = cwait_sleep(&accfull[b], (tc / NACC) & 1);
       tc_fence_after();
       uint32_t acc[kHalf];
       if (ok && c_lo < t.n_mma) {  // the same for the whole warp
@@ -888,8 +979,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0 && ok) mbar_arrive(&accempty[b]);  // the MMAs of tile tc + NACC may start
-      if (tid == 256 && ti == blockIdx.x) pf_mark(kMode, 3, 0);
+      if (lane == 0 && ok) mbar_arrive_cluster(accempty_cl + 8u * b);  // tile tc + NACC may start
+      if (tid == 256 && ti == pair) pf_mark(kMode, 3, 0);
       ++tc;
       named_bar_sync(1, kEpiThreads);  // every warp is done with the previous tile's multipliers
       if (!ok) s_epi_fail = 1;
@@ -951,11 +1042,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // neither CTA leaves while the other may still reach its memory
   if (tid == 0) pf_mark(kMode, 4, 1);
   if (s_fail && tid == 0) set_status(args.status, kStatusTimeout);
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(kTmemCols));
   }
 }
@@ -1016,6 +1108,26 @@ cudaError_t make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, u
                               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// Clusters of two GEMM CTAs that can be resident at once on this device.
+cudaError_t max_pairs(const void *fn, size_t smem, int *pairs) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, fn, &cfg);
+  if (e != cudaSuccess) return e;
+  *pairs = n > 0 ? n : 1;
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -1092,11 +1204,11 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
   const auto SW = CU_TENSOR_MAP_SWIZZLE_128B, NS = CU_TENSOR_MAP_SWIZZLE_NONE;
   if ((e = make_map(&mA1r, L.w13_q, U8, kH / 2, (uint64_t)kE * 2 * kI, kH / 2, 64, 64, NS)) ||
       (e = make_map(&mA1s, L.sh13_q, U8, kH / 2, 2 * kIs, kH / 2, 64, 64, NS)) ||
-      (e = make_map(&mB1, xp, F16, kH, (uint64_t)7 * T, kH * 2, 64, kPfN1, SW)) ||
+      (e = make_map(&mB1, xp, F16, kH, (uint64_t)7 * T, kH * 2, 64, GemmCfg<1>::kBRows, SW)) ||
       (e = make_map(&mA2r, L.w2_q, U8, kI / 2, (uint64_t)kE * kH, kI / 2, 64, 128, NS)) ||
       (e = make_map(&mA2s, L.sh2_q, U8, kIs / 2, kH, kIs / 2, 64, 128, NS)) ||
-      (e = make_map(&mB2r, hr, F16, kI, (uint64_t)P.mr, kI * 2, 64, kPfN2, SW)) ||
-      (e = make_map(&mB2s, hs, F16, kIs, (uint64_t)T, kIs * 2, 64, kPfN2, SW)))
+      (e = make_map(&mB2r, hr, F16, kI, (uint64_t)P.mr, kI * 2, 64, GemmCfg<2>::kBRows, SW)) ||
+      (e = make_map(&mB2s, hs, F16, kIs, (uint64_t)T, kIs * 2, 64, GemmCfg<2>::kBRows, SW)))
     return e;
   note_step("prefill GEMM attributes");
   if ((e = cudaFuncSetAttribute(k_pf_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1104,20 +1216,20 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
       (e = cudaFuncSetAttribute(k_pf_gemm<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)GemmCfg<2>::kSmem)) != cudaSuccess)
     return e;
-  // persistent GEMMs: one CTA per SM at most (the tile counts are on the device)
-  int dev = 0, sms = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (sms < 1) sms = 1;
+  // persistent GEMMs: as many CTA pairs as fit at once (the tile counts are on the device)
+  int pairs1 = 0, pairs2 = 0;
+  if ((e = max_pairs(reinterpret_cast<const void *>(k_pf_gemm<1>), GemmCfg<1>::kSmem, &pairs1)) ||
+      (e = max_pairs(reinterpret_cast<const void *>(k_pf_gemm<2>), GemmCfg<2>::kSmem, &pairs2)))
+    return e;
   GemmArgs a1{tiles1, ctrl, 3, ebase, ecount, T, L.w13_s, L.sh13_s, wst, rsc, rm3, hr, hs, ctrl + 1};
   note_step("prefill GEMM 1 launch");
-  k_pf_gemm<1><<<min(P.max_tiles1, sms), kGemmThreads, GemmCfg<1>::kSmem, st>>>(mA1r, mA1s, mB1,
-                                                                                mB1, a1);
+  k_pf_gemm<1><<<2 * min(P.max_tiles1, pairs1), kGemmThreads, GemmCfg<1>::kSmem, st>>>(
+      mA1r, mA1s, mB1, mB1, a1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   GemmArgs a2{tiles2, ctrl, 4, ebase, ecount, T, L.w2_s, L.sh2_s, wst, rsc, rm3, yw, ys, ctrl + 1};
   note_step("prefill GEMM 2 launch");
-  k_pf_gemm<2><<<min(P.max_tiles2, sms), kGemmThreads, GemmCfg<2>::kSmem, st>>>(mA2r, mA2s, mB2r,
-                                                                                mB2s, a2);
+  k_pf_gemm<2><<<2 * min(P.max_tiles2, pairs2), kGemmThreads, GemmCfg<2>::kSmem, st>>>(
+      mA2r, mA2s, mB2r, mB2s, a2);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // 5. combine
   note_step("prefill combine launch");
