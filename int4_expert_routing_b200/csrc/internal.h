@@ -85,8 +85,8 @@ inline PrefillLayout prefill_layout(int T) {
   L.ecount = take(sizeof(int32_t) * 256);
   L.perm = take(sizeof(int32_t) * (size_t)L.mr);
   L.pw = take(sizeof(float) * (size_t)L.mr);
-  L.tiles1 = take(sizeof(int32_t) * (size_t)L.max_tiles1);
-  L.tiles2 = take(sizeof(int32_t) * (size_t)L.max_tiles2);
+  L.tiles1 = take(sizeof(uint32_t) * 2 * (size_t)L.max_tiles1);  // tile descriptors (2 words)
+  L.tiles2 = take(sizeof(uint32_t) * 2 * (size_t)L.max_tiles2);
   L.wst = take(sizeof(float) * 4 * 257);   // per expert matrix pair: power-of-two shifts
   L.wbound = take(sizeof(float) * 257);    // per expert: bound factor of the SwiGLU output
   L.xstat = take(sizeof(float) * 2 * (size_t)T);     // per token: 2^-F, 2^E

@@ -208,8 +208,12 @@ FLINT_DEV int block_scan(int v, int *s_warp, int *total) {
   return off + incl - v;
 }
 
-FLINT_DEV uint32_t pack_tile(int e, int mt, int nt) {
-  return (uint32_t)e | ((uint32_t)mt << 9) | ((uint32_t)nt << 14);
+// Tile descriptor: x = expert | pair row tile << 9 | token tile << 14;
+// y = first row of the token tile in the per-row tables | valid tokens << 23
+// (rows < 7 * 2^20 < 2^23, valid tokens <= 256).
+FLINT_DEV uint2 pack_tile(int e, int mp, int nt, int b_row, int n_valid) {
+  return make_uint2((uint32_t)e | ((uint32_t)mp << 9) | ((uint32_t)nt << 14),
+                    (uint32_t)b_row | ((uint32_t)n_valid << 23));
 }
 
 // One CTA of 256 threads (one per expert): chunk offsets, expert counts,
@@ -219,8 +223,8 @@ FLINT_DEV uint32_t pack_tile(int e, int mt, int nt) {
 __global__ void __launch_bounds__(256)
     k_pf_scan(int T, int nchunks, const int32_t *__restrict__ chunk_cnt,
               int32_t *__restrict__ chunk_off, int32_t *__restrict__ ebase,
-              int32_t *__restrict__ ecount, uint32_t *__restrict__ tiles1,
-              uint32_t *__restrict__ tiles2, uint32_t *__restrict__ ctrl) {
+              int32_t *__restrict__ ecount, uint2 *__restrict__ tiles1,
+              uint2 *__restrict__ tiles2, uint32_t *__restrict__ ctrl) {
   __shared__ int s_warp[8];
   const int e = threadIdx.x;
   int off = 0;
@@ -238,13 +242,21 @@ __global__ void __launch_bounds__(256)
   ebase[e] = base;
   if (e == 0) ebase[kE] = total_rows;
   for (int nt = 0; nt < nt1; ++nt)
-    for (int mp = 0; mp < 4; ++mp) tiles1[o1 + nt * 4 + mp] = pack_tile(e, mp, nt);
+    for (int mp = 0; mp < 4; ++mp)
+      tiles1[o1 + nt * 4 + mp] =
+          pack_tile(e, mp, nt, base + nt * kPfN1, min(kPfN1, off - nt * kPfN1));
   for (int nt = 0; nt < nt2; ++nt)
-    for (int mp = 0; mp < 8; ++mp) tiles2[o2 + nt * 8 + mp] = pack_tile(e, mp, nt);
-  // the shared expert: one group over all T tokens
+    for (int mp = 0; mp < 8; ++mp)
+      tiles2[o2 + nt * 8 + mp] =
+          pack_tile(e, mp, nt, base + nt * kPfN2, min(kPfN2, off - nt * kPfN2));
+  // the shared expert: one group over all T tokens, rows 6T .. 7T - 1 of the tables
   const int nsh1 = (T + kPfN1 - 1) / kPfN1, nsh2 = (T + kPfN2 - 1) / kPfN2;
-  for (int i = e; i < 8 * nsh1; i += kE) tiles1[total1 + i] = pack_tile(kE, i & 7, i >> 3);
-  for (int i = e; i < 8 * nsh2; i += kE) tiles2[total2 + i] = pack_tile(kE, i & 7, i >> 3);
+  for (int i = e; i < 8 * nsh1; i += kE)
+    tiles1[total1 + i] =
+        pack_tile(kE, i & 7, i >> 3, 6 * T + (i >> 3) * kPfN1, min(kPfN1, T - (i >> 3) * kPfN1));
+  for (int i = e; i < 8 * nsh2; i += kE)
+    tiles2[total2 + i] =
+        pack_tile(kE, i & 7, i >> 3, 6 * T + (i >> 3) * kPfN2, min(kPfN2, T - (i >> 3) * kPfN2));
   if (e == 0) {
     ctrl[3] = (uint32_t)(total1 + 8 * nsh1);
     ctrl[4] = (uint32_t)(total2 + 8 * nsh2);
@@ -485,7 +497,7 @@ struct GemmCfg {
 };
 
 struct GemmArgs {
-  const uint32_t *tiles;
+  const uint2 *tiles;
   const uint32_t *ctrl;
   int count_word;
   const int32_t *ebase;
@@ -559,34 +571,12 @@ FLINT_DEV void cluster_sync_all() {
 FLINT_DEV void mbar_arrive_cluster(uint32_t cl_addr) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
 }
-// bounded waits with cluster-scope acquire (the arrivals come from the other
-// CTA of the pair or from its MMAs); the second form may suspend the thread
-FLINT_DEV bool cwait(uint64_t *bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kWaitPolls; ++i) {
-    uint32_t done;
-    asm volatile(
-        "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2; "
-        "selp.u32 %0, 1, 0, p; }"
-        : "=r"(done)
-        : "r"(smem_addr(bar)), "r"(parity)
-        : "memory");
-    if (done) return true;
-  }
-  return false;
-}
-FLINT_DEV bool cwait_sleep(uint64_t *bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kSleepPolls; ++i) {
-    uint32_t done;
-    asm volatile(
-        "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3; "
-        "selp.u32 %0, 1, 0, p; }"
-        : "=r"(done)
-        : "r"(smem_addr(bar)), "r"(parity), "r"(20000u)
-        : "memory");
-    if (done) return true;
-  }
-  return false;
-}
+// Waits on barriers that the other CTA of the pair or the pair's MMAs arrive
+// on: the default (CTA-scope) acquire, as for the other barriers; what must be
+// ordered is tensor-memory and shared-memory state completed before the
+// arrival (tcgen05.wait / fence, TMA and MMA completion).
+FLINT_DEV bool cwait(uint64_t *bar, uint32_t parity) { return mbar_wait(bar, parity); }
+FLINT_DEV bool cwait_sleep(uint64_t *bar, uint32_t parity) { return mbar_wait_sleep(bar, parity); }
 // TMA tile load into this CTA's shared memory whose completion is counted on
 // an mbarrier of either CTA of the pair (`bar_cl`, a shared::cluster address)
 FLINT_DEV void tma_load_2d_pair(void *dst, const CUtensorMap *map, int x, int y, uint32_t bar_cl) {
@@ -686,21 +676,19 @@ struct PfTile {
   int e, mt, n0, n_valid, n_mma, b_row, row0, row1, ng;
   bool sh;
 };
-// mt is this CTA's 128-row tile: 2 x (the pair's tile) + the CTA's rank
+// The tile a descriptor names, as every role of both CTAs derives it; mt is
+// this CTA's 128-row tile: 2 x (the pair's tile) + the CTA's rank.
 template <int kMode>
-FLINT_DEV bool pf_tile(const GemmArgs &args, uint32_t idx, uint32_t rank, PfTile &t) {
+FLINT_DEV bool pf_tile(const GemmArgs &args, uint2 w, uint32_t rank, PfTile &t) {
   constexpr int kN = GemmCfg<kMode>::kN;
-  const uint32_t packed = __ldcg(args.tiles + idx);
-  t.e = (int)(packed & 511u);
-  t.mt = 2 * (int)((packed >> 9) & 31u) + (int)rank;
-  const int nt = (int)(packed >> 14);
+  t.e = (int)(w.x & 511u);
+  t.mt = 2 * (int)((w.x >> 9) & 31u) + (int)rank;
+  t.n0 = (int)(w.x >> 14) * kN;
+  t.b_row = (int)(w.y & ((1u << 23) - 1u));
+  t.n_valid = (int)(w.y >> 23);
   t.sh = t.e == kE;
-  t.n0 = nt * kN;
-  t.n_valid = min(kN, (t.sh ? args.T : __ldcg(args.ecount + t.e)) - t.n0);
-  if (t.n_valid <= 0) return false;  // not produced by the scan; guards against an N = 0 MMA
+  if (t.n_valid <= 0) return false;  // guards against an N = 0 MMA
   t.n_mma = (t.n_valid + 31) & ~31;  // the pair MMA takes N in steps of 32
-  // row of the per-row tables (and of the fp16 token rows): routed rows, then the T shared rows
-  t.b_row = t.sh ? 6 * args.T + t.n0 : __ldcg(args.ebase + t.e) + t.n0;
   t.ng = (kMode == 1 ? kH : (t.sh ? kIs : kI)) / kG;  // 128-wide k-groups
   if (kMode == 1) {  // weight rows: gate (tile rows 2i) / up (2i+1)
     t.row0 = t.sh ? 64 * t.mt : t.e * 2 * kI + 64 * t.mt;
@@ -710,6 +698,12 @@ FLINT_DEV bool pf_tile(const GemmArgs &args, uint32_t idx, uint32_t rank, PfTile
     t.row1 = t.row0;
   }
   return true;
+}
+
+// Descriptor of the pair's tile `ti` (zero past the end): each role loads the
+// next one while it works on the current one.
+FLINT_DEV uint2 tile_word(const GemmArgs &args, uint32_t ti, uint32_t ntiles) {
+  return ti < ntiles ? __ldcg(args.tiles + ti) : make_uint2(0u, 0u);
 }
 
 // Persistent: pair c takes tiles c, c + pairs, ...  Every role of both CTAs
@@ -784,9 +778,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     if (warp == 0 && lane == 0) {
       // ---- token-tile producer, by TMA
       uint32_t it = 0;
+      uint2 wnext = tile_word(args, pair, ntiles);
       for (uint32_t ti = pair; ti < ntiles && !s_fail; ti += npairs) {
+        const uint2 w = wnext;
+        wnext = tile_word(args, ti + npairs, ntiles);
         PfTile t;
-        if (!pf_tile<kMode>(args, ti, rank, t)) continue;
+        if (!pf_tile<kMode>(args, w, rank, t)) continue;
         const CUtensorMap *tB = t.sh ? &tmB_s : &tmB_r;
         // this CTA's half of the token rows (GEMM 2's shared B is Hs)
         const int brow = ((kMode == 2 && t.sh) ? t.n0 : t.b_row) + (int)rank * (t.n_mma / 2);
@@ -807,9 +804,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     } else if (warp == 2 && lane == 0) {
       // ---- int4-code producer, by TMA
       uint32_t it = 0;
+      uint2 wnext = tile_word(args, pair, ntiles);
       for (uint32_t ti = pair; ti < ntiles && !s_fail; ti += npairs) {
+        const uint2 w = wnext;
+        wnext = tile_word(args, ti + npairs, ntiles);
         PfTile t;
-        if (!pf_tile<kMode>(args, ti, rank, t)) continue;
+        if (!pf_tile<kMode>(args, w, rank, t)) continue;
         const CUtensorMap *tA = t.sh ? &tmA_s : &tmA_r;
         for (int G = 0; G < t.ng; ++G, ++it) {
           const int r = it % R;
@@ -833,9 +833,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     } else if (warp == 1 && lane == 0) {
       // ---- MMA issuer (first CTA): tile tc accumulates into buffer tc % NACC of both CTAs
       uint32_t it = 0, tc = 0;
+      uint2 wnext = tile_word(args, pair, ntiles);
       for (uint32_t ti = pair; ti < ntiles && !s_fail; ti += npairs) {
+        const uint2 w = wnext;
+        wnext = tile_word(args, ti + npairs, ntiles);
         PfTile t;
-        if (!pf_tile<kMode>(args, ti, rank, t)) continue;
+        if (!pf_tile<kMode>(args, w, rank, t)) continue;
         const int b = tc % NACC;
         if (tc >= (uint32_t)NACC && !cwait_sleep(&accempty[b], ((tc / NACC) - 1) & 1)) {
           s_fail = 1;
@@ -884,20 +887,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // ---- dequant: thread i owns weight row i of every tile, TMEM lane i
     const int i = tid - 128, q = warp - 4;
     const int raw_row = kMode == 1 ? ((i & 1) ? 64 + (i >> 1) : (i >> 1)) : i;
+    // the row's bf16 scales for the whole K (16, 8 or 4 groups) and the matrix
+    // shift, fetched one tile ahead (tile descriptors two ahead)
+    auto fetch = [&](uint2 w, uint32_t (&sc)[8], float &mul) {
+      PfTile tn;
+      if (!pf_tile<kMode>(args, w, rank, tn)) return;
+      const int wrow = kMode == 1 ? ((i & 1) ? tn.row1 : tn.row0) + (i >> 1) : tn.row0 + i;
+      const uint32_t *srow = reinterpret_cast<const uint32_t *>(
+          (tn.sh ? args.sc_s : args.sc_r) + (size_t)wrow * tn.ng);
+#pragma unroll
+      for (int w2 = 0; w2 < 8; ++w2) sc[w2] = w2 < tn.ng / 2 ? __ldg(srow + w2) : 0u;
+      const float4 ws = __ldg(args.wst + tn.e);
+      mul = kMode == 1 ? ws.x : ws.z;
+    };
+    uint2 wa = tile_word(args, pair, ntiles), wb = tile_word(args, pair + npairs, ntiles);
+    uint32_t scn[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    float muln = 0.f;
+    fetch(wa, scn, muln);
     uint32_t it = 0;
     for (uint32_t ti = pair; ti < ntiles && !s_fail; ti += npairs) {
+      const uint2 w = wa;
+      wa = wb;
+      wb = tile_word(args, ti + 2 * npairs, ntiles);
       PfTile t;
-      if (!pf_tile<kMode>(args, ti, rank, t)) continue;
-      // the row's bf16 scales for the whole K (16, 8 or 4 groups) and the matrix shift
-      const int wrow = kMode == 1 ? ((i & 1) ? t.row1 : t.row0) + (i >> 1) : t.row0 + i;
-      const int gpr = t.ng;
-      const uint32_t *srow = reinterpret_cast<const uint32_t *>(
-          (t.sh ? args.sc_s : args.sc_r) + (size_t)wrow * gpr);
+      const bool valid = pf_tile<kMode>(args, w, rank, t);
       uint32_t scw[8];
 #pragma unroll
-      for (int w = 0; w < 8; ++w) scw[w] = w < gpr / 2 ? __ldg(srow + w) : 0u;
-      const float4 ws = __ldg(args.wst + t.e);
-      const float smul = kMode == 1 ? ws.x : ws.z;
+      for (int w2 = 0; w2 < 8; ++w2) scw[w2] = scn[w2];
+      const float smul = muln;
+      fetch(wa, scn, muln);  // the next tile's, in flight during this one
+      if (!valid) continue;
       bool ok = true;
       for (int G = 0; G < t.ng; ++G, ++it) {
         const int rr = it % R, a = it % NA;
@@ -957,9 +976,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // all eight warps leave in the same iteration.
     const int et = tid - 256;
     uint32_t tc = 0;
+    uint2 wnext = tile_word(args, pair, ntiles);
     for (uint32_t ti = pair; ti < ntiles; ti += npairs) {
+      const uint2 w = wnext;
+      wnext = tile_word(args, ti + npairs, ntiles);
       PfTile t;
-      if (!pf_tile<kMode>(args, ti, rank, t)) continue;
+      if (!pf_tile<kMode>(args, w, rank, t)) continue;
       const int b = tc % NACC;
       const float4 ws = __ldg(args.wst + t.e);
       float2 pre = make_float2(0.f, 0.f);
@@ -1165,8 +1187,8 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
   int32_t *ecount = reinterpret_cast<int32_t *>(ws + P.ecount);
   int32_t *perm = reinterpret_cast<int32_t *>(ws + P.perm);
   float *pw = reinterpret_cast<float *>(ws + P.pw);
-  uint32_t *tiles1 = reinterpret_cast<uint32_t *>(ws + P.tiles1);
-  uint32_t *tiles2 = reinterpret_cast<uint32_t *>(ws + P.tiles2);
+  uint2 *tiles1 = reinterpret_cast<uint2 *>(ws + P.tiles1);
+  uint2 *tiles2 = reinterpret_cast<uint2 *>(ws + P.tiles2);
   float4 *wst = reinterpret_cast<float4 *>(ws + P.wst);
   float *wbound = reinterpret_cast<float *>(ws + P.wbound);
   float2 *xstat = reinterpret_cast<float2 *>(ws + P.xstat);
