@@ -296,8 +296,11 @@ FLINT_DEV float exp2i(int n) { return __int_as_float((n + 127) << 23); }
 FLINT_DEV int clamp_shift(int n) { return min(max(n, -126), 126); }
 
 // One CTA per expert (expert 256 = the shared one).  For the gate/up matrix
-// and the down matrix the shift S puts the largest |code x scale| (|code| <= 8)
-// in [2^14, 2^15); wst[e] = (2^-S1, 2^S1, 2^-S2, 2^S2).  wbound[e] bounds the
+// and the down matrix the shift S puts the largest |scale| in [2^-10, 2^-9),
+// so the dequantization's fp16 multipliers scale x 2^24 stay below the fp16
+// maximum and every code x scale (at most 11 significant bits) is an exact
+// fp16 for scales down to 2^-17 (a 256-fold spread inside one matrix);
+// wst[e] = (2^-S1, 2^S1, 2^-S2, 2^S2).  wbound[e] bounds the
 // SwiGLU output per unit of |x|^2: by Cauchy-Schwarz |W1 x| <= |x| |W1 row| and
 // |silu(g)| <= |g|, so |silu(W1 x) (W3 x)| <= |x|^2 max|W1 row| max|W3 row|,
 // with |row| <= 8 sqrt(128 sum_g scale_g^2) for 128-wide groups of codes in [-8, 7].
@@ -349,8 +352,8 @@ __global__ void __launch_bounds__(256)
       m[k] = red[k][0];
       for (int w = 1; w < 8; ++w) m[k] = fmaxf(m[k], red[k][w]);
     }
-    const int S1 = m[0] > 0.f ? clamp_shift(ilogbf(m[0]) + 3 - 14) : 0;
-    const int S2 = m[1] > 0.f ? clamp_shift(ilogbf(m[1]) + 3 - 14) : 0;
+    const int S1 = m[0] > 0.f ? clamp_shift(ilogbf(m[0]) + 10) : 0;
+    const int S2 = m[1] > 0.f ? clamp_shift(ilogbf(m[1]) + 10) : 0;
     wst[e] = make_float4(exp2i(-S1), exp2i(S1), exp2i(-S2), exp2i(S2));
     wbound[e] = m[2] * m[3];
   }
@@ -647,17 +650,23 @@ FLINT_DEV void named_bar_sync(int id, int n) {
 FLINT_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 FLINT_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// 8 int4 codes (one 32-bit word, code k in bits 4k..4k+3) times an fp16x2
-// scale: pairs (k, k+4) for k = 0..3, exact.
-FLINT_DEV void codes8_f16(uint32_t w, uint32_t sc2, uint32_t *out) {
-#pragma unroll
-  for (int p = 0; p < 4; ++p) {
-    // (code ^ 8) + 1024 as fp16, exact; minus 1032 gives the signed code
-    const uint32_t t = ((w >> (4 * p)) & 0x000F000Fu) ^ 0x64086408u;
-    uint32_t c;
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(c) : "r"(t), "r"(0x64086408u));
-    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(out[p]) : "r"(c), "r"(sc2));
-  }
+// 8 int4 codes (one 32-bit word, code k in bits 4k..4k+3, two's complement)
+// times a scale s: fp16 pairs (k, k+4) for k = 0..3, exact.  A code field
+// XOR 8 is n = code + 8 in [0, 15]; left in bits 0..3 of an fp16 it is the
+// subnormal n 2^-24, in bits 4..7 it is n 2^-20.  One fused multiply-add
+// n 2^-24 (s 2^24) - 8 s (or with s 2^20) forms code x s exactly inside and
+// rounds once, and code x s is itself an fp16, so the result is exact.
+// m24 = s 2^24, m20 = s 2^20 and c8 = -8 s as fp16x2 (both halves equal).
+FLINT_DEV void codes8_f16(uint32_t w, uint32_t m24, uint32_t m20, uint32_t c8, uint32_t *out) {
+  const uint32_t w8 = w >> 8;
+  const uint32_t t0 = (w & 0x000F000Fu) ^ 0x00080008u;   // codes 0, 4
+  const uint32_t t1 = (w & 0x00F000F0u) ^ 0x00800080u;   // codes 1, 5
+  const uint32_t t2 = (w8 & 0x000F000Fu) ^ 0x00080008u;  // codes 2, 6
+  const uint32_t t3 = (w8 & 0x00F000F0u) ^ 0x00800080u;  // codes 3, 7
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(out[0]) : "r"(t0), "r"(m24), "r"(c8));
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(out[1]) : "r"(t1), "r"(m20), "r"(c8));
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(out[2]) : "r"(t2), "r"(m24), "r"(c8));
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(out[3]) : "r"(t3), "r"(m20), "r"(c8));
 }
 
 // 16-bit global store, skipped when `pred` is false (no branch)
@@ -926,11 +935,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           break;
         }
         tc_fence_after();
-        // the group's scale x 2^-S as fp16x2 (exact: 8 significant bits, normal range)
+        // the group's scale s x 2^-S and its multipliers as fp16x2 (exact: 8
+        // significant bits; s 2^24 < 2^15 by the choice of S)
         const uint32_t sw = scw[G >> 1] >> (16 * (G & 1));
         const float sf = __uint_as_float(sw << 16) * smul;
-        const uint32_t hs = __half_as_ushort(__float2half_rn(sf));
-        const uint32_t sc2 = hs | (hs << 16);
+        const uint32_t h24 = __half_as_ushort(__float2half_rn(sf * 16777216.f));
+        const uint32_t h20 = __half_as_ushort(__float2half_rn(sf * 1048576.f));
+        const uint32_t hc8 = __half_as_ushort(__float2half_rn(sf * -8.f));
+        const uint32_t m24 = h24 | (h24 << 16), m20 = h20 | (h20 << 16), c8 = hc8 | (hc8 << 16);
         const unsigned char *raw = sm + Cfg::raw_off(rr) + raw_row * 64;
         const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + Cfg::a_col(a);
 #pragma unroll
@@ -941,10 +953,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             // chunk j = codes 32 j .. 32 j + 31 of the group -> columns 16 j ..
             const int j = 2 * hf + jj;
             const uint4 w = *reinterpret_cast<const uint4 *>(raw + 16 * j);
-            codes8_f16(w.x, sc2, v + 16 * jj + 0);
-            codes8_f16(w.y, sc2, v + 16 * jj + 4);
-            codes8_f16(w.z, sc2, v + 16 * jj + 8);
-            codes8_f16(w.w, sc2, v + 16 * jj + 12);
+            codes8_f16(w.x, m24, m20, c8, v + 16 * jj + 0);
+            codes8_f16(w.y, m24, m20, c8, v + 16 * jj + 4);
+            codes8_f16(w.z, m24, m20, c8, v + 16 * jj + 8);
+            codes8_f16(w.w, m24, m20, c8, v + 16 * jj + 12);
           }
           tmem_st32(tbase + 32u * hf, v);
         }
