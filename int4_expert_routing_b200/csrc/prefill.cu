@@ -407,31 +407,40 @@ __global__ void __launch_bounds__(256)
 // in sorted order, rows [6T, 7T) every token for the shared expert.  Each
 // 8-element block is stored in the order 0,4,1,5,2,6,3,7.  Per row, rsc =
 // (2^F, 2^-E) for GEMM 1's read-out and rm3 = 2^E x routing weight for GEMM 2's.
+// One warp per row (grid-stride): each lane moves 8 16-byte chunks, all loads
+// issued before the first store.
 __global__ void __launch_bounds__(256)
     k_pf_gather(const uint16_t *__restrict__ x, int T, const int32_t *__restrict__ perm,
                 const float *__restrict__ pw, const float2 *__restrict__ xstat,
                 uint16_t *__restrict__ xp, float2 *__restrict__ rsc, float *__restrict__ rm3) {
+  const int lane = threadIdx.x & 31;
   const size_t rows = (size_t)7 * T;
-  const size_t n = rows * (kH / 8);
-  for (size_t i = (size_t)blockIdx.x * 256 + threadIdx.x; i < n; i += (size_t)gridDim.x * 256) {
-    const size_t row = i / (kH / 8), c = i % (kH / 8);
+  const size_t nwarps = (size_t)gridDim.x * 8;
+  for (size_t row = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5); row < rows; row += nwarps) {
     const bool routed = row < (size_t)6 * T;
-    const int tok = routed ? perm[row] : (int)(row - (size_t)6 * T);
-    const float2 st = xstat[tok];
-    const uint4 v = ld_cg_v4(x + (size_t)tok * kH + 8 * c);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t h[8];
+    const int tok = routed ? __ldg(perm + row) : (int)(row - (size_t)6 * T);
+    const float2 st = __ldg(xstat + tok);
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)tok * kH);
+    uint4 v[8];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      h[2 * q] = __half_as_ushort(__float2half_rn(__uint_as_float(w[q] << 16) * st.x));
-      h[2 * q + 1] = __half_as_ushort(__float2half_rn(__uint_as_float(w[q] & 0xffff0000u) * st.x));
+    for (int c = 0; c < 8; ++c) v[c] = ld_cg_v4(src + 32 * c + lane);
+    uint4 *dst = reinterpret_cast<uint4 *>(xp + row * kH);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+      uint32_t h[8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        h[2 * q] = __half_as_ushort(__float2half_rn(__uint_as_float(w[q] << 16) * st.x));
+        h[2 * q + 1] = __half_as_ushort(__float2half_rn(__uint_as_float(w[q] & 0xffff0000u) * st.x));
+      }
+      // natural h[0..7] -> pairs (0,4), (1,5), (2,6), (3,7)
+      dst[32 * c + lane] = make_uint4(h[0] | (h[4] << 16), h[1] | (h[5] << 16), h[2] | (h[6] << 16),
+                                      h[3] | (h[7] << 16));
     }
-    // natural h[0..7] -> pairs (0,4), (1,5), (2,6), (3,7)
-    *reinterpret_cast<uint4 *>(xp + row * kH + 8 * c) =
-        make_uint4(h[0] | (h[4] << 16), h[1] | (h[5] << 16), h[2] | (h[6] << 16), h[3] | (h[7] << 16));
-    if (c == 0) {
+    if (lane == 0) {
       rsc[row] = make_float2(1.f / st.x, 1.f / st.y);
-      rm3[row] = routed ? st.y * pw[row] : st.y;
+      rm3[row] = routed ? st.y * __ldg(pw + row) : st.y;
     }
   }
 }
@@ -1226,8 +1235,8 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
   k_pf_wstats<<<kE + 1, 256, 0, st>>>(L.w13_s, L.w2_s, L.sh13_s, L.sh2_s, wst, wbound);
   k_pf_xstats<<<(T + 7) / 8, 256, 0, st>>>(x, T, wbound, xstat);
   {
-    int blocks = (int)(((size_t)7 * T * (kH / 8) + 255) / 256);
-    if (blocks > 148 * 16) blocks = 148 * 16;
+    int blocks = (int)(((size_t)7 * T + 7) / 8);  // 8 rows (warps) per block
+    if (blocks > 148 * 8) blocks = 148 * 8;
     k_pf_gather<<<blocks, 256, 0, st>>>(x, T, perm, pw, xstat, xp, rsc, rm3);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
