@@ -47,7 +47,7 @@ inline DecodeLayout decode_layout(int B) {
 // ctrl words: [1] status, [3] GEMM1 tile count, [4] GEMM2 tile count,
 // [5] routed rows.
 constexpr int kPfN1 = 256;
-constexpr int kPfN2 = 192;
+constexpr int kPfN2 = 256;
 constexpr int kPfChunk = 256;
 struct PrefillLayout {
   size_t ctrl, z, sel_idx, sel_w, asc_e, asc_w, route_total;

@@ -487,9 +487,9 @@ constexpr int kTmemCols = 512;
 template <int kMode>
 struct GemmCfg {
   static constexpr int kN = kMode == 1 ? kPfN1 : kPfN2;
-  static constexpr int kAcc = kMode == 1 ? 1 : 2;
-  static constexpr int kNA = kMode == 1 ? 4 : 2;
-  static constexpr int kS = kMode == 1 ? 6 : 8;
+  static constexpr int kAcc = 1;
+  static constexpr int kNA = 4;
+  static constexpr int kS = 6;
   static constexpr int kR = 3;
   static constexpr int kBRows = kN / 2;       // token rows per CTA (the TMA box height)
   static constexpr int kBAtom = kBRows * 128;  // kN / 2 token rows x 64 fp16
@@ -497,14 +497,10 @@ struct GemmCfg {
   static constexpr size_t kSmem = (size_t)kS * kBStage + (size_t)kR * kRawBytes + 1024;
   static constexpr size_t b_off(int s) { return (size_t)s * kBStage; }
   static constexpr size_t raw_off(int r) { return (size_t)kS * kBStage + (size_t)r * kRawBytes; }
-  // TMEM columns: GEMM 1: accumulator 0..255, weight tiles 256, 320, 384, 448;
-  // GEMM 2: accumulators at 0 and 256 (192 columns each), weight tiles 192, 448
+  // TMEM columns: the accumulator 0..255, the weight tiles at 256, 320, 384, 448
   static constexpr uint32_t acc_col(int b) { return (uint32_t)(256 * b); }
-  static constexpr uint32_t a_col(int a) {
-    return kMode == 1 ? (uint32_t)(256 + 64 * a) : (uint32_t)(192 + 256 * a);
-  }
-  static_assert(kMode == 1 ? (kN <= 256 && kAcc == 1 && kNA == 4)
-                           : (kN <= 192 && kAcc == 2 && kNA == 2), "tensor memory");
+  static constexpr uint32_t a_col(int a) { return (uint32_t)(256 + 64 * a); }
+  static_assert(kN <= 256 && kAcc == 1 && kNA == 4, "tensor memory");
   static_assert(kBAtom % 1024 == 0 && kN % 32 == 0, "tile shape");
 };
 
