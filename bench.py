@@ -63,6 +63,10 @@ def parse():
 
 # router 2*256*2048 + routed 6 * 3 * 2 * 2048 * 512 + shared 3 * 2 * 2048 * 1024
 PREFILL_FLOP_PER_TOKEN = 2 * 256 * 2048 + 6 * 6 * 2048 * 512 + 6 * 2048 * 1024
+# grouped GEMM 1 (gate and up: 6 routed + shared), grouped GEMM 2 (down)
+GEMM1_FLOP_PER_TOKEN = 6 * 2 * 2 * 2048 * 512 + 2 * 2 * 2048 * 1024
+GEMM2_FLOP_PER_TOKEN = 6 * 2 * 2048 * 512 + 2 * 2048 * 1024
+assert PREFILL_FLOP_PER_TOKEN == 2 * 256 * 2048 + GEMM1_FLOP_PER_TOKEN + GEMM2_FLOP_PER_TOKEN
 
 
 def tensor_peak():
@@ -433,9 +437,26 @@ def main():
                     times.append(e0.elapsed_time(e1) * 1e3)
             us = statistics.median(times)
             tflops = T * PREFILL_FLOP_PER_TOKEN / (us * 1e-6) / 1e12
+            # per-stage CUDA-event times inside the call (library measurement hook)
+            stage_runs = []
+            F.flint_debug_prefill_events(True)
+            for it in range(3):
+                with torch.cuda.stream(stream):
+                    flush.zero_()
+                    F.flint_moe_prefill(structs[0], xt, T, out_t, wsp, nbp, stream=stream)
+                stage_runs.append(F.flint_debug_prefill_stage_ms())
+            F.flint_debug_prefill_events(False)
+            stages_us = {k: 1e3 * statistics.median(r[k] for r in stage_runs) for k in stage_runs[0]}
+            g1_tf = T * GEMM1_FLOP_PER_TOKEN / (stages_us["gemm1"] * 1e-6) / 1e12
+            g2_tf = T * GEMM2_FLOP_PER_TOKEN / (stages_us["gemm2"] * 1e-6) / 1e12
+            gg_tf = (T * (GEMM1_FLOP_PER_TOKEN + GEMM2_FLOP_PER_TOKEN)
+                     / ((stages_us["gemm1"] + stages_us["gemm2"]) * 1e-6) / 1e12)
             extra[f"prefill_T{T}"] = {"us": us, "tokens_per_s": T / (us * 1e-6),
                                       "TFLOPs": tflops, "tensor_frac": tflops / peak_tf,
-                                      "peak_kind": peak_kind_tf}
+                                      "peak_kind": peak_kind_tf, "stages_us": stages_us,
+                                      "gemm1_TFLOPs": g1_tf, "gemm1_frac": g1_tf / peak_tf,
+                                      "gemm2_TFLOPs": g2_tf, "gemm2_frac": g2_tf / peak_tf,
+                                      "grouped_gemms_frac": gg_tf / peak_tf}
             del wsp, out_t, xt
     sampler.stop()
 

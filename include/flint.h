@@ -127,6 +127,16 @@ FLINT_API int flint_read_status(const void *ws, int *status, void *stream);
  * ordinary latency into timeouts. */
 FLINT_API int flint_debug_set_wait_polls(uint32_t polls);
 
+/* Measurement hook: while enabled (enable != 0), flint_moe_prefill records a
+ * CUDA event on its stream before and after each of its six stages (routing;
+ * sort; operand scaling and token gather; grouped GEMM 1; grouped GEMM 2;
+ * combine).  flint_debug_prefill_stage_ms waits for the last call's final
+ * event and writes the six stage times in milliseconds to ms[0..5] (n >= 6).
+ * The events belong to the device that was current at the first enable; one
+ * call at a time; not for production use. */
+FLINT_API int flint_debug_prefill_events(int enable);
+FLINT_API int flint_debug_prefill_stage_ms(float *ms, int n);
+
 /*
  * Router for B rows ("How to Run Flint Locally", section "The architecture,
  * from config.json": sigmoid router over 256 experts, top 6 kept, weights

@@ -22,7 +22,8 @@ EXPORTS = ("flint_version", "flint_strerror", "flint_last_cuda_error", "flint_wo
            "flint_gemv_workspace_bytes", "flint_workspace_init", "flint_read_status",
            "flint_moe_route", "flint_moe_decode", "flint_moe_decode_residual",
            "flint_moe_prefill", "flint_int4_gemv", "flint_int4_gemv_noalloc",
-           "flint_debug_set_wait_polls")
+           "flint_debug_set_wait_polls", "flint_debug_prefill_events",
+           "flint_debug_prefill_stage_ms")
 
 _lib = None
 
@@ -64,6 +65,8 @@ def lib() -> C.CDLL:
         L.flint_workspace_init.argtypes = [vp, sz, vp]
         L.flint_read_status.argtypes = [vp, C.POINTER(C.c_int), vp]
         L.flint_debug_set_wait_polls.argtypes = [C.c_uint32]
+        L.flint_debug_prefill_events.argtypes = [C.c_int]
+        L.flint_debug_prefill_stage_ms.argtypes = [C.POINTER(C.c_float), C.c_int]
         lp = C.POINTER(flint_moe_layer)
         L.flint_moe_route.argtypes = [lp, vp, i, vp, vp, vp, sz, vp]
         L.flint_moe_decode.argtypes = [lp, vp, i, vp, vp, sz, vp]
@@ -131,6 +134,21 @@ def flint_debug_set_wait_polls(polls: int) -> None:
     """Poll bound of the decode kernels' first barrier waits (test hook for
     the timeout path); 0xFFFFFFFF restores the default."""
     _check(lib().flint_debug_set_wait_polls(polls), "flint_debug_set_wait_polls")
+
+
+PREFILL_STAGES = ("routing", "sort", "scaling+gather", "gemm1", "gemm2", "combine")
+
+
+def flint_debug_prefill_events(enable: bool) -> None:
+    """Record CUDA events between the stages of flint_moe_prefill (measurement)."""
+    _check(lib().flint_debug_prefill_events(1 if enable else 0), "flint_debug_prefill_events")
+
+
+def flint_debug_prefill_stage_ms() -> dict:
+    """Stage times (ms) of the last flint_moe_prefill call made with events on."""
+    buf = (C.c_float * 6)()
+    _check(lib().flint_debug_prefill_stage_ms(buf, 6), "flint_debug_prefill_stage_ms")
+    return dict(zip(PREFILL_STAGES, list(buf)))
 
 
 def flint_read_status(ws, stream=None) -> int:

@@ -101,6 +101,15 @@ int flint_read_status(const void *ws, int *status, void *stream) {
   return FLINT_OK;
 }
 
+int flint_debug_prefill_events(int enable) {
+  return from_cuda(noted(prefill_set_stage_events(enable), "prefill stage events"));
+}
+
+int flint_debug_prefill_stage_ms(float *ms, int n) {
+  if (!ms) return FLINT_EINVAL;
+  return from_cuda(noted(prefill_stage_times(ms, n), "prefill stage times"));
+}
+
 int flint_debug_set_wait_polls(uint32_t polls) {
   return from_cuda(noted(decode_set_wait_polls(polls), "debug wait bound"));
 }

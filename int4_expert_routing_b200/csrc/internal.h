@@ -51,7 +51,7 @@ constexpr int kPfN2 = 256;
 constexpr int kPfChunk = 256;
 struct PrefillLayout {
   size_t ctrl, z, sel_idx, sel_w, asc_e, asc_w, route_total;
-  size_t pos, chunk_cnt, chunk_off, ebase, ecount, perm, pw, tiles1, tiles2, wst, wbound, xstat,
+  size_t pos, chunk_cnt, chunk_off, ebase, ecount, tiles1, tiles2, wst, wbound, xstat,
       rsc, rm3, xp, hr, hs, yw, ys, total;
   int mr, max_tiles1, max_tiles2, nchunks;
 };
@@ -83,8 +83,6 @@ inline PrefillLayout prefill_layout(int T) {
   L.chunk_off = take(sizeof(int32_t) * (size_t)L.nchunks * 256);
   L.ebase = take(sizeof(int32_t) * 257);
   L.ecount = take(sizeof(int32_t) * 256);
-  L.perm = take(sizeof(int32_t) * (size_t)L.mr);
-  L.pw = take(sizeof(float) * (size_t)L.mr);
   L.tiles1 = take(sizeof(uint32_t) * 2 * (size_t)L.max_tiles1);  // tile descriptors (2 words)
   L.tiles2 = take(sizeof(uint32_t) * 2 * (size_t)L.max_tiles2);
   L.wst = take(sizeof(float) * 4 * 257);   // per expert matrix pair: power-of-two shifts
@@ -139,6 +137,8 @@ cudaError_t launch_gemv(const uint8_t *q, const uint16_t *s, int N, int K, const
                         int B, float *y, int32_t *argmax, char *ws, cudaStream_t st);
 size_t gemv_ws_bytes(int N, int B);
 cudaError_t decode_set_wait_polls(uint32_t polls);
+cudaError_t prefill_set_stage_events(int enable);
+cudaError_t prefill_stage_times(float *ms, int n);
 cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_t *out, char *ws,
                            cudaStream_t st);
 cudaError_t launch_route_many(const LayerArgs &L, const uint16_t *x, int T, int32_t *idx, float *w,

@@ -264,10 +264,10 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// pos[t][j]: the sorted row of token t's j-th expert (ascending expert order)
 __global__ void __launch_bounds__(256)
-    k_pf_place(const int32_t *__restrict__ asc_e, const float *__restrict__ asc_w, int T,
-               const int32_t *__restrict__ chunk_off, const int32_t *__restrict__ ebase,
-               int32_t *__restrict__ pos, int32_t *__restrict__ perm, float *__restrict__ pw) {
+    k_pf_place(const int32_t *__restrict__ asc_e, int T, const int32_t *__restrict__ chunk_off,
+               const int32_t *__restrict__ ebase, int32_t *__restrict__ pos) {
   __shared__ uint32_t bits[kE][8];
   const int c = blockIdx.x;
   chunk_bits(asc_e, T, c, bits);
@@ -280,8 +280,6 @@ __global__ void __launch_bounds__(256)
     for (int w = 0; w < warp; ++w) rank += __popc(bits[e][w]);
     const int p = ebase[e] + chunk_off[(size_t)c * kE + e] + rank;
     pos[(size_t)tok * kTopK + j] = p;
-    perm[p] = tok;
-    pw[p] = asc_w[(size_t)tok * kTopK + j];
   }
 }
 
@@ -407,24 +405,24 @@ __global__ void __launch_bounds__(256)
 // in sorted order, rows [6T, 7T) every token for the shared expert.  Each
 // 8-element block is stored in the order 0,4,1,5,2,6,3,7.  Per row, rsc =
 // (2^F, 2^-E) for GEMM 1's read-out and rm3 = 2^E x routing weight for GEMM 2's.
-// One warp per row (grid-stride): each lane moves 8 16-byte chunks, all loads
-// issued before the first store.
+// One warp per token (grid-stride): the row is read and converted once and
+// written to its shared row and its six routed rows.
 __global__ void __launch_bounds__(256)
-    k_pf_gather(const uint16_t *__restrict__ x, int T, const int32_t *__restrict__ perm,
-                const float *__restrict__ pw, const float2 *__restrict__ xstat,
+    k_pf_gather(const uint16_t *__restrict__ x, int T, const int32_t *__restrict__ pos,
+                const float *__restrict__ asc_w, const float2 *__restrict__ xstat,
                 uint16_t *__restrict__ xp, float2 *__restrict__ rsc, float *__restrict__ rm3) {
   const int lane = threadIdx.x & 31;
-  const size_t rows = (size_t)7 * T;
-  const size_t nwarps = (size_t)gridDim.x * 8;
-  for (size_t row = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5); row < rows; row += nwarps) {
-    const bool routed = row < (size_t)6 * T;
-    const int tok = routed ? __ldg(perm + row) : (int)(row - (size_t)6 * T);
+  const int nwarps = gridDim.x * 8;
+  for (int tok = blockIdx.x * 8 + (threadIdx.x >> 5); tok < T; tok += nwarps) {
     const float2 st = __ldg(xstat + tok);
+    // lanes 0..5: the token's routed rows; lane 6: its shared row
+    int myrow = 0;
+    if (lane < kTopK) myrow = __ldg(pos + (size_t)tok * kTopK + lane);
+    else if (lane == kTopK) myrow = 6 * T + tok;
     const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)tok * kH);
     uint4 v[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) v[c] = ld_cg_v4(src + 32 * c + lane);
-    uint4 *dst = reinterpret_cast<uint4 *>(xp + row * kH);
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
       const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
@@ -435,12 +433,19 @@ __global__ void __launch_bounds__(256)
         h[2 * q + 1] = __half_as_ushort(__float2half_rn(__uint_as_float(w[q] & 0xffff0000u) * st.x));
       }
       // natural h[0..7] -> pairs (0,4), (1,5), (2,6), (3,7)
-      dst[32 * c + lane] = make_uint4(h[0] | (h[4] << 16), h[1] | (h[5] << 16), h[2] | (h[6] << 16),
-                                      h[3] | (h[7] << 16));
+      v[c] = make_uint4(h[0] | (h[4] << 16), h[1] | (h[5] << 16), h[2] | (h[6] << 16),
+                        h[3] | (h[7] << 16));
     }
-    if (lane == 0) {
-      rsc[row] = make_float2(1.f / st.x, 1.f / st.y);
-      rm3[row] = routed ? st.y * __ldg(pw + row) : st.y;
+#pragma unroll
+    for (int j = 0; j <= kTopK; ++j) {
+      const int row = __shfl_sync(0xffffffffu, myrow, j);
+      uint4 *dst = reinterpret_cast<uint4 *>(xp + (size_t)row * kH);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) dst[32 * c + lane] = v[c];
+    }
+    if (lane <= kTopK) {
+      rsc[myrow] = make_float2(1.f / st.x, 1.f / st.y);
+      rm3[myrow] = lane < kTopK ? st.y * __ldg(asc_w + (size_t)tok * kTopK + lane) : st.y;
     }
   }
 }
@@ -1169,7 +1174,43 @@ cudaError_t max_pairs(const void *fn, size_t smem, int *pairs) {
   return cudaSuccess;
 }
 
+// Stage timing for measurement (flint_debug_prefill_events): events recorded
+// on the call's stream between the stages of flint_moe_prefill.
+constexpr int kPfStages = 6;  // routing, sort, scaling + gather, GEMM 1, GEMM 2, combine
+std::mutex g_ev_mu;
+bool g_ev_on = false;
+int g_ev_dev = -1;
+cudaEvent_t g_ev[kPfStages + 1];
+
+void stage_mark(int i, cudaStream_t st) {
+  if (g_ev_on) cudaEventRecord(g_ev[i], st);
+}
+
 }  // namespace
+
+cudaError_t prefill_set_stage_events(int enable) {
+  std::lock_guard<std::mutex> lock(g_ev_mu);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (enable && g_ev_dev != dev) {
+    if (g_ev_dev >= 0) return cudaErrorInvalidDevice;  // events live on the first device used
+    for (int i = 0; i <= kPfStages; ++i)
+      if ((e = cudaEventCreate(&g_ev[i])) != cudaSuccess) return e;
+    g_ev_dev = dev;
+  }
+  g_ev_on = enable != 0;
+  return cudaSuccess;
+}
+
+cudaError_t prefill_stage_times(float *ms, int n) {
+  std::lock_guard<std::mutex> lock(g_ev_mu);
+  if (g_ev_dev < 0 || n < kPfStages) return cudaErrorInvalidValue;
+  cudaError_t e = cudaEventSynchronize(g_ev[kPfStages]);
+  for (int i = 0; i < kPfStages && e == cudaSuccess; ++i)
+    e = cudaEventElapsedTime(ms + i, g_ev[i], g_ev[i + 1]);
+  return e;
+}
 
 cudaError_t launch_route_many(const LayerArgs &L, const uint16_t *x, int T, int32_t *idx, float *w,
                               char *ws, cudaStream_t st) {
@@ -1202,8 +1243,6 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
   int32_t *co = reinterpret_cast<int32_t *>(ws + P.chunk_off);
   int32_t *ebase = reinterpret_cast<int32_t *>(ws + P.ebase);
   int32_t *ecount = reinterpret_cast<int32_t *>(ws + P.ecount);
-  int32_t *perm = reinterpret_cast<int32_t *>(ws + P.perm);
-  float *pw = reinterpret_cast<float *>(ws + P.pw);
   uint2 *tiles1 = reinterpret_cast<uint2 *>(ws + P.tiles1);
   uint2 *tiles2 = reinterpret_cast<uint2 *>(ws + P.tiles2);
   float4 *wst = reinterpret_cast<float4 *>(ws + P.wst);
@@ -1218,24 +1257,28 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
   uint16_t *ys = reinterpret_cast<uint16_t *>(ws + P.ys);
 
   // 1. routing
+  stage_mark(0, st);
   e = launch_route_many(L, x, T, reinterpret_cast<int32_t *>(ws + P.sel_idx),
                         reinterpret_cast<float *>(ws + P.sel_w), ws, st);
   if (e != cudaSuccess) return e;
+  stage_mark(1, st);
   // 2. stable sort by expert
   note_step("prefill sort launches");
   k_pf_count<<<P.nchunks, 256, 0, st>>>(asc_e, T, cc);
   k_pf_scan<<<1, 256, 0, st>>>(T, P.nchunks, cc, co, ebase, ecount, tiles1, tiles2, ctrl);
-  k_pf_place<<<P.nchunks, 256, 0, st>>>(asc_e, asc_w, T, co, ebase, pos, perm, pw);
+  k_pf_place<<<P.nchunks, 256, 0, st>>>(asc_e, T, co, ebase, pos);
+  stage_mark(2, st);
   // 3. power-of-two shifts of the fp16 operands, and the fp16 token rows
   note_step("prefill operand scaling launches");
   k_pf_wstats<<<kE + 1, 256, 0, st>>>(L.w13_s, L.w2_s, L.sh13_s, L.sh2_s, wst, wbound);
   k_pf_xstats<<<(T + 7) / 8, 256, 0, st>>>(x, T, wbound, xstat);
   {
-    int blocks = (int)(((size_t)7 * T + 7) / 8);  // 8 rows (warps) per block
+    int blocks = (T + 7) / 8;  // 8 tokens (warps) per block
     if (blocks > 148 * 8) blocks = 148 * 8;
-    k_pf_gather<<<blocks, 256, 0, st>>>(x, T, perm, pw, xstat, xp, rsc, rm3);
+    k_pf_gather<<<blocks, 256, 0, st>>>(x, T, pos, asc_w, xstat, xp, rsc, rm3);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  stage_mark(3, st);
   // 4. tensor maps and the two grouped GEMMs
   CUtensorMap mA1r, mA1s, mB1, mA2r, mA2s, mB2r, mB2s;
   note_step("prefill tensor maps");
@@ -1265,11 +1308,13 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
   k_pf_gemm<1><<<2 * min(P.max_tiles1, pairs1), kGemmThreads, GemmCfg<1>::kSmem, st>>>(
       mA1r, mA1s, mB1, mB1, a1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  stage_mark(4, st);
   GemmArgs a2{tiles2, ctrl, 4, ebase, ecount, T, L.w2_s, L.sh2_s, wst, rsc, rm3, yw, ys, ctrl + 1};
   note_step("prefill GEMM 2 launch");
   k_pf_gemm<2><<<2 * min(P.max_tiles2, pairs2), kGemmThreads, GemmCfg<2>::kSmem, st>>>(
       mA2r, mA2s, mB2r, mB2s, a2);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  stage_mark(5, st);
   // 5. combine
   note_step("prefill combine launch");
   {
@@ -1277,6 +1322,7 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
     if (blocks > 148 * 16) blocks = 148 * 16;
     k_pf_combine<<<blocks, 256, 0, st>>>(pos, yw, ys, T, out);
   }
+  stage_mark(6, st);
   return cudaGetLastError();
 }
 
