@@ -184,12 +184,14 @@ FLINT_API int flint_moe_decode_residual(const flint_moe_layer *layer, float *h, 
 /*
  * Prefill of the MoE block for T >= 1 tokens: the same function as
  * flint_moe_decode row by row, computed as routing for T tokens, a stable
- * token-by-expert sort, grouped GEMMs on the tensor cores (weights
- * dequantized to bf16 tiles in shared memory; bf16 SwiGLU intermediate) and a
- * fixed-order combine.
+ * token-by-expert sort, grouped GEMMs on the tensor cores and a fixed-order
+ * combine.  The GEMMs multiply exact fp16 operands (code x scale with a
+ * power-of-two shift per weight matrix; token rows with one per token) in one
+ * fp32 accumulation per output; the SwiGLU intermediate is rounded once, to
+ * fp16 after a per-token power-of-two shift from a bound it cannot exceed.
  *   x bf16 [T][2048];  out bf16 [T][2048] (may not alias x);  1 <= T <= 2^20
- *   ws workspace of flint_workspace_bytes(FLINT_OP_PREFILL, T) (about 70 KB
- *      per token: routing tables, the gathered rows, the SwiGLU and expert
+ *   ws workspace of flint_workspace_bytes(FLINT_OP_PREFILL, T) (about 65 KB
+ *      per token: routing tables, the fp16 token rows, the SwiGLU and expert
  *      outputs)
  */
 FLINT_API int flint_moe_prefill(const flint_moe_layer *layer, const uint16_t *x, int T, uint16_t *out,

@@ -7,22 +7,24 @@
 //      top-6 with the same selection rule as decode;
 //   2. a stable token-by-expert counting sort: per-chunk bitmask counts, one
 //      scan over (expert, chunk), then positions in token order inside every
-//      expert; each expert's group is padded to the 128-token tile;
-//   3. a gather of the routed token rows;
+//      expert, and the GEMM tile lists;
+//   3. power-of-two shifts that make both GEMM operands exact fp16 values,
+//      and the fp16 token rows (each token's shared row and its six routed
+//      rows in sorted order);
 //   4. grouped GEMM 1 (gate/up + SwiGLU) and grouped GEMM 2 (down, scaled by
-//      the routing weight) on the tcgen05 tensor cores: the weights are the
-//      128-row A operand, their int4 codes land in shared memory by TMA and
-//      four warps dequantize them to bf16 tiles in the 128-byte-swizzled
-//      K-major layout the MMA reads; the tokens are the N operand, loaded by
-//      TMA; the fp32 accumulator lives in tensor memory.  The shared expert
-//      is one more group that covers every token;
+//      the routing weight) on the tcgen05 tensor cores, by pairs of CTAs: the
+//      int4 codes land in shared memory by TMA and four warps per CTA turn
+//      them into the fp16 weight tile in tensor memory, the token tile is
+//      loaded by TMA in two halves (one per CTA), and one MMA instruction
+//      covers 256 weight rows; the fp32 accumulator lives in tensor memory.
+//      The shared expert is one more group that covers every token;
 //   5. a fixed-order combine per token (its experts in ascending index, then
 //      the shared expert).
 // "What vLLM changed" on the same page: the small-batch MoE kernels that read
-// only the selected experts were also the largest prefill gain.  SwiGLU
-// intermediates travel as hi/lo bf16 pairs: bf16 range (TandemLLM "21 Flint",
-// section 21.2 reports routed activations up to 2.6e5, past fp16) with about
-// 16 significant bits.
+// only the selected experts were also the largest prefill gain.  The SwiGLU
+// intermediate is fp16 after a per-token shift from a bound it cannot exceed
+// (TandemLLM "21 Flint", section 21.2 reports routed activations up to 2.6e5,
+// past the unscaled fp16 range).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 

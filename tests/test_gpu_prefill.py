@@ -100,7 +100,8 @@ def test_prefill_deterministic_and_consistent_with_decode(layer0):
 
 def test_prefill_large_activations(layer0):
     """x scaled by 512 (exact in bf16): routed SwiGLU intermediates reach ~1e5
-    (past the fp16 range); the bf16 hi/lo intermediate keeps the bound."""
+    (past the unscaled fp16 range); the per-token shift of the fp16
+    intermediate keeps the bound."""
     x = synth.prefill_x(40, 4040)
     xs = synth.bf16_bits(synth.bf16_to_f64(x) * 512.0)
     out = prefill(layer0, xs)
@@ -113,8 +114,8 @@ def test_prefill_large_activations(layer0):
 
 
 def test_prefill_one_row_repeated(layer0):
-    """1,000 copies of one token: its 6 experts get 1,000 tokens each (eight
-    128-token tiles per expert), the other 250 none; every output row equals
+    """1,000 copies of one token: its 6 experts get 1,000 tokens each (four
+    256-token tiles per expert), the other 250 none; every output row equals
     the single-row oracle result."""
     T = 1000
     x1 = synth.prefill_x(1, 9001)
