@@ -79,6 +79,49 @@ def test_prefill_2048_sampled_rows(layer0):
     check_close(bf16_to_f64(out[rows]), ref, keep)
 
 
+@pytest.mark.parametrize("T", [4096, 32768])
+def test_prefill_full_size_sampled_rows(layer0, T):
+    """The 4,096- and 32,768-token workloads as the bench runs them (every
+    expert's group spans several 256-token tiles; both GEMMs run on all CTA
+    pairs): 24 sampled rows (first, last and a stride) against the oracle."""
+    x = synth.prefill_x(T, T)
+    out = prefill(layer0, x)
+    rows = sorted(set([0, 1, T - 1] + list(range(7, T, T // 21))))
+    ref, idx, w, gap = oracle.moe_layer(layer0["O"], x[rows])
+    ridx, _ = route(layer0, x)
+    keep = routing_rows(ridx[rows], idx, gap)
+    assert len(keep) >= len(rows) - 1
+    worst = check_close(bf16_to_f64(out[rows]), ref, keep)
+    print(f"prefill T={T} sampled: worst |err|/bound = {worst:.3e}")
+
+
+def test_prefill_stage_events(layer0):
+    """The measurement hook: six positive stage times whose sum matches the
+    call's own event timing."""
+    T = 2048
+    x = dev_bf16(synth.prefill_x(T, T))
+    out = torch().empty((T, 2048), dtype=torch().int16, device="cuda")
+    nb = F.flint_workspace_bytes(F.FLINT_OP_PREFILL, T)
+    ws = torch().zeros(nb, dtype=torch().uint8, device="cuda")
+    F.flint_workspace_init(ws, nb)
+    F.flint_moe_prefill(layer0["L"], x, T, out, ws, nb)  # warm-up
+    e0, e1 = torch().cuda.Event(enable_timing=True), torch().cuda.Event(enable_timing=True)
+    F.flint_debug_prefill_events(True)
+    try:
+        e0.record()
+        F.flint_moe_prefill(layer0["L"], x, T, out, ws, nb)
+        e1.record()
+        stages = F.flint_debug_prefill_stage_ms()
+    finally:
+        F.flint_debug_prefill_events(False)
+    e1.synchronize()
+    total = e0.elapsed_time(e1)
+    assert list(stages) == list(F.PREFILL_STAGES)
+    assert all(v > 0 for v in stages.values())
+    assert sum(stages.values()) <= total * 1.05 + 0.01
+    assert sum(stages.values()) >= total * 0.5
+
+
 def test_prefill_deterministic_and_consistent_with_decode(layer0):
     x = synth.prefill_x(16, 77)
     a = prefill(layer0, x)
