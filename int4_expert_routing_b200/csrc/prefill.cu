@@ -2,9 +2,9 @@
 //
 // The block is defined per token ("How to Run Flint Locally", section "The
 // architecture, from config.json"); for many tokens it is computed as
-//   1. router logits for all tokens (bf16 products on mma.sync, fp32
-//      partials of each 128-wide k-group summed in fp64) and a per-token
-//      top-6 with the same selection rule as decode;
+//   1. router logits for all tokens (bf16 products on the tcgen05 tensor
+//      cores, fp32 partials of each 128-wide k-group summed in fp64) and a
+//      per-token top-6 with the same selection rule as decode;
 //   2. a stable token-by-expert counting sort: per-chunk bitmask counts, one
 //      scan over (expert, chunk), then positions in token order inside every
 //      expert, and the GEMM tile lists;
@@ -35,74 +35,7 @@
 
 namespace flint {
 
-// ============================================================== router (T tokens)
-constexpr int kRtTok = 64;  // tokens per CTA (8 column blocks of 8)
-
-// 16 warps: warp w multiplies experts 16w .. 16w+15 against the CTA's 64 tokens.
-__global__ void __launch_bounds__(512)
-    k_pf_router(LayerArgs L, const uint16_t *__restrict__ x, int T, float *__restrict__ z) {
-  // fragment of one k-half: [8 groups][8 blocks][4 words q][32 lanes] (uint4),
-  // so the 32 lanes of a load read 512 consecutive bytes
-  extern __shared__ __align__(128) unsigned char sm[];
-  uint4 *frag = reinterpret_cast<uint4 *>(sm);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-  const int t0 = blockIdx.x * kRtTok, e0 = 16 * warp;
-  double acc[8][4];
-#pragma unroll
-  for (int nb = 0; nb < 8; ++nb)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) acc[nb][i] = 0.0;
-
-  for (int half = 0; half < 2; ++half) {
-    __syncthreads();
-    for (int task = tid; task < 8 * 8 * 32 * 4; task += 512) {
-      const int ln = task & 31, q = (task >> 5) & 3, nb = (task >> 7) & 7, Gl = task >> 10;
-      const int tok = t0 + 8 * nb + (ln >> 2);
-      const int k0 = 128 * (8 * half + Gl) + 32 * (ln & 3) + 8 * q;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (tok < T) v = ld_cg_v4(x + (size_t)tok * kH + k0);
-      frag[task] = bf16x8_to_pairs(v);
-    }
-    __syncthreads();
-#pragma unroll 1
-    for (int Gl = 0; Gl < 8; ++Gl) {
-      const int G = 8 * half + Gl;
-      const uint16_t *ra = L.router_w + (size_t)(e0 + g) * kH + 128 * G + 32 * t;
-      uint32_t a[16], b[16];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 p0 = bf16x8_to_pairs(ld_stream(ra + 8 * q));
-        const uint4 p1 = bf16x8_to_pairs(ld_stream(ra + 8 * kH + 8 * q));
-        a[4 * q] = p0.x, a[4 * q + 1] = p0.y, a[4 * q + 2] = p0.z, a[4 * q + 3] = p0.w;
-        b[4 * q] = p1.x, b[4 * q + 1] = p1.y, b[4 * q + 2] = p1.z, b[4 * q + 3] = p1.w;
-      }
-#pragma unroll
-      for (int nb = 0; nb < 8; ++nb) {
-        uint32_t xb[16];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint4 v = frag[((Gl * 8 + nb) * 4 + q) * 32 + lane];
-          xb[4 * q] = v.x, xb[4 * q + 1] = v.y, xb[4 * q + 2] = v.z, xb[4 * q + 3] = v.w;
-        }
-        float d[4];
-        group_mma(a, b, xb, d);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[nb][i] += (double)d[i];
-      }
-    }
-  }
-#pragma unroll
-  for (int nb = 0; nb < 8; ++nb)
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const int tok = t0 + 8 * nb + 2 * t + c;
-      if (tok < T) {
-        z[(size_t)tok * kE + e0 + g] = (float)acc[nb][c];
-        z[(size_t)tok * kE + e0 + g + 8] = (float)acc[nb][2 + c];
-      }
-    }
-}
-
+// ============================================================== top-6 (T tokens)
 // One warp per token: sigmoid, bias, top-6 (lower index wins ties), weights;
 // selection order to sel_*, ascending expert order to asc_*.
 __global__ void __launch_bounds__(256)
@@ -1098,6 +1031,185 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// ============================================================== router on tcgen05
+// z[t][e] = sum over the 16 k-groups of the fp32 sum of the group's 128 bf16
+// products, the groups added in fp64 in order (the same rule as the decode
+// router).  One tile = 128 tokens (the MMA's M: the token rows, TMA) x 128
+// experts (its N: router rows, TMA), K in 128-wide groups; each group's MMAs
+// write one of two TMEM slots (so the next group runs while this one is read)
+// and eight epilogue warps add the slot into fp64 registers.
+constexpr int kRtM = 128, kRtN = 128;
+constexpr int kRtThreads = 384;  // warp 0 producer, warp 1 MMA, 2-3 idle, 4-11 epilogue
+constexpr int kRtStages = 3;
+constexpr int kRtAtom = 128 * 128;                 // 128 rows x 64 bf16 (one SW128 atom)
+constexpr int kRtStageBytes = 4 * kRtAtom;         // x: 2 atoms, W: 2 atoms
+constexpr size_t kRtSmem = (size_t)kRtStages * kRtStageBytes + 1024;
+constexpr int kRtRegCtl = 40, kRtRegEpi = 232;
+static_assert(128 * kRtRegCtl + 256 * kRtRegEpi <= 384 * 168, "router register split");
+
+FLINT_DEV void umma_bf16_ss(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                            uint32_t accum) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, "
+      "%3, p;\n}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum));
+}
+FLINT_DEV void umma_commit1(uint64_t *bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_addr(bar))
+      : "memory");
+}
+
+// Persistent: CTA c takes tiles c, c + grid, ...; tile i = token tile i / 2,
+// expert half i % 2.
+__global__ void __launch_bounds__(kRtThreads, 1)
+    k_pf_router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                   int T, float *__restrict__ z, uint32_t *status) {
+  extern __shared__ unsigned char smraw[];
+  unsigned char *sm = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full[kRtStages], empty[kRtStages], sfull[2], sempty[2], done;
+  __shared__ uint32_t s_tmem;
+  __shared__ volatile int s_fail;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int ntiles = 2 * ((T + kRtM - 1) / kRtM);
+  if ((int)blockIdx.x >= ntiles) return;
+  if (tid == 0) {
+    for (int s = 0; s < kRtStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sfull[b], 1);
+      mbar_init(&sempty[b], 8);  // one arrival per epilogue warp
+    }
+    mbar_init(&done, 1);
+    s_fail = 0;
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(&s_tmem)),
+                 "r"(256));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  constexpr int kG = kH / 128;  // 16 k-groups
+
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRtRegCtl));
+    if (warp == 0 && lane == 0) {
+      // ---- producer: the token rows and the router rows of each k-group
+      uint32_t it = 0;
+      for (int ti = blockIdx.x; ti < ntiles && !s_fail; ti += gridDim.x) {
+        const int t0 = kRtM * (ti >> 1), e0 = kRtN * (ti & 1);
+        for (int G = 0; G < kG; ++G, ++it) {
+          const int s = it % kRtStages;
+          if (it >= (uint32_t)kRtStages &&
+              !mbar_wait_sleep(&empty[s], ((it / kRtStages) - 1) & 1)) {
+            s_fail = 1;
+            break;
+          }
+          unsigned char *st = sm + (size_t)s * kRtStageBytes;
+          mbar_expect_tx(&full[s], kRtStageBytes);
+          tma_load_2d(st, &tmX, 128 * G, t0, &full[s]);
+          tma_load_2d(st + kRtAtom, &tmX, 128 * G + 64, t0, &full[s]);
+          tma_load_2d(st + 2 * kRtAtom, &tmW, 128 * G, e0, &full[s]);
+          tma_load_2d(st + 3 * kRtAtom, &tmW, 128 * G + 64, e0, &full[s]);
+        }
+      }
+    } else if (warp == 1 && lane == 0) {
+      // ---- MMA issuer: k-group number it writes TMEM slot it % 2
+      // kind::f16, A = B = bf16, D = f32, K-major, N = 128, M = 128
+      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kRtN >> 3) << 17) |
+                             ((uint32_t)(kRtM >> 4) << 24);
+      uint32_t it = 0;
+      for (int ti = blockIdx.x; ti < ntiles && !s_fail; ti += gridDim.x) {
+        bool ok = true;
+        for (int G = 0; G < kG; ++G, ++it) {
+          const int s = it % kRtStages, b = it & 1;
+          if ((it >= 2 && !mbar_wait(&sempty[b], ((it >> 1) - 1) & 1)) ||
+              !mbar_wait(&full[s], (it / kRtStages) & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = smem_addr(sm + (size_t)s * kRtStageBytes);
+#pragma unroll
+          for (int atom = 0; atom < 2; ++atom)
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              umma_bf16_ss(tmem + (uint32_t)(128 * b), sw128_desc(st + atom * kRtAtom + 32 * k),
+                           sw128_desc(st + (2 + atom) * kRtAtom + 32 * k), idesc, (atom | k) != 0);
+          umma_commit1(&empty[s]);  // the stage is free for the producer
+          umma_commit1(&sfull[b]);  // the group's fp32 partials are in slot b
+        }
+        if (!ok) {
+          s_fail = 1;
+          break;
+        }
+      }
+      umma_commit1(&done);  // every MMA completes before tensor memory is freed
+      if (!mbar_wait(&done, 0)) s_fail = 1;
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRtRegEpi));
+    // ---- epilogue warps 4..11: TMEM lane quarter (warp % 4) = tokens; expert
+    // half (warp - 4) / 4 of the tile's 128 experts (64 columns)
+    const int q4 = warp & 3, c_lo = 64 * ((warp - 4) >> 2);
+    uint32_t it = 0;
+    for (int ti = blockIdx.x; ti < ntiles; ti += gridDim.x) {
+      const int t0 = kRtM * (ti >> 1), e0 = kRtN * (ti & 1);
+      double acc[64];
+#pragma unroll
+      for (int j = 0; j < 64; ++j) acc[j] = 0.0;
+      bool ok = true;
+      for (int G = 0; G < kG; ++G, ++it) {
+        const int b = it & 1;
+        if (!mbar_wait_sleep(&sfull[b], (it >> 1) & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t base = tmem + (uint32_t)(128 * b + c_lo) + ((uint32_t)(32 * q4) << 16);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t v[32];
+          tmem_ld32_async(base + 32u * h, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) acc[32 * h + j] += (double)__uint_as_float(v[j]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sempty[b]);
+      }
+      if (!ok) {
+        s_fail = 1;
+        break;
+      }
+      const int tok = t0 + 32 * q4 + lane;
+      if (tok < T) {
+        float4 *zr = reinterpret_cast<float4 *>(z + (size_t)tok * kE + e0 + c_lo);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          zr[j] = make_float4((float)acc[4 * j], (float)acc[4 * j + 1], (float)acc[4 * j + 2],
+                              (float)acc[4 * j + 3]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (s_fail && tid == 0) set_status(status, kStatusTimeout);
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256));
+  }
+}
+
 // ============================================================== combine
 __global__ void __launch_bounds__(256)
     k_pf_combine(const int32_t *__restrict__ pos, const uint16_t *__restrict__ yw,
@@ -1218,12 +1330,24 @@ cudaError_t launch_route_many(const LayerArgs &L, const uint16_t *x, int T, int3
                               char *ws, cudaStream_t st) {
   const PrefillLayout P = prefill_layout(T);
   float *z = reinterpret_cast<float *>(ws + P.z);
-  note_step("prefill router attribute");
-  cudaError_t e = cudaFuncSetAttribute(k_pf_router, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       8 * 8 * 32 * 64);
+  cudaError_t e = noted(get_encode(), "cuTensorMapEncodeTiled entry point");
   if (e != cudaSuccess) return e;
+  note_step("prefill router tensor maps");
+  CUtensorMap mX, mW;
+  const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if ((e = make_map(&mX, x, BF, kH, (uint64_t)T, kH * 2, 64, kRtM, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+      (e = make_map(&mW, L.router_w, BF, kH, kE, kH * 2, 64, kRtN, CU_TENSOR_MAP_SWIZZLE_128B)))
+    return e;
+  note_step("prefill router attribute");
+  if ((e = cudaFuncSetAttribute(k_pf_router_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kRtSmem)) != cudaSuccess)
+    return e;
   note_step("prefill router launch");
-  k_pf_router<<<(T + kRtTok - 1) / kRtTok, 512, 8 * 8 * 32 * 64, st>>>(L, x, T, z);
+  {
+    const int ntiles = 2 * ((T + kRtM - 1) / kRtM);
+    k_pf_router_tc<<<ntiles < 148 ? ntiles : 148, kRtThreads, kRtSmem, st>>>(
+        mX, mW, T, z, reinterpret_cast<uint32_t *>(ws + P.ctrl) + 1);
+  }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   note_step("prefill top-6 launch");
   k_pf_topk<<<(T + 7) / 8, 256, 0, st>>>(L.router_b, z, T, idx, w,
