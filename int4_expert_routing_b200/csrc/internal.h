@@ -51,7 +51,7 @@ constexpr int kPfN2 = 256;
 constexpr int kPfChunk = 256;
 struct PrefillLayout {
   size_t ctrl, z, sel_idx, sel_w, asc_e, asc_w, route_total;
-  size_t pos, chunk_cnt, chunk_off, ebase, ecount, tiles1, tiles2, wst, wbound, xstat,
+  size_t pos, chunk_cnt, chunk_off, ebase, ecount, tiles1, tiles2, wst, wbound,
       rsc, rm3, xp, hr, hs, yw, ys, total;
   int mr, max_tiles1, max_tiles2, nchunks;
 };
@@ -87,7 +87,6 @@ inline PrefillLayout prefill_layout(int T) {
   L.tiles2 = take(sizeof(uint32_t) * 2 * (size_t)L.max_tiles2);
   L.wst = take(sizeof(float) * 4 * 257);   // per expert matrix pair: power-of-two shifts
   L.wbound = take(sizeof(float) * 257);    // per expert: bound factor of the SwiGLU output
-  L.xstat = take(sizeof(float) * 2 * (size_t)T);     // per token: 2^-F, 2^E
   L.rsc = take(sizeof(float) * 2 * (size_t)7 * T);   // per row: 2^F, 2^-E
   L.rm3 = take(sizeof(float) * (size_t)7 * T);       // per row: 2^E x routing weight
   L.xp = take(sizeof(uint16_t) * (size_t)7 * T * 2048);  // fp16 token rows: routed, then all T

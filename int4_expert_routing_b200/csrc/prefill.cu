@@ -292,14 +292,21 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// One warp per token: F puts max|x| in [2^14, 2^15); E puts the SwiGLU output
-// bound |x|^2 max_e wbound[e] below 2^15.  xstat[t] = (2^-F, 2^E).
+// Token rows as the fp16 operand of GEMM 1: rows [0, 6T) are the routed rows
+// in sorted order, rows [6T, 7T) every token for the shared expert.  One warp
+// per token (grid-stride) reads the row once and takes its shifts: F puts
+// max|x| in [2^14, 2^15) (the row is stored as x 2^-F, exact), E puts the
+// SwiGLU output bound |x|^2 max_e wbound[e] below 2^15.  The converted row is
+// written to its shared row and its six routed rows, each 8-element block in
+// the order 0,4,1,5,2,6,3,7.  Per row, rsc = (2^F, 2^-E) for GEMM 1's read-out
+// and rm3 = 2^E x routing weight for GEMM 2's.
 __global__ void __launch_bounds__(256)
-    k_pf_xstats(const uint16_t *__restrict__ x, int T, const float *__restrict__ wbound,
-                float2 *__restrict__ xstat) {
+    k_pf_gather(const uint16_t *__restrict__ x, int T, const int32_t *__restrict__ pos,
+                const float *__restrict__ asc_w, const float *__restrict__ wbound,
+                uint16_t *__restrict__ xp, float2 *__restrict__ rsc, float *__restrict__ rm3) {
   __shared__ float s_k;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (warp == 0) {
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x < 32) {  // the bound factor: the largest over the experts
     float k = 0.f;
     for (int i = lane; i <= kE; i += 32) k = fmaxf(k, wbound[i]);
 #pragma unroll
@@ -307,49 +314,8 @@ __global__ void __launch_bounds__(256)
     if (lane == 0) s_k = k;
   }
   __syncthreads();
-  const int t = blockIdx.x * 8 + warp;
-  if (t >= T) return;
-  const uint4 *row = reinterpret_cast<const uint4 *>(x + (size_t)t * kH);
-  float mx = 0.f;
-  double ss = 0.0;
-#pragma unroll
-  for (int c = 0; c < kH / 8 / 32; ++c) {
-    const uint4 v = ld_cg_v4(reinterpret_cast<const uint16_t *>(row + c * 32 + lane));
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float a = __uint_as_float(w[q] << 16), b = __uint_as_float(w[q] & 0xffff0000u);
-      mx = fmaxf(mx, fmaxf(fabsf(a), fabsf(b)));
-      ss += (double)a * a + (double)b * b;
-    }
-  }
-#pragma unroll
-  for (int o = 16; o; o >>= 1) {
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  }
-  if (lane == 0) {
-    const int F = mx > 0.f ? clamp_shift(ilogbf(mx) - 14) : 0;
-    const double bound = ss * (double)s_k * (1.0 + 1.0 / 1024);  // rounding margin
-    const int E = bound > 0.0 ? clamp_shift(ilogb(bound) + 1 - 15) : 0;
-    xstat[t] = make_float2(exp2i(-F), exp2i(E));
-  }
-}
-
-// Token rows as the fp16 operand of GEMM 1: rows [0, 6T) are the routed rows
-// in sorted order, rows [6T, 7T) every token for the shared expert.  Each
-// 8-element block is stored in the order 0,4,1,5,2,6,3,7.  Per row, rsc =
-// (2^F, 2^-E) for GEMM 1's read-out and rm3 = 2^E x routing weight for GEMM 2's.
-// One warp per token (grid-stride): the row is read and converted once and
-// written to its shared row and its six routed rows.
-__global__ void __launch_bounds__(256)
-    k_pf_gather(const uint16_t *__restrict__ x, int T, const int32_t *__restrict__ pos,
-                const float *__restrict__ asc_w, const float2 *__restrict__ xstat,
-                uint16_t *__restrict__ xp, float2 *__restrict__ rsc, float *__restrict__ rm3) {
-  const int lane = threadIdx.x & 31;
   const int nwarps = gridDim.x * 8;
   for (int tok = blockIdx.x * 8 + (threadIdx.x >> 5); tok < T; tok += nwarps) {
-    const float2 st = __ldg(xstat + tok);
     // lanes 0..5: the token's routed rows; lane 6: its shared row
     int myrow = 0;
     if (lane < kTopK) myrow = __ldg(pos + (size_t)tok * kTopK + lane);
@@ -358,14 +324,35 @@ __global__ void __launch_bounds__(256)
     uint4 v[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) v[c] = ld_cg_v4(src + 32 * c + lane);
+    float mx = 0.f;
+    double ss = 0.0;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float a = __uint_as_float(w[q] << 16), b = __uint_as_float(w[q] & 0xffff0000u);
+        mx = fmaxf(mx, fmaxf(fabsf(a), fabsf(b)));
+        ss += (double)a * a + (double)b * b;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    }
+    const int F = mx > 0.f ? clamp_shift(ilogbf(mx) - 14) : 0;
+    const double bound = ss * (double)s_k * (1.0 + 1.0 / 1024);  // rounding margin
+    const int E = bound > 0.0 ? clamp_shift(ilogb(bound) + 1 - 15) : 0;
+    const float xs = exp2i(-F);
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
       const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
       uint32_t h[8];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        h[2 * q] = __half_as_ushort(__float2half_rn(__uint_as_float(w[q] << 16) * st.x));
-        h[2 * q + 1] = __half_as_ushort(__float2half_rn(__uint_as_float(w[q] & 0xffff0000u) * st.x));
+        h[2 * q] = __half_as_ushort(__float2half_rn(__uint_as_float(w[q] << 16) * xs));
+        h[2 * q + 1] = __half_as_ushort(__float2half_rn(__uint_as_float(w[q] & 0xffff0000u) * xs));
       }
       // natural h[0..7] -> pairs (0,4), (1,5), (2,6), (3,7)
       v[c] = make_uint4(h[0] | (h[4] << 16), h[1] | (h[5] << 16), h[2] | (h[6] << 16),
@@ -379,8 +366,8 @@ __global__ void __launch_bounds__(256)
       for (int c = 0; c < 8; ++c) dst[32 * c + lane] = v[c];
     }
     if (lane <= kTopK) {
-      rsc[myrow] = make_float2(1.f / st.x, 1.f / st.y);
-      rm3[myrow] = lane < kTopK ? st.y * __ldg(asc_w + (size_t)tok * kTopK + lane) : st.y;
+      rsc[myrow] = make_float2(exp2i(F), exp2i(-E));
+      rm3[myrow] = lane < kTopK ? exp2i(E) * __ldg(asc_w + (size_t)tok * kTopK + lane) : exp2i(E);
     }
   }
 }
@@ -1373,7 +1360,6 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
   uint2 *tiles2 = reinterpret_cast<uint2 *>(ws + P.tiles2);
   float4 *wst = reinterpret_cast<float4 *>(ws + P.wst);
   float *wbound = reinterpret_cast<float *>(ws + P.wbound);
-  float2 *xstat = reinterpret_cast<float2 *>(ws + P.xstat);
   float2 *rsc = reinterpret_cast<float2 *>(ws + P.rsc);
   float *rm3 = reinterpret_cast<float *>(ws + P.rm3);
   uint16_t *xp = reinterpret_cast<uint16_t *>(ws + P.xp);
@@ -1397,11 +1383,10 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
   // 3. power-of-two shifts of the fp16 operands, and the fp16 token rows
   note_step("prefill operand scaling launches");
   k_pf_wstats<<<kE + 1, 256, 0, st>>>(L.w13_s, L.w2_s, L.sh13_s, L.sh2_s, wst, wbound);
-  k_pf_xstats<<<(T + 7) / 8, 256, 0, st>>>(x, T, wbound, xstat);
   {
     int blocks = (T + 7) / 8;  // 8 tokens (warps) per block
     if (blocks > 148 * 8) blocks = 148 * 8;
-    k_pf_gather<<<blocks, 256, 0, st>>>(x, T, pos, asc_w, xstat, xp, rsc, rm3);
+    k_pf_gather<<<blocks, 256, 0, st>>>(x, T, pos, asc_w, wbound, xp, rsc, rm3);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   stage_mark(3, st);
