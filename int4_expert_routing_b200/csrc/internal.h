@@ -87,7 +87,7 @@ inline PrefillLayout prefill_layout(int T) {
   L.tiles2 = take(sizeof(uint32_t) * 2 * (size_t)L.max_tiles2);
   L.wst = take(sizeof(float) * 4 * 257);   // per expert matrix pair: power-of-two shifts
   L.wbound = take(sizeof(float) * 257);    // per expert: bound factor of the SwiGLU output
-  L.rsc = take(sizeof(float) * 2 * (size_t)7 * T);   // per row: 2^F, 2^-E
+  L.rsc = take(sizeof(uint32_t) * (size_t)7 * T);    // per row: F | E << 16
   L.rm3 = take(sizeof(float) * (size_t)7 * T);       // per row: 2^E x routing weight
   L.xp = take(sizeof(uint16_t) * (size_t)7 * T * 2048);  // fp16 token rows: routed, then all T
   L.hr = take(sizeof(uint16_t) * (size_t)L.mr * 512);    // fp16 SwiGLU intermediate, routed

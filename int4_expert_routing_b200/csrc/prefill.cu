@@ -298,12 +298,12 @@ __global__ void __launch_bounds__(256)
 // max|x| in [2^14, 2^15) (the row is stored as x 2^-F, exact), E puts the
 // SwiGLU output bound |x|^2 max_e wbound[e] below 2^15.  The converted row is
 // written to its shared row and its six routed rows, each 8-element block in
-// the order 0,4,1,5,2,6,3,7.  Per row, rsc = (2^F, 2^-E) for GEMM 1's read-out
-// and rm3 = 2^E x routing weight for GEMM 2's.
+// the order 0,4,1,5,2,6,3,7.  Per row, rsc = (F, E) for GEMM 1's read-out
+// (multipliers 2^F and 2^-E) and rm3 = 2^E x routing weight for GEMM 2's.
 __global__ void __launch_bounds__(256)
     k_pf_gather(const uint16_t *__restrict__ x, int T, const int32_t *__restrict__ pos,
                 const float *__restrict__ asc_w, const float *__restrict__ wbound,
-                uint16_t *__restrict__ xp, float2 *__restrict__ rsc, float *__restrict__ rm3) {
+                uint16_t *__restrict__ xp, uint32_t *__restrict__ rsc, float *__restrict__ rm3) {
   __shared__ float s_k;
   const int lane = threadIdx.x & 31;
   if (threadIdx.x < 32) {  // the bound factor: the largest over the experts
@@ -366,7 +366,7 @@ __global__ void __launch_bounds__(256)
       for (int c = 0; c < 8; ++c) dst[32 * c + lane] = v[c];
     }
     if (lane <= kTopK) {
-      rsc[myrow] = make_float2(exp2i(F), exp2i(-E));
+      rsc[myrow] = ((uint32_t)F & 0xffffu) | ((uint32_t)E << 16);
       rm3[myrow] = lane < kTopK ? exp2i(E) * __ldg(asc_w + (size_t)tok * kTopK + lane) : exp2i(E);
     }
   }
@@ -406,28 +406,30 @@ constexpr int kRegCtl = 40, kRegDeq = 88, kRegEpi = 184;
 static_assert(128 * kRegCtl + 128 * kRegDeq + 256 * kRegEpi <= 65536, "register split");
 constexpr int kTmemCols = 512;
 
-// kN tokens per tile, kAcc accumulators of kN columns, kNA weight tiles of 64
-// columns (128 fp16 k values per row) in TMEM; two rings in shared memory, one
-// 128-wide k-group per stage: kS half token tiles (freed when the MMAs that
-// read them complete) and kR int4-code tiles (freed once the dequant warps
-// have read them, so the codes run ahead of the MMAs).
+// kN tokens per tile, kAcc accumulators of kN columns, kNA weight tiles in
+// TMEM; a stage is kKS = 2 k-groups of 128 (one wait and one commit per 16
+// MMAs), with two rings in shared memory: kS half token tiles (freed when the
+// MMAs that read them complete) and kR int4-code tiles (freed once the
+// dequant warps have read them, so the codes run ahead of the MMAs).
 template <int kMode>
 struct GemmCfg {
   static constexpr int kN = kMode == 1 ? kPfN1 : kPfN2;
   static constexpr int kAcc = 1;
-  static constexpr int kNA = 4;
-  static constexpr int kS = 6;
-  static constexpr int kR = 3;
+  static constexpr int kKS = 2;   // k-groups per stage
+  static constexpr int kNA = 2;   // weight tiles (one stage each: 128 TMEM columns)
+  static constexpr int kS = 3;
+  static constexpr int kR = 2;
   static constexpr int kBRows = kN / 2;       // token rows per CTA (the TMA box height)
   static constexpr int kBAtom = kBRows * 128;  // kN / 2 token rows x 64 fp16
-  static constexpr int kBStage = 2 * kBAtom;
-  static constexpr size_t kSmem = (size_t)kS * kBStage + (size_t)kR * kRawBytes + 1024;
+  static constexpr int kBStage = kKS * 2 * kBAtom;
+  static constexpr int kRawStage = kKS * kRawBytes;
+  static constexpr size_t kSmem = (size_t)kS * kBStage + (size_t)kR * kRawStage + 1024;
   static constexpr size_t b_off(int s) { return (size_t)s * kBStage; }
-  static constexpr size_t raw_off(int r) { return (size_t)kS * kBStage + (size_t)r * kRawBytes; }
-  // TMEM columns: the accumulator 0..255, the weight tiles at 256, 320, 384, 448
+  static constexpr size_t raw_off(int r) { return (size_t)kS * kBStage + (size_t)r * kRawStage; }
+  // TMEM columns: the accumulator 0..255, the weight tiles at 256 and 384
   static constexpr uint32_t acc_col(int b) { return (uint32_t)(256 * b); }
-  static constexpr uint32_t a_col(int a) { return (uint32_t)(256 + 64 * a); }
-  static_assert(kN <= 256 && kAcc == 1 && kNA == 4, "tensor memory");
+  static constexpr uint32_t a_col(int a) { return (uint32_t)(256 + 64 * kKS * a); }
+  static_assert(kN <= 256 && kAcc == 1 && 256 + 64 * kKS * kNA <= kTmemCols, "tensor memory");
   static_assert(kBAtom % 1024 == 0 && kN % 32 == 0, "tile shape");
 };
 
@@ -441,7 +443,7 @@ struct GemmArgs {
   const uint16_t *sc_r;  // scales of the routed weight tensor
   const uint16_t *sc_s;  // scales of the shared expert's tensor
   const float4 *wst;     // per expert: 2^-S1, 2^S1, 2^-S2, 2^S2
-  const float2 *rsc;     // per row: 2^F, 2^-E
+  const uint32_t *rsc;   // per row: F | E << 16 (int16 each): multipliers 2^F, 2^-E
   const float *rm3;      // per row: 2^E x routing weight
   uint16_t *out_r;       // GEMM 1: Hr fp16 [6T][512]; GEMM 2: Yw bf16 [6T][2048]
   uint16_t *out_s;       // GEMM 1: Hs fp16 [T][1024]; GEMM 2: Ys bf16 [T][2048]
@@ -660,6 +662,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
               GemmArgs args) {
   using Cfg = GemmCfg<kMode>;
   constexpr int S = Cfg::kS, R = Cfg::kR, NA = Cfg::kNA, NACC = Cfg::kAcc, kN = Cfg::kN;
+  constexpr int KS = Cfg::kKS;
   constexpr int kHalf = kN / 2;
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>(
@@ -668,7 +671,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       accfull[NACC], accempty[NACC], mma_done;
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_fail, s_epi_fail;
-  __shared__ float2 s_mul[kN];  // per token of the tile: (2^F, 2^-E) or (2^E x weight, -)
+  __shared__ uint32_t s_mul[kN];  // per token of the tile: GEMM 1 F | E << 16; GEMM 2 2^E x weight
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_rank();
@@ -728,7 +731,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const CUtensorMap *tB = t.sh ? &tmB_s : &tmB_r;
         // this CTA's half of the token rows (GEMM 2's shared B is Hs)
         const int brow = ((kMode == 2 && t.sh) ? t.n0 : t.b_row) + (int)rank * (t.n_mma / 2);
-        for (int G = 0; G < t.ng; ++G, ++it) {
+        for (int G0 = 0; G0 < t.ng; G0 += KS, ++it) {
           const int s = it % S;
           if (it >= (uint32_t)S && !cwait_sleep(&empty[s], ((it / S) - 1) & 1)) {
             s_fail = 1;
@@ -737,9 +740,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           unsigned char *st = sm + Cfg::b_off(s);
           if (rank == 0) mbar_expect_tx(&full[s], 2 * Cfg::kBStage);  // both halves
           const uint32_t fb = full_cl + 8u * s;
-          tma_load_2d_pair(st, tB, G * 128, brow, fb);
-          tma_load_2d_pair(st + Cfg::kBAtom, tB, G * 128 + 64, brow, fb);
-          if (ti == pair) pf_mark(kMode, 0, G);
+#pragma unroll
+          for (int j = 0; j < 2 * KS; ++j)  // (group G0 + j / 2, atom j % 2)
+            tma_load_2d_pair(st + j * Cfg::kBAtom, tB, G0 * 128 + 64 * j, brow, fb);
+          if (ti == pair) pf_mark(kMode, 0, G0 / KS);
         }
       }
     } else if (warp == 2 && lane == 0) {
@@ -752,19 +756,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         PfTile t;
         if (!pf_tile<kMode>(args, w, rank, t)) continue;
         const CUtensorMap *tA = t.sh ? &tmA_s : &tmA_r;
-        for (int G = 0; G < t.ng; ++G, ++it) {
+        for (int G0 = 0; G0 < t.ng; G0 += KS, ++it) {
           const int r = it % R;
           if (it >= (uint32_t)R && !mbar_wait_sleep(&rempty[r], ((it / R) - 1) & 1)) {
             s_fail = 1;
             break;
           }
           unsigned char *rw = sm + Cfg::raw_off(r);
-          mbar_expect_tx(&rfull[r], kRawBytes);
-          if (kMode == 1) {  // gate rows then up rows, 128 codes (64 B) each
-            tma_load_2d(rw, tA, G * 64, t.row0, &rfull[r]);
-            tma_load_2d(rw + 64 * 64, tA, G * 64, t.row1, &rfull[r]);
-          } else {  // 128 rows x 128 codes
-            tma_load_2d(rw, tA, G * 64, t.row0, &rfull[r]);
+          mbar_expect_tx(&rfull[r], Cfg::kRawStage);
+#pragma unroll
+          for (int g = 0; g < KS; ++g) {  // group G0 + g at rw + g * kRawBytes
+            if (kMode == 1) {  // gate rows then up rows, 128 codes (64 B) each
+              tma_load_2d(rw + g * kRawBytes, tA, (G0 + g) * 64, t.row0, &rfull[r]);
+              tma_load_2d(rw + g * kRawBytes + 64 * 64, tA, (G0 + g) * 64, t.row1, &rfull[r]);
+            } else {  // 128 rows x 128 codes
+              tma_load_2d(rw + g * kRawBytes, tA, (G0 + g) * 64, t.row0, &rfull[r]);
+            }
           }
         }
       }
@@ -791,7 +798,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const uint32_t idesc =
             (1u << 4) | ((uint32_t)(t.n_mma >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
         bool ok = true;
-        for (int G = 0; G < t.ng; ++G, ++it) {
+        for (int G0 = 0; G0 < t.ng; G0 += KS, ++it) {
           const int s = it % S, a = it % NA;
           if (!cwait_sleep(&afull[a], (it / NA) & 1) || !cwait_sleep(&full[s], (it / S) & 1)) {
             ok = false;
@@ -801,16 +808,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           const uint32_t b_addr = smem_addr(sm + Cfg::b_off(s));
           const uint32_t a_tm = tmem + Cfg::a_col(a);
 #pragma unroll
-          for (int atom = 0; atom < 2; ++atom) {
+          for (int j = 0; j < 2 * KS; ++j) {  // (group G0 + j / 2, atom j % 2): 64 k each
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-              umma_f16_ts_pair(d, a_tm + 8u * (4 * atom + k),
-                               sw128_desc(b_addr + atom * Cfg::kBAtom + 32 * k), idesc,
-                               (G | atom | k) != 0);
+              umma_f16_ts_pair(d, a_tm + 8u * (4 * j + k),
+                               sw128_desc(b_addr + j * Cfg::kBAtom + 32 * k), idesc,
+                               (G0 | j | k) != 0);
           }
           umma_commit_pair(&empty[s]);   // both halves of the stage are free for the producers
           umma_commit_pair(&aempty[a]);  // both weight tiles are free for the dequant warps
-          if (ti == pair) pf_mark(kMode, 2, G);
+          if (ti == pair) pf_mark(kMode, 2, G0 / KS);
         }
         if (!ok) {
           s_fail = 1;
@@ -859,7 +866,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       fetch(wa, scn, muln);  // the next tile's, in flight during this one
       if (!valid) continue;
       bool ok = true;
-      for (int G = 0; G < t.ng; ++G, ++it) {
+      for (int G0 = 0; G0 < t.ng; G0 += KS, ++it) {
         const int rr = it % R, a = it % NA;
         if (!mbar_wait_sleep(&rfull[rr], (it / R) & 1) ||
             (it >= (uint32_t)NA && !cwait_sleep(&aempty[a], ((it / NA) - 1) & 1))) {
@@ -867,30 +874,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           break;
         }
         tc_fence_after();
-        // the group's scale s x 2^-S and its multipliers as fp16x2 (exact: 8
-        // significant bits; s 2^24 < 2^15 by the choice of S)
-        const uint32_t sw = scw[G >> 1] >> (16 * (G & 1));
-        const float sf = __uint_as_float(sw << 16) * smul;
-        const uint32_t h24 = __half_as_ushort(__float2half_rn(sf * 16777216.f));
-        const uint32_t h20 = __half_as_ushort(__float2half_rn(sf * 1048576.f));
-        const uint32_t hc8 = __half_as_ushort(__float2half_rn(sf * -8.f));
-        const uint32_t m24 = h24 | (h24 << 16), m20 = h20 | (h20 << 16), c8 = hc8 | (hc8 << 16);
-        const unsigned char *raw = sm + Cfg::raw_off(rr) + raw_row * 64;
-        const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + Cfg::a_col(a);
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {  // TMEM columns 32 hf .. 32 hf + 31: chunks 2 hf, 2 hf + 1
-          uint32_t v[32];
+        for (int g = 0; g < KS; ++g) {  // group G0 + g -> TMEM columns 64 g .. of the tile
+          const int G = G0 + g;
+          // the group's scale s x 2^-S and its multipliers as fp16x2 (exact: 8
+          // significant bits; s 2^24 < 2^15 by the choice of S)
+          const uint32_t sw = scw[G >> 1] >> (16 * (G & 1));
+          const float sf = __uint_as_float(sw << 16) * smul;
+          const uint32_t h24 = __half_as_ushort(__float2half_rn(sf * 16777216.f));
+          const uint32_t h20 = __half_as_ushort(__float2half_rn(sf * 1048576.f));
+          const uint32_t hc8 = __half_as_ushort(__float2half_rn(sf * -8.f));
+          const uint32_t m24 = h24 | (h24 << 16), m20 = h20 | (h20 << 16),
+                         c8 = hc8 | (hc8 << 16);
+          const unsigned char *raw = sm + Cfg::raw_off(rr) + g * kRawBytes + raw_row * 64;
+          const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + Cfg::a_col(a) + 64u * g;
 #pragma unroll
-          for (int jj = 0; jj < 2; ++jj) {
-            // chunk j = codes 32 j .. 32 j + 31 of the group -> columns 16 j ..
-            const int j = 2 * hf + jj;
-            const uint4 w = *reinterpret_cast<const uint4 *>(raw + 16 * j);
-            codes8_f16(w.x, m24, m20, c8, v + 16 * jj + 0);
-            codes8_f16(w.y, m24, m20, c8, v + 16 * jj + 4);
-            codes8_f16(w.z, m24, m20, c8, v + 16 * jj + 8);
-            codes8_f16(w.w, m24, m20, c8, v + 16 * jj + 12);
+          for (int hf = 0; hf < 2; ++hf) {  // columns 32 hf .. 32 hf + 31: chunks 2 hf, 2 hf + 1
+            uint32_t v[32];
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+              // chunk j = codes 32 j .. 32 j + 31 of the group -> columns 16 j ..
+              const int j = 2 * hf + jj;
+              const uint4 w = *reinterpret_cast<const uint4 *>(raw + 16 * j);
+              codes8_f16(w.x, m24, m20, c8, v + 16 * jj + 0);
+              codes8_f16(w.y, m24, m20, c8, v + 16 * jj + 4);
+              codes8_f16(w.z, m24, m20, c8, v + 16 * jj + 8);
+              codes8_f16(w.w, m24, m20, c8, v + 16 * jj + 12);
+            }
+            tmem_st32(tbase + 32u * hf, v);
           }
-          tmem_st32(tbase + 32u * hf, v);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -899,7 +911,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           mbar_arrive(&rempty[rr]);  // the codes are in registers and TMEM
           mbar_arrive_cluster(afull_cl + 8u * a);
         }
-        if (tid == 128 && ti == pair) pf_mark(kMode, 1, G);
+        if (tid == 128 && ti == pair) pf_mark(kMode, 1, G0 / KS);
       }
       if (!ok) {
         s_fail = 1;
@@ -928,11 +940,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       if (!pf_tile<kMode>(args, w, rank, t)) continue;
       const int b = tc % NACC;
       const float4 ws = __ldg(args.wst + t.e);
-      float2 pre = make_float2(0.f, 0.f);
-      if (et < t.n_valid) {
-        if (kMode == 1) pre = __ldg(args.rsc + t.b_row + et);
-        else pre.x = __ldg(args.rm3 + t.b_row + et);
-      }
+      uint32_t pre = 0u;
+      if (et < t.n_valid)
+        pre = kMode == 1 ? __ldg(args.rsc + t.b_row + et)
+                         : __float_as_uint(__ldg(args.rm3 + t.b_row + et));
       const bool ok = cwait_sleep(&accfull[b], (tc / NACC) & 1);
       tc_fence_after();
       uint32_t acc[kHalf];
@@ -980,10 +991,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             const float mine = __uint_as_float(up_lane ? acc[kQ + jj] : acc[jj]);
             const float theirs =
                 __shfl_xor_sync(0xffffffffu, __uint_as_float(up_lane ? acc[jj] : acc[kQ + jj]), 1);
-            const float2 rs = s_mul[c_lo + j0 + jj];
-            const float m = mw * rs.x;
+            const uint32_t fe = s_mul[c_lo + j0 + jj];  // F | E << 16
+            const float m = mw * exp2i((int)(int16_t)(fe & 0xffffu));
             const float g = (up_lane ? theirs : mine) * m, uu = (up_lane ? mine : theirs) * m;
-            const float h = __fdividef(g, 1.f + __expf(-g)) * uu * rs.y;  // silu(gate) * up / 2^E
+            const float h = __fdividef(g, 1.f + __expf(-g)) * uu *
+                            exp2i(-(int)(int16_t)(fe >> 16));  // silu(gate) * up / 2^E
             const uint32_t hv = __half_as_ushort(__float2half_rn(h));
             hp[u >> 1] = (u & 1) ? (hp[u >> 1] | (hv << 16)) : hv;
           }
@@ -1000,7 +1012,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                             : args.out_r + (size_t)t.b_row * kH + col;
 #pragma unroll
         for (int j = 0; j < kHalf; ++j) {
-          const float m = mw * s_mul[c_lo + j].x;
+          const float m = mw * __uint_as_float(s_mul[c_lo + j]);
           st_u16_if(yb + (size_t)(c_lo + j) * kH, f32_to_bf16_bits(__uint_as_float(acc[j]) * m), j < nv);
         }
       }
@@ -1360,7 +1372,7 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
   uint2 *tiles2 = reinterpret_cast<uint2 *>(ws + P.tiles2);
   float4 *wst = reinterpret_cast<float4 *>(ws + P.wst);
   float *wbound = reinterpret_cast<float *>(ws + P.wbound);
-  float2 *rsc = reinterpret_cast<float2 *>(ws + P.rsc);
+  uint32_t *rsc = reinterpret_cast<uint32_t *>(ws + P.rsc);
   float *rm3 = reinterpret_cast<float *>(ws + P.rm3);
   uint16_t *xp = reinterpret_cast<uint16_t *>(ws + P.xp);
   uint16_t *hr = reinterpret_cast<uint16_t *>(ws + P.hr);
