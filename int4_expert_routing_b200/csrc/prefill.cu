@@ -42,6 +42,8 @@ __global__ void __launch_bounds__(256)
     k_pf_topk(const float *__restrict__ router_b, const float *__restrict__ z, int T,
               int32_t *__restrict__ sel_idx, float *__restrict__ sel_w, int32_t *__restrict__ asc_e,
               float *__restrict__ asc_w) {
+  pdl_wait();  // the previous kernel in the stream is complete (programmatic launch)
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tok = blockIdx.x * 8 + warp;
   if (tok >= T) return;
@@ -112,6 +114,8 @@ FLINT_DEV void chunk_bits(const int32_t *asc_e, int T, int c, uint32_t (*bits)[8
 
 __global__ void __launch_bounds__(256)
     k_pf_count(const int32_t *__restrict__ asc_e, int T, int32_t *__restrict__ chunk_cnt) {
+  pdl_wait();  // the previous kernel in the stream is complete (programmatic launch)
+  pdl_trigger();
   __shared__ uint32_t bits[kE][8];
   chunk_bits(asc_e, T, blockIdx.x, bits);
   const int e = threadIdx.x;
@@ -160,6 +164,8 @@ __global__ void __launch_bounds__(256)
               int32_t *__restrict__ chunk_off, int32_t *__restrict__ ebase,
               int32_t *__restrict__ ecount, uint2 *__restrict__ tiles1,
               uint2 *__restrict__ tiles2, uint32_t *__restrict__ ctrl) {
+  pdl_wait();  // the previous kernel in the stream is complete (programmatic launch)
+  pdl_trigger();
   __shared__ int s_warp[8];
   const int e = threadIdx.x;
   int off = 0;
@@ -203,6 +209,8 @@ __global__ void __launch_bounds__(256)
 __global__ void __launch_bounds__(256)
     k_pf_place(const int32_t *__restrict__ asc_e, int T, const int32_t *__restrict__ chunk_off,
                const int32_t *__restrict__ ebase, int32_t *__restrict__ pos) {
+  pdl_wait();  // the previous kernel in the stream is complete (programmatic launch)
+  pdl_trigger();
   __shared__ uint32_t bits[kE][8];
   const int c = blockIdx.x;
   chunk_bits(asc_e, T, c, bits);
@@ -241,6 +249,8 @@ __global__ void __launch_bounds__(256)
     k_pf_wstats(const uint16_t *__restrict__ w13_s, const uint16_t *__restrict__ w2_s,
                 const uint16_t *__restrict__ sh13_s, const uint16_t *__restrict__ sh2_s,
                 float4 *__restrict__ wst, float *__restrict__ wbound) {
+  pdl_wait();  // the previous kernel in the stream is complete (programmatic launch)
+  pdl_trigger();
   __shared__ float red[4][8];
   const int e = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool sh = e == kE;
@@ -304,6 +314,8 @@ __global__ void __launch_bounds__(256)
     k_pf_gather(const uint16_t *__restrict__ x, int T, const int32_t *__restrict__ pos,
                 const float *__restrict__ asc_w, const float *__restrict__ wbound,
                 uint16_t *__restrict__ xp, uint32_t *__restrict__ rsc, float *__restrict__ rm3) {
+  pdl_wait();  // the previous kernel in the stream is complete (programmatic launch)
+  pdl_trigger();
   __shared__ float s_k;
   const int lane = threadIdx.x & 31;
   if (threadIdx.x < 32) {  // the bound factor: the largest over the experts
@@ -660,6 +672,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     k_pf_gemm(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
               const __grid_constant__ CUtensorMap tmB_r, const __grid_constant__ CUtensorMap tmB_s,
               GemmArgs args) {
+  pdl_wait();  // the previous kernel in the stream is complete (programmatic launch)
+  pdl_trigger();
   using Cfg = GemmCfg<kMode>;
   constexpr int S = Cfg::kS, R = Cfg::kR, NA = Cfg::kNA, NACC = Cfg::kAcc, kN = Cfg::kN;
   constexpr int KS = Cfg::kKS;
@@ -1065,6 +1079,8 @@ FLINT_DEV void umma_commit1(uint64_t *bar) {
 __global__ void __launch_bounds__(kRtThreads, 1)
     k_pf_router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                    int T, float *__restrict__ z, uint32_t *status) {
+  pdl_wait();  // the previous kernel in the stream is complete (programmatic launch)
+  pdl_trigger();
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
@@ -1213,6 +1229,8 @@ __global__ void __launch_bounds__(kRtThreads, 1)
 __global__ void __launch_bounds__(256)
     k_pf_combine(const int32_t *__restrict__ pos, const uint16_t *__restrict__ yw,
                  const uint16_t *__restrict__ ys, int T, uint16_t *__restrict__ out) {
+  pdl_wait();  // the previous kernel in the stream is complete (programmatic launch)
+  pdl_trigger();
   const size_t n = (size_t)T * (kH / 8);
   for (size_t i = (size_t)blockIdx.x * 256 + threadIdx.x; i < n; i += (size_t)gridDim.x * 256) {
     const size_t tok = i / (kH / 8), c = i % (kH / 8);
@@ -1265,6 +1283,25 @@ cudaError_t make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, u
                               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// Every prefill kernel is launched with programmatic stream serialization: its
+// CTAs may be scheduled while the previous kernel drains, and each waits
+// (griddepcontrol.wait, first thing) until that kernel is complete.
+template <typename... KArgs, typename... Args>
+cudaError_t pf_launch(void (*kernel)(KArgs...), int grid, int block, size_t smem, cudaStream_t st,
+                      Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
 // Clusters of two GEMM CTAs that can be resident at once on this device.
@@ -1344,15 +1381,13 @@ cudaError_t launch_route_many(const LayerArgs &L, const uint16_t *x, int T, int3
   note_step("prefill router launch");
   {
     const int ntiles = 2 * ((T + kRtM - 1) / kRtM);
-    k_pf_router_tc<<<ntiles < 148 ? ntiles : 148, kRtThreads, kRtSmem, st>>>(
-        mX, mW, T, z, reinterpret_cast<uint32_t *>(ws + P.ctrl) + 1);
+    e = pf_launch(k_pf_router_tc, ntiles < 148 ? ntiles : 148, kRtThreads, kRtSmem, st, mX, mW, T,
+                  z, reinterpret_cast<uint32_t *>(ws + P.ctrl) + 1);
   }
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (e != cudaSuccess) return e;
   note_step("prefill top-6 launch");
-  k_pf_topk<<<(T + 7) / 8, 256, 0, st>>>(L.router_b, z, T, idx, w,
-                                          reinterpret_cast<int32_t *>(ws + P.asc_e),
-                                          reinterpret_cast<float *>(ws + P.asc_w));
-  return cudaGetLastError();
+  return pf_launch(k_pf_topk, (T + 7) / 8, 256, 0, st, L.router_b, z, T, idx, w,
+                   reinterpret_cast<int32_t *>(ws + P.asc_e), reinterpret_cast<float *>(ws + P.asc_w));
 }
 
 cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_t *out, char *ws,
@@ -1388,17 +1423,22 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
   stage_mark(1, st);
   // 2. stable sort by expert
   note_step("prefill sort launches");
-  k_pf_count<<<P.nchunks, 256, 0, st>>>(asc_e, T, cc);
-  k_pf_scan<<<1, 256, 0, st>>>(T, P.nchunks, cc, co, ebase, ecount, tiles1, tiles2, ctrl);
-  k_pf_place<<<P.nchunks, 256, 0, st>>>(asc_e, T, co, ebase, pos);
+  if ((e = pf_launch(k_pf_count, P.nchunks, 256, 0, st, asc_e, T, cc)) ||
+      (e = pf_launch(k_pf_scan, 1, 256, 0, st, T, P.nchunks, cc, co, ebase, ecount, tiles1, tiles2,
+                     ctrl)) ||
+      (e = pf_launch(k_pf_place, P.nchunks, 256, 0, st, asc_e, T, co, ebase, pos)))
+    return e;
   stage_mark(2, st);
   // 3. power-of-two shifts of the fp16 operands, and the fp16 token rows
   note_step("prefill operand scaling launches");
-  k_pf_wstats<<<kE + 1, 256, 0, st>>>(L.w13_s, L.w2_s, L.sh13_s, L.sh2_s, wst, wbound);
+  if ((e = pf_launch(k_pf_wstats, kE + 1, 256, 0, st, L.w13_s, L.w2_s, L.sh13_s, L.sh2_s, wst,
+                     wbound)))
+    return e;
   {
     int blocks = (T + 7) / 8;  // 8 tokens (warps) per block
     if (blocks > 148 * 8) blocks = 148 * 8;
-    k_pf_gather<<<blocks, 256, 0, st>>>(x, T, pos, asc_w, wbound, xp, rsc, rm3);
+    if ((e = pf_launch(k_pf_gather, blocks, 256, 0, st, x, T, pos, asc_w, wbound, xp, rsc, rm3)))
+      return e;
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   stage_mark(3, st);
@@ -1428,22 +1468,22 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
     return e;
   GemmArgs a1{tiles1, ctrl, 3, ebase, ecount, T, L.w13_s, L.sh13_s, wst, rsc, rm3, hr, hs, ctrl + 1};
   note_step("prefill GEMM 1 launch");
-  k_pf_gemm<1><<<2 * min(P.max_tiles1, pairs1), kGemmThreads, GemmCfg<1>::kSmem, st>>>(
-      mA1r, mA1s, mB1, mB1, a1);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  e = pf_launch(k_pf_gemm<1>, 2 * min(P.max_tiles1, pairs1), kGemmThreads, GemmCfg<1>::kSmem, st,
+                mA1r, mA1s, mB1, mB1, a1);
+  if (e != cudaSuccess) return e;
   stage_mark(4, st);
   GemmArgs a2{tiles2, ctrl, 4, ebase, ecount, T, L.w2_s, L.sh2_s, wst, rsc, rm3, yw, ys, ctrl + 1};
   note_step("prefill GEMM 2 launch");
-  k_pf_gemm<2><<<2 * min(P.max_tiles2, pairs2), kGemmThreads, GemmCfg<2>::kSmem, st>>>(
-      mA2r, mA2s, mB2r, mB2s, a2);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  e = pf_launch(k_pf_gemm<2>, 2 * min(P.max_tiles2, pairs2), kGemmThreads, GemmCfg<2>::kSmem, st,
+                mA2r, mA2s, mB2r, mB2s, a2);
+  if (e != cudaSuccess) return e;
   stage_mark(5, st);
   // 5. combine
   note_step("prefill combine launch");
   {
     int blocks = (int)(((size_t)T * (kH / 8) + 255) / 256);
     if (blocks > 148 * 16) blocks = 148 * 16;
-    k_pf_combine<<<blocks, 256, 0, st>>>(pos, yw, ys, T, out);
+    if ((e = pf_launch(k_pf_combine, blocks, 256, 0, st, pos, yw, ys, T, out))) return e;
   }
   stage_mark(6, st);
   return cudaGetLastError();
