@@ -147,33 +147,6 @@ FLINT_DEV void group_mma_acc(const uint32_t (&ra)[16], const uint32_t (&rb)[16],
     mma_bf16_16816(d, ra[2 * s], rb[2 * s], ra[2 * s + 1], rb[2 * s + 1], xb[2 * s], xb[2 * s + 1]);
 }
 
-FLINT_DEV void load_frag(const uint4 *p, uint32_t (&x)[16]) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint4 v = p[i];
-    x[4 * i] = v.x;
-    x[4 * i + 1] = v.y;
-    x[4 * i + 2] = v.z;
-    x[4 * i + 3] = v.w;
-  }
-}
-
-// Activation fragment of `ngroups` groups for up to 8 bf16 rows, in shared
-// memory: frag[(G * 32 + lane) * 4 + q] holds, for column g = lane / 4 and
-// slice t = lane % 4, the pairs of elements 128G + 32t + 8q .. +7 of row g
-// (zero for g >= rows).  rowptr(g) returns the row's bf16 bits.
-template <typename RowPtr>
-FLINT_DEV void build_x_frag(uint4 *frag, int ngroups, int rows, RowPtr rowptr, int tid,
-                            int nthreads) {
-  for (int task = tid; task < ngroups * 128; task += nthreads) {
-    const int G = task >> 7, lane = (task >> 2) & 31, q = task & 3;
-    const int g = lane >> 2, t = lane & 3;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (g < rows) v = ld_cg_v4(rowptr(g) + 128 * G + 32 * t + 8 * q);
-    frag[task] = bf16x8_to_pairs(v);
-  }
-}
-
 // Position of element k (0 <= k < K) of a column inside a hi/lo fragment
 // image laid out [G][t][16 words] (one column): returns the bf16 slot index.
 FLINT_DEV int frag_slot(int k) {
@@ -219,9 +192,6 @@ FLINT_DEV void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *ba
       "l"(src), "r"(bytes), "r"(smem_addr(bar))
       : "memory");
 }
-// Order this thread's earlier generic-proxy shared-memory accesses before
-// later async-proxy (bulk copy / tensor core) accesses of the same memory.
-FLINT_DEV void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // One poll of phase `parity` of `bar`.
 FLINT_DEV bool mbar_try(uint64_t *bar, uint32_t parity) {

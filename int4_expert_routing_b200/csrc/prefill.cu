@@ -520,12 +520,13 @@ FLINT_DEV void cluster_sync_all() {
 FLINT_DEV void mbar_arrive_cluster(uint32_t cl_addr) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
 }
-// Waits on barriers that the other CTA of the pair or the pair's MMAs arrive
-// on: the default (CTA-scope) acquire, as for the other barriers; what must be
+// Wait on a barrier that the other CTA of the pair or the pair's MMAs arrive
+// on: the default (CTA-scope) acquire, as for the other barriers (what must be
 // ordered is tensor-memory and shared-memory state completed before the
-// arrival (tcgen05.wait / fence, TMA and MMA completion).
-FLINT_DEV bool cwait(uint64_t *bar, uint32_t parity) { return mbar_wait(bar, parity); }
+// arrival: tcgen05.wait / fence, TMA and MMA completion); the thread may
+// suspend until the phase completes.
 FLINT_DEV bool cwait_sleep(uint64_t *bar, uint32_t parity) { return mbar_wait_sleep(bar, parity); }
+
 // TMA tile load into this CTA's shared memory whose completion is counted on
 // an mbarrier of either CTA of the pair (`bar_cl`, a shared::cluster address)
 FLINT_DEV void tma_load_2d_pair(void *dst, const CUtensorMap *map, int x, int y, uint32_t bar_cl) {
