@@ -679,6 +679,9 @@ __global__ void __launch_bounds__(kK3Threads)
   __shared__ int s_ns;
   __shared__ uint32_t s_rows[kE];
   __shared__ int s_asc[kMaxB * kTopK];
+  // slot u's i-th row (ascending) b and the slot's place j among that row's
+  // experts (ascending), as b | j << 4
+  __shared__ uint8_t s_rbj[kMaxB * kTopK][kMaxB];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const int n0 = blockIdx.x * 16;
@@ -687,7 +690,10 @@ __global__ void __launch_bounds__(kK3Threads)
 
   // Routing is final here (K2 triggered this launch after its own wait on
   // K1): fetch the chosen experts' down rows before waiting on K2.
-  if (tid == 0) mbar_init(&bar, 1);
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    s_ns = 0;  // stays 0 if slot 0 is invalid (a routing left by a failed K1)
+  }
   __syncthreads();
   float h_old = 0.f;  // this thread's residual element (final: K1 waited for it)
   if (kResidual && tid < 16 * B) h_old = ld_cg_f32(h + (size_t)(tid >> 4) * kH + n0 + (tid & 15));
@@ -695,9 +701,10 @@ __global__ void __launch_bounds__(kK3Threads)
     const uint32_t word = ld_cg_u32(reinterpret_cast<const uint32_t *>(ws + lay.slot_word) + tid);
     // at most umax slots have room here; a routing left by a failed K1 may
     // hold more, and none of it is used after the status is set
+    s_rows[tid] = 0u;  // rows of an invalid slot: none
     if (word != kSlotInvalid && tid < umax) {
       const size_t e = slot_expert(word);
-      s_rows[tid] = slot_mask(word);
+      s_rows[tid] = slot_mask(word) & ((1u << B) - 1u);
       mbar_add_tx(&bar, 4096 + 128);
       bulk_g2s(wsm + tid * 4096, L.w2_q + (e * kH + n0) * (kI / 2), 4096, &bar);
       bulk_g2s(ssm + tid * 128, L.w2_s + (e * kH + n0) * (kI / kG), 128, &bar);
@@ -713,6 +720,16 @@ __global__ void __launch_bounds__(kK3Threads)
   }
   __syncthreads();
   if (tid == 0) mbar_arrive(&bar);
+  if (tid < s_ns) {  // read by the tasks after the barrier that follows the wait
+    uint32_t m = s_rows[tid];
+    for (int i = 0; m != 0u; ++i, m &= m - 1u) {
+      const int b = __ffs(m) - 1;
+      int j = 0;
+      for (int jj = 0; jj < kTopK; ++jj)
+        if (s_asc[b * kTopK + jj] == tid) j = jj;
+      s_rbj[tid][i] = (uint8_t)(b | (j << 4));
+    }
+  }
 
   pdl_wait();
   pdl_trigger();
@@ -760,24 +777,24 @@ __global__ void __launch_bounds__(kK3Threads)
 #pragma unroll
     for (int p = 0; p < 2; ++p) {
       const int ic = 4 * p + (g >> 1), io = 4 * p + t;
-      if (ic < nr) {
-        const int b = nth_bit(mask, ic), hl = g & 1;
+      if (ic < nr) {  // the shared expert takes every row: its i-th row is row i
+        const int hl = g & 1;
         if (sh) {
-          img[p] = gs + (size_t)(2 * b + hl) * kIs;
+          img[p] = gs + (size_t)(2 * ic + hl) * kIs;
         } else {
-          int j = 0;
-          for (int jj = 0; jj < kTopK; ++jj)
-            if (s_asc[b * kTopK + jj] == slot) j = jj;
-          img[p] = gr + (size_t)((b * kTopK + j) * 2 + hl) * kI;
+          const int bj = s_rbj[slot][ic];
+          img[p] = gr + (size_t)(((bj & 15) * kTopK + (bj >> 4)) * 2 + hl) * kI;
         }
       }
       if (io < nr) {
-        const int b = nth_bit(mask, io);
-        orow[p] = b;
-        om[p] = 12 + part;
-        if (!sh)
-          for (int jj = 0; jj < kTopK; ++jj)
-            if (s_asc[b * kTopK + jj] == slot) om[p] = 2 * jj + part;
+        if (sh) {
+          orow[p] = io;
+          om[p] = 12 + part;
+        } else {
+          const int bj = s_rbj[slot][io];
+          orow[p] = bj & 15;
+          om[p] = 2 * (bj >> 4) + part;
+        }
       }
     }
     float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
