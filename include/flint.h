@@ -190,9 +190,10 @@ FLINT_API int flint_moe_decode_residual(const flint_moe_layer *layer, float *h, 
  * fp32 accumulation per output; the SwiGLU intermediate is rounded once, to
  * fp16 after a per-token power-of-two shift from a bound it cannot exceed.
  *   x bf16 [T][2048];  out bf16 [T][2048] (may not alias x);  1 <= T <= 2^20
- *   ws workspace of flint_workspace_bytes(FLINT_OP_PREFILL, T) (about 65 KB
- *      per token: routing tables, the fp16 token rows, the SwiGLU and expert
- *      outputs)
+ *   ws workspace of flint_workspace_bytes(FLINT_OP_PREFILL, T) (about 67 KB
+ *      per token, 70 KB up to T = 4,608 where the router keeps two fp64
+ *      partial logits per token and expert: routing tables, the fp16 token
+ *      rows, the SwiGLU and expert outputs)
  */
 FLINT_API int flint_moe_prefill(const flint_moe_layer *layer, const uint16_t *x, int T, uint16_t *out,
                       void *ws, size_t ws_bytes, void *stream);

@@ -56,6 +56,12 @@ struct PrefillLayout {
   int mr, max_tiles1, max_tiles2, nchunks;
 };
 
+// Up to this many tokens the prefill router splits every tile's K between two
+// CTAs (the tiles alone would leave most SMs idle) and publishes the two
+// k-half partial logits in fp64; above it, one CTA per tile publishes fp32.
+constexpr int kRouteSplitMaxT = 4608;
+inline int route_split(int T) { return T <= kRouteSplitMaxT ? 2 : 1; }
+
 inline PrefillLayout prefill_layout(int T) {
   PrefillLayout L{};
   L.nchunks = (T + kPfChunk - 1) / kPfChunk;
@@ -72,7 +78,7 @@ inline PrefillLayout prefill_layout(int T) {
     return at;
   };
   L.ctrl = take(256);
-  L.z = take(sizeof(float) * (size_t)T * 256);
+  L.z = take((route_split(T) == 2 ? 2 * sizeof(double) : sizeof(float)) * (size_t)T * 256);
   L.sel_idx = take(sizeof(int32_t) * (size_t)T * 6);
   L.sel_w = take(sizeof(float) * (size_t)T * 6);
   L.asc_e = take(sizeof(int32_t) * (size_t)T * 6);

@@ -3,7 +3,8 @@
 // The block is defined per token ("How to Run Flint Locally", section "The
 // architecture, from config.json"); for many tokens it is computed as
 //   1. router logits for all tokens (bf16 products on the tcgen05 tensor
-//      cores, fp32 partials of each 128-wide k-group summed in fp64) and a
+//      cores, fp32 partials of each 128-wide k-group summed in fp64; for
+//      small T in two k-halves on two CTAs, added as decode adds them) and a
 //      per-token top-6 with the same selection rule as decode;
 //   2. a stable token-by-expert counting sort: per-chunk bitmask counts, one
 //      scan over (expert, chunk), then positions in token order inside every
@@ -37,9 +38,12 @@ namespace flint {
 
 // ============================================================== top-6 (T tokens)
 // One warp per token: sigmoid, bias, top-6 (lower index wins ties), weights;
-// selection order to sel_*, ascending expert order to asc_*.
+// selection order to sel_*, ascending expert order to asc_*.  The logits are
+// fp32 z[T][256], or (zh non-null) two fp64 k-half partials zh[2][T][256]
+// added here, half 0 + half 1, as the decode router adds its halves.
 __global__ void __launch_bounds__(256)
-    k_pf_topk(const float *__restrict__ router_b, const float *__restrict__ z, int T,
+    k_pf_topk(const float *__restrict__ router_b, const float *__restrict__ z,
+              const double *__restrict__ zh, int T,
               int32_t *__restrict__ sel_idx, float *__restrict__ sel_w, int32_t *__restrict__ asc_e,
               float *__restrict__ asc_w) {
   pdl_wait();  // the previous kernel in the stream is complete (programmatic launch)
@@ -51,7 +55,8 @@ __global__ void __launch_bounds__(256)
   uint32_t key[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float zf = z[(size_t)tok * kE + lane + 32 * i];
+    const size_t zi = (size_t)tok * kE + lane + 32 * i;
+    const float zf = zh ? (float)(zh[zi] + zh[(size_t)T * kE + zi]) : z[zi];
     const float s = 1.f / (1.f + expf(-zf));
     sv[i] = s;
     key[i] = float_key(s + router_b[lane + 32 * i]);
@@ -1075,11 +1080,14 @@ FLINT_DEV void umma_commit1(uint64_t *bar) {
       : "memory");
 }
 
-// Persistent: CTA c takes tiles c, c + grid, ...; tile i = token tile i / 2,
-// expert half i % 2.
+// Persistent: CTA c takes work items c, c + grid, ...; item i is tile
+// i / nsplit (token tile tile / 2, expert half tile % 2) over the k-groups of
+// k-part i % nsplit.  nsplit = 1: the tile's fp32 logits to z[T][256];
+// nsplit = 2: the k-half's fp64 partial sums to zh[half][T][256].
 __global__ void __launch_bounds__(kRtThreads, 1)
     k_pf_router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                   int T, float *__restrict__ z, uint32_t *status) {
+                   int T, int nsplit, float *__restrict__ z, double *__restrict__ zh,
+                   uint32_t *status) {
   pdl_wait();  // the previous kernel in the stream is complete (programmatic launch)
   pdl_trigger();
   extern __shared__ unsigned char smraw[];
@@ -1089,8 +1097,8 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_fail;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int ntiles = 2 * ((T + kRtM - 1) / kRtM);
-  if ((int)blockIdx.x >= ntiles) return;
+  const int ntiles = 2 * ((T + kRtM - 1) / kRtM), nitems = ntiles * nsplit;
+  if ((int)blockIdx.x >= nitems) return;
   if (tid == 0) {
     for (int s = 0; s < kRtStages; ++s) {
       mbar_init(&full[s], 1);
@@ -1114,15 +1122,17 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s_tmem;
   constexpr int kG = kH / 128;  // 16 k-groups
+  const int gper = kG / nsplit;  // k-groups per work item
 
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRtRegCtl));
     if (warp == 0 && lane == 0) {
       // ---- producer: the token rows and the router rows of each k-group
       uint32_t it = 0;
-      for (int ti = blockIdx.x; ti < ntiles && !s_fail; ti += gridDim.x) {
+      for (int wi = blockIdx.x; wi < nitems && !s_fail; wi += gridDim.x) {
+        const int ti = wi / nsplit, g0 = gper * (wi % nsplit);
         const int t0 = kRtM * (ti >> 1), e0 = kRtN * (ti & 1);
-        for (int G = 0; G < kG; ++G, ++it) {
+        for (int G = g0; G < g0 + gper; ++G, ++it) {
           const int s = it % kRtStages;
           if (it >= (uint32_t)kRtStages &&
               !mbar_wait_sleep(&empty[s], ((it / kRtStages) - 1) & 1)) {
@@ -1143,9 +1153,9 @@ __global__ void __launch_bounds__(kRtThreads, 1)
       const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kRtN >> 3) << 17) |
                              ((uint32_t)(kRtM >> 4) << 24);
       uint32_t it = 0;
-      for (int ti = blockIdx.x; ti < ntiles && !s_fail; ti += gridDim.x) {
+      for (int wi = blockIdx.x; wi < nitems && !s_fail; wi += gridDim.x) {
         bool ok = true;
-        for (int G = 0; G < kG; ++G, ++it) {
+        for (int G = 0; G < gper; ++G, ++it) {
           const int s = it % kRtStages, b = it & 1;
           if ((it >= 2 && !mbar_wait(&sempty[b], ((it >> 1) - 1) & 1)) ||
               !mbar_wait(&full[s], (it / kRtStages) & 1)) {
@@ -1177,13 +1187,14 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     // half (warp - 4) / 4 of the tile's 128 experts (64 columns)
     const int q4 = warp & 3, c_lo = 64 * ((warp - 4) >> 2);
     uint32_t it = 0;
-    for (int ti = blockIdx.x; ti < ntiles; ti += gridDim.x) {
+    for (int wi = blockIdx.x; wi < nitems; wi += gridDim.x) {
+      const int ti = wi / nsplit, kh = wi % nsplit;
       const int t0 = kRtM * (ti >> 1), e0 = kRtN * (ti & 1);
       double acc[64];
 #pragma unroll
       for (int j = 0; j < 64; ++j) acc[j] = 0.0;
       bool ok = true;
-      for (int G = 0; G < kG; ++G, ++it) {
+      for (int G = 0; G < gper; ++G, ++it) {
         const int b = it & 1;
         if (!mbar_wait_sleep(&sfull[b], (it >> 1) & 1)) {
           ok = false;
@@ -1208,12 +1219,16 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         break;
       }
       const int tok = t0 + 32 * q4 + lane;
-      if (tok < T) {
+      if (tok < T && nsplit == 1) {
         float4 *zr = reinterpret_cast<float4 *>(z + (size_t)tok * kE + e0 + c_lo);
 #pragma unroll
         for (int j = 0; j < 16; ++j)
           zr[j] = make_float4((float)acc[4 * j], (float)acc[4 * j + 1], (float)acc[4 * j + 2],
                               (float)acc[4 * j + 3]);
+      } else if (tok < T) {
+        double2 *zr = reinterpret_cast<double2 *>(zh + ((size_t)kh * T + tok) * kE + e0 + c_lo);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) zr[j] = make_double2(acc[2 * j], acc[2 * j + 1]);
       }
     }
   }
@@ -1380,14 +1395,17 @@ cudaError_t launch_route_many(const LayerArgs &L, const uint16_t *x, int T, int3
                                 (int)kRtSmem)) != cudaSuccess)
     return e;
   note_step("prefill router launch");
+  const int nsplit = route_split(T);
+  double *zh = nsplit == 2 ? reinterpret_cast<double *>(ws + P.z) : nullptr;
   {
-    const int ntiles = 2 * ((T + kRtM - 1) / kRtM);
-    e = pf_launch(k_pf_router_tc, ntiles < 148 ? ntiles : 148, kRtThreads, kRtSmem, st, mX, mW, T,
-                  z, reinterpret_cast<uint32_t *>(ws + P.ctrl) + 1);
+    const int nitems = 2 * ((T + kRtM - 1) / kRtM) * nsplit;
+    e = pf_launch(k_pf_router_tc, nitems < 148 ? nitems : 148, kRtThreads, kRtSmem, st, mX, mW, T,
+                  nsplit, z, zh, reinterpret_cast<uint32_t *>(ws + P.ctrl) + 1);
   }
   if (e != cudaSuccess) return e;
   note_step("prefill top-6 launch");
-  return pf_launch(k_pf_topk, (T + 7) / 8, 256, 0, st, L.router_b, z, T, idx, w,
+  return pf_launch(k_pf_topk, (T + 7) / 8, 256, 0, st, L.router_b, (const float *)z,
+                   (const double *)zh, T, idx, w,
                    reinterpret_cast<int32_t *>(ws + P.asc_e), reinterpret_cast<float *>(ws + P.asc_w));
 }
 
