@@ -36,10 +36,10 @@ H = synth.HIDDEN
 LAYER_FIXED_BYTES = 256 * 2048 * 2 + 256 * 4 + 2048 * (1024 + 32) + 2048 * (512 + 16)
 # DRAM bytes per decode layer over algorithmic bytes, from the ncu capture in
 # profiles/decode_layer_b4_stack.md (4 layers of this workload at batch 4:
-# 110.70 MB read against 109.63 MB algorithmic); traffic grows with the
+# 110.68 MB read against 109.63 MB algorithmic); traffic grows with the
 # expert count the same way, so a full layer's traffic is this ratio times
 # its algorithmic bytes.
-DECODE_TRAFFIC_RATIO = 110.70 / 109.63
+DECODE_TRAFFIC_RATIO = 110.68 / 109.63
 EXPERT_BYTES = 1024 * (1024 + 32) + 2048 * (256 + 8)
 HEAD_BYTES = synth.VOCAB * (1024 + 32)
 METRIC = "us per MoE-layer decode (B=4), fraction of HBM roofline"
