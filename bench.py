@@ -142,6 +142,14 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ workload
+def decode_config(B, layers):
+    """The workload both arms time (the reference arm on a bounded sample of it)."""
+    return {"workload": f"flint moe decode, 47-layer stack (RMSNorm->MoE->residual), "
+                        f"batch {B}, fresh rows per step",
+            "batch": B, "layers": layers, "hidden": H, "experts": 256, "top_k": 6,
+            "l2": "inputs larger than L2: 47 layers x 420 MB of int4 weights rotate"}
+
+
 def step_inputs(steps: int, B: int) -> np.ndarray:
     """Fresh residual rows for each step: seed 10000 + 4*step + row."""
     return np.stack([synth.residual_h([10000 + 4 * s + r for r in range(B)]) for s in range(steps)])
@@ -239,8 +247,7 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": per_layer_us * args.layers / 1e3, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"flint moe decode, 47-layer stack, batch {B}",
-                       "batch": B, "layers": args.layers},
+            "config": decode_config(B, args.layers),
             "cpu_baseline": {"value": per_layer_us, "unit": "us/layer", "cores": 1,
                              "kind": "oracle",
                              "sample": f"{args.steps} stack-layer calls of one row each, "
@@ -468,14 +475,11 @@ def main():
         "metric": METRIC, "value": us_per_layer, "unit": "us/layer", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms / args.steps, "higher_is_better": False, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16 activations x int4 weights, fp32 accumulate",
+        "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; weights as the workload recipe)",
-        "config": {"workload": f"flint moe decode, 47-layer stack (RMSNorm->MoE->residual), "
-                               f"batch {B}, fresh rows per step",
-                   "batch": B, "layers": nl, "hidden": H, "experts": 256, "top_k": 6,
-                   "l2": "inputs larger than L2: 47 layers x 420 MB of int4 weights rotate",
-                   "stack_tokens_per_s": B * 1e6 / (us_per_layer * nl * world) * world,
-                   "mean_distinct_experts": U},
+        "config": dict(decode_config(B, nl),
+                       stack_tokens_per_s=B * 1e6 / (us_per_layer * nl * world) * world,
+                       mean_distinct_experts=U),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm,
                      "traffic": DECODE_TRAFFIC_RATIO * bytes_per_layer,
