@@ -186,14 +186,21 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(world, v: float) -> float:
+def max_over_ranks(world, v: float, device: str = "cuda") -> float:
+    """The largest of the ranks' values (every rank gets it); device is where
+    the reduction runs: the GPU under NCCL, the CPU under gloo."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_us_per_layer(ms: float, steps: int, layers: int, world: int) -> float:
+    """Whole-job figure: the slowest rank's time over every layer-step all ranks ran."""
+    return ms * 1e3 / (steps * layers) / world
 
 
 def cpu_baseline(B: int, n_samples: int = 6):
@@ -341,7 +348,7 @@ def main():
     clocks = sampler.summary(tw0 - 0.5, tw1 + 0.5)
 
     layers_done = args.steps * nl * world
-    us_per_layer = ms * 1e3 / (args.steps * nl) / world
+    us_per_layer = job_us_per_layer(ms, args.steps, nl, world)
     achieved = bytes_per_layer / (ms * 1e-3 / (args.steps * nl)) / 1e9
 
     # ---- batch 1, same stack (context figure)
@@ -394,7 +401,7 @@ def main():
     e1.synchronize()
     barrier(world)
     mse = max_over_ranks(world, e0.elapsed_time(e1))
-    e2e_us = mse * 1e3 / (args.steps * nl) / world
+    e2e_us = job_us_per_layer(mse, args.steps, nl, world)
 
     # ---- output head int4 GEMV (B = 1 and the bench batch), context
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
