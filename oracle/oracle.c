@@ -23,15 +23,19 @@ typedef struct {
   int64_t lo, hi;
 } chunk;
 
+/* set inside a worker: a par_for called from one runs its loop itself */
+static __thread int t_in_worker = 0;
+
 static void *run_chunk(void *p) {
   chunk *c = (chunk *)p;
+  t_in_worker = 1;
   for (int64_t i = c->lo; i < c->hi; ++i) c->fn(c->ctx, i);
   return NULL;
 }
 
 /* fn(ctx, i) for i in [0, n): contiguous chunks, one per thread. */
 static void par_for(int64_t n, range_fn fn, void *ctx) {
-  int t = g_threads;
+  int t = t_in_worker ? 1 : g_threads;
   if (t > n) t = (int)n;
   if (t <= 1) {
     for (int64_t i = 0; i < n; ++i) fn(ctx, i);
@@ -201,15 +205,55 @@ void oracle_route(const oracle_layer *L, const uint16_t *x, int B, double *z, do
 }
 
 /* ------------------------------------------------------------ experts */
+/* Several matrix-vector products whose output rows are numbered one after
+ * the other, so that one par_for covers them all; each output element is the
+ * plain left-to-right row_dot. */
+typedef struct {
+  int n;
+  const uint8_t *q[8];
+  const uint16_t *s[8];
+  int64_t K[8], rows[8];
+  const double *x[8];
+  double *y[8];
+} matvec_set;
+
+static void matvec_set_row(void *p, int64_t i) {
+  matvec_set *m = (matvec_set *)p;
+  int j = 0;
+  while (i >= m->rows[j]) i -= m->rows[j++];
+  m->y[j][i] = row_dot(m->q[j], m->s[j], m->K[j], i, m->x[j]);
+}
+
+static void matvec_set_add(matvec_set *m, const uint8_t *q, const uint16_t *s, int64_t rows,
+                           int64_t K, const double *x, double *y) {
+  m->q[m->n] = q, m->s[m->n] = s, m->rows[m->n] = rows, m->K[m->n] = K;
+  m->x[m->n] = x, m->y[m->n] = y;
+  ++m->n;
+}
+
+static void matvec_set_run(matvec_set *m) {
+  int64_t total = 0;
+  for (int j = 0; j < m->n; ++j) total += m->rows[j];
+  par_for(total, matvec_set_row, m);
+}
+
+/* h[r] = silu(gate[r]) * up[r], with gate rows 0..I-1 and up rows I..2I-1 of g */
+static void swiglu_mid(const double *g, int inter, double *hmid) {
+  for (int r = 0; r < inter; ++r) hmid[r] = g[r] * sigmoid(g[r]) * g[inter + r];
+}
+
 void oracle_swiglu_expert(const uint8_t *q13, const uint16_t *s13, const uint8_t *q2,
                           const uint16_t *s2, int hidden, int inter, const double *x, double *y) {
+  double *g = (double *)malloc(sizeof(double) * 2 * inter);
   double *hmid = (double *)malloc(sizeof(double) * inter);
-  for (int r = 0; r < inter; ++r) {
-    double gate = row_dot(q13, s13, hidden, r, x);
-    double up = row_dot(q13, s13, hidden, inter + r, x);
-    hmid[r] = gate * sigmoid(gate) * up; /* silu(gate) * up */
-  }
-  for (int n = 0; n < hidden; ++n) y[n] = row_dot(q2, s2, inter, n, hmid);
+  matvec_set m = {0};
+  matvec_set_add(&m, q13, s13, 2 * inter, hidden, x, g);
+  matvec_set_run(&m);
+  swiglu_mid(g, inter, hmid);
+  matvec_set m2 = {0};
+  matvec_set_add(&m2, q2, s2, hidden, inter, hmid, y);
+  matvec_set_run(&m2);
+  free(g);
   free(hmid);
 }
 
@@ -227,33 +271,58 @@ static void moe_row(void *p, int64_t b) {
   const int E = L->n_experts, H = L->hidden, k = L->top_k, I = L->expert_i, Is = L->shared_i;
   double *xd = (double *)malloc(sizeof(double) * H);
   double *scr = (double *)malloc(sizeof(double) * 3 * E);
-  double *y = (double *)malloc(sizeof(double) * H);
   int32_t idx[64];
   double w[64], gap;
   to_double(c->x + b * H, H, xd);
   route_row(L, xd, scr, scr + E, scr + 2 * E, idx, w, &gap);
   double *out = c->out + b * H;
-  for (int n = 0; n < H; ++n) out[n] = 0.0;
-  for (int j = 0; j < k; ++j) {
-    const int64_t e = idx[j];
-    oracle_swiglu_expert(L->w13_q + e * (2 * I) * (H / 2), L->w13_s + e * (2 * I) * (H / 128),
-                         L->w2_q + e * H * (I / 2), L->w2_s + e * H * (I / 128), H, I, xd, y);
-    for (int n = 0; n < H; ++n) out[n] += w[j] * y[n];
+  /* the k chosen experts and the shared expert (slot k), each
+   * y = W2 (silu(W1 x) * (W3 x)): all gate/up rows in one set of products,
+   * then all down rows in another */
+  double *g = (double *)malloc(sizeof(double) * (2 * (size_t)I * k + 2 * (size_t)Is));
+  double *hmid = (double *)malloc(sizeof(double) * ((size_t)I * k + Is));
+  double *ys = (double *)malloc(sizeof(double) * (size_t)H * (k + 1));
+  matvec_set m13 = {0}, m2 = {0};
+  for (int j = 0; j <= k; ++j) {
+    const int64_t e = j < k ? idx[j] : 0;
+    const int inter = j < k ? I : Is;
+    const size_t go = 2 * (size_t)I * j, ho = (size_t)I * j;
+    if (j < k) {
+      matvec_set_add(&m13, L->w13_q + e * (2 * I) * (H / 2), L->w13_s + e * (2 * I) * (H / 128),
+                     2 * inter, H, xd, g + go);
+      matvec_set_add(&m2, L->w2_q + e * H * (I / 2), L->w2_s + e * H * (I / 128), H, inter,
+                     hmid + ho, ys + (size_t)H * j);
+    } else {
+      matvec_set_add(&m13, L->sh13_q, L->sh13_s, 2 * inter, H, xd, g + go);
+      matvec_set_add(&m2, L->sh2_q, L->sh2_s, H, inter, hmid + ho, ys + (size_t)H * j);
+    }
   }
-  oracle_swiglu_expert(L->sh13_q, L->sh13_s, L->sh2_q, L->sh2_s, H, Is, xd, y);
-  for (int n = 0; n < H; ++n) out[n] += y[n];
+  matvec_set_run(&m13);
+  for (int j = 0; j <= k; ++j)
+    swiglu_mid(g + 2 * (size_t)I * j, j < k ? I : Is, hmid + (size_t)I * j);
+  matvec_set_run(&m2);
+  for (int n = 0; n < H; ++n) out[n] = 0.0;
+  for (int j = 0; j < k; ++j)
+    for (int n = 0; n < H; ++n) out[n] += w[j] * ys[(size_t)H * j + n];
+  for (int n = 0; n < H; ++n) out[n] += ys[(size_t)H * k + n];
+  free(g);
+  free(hmid);
+  free(ys);
   if (c->idx) memcpy(c->idx + b * k, idx, sizeof(int32_t) * k);
   if (c->w) memcpy(c->w + b * k, w, sizeof(double) * k);
   if (c->gap) c->gap[b] = gap;
   free(xd);
   free(scr);
-  free(y);
 }
 
 void oracle_moe_layer(const oracle_layer *L, const uint16_t *x, int B, double *out,
                       int32_t *idx, double *w, double *gap) {
   moe_ctx c = {L, x, out, idx, w, gap};
-  par_for(B, moe_row, &c);
+  if (B >= g_threads) {
+    par_for(B, moe_row, &c); /* one row per worker, its products in turn */
+  } else {
+    for (int b = 0; b < B; ++b) moe_row(&c, b); /* rows in turn, their products threaded */
+  }
 }
 
 /* ------------------------------------------------------------ stack layer */

@@ -38,10 +38,12 @@ MUTANTS = {
     "weights not normalized": [("w[j] = sig[order[j]] / ssum;", "w[j] = sig[order[j]];")],
     "ties to the higher expert": [("(bi == bj && i < j)", "(bi == bj && i > j)")],
     "router transposed": [("L->router_w[(int64_t)e * H + h]", "L->router_w[(int64_t)h * E + e]")],
-    "gate and up swapped": [("hmid[r] = gate * sigmoid(gate) * up;",
-                             "hmid[r] = up * sigmoid(up) * gate;")],
-    "activation dropped": [("hmid[r] = gate * sigmoid(gate) * up;", "hmid[r] = gate * up;")],
-    "shared expert dropped": [("for (int n = 0; n < H; ++n) out[n] += y[n];", "(void)y;")],
+    "gate and up swapped": [("hmid[r] = g[r] * sigmoid(g[r]) * g[inter + r];",
+                             "hmid[r] = g[inter + r] * sigmoid(g[inter + r]) * g[r];")],
+    "activation dropped": [("hmid[r] = g[r] * sigmoid(g[r]) * g[inter + r];",
+                            "hmid[r] = g[r] * g[inter + r];")],
+    "shared expert dropped": [("for (int n = 0; n < H; ++n) out[n] += ys[(size_t)H * k + n];",
+                               "(void)0;")],
     "rmsnorm without the mean": [("1.0 / sqrt(ss / H + eps)", "1.0 / sqrt(ss + eps)")],
     "residual adds the fp64 block output": [
         ("double o = oracle_bf16_to_double(oracle_double_to_bf16(out[i]));", "double o = out[i];")],
