@@ -34,12 +34,13 @@ import synth  # noqa: E402
 N_LAYERS = synth.N_MOE_LAYERS
 H = synth.HIDDEN
 LAYER_FIXED_BYTES = 256 * 2048 * 2 + 256 * 4 + 2048 * (1024 + 32) + 2048 * (512 + 16)
-# DRAM bytes per decode layer over algorithmic bytes, from the ncu capture in
-# profiles/decode_layer_b4_stack.md (4 layers of this workload at batch 4:
-# 110.68 MB read against 109.63 MB algorithmic); traffic grows with the
-# expert count the same way, so a full layer's traffic is this ratio times
-# its algorithmic bytes.
+# DRAM bytes per decode layer over algorithmic bytes, from one ncu capture of
+# four stacked layers of this workload at batch 4 (110.68 MB read against
+# 109.63 MB algorithmic).  Traffic grows with the expert count the same way,
+# so a full layer's traffic is reported as this ratio times its algorithmic
+# bytes: a figure scaled from that capture, not measured in this run.
 DECODE_TRAFFIC_RATIO = 110.68 / 109.63
+TIMING_REPEATS = 20
 EXPERT_BYTES = 1024 * (1024 + 32) + 2048 * (256 + 8)
 HEAD_BYTES = synth.VOCAB * (1024 + 32)
 METRIC = "us per MoE-layer decode (B=4), fraction of HBM roofline"
@@ -48,7 +49,7 @@ METRIC = "us per MoE-layer decode (B=4), fraction of HBM roofline"
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--batch", type=int, default=4)
     p.add_argument("--impl", default="flint", choices=["flint", "reference"])
@@ -203,12 +204,16 @@ def job_us_per_layer(ms: float, steps: int, layers: int, world: int) -> float:
     return ms * 1e3 / (steps * layers) / world
 
 
-def cpu_baseline(B: int, n_samples: int = 6):
-    """The fp64 oracle on the host cores: n_samples stack-layer calls at batch
-    B (layer l, rows of step l), timed; reported as us per MoE layer."""
+def host_cores() -> int:
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(B: int, n_samples: int = 3):
+    """The fp64 oracle on every host core: n_samples stack-layer calls at
+    batch B (layer i on the rows of step i), timed; us per MoE layer."""
     import oracle
-    threads = os.cpu_count() or 1
-    oracle.set_threads(threads)
+    cores = host_cores()
+    oracle.set_threads(cores)
     hs = step_inputs(n_samples, B)
     t = 0.0
     for i in range(n_samples):
@@ -216,49 +221,87 @@ def cpu_baseline(B: int, n_samples: int = 6):
         t0 = time.perf_counter()
         oracle.stack_layer(L, hs[i])
         t += time.perf_counter() - t0
-    return {"value": t / n_samples * 1e6, "unit": "us/layer", "cores": min(threads, B),
+    return {"value": t / n_samples * 1e6, "unit": "us/layer", "cores": cores, "nproc": cores,
             "kind": "oracle",
-            "sample": f"{n_samples} stack-layer calls at batch {B} (layers 0..{n_samples - 1}, "
-                      f"fp64 oracle threaded over the {B} rows)"}
+            "sample": f"{n_samples} stack-layer calls at batch {B} (layers 0..{n_samples - 1}), "
+                      f"fp64 oracle threaded over each matrix's output rows on {cores} threads"}
+
+
+def cpu_baselines_other(B: int):
+    """The oracle on the other workloads, each a bounded sample, all cores:
+    one layer at batch 1 and at batch B (layer 0, decode rows), the output
+    head at batch 1, and prefill of the first 64 tokens of the 2,048-token
+    input (per-token work is the same for every token)."""
+    import oracle
+    cores = host_cores()
+    oracle.set_threads(cores)
+    out = {}
+    L0 = oracle.Layer(synth.layer_host(0))
+    for b, seeds in ((1, [0]), (B, list(range(1, B + 1)))):
+        x = synth.decode_x(seeds)
+        t0 = time.perf_counter()
+        oracle.moe_layer(L0, x)
+        dt = time.perf_counter() - t0
+        out[f"layer_b{b}"] = {"value": dt * 1e6, "unit": "us/layer", "cores": cores,
+                              "kind": "oracle", "sample": f"layer 0, batch {b}, in full"}
+    head = synth.head_host()
+    x = synth.head_x([0])
+    t0 = time.perf_counter()
+    oracle.int4_gemv(head["q"], head["s"], x)
+    dt = time.perf_counter() - t0
+    out["head_gemv_b1"] = {"value": dt * 1e6, "unit": "us", "cores": cores, "kind": "oracle",
+                           "sample": "150,144 x 2,048 head, batch 1, in full"}
+    xp = synth.prefill_x(2048, 2048)[:64]
+    t0 = time.perf_counter()
+    oracle.moe_layer(L0, xp)
+    dt = time.perf_counter() - t0
+    out["prefill_T2048"] = {"value": 64 / dt, "unit": "tokens/s", "cores": cores,
+                            "kind": "oracle",
+                            "sample": "first 64 of the 2,048 prefill tokens (layer 0), "
+                                      "scaled per token"}
+    return out
 
 
 def run_reference(args):
-    """Reference arm: the fp64 CPU oracle, each step one stack-layer call for
-    ONE row (layer = step mod 47); value scaled to us per layer at batch B."""
+    """Reference arm: the fp64 CPU oracle as it stands, on every host core.
+    Each step is one stack-layer call at the benchmark's batch (RMSNorm ->
+    block -> residual add for B rows; layers cycle through the first four of
+    the stack), so the value is us per MoE layer at batch B, the arm's own
+    metric, and ms_per_step is the time one such step took."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if world > 1 and rank != 0:
         return
     import oracle
-    oracle.set_threads(1)
+    cores = host_cores()
+    oracle.set_threads(cores)
     B = args.batch
-    hs = step_inputs(args.steps + args.warmup, 1)
+    hs = step_inputs(args.steps + args.warmup, B)
     cache = {}
 
     def layer(l):
         if l not in cache:
-            cache.clear()
             cache[l] = oracle.Layer(synth.layer_host(l))
         return cache[l]
 
     for s in range(args.warmup):
-        oracle.stack_layer(layer(s % args.layers), hs[s])
+        oracle.stack_layer(layer(s % 4), hs[s])
     t = 0.0
     for s in range(args.warmup, args.warmup + args.steps):
-        L = layer(s % args.layers)
+        L = layer(s % 4)
         t0 = time.perf_counter()
         oracle.stack_layer(L, hs[s])
         t += time.perf_counter() - t0
-    per_layer_us = t / args.steps * 1e6 * B
+    per_layer_us = t / args.steps * 1e6
     line = {"impl": "reference", "metric": METRIC, "value": per_layer_us, "unit": "us/layer",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": per_layer_us * args.layers / 1e3, "higher_is_better": False,
+            "ms_per_step": per_layer_us / 1e3, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": decode_config(B, args.layers),
-            "cpu_baseline": {"value": per_layer_us, "unit": "us/layer", "cores": 1,
-                             "kind": "oracle",
-                             "sample": f"{args.steps} stack-layer calls of one row each, "
-                                       f"scaled x{B} to a batch-{B} layer"},
+            "cpu_baseline": {"value": per_layer_us, "unit": "us/layer", "cores": cores,
+                             "nproc": cores, "kind": "oracle",
+                             "sample": f"{args.steps} stack-layer calls at batch {B} (layers "
+                                       f"0..3 in turn), fp64 oracle on {cores} threads"},
             "e2e": {"value": per_layer_us, "unit": "us/layer", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
@@ -277,6 +320,7 @@ def main():
     hbm, peak_kind = peaks()
 
     layers, structs = build_layers(nl, dev)
+    layer_arr = F.layer_array(structs)
     total = args.steps + args.warmup
     h_host = torch.from_numpy(step_inputs(total, B)).pin_memory()          # [S][B][H]
     h_dev = h_host.to(dev)
@@ -286,10 +330,9 @@ def main():
     F.flint_workspace_init(ws, nb)
     stream = torch.cuda.Stream(dev)
 
-    def one_step(s, st):
-        h_work.copy_(h_dev[s], non_blocking=True)
-        for l in range(nl):
-            F.flint_moe_decode_residual(structs[l], h_work, B, None, None, ws, nb, stream=st)
+    def one_step(s, st, hw=h_work, b=B, w=ws, n=nb, src=None):
+        hw.copy_(h_dev[s, :b] if src is None else src[s], non_blocking=True)
+        F.flint_moe_decode_stack(layer_arr, nl, hw, b, None, None, None, w, n, stream=st)
 
     # routing of every (step, layer), outside the timed region, for the bytes count
     idx = torch.empty((nl, B, 6), dtype=torch.int32, device=dev)
@@ -297,32 +340,54 @@ def main():
     with torch.cuda.stream(stream):
         for s in range(args.warmup, total):
             h_work.copy_(h_dev[s])
-            for l in range(nl):
-                F.flint_moe_decode_residual(structs[l], h_work, B, idx[l], None, ws, nb,
-                                            stream=stream)
+            F.flint_moe_decode_stack(layer_arr, nl, h_work, B, idx, None, None, ws, nb,
+                                     stream=stream)
             distinct.append(idx.cpu().numpy())
     stream.synchronize()
     U = float(np.mean([len(set(a[l].ravel().tolist())) for a in distinct for l in range(nl)]))
     bytes_per_layer = LAYER_FIXED_BYTES + U * EXPERT_BYTES + 2 * B * H * 4
 
-    # capture the K timed steps (and warmup steps) as CUDA graphs
-    with torch.cuda.stream(stream):
-        for s in range(args.warmup):
-            one_step(s, stream)
-    stream.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        for s in range(args.warmup, total):
-            one_step(s, stream)
-    gw = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(gw, stream=stream):
-        for s in range(min(args.warmup, total)):
-            one_step(s, stream)
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            gw.replay()
-    stream.synchronize()
+    def capture(step_fn):
+        """CUDA graphs of the warm-up steps and of the K timed steps."""
+        with torch.cuda.stream(stream):
+            for s in range(args.warmup):
+                step_fn(s, stream)
+        stream.synchronize()
+        gt = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gt, stream=stream):
+            for s in range(args.warmup, total):
+                step_fn(s, stream)
+        gwu = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gwu, stream=stream):
+            for s in range(min(args.warmup, total)):
+                step_fn(s, stream)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                gwu.replay()
+        stream.synchronize()
+        return gt, gwu
 
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timed(gt):
+        """TIMING_REPEATS replays of the K-step graph, each bracketed by a
+        barrier and a synchronize, timed with events on the launching stream;
+        per replay the max over ranks.  Returns the per-replay ms list."""
+        out = []
+        for _ in range(TIMING_REPEATS):
+            barrier(world)
+            torch.cuda.synchronize()
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                gt.replay()
+                e1.record(stream)
+            e1.synchronize()
+            barrier(world)
+            torch.cuda.synchronize()
+            out.append(max_over_ranks(world, e0.elapsed_time(e1)))
+        return out
+
+    g, gw = capture(one_step)
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
@@ -332,24 +397,18 @@ def main():
         with torch.cuda.stream(stream):
             g.replay()
         stream.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
     tw0 = time.time()
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        g.replay()
-        e1.record(stream)
-    e1.synchronize()
+    reps = timed(g)
     tw1 = time.time()
-    barrier(world)
-    torch.cuda.synchronize()
-    ms = max_over_ranks(world, e0.elapsed_time(e1))
     clocks = sampler.summary(tw0 - 0.5, tw1 + 0.5)
+    ms = statistics.median(reps)
 
-    layers_done = args.steps * nl * world
     us_per_layer = job_us_per_layer(ms, args.steps, nl, world)
     achieved = bytes_per_layer / (ms * 1e-3 / (args.steps * nl)) / 1e9
+    timing = {"repeats": TIMING_REPEATS, "steps_per_repeat": args.steps,
+              "us_per_layer_median": us_per_layer,
+              "us_per_layer_min": job_us_per_layer(min(reps), args.steps, nl, world),
+              "us_per_layer_max": job_us_per_layer(max(reps), args.steps, nl, world)}
 
     # ---- batch 1, same stack (context figure)
     extra = {}
@@ -358,50 +417,32 @@ def main():
         nb1 = F.flint_workspace_bytes(F.FLINT_OP_DECODE, 1)
         ws1 = torch.zeros(nb1, dtype=torch.uint8, device=dev)
         F.flint_workspace_init(ws1, nb1)
-        g1 = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g1, stream=stream):
-            for s in range(args.warmup, total):
-                h1.copy_(h_dev[s, :1], non_blocking=True)
-                for l in range(nl):
-                    F.flint_moe_decode_residual(structs[l], h1, 1, None, None, ws1, nb1,
-                                                stream=stream)
-        with torch.cuda.stream(stream):
-            g1.replay()
-            stream.synchronize()
-            e0.record(stream)
-            g1.replay()
-            e1.record(stream)
-        e1.synchronize()
-        ms1 = e0.elapsed_time(e1)
+        g1, gw1 = capture(lambda s, st: one_step(s, st, hw=h1, b=1, w=ws1, n=nb1))
+        reps1 = timed(g1)
+        ms1 = statistics.median(reps1)
         us1 = ms1 * 1e3 / (args.steps * nl)
         b1_bytes = LAYER_FIXED_BYTES + 6 * EXPERT_BYTES + 2 * H * 4
-        extra["batch1"] = {"us_per_layer": us1, "stack_tokens_per_s": 1e6 / (us1 * nl),
+        extra["batch1"] = {"us_per_layer": us1, "us_per_layer_min": min(reps1) * 1e3 / (args.steps * nl),
+                           "us_per_layer_max": max(reps1) * 1e3 / (args.steps * nl),
+                           "stack_tokens_per_s": 1e6 / (us1 * nl),
                            "roofline_frac": b1_bytes / (us1 * 1e-6) / 1e9 / hbm,
                            "bytes_per_layer": b1_bytes}
+        del g1, gw1
 
     # ---- e2e through the C ABI with host buffers: H2D of the step's rows,
-    # 47 layer calls, D2H of the result rows, every step
-    out_host = torch.empty((args.steps, B, H), dtype=torch.float32).pin_memory()
-    ge = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(ge, stream=stream):
-        for i, s in enumerate(range(args.warmup, total)):
-            h_work.copy_(h_host[s], non_blocking=True)
-            for l in range(nl):
-                F.flint_moe_decode_residual(structs[l], h_work, B, None, None, ws, nb,
-                                            stream=stream)
-            out_host[i].copy_(h_work, non_blocking=True)
-    with torch.cuda.stream(stream):
-        ge.replay()
-    stream.synchronize()
-    barrier(world)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        ge.replay()
-        e1.record(stream)
-    e1.synchronize()
-    barrier(world)
-    mse = max_over_ranks(world, e0.elapsed_time(e1))
+    # the stack call, D2H of the result rows, every step
+    out_host = torch.empty((total, B, H), dtype=torch.float32).pin_memory()
+
+    def e2e_step(s, st):
+        h_work.copy_(h_host[s], non_blocking=True)
+        F.flint_moe_decode_stack(layer_arr, nl, h_work, B, None, None, None, ws, nb, stream=st)
+        out_host[s].copy_(h_work, non_blocking=True)
+
+    ge, gwe = capture(e2e_step)
+    repse = timed(ge)
+    mse = statistics.median(repse)
     e2e_us = job_us_per_layer(mse, args.steps, nl, world)
+    del ge, gwe
 
     # ---- output head int4 GEMV (B = 1 and the bench batch), context
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -477,6 +518,7 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline(B)
+        extra["cpu_baselines"] = cpu_baselines_other(B)
 
     line = {
         "metric": METRIC, "value": us_per_layer, "unit": "us/layer", "n_gpus": world,
@@ -487,9 +529,13 @@ def main():
         "config": dict(decode_config(B, nl),
                        stack_tokens_per_s=B * 1e6 / (us_per_layer * nl * world) * world,
                        mean_distinct_experts=U),
+        "timing": timing,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm,
                      "traffic": DECODE_TRAFFIC_RATIO * bytes_per_layer,
+                     "traffic_source": "scaled: this layer's algorithmic bytes x the DRAM/"
+                                       "algorithmic ratio of one ncu capture of the same "
+                                       "kernels (four stacked layers, batch 4)",
                      "kernel": "decode layer (3 PDL-chained kernels)",
                      "peak_kind": peak_kind, "bytes_per_layer": bytes_per_layer},
         "e2e": {"value": e2e_us, "unit": "us/layer", "h2d_bytes_per_step": B * H * 4,
@@ -503,7 +549,7 @@ def main():
         print(json.dumps(line))
     if world > 1:
         import torch.distributed as dist
-        del g, gw, ge
+        del g, gw
         dist.destroy_process_group()
 
 

@@ -54,6 +54,7 @@ extern "C" {
 #define FLINT_GROUP 128
 #define FLINT_MAX_DECODE_B 8
 #define FLINT_MAX_PREFILL_T (1 << 20)
+#define FLINT_MAX_STACK_LAYERS 256
 #define FLINT_RMS_EPS 1e-6
 
 enum {
@@ -108,7 +109,8 @@ FLINT_API const char *flint_strerror(int code);
 FLINT_API size_t flint_workspace_bytes(int op, int n);
 FLINT_API size_t flint_gemv_workspace_bytes(int N, int B);
 
-/* Zero a workspace's counters and status word (async on `stream`). */
+/* Zero a whole workspace (async on `stream`), counters and status word
+ * included. */
 FLINT_API int flint_workspace_init(void *ws, size_t ws_bytes, void *stream);
 
 /* Copy the workspace's device status word to *status (synchronizes `stream`).
@@ -116,7 +118,8 @@ FLINT_API int flint_workspace_init(void *ws, size_t ws_bytes, void *stream);
 FLINT_API int flint_read_status(const void *ws, int *status, void *stream);
 
 /* Test hook for the failure path: the poll bound of the decode kernels'
- * (flint_moe_route, flint_moe_decode, flint_moe_decode_residual) first wait
+ * (flint_moe_route, flint_moe_decode, flint_moe_decode_residual) and the
+ * int4 GEMV's (flint_int4_gemv and its allocation-free variant) first wait
  * on each shared-memory barrier.  The default is 1 << 26 polls (seconds); a
  * small value, 0 included, makes those waits give up at once, so the call
  * records FLINT_ETIMEOUT in the workspace status word and returns without a
@@ -182,6 +185,26 @@ FLINT_API int flint_moe_decode_residual(const flint_moe_layer *layer, float *h, 
                               float *w, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * L stacked decode layers on an fp32 residual stream h [B][2048], B in
+ * [1, 8], 1 <= L <= FLINT_MAX_STACK_LAYERS: flint_moe_decode_residual applied
+ * with layers[0], then layers[1], ..., in one call (three programmatic-
+ * dependent kernels per layer on `stream`: each layer's router and shared
+ * expert weights are fetched while the previous kernel runs).  Bitwise equal
+ * to L calls of flint_moe_decode_residual.
+ *   layers   HOST array of L layer structs (read during the call only)
+ *   h        fp32 [B][2048], updated in place
+ *   idx, w   optional outputs (NULL to skip): int32 / fp32 [L][B][6], each
+ *            layer's selection as flint_moe_route returns it
+ *   h_trace  optional output (NULL to skip): fp32 [L][B][2048], the residual
+ *            h entering each layer (for layer-by-layer checks; one
+ *            device-to-device copy per layer)
+ *   ws       workspace of flint_workspace_bytes(FLINT_OP_DECODE, B)
+ */
+FLINT_API int flint_moe_decode_stack(const flint_moe_layer *layers, int L, float *h, int B,
+                                     int32_t *idx, float *w, float *h_trace, void *ws,
+                                     size_t ws_bytes, void *stream);
+
+/*
  * Prefill of the MoE block for T >= 1 tokens: the same function as
  * flint_moe_decode row by row, computed as routing for T tokens, a stable
  * token-by-expert sort, grouped GEMMs on the tensor cores and a fixed-order
@@ -218,22 +241,36 @@ FLINT_API int flint_int4_gemv(const uint8_t *q, const uint16_t *s, int N, int K,
  * allocation.  The pages have no counterpart: this entry point is an
  * integration convenience, not part of the method.
  *
- * Same arguments, results and errors as flint_int4_gemv, minus `ws`.  The
- * scratch (a counter, a status word and per-CTA argmax partials) is a
- * 65,792-byte array inside the library, one per GPU that loads it, kept until
- * the process exits; calls whose scratch would not fit are rejected with
- * FLINT_EINVAL (none with B <= 8 do).  Nothing is allocated: the call clears
- * the counter and status word with an asynchronous memset on `stream`, then
- * launches.  The first call on a device looks the array's device address up
- * (cudaGetSymbolAddress, with that device current) and caches it; make that
- * first call before any stream capture.  All calls on a device share the one
- * array and it keeps the last call's contents, so calls that may overlap on
- * the GPU (different streams without ordering between them) race and must
- * not be issued; order them on one stream.
+ * Same arguments and results as flint_int4_gemv, minus `ws`; argument errors
+ * are returned the same way, and a device-side timeout is recorded in the
+ * array's status word, read with flint_int4_gemv_noalloc_status.  The scratch
+ * (a counter, a status word and per-CTA argmax partials) is a 65,792-byte
+ * array inside the library, one per GPU that loads it, kept until the process
+ * exits; calls whose scratch would not fit are rejected with FLINT_EINVAL
+ * (none with B <= 8 do; B = 8 fills it).  Nothing is allocated: the call
+ * clears the counter and status word with an asynchronous memset on
+ * `stream`, then launches.  Outside a stream capture every call looks the
+ * array's device address up (cudaGetSymbolAddress, with the device current)
+ * and keeps it per device; inside a capture the kept address is used, so the
+ * first call on a device must be made before any capture (a capture without
+ * it returns FLINT_ECUDA).  All calls on a device share the one array and it
+ * keeps the last call's contents, so calls that may overlap on the GPU
+ * (different streams without ordering between them) race and must not be
+ * issued; order them on one stream.
  */
 FLINT_API int flint_int4_gemv_noalloc(const uint8_t *q, const uint16_t *s, int N, int K,
                                       const uint16_t *x, int B, float *y, int32_t *argmax,
                                       void *stream);
+
+/*
+ * Status word of the allocation-free GEMV's array on the current device:
+ * FLINT_OK, or FLINT_ETIMEOUT if a bounded wait of the last
+ * flint_int4_gemv_noalloc call on this device gave up (its y and argmax are
+ * then incomplete).  Copies the word to *status and synchronizes `stream`
+ * (use the stream of that call, outside any stream capture).  The next
+ * flint_int4_gemv_noalloc call clears the word.  Allocates nothing.
+ */
+FLINT_API int flint_int4_gemv_noalloc_status(int *status, void *stream);
 
 #ifdef __cplusplus
 }

@@ -20,8 +20,9 @@ HIDDEN, EXPERTS, TOP_K, EXPERT_I, SHARED_I, GROUP, MAX_DECODE_B = 2048, 256, 6, 
 
 EXPORTS = ("flint_version", "flint_strerror", "flint_last_cuda_error", "flint_workspace_bytes",
            "flint_gemv_workspace_bytes", "flint_workspace_init", "flint_read_status",
-           "flint_moe_route", "flint_moe_decode", "flint_moe_decode_residual",
+           "flint_moe_route", "flint_moe_decode", "flint_moe_decode_residual", "flint_moe_decode_stack",
            "flint_moe_prefill", "flint_int4_gemv", "flint_int4_gemv_noalloc",
+           "flint_int4_gemv_noalloc_status",
            "flint_debug_set_wait_polls", "flint_debug_prefill_events",
            "flint_debug_prefill_stage_ms")
 
@@ -71,9 +72,11 @@ def lib() -> C.CDLL:
         L.flint_moe_route.argtypes = [lp, vp, i, vp, vp, vp, sz, vp]
         L.flint_moe_decode.argtypes = [lp, vp, i, vp, vp, sz, vp]
         L.flint_moe_decode_residual.argtypes = [lp, vp, i, vp, vp, vp, sz, vp]
+        L.flint_moe_decode_stack.argtypes = [lp, i, vp, i, vp, vp, vp, vp, sz, vp]
         L.flint_moe_prefill.argtypes = [lp, vp, i, vp, vp, sz, vp]
         L.flint_int4_gemv.argtypes = [vp, vp, i, i, vp, i, vp, vp, vp, sz, vp]
         L.flint_int4_gemv_noalloc.argtypes = [vp, vp, i, i, vp, i, vp, vp, vp]
+        L.flint_int4_gemv_noalloc_status.argtypes = [C.POINTER(C.c_int), vp]
         for name in EXPORTS:
             getattr(L, name).restype = getattr(L, name).restype or i
         _lib = L
@@ -174,6 +177,24 @@ def flint_moe_decode_residual(layer: flint_moe_layer, h, B: int, idx, w, ws, ws_
            "flint_moe_decode_residual")
 
 
+def layer_array(layers) -> C.Array:
+    """A contiguous host array of layer structs (for flint_moe_decode_stack);
+    keeps the structs' tensors alive."""
+    arr = (flint_moe_layer * len(layers))(*layers)
+    arr._keep = list(layers)
+    return arr
+
+
+def flint_moe_decode_stack(layers, L: int, h, B: int, idx, w, h_trace, ws, ws_bytes: int,
+                           stream=None):
+    """``layers``: an array from ``layer_array`` (or a list of structs)."""
+    if not isinstance(layers, C.Array):
+        layers = layer_array(layers)
+    _check(lib().flint_moe_decode_stack(layers, L, _ptr(h), B, _ptr(idx), _ptr(w), _ptr(h_trace),
+                                        _ptr(ws), ws_bytes, _stream(stream)),
+           "flint_moe_decode_stack")
+
+
 def flint_moe_prefill(layer: flint_moe_layer, x, T: int, out, ws, ws_bytes: int, stream=None):
     _check(lib().flint_moe_prefill(C.byref(layer), _ptr(x), T, _ptr(out), _ptr(ws), ws_bytes,
                                    _stream(stream)), "flint_moe_prefill")
@@ -188,3 +209,12 @@ def flint_int4_gemv_noalloc(q, s, N: int, K: int, x, B: int, y, argmax, stream=N
     """flint_int4_gemv with the library's own static scratch (no workspace)."""
     _check(lib().flint_int4_gemv_noalloc(_ptr(q), _ptr(s), N, K, _ptr(x), B, _ptr(y),
                                          _ptr(argmax), _stream(stream)), "flint_int4_gemv_noalloc")
+
+
+def flint_int4_gemv_noalloc_status(stream=None) -> int:
+    """Status word of the allocation-free GEMV's static array on the current
+    device (synchronizes the stream)."""
+    st = C.c_int(0)
+    _check(lib().flint_int4_gemv_noalloc_status(C.byref(st), _stream(stream)),
+           "flint_int4_gemv_noalloc_status")
+    return st.value

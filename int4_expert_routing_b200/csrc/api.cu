@@ -87,7 +87,7 @@ size_t flint_gemv_workspace_bytes(int N, int B) {
 
 int flint_workspace_init(void *ws, size_t ws_bytes, void *stream) {
   if (!aligned16(ws) || ws_bytes < 256) return FLINT_EINVAL;
-  return from_cuda(cudaMemsetAsync(ws, 0, 256, static_cast<cudaStream_t>(stream)));
+  return from_cuda(cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)));
 }
 
 int flint_read_status(const void *ws, int *status, void *stream) {
@@ -111,7 +111,9 @@ int flint_debug_prefill_stage_ms(float *ms, int n) {
 }
 
 int flint_debug_set_wait_polls(uint32_t polls) {
-  return from_cuda(noted(decode_set_wait_polls(polls), "debug wait bound"));
+  cudaError_t e = noted(decode_set_wait_polls(polls), "debug wait bound (decode)");
+  if (e == cudaSuccess) e = noted(gemv_set_wait_polls(polls), "debug wait bound (gemv)");
+  return from_cuda(e);
 }
 
 int flint_moe_route(const flint_moe_layer *layer, const uint16_t *x, int B, int32_t *idx,
@@ -146,6 +148,33 @@ int flint_moe_decode_residual(const flint_moe_layer *layer, float *h, int B, int
   return from_cuda(launch_decode(layer_args(layer), nullptr, h, h, B, nullptr, idx, w,
                                  static_cast<char *>(ws), static_cast<cudaStream_t>(stream),
                                  false));
+}
+
+int flint_moe_decode_stack(const flint_moe_layer *layers, int L, float *h, int B, int32_t *idx,
+                           float *w, float *h_trace, void *ws, size_t ws_bytes, void *stream) {
+  if (!layers || L < 1 || L > FLINT_MAX_STACK_LAYERS || !aligned16(h) || B < 1 ||
+      B > FLINT_MAX_DECODE_B || !aligned16(ws) ||
+      ws_bytes < flint_workspace_bytes(FLINT_OP_DECODE, B) ||
+      (h_trace && !aligned16(h_trace)))
+    return FLINT_EINVAL;
+  for (int l = 0; l < L; ++l)
+    if (!layer_ok(&layers[l])) return FLINT_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int l = 0; l < L; ++l) {
+    cudaError_t e = cudaSuccess;
+    if (h_trace)
+      e = noted(cudaMemcpyAsync(h_trace + (size_t)l * B * FLINT_HIDDEN, h,
+                                sizeof(float) * (size_t)B * FLINT_HIDDEN, cudaMemcpyDeviceToDevice,
+                                st),
+                "stack trace copy");
+    if (e == cudaSuccess)
+      e = launch_decode(layer_args(&layers[l]), nullptr, h, h, B, nullptr,
+                        idx ? idx + (size_t)l * B * FLINT_TOPK : nullptr,
+                        w ? w + (size_t)l * B * FLINT_TOPK : nullptr, static_cast<char *>(ws), st,
+                        false);
+    if (e != cudaSuccess) return from_cuda(e);
+  }
+  return FLINT_OK;
 }
 
 int flint_int4_gemv(const uint8_t *q, const uint16_t *s, int N, int K, const uint16_t *x, int B,

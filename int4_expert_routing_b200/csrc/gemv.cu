@@ -36,6 +36,18 @@ FLINT_DEV bool better(float v, int i, float bv, int bi) {
   return bi < 0 ? (v == v) : (v > bv || (v == bv && i < bi));
 }
 
+// Poll bound of the GEMV's first wait on each ring barrier (a consumer's wait
+// for a stage to land, the producer's wait for a stage to be released).
+// flint_debug_set_wait_polls lowers it so that a test can drive the timeout
+// path; the error path's waits for copies still in flight keep kWaitPolls.
+static __device__ uint32_t g_gemv_polls = kWaitPolls;
+FLINT_DEV bool gwait(uint64_t *bar, uint32_t parity) {
+  const uint32_t n = *reinterpret_cast<volatile uint32_t *>(&g_gemv_polls);
+  for (uint32_t i = 0; i < n; ++i)
+    if (mbar_try(bar, parity)) return true;
+  return false;
+}
+
 static int gemv_grid(int N) {
   const int tiles = (N + 15) / 16;
   int sms = 148, dev = 0;
@@ -168,6 +180,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 1)
   }
   __syncthreads();
   bool failed = false;
+  int issued = 0;  // producer lane: tiles whose copies it issued
   float best_v[2] = {0.f, 0.f};
   int best_i[2] = {-1, -1};
 
@@ -177,10 +190,11 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 1)
       int k = 0;
       for (int tile = blockIdx.x; tile < full_tiles; tile += gridDim.x, ++k) {
         const int st = k % stages;
-        if (k >= stages && !mbar_wait(&empty[st], ((k / stages) - 1) & 1)) {
+        if (k >= stages && !gwait(&empty[st], ((k / stages) - 1) & 1)) {
           failed = true;
           break;
         }
+        issued = k + 1;
         unsigned char *dst = ring + (size_t)st * stage_bytes;
         mbar_expect_tx(&full[st], wbytes + sbytes);
         bulk_g2s(dst, q + (size_t)tile * wbytes, wbytes, &full[st]);
@@ -211,7 +225,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 1)
       if (k >= my_tiles) break;
       const int tile = (int)blockIdx.x + k * (int)gridDim.x;
       const int st = k % stages;
-      if (!mbar_wait(&full[st], (k / stages) & 1)) {
+      if (!gwait(&full[st], (k / stages) & 1)) {
         failed = true;
         break;
       }
@@ -248,6 +262,11 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 1)
   }
   if (__syncthreads_or(failed)) {
     if (tid == 0) set_status(ctrl + 1, kStatusTimeout);
+    // copies still in flight land before the CTA exits: the last phase issued
+    // on each stage (a completed phase passes at once)
+    if (warp == ncons && lane == 0)
+      for (int k = issued > stages ? issued - stages : 0; k < issued; ++k)
+        mbar_wait(&full[k % stages], (uint32_t)((k / stages) & 1));
     return;
   }
   if (!argmax) return;
@@ -298,6 +317,11 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 1)
   if (tid == 0) ctrl[0] = 0;
 }
 
+cudaError_t gemv_set_wait_polls(uint32_t polls) {
+  if (polls == 0xFFFFFFFFu) polls = kWaitPolls;
+  return cudaMemcpyToSymbol(g_gemv_polls, &polls, sizeof(polls));
+}
+
 cudaError_t launch_gemv(const uint8_t *q, const uint16_t *s, int N, int K, const uint16_t *x,
                         int B, float *y, int32_t *argmax, char *ws, cudaStream_t st) {
   const GemvPlan p = gemv_plan(K, B);
@@ -330,9 +354,11 @@ cudaError_t launch_gemv(const uint8_t *q, const uint16_t *s, int N, int K, const
 // status word, one argmax partial per CTA and row) lives in this file-scope
 // device array instead of a caller workspace.  Every GPU that loads the
 // library holds it until the process exits.  In host code the array's name is
-// only a host-side stand-in, so its device address is looked up once per
-// device (cudaGetSymbolAddress, on the first call made with that device
-// current) and cached.
+// only a host-side stand-in, so its device address is looked up with
+// cudaGetSymbolAddress, with the device current: on every call made outside a
+// stream capture (so a context torn down by cudaDeviceReset and rebuilt gets
+// the new address), and taken from the per-device cache inside a capture,
+// where only a device that already made an uncaptured call can be used.
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = 256 + 8 * 1024 * 8;  // counter/status + 1024 CTAs x 8 rows
@@ -341,18 +367,23 @@ static __device__ __align__(256) unsigned char g_gemv_scratch[kNoAllocScratchByt
 std::mutex g_scratch_mu;
 void *g_scratch_ptr[64] = {};
 
-// Device address of g_gemv_scratch on the current device (looked up once).
-cudaError_t scratch_address(void **out) {
+// Device address of g_gemv_scratch on the current device.
+cudaError_t scratch_address(cudaStream_t st, void **out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(st, &cap);
+  if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void *ptr = nullptr;
     e = cudaGetSymbolAddress(&ptr, g_gemv_scratch);
     if (e != cudaSuccess) return e;
     g_scratch_ptr[dev] = ptr;
+  } else if (!g_scratch_ptr[dev]) {
+    return cudaErrorStreamCaptureUnsupported;  // no uncaptured call on this device yet
   }
   *out = g_scratch_ptr[dev];
   return cudaSuccess;
@@ -370,12 +401,27 @@ extern "C" FLINT_API int flint_int4_gemv_noalloc(const uint8_t *q, const uint16_
       K % 128 || K > 8192 || B < 1 || B > FLINT_MAX_DECODE_B)
     return FLINT_EINVAL;
   if (flint::gemv_ws_bytes(N, B) > kNoAllocScratchBytes) return FLINT_EINVAL;  // cannot happen for B <= 8
-  void *scratch = nullptr;
-  cudaError_t e = flint::noted(scratch_address(&scratch), "no-alloc scratch address");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void *scratch = nullptr;
+  cudaError_t e = flint::noted(scratch_address(st, &scratch), "no-alloc scratch address");
   // the counter and status word must start at zero; the partials need not
   if (e == cudaSuccess) e = flint::noted(cudaMemsetAsync(scratch, 0, 256, st), "no-alloc scratch clear");
   if (e == cudaSuccess)
     e = flint::launch_gemv(q, s, N, K, x, B, y, argmax, static_cast<char *>(scratch), st);
   return flint_from_cuda(e);
+}
+
+extern "C" FLINT_API int flint_int4_gemv_noalloc_status(int *status, void *stream) {
+  if (!status) return FLINT_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void *scratch = nullptr;
+  cudaError_t e = flint::noted(scratch_address(st, &scratch), "no-alloc scratch address");
+  uint32_t ctrl[2] = {0, 0};
+  if (e == cudaSuccess)
+    e = flint::noted(cudaMemcpyAsync(ctrl, scratch, sizeof(ctrl), cudaMemcpyDeviceToHost, st),
+                     "no-alloc status copy");
+  if (e == cudaSuccess) e = flint::noted(cudaStreamSynchronize(st), "no-alloc status sync");
+  if (e != cudaSuccess) return flint_from_cuda(e);
+  *status = static_cast<int>(ctrl[1]);
+  return FLINT_OK;
 }

@@ -142,6 +142,7 @@ cudaError_t launch_gemv(const uint8_t *q, const uint16_t *s, int N, int K, const
                         int B, float *y, int32_t *argmax, char *ws, cudaStream_t st);
 size_t gemv_ws_bytes(int N, int B);
 cudaError_t decode_set_wait_polls(uint32_t polls);
+cudaError_t gemv_set_wait_polls(uint32_t polls);
 cudaError_t prefill_set_stage_events(int enable);
 cudaError_t prefill_stage_times(float *ms, int n);
 cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_t *out, char *ws,

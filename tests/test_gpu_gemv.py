@@ -84,3 +84,43 @@ def test_argmax_ties_go_to_lowest_row():
     y, am = gemv(q, s, x, N, K)
     assert list(am) == [17, 17]
     assert y[0, 17] == 3.5 and y[0, 100] == 2.5
+
+
+def test_gemv_timeout_reports_status_and_recovers():
+    """The GEMV's timeout path, driven without a GPU fault: with the first-wait
+    bound lowered to zero every CTA gives up at once, records FLINT_ETIMEOUT in
+    the workspace status word and returns after the copies it issued have
+    landed; with the bound restored the same workspace gives the normal,
+    bitwise-equal result."""
+    import time
+    F.build()
+    N, K, B = 150144, 2048, 2
+    q = synth.random_bytes_torch(0, synth.T_HEAD_Q, N * K // 2, "cuda").view(N, K // 2)
+    s = synth.to_device({"s": synth.head_host(with_codes=False)["s"]}, "cuda")["s"]
+    x = synth.to_device({"x": synth.head_x([0, 1])}, "cuda")["x"]
+    nb = F.flint_gemv_workspace_bytes(N, B)
+    ws = torch().zeros(nb, dtype=torch().uint8, device="cuda")
+
+    def call():
+        F.flint_workspace_init(ws, nb)
+        y = torch().full((B, N), 7.0, dtype=torch().float32, device="cuda")
+        am = torch().full((B,), -7, dtype=torch().int32, device="cuda")
+        F.flint_int4_gemv(q, s, N, K, x, B, y, am, ws, nb)
+        torch().cuda.synchronize()
+        return y.cpu().numpy(), am.cpu().numpy(), F.flint_read_status(ws)
+
+    y0, am0, st0 = call()
+    assert st0 == F.FLINT_OK
+    F.flint_debug_set_wait_polls(0)
+    try:
+        t0 = time.time()
+        y1, am1, st1 = call()
+        elapsed = time.time() - t0
+    finally:
+        F.flint_debug_set_wait_polls(0xFFFFFFFF)
+    assert st1 == F.FLINT_ETIMEOUT
+    assert elapsed < 5.0
+    assert (am1 == -7).all() and (y1 == 7.0).all()   # nothing written
+    y2, am2, st2 = call()
+    assert st2 == F.FLINT_OK
+    assert np.array_equal(y2, y0) and np.array_equal(am2, am0)
