@@ -109,6 +109,37 @@ static double row_dot(const uint8_t *q, const uint16_t *s, int64_t K, int64_t n,
 
 static double sigmoid(double z) { return 1.0 / (1.0 + exp(-z)); }
 
+/* ------------------------------------------------------------ group-64 affine int4 */
+/* IEEE binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits. */
+double oracle_fp16_to_double(uint16_t v) {
+  const int sign = v >> 15, e = (v >> 10) & 31, f = v & 1023;
+  double mag;
+  if (e == 0) mag = ldexp((double)f, -24);                 /* subnormal: f * 2^-24 */
+  else if (e == 31) mag = f ? NAN : INFINITY;
+  else mag = ldexp((double)(1024 + f), e - 25);            /* (1 + f/1024) * 2^(e-15) */
+  return sign ? -mag : mag;
+}
+
+/* The unsigned code of element k of a packed row (low nibble = even element). */
+static int ucode_of(const uint8_t *row, int64_t k) {
+  uint8_t byte = row[k / 2];
+  return (k % 2 == 0) ? (byte & 0x0F) : (byte >> 4);
+}
+
+/* Weight element (n, k): code * scale + offset of its 64-element group. */
+static double weight_affine(const uint8_t *q, const uint16_t *s, const uint16_t *m, int64_t K,
+                            int64_t n, int64_t k) {
+  const int64_t g = n * (K / 64) + k / 64;
+  return (double)ucode_of(q + n * (K / 2), k) * oracle_fp16_to_double(s[g]) +
+         oracle_fp16_to_double(m[g]);
+}
+
+void oracle_dequant_affine(const uint8_t *q, const uint16_t *s, const uint16_t *m, int64_t N,
+                           int64_t K, double *W) {
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k) W[n * K + k] = weight_affine(q, s, m, K, n, k);
+}
+
 /* ------------------------------------------------------------ int4 GEMV */
 typedef struct {
   const uint8_t *q;
@@ -127,6 +158,18 @@ static void to_double(const uint16_t *x, int64_t n, double *out) {
   for (int64_t i = 0; i < n; ++i) out[i] = oracle_bf16_to_double(x[i]);
 }
 
+/* argmax[b] = lowest index of the row maximum; gap[b] = top-1 minus top-2 */
+static void argmax_row(const double *yb, int64_t N, int32_t *argmax, double *gap) {
+  int64_t best = 0;
+  for (int64_t n = 1; n < N; ++n)
+    if (yb[n] > yb[best]) best = n;
+  double second = -INFINITY;
+  for (int64_t n = 0; n < N; ++n)
+    if (n != best && yb[n] > second) second = yb[n];
+  if (argmax) *argmax = (int32_t)best;
+  if (gap) *gap = yb[best] - second;
+}
+
 void oracle_int4_gemv(const uint8_t *q, const uint16_t *s, int64_t N, int64_t K,
                       const uint16_t *x, int B, double *y, int32_t *argmax, double *gap) {
   double *xd = (double *)malloc(sizeof(double) * K);
@@ -134,16 +177,35 @@ void oracle_int4_gemv(const uint8_t *q, const uint16_t *s, int64_t N, int64_t K,
     to_double(x + (int64_t)b * K, K, xd);
     gemv_ctx c = {q, s, N, K, xd, y + (int64_t)b * N};
     par_for(N, gemv_row, &c);
-    /* argmax, lowest index on ties; gap = best minus second best value */
-    const double *yb = y + (int64_t)b * N;
-    int64_t best = 0;
-    for (int64_t n = 1; n < N; ++n)
-      if (yb[n] > yb[best]) best = n;
-    double second = -INFINITY;
-    for (int64_t n = 0; n < N; ++n)
-      if (n != best && yb[n] > second) second = yb[n];
-    if (argmax) argmax[b] = (int32_t)best;
-    if (gap) gap[b] = yb[best] - second;
+    argmax_row(y + (int64_t)b * N, N, argmax ? argmax + b : NULL, gap ? gap + b : NULL);
+  }
+  free(xd);
+}
+
+typedef struct {
+  const uint8_t *q;
+  const uint16_t *s, *m;
+  int64_t K;
+  const double *x;
+  double *y;
+} gemv_affine_ctx;
+
+static void gemv_affine_row(void *p, int64_t n) {
+  gemv_affine_ctx *c = (gemv_affine_ctx *)p;
+  double acc = 0.0;
+  for (int64_t k = 0; k < c->K; ++k) acc += weight_affine(c->q, c->s, c->m, c->K, n, k) * c->x[k];
+  c->y[n] = acc;
+}
+
+void oracle_int4_gemv_affine(const uint8_t *q, const uint16_t *s, const uint16_t *m, int64_t N,
+                             int64_t K, const uint16_t *x, int B, double *y, int32_t *argmax,
+                             double *gap) {
+  double *xd = (double *)malloc(sizeof(double) * K);
+  for (int b = 0; b < B; ++b) {
+    to_double(x + (int64_t)b * K, K, xd);
+    gemv_affine_ctx c = {q, s, m, K, xd, y + (int64_t)b * N};
+    par_for(N, gemv_affine_row, &c);
+    argmax_row(y + (int64_t)b * N, N, argmax ? argmax + b : NULL, gap ? gap + b : NULL);
   }
   free(xd);
 }

@@ -64,6 +64,18 @@ uint16_t oracle_double_to_bf16(double v); /* round to nearest, ties to even */
 void oracle_int4_gemv(const uint8_t *q, const uint16_t *s, int64_t N, int64_t K,
                       const uint16_t *x, int B, double *y, int32_t *argmax, double *gap);
 
+/* Group-64 affine int4 ("How to Run Flint Locally", section "Every build and
+ * its size": the MLX int4 build quantizes to group-64 affine int4; the Q4_1
+ * GGUF stores the same codes with FP16 scales and offsets).  Row n of an
+ * [N, K] matrix: q as above but each nibble an UNSIGNED code 0..15, s and m
+ * [N, K/64] fp16 bits; weight = code * s + m, exactly, in fp64. */
+double oracle_fp16_to_double(uint16_t v);
+void oracle_dequant_affine(const uint8_t *q, const uint16_t *s, const uint16_t *m, int64_t N,
+                           int64_t K, double *W);
+void oracle_int4_gemv_affine(const uint8_t *q, const uint16_t *s, const uint16_t *m, int64_t N,
+                             int64_t K, const uint16_t *x, int B, double *y, int32_t *argmax,
+                             double *gap);
+
 /* Router for B rows.  z, sig, biased: [B][E] (any may be NULL); idx, w: [B][k];
  * gap[b] = k-th minus (k+1)-th biased score in selection order. */
 void oracle_route(const oracle_layer *L, const uint16_t *x, int B, double *z, double *sig,

@@ -131,6 +131,72 @@ def test_int4_gemv_argmax_ties_go_to_lowest_index():
     assert y[0, 1] == 3.5 and y[0, 2] == 1.5
 
 
+# ------------------------------------------------------------------ group-64 affine int4
+def fp16(v):
+    return np.asarray(v, np.float64).astype(np.float16).view(np.uint16)
+
+
+def test_fp16_decode_every_finite_bit_pattern():
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    ref = bits.view(np.float16).astype(np.float64)
+    finite = np.isfinite(ref)
+    got = np.array([oracle.fp16_to_double(int(b)) for b in bits[finite]])
+    assert np.array_equal(got, ref[finite])
+    assert math.isinf(oracle.fp16_to_double(0x7C00)) and math.isnan(oracle.fp16_to_double(0x7E00))
+
+
+def dequant_affine_np(q, s, m):
+    """Independent statement: unsigned nibbles (low = even element) times the
+    fp16 scale of the element's 64-group, plus that group's fp16 offset."""
+    q = np.asarray(q, np.int64)
+    codes = np.stack([q & 0xF, q >> 4], axis=-1).reshape(q.shape[0], -1).astype(np.float64)
+    sd = np.repeat(np.asarray(s, np.uint16).view(np.float16).astype(np.float64), 64, axis=1)
+    md = np.repeat(np.asarray(m, np.uint16).view(np.float16).astype(np.float64), 64, axis=1)
+    return codes * sd + md
+
+
+def test_affine_hand_case():
+    """One row of 128: group 0 has scale 0.5 and offset -1, group 1 scale 0.25
+    and offset 2; codes 0..15 then 15..0 in each group (all exact in binary)."""
+    codes = np.concatenate([np.arange(64) % 16, 15 - np.arange(64) % 16])
+    q = (codes[0::2] | (codes[1::2] << 4)).astype(np.uint8)[None, :]
+    s = fp16([[0.5, 0.25]])
+    m = fp16([[-1.0, 2.0]])
+    W = oracle.dequant_affine(q, s, m)
+    expect = np.concatenate([(np.arange(64) % 16) * 0.5 - 1.0, (15 - np.arange(64) % 16) * 0.25 + 2.0])
+    assert np.array_equal(W[0], expect)
+    x = np.zeros((1, 128), np.uint16)
+    x[0, 3], x[0, 70] = bf16(1.0), bf16(-2.0)   # 3 * 0.5 - 1 = 0.5; -2 * ((15 - 6) * 0.25 + 2) = -8.5
+    y, am, gap = oracle.int4_gemv_affine(q, s, m, x)
+    assert y[0, 0] == 0.5 - 8.5
+
+
+def test_affine_gemv_matches_numpy_fp64_matmul():
+    rng = np.random.default_rng(12)
+    N, K, B = 41, 448, 3
+    q = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    s = fp16(rng.uniform(1e-3, 5e-3, size=(N, K // 64)))
+    m = fp16(-rng.uniform(1e-2, 4e-2, size=(N, K // 64)))
+    x = bf16(rng.normal(size=(B, K)))
+    assert np.array_equal(oracle.dequant_affine(q, s, m), dequant_affine_np(q, s, m))
+    y, am, gap = oracle.int4_gemv_affine(q, s, m, x)
+    ref = synth.bf16_to_f64(x) @ dequant_affine_np(q, s, m).T
+    np.testing.assert_allclose(y, ref, rtol=1e-13, atol=1e-15)
+    assert np.array_equal(am, ref.argmax(axis=1))
+
+
+def test_affine_argmax_ties_go_to_lowest_index():
+    K = 64
+    q = np.zeros((5, K // 2), np.uint8)
+    q[1, 0] = q[3, 0] = 0x0F   # code 15 at element 0
+    s = fp16(np.full((5, 1), 0.5))
+    m = fp16(np.zeros((5, 1)))
+    x = np.zeros((1, K), np.uint16)
+    x[0, 0] = bf16(1.0)
+    y, am, gap = oracle.int4_gemv_affine(q, s, m, x)
+    assert am[0] == 1 and gap[0] == 0.0 and y[0, 1] == 7.5
+
+
 # ------------------------------------------------------------------ routing
 def brute_force_topk(b, k):
     """The unique k-subset whose members all rank above every non-member

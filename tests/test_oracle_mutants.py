@@ -50,6 +50,16 @@ MUTANTS = {
     "bf16 rounding truncates": [("nearbyint(m * 256.0)", "trunc(m * 256.0)")],
     "head ties to the highest row": [("if (yb[n] > yb[best]) best = n;",
                                       "if (yb[n] >= yb[best]) best = n;")],
+    "affine codes read as signed": [("return (k % 2 == 0) ? (byte & 0x0F) : (byte >> 4);",
+                                     "return ((k % 2 == 0) ? (byte & 0x0F) : (byte >> 4)) ^ 8;")],
+    "affine offset dropped": [("oracle_fp16_to_double(s[g]) +\n         oracle_fp16_to_double(m[g]);",
+                               "oracle_fp16_to_double(s[g]);")],
+    "affine group of 128": [("const int64_t g = n * (K / 64) + k / 64;",
+                             "const int64_t g = n * (K / 64) + (k / 128) % (K / 64);")],
+    "affine scale and offset swapped": [
+        ("(double)ucode_of(q + n * (K / 2), k) * oracle_fp16_to_double(s[g]) +\n         oracle_fp16_to_double(m[g]);",
+         "(double)ucode_of(q + n * (K / 2), k) * oracle_fp16_to_double(m[g]) +\n         oracle_fp16_to_double(s[g]);")],
+    "fp16 exponent bias 16": [("mag = ldexp((double)(1024 + f), e - 25);", "mag = ldexp((double)(1024 + f), e - 26);")],
 }
 
 
