@@ -471,6 +471,33 @@ def main():
             us = statistics.median(times)
             extra[f"head_gemv_b{hb}"] = {"us": us, "GBps": HEAD_BYTES / (us * 1e-6) / 1e9,
                                         "roofline_frac": HEAD_BYTES / (us * 1e-6) / 1e9 / hbm}
+    # ---- the head in the group-64 affine int4 format (MLX int4 / Q4_1 layout)
+    if not args.no_head and rank == 0:
+        wa = synth.to_device(synth.affine_head_host(), dev)
+        abytes = synth.VOCAB * (1024 + 2 * 64)
+        for hb in sorted({1, min(B, 8)}):
+            xh = synth.to_device({"x": synth.head_x(list(range(hb)))}, dev)["x"]
+            y = torch.empty((hb, synth.VOCAB), dtype=torch.float32, device=dev)
+            am = torch.empty(hb, dtype=torch.int32, device=dev)
+            nbh = F.flint_gemv_workspace_bytes(synth.VOCAB, hb)
+            wsh = torch.zeros(nbh, dtype=torch.uint8, device=dev)
+            F.flint_workspace_init(wsh, nbh)
+            times = []
+            for it in range(23):
+                with torch.cuda.stream(stream):
+                    flush.zero_()              # evict the head from L2 between launches
+                e0.record(stream)
+                F.flint_int4_gemv_affine(wa["q"], wa["s"], wa["m"], synth.VOCAB, H, xh, hb, y, am,
+                                         wsh, nbh, stream=stream)
+                e1.record(stream)
+                e1.synchronize()
+                if it >= 3:
+                    times.append(e0.elapsed_time(e1) * 1e3)
+            us = statistics.median(times)
+            extra[f"head_gemv_affine_b{hb}"] = {"us": us, "GBps": abytes / (us * 1e-6) / 1e9,
+                                               "roofline_frac": abytes / (us * 1e-6) / 1e9 / hbm,
+                                               "bytes": abytes}
+        del wa
     # ---- prefill of one MoE layer (layer 0): tokens/s and tensor-pipe roofline
     if not args.no_prefill and rank == 0:
         peak_tf, peak_kind_tf = tensor_peak()

@@ -234,6 +234,25 @@ FLINT_API int flint_int4_gemv(const uint8_t *q, const uint16_t *s, int N, int K,
                     float *y, int32_t *argmax, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Int4 GEMV on group-64 affine weights, the format of the MLX int4 build and
+ * of the Q4_1 GGUF ("How to Run Flint Locally", section "Every build and its
+ * size": group-64 affine int4; the same int4 codes with FP16 scales and
+ * offsets), for B in [1, 8] rows:
+ *   W[n][k] = code(n, k) * s[n][k/64] + m[n][k/64]   (code unsigned, 0..15)
+ *   y[r][n] = sum_k W[n][k] x[r][k]  (fp32 accumulation: per 64-group
+ *             scale * (codes . x) + offset * sum(x over the group))
+ *   argmax[r] = the lowest n with the largest y[r][n]   (argmax may be NULL)
+ *   q packed [N][K/2] (byte j: element 2j low nibble, 2j+1 high nibble, each
+ *     an unsigned code); s, m fp16 bits [N][K/64]; K a multiple of 128, at
+ *     most 8192
+ *   x bf16 [B][K];  y fp32 [B][N];  ws as for flint_int4_gemv
+ * Rows are batch-invariant; errors as flint_int4_gemv.
+ */
+FLINT_API int flint_int4_gemv_affine(const uint8_t *q, const uint16_t *s, const uint16_t *m, int N,
+                                     int K, const uint16_t *x, int B, float *y, int32_t *argmax,
+                                     void *ws, size_t ws_bytes, void *stream);
+
+/*
  * flint_int4_gemv without a workspace, for callers that cannot allocate
  * device memory themselves: code embedded in a host program that owns every
  * device allocation (and forbids cudaMalloc from libraries), or a hot path

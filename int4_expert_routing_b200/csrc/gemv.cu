@@ -67,10 +67,15 @@ struct GemvPlan {
   int stages;
 };
 
-static GemvPlan gemv_plan(int K, int B) {
+// Stage of one 16-row tile: codes (16 x K/2 bytes), then the symmetric
+// format's bf16 scales (16 x K/128) or the affine format's fp16 scales and
+// offsets (16 x K/64 each).  The affine fragment is followed by the per-row
+// sums of x over every 64-group (fp32, [K/64][B]).
+static GemvPlan gemv_plan(int K, int B, bool affine) {
   GemvPlan p;
-  p.stage_bytes = align256((size_t)8 * K + (size_t)K / 4);
-  p.frag_bytes = align256((size_t)(K / kG) * 4 * B * 64);
+  p.stage_bytes = align256((size_t)8 * K + (affine ? (size_t)K : (size_t)K / 4));
+  p.frag_bytes = align256((size_t)(K / kG) * 4 * B * 64) +
+                 (affine ? align256((size_t)(K / 64) * B * 4) : 0);
   p.stages = (int)((kGemvSmemCap - p.frag_bytes) / p.stage_bytes);
   if (p.stages > 16) p.stages = 16;
   p.smem = p.frag_bytes + (size_t)p.stages * p.stage_bytes;
@@ -132,6 +137,74 @@ FLINT_DEV void rows_dot(const uint8_t *qa, const uint8_t *qb, const uint16_t *sa
   }
 }
 
+// 16 unsigned codes (two words) -> 8 bf16 pairs {c(8q+p), c(8q+p+4)} at
+// register 4q+p, exact: (w & 0x000F000F) | 0x43004300 is bf16 128 + code.
+FLINT_DEV void uint4x16_to_bf16x2(const uint2 w, uint32_t (&r)[8]) {
+  const uint32_t words[2] = {w.x, w.y};
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const uint32_t t = ((words[q] >> (4 * p)) & 0x000F000Fu) | 0x43004300u;
+      uint32_t c;
+      asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(c) : "r"(t), "r"(0x43004300u));
+      r[4 * q + p] = c;
+    }
+  }
+}
+
+// Affine rows ra, rb: codes at row stride K/2 bytes; fp16 scales and offsets
+// at row stride K/64.  Lane t takes elements 64h + 16t .. 64h + 16t + 15 of
+// half h of each 128-element block, so MMAs 4h .. 4h+3 cover 64-group 2G + h
+// alone: y += scale * (codes . x) + offset * sum(x over the group).
+template <bool kGlobal>
+FLINT_DEV void rows_dot_affine(const uint8_t *qa, const uint8_t *qb, const uint16_t *sa,
+                               const uint16_t *sb, const uint16_t *ma, const uint16_t *mb, int K,
+                               int B, const uint4 *frag, const float *xsum, int lane,
+                               float (&acc)[4]) {
+  const int t = lane & 3;
+  const int ng = K / kG;
+  acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+  for (int G = 0; G < ng; ++G) {
+    uint32_t xb[16];
+    load_frag_compact(frag, G, B, lane, xb);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int off = 64 * G + 32 * h + 8 * t, grp = 2 * G + h;
+      uint2 w0, w1;
+      uint32_t s0b, s1b, m0b, m1b;
+      if (kGlobal) {
+        w0 = __ldg(reinterpret_cast<const uint2 *>(qa + off));
+        w1 = __ldg(reinterpret_cast<const uint2 *>(qb + off));
+        s0b = ld_nc_u16(sa + grp), s1b = ld_nc_u16(sb + grp);
+        m0b = ld_nc_u16(ma + grp), m1b = ld_nc_u16(mb + grp);
+      } else {
+        w0 = *reinterpret_cast<const uint2 *>(qa + off);
+        w1 = *reinterpret_cast<const uint2 *>(qb + off);
+        s0b = sa[grp], s1b = sb[grp], m0b = ma[grp], m1b = mb[grp];
+      }
+      uint32_t ra[8], rb[8];
+      uint4x16_to_bf16x2(w0, ra);
+      uint4x16_to_bf16x2(w1, rb);
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        mma_bf16_16816(d, ra[2 * j], rb[2 * j], ra[2 * j + 1], rb[2 * j + 1], xb[8 * h + 2 * j],
+                       xb[8 * h + 2 * j + 1]);
+      const float s0 = __half2float(__ushort_as_half((unsigned short)s0b));
+      const float s1 = __half2float(__ushort_as_half((unsigned short)s1b));
+      const float m0 = __half2float(__ushort_as_half((unsigned short)m0b));
+      const float m1 = __half2float(__ushort_as_half((unsigned short)m1b));
+      const int c0 = 2 * t, c1 = 2 * t + 1;
+      const float x0 = c0 < B ? xsum[grp * B + c0] : 0.f, x1 = c1 < B ? xsum[grp * B + c1] : 0.f;
+      acc[0] = fmaf(m0, x0, fmaf(d[0], s0, acc[0]));
+      acc[1] = fmaf(m0, x1, fmaf(d[1], s0, acc[1]));
+      acc[2] = fmaf(m1, x0, fmaf(d[2], s1, acc[2]));
+      acc[3] = fmaf(m1, x1, fmaf(d[3], s1, acc[3]));
+    }
+  }
+}
+
 FLINT_DEV void rows_store(const float (&acc)[4], int n_a, int n_b, int N, int B, float *y, int t,
                           float (&best_v)[2], int (&best_i)[2]) {
 #pragma unroll
@@ -150,13 +223,16 @@ FLINT_DEV void rows_store(const float (&acc)[4], int n_a, int n_b, int N, int B,
   }
 }
 
+template <bool kAffine>
 __global__ void __launch_bounds__(kGemvWarps * 32, 1)
-    k_int4_gemv(const uint8_t *__restrict__ q, const uint16_t *__restrict__ s, int N, int K,
-                const uint16_t *__restrict__ x, int B, float *__restrict__ y,
-                int32_t *__restrict__ argmax, char *__restrict__ ws, int stages,
-                uint32_t stage_bytes, uint32_t frag_bytes) {
+    k_int4_gemv(const uint8_t *__restrict__ q, const uint16_t *__restrict__ s,
+                const uint16_t *__restrict__ moff, int N, int K, const uint16_t *__restrict__ x,
+                int B, float *__restrict__ y, int32_t *__restrict__ argmax,
+                char *__restrict__ ws, int stages, uint32_t stage_bytes, uint32_t frag_bytes) {
   extern __shared__ __align__(128) unsigned char sm[];
   uint4 *frag = reinterpret_cast<uint4 *>(sm);
+  // affine: per-row sums of x over every 64-group, after the fragment
+  float *xsum = reinterpret_cast<float *>(sm + align256((size_t)(K / kG) * 4 * B * 64));
   unsigned char *ring = sm + frag_bytes;
   __shared__ __align__(8) uint64_t full[16], empty[16];
   __shared__ ArgPartial s_part[kGemvWarps][kMaxB];
@@ -168,8 +244,9 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 1)
   ArgPartial *parts = reinterpret_cast<ArgPartial *>(ws + align256(256));
   const int full_tiles = N / 16;
   const size_t rbytes = (size_t)K / 2;
-  const int ng = K / kG;
-  const uint32_t wbytes = (uint32_t)(8 * K), sbytes = (uint32_t)(K / 4);
+  const int ng = K / kG, ng64 = K / 64;
+  // per tile: codes, then scales (and, affine, offsets) of its 16 rows
+  const uint32_t wbytes = (uint32_t)(8 * K), sbytes = (uint32_t)(kAffine ? K / 2 : K / 4);
 
   if (tid == 0) {
     s_next = 0;
@@ -196,10 +273,14 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 1)
         }
         issued = k + 1;
         unsigned char *dst = ring + (size_t)st * stage_bytes;
-        mbar_expect_tx(&full[st], wbytes + sbytes);
+        mbar_expect_tx(&full[st], wbytes + (kAffine ? 2 : 1) * sbytes);
         bulk_g2s(dst, q + (size_t)tile * wbytes, wbytes, &full[st]);
         bulk_g2s(dst + wbytes, reinterpret_cast<const unsigned char *>(s) + (size_t)tile * sbytes,
                  sbytes, &full[st]);
+        if (kAffine)
+          bulk_g2s(dst + wbytes + sbytes,
+                   reinterpret_cast<const unsigned char *>(moff) + (size_t)tile * sbytes, sbytes,
+                   &full[st]);
       }
     }
     pdl_wait();
@@ -212,7 +293,20 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 1)
     for (int task = tid; task < nfrag; task += ncons * 32) {
       const int q4 = task & 3, gt = (task >> 2) % (4 * B), G = (task >> 2) / (4 * B);
       const int gg = gt >> 2, tt = gt & 3;
-      frag[task] = bf16x8_to_pairs(ld_cg_v4(x + (size_t)gg * K + 128 * G + 32 * tt + 8 * q4));
+      // symmetric: lane tt's 32 elements 32 tt ..; affine: 16 elements of each
+      // 64-half, 64 (q4 / 2) + 16 tt + 8 (q4 % 2)
+      const int e0 = kAffine ? 64 * (q4 >> 1) + 16 * tt + 8 * (q4 & 1) : 32 * tt + 8 * q4;
+      frag[task] = bf16x8_to_pairs(ld_cg_v4(x + (size_t)gg * K + 128 * G + e0));
+    }
+    if (kAffine) {  // sum of x over 64-group j of row b, elements in ascending order
+      for (int task = tid; task < ng64 * B; task += ncons * 32) {
+        const int j = task / B, b = task % B;
+        const uint16_t *xr = x + (size_t)b * K + 64 * j;
+        float sx = 0.f;
+        for (int k = 0; k < 64; ++k)
+          sx += bf16_bits_to_f32((uint32_t)__ldcg(reinterpret_cast<const unsigned short *>(xr + k)));
+        xsum[task] = sx;
+      }
     }
     asm volatile("bar.sync 1, %0;" ::"r"(ncons * 32) : "memory");  // consumers only
     const int my_tiles = full_tiles > (int)blockIdx.x
@@ -232,8 +326,15 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 1)
       const unsigned char *src = ring + (size_t)st * stage_bytes;
       const uint16_t *sc = reinterpret_cast<const uint16_t *>(src + wbytes);
       float acc[4];
-      rows_dot<false>(src + g * rbytes, src + (g + 8) * rbytes, sc + g * ng, sc + (g + 8) * ng,
-                      K, B, frag, lane, acc);
+      if (kAffine) {
+        const uint16_t *mo = reinterpret_cast<const uint16_t *>(src + wbytes + sbytes);
+        rows_dot_affine<false>(src + g * rbytes, src + (g + 8) * rbytes, sc + g * ng64,
+                               sc + (g + 8) * ng64, mo + g * ng64, mo + (g + 8) * ng64, K, B, frag,
+                               xsum, lane, acc);
+      } else {
+        rows_dot<false>(src + g * rbytes, src + (g + 8) * rbytes, sc + g * ng, sc + (g + 8) * ng,
+                        K, B, frag, lane, acc);
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);
       rows_store(acc, tile * 16 + g, tile * 16 + g + 8, N, B, y, t, best_v, best_i);
@@ -243,8 +344,12 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 1)
       const int n_a = full_tiles * 16 + g, n_b = n_a + 8;
       const size_t ra = n_a < N ? (size_t)n_a : 0, rb = n_b < N ? (size_t)n_b : 0;
       float acc[4];
-      rows_dot<true>(q + ra * rbytes, q + rb * rbytes, s + ra * ng, s + rb * ng, K, B, frag, lane,
-                     acc);
+      if (kAffine)
+        rows_dot_affine<true>(q + ra * rbytes, q + rb * rbytes, s + ra * ng64, s + rb * ng64,
+                              moff + ra * ng64, moff + rb * ng64, K, B, frag, xsum, lane, acc);
+      else
+        rows_dot<true>(q + ra * rbytes, q + rb * rbytes, s + ra * ng, s + rb * ng, K, B, frag,
+                       lane, acc);
       rows_store(acc, n_a, n_b, N, B, y, t, best_v, best_i);
     }
   }
@@ -322,13 +427,16 @@ cudaError_t gemv_set_wait_polls(uint32_t polls) {
   return cudaMemcpyToSymbol(g_gemv_polls, &polls, sizeof(polls));
 }
 
-cudaError_t launch_gemv(const uint8_t *q, const uint16_t *s, int N, int K, const uint16_t *x,
-                        int B, float *y, int32_t *argmax, char *ws, cudaStream_t st) {
-  const GemvPlan p = gemv_plan(K, B);
+template <bool kAffine>
+static cudaError_t launch_gemv_t(const uint8_t *q, const uint16_t *s, const uint16_t *m, int N,
+                                 int K, const uint16_t *x, int B, float *y, int32_t *argmax,
+                                 char *ws, cudaStream_t st) {
+  const GemvPlan p = gemv_plan(K, B, kAffine);
   note_step("k_int4_gemv plan");
   if (p.stages < 2) return cudaErrorInvalidValue;
   note_step("k_int4_gemv smem attribute");
-  cudaError_t e = cudaFuncSetAttribute(k_int4_gemv, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(k_int4_gemv<kAffine>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kGemvSmemCap);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -343,8 +451,19 @@ cudaError_t launch_gemv(const uint8_t *q, const uint16_t *s, int N, int K, const
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   note_step("k_int4_gemv launch");
-  return cudaLaunchKernelEx(&cfg, k_int4_gemv, q, s, N, K, x, B, y, argmax, ws, p.stages,
-                            (uint32_t)p.stage_bytes, (uint32_t)p.frag_bytes);
+  return cudaLaunchKernelEx(&cfg, k_int4_gemv<kAffine>, q, s, m, N, K, x, B, y, argmax, ws,
+                            p.stages, (uint32_t)p.stage_bytes, (uint32_t)p.frag_bytes);
+}
+
+cudaError_t launch_gemv(const uint8_t *q, const uint16_t *s, int N, int K, const uint16_t *x,
+                        int B, float *y, int32_t *argmax, char *ws, cudaStream_t st) {
+  return launch_gemv_t<false>(q, s, nullptr, N, K, x, B, y, argmax, ws, st);
+}
+
+cudaError_t launch_gemv_affine(const uint8_t *q, const uint16_t *s, const uint16_t *m, int N,
+                               int K, const uint16_t *x, int B, float *y, int32_t *argmax,
+                               char *ws, cudaStream_t st) {
+  return launch_gemv_t<true>(q, s, m, N, K, x, B, y, argmax, ws, st);
 }
 
 }  // namespace flint

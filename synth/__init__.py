@@ -73,6 +73,9 @@ T_RESID = 14
 T_HEAD_Q = 20
 T_HEAD_S = 21
 T_HEAD_X = 22
+T_AFF_Q = 30
+T_AFF_S = 31
+T_AFF_M = 32
 
 N_OUTLIERS = 8
 OUTLIER_GAIN = 20.0
@@ -148,6 +151,25 @@ def scale_bits(seed: int, tensor_id: int, count: int, start: int = 0) -> np.ndar
     """Group scales bf16(0.02 * U(0.5, 1.5) / 7)."""
     u = uniforms(seed, tensor_id, count, start)
     return bf16_bits(0.02 * (0.5 + u) / 7.0)
+
+
+def fp16_bits(v: np.ndarray) -> np.ndarray:
+    """fp16 bit patterns of fp64 values, rounded to nearest-even (numpy's IEEE
+    half conversion)."""
+    return np.asarray(v, np.float64).astype(np.float16).view(np.uint16)
+
+
+def affine_head_host(rows: int = VOCAB, hidden: int = HIDDEN, seed: int = 0) -> dict:
+    """A group-64 affine int4 matrix [rows, hidden] (the MLX int4 / Q4_1
+    layout): unsigned codes uniform in 0..15 (raw random bytes), per 64-group
+    fp16 scale 0.02 * U(0.5, 1.5) / 7.5 and fp16 offset -7.5 * scale * U(0.9,
+    1.1), so each group spans about [-0.02, 0.02] like the symmetric recipe."""
+    g = rows * (hidden // 64)
+    sc = 0.02 * (0.5 + uniforms(seed, T_AFF_S, g)) / 7.5
+    off = -7.5 * sc * (0.9 + 0.2 * uniforms(seed, T_AFF_M, g))
+    return {"q": random_bytes(seed, T_AFF_Q, rows * hidden // 2).reshape(rows, hidden // 2),
+            "s": fp16_bits(sc).reshape(rows, hidden // 64),
+            "m": fp16_bits(off).reshape(rows, hidden // 64)}
 
 
 def outlier_channels(hidden: int = HIDDEN, n: int = N_OUTLIERS) -> np.ndarray:
