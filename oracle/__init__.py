@@ -60,7 +60,8 @@ class _LayerC(C.Structure):
     _fields_ = [("n_experts", C.c_int), ("top_k", C.c_int), ("hidden", C.c_int),
                 ("expert_i", C.c_int), ("shared_i", C.c_int)] + [
         (n, C.c_void_p) for n in ("router_w", "router_b", "w13_q", "w13_s", "w2_q", "w2_s",
-                                  "sh13_q", "sh13_s", "sh2_q", "sh2_s")]
+                                  "sh13_q", "sh13_s", "sh2_q", "sh2_s")] + [
+        ("expert_interm_div", C.c_double)]
 
 
 _DT = {"router_w": np.uint16, "router_b": np.float32, "w13_q": np.uint8, "w13_s": np.uint16,
@@ -71,13 +72,14 @@ _DT = {"router_w": np.uint16, "router_b": np.float32, "w13_q": np.uint8, "w13_s"
 class Layer:
     """A MoE layer's host tensors (the dict ``synth.layer_host`` returns)."""
 
-    def __init__(self, t: dict, top_k: int = 6):
+    def __init__(self, t: dict, top_k: int = 6, expert_interm_div: float = 0.0):
         self.t = {k: np.ascontiguousarray(t[k], dtype=_DT[k]) for k in _DT}
         E, H = self.t["router_w"].shape
         self.E, self.H, self.k = E, H, top_k
         self.I = self.t["w13_s"].shape[1] // 2
         self.Is = self.t["sh13_s"].shape[0] // 2
-        self.c = _LayerC(E, top_k, H, self.I, self.Is, *[_p(self.t[n]).value for n in _DT])
+        self.c = _LayerC(E, top_k, H, self.I, self.Is, *[_p(self.t[n]).value for n in _DT],
+                         float(expert_interm_div))
 
 
 def unpack_int4(q: np.ndarray) -> np.ndarray:

@@ -363,9 +363,11 @@ static void moe_row(void *p, int64_t b) {
   for (int j = 0; j <= k; ++j)
     swiglu_mid(g + 2 * (size_t)I * j, j < k ? I : Is, hmid + (size_t)I * j);
   matvec_set_run(&m2);
+  /* routing weight times the divisor of the stored up projections */
+  const double div = L->expert_interm_div > 1.0 ? L->expert_interm_div : 1.0;
   for (int n = 0; n < H; ++n) out[n] = 0.0;
   for (int j = 0; j < k; ++j)
-    for (int n = 0; n < H; ++n) out[n] += w[j] * ys[(size_t)H * j + n];
+    for (int n = 0; n < H; ++n) out[n] += (w[j] * div) * ys[(size_t)H * j + n];
   for (int n = 0; n < H; ++n) out[n] += ys[(size_t)H * k + n];
   free(g);
   free(hmid);

@@ -47,6 +47,10 @@ typedef struct {
   const uint16_t *sh13_s;   /* [2Is][H/128] */
   const uint8_t *sh2_q;     /* [H][Is/2] */
   const uint16_t *sh2_s;    /* [H][Is/128] */
+  /* Routed up projections stored divided by this (TandemLLM "21 Flint",
+   * section 21.2 "The packs": expert_interm_div, the routing weights
+   * multiplied back in the combine); 0 or 1: not divided. */
+  double expert_interm_div;
 } oracle_layer;
 
 void oracle_set_threads(int n);

@@ -172,6 +172,20 @@ def affine_head_host(rows: int = VOCAB, hidden: int = HIDDEN, seed: int = 0) -> 
             "m": fp16_bits(off).reshape(rows, hidden // 64)}
 
 
+def divide_routed_up(layer: dict, log2_div: int = 7) -> dict:
+    """A copy of a layer whose routed experts' up-projection scales (rows I ..
+    2I-1 of each expert's gate/up block) are divided by 2^log2_div: the bf16
+    exponent field lowered, exact while the scales stay normal."""
+    out = dict(layer)
+    s = layer["w13_s"].copy()
+    I = s.shape[1] // 2
+    up = s[:, I:, :].astype(np.int32)
+    assert ((up >> 7) & 0xFF).min() > log2_div, "scale would leave the normal range"
+    s[:, I:, :] = (up - (log2_div << 7)).astype(np.uint16)
+    out["w13_s"] = s
+    return out
+
+
 def outlier_channels(hidden: int = HIDDEN, n: int = N_OUTLIERS) -> np.ndarray:
     """The fixed outlier channels: a partial Fisher-Yates shuffle of 0..hidden-1
     drawn from stream (0, T_OUTLIER); the first n entries, in draw order."""

@@ -405,6 +405,21 @@ def test_layer_matches_numpy_definition_random():
 
 
 # ------------------------------------------------------------------ stack
+def test_interm_div_layer_equals_undivided_layer_exactly():
+    """Routed up projections stored / 128 with the routing weights multiplied
+    back (TandemLLM "21 Flint" section 21.2, expert_interm_div): every step is
+    scaled by a power of two, so the block output equals the undivided one
+    exactly; without multiplying back it is not."""
+    t, _ = tiny_layer(E=8, H=128, I=128, Is=128, seed=21)
+    x = bf16(np.random.default_rng(22).normal(size=(3, 128)))
+    ref, idx, w, gap = oracle.moe_layer(oracle.Layer(t), x)
+    td = synth.divide_routed_up(t, 7)
+    got, idx2, w2, gap2 = oracle.moe_layer(oracle.Layer(td, expert_interm_div=128.0), x)
+    assert np.array_equal(got, ref) and np.array_equal(idx, idx2)
+    plain, *_ = oracle.moe_layer(oracle.Layer(td), x)
+    assert not np.allclose(plain, ref)
+
+
 def test_rmsnorm_closed_forms():
     h = np.zeros((2, 4), np.float32)
     h[0] = [3.0, 4.0, 0.0, 0.0]           # mean square 25/4

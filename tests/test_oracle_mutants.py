@@ -59,6 +59,8 @@ MUTANTS = {
     "affine scale and offset swapped": [
         ("(double)ucode_of(q + n * (K / 2), k) * oracle_fp16_to_double(s[g]) +\n         oracle_fp16_to_double(m[g]);",
          "(double)ucode_of(q + n * (K / 2), k) * oracle_fp16_to_double(m[g]) +\n         oracle_fp16_to_double(s[g]);")],
+    "interm_div not multiplied back": [("out[n] += (w[j] * div) * ys[(size_t)H * j + n];",
+                                        "out[n] += w[j] * ys[(size_t)H * j + n];")],
     "fp16 exponent bias 16": [("mag = ldexp((double)(1024 + f), e - 25);", "mag = ldexp((double)(1024 + f), e - 26);")],
 }
 
