@@ -78,7 +78,7 @@ enum { FLINT_OP_ROUTE = 0, FLINT_OP_DECODE = 1, FLINT_OP_PREFILL = 2, FLINT_OP_G
  *  sh13_q/s  packed [2048][2048]: shared expert, rows 0..1023 gate, 1024..2047 up
  *  sh2_q/s   packed [2048][1024]: shared expert down projection
  * Expert e's block starts at e * rows * row_bytes; the struct holds only base
- * pointers.
+ * pointers (and the up-projection divisor below).
  */
 typedef struct {
   const uint16_t *router_w;
@@ -91,6 +91,13 @@ typedef struct {
   const uint16_t *sh13_s;
   const uint8_t *sh2_q;
   const uint16_t *sh2_s;
+  /* Routed experts' up projections stored divided by this power of two (the
+   * packs' expert_interm_div of TandemLLM "21 Flint", section 21.2 "The
+   * packs": the up projection / 128 keeps SwiGLU intermediates in fp16 range;
+   * the engine multiplies the routing weights back).  0 or 1: not divided;
+   * otherwise 2^n with 1 <= n <= 16.  The block computes the same function
+   * either way: outputs equal those of the undivided weights. */
+  int expert_interm_div;
 } flint_moe_layer;
 
 /* Library version (major*10000 + minor*100 + patch). */

@@ -39,7 +39,7 @@ class FlintError(RuntimeError):
 class flint_moe_layer(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in (
         "router_w", "router_b", "w13_q", "w13_s", "w2_q", "w2_s",
-        "sh13_q", "sh13_s", "sh2_q", "sh2_s")]
+        "sh13_q", "sh13_s", "sh2_q", "sh2_s")] + [("expert_interm_div", C.c_int)]
 
 
 def build(force: bool = False) -> str:
@@ -113,11 +113,13 @@ def _check(code: int, where: str):
         raise FlintError(code, where)
 
 
-def make_layer(t: dict) -> flint_moe_layer:
-    """The C layer struct from a dict of device tensors (keys as in flint.h).
-    The struct keeps a reference to the tensors, so their memory stays
-    allocated while the struct is alive."""
-    layer = flint_moe_layer(*[_ptr(t[n]) for n, _ in flint_moe_layer._fields_])
+def make_layer(t: dict, expert_interm_div: int = 0) -> flint_moe_layer:
+    """The C layer struct from a dict of device tensors (keys as in flint.h)
+    and the divisor of the routed up projections (0: not divided).  The
+    struct keeps a reference to the tensors, so their memory stays allocated
+    while the struct is alive."""
+    layer = flint_moe_layer(*[_ptr(t[n]) for n, _ in flint_moe_layer._fields_[:-1]],
+                            int(expert_interm_div))
     layer._tensors = t
     return layer
 

@@ -13,8 +13,12 @@ namespace {
 
 bool aligned16(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// 0 or 1 (not divided), or a power of two from 2 to 2^16
+bool div_ok(int d) { return d == 0 || (d > 0 && d <= 65536 && (d & (d - 1)) == 0); }
+
 bool layer_ok(const flint_moe_layer *l) {
-  return l && aligned16(l->router_w) && aligned16(l->router_b) && aligned16(l->w13_q) &&
+  return l && div_ok(l->expert_interm_div) && aligned16(l->router_w) && aligned16(l->router_b) &&
+         aligned16(l->w13_q) &&
          aligned16(l->w13_s) && aligned16(l->w2_q) && aligned16(l->w2_s) && aligned16(l->sh13_q) &&
          aligned16(l->sh13_s) && aligned16(l->sh2_q) && aligned16(l->sh2_s);
 }

@@ -631,7 +631,9 @@ __global__ void __launch_bounds__(kK2Warps * 32)
 #pragma unroll
             for (int q = 0; q < kTopK; ++q)
               if (s_aslot[b * kTopK + q] == u) jj = q;
-            const float w = s_aw[b * kTopK + jj];
+            // the routing weight, times the divisor of the stored up rows
+            // (a power of two: the product equals the undivided one exactly)
+            const float w = s_aw[b * kTopK + jj] * L.interm_div;
             uint16_t *img = hfr + (size_t)((b * kTopK + jj) * 2) * kI;
             write_hilo(img, img + kI, r0 + g, w * (silu_f(acc[c]) * acc[2 + c]));
           }

@@ -115,11 +115,13 @@ struct LayerArgs {
   const uint16_t *sh13_s;
   const uint8_t *sh2_q;
   const uint16_t *sh2_s;
+  float interm_div;  // routed up projections stored divided by this (a power of two, >= 1)
 };
 
 inline LayerArgs layer_args(const flint_moe_layer *l) {
-  return LayerArgs{l->router_w, l->router_b, l->w13_q, l->w13_s, l->w2_q,
-                   l->w2_s,     l->sh13_q,   l->sh13_s, l->sh2_q, l->sh2_s};
+  const int d = l->expert_interm_div > 1 ? l->expert_interm_div : 1;
+  return LayerArgs{l->router_w, l->router_b, l->w13_q,  l->w13_s, l->w2_q,
+                   l->w2_s,     l->sh13_q,   l->sh13_s, l->sh2_q, l->sh2_s, (float)d};
 }
 
 // Where the calling thread's last failing CUDA call was made (for

@@ -250,10 +250,13 @@ FLINT_DEV int clamp_shift(int n) { return min(max(n, -126), 126); }
 // SwiGLU output per unit of |x|^2: by Cauchy-Schwarz |W1 x| <= |x| |W1 row| and
 // |silu(g)| <= |g|, so |silu(W1 x) (W3 x)| <= |x|^2 max|W1 row| max|W3 row|,
 // with |row| <= 8 sqrt(128 sum_g scale_g^2) for 128-wide groups of codes in [-8, 7].
+// Routed experts' up rows stored divided by `up_mul` (a power of two) count
+// with their scales times up_mul here and in the dequantization, so the
+// GEMMs see the undivided weights.
 __global__ void __launch_bounds__(256)
     k_pf_wstats(const uint16_t *__restrict__ w13_s, const uint16_t *__restrict__ w2_s,
                 const uint16_t *__restrict__ sh13_s, const uint16_t *__restrict__ sh2_s,
-                float4 *__restrict__ wst, float *__restrict__ wbound) {
+                float up_mul, float4 *__restrict__ wst, float *__restrict__ wbound) {
   pdl_wait();  // the previous kernel in the stream is complete (programmatic launch)
   pdl_trigger();
   __shared__ float red[4][8];
@@ -266,6 +269,7 @@ __global__ void __launch_bounds__(256)
   float mx1 = 0.f, mx2 = 0.f, bg = 0.f, bu = 0.f;
   for (int r = tid; r < r13; r += 256) {
     const uint4 *p = reinterpret_cast<const uint4 *>(s13 + (size_t)r * (kH / kG));
+    const float um = (!sh && r >= r13 / 2) ? up_mul : 1.f;
     float ss = 0.f;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -273,7 +277,8 @@ __global__ void __launch_bounds__(256)
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const float a = fabsf(__uint_as_float(w[q] << 16)), b = fabsf(__uint_as_float(w[q] & 0xffff0000u));
+        const float a = fabsf(__uint_as_float(w[q] << 16)) * um,
+                    b = fabsf(__uint_as_float(w[q] & 0xffff0000u)) * um;
         mx1 = fmaxf(mx1, fmaxf(a, b));
         ss = fmaf(a, a, fmaf(b, b, ss));
       }
@@ -465,6 +470,7 @@ struct GemmArgs {
   uint16_t *out_r;       // GEMM 1: Hr fp16 [6T][512]; GEMM 2: Yw bf16 [6T][2048]
   uint16_t *out_s;       // GEMM 1: Hs fp16 [T][1024]; GEMM 2: Ys bf16 [T][2048]
   uint32_t *status;
+  float up_mul;          // GEMM 1: routed up rows' scales times this (the stored divisor)
 };
 
 FLINT_DEV uint64_t sw128_desc(uint32_t saddr) {
@@ -867,6 +873,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       for (int w2 = 0; w2 < 8; ++w2) sc[w2] = w2 < tn.ng / 2 ? __ldg(srow + w2) : 0u;
       const float4 ws = __ldg(args.wst + tn.e);
       mul = kMode == 1 ? ws.x : ws.z;
+      if (kMode == 1 && (i & 1) && !tn.sh) mul *= args.up_mul;  // routed up rows: undo the divisor
     };
     uint2 wa = tile_word(args, pair, ntiles), wb = tile_word(args, pair + npairs, ntiles);
     uint32_t scn[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
@@ -1450,8 +1457,8 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
   stage_mark(2, st);
   // 3. power-of-two shifts of the fp16 operands, and the fp16 token rows
   note_step("prefill operand scaling launches");
-  if ((e = pf_launch(k_pf_wstats, kE + 1, 256, 0, st, L.w13_s, L.w2_s, L.sh13_s, L.sh2_s, wst,
-                     wbound)))
+  if ((e = pf_launch(k_pf_wstats, kE + 1, 256, 0, st, L.w13_s, L.w2_s, L.sh13_s, L.sh2_s,
+                     L.interm_div, wst, wbound)))
     return e;
   {
     int blocks = (T + 7) / 8;  // 8 tokens (warps) per block
@@ -1485,13 +1492,15 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
   if ((e = max_pairs(reinterpret_cast<const void *>(k_pf_gemm<1>), GemmCfg<1>::kSmem, &pairs1)) ||
       (e = max_pairs(reinterpret_cast<const void *>(k_pf_gemm<2>), GemmCfg<2>::kSmem, &pairs2)))
     return e;
-  GemmArgs a1{tiles1, ctrl, 3, ebase, ecount, T, L.w13_s, L.sh13_s, wst, rsc, rm3, hr, hs, ctrl + 1};
+  GemmArgs a1{tiles1, ctrl,    3,  ebase, ecount, T,  L.w13_s,   L.sh13_s,
+              wst,    rsc,     rm3, hr,   hs,     ctrl + 1, L.interm_div};
   note_step("prefill GEMM 1 launch");
   e = pf_launch(k_pf_gemm<1>, 2 * min(P.max_tiles1, pairs1), kGemmThreads, GemmCfg<1>::kSmem, st,
                 mA1r, mA1s, mB1, mB1, a1);
   if (e != cudaSuccess) return e;
   stage_mark(4, st);
-  GemmArgs a2{tiles2, ctrl, 4, ebase, ecount, T, L.w2_s, L.sh2_s, wst, rsc, rm3, yw, ys, ctrl + 1};
+  GemmArgs a2{tiles2, ctrl, 4,  ebase, ecount, T,  L.w2_s,   L.sh2_s,
+              wst,    rsc,  rm3, yw,   ys,     ctrl + 1, 1.f};
   note_step("prefill GEMM 2 launch");
   e = pf_launch(k_pf_gemm<2>, 2 * min(P.max_tiles2, pairs2), kGemmThreads, GemmCfg<2>::kSmem, st,
                 mA2r, mA2s, mB2r, mB2s, a2);
