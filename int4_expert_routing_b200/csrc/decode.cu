@@ -431,9 +431,14 @@ __global__ void __launch_bounds__(kK1Threads)
 // items 0..127; routed: item 128 + 64u + r/8 for slot u).  The item's bytes
 // (8 gate rows, 8 up rows, their scales; 16.5 KB) arrive in shared memory by
 // four bulk copies (the shared expert's before the wait on K1), the block
-// input fragment K1 published by one more after it; the 4 warps split the 16
+// input fragment K1 published by one more after it; the warps split the 16
 // k-groups and their partial sums are added in warp order.
-constexpr int kK2Warps = 4;
+#ifndef FLINT_K2_WARPS
+#define FLINT_K2_WARPS 4
+#endif
+constexpr int kK2Warps = FLINT_K2_WARPS;
+constexpr int kK2Groups = 16 / kK2Warps;  // k-groups per warp
+static_assert(kK2Warps * kK2Groups == 16, "the warps split the 16 k-groups evenly");
 constexpr int kItemBytes = 16384 + 512;
 constexpr int kSharedItems = kIs / 8;
 
@@ -462,7 +467,7 @@ FLINT_DEV void issue_item(const ItemSrc &src, unsigned char *buf, uint64_t *bar)
   bulk_g2s(buf + 16640, src.up_s, 256, bar);
 }
 
-// This warp's 4 k-groups of the item: acc[0..1] gate, [2..3] up partials for
+// This warp's k-groups of the item: acc[0..1] gate, [2..3] up partials for
 // columns 2t, 2t+1 of row r0 + g.
 FLINT_DEV void item_part(const unsigned char *buf, const uint4 *frag, int B, int warp, int lane,
                          float (&acc)[4]) {
@@ -471,8 +476,8 @@ FLINT_DEV void item_part(const unsigned char *buf, const uint4 *frag, int B, int
   const uint16_t *sg = reinterpret_cast<const uint16_t *>(buf + 16384 + g * 32);
   const uint16_t *su = reinterpret_cast<const uint16_t *>(buf + 16640 + g * 32);
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int G = 4 * warp + k;
+  for (int k = 0; k < kK2Groups; ++k) {
+    const int G = kK2Groups * warp + k;
     const uint4 wg = *reinterpret_cast<const uint4 *>(buf + g * 1024 + 64 * G + 16 * t);
     const uint4 wu = *reinterpret_cast<const uint4 *>(buf + 8192 + g * 1024 + 64 * G + 16 * t);
     uint32_t ra[16], rb[16], xb[16];
@@ -607,8 +612,12 @@ __global__ void __launch_bounds__(kK2Warps * 32)
     }
     if (warp == 0) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        acc[i] = ((s_acc[0][lane][i] + s_acc[1][lane][i]) + s_acc[2][lane][i]) + s_acc[3][lane][i];
+      for (int i = 0; i < 4; ++i) {
+        float a = s_acc[0][lane][i];
+#pragma unroll
+        for (int w = 1; w < kK2Warps; ++w) a += s_acc[w][lane][i];
+        acc[i] = a;
+      }
       if (it < kSharedItems) {
         uint16_t *hfs = reinterpret_cast<uint16_t *>(ws + lay.hfs);
         const int r = 8 * it + g;
