@@ -39,6 +39,10 @@ def lib():
         _lib.oracle_double_to_bf16.argtypes = [C.c_double]
         _lib.oracle_fp16_to_double.restype = C.c_double
         _lib.oracle_fp16_to_double.argtypes = [C.c_uint16]
+        _lib.oracle_e2m1_to_double.restype = C.c_double
+        _lib.oracle_e2m1_to_double.argtypes = [C.c_uint8]
+        _lib.oracle_e4m3_to_double.restype = C.c_double
+        _lib.oracle_e4m3_to_double.argtypes = [C.c_uint8]
         _lib.oracle_get_threads.restype = C.c_int
         set_threads(os.cpu_count() or 1)
     return _lib
@@ -144,6 +148,39 @@ def int4_gemv_affine(q: np.ndarray, s: np.ndarray, m: np.ndarray, x: np.ndarray)
     gap = np.empty(B, np.float64)
     lib().oracle_int4_gemv_affine(_p(q), _p(s), _p(m), C.c_int64(N), C.c_int64(K), _p(x),
                                   C.c_int(B), _p(y), _p(am), _p(gap))
+    return y, am, gap
+
+
+def e2m1_to_double(v: int) -> float:
+    return float(lib().oracle_e2m1_to_double(C.c_uint8(int(v))))
+
+
+def e4m3_to_double(v: int) -> float:
+    return float(lib().oracle_e4m3_to_double(C.c_uint8(int(v))))
+
+
+def dequant_nvfp4(q: np.ndarray, s: np.ndarray, global_scale: float) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    s = np.ascontiguousarray(s, dtype=np.uint8)
+    N, K = q.shape[0], 2 * q.shape[1]
+    W = np.empty((N, K), np.float64)
+    lib().oracle_dequant_nvfp4(_p(q), _p(s), C.c_float(global_scale), C.c_int64(N), C.c_int64(K),
+                               _p(W))
+    return W
+
+
+def int4_gemv_nvfp4(q: np.ndarray, s: np.ndarray, global_scale: float, x: np.ndarray):
+    """NVFP4 weight-only GEMV: (y[B,N] fp64, argmax[B] int32, top1-top2 gap[B])."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    s = np.ascontiguousarray(s, dtype=np.uint8)
+    x = np.ascontiguousarray(np.atleast_2d(x), dtype=np.uint16)
+    N, K = q.shape[0], 2 * q.shape[1]
+    B = x.shape[0]
+    y = np.empty((B, N), np.float64)
+    am = np.empty(B, np.int32)
+    gap = np.empty(B, np.float64)
+    lib().oracle_int4_gemv_nvfp4(_p(q), _p(s), C.c_float(global_scale), C.c_int64(N),
+                                 C.c_int64(K), _p(x), C.c_int(B), _p(y), _p(am), _p(gap))
     return y, am, gap
 
 

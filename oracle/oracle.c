@@ -182,6 +182,50 @@ void oracle_int4_gemv(const uint8_t *q, const uint16_t *s, int64_t N, int64_t K,
   free(xd);
 }
 
+/* ------------------------------------------------------------ NVFP4 */
+double oracle_e2m1_to_double(uint8_t v) {
+  const int sign = (v >> 3) & 1, e = (v >> 1) & 3, m = v & 1;
+  const double mag = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+  return sign ? -mag : mag;
+}
+
+double oracle_e4m3_to_double(uint8_t v) {
+  const int sign = v >> 7, e = (v >> 3) & 15, m = v & 7;
+  double mag;
+  if (e == 15 && m == 7) mag = NAN;
+  else if (e == 0) mag = ldexp((double)m, -9);            /* subnormal: m/8 * 2^-6 */
+  else mag = ldexp(1.0 + m / 8.0, e - 7);
+  return sign ? -mag : mag;
+}
+
+/* Weight element (n, k): its E2M1 code times its 16-block's E4M3 scale times the global scale. */
+static double weight_nvfp4(const uint8_t *q, const uint8_t *s, double global, int64_t K, int64_t n,
+                           int64_t k) {
+  return oracle_e2m1_to_double((uint8_t)ucode_of(q + n * (K / 2), k)) *
+         oracle_e4m3_to_double(s[n * (K / 16) + k / 16]) * global;
+}
+
+void oracle_dequant_nvfp4(const uint8_t *q, const uint8_t *s, float global, int64_t N, int64_t K,
+                          double *W) {
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k) W[n * K + k] = weight_nvfp4(q, s, (double)global, K, n, k);
+}
+
+typedef struct {
+  const uint8_t *q, *s;
+  double global;
+  int64_t K;
+  const double *x;
+  double *y;
+} gemv_nvfp4_ctx;
+
+static void gemv_nvfp4_row(void *p, int64_t n) {
+  gemv_nvfp4_ctx *c = (gemv_nvfp4_ctx *)p;
+  double acc = 0.0;
+  for (int64_t k = 0; k < c->K; ++k) acc += weight_nvfp4(c->q, c->s, c->global, c->K, n, k) * c->x[k];
+  c->y[n] = acc;
+}
+
 typedef struct {
   const uint8_t *q;
   const uint16_t *s, *m;
@@ -205,6 +249,19 @@ void oracle_int4_gemv_affine(const uint8_t *q, const uint16_t *s, const uint16_t
     to_double(x + (int64_t)b * K, K, xd);
     gemv_affine_ctx c = {q, s, m, K, xd, y + (int64_t)b * N};
     par_for(N, gemv_affine_row, &c);
+    argmax_row(y + (int64_t)b * N, N, argmax ? argmax + b : NULL, gap ? gap + b : NULL);
+  }
+  free(xd);
+}
+
+void oracle_int4_gemv_nvfp4(const uint8_t *q, const uint8_t *s, float global, int64_t N,
+                            int64_t K, const uint16_t *x, int B, double *y, int32_t *argmax,
+                            double *gap) {
+  double *xd = (double *)malloc(sizeof(double) * K);
+  for (int b = 0; b < B; ++b) {
+    to_double(x + (int64_t)b * K, K, xd);
+    gemv_nvfp4_ctx c = {q, s, (double)global, K, xd, y + (int64_t)b * N};
+    par_for(N, gemv_nvfp4_row, &c);
     argmax_row(y + (int64_t)b * N, N, argmax ? argmax + b : NULL, gap ? gap + b : NULL);
   }
   free(xd);

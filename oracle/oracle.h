@@ -80,6 +80,21 @@ void oracle_int4_gemv_affine(const uint8_t *q, const uint16_t *s, const uint16_t
                              int64_t K, const uint16_t *x, int B, double *y, int32_t *argmax,
                              double *gap);
 
+/* NVFP4 weight-only ("How to Run Flint Locally", section "What vLLM changed":
+ * the NVFP4 checkpoint runs weight-only with BF16 activations; FP4 E2M1
+ * elements, one FP8 E4M3 scale per 16 elements, one FP32 scale per tensor).
+ * Row n of an [N, K] matrix: q packed as above, each nibble an E2M1 code
+ * (sign bit 3, exponent bits 2-1 with bias 1, mantissa bit 0); s [N, K/16]
+ * E4M3 codes (sign bit 7, exponent bits 6-3 with bias 7, mantissa bits 2-0;
+ * 0x7F / 0xFF NaN); weight = e2m1 * e4m3 * global, exactly, in fp64. */
+double oracle_e2m1_to_double(uint8_t v);
+double oracle_e4m3_to_double(uint8_t v);
+void oracle_dequant_nvfp4(const uint8_t *q, const uint8_t *s, float global, int64_t N, int64_t K,
+                          double *W);
+void oracle_int4_gemv_nvfp4(const uint8_t *q, const uint8_t *s, float global, int64_t N,
+                            int64_t K, const uint16_t *x, int B, double *y, int32_t *argmax,
+                            double *gap);
+
 /* Router for B rows.  z, sig, biased: [B][E] (any may be NULL); idx, w: [B][k];
  * gap[b] = k-th minus (k+1)-th biased score in selection order. */
 void oracle_route(const oracle_layer *L, const uint16_t *x, int B, double *z, double *sig,

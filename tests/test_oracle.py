@@ -197,6 +197,67 @@ def test_affine_argmax_ties_go_to_lowest_index():
     assert am[0] == 1 and gap[0] == 0.0 and y[0, 1] == 7.5
 
 
+# ------------------------------------------------------------------ NVFP4
+def test_e2m1_values_match_the_published_table():
+    rows = [ln.split() for ln in open(os.path.join(GOLDEN, "e2m1_values.txt"))
+            if ln.strip() and not ln.startswith("#")]
+    assert len(rows) == 16
+    for code, val in rows:
+        got = oracle.e2m1_to_double(int(code, 16))
+        assert got == float(val) and math.copysign(1.0, got) == math.copysign(1.0, float(val))
+
+
+def test_e4m3_decode_every_code_against_torch():
+    import torch
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([oracle.e4m3_to_double(v) for v in range(256)])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan) and nan.sum() == 2
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+def nvfp4_dequant_np(q, s, g):
+    """Independent statement: E2M1 value of each nibble (low = even element) from
+    the published table, times the E4M3 scale of its 16-block (torch's decoder),
+    times the global scale."""
+    import torch
+    table = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6, -0.0, -0.5, -1, -1.5, -2, -3, -4, -6])
+    q = np.asarray(q, np.int64)
+    codes = np.stack([q & 0xF, q >> 4], axis=-1).reshape(q.shape[0], -1)
+    sv = torch.from_numpy(np.ascontiguousarray(s, np.uint8)).view(torch.float8_e4m3fn)
+    sv = sv.to(torch.float64).numpy()
+    return table[codes] * np.repeat(sv, 16, axis=1) * float(np.float32(g))
+
+
+def test_nvfp4_gemv_matches_numpy_fp64_matmul():
+    rng = np.random.default_rng(31)
+    N, K, B = 29, 256, 3
+    q = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    s = rng.integers(0x30, 0x70, size=(N, K // 16), dtype=np.uint8)   # finite E4M3 codes
+    g = 2.0 ** -9
+    x = bf16(rng.normal(size=(B, K)))
+    W = oracle.dequant_nvfp4(q, s, g)
+    assert np.array_equal(W, nvfp4_dequant_np(q, s, g))
+    y, am, gap = oracle.int4_gemv_nvfp4(q, s, g, x)
+    ref = synth.bf16_to_f64(x) @ W.T
+    np.testing.assert_allclose(y, ref, rtol=1e-13, atol=1e-15)
+    assert np.array_equal(am, ref.argmax(axis=1))
+
+
+def test_nvfp4_hand_case():
+    """One row of 32: block 0 scale 2 (E4M3 0x40), block 1 scale 0.25 (0x28);
+    global 0.5; x picks element 1 (code 0x3 = 1.5) with 1 and element 17 (code
+    0xF = -6) with 0.5: 1.5 * 2 * 0.5 * 1 - 6 * 0.25 * 0.5 * 0.5 = 1.125."""
+    q = np.zeros((1, 16), np.uint8)
+    q[0, 0] = 0x30          # element 1: 1.5
+    q[0, 8] = 0xF0          # element 17: -6
+    s = np.array([[0x40, 0x28]], np.uint8)
+    x = np.zeros((1, 32), np.uint16)
+    x[0, 1], x[0, 17] = bf16(1.0), bf16(0.5)
+    y, am, gap = oracle.int4_gemv_nvfp4(q, s, 0.5, x)
+    assert y[0, 0] == 1.125
+
+
 # ------------------------------------------------------------------ routing
 def brute_force_topk(b, k):
     """The unique k-subset whose members all rank above every non-member

@@ -61,6 +61,11 @@ MUTANTS = {
          "(double)ucode_of(q + n * (K / 2), k) * oracle_fp16_to_double(m[g]) +\n         oracle_fp16_to_double(s[g]);")],
     "interm_div not multiplied back": [("out[n] += (w[j] * div) * ys[(size_t)H * j + n];",
                                         "out[n] += w[j] * ys[(size_t)H * j + n];")],
+    "e2m1 exponent bias 0": [("ldexp(1.0 + 0.5 * m, e - 1)", "ldexp(1.0 + 0.5 * m, e)")],
+    "e4m3 exponent bias 8": [("mag = ldexp(1.0 + m / 8.0, e - 7);", "mag = ldexp(1.0 + m / 8.0, e - 8);")],
+    "nvfp4 scale block of 32": [("s[n * (K / 16) + k / 16]", "s[n * (K / 16) + (k / 32) % (K / 16)]")],
+    "nvfp4 global scale dropped": [("oracle_e4m3_to_double(s[n * (K / 16) + k / 16]) * global;",
+                                    "oracle_e4m3_to_double(s[n * (K / 16) + k / 16]);")],
     "fp16 exponent bias 16": [("mag = ldexp((double)(1024 + f), e - 25);", "mag = ldexp((double)(1024 + f), e - 26);")],
 }
 
