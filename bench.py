@@ -498,6 +498,32 @@ def main():
                                                "roofline_frac": abytes / (us * 1e-6) / 1e9 / hbm,
                                                "bytes": abytes}
         del wa
+        wn = synth.nvfp4_head_host()
+        wnd = synth.to_device({"q": wn["q"], "s": wn["s"]}, dev)
+        nbytes = synth.VOCAB * (1024 + 128)
+        for hb in sorted({1, min(B, 8)}):
+            xh = synth.to_device({"x": synth.head_x(list(range(hb)))}, dev)["x"]
+            y = torch.empty((hb, synth.VOCAB), dtype=torch.float32, device=dev)
+            am = torch.empty(hb, dtype=torch.int32, device=dev)
+            nbh = F.flint_gemv_workspace_bytes(synth.VOCAB, hb)
+            wsh = torch.zeros(nbh, dtype=torch.uint8, device=dev)
+            F.flint_workspace_init(wsh, nbh)
+            times = []
+            for it in range(23):
+                with torch.cuda.stream(stream):
+                    flush.zero_()              # evict the head from L2 between launches
+                e0.record(stream)
+                F.flint_int4_gemv_nvfp4(wnd["q"], wnd["s"], wn["g"], synth.VOCAB, H, xh, hb, y, am,
+                                        wsh, nbh, stream=stream)
+                e1.record(stream)
+                e1.synchronize()
+                if it >= 3:
+                    times.append(e0.elapsed_time(e1) * 1e3)
+            us = statistics.median(times)
+            extra[f"head_gemv_nvfp4_b{hb}"] = {"us": us, "GBps": nbytes / (us * 1e-6) / 1e9,
+                                              "roofline_frac": nbytes / (us * 1e-6) / 1e9 / hbm,
+                                              "bytes": nbytes}
+        del wnd
     # ---- prefill of one MoE layer (layer 0): tokens/s and tensor-pipe roofline
     if not args.no_prefill and rank == 0:
         peak_tf, peak_kind_tf = tensor_peak()

@@ -260,6 +260,27 @@ FLINT_API int flint_int4_gemv_affine(const uint8_t *q, const uint16_t *s, const 
                                      void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * GEMV on NVFP4 weights run weight-only with bf16 activations (the checkpoint
+ * the vLLM path of "How to Run Flint Locally", section "What vLLM changed",
+ * benchmarks: NVIDIA's NVFP4 format, repacked losslessly and run W4A16), for B
+ * in [1, 8] rows:
+ *   W[n][k] = e2m1(code(n, k)) * e4m3(s[n][k/16]) * global_scale
+ *   y[r][n] = sum_k W[n][k] x[r][k]  (fp32 accumulation)
+ *   argmax[r] = the lowest n with the largest y[r][n]   (argmax may be NULL)
+ *   q packed [N][K/2] (byte j: element 2j in the low nibble, 2j+1 in the high
+ *     nibble, each an FP4 E2M1 code: sign bit 3, exponent bits 2-1, mantissa
+ *     bit 0); s [N][K/16] FP8 E4M3 block scales (one byte each); K a multiple
+ *     of 128, at most 8192; global_scale a finite fp32
+ *   x bf16 [B][K];  y fp32 [B][N];  ws as for flint_int4_gemv
+ * Every code times its block scale is exact in fp16 and is multiplied on the
+ * tensor cores with x as fp16 scaled by a power of two per row (exact for
+ * elements down to 2^-24 of the row's largest); errors as flint_int4_gemv.
+ */
+FLINT_API int flint_int4_gemv_nvfp4(const uint8_t *q, const uint8_t *s, float global_scale, int N,
+                                    int K, const uint16_t *x, int B, float *y, int32_t *argmax,
+                                    void *ws, size_t ws_bytes, void *stream);
+
+/*
  * flint_int4_gemv without a workspace, for callers that cannot allocate
  * device memory themselves: code embedded in a host program that owns every
  * device allocation (and forbids cudaMalloc from libraries), or a hot path

@@ -21,7 +21,8 @@ HIDDEN, EXPERTS, TOP_K, EXPERT_I, SHARED_I, GROUP, MAX_DECODE_B = 2048, 256, 6, 
 EXPORTS = ("flint_version", "flint_strerror", "flint_last_cuda_error", "flint_workspace_bytes",
            "flint_gemv_workspace_bytes", "flint_workspace_init", "flint_read_status",
            "flint_moe_route", "flint_moe_decode", "flint_moe_decode_residual", "flint_moe_decode_stack",
-           "flint_moe_prefill", "flint_int4_gemv", "flint_int4_gemv_affine", "flint_int4_gemv_noalloc",
+           "flint_moe_prefill", "flint_int4_gemv", "flint_int4_gemv_affine", "flint_int4_gemv_nvfp4",
+           "flint_int4_gemv_noalloc",
            "flint_int4_gemv_noalloc_status",
            "flint_debug_set_wait_polls", "flint_debug_prefill_events",
            "flint_debug_prefill_stage_ms")
@@ -76,6 +77,7 @@ def lib() -> C.CDLL:
         L.flint_moe_prefill.argtypes = [lp, vp, i, vp, vp, sz, vp]
         L.flint_int4_gemv.argtypes = [vp, vp, i, i, vp, i, vp, vp, vp, sz, vp]
         L.flint_int4_gemv_affine.argtypes = [vp, vp, vp, i, i, vp, i, vp, vp, vp, sz, vp]
+        L.flint_int4_gemv_nvfp4.argtypes = [vp, vp, C.c_float, i, i, vp, i, vp, vp, vp, sz, vp]
         L.flint_int4_gemv_noalloc.argtypes = [vp, vp, i, i, vp, i, vp, vp, vp]
         L.flint_int4_gemv_noalloc_status.argtypes = [C.POINTER(C.c_int), vp]
         for name in EXPORTS:
@@ -213,6 +215,13 @@ def flint_int4_gemv_affine(q, s, m, N: int, K: int, x, B: int, y, argmax, ws, ws
     _check(lib().flint_int4_gemv_affine(_ptr(q), _ptr(s), _ptr(m), N, K, _ptr(x), B, _ptr(y),
                                         _ptr(argmax), _ptr(ws), ws_bytes, _stream(stream)),
            "flint_int4_gemv_affine")
+
+
+def flint_int4_gemv_nvfp4(q, s, global_scale: float, N: int, K: int, x, B: int, y, argmax, ws,
+                          ws_bytes: int, stream=None):
+    _check(lib().flint_int4_gemv_nvfp4(_ptr(q), _ptr(s), float(global_scale), N, K, _ptr(x), B,
+                                       _ptr(y), _ptr(argmax), _ptr(ws), ws_bytes, _stream(stream)),
+           "flint_int4_gemv_nvfp4")
 
 
 def flint_int4_gemv_noalloc(q, s, N: int, K: int, x, B: int, y, argmax, stream=None):

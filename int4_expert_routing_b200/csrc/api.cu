@@ -204,6 +204,17 @@ int flint_int4_gemv_affine(const uint8_t *q, const uint16_t *s, const uint16_t *
                                       static_cast<cudaStream_t>(stream)));
 }
 
+int flint_int4_gemv_nvfp4(const uint8_t *q, const uint8_t *s, float global_scale, int N, int K,
+                          const uint16_t *x, int B, float *y, int32_t *argmax, void *ws,
+                          size_t ws_bytes, void *stream) {
+  if (!aligned16(q) || !aligned16(s) || !aligned16(x) || !aligned16(y) || N < 1 || K < 128 ||
+      K % 128 || K > 8192 || B < 1 || B > FLINT_MAX_DECODE_B || !aligned16(ws) ||
+      ws_bytes < flint_gemv_workspace_bytes(N, B) || !(global_scale == global_scale))
+    return FLINT_EINVAL;
+  return from_cuda(launch_gemv_nvfp4(q, s, global_scale, N, K, x, B, y, argmax,
+                                     static_cast<char *>(ws), static_cast<cudaStream_t>(stream)));
+}
+
 int flint_moe_prefill(const flint_moe_layer *layer, const uint16_t *x, int T, uint16_t *out,
                       void *ws, size_t ws_bytes, void *stream) {
   if (!layer_ok(layer) || !aligned16(x) || !aligned16(out) || T < 1 || T > FLINT_MAX_PREFILL_T ||

@@ -71,9 +71,13 @@ struct GemvPlan {
 // format's bf16 scales (16 x K/128) or the affine format's fp16 scales and
 // offsets (16 x K/64 each).  The affine fragment is followed by the per-row
 // sums of x over every 64-group (fp32, [K/64][B]).
-static GemvPlan gemv_plan(int K, int B, bool affine) {
+// NVFP4: codes, then the 16 rows' E4M3 block scales (16 x K/16 bytes).
+enum { kFmtSym = 0, kFmtAffine = 1, kFmtNvfp4 = 2 };
+
+static GemvPlan gemv_plan(int K, int B, int fmt) {
+  const bool affine = fmt == kFmtAffine;
   GemvPlan p;
-  p.stage_bytes = align256((size_t)8 * K + (affine ? (size_t)K : (size_t)K / 4));
+  p.stage_bytes = align256((size_t)8 * K + (fmt == kFmtSym ? (size_t)K / 4 : (size_t)K));
   p.frag_bytes = align256((size_t)(K / kG) * 4 * B * 64) +
                  (affine ? align256((size_t)(K / 64) * B * 4) : 0);
   p.stages = (int)((kGemvSmemCap - p.frag_bytes) / p.stage_bytes);
@@ -205,6 +209,84 @@ FLINT_DEV void rows_dot_affine(const uint8_t *qa, const uint8_t *qb, const uint1
   }
 }
 
+// 8 E2M1 codes (one word; byte j = elements 2j, 2j+1 of the word's bytes)
+// -> 4 f16 pairs, exact (hardware conversion, the lower nibble to the lower
+// half).
+FLINT_DEV void e2m1x8_to_f16x2(uint32_t w, uint32_t *r) {
+  asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %4;\n"
+      "cvt.rn.f16x2.e2m1x2 %0, b0; cvt.rn.f16x2.e2m1x2 %1, b1;\n"
+      "cvt.rn.f16x2.e2m1x2 %2, b2; cvt.rn.f16x2.e2m1x2 %3, b3; }"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+      : "r"(w));
+}
+// two E4M3 codes (the lower byte first) -> f16 pair, exact
+FLINT_DEV uint32_t e4m3x2_to_f16x2(uint32_t v) {
+  uint32_t d;
+  asm("{ .reg .b16 h; cvt.u16.u32 h, %1; cvt.rn.f16x2.e4m3x2 %0, h; }" : "=r"(d) : "r"(v));
+  return d;
+}
+FLINT_DEV uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+FLINT_DEV void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                             uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// NVFP4 rows ra, rb: codes at row stride K/2 bytes, E4M3 block scales at row
+// stride K/16 bytes.  Lane t's 32 elements of a 128-block are two 16-element
+// scale blocks (2t, 2t+1); every code times its block scale is exact in fp16
+// (at most 5 significant bits, magnitudes 2^-10 .. 2,688), so the f16 MMAs
+// accumulate the exact products of the weights and the f16 activations in
+// fp32, block after block, with no per-block step (the fragment holds x in
+// natural order: pair j = elements 2j, 2j+1 of the lane's slice).
+template <bool kGlobal>
+FLINT_DEV void rows_dot_nvfp4(const uint8_t *qa, const uint8_t *qb, const uint8_t *sa,
+                              const uint8_t *sb, int K, int B, const uint4 *frag, int lane,
+                              float (&acc)[4]) {
+  const int t = lane & 3;
+  const int ng = K / kG;
+  acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+  for (int G = 0; G < ng; ++G) {
+    uint4 w0, w1;
+    uint32_t s0b, s1b;
+    if (kGlobal) {
+      w0 = ld_stream(qa + 64 * G + 16 * t);
+      w1 = ld_stream(qb + 64 * G + 16 * t);
+      s0b = ld_nc_u16(sa + 8 * G + 2 * t);
+      s1b = ld_nc_u16(sb + 8 * G + 2 * t);
+    } else {
+      w0 = *reinterpret_cast<const uint4 *>(qa + 64 * G + 16 * t);
+      w1 = *reinterpret_cast<const uint4 *>(qb + 64 * G + 16 * t);
+      s0b = *reinterpret_cast<const uint16_t *>(sa + 8 * G + 2 * t);
+      s1b = *reinterpret_cast<const uint16_t *>(sb + 8 * G + 2 * t);
+    }
+    uint32_t ra[16], rb[16], xb[16];
+    e2m1x8_to_f16x2(w0.x, ra), e2m1x8_to_f16x2(w0.y, ra + 4);
+    e2m1x8_to_f16x2(w0.z, ra + 8), e2m1x8_to_f16x2(w0.w, ra + 12);
+    e2m1x8_to_f16x2(w1.x, rb), e2m1x8_to_f16x2(w1.y, rb + 4);
+    e2m1x8_to_f16x2(w1.z, rb + 8), e2m1x8_to_f16x2(w1.w, rb + 12);
+    const uint32_t sa2 = e4m3x2_to_f16x2(s0b), sb2 = e4m3x2_to_f16x2(s1b);
+    const uint32_t sa_lo = __byte_perm(sa2, 0, 0x1010), sa_hi = __byte_perm(sa2, 0, 0x3232);
+    const uint32_t sb_lo = __byte_perm(sb2, 0, 0x1010), sb_hi = __byte_perm(sb2, 0, 0x3232);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      ra[j] = hmul2(ra[j], sa_lo), ra[8 + j] = hmul2(ra[8 + j], sa_hi);
+      rb[j] = hmul2(rb[j], sb_lo), rb[8 + j] = hmul2(rb[8 + j], sb_hi);
+    }
+    load_frag_compact(frag, G, B, lane, xb);
+#pragma unroll
+    for (int s2 = 0; s2 < 8; ++s2)
+      mma_f16_16816(acc, ra[2 * s2], rb[2 * s2], ra[2 * s2 + 1], rb[2 * s2 + 1], xb[2 * s2],
+                    xb[2 * s2 + 1]);
+  }
+}
+
 FLINT_DEV void rows_store(const float (&acc)[4], int n_a, int n_b, int N, int B, float *y, int t,
                           float (&best_v)[2], int (&best_i)[2]) {
 #pragma unroll
@@ -223,13 +305,24 @@ FLINT_DEV void rows_store(const float (&acc)[4], int n_a, int n_b, int N, int B,
   }
 }
 
-template <bool kAffine>
+// NVFP4 read-out: column c's sums times the global scale and 2^F of row c
+FLINT_DEV void nv_scale(float (&acc)[4], int t, int B, const float *ymul) {
+  const int c0 = 2 * t, c1 = 2 * t + 1;
+  const float m0 = c0 < B ? ymul[c0] : 0.f, m1 = c1 < B ? ymul[c1] : 0.f;
+  acc[0] *= m0, acc[1] *= m1, acc[2] *= m0, acc[3] *= m1;
+}
+
+template <int kFmt>
 __global__ void __launch_bounds__(kGemvWarps * 32, 1)
     k_int4_gemv(const uint8_t *__restrict__ q, const uint16_t *__restrict__ s,
-                const uint16_t *__restrict__ moff, int N, int K, const uint16_t *__restrict__ x,
-                int B, float *__restrict__ y, int32_t *__restrict__ argmax,
-                char *__restrict__ ws, int stages, uint32_t stage_bytes, uint32_t frag_bytes) {
+                const uint16_t *__restrict__ moff, float gsc, int N, int K,
+                const uint16_t *__restrict__ x, int B, float *__restrict__ y,
+                int32_t *__restrict__ argmax, char *__restrict__ ws, int stages,
+                uint32_t stage_bytes, uint32_t frag_bytes) {
+  constexpr bool kAffine = kFmt == kFmtAffine, kNv = kFmt == kFmtNvfp4;
   extern __shared__ __align__(128) unsigned char sm[];
+  __shared__ unsigned int s_xmax[kMaxB];  // NVFP4: max |x| of each row (float bits)
+  __shared__ float s_ymul[kMaxB];         // NVFP4: global scale x 2^F of each row
   uint4 *frag = reinterpret_cast<uint4 *>(sm);
   // affine: per-row sums of x over every 64-group, after the fragment
   float *xsum = reinterpret_cast<float *>(sm + align256((size_t)(K / kG) * 4 * B * 64));
@@ -246,8 +339,10 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 1)
   const size_t rbytes = (size_t)K / 2;
   const int ng = K / kG, ng64 = K / 64;
   // per tile: codes, then scales (and, affine, offsets) of its 16 rows
-  const uint32_t wbytes = (uint32_t)(8 * K), sbytes = (uint32_t)(kAffine ? K / 2 : K / 4);
+  const uint32_t wbytes = (uint32_t)(8 * K),
+                 sbytes = (uint32_t)(kAffine ? K / 2 : (kNv ? K : K / 4));
 
+  if (tid < kMaxB) s_xmax[tid] = 0u;
   if (tid == 0) {
     s_next = 0;
     for (int i = 0; i < stages; ++i) {
@@ -290,13 +385,52 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 1)
     pdl_wait();
     pdl_trigger();
     const int nfrag = ng * 4 * B * 4;
+    if (kNv) {
+      // f16 activations: row b as x 2^-F_b with F_b putting max |x| in
+      // [2^14, 2^15) (exact down to 2^-24 of the row's largest element);
+      // the output is scaled back by 2^F_b and the global scale
+      for (int task = tid; task < B * (K / 8); task += ncons * 32) {
+        const int b = task / (K / 8), c = task % (K / 8);
+        const uint4 v = ld_cg_v4(x + (size_t)b * K + 8 * c);
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+        float m = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          m = fmaxf(m, fmaxf(fabsf(__uint_as_float(wv[i] << 16)),
+                             fabsf(__uint_as_float(wv[i] & 0xffff0000u))));
+        atomicMax(&s_xmax[b], __float_as_uint(m));
+      }
+      asm volatile("bar.sync 1, %0;" ::"r"(ncons * 32) : "memory");
+      if (tid < B) {
+        const float m = __uint_as_float(s_xmax[tid]);
+        const int F = m > 0.f ? min(max(ilogbf(m) - 14, -100), 100) : 0;
+        s_ymul[tid] = gsc * ldexpf(1.f, F);
+        s_xmax[tid] = (unsigned)(F + 128);  // reused: the shift, offset by 128
+      }
+      asm volatile("bar.sync 1, %0;" ::"r"(ncons * 32) : "memory");
+    }
     for (int task = tid; task < nfrag; task += ncons * 32) {
       const int q4 = task & 3, gt = (task >> 2) % (4 * B), G = (task >> 2) / (4 * B);
       const int gg = gt >> 2, tt = gt & 3;
       // symmetric: lane tt's 32 elements 32 tt ..; affine: 16 elements of each
-      // 64-half, 64 (q4 / 2) + 16 tt + 8 (q4 % 2)
+      // 64-half, 64 (q4 / 2) + 16 tt + 8 (q4 % 2); NVFP4: 32 tt .. in natural
+      // order, as f16
       const int e0 = kAffine ? 64 * (q4 >> 1) + 16 * tt + 8 * (q4 & 1) : 32 * tt + 8 * q4;
-      frag[task] = bf16x8_to_pairs(ld_cg_v4(x + (size_t)gg * K + 128 * G + e0));
+      const uint4 v = ld_cg_v4(x + (size_t)gg * K + 128 * G + e0);
+      if (kNv) {
+        const float sc = ldexpf(1.f, 128 - (int)s_xmax[gg]);
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+        uint32_t h[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const __half lo = __float2half_rn(__uint_as_float(wv[i] << 16) * sc);
+          const __half hi = __float2half_rn(__uint_as_float(wv[i] & 0xffff0000u) * sc);
+          h[i] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+        }
+        frag[task] = make_uint4(h[0], h[1], h[2], h[3]);
+      } else {
+        frag[task] = bf16x8_to_pairs(v);
+      }
     }
     if (kAffine) {  // sum of x over 64-group j of row b, elements in ascending order
       for (int task = tid; task < ng64 * B; task += ncons * 32) {
@@ -331,6 +465,11 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 1)
         rows_dot_affine<false>(src + g * rbytes, src + (g + 8) * rbytes, sc + g * ng64,
                                sc + (g + 8) * ng64, mo + g * ng64, mo + (g + 8) * ng64, K, B, frag,
                                xsum, lane, acc);
+      } else if (kNv) {
+        const uint8_t *sc8 = src + wbytes;
+        rows_dot_nvfp4<false>(src + g * rbytes, src + (g + 8) * rbytes, sc8 + g * (K / 16),
+                              sc8 + (g + 8) * (K / 16), K, B, frag, lane, acc);
+        nv_scale(acc, t, B, s_ymul);
       } else {
         rows_dot<false>(src + g * rbytes, src + (g + 8) * rbytes, sc + g * ng, sc + (g + 8) * ng,
                         K, B, frag, lane, acc);
@@ -344,10 +483,15 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 1)
       const int n_a = full_tiles * 16 + g, n_b = n_a + 8;
       const size_t ra = n_a < N ? (size_t)n_a : 0, rb = n_b < N ? (size_t)n_b : 0;
       float acc[4];
-      if (kAffine)
+      if (kAffine) {
         rows_dot_affine<true>(q + ra * rbytes, q + rb * rbytes, s + ra * ng64, s + rb * ng64,
                               moff + ra * ng64, moff + rb * ng64, K, B, frag, xsum, lane, acc);
-      else
+      } else if (kNv) {
+        const uint8_t *s8 = reinterpret_cast<const uint8_t *>(s);
+        rows_dot_nvfp4<true>(q + ra * rbytes, q + rb * rbytes, s8 + ra * (K / 16),
+                             s8 + rb * (K / 16), K, B, frag, lane, acc);
+        nv_scale(acc, t, B, s_ymul);
+      } else
         rows_dot<true>(q + ra * rbytes, q + rb * rbytes, s + ra * ng, s + rb * ng, K, B, frag,
                        lane, acc);
       rows_store(acc, n_a, n_b, N, B, y, t, best_v, best_i);
@@ -427,15 +571,15 @@ cudaError_t gemv_set_wait_polls(uint32_t polls) {
   return cudaMemcpyToSymbol(g_gemv_polls, &polls, sizeof(polls));
 }
 
-template <bool kAffine>
-static cudaError_t launch_gemv_t(const uint8_t *q, const uint16_t *s, const uint16_t *m, int N,
-                                 int K, const uint16_t *x, int B, float *y, int32_t *argmax,
-                                 char *ws, cudaStream_t st) {
-  const GemvPlan p = gemv_plan(K, B, kAffine);
+template <int kFmt>
+static cudaError_t launch_gemv_t(const uint8_t *q, const uint16_t *s, const uint16_t *m,
+                                 float gsc, int N, int K, const uint16_t *x, int B, float *y,
+                                 int32_t *argmax, char *ws, cudaStream_t st) {
+  const GemvPlan p = gemv_plan(K, B, kFmt);
   note_step("k_int4_gemv plan");
   if (p.stages < 2) return cudaErrorInvalidValue;
   note_step("k_int4_gemv smem attribute");
-  cudaError_t e = cudaFuncSetAttribute(k_int4_gemv<kAffine>,
+  cudaError_t e = cudaFuncSetAttribute(k_int4_gemv<kFmt>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kGemvSmemCap);
   if (e != cudaSuccess) return e;
@@ -451,19 +595,26 @@ static cudaError_t launch_gemv_t(const uint8_t *q, const uint16_t *s, const uint
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   note_step("k_int4_gemv launch");
-  return cudaLaunchKernelEx(&cfg, k_int4_gemv<kAffine>, q, s, m, N, K, x, B, y, argmax, ws,
+  return cudaLaunchKernelEx(&cfg, k_int4_gemv<kFmt>, q, s, m, gsc, N, K, x, B, y, argmax, ws,
                             p.stages, (uint32_t)p.stage_bytes, (uint32_t)p.frag_bytes);
 }
 
 cudaError_t launch_gemv(const uint8_t *q, const uint16_t *s, int N, int K, const uint16_t *x,
                         int B, float *y, int32_t *argmax, char *ws, cudaStream_t st) {
-  return launch_gemv_t<false>(q, s, nullptr, N, K, x, B, y, argmax, ws, st);
+  return launch_gemv_t<kFmtSym>(q, s, nullptr, 0.f, N, K, x, B, y, argmax, ws, st);
 }
 
 cudaError_t launch_gemv_affine(const uint8_t *q, const uint16_t *s, const uint16_t *m, int N,
                                int K, const uint16_t *x, int B, float *y, int32_t *argmax,
                                char *ws, cudaStream_t st) {
-  return launch_gemv_t<true>(q, s, m, N, K, x, B, y, argmax, ws, st);
+  return launch_gemv_t<kFmtAffine>(q, s, m, 0.f, N, K, x, B, y, argmax, ws, st);
+}
+
+cudaError_t launch_gemv_nvfp4(const uint8_t *q, const uint8_t *s, float gsc, int N, int K,
+                              const uint16_t *x, int B, float *y, int32_t *argmax, char *ws,
+                              cudaStream_t st) {
+  return launch_gemv_t<kFmtNvfp4>(q, reinterpret_cast<const uint16_t *>(s), nullptr, gsc, N, K, x,
+                                  B, y, argmax, ws, st);
 }
 
 }  // namespace flint

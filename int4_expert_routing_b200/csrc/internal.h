@@ -145,6 +145,9 @@ cudaError_t launch_gemv(const uint8_t *q, const uint16_t *s, int N, int K, const
 cudaError_t launch_gemv_affine(const uint8_t *q, const uint16_t *s, const uint16_t *m, int N,
                                int K, const uint16_t *x, int B, float *y, int32_t *argmax,
                                char *ws, cudaStream_t st);
+cudaError_t launch_gemv_nvfp4(const uint8_t *q, const uint8_t *s, float gsc, int N, int K,
+                              const uint16_t *x, int B, float *y, int32_t *argmax, char *ws,
+                              cudaStream_t st);
 size_t gemv_ws_bytes(int N, int B);
 cudaError_t decode_set_wait_polls(uint32_t polls);
 cudaError_t gemv_set_wait_polls(uint32_t polls);

@@ -76,6 +76,8 @@ T_HEAD_X = 22
 T_AFF_Q = 30
 T_AFF_S = 31
 T_AFF_M = 32
+T_NV_Q = 33
+T_NV_S = 34
 
 N_OUTLIERS = 8
 OUTLIER_GAIN = 20.0
@@ -170,6 +172,20 @@ def affine_head_host(rows: int = VOCAB, hidden: int = HIDDEN, seed: int = 0) -> 
     return {"q": random_bytes(seed, T_AFF_Q, rows * hidden // 2).reshape(rows, hidden // 2),
             "s": fp16_bits(sc).reshape(rows, hidden // 64),
             "m": fp16_bits(off).reshape(rows, hidden // 64)}
+
+
+NVFP4_GLOBAL = 2.0 ** -13
+
+
+def nvfp4_head_host(rows: int = VOCAB, hidden: int = HIDDEN, seed: int = 0) -> dict:
+    """An NVFP4 matrix [rows, hidden]: E2M1 codes uniform over the 16 codes
+    (raw random bytes), one E4M3 block scale per 16 elements with exponent
+    field 13 or 14 and any mantissa (values 64 .. 240), global scale 2^-13: the
+    weights span about [-0.18, 0.18]."""
+    r = random_bytes(seed, T_NV_S, rows * (hidden // 16)).astype(np.uint32)
+    sc = (((13 + (r & 1)) << 3) | ((r >> 1) & 7)).astype(np.uint8)
+    return {"q": random_bytes(seed, T_NV_Q, rows * hidden // 2).reshape(rows, hidden // 2),
+            "s": sc.reshape(rows, hidden // 16), "g": NVFP4_GLOBAL}
 
 
 def divide_routed_up(layer: dict, log2_div: int = 7) -> dict:
