@@ -222,6 +222,17 @@ def moe_layer(L: Layer, x: np.ndarray):
     return out, idx, w, gap
 
 
+def moe_layer_partial(L: Layer, x: np.ndarray, e_lo: int, e_hi: int, with_shared: bool):
+    """out[B,H] fp64: the block's terms from routed experts [e_lo, e_hi) and,
+    with with_shared, the shared expert."""
+    x = np.ascontiguousarray(np.atleast_2d(x), dtype=np.uint16)
+    B = x.shape[0]
+    out = np.empty((B, L.H), np.float64)
+    lib().oracle_moe_layer_partial(C.byref(L.c), _p(x), C.c_int(B), C.c_int(e_lo), C.c_int(e_hi),
+                                   C.c_int(1 if with_shared else 0), _p(out))
+    return out
+
+
 def rmsnorm_bf16(h: np.ndarray, eps: float = 1e-6) -> np.ndarray:
     h = np.ascontiguousarray(np.atleast_2d(h), dtype=np.float32)
     x = np.empty(h.shape, np.uint16)

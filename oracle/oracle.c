@@ -382,6 +382,7 @@ typedef struct {
   double *out;
   int32_t *idx;
   double *w, *gap;
+  int e_lo, e_hi, with_shared; /* the experts whose terms are summed */
 } moe_ctx;
 
 static void moe_row(void *p, int64_t b) {
@@ -406,6 +407,7 @@ static void moe_row(void *p, int64_t b) {
     const int64_t e = j < k ? idx[j] : 0;
     const int inter = j < k ? I : Is;
     const size_t go = 2 * (size_t)I * j, ho = (size_t)I * j;
+    if (j < k ? (e < c->e_lo || e >= c->e_hi) : !c->with_shared) continue; /* term not summed */
     if (j < k) {
       matvec_set_add(&m13, L->w13_q + e * (2 * I) * (H / 2), L->w13_s + e * (2 * I) * (H / 128),
                      2 * inter, H, xd, g + go);
@@ -423,9 +425,12 @@ static void moe_row(void *p, int64_t b) {
   /* routing weight times the divisor of the stored up projections */
   const double div = L->expert_interm_div > 1.0 ? L->expert_interm_div : 1.0;
   for (int n = 0; n < H; ++n) out[n] = 0.0;
-  for (int j = 0; j < k; ++j)
+  for (int j = 0; j < k; ++j) {
+    if (idx[j] < c->e_lo || idx[j] >= c->e_hi) continue;
     for (int n = 0; n < H; ++n) out[n] += (w[j] * div) * ys[(size_t)H * j + n];
-  for (int n = 0; n < H; ++n) out[n] += ys[(size_t)H * k + n];
+  }
+  if (c->with_shared)
+    for (int n = 0; n < H; ++n) out[n] += ys[(size_t)H * k + n];
   free(g);
   free(hmid);
   free(ys);
@@ -436,14 +441,24 @@ static void moe_row(void *p, int64_t b) {
   free(scr);
 }
 
-void oracle_moe_layer(const oracle_layer *L, const uint16_t *x, int B, double *out,
-                      int32_t *idx, double *w, double *gap) {
-  moe_ctx c = {L, x, out, idx, w, gap};
+static void moe_rows(const oracle_layer *L, const uint16_t *x, int B, double *out, int32_t *idx,
+                     double *w, double *gap, int e_lo, int e_hi, int with_shared) {
+  moe_ctx c = {L, x, out, idx, w, gap, e_lo, e_hi, with_shared};
   if (B >= g_threads) {
     par_for(B, moe_row, &c); /* one row per worker, its products in turn */
   } else {
     for (int b = 0; b < B; ++b) moe_row(&c, b); /* rows in turn, their products threaded */
   }
+}
+
+void oracle_moe_layer(const oracle_layer *L, const uint16_t *x, int B, double *out,
+                      int32_t *idx, double *w, double *gap) {
+  moe_rows(L, x, B, out, idx, w, gap, 0, L->n_experts, 1);
+}
+
+void oracle_moe_layer_partial(const oracle_layer *L, const uint16_t *x, int B, int e_lo, int e_hi,
+                              int with_shared, double *out) {
+  moe_rows(L, x, B, out, NULL, NULL, NULL, e_lo, e_hi, with_shared);
 }
 
 /* ------------------------------------------------------------ stack layer */

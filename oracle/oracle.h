@@ -109,6 +109,13 @@ void oracle_swiglu_expert(const uint8_t *q13, const uint16_t *s13, const uint8_t
 void oracle_moe_layer(const oracle_layer *L, const uint16_t *x, int B, double *out,
                       int32_t *idx, double *w, double *gap);
 
+/* The terms of the block from the routed experts e_lo <= e < e_hi and (with
+ * with_shared) the shared expert: one rank's share under expert parallelism;
+ * the sum over a partition of the experts is the block output.  Routing is
+ * over all experts. */
+void oracle_moe_layer_partial(const oracle_layer *L, const uint16_t *x, int B, int e_lo, int e_hi,
+                              int with_shared, double *out);
+
 /* x = bf16(h / sqrt(mean(h^2) + eps)) for B rows of length H (unit weight). */
 void oracle_rmsnorm_bf16(const float *h, int B, int H, double eps, uint16_t *x);
 

@@ -481,6 +481,26 @@ def test_interm_div_layer_equals_undivided_layer_exactly():
     assert not np.allclose(plain, ref)
 
 
+@pytest.mark.parametrize("world", [2, 3, 4])
+def test_expert_partition_partials_sum_to_the_block(world):
+    """Expert parallelism's decomposition: the partials of a partition of the
+    experts (the shared expert in one of them) sum to the block output, and a
+    shard's partial does not depend on the weights of experts outside it."""
+    t, dims = tiny_layer(E=8, H=128, I=128, Is=128, seed=31)
+    x = bf16(np.random.default_rng(32).normal(size=(4, 128)))
+    L = oracle.Layer(t)
+    full, idx, w, gap = oracle.moe_layer(L, x)
+    bounds = [r * 8 // world for r in range(world + 1)]
+    parts = [oracle.moe_layer_partial(L, x, bounds[r], bounds[r + 1], r == 0) for r in range(world)]
+    np.testing.assert_allclose(sum(parts), full, rtol=1e-12, atol=1e-14)
+    assert np.array_equal(oracle.moe_layer_partial(L, x, 0, 8, True), full)
+    # experts outside shard 0 altered: shard 0's partial is unchanged
+    t2 = dict(t)
+    t2["w2_s"] = t["w2_s"].copy()
+    t2["w2_s"][bounds[1]:] = 0
+    assert np.array_equal(oracle.moe_layer_partial(oracle.Layer(t2), x, 0, bounds[1], True), parts[0])
+
+
 def test_rmsnorm_closed_forms():
     h = np.zeros((2, 4), np.float32)
     h[0] = [3.0, 4.0, 0.0, 0.0]           # mean square 25/4
