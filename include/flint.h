@@ -192,6 +192,41 @@ FLINT_API int flint_moe_decode_residual(const flint_moe_layer *layer, float *h, 
                               float *w, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * One rank's share of the decode block under expert parallelism (experts
+ * sharded by index across ranks, routing replicated; the split is the next
+ * step the workload's scope names for this path):
+ *   partial[r] = sum over row r's chosen experts e with expert_lo <= e <
+ *                expert_hi of w[r][j] * W2_e (silu(W1_e x) * (W3_e x)), in the
+ *                row's ascending expert order
+ *              + (with_shared != 0) W2_sh (silu(W1_sh x) * (W3_sh x))
+ * in fp32, before any rounding.  Routing is computed over all 256 experts (as
+ * flint_moe_route), so every rank agrees on it.  The block output is the sum
+ * of the ranks' partials (an all-reduce), finished by
+ * flint_moe_combine_partials.  Exactly one of the inputs is given: x bf16
+ * [B][2048] (the block input, as flint_moe_decode) or h fp32 [B][2048] (the
+ * residual stream, read only: x = its RMSNorm, as flint_moe_decode_residual).
+ * Only the shard's experts' weights are read, so a rank may hold only those:
+ * the layer's routed base pointers may be offset so that expert expert_lo's
+ * block sits at the rank's first shard byte (they must stay 16-byte aligned).
+ *   partial fp32 [B][2048];  0 <= expert_lo < expert_hi <= 256;  B in [1, 8]
+ *   ws  workspace of flint_workspace_bytes(FLINT_OP_DECODE, B)
+ */
+FLINT_API int flint_moe_decode_partial(const flint_moe_layer *layer, const uint16_t *x,
+                                       const float *h, int B, int expert_lo, int expert_hi,
+                                       int with_shared, float *partial, void *ws,
+                                       size_t ws_bytes, void *stream);
+
+/*
+ * The last step of a block whose output was summed from partials:
+ *   out[i] = bf16(sum[i])            (if out != NULL)
+ *   h[i]   = h[i] + bf16(sum[i])     (if h != NULL; the residual add in fp32)
+ * sum fp32 [B][2048]; out bf16 [B][2048]; h fp32 [B][2048]; at least one of
+ * out and h.
+ */
+FLINT_API int flint_moe_combine_partials(const float *sum, int B, uint16_t *out, float *h,
+                                         void *stream);
+
+/*
  * L stacked decode layers on an fp32 residual stream h [B][2048], B in
  * [1, 8], 1 <= L <= FLINT_MAX_STACK_LAYERS: flint_moe_decode_residual applied
  * with layers[0], then layers[1], ..., in one call (three programmatic-

@@ -21,6 +21,7 @@ HIDDEN, EXPERTS, TOP_K, EXPERT_I, SHARED_I, GROUP, MAX_DECODE_B = 2048, 256, 6, 
 EXPORTS = ("flint_version", "flint_strerror", "flint_last_cuda_error", "flint_workspace_bytes",
            "flint_gemv_workspace_bytes", "flint_workspace_init", "flint_read_status",
            "flint_moe_route", "flint_moe_decode", "flint_moe_decode_residual", "flint_moe_decode_stack",
+           "flint_moe_decode_partial", "flint_moe_combine_partials",
            "flint_moe_prefill", "flint_int4_gemv", "flint_int4_gemv_affine", "flint_int4_gemv_nvfp4",
            "flint_int4_gemv_noalloc",
            "flint_int4_gemv_noalloc_status",
@@ -74,6 +75,8 @@ def lib() -> C.CDLL:
         L.flint_moe_decode.argtypes = [lp, vp, i, vp, vp, sz, vp]
         L.flint_moe_decode_residual.argtypes = [lp, vp, i, vp, vp, vp, sz, vp]
         L.flint_moe_decode_stack.argtypes = [lp, i, vp, i, vp, vp, vp, vp, sz, vp]
+        L.flint_moe_decode_partial.argtypes = [lp, vp, vp, i, i, i, i, vp, vp, sz, vp]
+        L.flint_moe_combine_partials.argtypes = [vp, i, vp, vp, vp]
         L.flint_moe_prefill.argtypes = [lp, vp, i, vp, vp, sz, vp]
         L.flint_int4_gemv.argtypes = [vp, vp, i, i, vp, i, vp, vp, vp, sz, vp]
         L.flint_int4_gemv_affine.argtypes = [vp, vp, vp, i, i, vp, i, vp, vp, vp, sz, vp]
@@ -198,6 +201,22 @@ def flint_moe_decode_stack(layers, L: int, h, B: int, idx, w, h_trace, ws, ws_by
     _check(lib().flint_moe_decode_stack(layers, L, _ptr(h), B, _ptr(idx), _ptr(w), _ptr(h_trace),
                                         _ptr(ws), ws_bytes, _stream(stream)),
            "flint_moe_decode_stack")
+
+
+def flint_moe_decode_partial(layer: flint_moe_layer, x, h, B: int, expert_lo: int,
+                             expert_hi: int, with_shared: bool, partial, ws, ws_bytes: int,
+                             stream=None):
+    """One expert shard's fp32 share of the decode block (exactly one of x, h)."""
+    _check(lib().flint_moe_decode_partial(C.byref(layer), _ptr(x), _ptr(h), B, expert_lo,
+                                          expert_hi, 1 if with_shared else 0, _ptr(partial),
+                                          _ptr(ws), ws_bytes, _stream(stream)),
+           "flint_moe_decode_partial")
+
+
+def flint_moe_combine_partials(total, B: int, out, h, stream=None):
+    """out = bf16(total) and / or h += bf16(total)."""
+    _check(lib().flint_moe_combine_partials(_ptr(total), B, _ptr(out), _ptr(h), _stream(stream)),
+           "flint_moe_combine_partials")
 
 
 def flint_moe_prefill(layer: flint_moe_layer, x, T: int, out, ws, ws_bytes: int, stream=None):

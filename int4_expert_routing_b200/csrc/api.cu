@@ -154,6 +154,28 @@ int flint_moe_decode_residual(const flint_moe_layer *layer, float *h, int B, int
                                  false));
 }
 
+int flint_moe_decode_partial(const flint_moe_layer *layer, const uint16_t *x, const float *h, int B,
+                             int expert_lo, int expert_hi, int with_shared, float *partial, void *ws,
+                             size_t ws_bytes, void *stream) {
+  if (!layer_ok(layer) || (x == nullptr) == (h == nullptr) || (x && !aligned16(x)) ||
+      (h && !aligned16(h)) || !aligned16(partial) || B < 1 || B > FLINT_MAX_DECODE_B ||
+      expert_lo < 0 || expert_hi > FLINT_EXPERTS || expert_lo >= expert_hi || !aligned16(ws) ||
+      ws_bytes < flint_workspace_bytes(FLINT_OP_DECODE, B))
+    return FLINT_EINVAL;
+  DecodeShard sh;
+  sh.e_lo = expert_lo, sh.e_hi = expert_hi, sh.with_shared = with_shared != 0, sh.partial = partial;
+  return from_cuda(launch_decode(layer_args(layer), x, h, nullptr, B, nullptr, nullptr, nullptr,
+                                 static_cast<char *>(ws), static_cast<cudaStream_t>(stream), false,
+                                 sh));
+}
+
+int flint_moe_combine_partials(const float *sum, int B, uint16_t *out, float *h, void *stream) {
+  if (!aligned16(sum) || B < 1 || B > FLINT_MAX_DECODE_B || (!out && !h) ||
+      (out && !aligned16(out)) || (h && !aligned16(h)))
+    return FLINT_EINVAL;
+  return from_cuda(launch_combine_partials(sum, B, out, h, static_cast<cudaStream_t>(stream)));
+}
+
 int flint_moe_decode_stack(const flint_moe_layer *layers, int L, float *h, int B, int32_t *idx,
                            float *w, float *h_trace, void *ws, size_t ws_bytes, void *stream) {
   if (!layers || L < 1 || L > FLINT_MAX_STACK_LAYERS || !aligned16(h) || B < 1 ||

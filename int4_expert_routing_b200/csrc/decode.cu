@@ -234,7 +234,7 @@ template <bool kResidual>
 __global__ void __launch_bounds__(kK1Threads)
     k1_router(LayerArgs L, const uint16_t *__restrict__ x_in, const float *__restrict__ h, int B,
               char *__restrict__ ws, DecodeLayout lay, int32_t *__restrict__ idx_out,
-              float *__restrict__ w_out) {
+              float *__restrict__ w_out, int e_lo, int e_hi) {
   extern __shared__ __align__(128) unsigned char sm[];  // [16 rows][2064 B] | compact x fragment
   uint4 *frag = reinterpret_cast<uint4 *>(sm + 16 * kRouterRowStride);
   __shared__ __align__(8) uint64_t bar;
@@ -387,12 +387,15 @@ __global__ void __launch_bounds__(kK1Threads)
   }
   __syncthreads();
   trace_point(1, 7);
-  // slot table: experts used by any row, ascending; one expert per thread
+  // slot table: experts of this call's range [e_lo, e_hi) used by any row,
+  // ascending; one expert per thread (an expert without a slot maps to -1)
   const int e = tid;
   uint32_t m = 0;
-  for (int b = 0; b < B; ++b)
-    for (int j = 0; j < kTopK; ++j)
-      if (s_asc_e[b][j] == e) m |= 1u << b;
+  s_slot_of[e] = -1;
+  if (e >= e_lo && e < e_hi)
+    for (int b = 0; b < B; ++b)
+      for (int j = 0; j < kTopK; ++j)
+        if (s_asc_e[b][j] == e) m |= 1u << b;
   const uint32_t bal = __ballot_sync(0xffffffffu, m != 0);
   if (lane == 0) s_wcount[warp] = __popc(bal);
   __syncthreads();
@@ -497,11 +500,13 @@ FLINT_DEV void item_part(const unsigned char *buf, const uint4 *frag, int B, int
 constexpr int kK2Stages = 2;     // items in flight per CTA
 constexpr int kK2MaxItems = 16;  // items per CTA (the host sizes the grid to keep within it)
 
-// Item list of one call: shared items 0..127, then 64 items per routed slot.
+// Item list of one call: shared items 0..sh_items-1 (128, or none when the
+// shared expert is left to another call), then 64 items per routed slot.
 // CTA c takes items c, c + grid, c + 2 grid, ...; a CTA's first item is
 // fetched before the wait when it is a shared one.
 __global__ void __launch_bounds__(kK2Warps * 32)
-    k2_gateup(LayerArgs L, int B, int n_items, char *__restrict__ ws, DecodeLayout lay) {
+    k2_gateup(LayerArgs L, int B, int n_items, int sh_items, char *__restrict__ ws,
+              DecodeLayout lay) {
   extern __shared__ __align__(128) unsigned char sm[];  // stages | x fragment (compact)
   uint4 *frag = reinterpret_cast<uint4 *>(sm + kK2Stages * kItemBytes);
   __shared__ __align__(8) uint64_t bar[kK2Stages];
@@ -522,7 +527,7 @@ __global__ void __launch_bounds__(kK2Warps * 32)
   if (tid == 0) {
     for (int i = 0; i < kK2Stages; ++i) mbar_init(&bar[i], 1);
     mbar_init(&fbar, 1);
-    if (c0 < kSharedItems) {
+    if (c0 < sh_items) {
       mbar_add_tx(&bar[0], kItemBytes);
       issue_item(shared_item(L, c0), sm, &bar[0]);
     }
@@ -540,8 +545,8 @@ __global__ void __launch_bounds__(kK2Warps * 32)
   if (tid < kK2MaxItems) {
     const int it = c0 + tid * step;
     uint32_t w = kSlotInvalid;
-    if (it < kSharedItems) w = 0u;
-    else if (it < n_items) w = ld_cg_u32(slot_word + ((it - kSharedItems) >> 6));
+    if (it < sh_items) w = 0u;
+    else if (it < n_items) w = ld_cg_u32(slot_word + ((it - sh_items) >> 6));
     s_word[tid] = w;
   } else if (tid >= 32 && tid < 32 + B * kTopK) {
     s_aslot[tid - 32] = (int)ld_cg_u32(reinterpret_cast<const uint32_t *>(ws + lay.asc_slot) + tid - 32);
@@ -555,13 +560,13 @@ __global__ void __launch_bounds__(kK2Warps * 32)
     if (n > 0) {
       for (int j = 0; j < n && j < kK2Stages; ++j) {
         const int it = c0 + j * step;
-        if (j == 0 && it < kSharedItems) {
+        if (j == 0 && it < sh_items) {
           mbar_arrive(&bar[0]);  // fetched before the wait
         } else {
           mbar_add_tx(&bar[j], kItemBytes);
-          issue_item(it < kSharedItems ? shared_item(L, it)
+          issue_item(it < sh_items ? shared_item(L, it)
                                        : routed_item(L, (int)slot_expert(s_word[j]),
-                                                     8 * ((it - kSharedItems) & 63)),
+                                                     8 * ((it - sh_items) & 63)),
                      sm + j * kItemBytes, &bar[j]);
           mbar_arrive(&bar[j]);
         }
@@ -604,9 +609,9 @@ __global__ void __launch_bounds__(kK2Warps * 32)
     if (tid == 0 && j + kK2Stages < n) {
       const int jn = j + kK2Stages, itn = c0 + jn * step;
       mbar_add_tx(&bar[st], kItemBytes);
-      issue_item(itn < kSharedItems ? shared_item(L, itn)
+      issue_item(itn < sh_items ? shared_item(L, itn)
                                     : routed_item(L, (int)slot_expert(s_word[jn]),
-                                                  8 * ((itn - kSharedItems) & 63)),
+                                                  8 * ((itn - sh_items) & 63)),
                  buf, &bar[st]);
       mbar_arrive(&bar[st]);
     }
@@ -618,7 +623,7 @@ __global__ void __launch_bounds__(kK2Warps * 32)
         for (int w = 1; w < kK2Warps; ++w) a += s_acc[w][lane][i];
         acc[i] = a;
       }
-      if (it < kSharedItems) {
+      if (it < sh_items) {
         uint16_t *hfs = reinterpret_cast<uint16_t *>(ws + lay.hfs);
         const int r = 8 * it + g;
 #pragma unroll
@@ -629,7 +634,7 @@ __global__ void __launch_bounds__(kK2Warps * 32)
                        silu_f(acc[c]) * acc[2 + c]);
         }
       } else {
-        const int u = (it - kSharedItems) >> 6, r0 = 8 * ((it - kSharedItems) & 63);
+        const int u = (it - sh_items) >> 6, r0 = 8 * ((it - sh_items) & 63);
         const uint32_t mask = slot_mask(word);
         uint16_t *hfr = reinterpret_cast<uint16_t *>(ws + lay.hfr);
 #pragma unroll
@@ -676,7 +681,8 @@ struct K3Smem {
 template <bool kResidual, bool kStage>
 __global__ void __launch_bounds__(kK3Threads)
     k3_down_combine(LayerArgs L, int B, uint16_t *__restrict__ out, float *__restrict__ h,
-                    char *__restrict__ ws, DecodeLayout lay, int umax) {
+                    float *__restrict__ pout, int with_shared, char *__restrict__ ws,
+                    DecodeLayout lay, int umax) {
   extern __shared__ __align__(128) unsigned char sm[];
   const K3Smem P{umax, B};
   unsigned char *wsm = sm + P.w();
@@ -721,7 +727,7 @@ __global__ void __launch_bounds__(kK3Threads)
       bulk_g2s(ssm + tid * 128, L.w2_s + (e * kH + n0) * (kI / kG), 128, &bar);
       if (tid == 0) s_ns = min(slot_count(word), umax);
     }
-  } else if (tid == kE) {
+  } else if (tid == kE && with_shared) {
     mbar_add_tx(&bar, 8192 + 256);
     bulk_g2s(shm, L.sh2_q + (size_t)n0 * (kIs / 2), 8192, &bar);
     bulk_g2s(shs, L.sh2_s + (size_t)n0 * (kIs / kG), 256, &bar);
@@ -755,6 +761,9 @@ __global__ void __launch_bounds__(kK3Threads)
       cp_async16(reinterpret_cast<unsigned char *>(himg_s) + 16 * i, src_s + 16 * i);
     cp_async_wait_all();
   }
+  // parts no task writes (experts outside this call's range, the shared
+  // expert when it is left out) add zero
+  for (int i = tid; i < 16 * 16 * B; i += kK3Threads) ysel[i] = 0.f;
   const bool arrived = dwait(&bar, 0);
   if (__syncthreads_or(!arrived)) {
     if (tid == 0) set_status(ctrl + 1, kStatusTimeout);
@@ -772,7 +781,7 @@ __global__ void __launch_bounds__(kK3Threads)
   // The MMA's columns carry the task's rows R (those that chose the expert,
   // every row for the shared one) as pairs: column 2i the hi image of row
   // R[4p + i], column 2i+1 its lo image; one pass p per 4 rows.
-  for (int task = warp; task < 2 * ns + 4; task += kK3Threads / 32) {
+  for (int task = warp; task < 2 * ns + (with_shared ? 4 : 0); task += kK3Threads / 32) {
     const bool sh = task >= 2 * ns;
     const int slot = task >> 1;
     const int part = sh ? task - 2 * ns : task & 1;
@@ -860,7 +869,9 @@ __global__ void __launch_bounds__(kK3Threads)
 #pragma unroll
     for (int m = 0; m < 16; ++m) y += ysel[(b * 16 + m) * 16 + n];
     const size_t o = (size_t)b * kH + n0 + n;
-    if (kResidual) {
+    if (pout) {
+      pout[o] = y;  // this call's share of the block output, before any rounding
+    } else if (kResidual) {
       const float yb = __bfloat162float(__float2bfloat16_rn(y));
       h[o] = h_old + yb;
     } else {
@@ -942,27 +953,30 @@ static cudaError_t set_attrs(int dev) {
 template <bool kResidual>
 static cudaError_t launch_decode_t(const LayerArgs &L, const uint16_t *x, float *h, int B,
                                    uint16_t *out, int32_t *idx_out, float *w_out, char *ws,
-                                   cudaStream_t st, bool route_only) {
+                                   cudaStream_t st, bool route_only, const DecodeShard &sh) {
   cudaError_t err = set_attrs<kResidual>(current_device());
   if (err != cudaSuccess) return err;
   const DecodeLayout lay = decode_layout(B);
   note_step("k1_router launch");
   err = launch_pdl(k1_router<kResidual>, kRouterCtas, kK1Threads, kK1Smem, st, L, x,
-                   (const float *)h, B, ws, lay, idx_out, w_out);
+                   (const float *)h, B, ws, lay, idx_out, w_out, sh.e_lo, sh.e_hi);
   if (err != cudaSuccess || route_only) return err;
-  const int umax = kTopK * B < kE ? kTopK * B : kE;
-  const int n_items = kSharedItems + 64 * umax;
+  const int span = sh.e_hi - sh.e_lo;
+  const int umax = kTopK * B < span ? kTopK * B : span;
+  const int sh_items = sh.with_shared ? kSharedItems : 0;
+  const int n_items = sh_items + 64 * umax;
   note_step("k2_gateup launch");
-  err = launch_pdl(k2_gateup, k2_grid(current_device(), B, n_items), kK2Warps * 32, k2_smem(B),
-                   st, L, B, n_items, ws, lay);
+  err = launch_pdl(k2_gateup, k2_grid(current_device(), B, n_items > 0 ? n_items : 1),
+                   kK2Warps * 32, k2_smem(B), st, L, B, n_items, sh_items, ws, lay);
   if (err != cudaSuccess) return err;
   const K3Smem P{umax, B};
+  const int wsh = sh.with_shared ? 1 : 0;
   note_step("k3_down_combine launch");
   if (P.total(true) <= kK3MaxSmem)
     return launch_pdl(k3_down_combine<kResidual, true>, kH / 16, kK3Threads, P.total(true), st,
-                      L, B, out, h, ws, lay, umax);
+                      L, B, out, h, sh.partial, wsh, ws, lay, umax);
   return launch_pdl(k3_down_combine<kResidual, false>, kH / 16, kK3Threads, P.total(false), st, L,
-                    B, out, h, ws, lay, umax);
+                    B, out, h, sh.partial, wsh, ws, lay, umax);
 }
 
 cudaError_t decode_set_wait_polls(uint32_t polls) {
@@ -989,11 +1003,31 @@ extern "C" FLINT_API int flint_trace_dump(unsigned long long *t, unsigned int *t
 
 cudaError_t launch_decode(const LayerArgs &L, const uint16_t *x, const float *h_in, float *h_out,
                           int B, uint16_t *out, int32_t *idx_out, float *w_out, char *ws,
-                          cudaStream_t st, bool route_only) {
-  (void)h_in;
-  if (h_out)
-    return launch_decode_t<true>(L, nullptr, h_out, B, nullptr, idx_out, w_out, ws, st, false);
-  return launch_decode_t<false>(L, x, nullptr, B, out, idx_out, w_out, ws, st, route_only);
+                          cudaStream_t st, bool route_only, const DecodeShard &sh) {
+  if (h_out || h_in)
+    return launch_decode_t<true>(L, nullptr, h_out ? h_out : const_cast<float *>(h_in), B, nullptr,
+                                 idx_out, w_out, ws, st, false, sh);
+  return launch_decode_t<false>(L, x, nullptr, B, out, idx_out, w_out, ws, st, route_only, sh);
+}
+
+// out = bf16(sum) and / or h += bf16(sum): the last step of a block whose
+// output was summed from partials (one thread per element)
+__global__ void k_combine_partials(const float *__restrict__ sum, int n, uint16_t *__restrict__ out,
+                                   float *__restrict__ h) {
+  pdl_wait();
+  pdl_trigger();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float y = sum[i];
+  if (out) out[i] = f32_to_bf16_bits(y);
+  if (h) h[i] = h[i] + __bfloat162float(__float2bfloat16_rn(y));
+}
+
+cudaError_t launch_combine_partials(const float *sum, int B, uint16_t *out, float *h,
+                                    cudaStream_t st) {
+  note_step("k_combine_partials launch");
+  const int n = B * kH;
+  return launch_pdl(k_combine_partials, (n + 255) / 256, 256, 0, st, sum, n, out, h);
 }
 
 }  // namespace flint

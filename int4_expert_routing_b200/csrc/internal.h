@@ -137,9 +137,19 @@ int flint_from_cuda(cudaError_t e);
 namespace flint {
 
 // Launchers (return a cudaError_t from the launches).
+// The experts a decode call computes: [e_lo, e_hi) of the routed ones and,
+// with with_shared, the shared expert; with `partial` set, K3 writes that
+// share of the block output in fp32 instead of the bf16 output or residual.
+struct DecodeShard {
+  int e_lo = 0, e_hi = 256;
+  bool with_shared = true;
+  float *partial = nullptr;
+};
 cudaError_t launch_decode(const LayerArgs &L, const uint16_t *x, const float *h_in, float *h_out,
                           int B, uint16_t *out, int32_t *idx_out, float *w_out, char *ws,
-                          cudaStream_t st, bool route_only);
+                          cudaStream_t st, bool route_only, const DecodeShard &sh = DecodeShard());
+cudaError_t launch_combine_partials(const float *sum, int B, uint16_t *out, float *h,
+                                    cudaStream_t st);
 cudaError_t launch_gemv(const uint8_t *q, const uint16_t *s, int N, int K, const uint16_t *x,
                         int B, float *y, int32_t *argmax, char *ws, cudaStream_t st);
 cudaError_t launch_gemv_affine(const uint8_t *q, const uint16_t *s, const uint16_t *m, int N,
