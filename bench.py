@@ -35,11 +35,11 @@ N_LAYERS = synth.N_MOE_LAYERS
 H = synth.HIDDEN
 LAYER_FIXED_BYTES = 256 * 2048 * 2 + 256 * 4 + 2048 * (1024 + 32) + 2048 * (512 + 16)
 # DRAM bytes per decode layer over algorithmic bytes, from one ncu capture of
-# four stacked layers of this workload at batch 4 (110.68 MB read against
-# 109.63 MB algorithmic).  Traffic grows with the expert count the same way,
+# four stacked layers of this workload at batch 4 (110.69 MB read against
+# 109.89 MB algorithmic, caches flushed before every launch).  Traffic grows with the expert count the same way,
 # so a full layer's traffic is reported as this ratio times its algorithmic
 # bytes: a figure scaled from that capture, not measured in this run.
-DECODE_TRAFFIC_RATIO = 110.68 / 109.63
+DECODE_TRAFFIC_RATIO = 110.687744 / 109.891584
 TIMING_REPEATS = 20
 EXPERT_BYTES = 1024 * (1024 + 32) + 2048 * (256 + 8)
 HEAD_BYTES = synth.VOCAB * (1024 + 32)
