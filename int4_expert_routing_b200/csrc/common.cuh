@@ -97,13 +97,27 @@ FLINT_DEV uint32_t float_key(float f) {
 // 32 int4 codes -> 16 bf16 pairs {c(8q+p), c(8q+p+4)} at register 4q+p, exact.
 // (w & 0x000F000F) ^ 0x43084308 is bf16 128 + (nibble ^ 8) = 136 + code in
 // each half; subtracting 136 (bf16 0x4308) leaves the code.
+// (a & b) ^ c and (a & b) | c as one three-input logic operation each
+// (truth tables 0x6A and 0xEA); written out because the compiler does not
+// always fuse the pair
+FLINT_DEV uint32_t and_xor(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+FLINT_DEV uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
 FLINT_DEV void int4x32_to_bf16x2(const uint4 w, uint32_t (&r)[16]) {
   const uint32_t words[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
-      uint32_t t = ((words[q] >> (4 * p)) & 0x000F000Fu) ^ 0x43084308u;
+      const uint32_t t = and_xor(words[q] >> (4 * p), 0x000F000Fu, 0x43084308u);
       uint32_t c;
       asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(c) : "r"(t), "r"(0x43084308u));
       r[4 * q + p] = c;

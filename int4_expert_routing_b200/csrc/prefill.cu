@@ -617,10 +617,10 @@ FLINT_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync
 // m24 = s 2^24, m20 = s 2^20 and c8 = -8 s as fp16x2 (both halves equal).
 FLINT_DEV void codes8_f16(uint32_t w, uint32_t m24, uint32_t m20, uint32_t c8, uint32_t *out) {
   const uint32_t w8 = w >> 8;
-  const uint32_t t0 = (w & 0x000F000Fu) ^ 0x00080008u;   // codes 0, 4
-  const uint32_t t1 = (w & 0x00F000F0u) ^ 0x00800080u;   // codes 1, 5
-  const uint32_t t2 = (w8 & 0x000F000Fu) ^ 0x00080008u;  // codes 2, 6
-  const uint32_t t3 = (w8 & 0x00F000F0u) ^ 0x00800080u;  // codes 3, 7
+  const uint32_t t0 = and_xor(w, 0x000F000Fu, 0x00080008u);   // codes 0, 4
+  const uint32_t t1 = and_xor(w, 0x00F000F0u, 0x00800080u);   // codes 1, 5
+  const uint32_t t2 = and_xor(w8, 0x000F000Fu, 0x00080008u);  // codes 2, 6
+  const uint32_t t3 = and_xor(w8, 0x00F000F0u, 0x00800080u);  // codes 3, 7
   asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(out[0]) : "r"(t0), "r"(m24), "r"(c8));
   asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(out[1]) : "r"(t1), "r"(m20), "r"(c8));
   asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(out[2]) : "r"(t2), "r"(m24), "r"(c8));
