@@ -36,11 +36,13 @@ H = synth.HIDDEN
 LAYER_FIXED_BYTES = 256 * 2048 * 2 + 256 * 4 + 2048 * (1024 + 32) + 2048 * (512 + 16)
 # DRAM bytes per decode layer over algorithmic bytes, from one ncu capture of
 # four stacked layers of this workload at batch 4 (110.69 MB read against
-# 109.89 MB algorithmic, caches flushed before every launch).  Traffic grows with the expert count the same way,
-# so a full layer's traffic is reported as this ratio times its algorithmic
-# bytes: a figure scaled from that capture, not measured in this run.
+# 109.89 MB algorithmic, caches flushed before every launch).  Traffic grows
+# with the expert count the same way, so a full layer's traffic is reported as
+# this ratio times its algorithmic bytes: a figure scaled from that capture,
+# not measured in this run.
 DECODE_TRAFFIC_RATIO = 110.687744 / 109.891584
 TIMING_REPEATS = 20
+HEAD_COPIES = 3  # copies of the head the head timing rotates over (3 x 158.6 MB > L2)
 EXPERT_BYTES = 1024 * (1024 + 32) + 2048 * (256 + 8)
 HEAD_BYTES = synth.VOCAB * (1024 + 32)
 METRIC = "us per MoE-layer decode (B=4), fraction of HBM roofline"
@@ -444,86 +446,67 @@ def main():
     e2e_us = job_us_per_layer(mse, args.steps, nl, world)
     del ge, gwe
 
-    # ---- output head int4 GEMV (B = 1 and the bench batch), context
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    # ---- output head int4 GEMV (B = 1 and the bench batch), context.  Timed
+    # on inputs larger than L2: the launches rotate over HEAD_COPIES copies of
+    # the head (158.6 MB each), so a launch never finds its weights in L2 and
+    # no flush writes are left in L2 for it to write back.
+
+    def rotating_us(calls, iters=23, skip=3, spin_cycles=400_000):
+        """Median device time of single calls, call i on input copy i % len:
+        a GPU spin queued ahead of each start event lets the host enqueue the
+        call before the GPU reaches the event, so host launch overhead stays
+        outside the timed region."""
+        times = []
+        for it in range(iters):
+            with torch.cuda.stream(stream):
+                torch.cuda._sleep(spin_cycles)
+                e0.record(stream)
+                calls[it % len(calls)]()
+                e1.record(stream)
+            e1.synchronize()
+            if it >= skip:
+                times.append(e0.elapsed_time(e1) * 1e3)
+        return statistics.median(times)
+
+    def head_case(name, nbytes, launch, copies):
+        for hb in sorted({1, min(B, 8)}):
+            xh = synth.to_device({"x": synth.head_x(list(range(hb)))}, dev)["x"]
+            y = torch.empty((hb, synth.VOCAB), dtype=torch.float32, device=dev)
+            am = torch.empty(hb, dtype=torch.int32, device=dev)
+            nbh = F.flint_gemv_workspace_bytes(synth.VOCAB, hb)
+            wsh = torch.zeros(nbh, dtype=torch.uint8, device=dev)
+            F.flint_workspace_init(wsh, nbh)
+            us = rotating_us([lambda c=c: launch(c, xh, hb, y, am, wsh, nbh) for c in copies])
+            extra[f"{name}_b{hb}"] = {"us": us, "GBps": nbytes / (us * 1e-6) / 1e9,
+                                      "roofline_frac": nbytes / (us * 1e-6) / 1e9 / hbm,
+                                      "bytes": nbytes}
+
     if not args.no_head and rank == 0:
         hq = synth.random_bytes_torch(0, synth.T_HEAD_Q, synth.VOCAB * H // 2, dev).view(
             synth.VOCAB, H // 2)
         hs_ = synth.to_device({"s": synth.head_host(with_codes=False)["s"]}, dev)["s"]
-        for hb in sorted({1, min(B, 8)}):
-            xh = synth.to_device({"x": synth.head_x(list(range(hb)))}, dev)["x"]
-            y = torch.empty((hb, synth.VOCAB), dtype=torch.float32, device=dev)
-            am = torch.empty(hb, dtype=torch.int32, device=dev)
-            nbh = F.flint_gemv_workspace_bytes(synth.VOCAB, hb)
-            wsh = torch.zeros(nbh, dtype=torch.uint8, device=dev)
-            F.flint_workspace_init(wsh, nbh)
-            times = []
-            for it in range(23):
-                with torch.cuda.stream(stream):
-                    flush.zero_()              # evict the head from L2 between launches
-                e0.record(stream)
-                F.flint_int4_gemv(hq, hs_, synth.VOCAB, H, xh, hb, y, am, wsh, nbh,
-                                  stream=stream)
-                e1.record(stream)
-                e1.synchronize()
-                if it >= 3:
-                    times.append(e0.elapsed_time(e1) * 1e3)
-            us = statistics.median(times)
-            extra[f"head_gemv_b{hb}"] = {"us": us, "GBps": HEAD_BYTES / (us * 1e-6) / 1e9,
-                                        "roofline_frac": HEAD_BYTES / (us * 1e-6) / 1e9 / hbm}
-    # ---- the head in the group-64 affine int4 format (MLX int4 / Q4_1 layout)
-    if not args.no_head and rank == 0:
+        copies = [(hq, hs_)] + [(hq.clone(), hs_.clone()) for _ in range(HEAD_COPIES - 1)]
+        head_case("head_gemv", HEAD_BYTES,
+                  lambda c, xh, hb, y, am, w, n: F.flint_int4_gemv(
+                      c[0], c[1], synth.VOCAB, H, xh, hb, y, am, w, n, stream=stream), copies)
+        del copies, hq, hs_
+        # the group-64 affine int4 format (MLX int4 / Q4_1 layout)
         wa = synth.to_device(synth.affine_head_host(), dev)
-        abytes = synth.VOCAB * (1024 + 2 * 64)
-        for hb in sorted({1, min(B, 8)}):
-            xh = synth.to_device({"x": synth.head_x(list(range(hb)))}, dev)["x"]
-            y = torch.empty((hb, synth.VOCAB), dtype=torch.float32, device=dev)
-            am = torch.empty(hb, dtype=torch.int32, device=dev)
-            nbh = F.flint_gemv_workspace_bytes(synth.VOCAB, hb)
-            wsh = torch.zeros(nbh, dtype=torch.uint8, device=dev)
-            F.flint_workspace_init(wsh, nbh)
-            times = []
-            for it in range(23):
-                with torch.cuda.stream(stream):
-                    flush.zero_()              # evict the head from L2 between launches
-                e0.record(stream)
-                F.flint_int4_gemv_affine(wa["q"], wa["s"], wa["m"], synth.VOCAB, H, xh, hb, y, am,
-                                         wsh, nbh, stream=stream)
-                e1.record(stream)
-                e1.synchronize()
-                if it >= 3:
-                    times.append(e0.elapsed_time(e1) * 1e3)
-            us = statistics.median(times)
-            extra[f"head_gemv_affine_b{hb}"] = {"us": us, "GBps": abytes / (us * 1e-6) / 1e9,
-                                               "roofline_frac": abytes / (us * 1e-6) / 1e9 / hbm,
-                                               "bytes": abytes}
-        del wa
+        copies = [wa] + [{k: v.clone() for k, v in wa.items()} for _ in range(HEAD_COPIES - 1)]
+        head_case("head_gemv_affine", synth.VOCAB * (1024 + 2 * 64),
+                  lambda c, xh, hb, y, am, w, n: F.flint_int4_gemv_affine(
+                      c["q"], c["s"], c["m"], synth.VOCAB, H, xh, hb, y, am, w, n,
+                      stream=stream), copies)
+        del copies, wa
+        # NVFP4 (E2M1 codes, E4M3 scale per 16, fp32 global scale)
         wn = synth.nvfp4_head_host()
         wnd = synth.to_device({"q": wn["q"], "s": wn["s"]}, dev)
-        nbytes = synth.VOCAB * (1024 + 128)
-        for hb in sorted({1, min(B, 8)}):
-            xh = synth.to_device({"x": synth.head_x(list(range(hb)))}, dev)["x"]
-            y = torch.empty((hb, synth.VOCAB), dtype=torch.float32, device=dev)
-            am = torch.empty(hb, dtype=torch.int32, device=dev)
-            nbh = F.flint_gemv_workspace_bytes(synth.VOCAB, hb)
-            wsh = torch.zeros(nbh, dtype=torch.uint8, device=dev)
-            F.flint_workspace_init(wsh, nbh)
-            times = []
-            for it in range(23):
-                with torch.cuda.stream(stream):
-                    flush.zero_()              # evict the head from L2 between launches
-                e0.record(stream)
-                F.flint_int4_gemv_nvfp4(wnd["q"], wnd["s"], wn["g"], synth.VOCAB, H, xh, hb, y, am,
-                                        wsh, nbh, stream=stream)
-                e1.record(stream)
-                e1.synchronize()
-                if it >= 3:
-                    times.append(e0.elapsed_time(e1) * 1e3)
-            us = statistics.median(times)
-            extra[f"head_gemv_nvfp4_b{hb}"] = {"us": us, "GBps": nbytes / (us * 1e-6) / 1e9,
-                                              "roofline_frac": nbytes / (us * 1e-6) / 1e9 / hbm,
-                                              "bytes": nbytes}
-        del wnd
+        copies = [wnd] + [{k: v.clone() for k, v in wnd.items()} for _ in range(HEAD_COPIES - 1)]
+        head_case("head_gemv_nvfp4", synth.VOCAB * (1024 + 128),
+                  lambda c, xh, hb, y, am, w, n: F.flint_int4_gemv_nvfp4(
+                      c["q"], c["s"], wn["g"], synth.VOCAB, H, xh, hb, y, am, w, n,
+                      stream=stream), copies)
+        del copies, wnd
     # ---- prefill of one MoE layer (layer 0): tokens/s and tensor-pipe roofline
     if not args.no_prefill and rank == 0:
         peak_tf, peak_kind_tf = tensor_peak()
@@ -533,25 +516,20 @@ def main():
             nbp = F.flint_workspace_bytes(F.FLINT_OP_PREFILL, T)
             wsp = torch.zeros(nbp, dtype=torch.uint8, device=dev)
             F.flint_workspace_init(wsp, nbp)
-            times = []
-            for it in range(7):
-                with torch.cuda.stream(stream):
-                    flush.zero_()  # evict L2 between runs
-                    e0.record(stream)
-                    F.flint_moe_prefill(structs[0], xt, T, out_t, wsp, nbp, stream=stream)
-                    e1.record(stream)
-                e1.synchronize()
-                if it >= 2:
-                    times.append(e0.elapsed_time(e1) * 1e3)
-            us = statistics.median(times)
+            # inputs larger than L2: the runs rotate over layers 0..2 (420 MB of
+            # weights each), so no run finds its weights in L2
+            pf_layers = structs[:min(3, nl)]
+            us = rotating_us([lambda l=l: F.flint_moe_prefill(l, xt, T, out_t, wsp, nbp,
+                                                              stream=stream)
+                              for l in pf_layers], iters=8, skip=2, spin_cycles=2_000_000)
             tflops = T * PREFILL_FLOP_PER_TOKEN / (us * 1e-6) / 1e12
             # per-stage CUDA-event times inside the call (library measurement hook)
             stage_runs = []
             F.flint_debug_prefill_events(True)
             for it in range(3):
                 with torch.cuda.stream(stream):
-                    flush.zero_()
-                    F.flint_moe_prefill(structs[0], xt, T, out_t, wsp, nbp, stream=stream)
+                    F.flint_moe_prefill(pf_layers[it % len(pf_layers)], xt, T, out_t, wsp, nbp,
+                                        stream=stream)
                 stage_runs.append(F.flint_debug_prefill_stage_ms())
             F.flint_debug_prefill_events(False)
             stages_us = {k: 1e3 * statistics.median(r[k] for r in stage_runs) for k in stage_runs[0]}
