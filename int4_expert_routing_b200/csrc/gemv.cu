@@ -135,23 +135,6 @@ static GemvPlan gemv_plan(int K, int B, int fmt) {
   return p;
 }
 
-// Compact activation fragment: only the B live columns (lanes g < B) are
-// stored, frag[(G * 4B + g * 4 + t) * 4 + q] (uint4); other lanes read zeros.
-FLINT_DEV void load_frag_compact(const uint4 *frag, int G, int B, int lane, uint32_t (&x)[16]) {
-  const int g = lane >> 2, t = lane & 3;
-  if (g < B) {
-    const uint4 *p = frag + (size_t)(G * 4 * B + g * 4 + t) * 4;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 v = p[i];
-      x[4 * i] = v.x, x[4 * i + 1] = v.y, x[4 * i + 2] = v.z, x[4 * i + 3] = v.w;
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) x[i] = 0u;
-  }
-}
-
 // The lane's 16 fragment registers of k-group G for the live columns (lanes
 // g < B); lanes g >= B keep what they hold (zeros from the caller): their MMA
 // columns are never stored.
@@ -272,26 +255,13 @@ FLINT_DEV void rows_dot_reg(const uint8_t *qa, const uint8_t *qb, const uint16_t
   }
 }
 
-// 16 unsigned codes (two words) -> 8 bf16 pairs {c(8q+p), c(8q+p+4)} at
-// register 4q+p, exact: (w & 0x000F000F) | 0x43004300 is bf16 128 + code.
-FLINT_DEV void uint4x16_to_bf16x2(const uint2 w, uint32_t (&r)[8]) {
-  const uint32_t words[2] = {w.x, w.y};
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      const uint32_t t = and_or(words[q] >> (4 * p), 0x000F000Fu, 0x43004300u);
-      uint32_t c;
-      asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(c) : "r"(t), "r"(0x43004300u));
-      r[4 * q + p] = c;
-    }
-  }
-}
-
 // Affine rows ra, rb: codes at row stride K/2 bytes; fp16 scales and offsets
 // at row stride K/64.  Lane t takes elements 64h + 16t .. 64h + 16t + 15 of
 // half h of each 128-element block, so MMAs 4h .. 4h+3 cover 64-group 2G + h
-// alone: y += scale * (codes . x) + offset * sum(x over the group).
+// alone: the f16 MMAs sum the exact products n 2^-24 x of the unsigned codes
+// n (fields read as subnormals, as in the symmetric path), and
+// y += scale * 2^24 d + offset * sum(x over the group), in the activations'
+// shifted units.  xsum: [K/64][B] sums of the shifted x.
 template <bool kGlobal>
 FLINT_DEV void rows_dot_affine(const uint8_t *qa, const uint8_t *qb, const uint16_t *sa,
                                const uint16_t *sb, const uint16_t *ma, const uint16_t *mb, int G0,
@@ -299,9 +269,11 @@ FLINT_DEV void rows_dot_affine(const uint8_t *qa, const uint8_t *qb, const uint1
                                float (&acc)[4]) {
   const int t = lane & 3;
   acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+  uint32_t xb[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) xb[i] = 0u;
   for (int G = G0; G < G1; ++G) {
-    uint32_t xb[16];
-    load_frag_compact(frag, G, B, lane, xb);
+    load_frag_live(frag, G, B, lane, xb);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int off = 64 * G + 32 * h + 8 * t, grp = 2 * G + h;
@@ -318,15 +290,15 @@ FLINT_DEV void rows_dot_affine(const uint8_t *qa, const uint8_t *qb, const uint1
         s0b = sa[grp], s1b = sb[grp], m0b = ma[grp], m1b = mb[grp];
       }
       uint32_t ra[8], rb[8];
-      uint4x16_to_bf16x2(w0, ra);
-      uint4x16_to_bf16x2(w1, rb);
+      fields8_f16sub<0>(w0.x, ra), fields8_f16sub<0>(w0.y, ra + 4);
+      fields8_f16sub<0>(w1.x, rb), fields8_f16sub<0>(w1.y, rb + 4);
       float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int j = 0; j < 4; ++j)
-        mma_bf16_16816(d, ra[2 * j], rb[2 * j], ra[2 * j + 1], rb[2 * j + 1], xb[8 * h + 2 * j],
-                       xb[8 * h + 2 * j + 1]);
-      const float s0 = __half2float(__ushort_as_half((unsigned short)s0b));
-      const float s1 = __half2float(__ushort_as_half((unsigned short)s1b));
+        mma_f16_16816(d, ra[2 * j], rb[2 * j], ra[2 * j + 1], rb[2 * j + 1], xb[8 * h + 2 * j],
+                      xb[8 * h + 2 * j + 1]);
+      const float s0 = __half2float(__ushort_as_half((unsigned short)s0b)) * 0x1p24f;
+      const float s1 = __half2float(__ushort_as_half((unsigned short)s1b)) * 0x1p24f;
       const float m0 = __half2float(__ushort_as_half((unsigned short)m0b));
       const float m1 = __half2float(__ushort_as_half((unsigned short)m1b));
       const int c0 = 2 * t, c1 = 2 * t + 1;
@@ -448,7 +420,6 @@ __global__ void __launch_bounds__((kGW ? kRegWarps : kGemvWarps) * 32, 1)
                 int32_t *__restrict__ argmax, char *__restrict__ ws, int stages,
                 uint32_t stage_bytes, uint32_t frag_bytes) {
   constexpr bool kAffine = kFmt == kFmtAffine, kNv = kFmt == kFmtNvfp4, kSym = kFmt == kFmtSym;
-  constexpr bool kF16x = kNv || kSym;  // f16 activations, shifted by a power of two per row
   extern __shared__ __align__(128) unsigned char sm[];
   __shared__ unsigned int s_xmax[kMaxB];  // max |x| of each row (float bits), then its shift
   __shared__ float s_ymul[kMaxB];         // 2^F of each row (NVFP4: times the global scale)
@@ -526,11 +497,11 @@ __global__ void __launch_bounds__((kGW ? kRegWarps : kGemvWarps) * 32, 1)
     const int nfrag = ng * 4 * B * 4;
     if (kSym)
       for (int i = tid; i < ng * 8; i += ncons * 32) xsum[i] = 0.f;
-    if (kF16x) {
+    {
       // f16 activations: row b as x 2^-F_b with F_b putting max |x| in
       // [2^14, 2^15) (exact down to 2^-24 of the row's largest element);
-      // the output is scaled back by 2^F_b and the global scale
-      // one 16-byte chunk per thread, a maximum over each half-warp (16
+      // the output is scaled back by 2^F_b (NVFP4: and the global scale).
+      // One 16-byte chunk per thread, a maximum over each half-warp (16
       // consecutive chunks of one row, K/8 being a multiple of 16), then one
       // shared atomic per half-warp
       for (int task = tid; task < B * (K / 8); task += ncons * 32) {
@@ -564,54 +535,44 @@ __global__ void __launch_bounds__((kGW ? kRegWarps : kGemvWarps) * 32, 1)
       // affine: 16 elements of each 64-half, 64 (q4 / 2) + 16 tt + 8 (q4 % 2)
       const int e0 = kAffine ? 64 * (q4 >> 1) + 16 * tt + 8 * (q4 & 1) : 32 * tt + 8 * q4;
       const uint4 v = ld_cg_v4(x + (size_t)gg * K + 128 * G + e0);
-      if (kF16x) {
-        const float sc = ldexpf(1.f, 128 - (int)s_xmax[gg]);
-        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-        uint32_t h[4];
-        float part = 0.f;  // symmetric: sum of the 8 shifted values, in element order
+      const float sc = ldexpf(1.f, 128 - (int)s_xmax[gg]);
+      const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+      uint32_t h[4];
+      float part = 0.f;  // sum of the 8 shifted values, in element order
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          if (kNv) {  // natural order: pair i = elements 2i, 2i+1
-            const __half lo = __float2half_rn(__uint_as_float(wv[i] << 16) * sc);
-            const __half hi = __float2half_rn(__uint_as_float(wv[i] & 0xffff0000u) * sc);
-            h[i] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
-          } else {    // pair i = elements i, i + 4; odd i carry 2^-4
-            const uint32_t wl = wv[i >> 1], wh = wv[(i >> 1) + 2];
-            const float xl = __uint_as_float((i & 1) ? (wl & 0xffff0000u) : (wl << 16)) * sc;
-            const float xh = __uint_as_float((i & 1) ? (wh & 0xffff0000u) : (wh << 16)) * sc;
-            const float m = (i & 1) ? 0.0625f : 1.f;
-            const __half lo = __float2half_rn(xl * m), hi = __float2half_rn(xh * m);
-            h[i] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
-          }
+      for (int i = 0; i < 4; ++i) {
+        if (kNv) {  // natural order: pair i = elements 2i, 2i+1
+          const __half lo = __float2half_rn(__uint_as_float(wv[i] << 16) * sc);
+          const __half hi = __float2half_rn(__uint_as_float(wv[i] & 0xffff0000u) * sc);
+          h[i] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+        } else {    // symmetric, affine: pair i = elements i, i + 4; odd i carry 2^-4
+          const uint32_t wl = wv[i >> 1], wh = wv[(i >> 1) + 2];
+          const float xl = __uint_as_float((i & 1) ? (wl & 0xffff0000u) : (wl << 16)) * sc;
+          const float xh = __uint_as_float((i & 1) ? (wh & 0xffff0000u) : (wh << 16)) * sc;
+          const float m = (i & 1) ? 0.0625f : 1.f;
+          const __half lo = __float2half_rn(xl * m), hi = __float2half_rn(xh * m);
+          h[i] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
         }
-        if (kSym) {
+      }
+      if (!kNv) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const uint32_t we = wv[e >> 1];
-            part += __half2float(__float2half_rn(
-                __uint_as_float((e & 1) ? (we & 0xffff0000u) : (we << 16)) * sc));
-          }
-          // the 16 tasks of one (group, row) are consecutive and share a
-          // half-warp: a fixed tree over them
-          const unsigned hmask = 0xFFFFu << (lane & 16);
-#pragma unroll
-          for (int o = 1; o < 16; o <<= 1) part += __shfl_xor_sync(hmask, part, o);
-          if ((task & 15) == 0) xsum[G * 8 + gg] = -8.f * part;
+        for (int e = 0; e < 8; ++e) {
+          const uint32_t we = wv[e >> 1];
+          part += __half2float(__float2half_rn(
+              __uint_as_float((e & 1) ? (we & 0xffff0000u) : (we << 16)) * sc));
         }
-        frag[task] = make_uint4(h[0], h[1], h[2], h[3]);
-      } else {
-        frag[task] = bf16x8_to_pairs(v);
+        // the 16 tasks of one (group, row) are consecutive and share a
+        // half-warp, lane (tt, q4) at 4 tt + q4: a fixed tree over them;
+        // affine keeps the 64-groups q4 / 2 = 0, 1 apart (no xor 2)
+        const unsigned hmask = 0xFFFFu << (lane & 16);
+        part += __shfl_xor_sync(hmask, part, 1);
+        if (kSym) part += __shfl_xor_sync(hmask, part, 2);
+        part += __shfl_xor_sync(hmask, part, 4);
+        part += __shfl_xor_sync(hmask, part, 8);
+        if (kSym && (task & 15) == 0) xsum[G * 8 + gg] = -8.f * part;
+        if (kAffine && (task & 13) == 0) xsum[(2 * G + (q4 >> 1)) * B + gg] = part;
       }
-    }
-    if (kAffine) {  // sum of x over 64-group j of row b, elements in ascending order
-      for (int task = tid; task < ng64 * B; task += ncons * 32) {
-        const int j = task / B, b = task % B;
-        const uint16_t *xr = x + (size_t)b * K + 64 * j;
-        float sx = 0.f;
-        for (int k = 0; k < 64; ++k)
-          sx += bf16_bits_to_f32((uint32_t)__ldcg(reinterpret_cast<const unsigned short *>(xr + k)));
-        xsum[task] = sx;
-      }
+      frag[task] = make_uint4(h[0], h[1], h[2], h[3]);
     }
     asm volatile("bar.sync 1, %0;" ::"r"(ncons * 32) : "memory");  // consumers only
     const int my_tiles = full_tiles > (int)blockIdx.x
@@ -675,7 +636,7 @@ __global__ void __launch_bounds__((kGW ? kRegWarps : kGemvWarps) * 32, 1)
           const float4 o = s_red[grp][i & 1][j][lane];
           acc[0] += o.x, acc[1] += o.y, acc[2] += o.z, acc[3] += o.w;
         }
-        if (kF16x) col_scale(acc, t, B, s_ymul);
+        col_scale(acc, t, B, s_ymul);
         if (lane == 0) mbar_arrive(&empty[st]);
         rows_store(acc, tile * 16 + ra_t, tile * 16 + rb_t, N, B, y, t, best_v, best_i);
       }
@@ -689,6 +650,7 @@ __global__ void __launch_bounds__((kGW ? kRegWarps : kGemvWarps) * 32, 1)
         rows_dot_affine<true>(q + ra * rbytes, q + rb * rbytes, s + ra * ng64, s + rb * ng64,
                               moff + ra * ng64, moff + rb * ng64, 0, ng, B, frag, xsum, lane,
                               acc);
+        col_scale(acc, t, B, s_ymul);
       } else if (kNv) {
         const uint8_t *s8 = reinterpret_cast<const uint8_t *>(s);
         rows_dot_nvfp4<true>(q + ra * rbytes, q + rb * rbytes, s8 + ra * (K / 16),
