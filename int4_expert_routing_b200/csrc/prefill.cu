@@ -257,7 +257,8 @@ __global__ void __launch_bounds__(256)
     k_pf_wstats(const uint16_t *__restrict__ w13_s, const uint16_t *__restrict__ w2_s,
                 const uint16_t *__restrict__ sh13_s, const uint16_t *__restrict__ sh2_s,
                 float up_mul, float4 *__restrict__ wst, float *__restrict__ wbound) {
-  pdl_wait();  // the previous kernel in the stream is complete (programmatic launch)
+  // the scales are weights, not the previous kernel's output: they are read
+  // before the programmatic-launch wait, which only guards the writes
   pdl_trigger();
   __shared__ float red[4][8];
   const int e = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -267,30 +268,63 @@ __global__ void __launch_bounds__(256)
   const int g2 = (sh ? kIs : kI) / kG;
   const uint16_t *s2 = sh ? sh2_s : w2_s + (size_t)e * kH * g2;
   float mx1 = 0.f, mx2 = 0.f, bg = 0.f, bu = 0.f;
-  for (int r = tid; r < r13; r += 256) {
-    const uint4 *p = reinterpret_cast<const uint4 *>(s13 + (size_t)r * (kH / kG));
-    const float um = (!sh && r >= r13 / 2) ? up_mul : 1.f;
-    float ss = 0.f;
+  // gate/up: a row's 16 scales are two 16-byte words; every row of the thread
+  // loaded before any is used (at most 8 rows: 2,048 rows over 256 threads)
+  {
+    constexpr int kMaxRows = 2 * kIs / 256;
+    uint4 rv[kMaxRows][2];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint4 v = __ldg(p + h);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float a = fabsf(__uint_as_float(w[q] << 16)) * um,
-                    b = fabsf(__uint_as_float(w[q] & 0xffff0000u)) * um;
-        mx1 = fmaxf(mx1, fmaxf(a, b));
-        ss = fmaf(a, a, fmaf(b, b, ss));
+    for (int i = 0; i < kMaxRows; ++i) {
+      const int r = tid + 256 * i;
+      if (r < r13) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(s13 + (size_t)r * (kH / kG));
+        rv[i][0] = __ldg(p), rv[i][1] = __ldg(p + 1);
       }
     }
-    const float rb = 8.f * sqrtf(128.f * ss);
-    if (r < r13 / 2) bg = fmaxf(bg, rb);
-    else bu = fmaxf(bu, rb);
+#pragma unroll
+    for (int i = 0; i < kMaxRows; ++i) {
+      const int r = tid + 256 * i;
+      if (r >= r13) continue;
+      const float um = (!sh && r >= r13 / 2) ? up_mul : 1.f;
+      float ss = 0.f;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t w[4] = {rv[i][h].x, rv[i][h].y, rv[i][h].z, rv[i][h].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float a = fabsf(__uint_as_float(w[q] << 16)) * um,
+                      b = fabsf(__uint_as_float(w[q] & 0xffff0000u)) * um;
+          mx1 = fmaxf(mx1, fmaxf(a, b));
+          ss = fmaf(a, a, fmaf(b, b, ss));
+        }
+      }
+      const float rb = 8.f * sqrtf(128.f * ss);
+      if (r < r13 / 2) bg = fmaxf(bg, rb);
+      else bu = fmaxf(bu, rb);
+    }
   }
-  for (int i = tid; i < kH * g2 / 2; i += 256) {
-    const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(s2) + i);
-    mx2 = fmaxf(mx2, fmaxf(fabsf(__uint_as_float(w << 16)), fabsf(__uint_as_float(w & 0xffff0000u))));
+  // down: 16-byte words of scales, all of the thread's in flight at once
+  // (routed: 2,048 x 4 scales = 1,024 words; shared: 2,048 x 8 = 2,048)
+  {
+    constexpr int kMaxWords = kH * (kIs / kG) / 8 / 256;
+    const int nw = kH * g2 / 8;
+    uint4 dv[kMaxWords];
+#pragma unroll
+    for (int i = 0; i < kMaxWords; ++i) {
+      const int k = tid + 256 * i;
+      if (k < nw) dv[i] = __ldg(reinterpret_cast<const uint4 *>(s2) + k);
+    }
+#pragma unroll
+    for (int i = 0; i < kMaxWords; ++i) {
+      if (tid + 256 * i >= nw) continue;
+      const uint32_t w[4] = {dv[i].x, dv[i].y, dv[i].z, dv[i].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        mx2 = fmaxf(mx2, fmaxf(fabsf(__uint_as_float(w[q] << 16)),
+                               fabsf(__uint_as_float(w[q] & 0xffff0000u))));
+    }
   }
+  pdl_wait();  // the previous kernel in the stream is complete before any write
   float v[4] = {mx1, mx2, bg, bu};
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
@@ -1403,7 +1437,7 @@ cudaError_t launch_route_many(const LayerArgs &L, const uint16_t *x, int T, int3
     return e;
   note_step("prefill router launch");
   const int nsplit = route_split(T);
-  double *zh = nsplit == 2 ? reinterpret_cast<double *>(ws + P.z) : nullptr;
+  double *zh = nsplit > 1 ? reinterpret_cast<double *>(ws + P.z) : nullptr;
   {
     const int nitems = 2 * ((T + kRtM - 1) / kRtM) * nsplit;
     e = pf_launch(k_pf_router_tc, nitems < 148 ? nitems : 148, kRtThreads, kRtSmem, st, mX, mW, T,
