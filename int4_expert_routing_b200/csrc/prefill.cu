@@ -954,9 +954,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             uint32_t v[32];
 #pragma unroll
             for (int jj = 0; jj < 2; ++jj) {
-              // chunk j = codes 32 j .. 32 j + 31 of the group -> columns 16 j ..
+              // chunk j = codes 32 j .. 32 j + 31 of the group -> columns 16 j ..;
+              // the box is 64-byte swizzled: chunk j of box row r sits at
+              // chunk j ^ ((r >> 1) & 3) (address bits 7-8 of a 1024-aligned box)
               const int j = 2 * hf + jj;
-              const uint4 w = *reinterpret_cast<const uint4 *>(raw + 16 * j);
+              const uint4 w = *reinterpret_cast<const uint4 *>(raw + 16 * (j ^ ((raw_row >> 1) & 3)));
               codes8_f16(w.x, m24, m20, c8, v + 16 * jj + 0);
               codes8_f16(w.y, m24, m20, c8, v + 16 * jj + 4);
               codes8_f16(w.z, m24, m20, c8, v + 16 * jj + 8);
@@ -1506,12 +1508,15 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
   CUtensorMap mA1r, mA1s, mB1, mA2r, mA2s, mB2r, mB2s;
   note_step("prefill tensor maps");
   const auto F16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16, U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
-  const auto SW = CU_TENSOR_MAP_SWIZZLE_128B, NS = CU_TENSOR_MAP_SWIZZLE_NONE;
-  if ((e = make_map(&mA1r, L.w13_q, U8, kH / 2, (uint64_t)kE * 2 * kI, kH / 2, 64, 64, NS)) ||
-      (e = make_map(&mA1s, L.sh13_q, U8, kH / 2, 2 * kIs, kH / 2, 64, 64, NS)) ||
+  const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
+  // code boxes of 64-byte rows, 64-byte swizzled: the dequant warps' row reads
+  // (8 consecutive rows per 16-byte load phase) hit every bank once
+  const auto SW64 = CU_TENSOR_MAP_SWIZZLE_64B;
+  if ((e = make_map(&mA1r, L.w13_q, U8, kH / 2, (uint64_t)kE * 2 * kI, kH / 2, 64, 64, SW64)) ||
+      (e = make_map(&mA1s, L.sh13_q, U8, kH / 2, 2 * kIs, kH / 2, 64, 64, SW64)) ||
       (e = make_map(&mB1, xp, F16, kH, (uint64_t)7 * T, kH * 2, 64, GemmCfg<1>::kBRows, SW)) ||
-      (e = make_map(&mA2r, L.w2_q, U8, kI / 2, (uint64_t)kE * kH, kI / 2, 64, 128, NS)) ||
-      (e = make_map(&mA2s, L.sh2_q, U8, kIs / 2, kH, kIs / 2, 64, 128, NS)) ||
+      (e = make_map(&mA2r, L.w2_q, U8, kI / 2, (uint64_t)kE * kH, kI / 2, 64, 128, SW64)) ||
+      (e = make_map(&mA2s, L.sh2_q, U8, kIs / 2, kH, kIs / 2, 64, 128, SW64)) ||
       (e = make_map(&mB2r, hr, F16, kI, (uint64_t)P.mr, kI * 2, 64, GemmCfg<2>::kBRows, SW)) ||
       (e = make_map(&mB2s, hs, F16, kIs, (uint64_t)T, kIs * 2, 64, GemmCfg<2>::kBRows, SW)))
     return e;
