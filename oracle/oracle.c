@@ -134,6 +134,13 @@ static double weight_affine(const uint8_t *q, const uint16_t *s, const uint16_t 
          oracle_fp16_to_double(m[g]);
 }
 
+static double row_dot_affine(const uint8_t *q, const uint16_t *s, const uint16_t *m, int64_t K,
+                             int64_t n, const double *x) {
+  double acc = 0.0;
+  for (int64_t k = 0; k < K; ++k) acc += weight_affine(q, s, m, K, n, k) * x[k];
+  return acc;
+}
+
 void oracle_dequant_affine(const uint8_t *q, const uint16_t *s, const uint16_t *m, int64_t N,
                            int64_t K, double *W) {
   for (int64_t n = 0; n < N; ++n)
@@ -331,6 +338,7 @@ typedef struct {
   int n;
   const uint8_t *q[8];
   const uint16_t *s[8];
+  const uint16_t *m[8]; /* affine offsets, or NULL for the symmetric format */
   int64_t K[8], rows[8];
   const double *x[8];
   double *y[8];
@@ -340,12 +348,14 @@ static void matvec_set_row(void *p, int64_t i) {
   matvec_set *m = (matvec_set *)p;
   int j = 0;
   while (i >= m->rows[j]) i -= m->rows[j++];
-  m->y[j][i] = row_dot(m->q[j], m->s[j], m->K[j], i, m->x[j]);
+  m->y[j][i] = m->m[j] ? row_dot_affine(m->q[j], m->s[j], m->m[j], m->K[j], i, m->x[j])
+                       : row_dot(m->q[j], m->s[j], m->K[j], i, m->x[j]);
 }
 
-static void matvec_set_add(matvec_set *m, const uint8_t *q, const uint16_t *s, int64_t rows,
-                           int64_t K, const double *x, double *y) {
-  m->q[m->n] = q, m->s[m->n] = s, m->rows[m->n] = rows, m->K[m->n] = K;
+static void matvec_set_add(matvec_set *m, const uint8_t *q, const uint16_t *s,
+                           const uint16_t *off, int64_t rows, int64_t K, const double *x,
+                           double *y) {
+  m->q[m->n] = q, m->s[m->n] = s, m->m[m->n] = off, m->rows[m->n] = rows, m->K[m->n] = K;
   m->x[m->n] = x, m->y[m->n] = y;
   ++m->n;
 }
@@ -366,11 +376,11 @@ void oracle_swiglu_expert(const uint8_t *q13, const uint16_t *s13, const uint8_t
   double *g = (double *)malloc(sizeof(double) * 2 * inter);
   double *hmid = (double *)malloc(sizeof(double) * inter);
   matvec_set m = {0};
-  matvec_set_add(&m, q13, s13, 2 * inter, hidden, x, g);
+  matvec_set_add(&m, q13, s13, NULL, 2 * inter, hidden, x, g);
   matvec_set_run(&m);
   swiglu_mid(g, inter, hmid);
   matvec_set m2 = {0};
-  matvec_set_add(&m2, q2, s2, hidden, inter, hmid, y);
+  matvec_set_add(&m2, q2, s2, NULL, hidden, inter, hmid, y);
   matvec_set_run(&m2);
   free(g);
   free(hmid);
@@ -408,14 +418,19 @@ static void moe_row(void *p, int64_t b) {
     const int inter = j < k ? I : Is;
     const size_t go = 2 * (size_t)I * j, ho = (size_t)I * j;
     if (j < k ? (e < c->e_lo || e >= c->e_hi) : !c->with_shared) continue; /* term not summed */
+    /* scales (and affine offsets) per 128 (symmetric) or 64 (affine) elements */
+    const int gs = L->format == 1 ? 64 : 128;
+    const int aff = L->format == 1;
     if (j < k) {
-      matvec_set_add(&m13, L->w13_q + e * (2 * I) * (H / 2), L->w13_s + e * (2 * I) * (H / 128),
-                     2 * inter, H, xd, g + go);
-      matvec_set_add(&m2, L->w2_q + e * H * (I / 2), L->w2_s + e * H * (I / 128), H, inter,
-                     hmid + ho, ys + (size_t)H * j);
+      const int64_t g13 = e * (2 * I) * (H / gs), g2 = e * H * (I / gs);
+      matvec_set_add(&m13, L->w13_q + e * (2 * I) * (H / 2), L->w13_s + g13,
+                     aff ? L->w13_m + g13 : NULL, 2 * inter, H, xd, g + go);
+      matvec_set_add(&m2, L->w2_q + e * H * (I / 2), L->w2_s + g2, aff ? L->w2_m + g2 : NULL, H,
+                     inter, hmid + ho, ys + (size_t)H * j);
     } else {
-      matvec_set_add(&m13, L->sh13_q, L->sh13_s, 2 * inter, H, xd, g + go);
-      matvec_set_add(&m2, L->sh2_q, L->sh2_s, H, inter, hmid + ho, ys + (size_t)H * j);
+      matvec_set_add(&m13, L->sh13_q, L->sh13_s, aff ? L->sh13_m : NULL, 2 * inter, H, xd, g + go);
+      matvec_set_add(&m2, L->sh2_q, L->sh2_s, aff ? L->sh2_m : NULL, H, inter, hmid + ho,
+                     ys + (size_t)H * j);
     }
   }
   matvec_set_run(&m13);

@@ -51,6 +51,14 @@ typedef struct {
    * section 21.2 "The packs": expert_interm_div, the routing weights
    * multiplied back in the combine); 0 or 1: not divided. */
   double expert_interm_div;
+  /* Format of the expert matrices (the router is bf16 in both): 0 the
+   * symmetric int4 above; 1 group-64 affine int4 ("How to Run Flint Locally",
+   * section "Every build and its size": the MLX int4 build, the Q4_1 GGUF):
+   * unsigned codes 0..15 in the same nibble order, the *_s arrays fp16 scales
+   * [rows][K/64] and the *_m arrays fp16 offsets [rows][K/64],
+   * weight = code * scale + offset. */
+  int format;
+  const uint16_t *w13_m, *w2_m, *sh13_m, *sh2_m;
 } oracle_layer;
 
 void oracle_set_threads(int n);

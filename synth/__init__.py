@@ -78,6 +78,14 @@ T_AFF_S = 31
 T_AFF_M = 32
 T_NV_Q = 33
 T_NV_S = 34
+T_AFL_W13_S = 40
+T_AFL_W13_M = 41
+T_AFL_W2_S = 42
+T_AFL_W2_M = 43
+T_AFL_SH13_S = 44
+T_AFL_SH13_M = 45
+T_AFL_SH2_S = 46
+T_AFL_SH2_M = 47
 
 N_OUTLIERS = 8
 OUTLIER_GAIN = 20.0
@@ -313,6 +321,51 @@ def layer_host(seed: int, dims: Dims = FLINT, with_codes: bool = True) -> dict:
     return d
 
 
+def _affine_groups(seed: int, tid_s: int, tid_m: int, rows: int, k: int):
+    """fp16 scale and offset bits [rows, k/64] of the affine recipe: scale
+    0.02 * U(0.5, 1.5) / 7.5, offset -7.5 * scale * U(0.9, 1.1)."""
+    g = rows * (k // 64)
+    sc = 0.02 * (0.5 + uniforms(seed, tid_s, g)) / 7.5
+    off = -7.5 * sc * (0.9 + 0.2 * uniforms(seed, tid_m, g))
+    return fp16_bits(sc).reshape(rows, k // 64), fp16_bits(off).reshape(rows, k // 64)
+
+
+def affine_layer_host(seed: int, dims: Dims = FLINT, with_codes: bool = True) -> dict:
+    """A MoE layer whose expert matrices are group-64 affine int4 (the MLX
+    int4 / Q4_1 layout): the router as in ``layer_host``; the same packed
+    bytes as the symmetric layer of this seed, each nibble read as an unsigned
+    code 0..15; per 64 elements along K an fp16 scale and an fp16 offset
+    (``_affine_groups``).  Scale and offset arrays are [rows, K/64] per
+    matrix (w13_s [E, 2I, H/64], w2_s [E, H, I/64], sh13_s [2Is, H/64],
+    sh2_s [H, Is/64]), the offsets under the *_m names."""
+    dims.check()
+    E, H, I, Is = dims.n_experts, dims.hidden, dims.expert_i, dims.shared_i
+    d = layer_host(seed, dims, with_codes=with_codes)
+    for name, tid_s, tid_m, rows, k, shape in (
+            ("w13", T_AFL_W13_S, T_AFL_W13_M, E * 2 * I, H, (E, 2 * I, H // 64)),
+            ("w2", T_AFL_W2_S, T_AFL_W2_M, E * H, I, (E, H, I // 64)),
+            ("sh13", T_AFL_SH13_S, T_AFL_SH13_M, 2 * Is, H, (2 * Is, H // 64)),
+            ("sh2", T_AFL_SH2_S, T_AFL_SH2_M, H, Is, (H, Is // 64))):
+        sc, off = _affine_groups(seed, tid_s, tid_m, rows, k)
+        d[name + "_s"], d[name + "_m"] = sc.reshape(shape), off.reshape(shape)
+    return d
+
+
+def affine_from_symmetric(t: dict) -> dict:
+    """The same weights in the affine format, exactly: code c -> c + 8 (each
+    nibble XOR 8), each bf16 scale -> two fp16 scales of the same value (one
+    per 64-half of its 128-group), offset -8 x scale.  Both conversions are
+    exact for the recipe's scales (normal fp16, 8 significant bits)."""
+    out = dict(t)
+    for name in ("w13", "w2", "sh13", "sh2"):
+        out[name + "_q"] = np.asarray(t[name + "_q"], np.uint8) ^ np.uint8(0x88)
+        b = np.asarray(t[name + "_s"], np.uint16).astype(np.uint32) << np.uint32(16)
+        sc = np.repeat(b.view(np.float32).astype(np.float64), 2, axis=-1)
+        out[name + "_s"] = fp16_bits(sc)
+        out[name + "_m"] = fp16_bits(-8.0 * sc)
+    return out
+
+
 def expert_codes_host(seed: int, expert: int, dims: Dims = FLINT):
     """(w13_q[e], w2_q[e]) of one expert, drawn on their own (counter-based)."""
     n13 = 2 * dims.expert_i * dims.hidden // 2
@@ -385,6 +438,13 @@ def to_device(arrays: dict, device) -> dict:
             a = a.view(np.int16)
         out[k] = torch.from_numpy(a).to(device)
     return out
+
+
+def affine_layer_device(seed: int, device, dims: Dims = FLINT) -> dict:
+    """``affine_layer_host`` on ``device``, the codes drawn on the device."""
+    d = to_device(affine_layer_host(seed, dims, with_codes=False), device)
+    d.update(layer_codes_torch(seed, device, dims))
+    return d
 
 
 def layer_device(seed: int, device, dims: Dims = FLINT, host: dict | None = None) -> dict:

@@ -465,6 +465,55 @@ def test_layer_matches_numpy_definition_random():
         np.testing.assert_allclose(out[row], expect, rtol=1e-10, atol=1e-13)
 
 
+def dequant_affine_np(q, s, m):
+    """Group-64 affine weights from their definition, in numpy: unsigned
+    nibbles (low nibble = even element) x fp16 scale + fp16 offset."""
+    q = np.asarray(q, np.uint8)
+    u = np.stack([q & 15, q >> 4], axis=-1).reshape(q.shape[0], -1).astype(np.float64)
+    sc = np.asarray(s, np.uint16).view(np.float16).astype(np.float64)
+    off = np.asarray(m, np.uint16).view(np.float16).astype(np.float64)
+    return u * np.repeat(sc, 64, axis=1) + np.repeat(off, 64, axis=1)
+
+
+def test_affine_layer_matches_numpy_definition_random():
+    """The block with group-64 affine experts ("How to Run Flint Locally",
+    section "Every build and its size"), against a numpy statement of the
+    same definition."""
+    dims = synth.Dims(hidden=256, n_experts=16, top_k=6, expert_i=128, shared_i=256)
+    t = synth.affine_layer_host(15, dims)
+    x = bf16(np.random.default_rng(9).normal(size=(2, 256)))
+    out, idx, w, gap = oracle.moe_layer(oracle.Layer(t), x)
+
+    def expert(q13, s13, m13, q2, s2, m2, xd):
+        W13 = dequant_affine_np(q13, s13, m13)
+        I = W13.shape[0] // 2
+        g, u = W13[:I] @ xd, W13[I:] @ xd
+        return dequant_affine_np(q2, s2, m2) @ (g / (1 + np.exp(-g)) * u)
+
+    for row in range(2):
+        xd = synth.bf16_to_f64(x[row])
+        s = 1 / (1 + np.exp(-(synth.bf16_to_f64(t["router_w"]) @ xd)))
+        sel = np.lexsort((np.arange(16), -(s + t["router_b"].astype(np.float64))))[:6]
+        assert list(sel) == list(idx[row])
+        expect = sum(s[e] / s[sel].sum() * expert(t["w13_q"][e], t["w13_s"][e], t["w13_m"][e],
+                                                  t["w2_q"][e], t["w2_s"][e], t["w2_m"][e], xd)
+                     for e in sel)
+        expect = expect + expert(t["sh13_q"], t["sh13_s"], t["sh13_m"], t["sh2_q"], t["sh2_s"],
+                                 t["sh2_m"], xd)
+        np.testing.assert_allclose(out[row], expect, rtol=1e-10, atol=1e-13)
+
+
+def test_affine_layer_equals_symmetric_layer_exactly():
+    """A symmetric layer rewritten in the affine format (codes + 8, each bf16
+    scale as two fp16 scales, offsets -8 x scale) has the same weights, so
+    the affine block output equals the symmetric one bit for bit."""
+    t, _ = tiny_layer(E=8, H=256, I=128, Is=256, seed=23)
+    x = bf16(np.random.default_rng(24).normal(size=(3, 256)))
+    ref, idx, *_ = oracle.moe_layer(oracle.Layer(t), x)
+    got, idx2, *_ = oracle.moe_layer(oracle.Layer(synth.affine_from_symmetric(t)), x)
+    assert np.array_equal(got, ref) and np.array_equal(idx, idx2)
+
+
 # ------------------------------------------------------------------ stack
 def test_interm_div_layer_equals_undivided_layer_exactly():
     """Routed up projections stored / 128 with the routing weights multiplied

@@ -24,6 +24,10 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
 # name -> [(text in oracle.c, replacement)]; every text occurs exactly once,
 # and every mutant keeps its indexes inside the arrays it reads
 MUTANTS = {
+    "affine layer read as symmetric": [("m->m[j] ? row_dot_affine(", "0 ? row_dot_affine(")],
+    "affine layer with 128-groups": [("const int gs = L->format == 1 ? 64 : 128;",
+                                      "const int gs = 128;")],
+    "affine down offsets from gate/up": [("aff ? L->w2_m + g2 : NULL", "aff ? L->w13_m + g2 : NULL")],
     "nibble as offset binary": [("return nib >= 8 ? nib - 16 : nib;", "return nib - 8;")],
     "nibble order swapped": [("int nib = (k % 2 == 0) ? (byte & 0x0F) : (byte >> 4);",
                               "int nib = (k % 2 == 0) ? (byte >> 4) : (byte & 0x0F);")],
