@@ -53,6 +53,11 @@ extern "C" {
 #define FLINT_SHARED_I 1024
 #define FLINT_GROUP 128
 #define FLINT_MAX_DECODE_B 8
+/* The decode calls on a layer in the group-64 affine format take B <= 7:
+ * each of the 128 down-projection CTAs holds up to 6B experts' rows with
+ * their fp16 scales and offsets, and 48 of them do not fit its shared
+ * memory.  (flint_moe_route takes B <= 8 in both formats.) */
+#define FLINT_MAX_DECODE_B_AFFINE 7
 #define FLINT_MAX_PREFILL_T (1 << 20)
 #define FLINT_MAX_STACK_LAYERS 256
 #define FLINT_RMS_EPS 1e-6
@@ -98,7 +103,27 @@ typedef struct {
    * otherwise 2^n with 1 <= n <= 16.  The block computes the same function
    * either way: outputs equal those of the undivided weights. */
   int expert_interm_div;
+  /* Weight format of the routed and shared experts (the router is bf16 in
+   * both).  FLINT_FMT_SYM_INT4 (0): the layout above.  FLINT_FMT_AFFINE_INT4
+   * (1): group-64 affine int4 ("How to Run Flint Locally", section "Every
+   * build and its size": the MLX int4 build, and the Q4_1 GGUF's codes with
+   * FP16 scales and offsets): the *_q arrays as above but each nibble an
+   * unsigned code 0..15; the *_s arrays fp16 scales and the *_m arrays fp16
+   * offsets, one per 64 elements along K: w13_s / w13_m [E][2I][H/64],
+   * w2_s / w2_m [E][H][I/64], sh13_s / sh13_m [2Is][H/64], sh2_s / sh2_m
+   * [H][Is/64]; weight = code * scale + offset.  The *_m pointers are read
+   * only for format 1 (16-byte aligned there).  Decode, route and the stack
+   * and expert-parallel calls take both formats; prefill takes format 0
+   * only (FLINT_EINVAL otherwise). */
+  int format;
+  const uint16_t *w13_m;
+  const uint16_t *w2_m;
+  const uint16_t *sh13_m;
+  const uint16_t *sh2_m;
 } flint_moe_layer;
+
+#define FLINT_FMT_SYM_INT4 0
+#define FLINT_FMT_AFFINE_INT4 1
 
 /* Library version (major*10000 + minor*100 + patch). */
 FLINT_API int flint_version(void);

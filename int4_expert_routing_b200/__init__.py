@@ -38,10 +38,17 @@ class FlintError(RuntimeError):
         super().__init__(f"{where}: {strerror(code)} ({code}){detail}")
 
 
+_WEIGHTS = ("router_w", "router_b", "w13_q", "w13_s", "w2_q", "w2_s",
+            "sh13_q", "sh13_s", "sh2_q", "sh2_s")
+_OFFSETS = ("w13_m", "w2_m", "sh13_m", "sh2_m")
+FLINT_FMT_SYM_INT4 = 0
+FLINT_FMT_AFFINE_INT4 = 1
+
+
 class flint_moe_layer(C.Structure):
-    _fields_ = [(n, C.c_void_p) for n in (
-        "router_w", "router_b", "w13_q", "w13_s", "w2_q", "w2_s",
-        "sh13_q", "sh13_s", "sh2_q", "sh2_s")] + [("expert_interm_div", C.c_int)]
+    _fields_ = [(n, C.c_void_p) for n in _WEIGHTS] + [
+        ("expert_interm_div", C.c_int), ("format", C.c_int)] + [
+        (n, C.c_void_p) for n in _OFFSETS]
 
 
 def build(force: bool = False) -> str:
@@ -120,11 +127,14 @@ def _check(code: int, where: str):
 
 def make_layer(t: dict, expert_interm_div: int = 0) -> flint_moe_layer:
     """The C layer struct from a dict of device tensors (keys as in flint.h)
-    and the divisor of the routed up projections (0: not divided).  The
-    struct keeps a reference to the tensors, so their memory stays allocated
-    while the struct is alive."""
-    layer = flint_moe_layer(*[_ptr(t[n]) for n, _ in flint_moe_layer._fields_[:-1]],
-                            int(expert_interm_div))
+    and the divisor of the routed up projections (0: not divided).  With the
+    *_m offset tensors the experts are group-64 affine int4
+    (FLINT_FMT_AFFINE_INT4).  The struct keeps a reference to the tensors, so
+    their memory stays allocated while the struct is alive."""
+    affine = "w13_m" in t
+    layer = flint_moe_layer(*[_ptr(t[n]) for n in _WEIGHTS], int(expert_interm_div),
+                            FLINT_FMT_AFFINE_INT4 if affine else FLINT_FMT_SYM_INT4,
+                            *[_ptr(t[n]) if affine else None for n in _OFFSETS])
     layer._tensors = t
     return layer
 

@@ -17,10 +17,22 @@ bool aligned16(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 15
 bool div_ok(int d) { return d == 0 || (d > 0 && d <= 65536 && (d & (d - 1)) == 0); }
 
 bool layer_ok(const flint_moe_layer *l) {
-  return l && div_ok(l->expert_interm_div) && aligned16(l->router_w) && aligned16(l->router_b) &&
+  if (!l || (l->format != FLINT_FMT_SYM_INT4 && l->format != FLINT_FMT_AFFINE_INT4)) return false;
+  if (l->format == FLINT_FMT_AFFINE_INT4 &&
+      !(aligned16(l->w13_m) && aligned16(l->w2_m) && aligned16(l->sh13_m) && aligned16(l->sh2_m)))
+    return false;
+  return div_ok(l->expert_interm_div) && aligned16(l->router_w) && aligned16(l->router_b) &&
          aligned16(l->w13_q) &&
          aligned16(l->w13_s) && aligned16(l->w2_q) && aligned16(l->w2_s) && aligned16(l->sh13_q) &&
          aligned16(l->sh13_s) && aligned16(l->sh2_q) && aligned16(l->sh2_s);
+}
+
+// the decode calls' batch limit for a layer: K3 stages up to 6B experts'
+// down rows of its 16 output rows; the affine format's fp16 scales and
+// offsets (4.5 KB a slot instead of 4.1 KB) fit 42 slots, not 48
+bool decode_batch_ok(const flint_moe_layer *l, int B) {
+  return B >= 1 && B <= (l->format == FLINT_FMT_AFFINE_INT4 ? FLINT_MAX_DECODE_B_AFFINE
+                                                            : FLINT_MAX_DECODE_B);
 }
 
 thread_local cudaError_t g_last_cuda = cudaSuccess;
@@ -135,7 +147,7 @@ int flint_moe_route(const flint_moe_layer *layer, const uint16_t *x, int B, int3
 
 int flint_moe_decode(const flint_moe_layer *layer, const uint16_t *x, int B, uint16_t *out,
                      void *ws, size_t ws_bytes, void *stream) {
-  if (!layer_ok(layer) || !aligned16(x) || !aligned16(out) || B < 1 || B > FLINT_MAX_DECODE_B ||
+  if (!layer_ok(layer) || !aligned16(x) || !aligned16(out) || !decode_batch_ok(layer, B) ||
       !aligned16(ws) || ws_bytes < flint_workspace_bytes(FLINT_OP_DECODE, B) ||
       static_cast<const void *>(x) == static_cast<const void *>(out))
     return FLINT_EINVAL;
@@ -146,7 +158,7 @@ int flint_moe_decode(const flint_moe_layer *layer, const uint16_t *x, int B, uin
 
 int flint_moe_decode_residual(const flint_moe_layer *layer, float *h, int B, int32_t *idx,
                               float *w, void *ws, size_t ws_bytes, void *stream) {
-  if (!layer_ok(layer) || !aligned16(h) || B < 1 || B > FLINT_MAX_DECODE_B || !aligned16(ws) ||
+  if (!layer_ok(layer) || !aligned16(h) || !decode_batch_ok(layer, B) || !aligned16(ws) ||
       ws_bytes < flint_workspace_bytes(FLINT_OP_DECODE, B))
     return FLINT_EINVAL;
   return from_cuda(launch_decode(layer_args(layer), nullptr, h, h, B, nullptr, idx, w,
@@ -158,7 +170,7 @@ int flint_moe_decode_partial(const flint_moe_layer *layer, const uint16_t *x, co
                              int expert_lo, int expert_hi, int with_shared, float *partial, void *ws,
                              size_t ws_bytes, void *stream) {
   if (!layer_ok(layer) || (x == nullptr) == (h == nullptr) || (x && !aligned16(x)) ||
-      (h && !aligned16(h)) || !aligned16(partial) || B < 1 || B > FLINT_MAX_DECODE_B ||
+      (h && !aligned16(h)) || !aligned16(partial) || !decode_batch_ok(layer, B) ||
       expert_lo < 0 || expert_hi > FLINT_EXPERTS || expert_lo >= expert_hi || !aligned16(ws) ||
       ws_bytes < flint_workspace_bytes(FLINT_OP_DECODE, B))
     return FLINT_EINVAL;
@@ -184,7 +196,7 @@ int flint_moe_decode_stack(const flint_moe_layer *layers, int L, float *h, int B
       (h_trace && !aligned16(h_trace)))
     return FLINT_EINVAL;
   for (int l = 0; l < L; ++l)
-    if (!layer_ok(&layers[l])) return FLINT_EINVAL;
+    if (!layer_ok(&layers[l]) || !decode_batch_ok(&layers[l], B)) return FLINT_EINVAL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   for (int l = 0; l < L; ++l) {
     cudaError_t e = cudaSuccess;
@@ -239,8 +251,9 @@ int flint_int4_gemv_nvfp4(const uint8_t *q, const uint8_t *s, float global_scale
 
 int flint_moe_prefill(const flint_moe_layer *layer, const uint16_t *x, int T, uint16_t *out,
                       void *ws, size_t ws_bytes, void *stream) {
-  if (!layer_ok(layer) || !aligned16(x) || !aligned16(out) || T < 1 || T > FLINT_MAX_PREFILL_T ||
-      !aligned16(ws) || ws_bytes < flint_workspace_bytes(FLINT_OP_PREFILL, T) ||
+  if (!layer_ok(layer) || layer->format != FLINT_FMT_SYM_INT4 || !aligned16(x) ||
+      !aligned16(out) || T < 1 || T > FLINT_MAX_PREFILL_T || !aligned16(ws) ||
+      ws_bytes < flint_workspace_bytes(FLINT_OP_PREFILL, T) ||
       static_cast<const void *>(x) == static_cast<const void *>(out))
     return FLINT_EINVAL;
   return from_cuda(launch_prefill(layer_args(layer), x, T, out, static_cast<char *>(ws),

@@ -125,6 +125,22 @@ FLINT_DEV void int4x32_to_bf16x2(const uint4 w, uint32_t (&r)[16]) {
   }
 }
 
+// The same for unsigned codes 0..15 (the affine format): (w & 0x000F000F) |
+// 0x43004300 is the bf16 pair 128 + code, less 128 exact.
+FLINT_DEV void uint4x32_to_bf16x2(const uint4 w, uint32_t (&r)[16]) {
+  const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const uint32_t t = and_or(words[q] >> (4 * p), 0x000F000Fu, 0x43004300u);
+      uint32_t c;
+      asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(c) : "r"(t), "r"(0x43004300u));
+      r[4 * q + p] = c;
+    }
+  }
+}
+
 // 8 consecutive bf16 (one 16-byte load, 4 words) -> pairs {v[p], v[p+4]}.
 FLINT_DEV uint4 bf16x8_to_pairs(const uint4 v) {
   uint4 o;

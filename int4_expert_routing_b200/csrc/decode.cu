@@ -442,32 +442,59 @@ __global__ void __launch_bounds__(kK1Threads)
 constexpr int kK2Warps = FLINT_K2_WARPS;
 constexpr int kK2Groups = 16 / kK2Warps;  // k-groups per warp
 static_assert(kK2Warps * kK2Groups == 16, "the warps split the 16 k-groups evenly");
-constexpr int kItemBytes = 16384 + 512;
+constexpr int kItemBytes = 16384 + 512;      // codes, bf16 scales per 128
+constexpr int kItemBytesAff = 16384 + 2048;  // codes, fp16 scales and offsets per 64
 constexpr int kSharedItems = kIs / 8;
+template <bool kAff>
+constexpr int item_bytes() {
+  return kAff ? kItemBytesAff : kItemBytes;
+}
 
 struct ItemSrc {
   const uint8_t *gate;
   const uint8_t *up;
   const uint16_t *gate_s;
   const uint16_t *up_s;
+  const uint16_t *gate_m;  // affine offsets
+  const uint16_t *up_m;
 };
 
+// scale (and offset) groups per gate/up row: 16 of 128 or 32 of 64
+template <bool kAff>
+constexpr int item_groups() {
+  return kAff ? kH / 64 : kH / kG;
+}
+template <bool kAff>
 FLINT_DEV ItemSrc shared_item(const LayerArgs &L, int it) {
   const int r = 8 * it;
+  constexpr int gpr = item_groups<kAff>();
   return ItemSrc{L.sh13_q + (size_t)r * (kH / 2), L.sh13_q + (size_t)(kIs + r) * (kH / 2),
-                 L.sh13_s + (size_t)r * (kH / kG), L.sh13_s + (size_t)(kIs + r) * (kH / kG)};
+                 L.sh13_s + (size_t)r * gpr, L.sh13_s + (size_t)(kIs + r) * gpr,
+                 kAff ? L.sh13_m + (size_t)r * gpr : nullptr,
+                 kAff ? L.sh13_m + (size_t)(kIs + r) * gpr : nullptr};
 }
+template <bool kAff>
 FLINT_DEV ItemSrc routed_item(const LayerArgs &L, int e, int r0) {
   const size_t row = (size_t)e * (2 * kI) + r0;
+  constexpr int gpr = item_groups<kAff>();
   return ItemSrc{L.w13_q + row * (kH / 2), L.w13_q + (row + kI) * (kH / 2),
-                 L.w13_s + row * (kH / kG), L.w13_s + (row + kI) * (kH / kG)};
+                 L.w13_s + row * gpr, L.w13_s + (row + kI) * gpr,
+                 kAff ? L.w13_m + row * gpr : nullptr, kAff ? L.w13_m + (row + kI) * gpr : nullptr};
 }
-// one thread; the caller accounts the bytes on the barrier (mbar_add_tx)
+// one thread; the caller accounts the bytes on the barrier (mbar_add_tx).
+// Item layout: gate codes, up codes (8 rows x 1 KB each), then the gate and
+// up rows' scales (8 rows x groups) and, affine, their offsets.
+template <bool kAff>
 FLINT_DEV void issue_item(const ItemSrc &src, unsigned char *buf, uint64_t *bar) {
+  constexpr uint32_t sb = 8 * item_groups<kAff>() * 2;  // 256 or 512 bytes
   bulk_g2s(buf, src.gate, 8192, bar);
   bulk_g2s(buf + 8192, src.up, 8192, bar);
-  bulk_g2s(buf + 16384, src.gate_s, 256, bar);
-  bulk_g2s(buf + 16640, src.up_s, 256, bar);
+  bulk_g2s(buf + 16384, src.gate_s, sb, bar);
+  bulk_g2s(buf + 16384 + sb, src.up_s, sb, bar);
+  if (kAff) {
+    bulk_g2s(buf + 16384 + 2 * sb, src.gate_m, sb, bar);
+    bulk_g2s(buf + 16384 + 3 * sb, src.up_m, sb, bar);
+  }
 }
 
 // This warp's k-groups of the item: acc[0..1] gate, [2..3] up partials for
@@ -497,6 +524,47 @@ FLINT_DEV void item_part(const unsigned char *buf, const uint4 *frag, int B, int
   }
 }
 
+// The affine item: lane t's 32 elements of a 128-group lie in its 64-group
+// 2G (t < 2) or 2G + 1 (t >= 2).  Two MMAs per group on the same codes, each
+// with the other half's activation lanes zeroed, give the two 64-groups'
+// exact sums dA, dB; then y += s_A dA + m_A sum(x over 2G) + s_B dB + m_B
+// sum(x over 2G+1) per row (xs: [32 groups][kMaxB] sums of the block input).
+FLINT_DEV void item_part_aff(const unsigned char *buf, const uint4 *frag, const float *xs, int B,
+                             int warp, int lane, float (&acc)[4]) {
+  const int g = lane >> 2, t = lane & 3;
+  acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+  const uint16_t *sg = reinterpret_cast<const uint16_t *>(buf + 16384 + g * 64);
+  const uint16_t *su = reinterpret_cast<const uint16_t *>(buf + 16384 + 512 + g * 64);
+  const uint16_t *mg = reinterpret_cast<const uint16_t *>(buf + 16384 + 1024 + g * 64);
+  const uint16_t *mu = reinterpret_cast<const uint16_t *>(buf + 16384 + 1536 + g * 64);
+  const uint32_t mA = t < 2 ? 0xffffffffu : 0u, mB = ~mA;
+  const int c0 = 2 * t, c1 = 2 * t + 1;
+  auto h2f = [](uint16_t v) { return __half2float(__ushort_as_half(v)); };
+#pragma unroll
+  for (int k = 0; k < kK2Groups; ++k) {
+    const int G = kK2Groups * warp + k, gA = 2 * G, gB = 2 * G + 1;
+    const uint4 wg = *reinterpret_cast<const uint4 *>(buf + g * 1024 + 64 * G + 16 * t);
+    const uint4 wu = *reinterpret_cast<const uint4 *>(buf + 8192 + g * 1024 + 64 * G + 16 * t);
+    uint32_t ra[16], rb[16], xb[16], xa[16], xo[16];
+    uint4x32_to_bf16x2(wg, ra);
+    uint4x32_to_bf16x2(wu, rb);
+    load_frag_compact(frag, G, B, lane, xb);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) xa[i] = xb[i] & mA, xo[i] = xb[i] & mB;
+    float dA[4], dB[4];
+    group_mma(ra, rb, xa, dA);
+    group_mma(ra, rb, xo, dB);
+    const float xa0 = c0 < B ? xs[gA * kMaxB + c0] : 0.f, xa1 = c1 < B ? xs[gA * kMaxB + c1] : 0.f;
+    const float xb0 = c0 < B ? xs[gB * kMaxB + c0] : 0.f, xb1 = c1 < B ? xs[gB * kMaxB + c1] : 0.f;
+    const float sgA = h2f(sg[gA]), sgB = h2f(sg[gB]), suA = h2f(su[gA]), suB = h2f(su[gB]);
+    const float mgA = h2f(mg[gA]), mgB = h2f(mg[gB]), muA = h2f(mu[gA]), muB = h2f(mu[gB]);
+    acc[0] += fmaf(sgA, dA[0], mgA * xa0) + fmaf(sgB, dB[0], mgB * xb0);
+    acc[1] += fmaf(sgA, dA[1], mgA * xa1) + fmaf(sgB, dB[1], mgB * xb1);
+    acc[2] += fmaf(suA, dA[2], muA * xa0) + fmaf(suB, dB[2], muB * xb0);
+    acc[3] += fmaf(suA, dA[3], muA * xa1) + fmaf(suB, dB[3], muB * xb1);
+  }
+}
+
 constexpr int kK2Stages = 2;     // items in flight per CTA
 constexpr int kK2MaxItems = 16;  // items per CTA (the host sizes the grid to keep within it)
 
@@ -504,11 +572,13 @@ constexpr int kK2MaxItems = 16;  // items per CTA (the host sizes the grid to ke
 // shared expert is left to another call), then 64 items per routed slot.
 // CTA c takes items c, c + grid, c + 2 grid, ...; a CTA's first item is
 // fetched before the wait when it is a shared one.
+template <bool kAff>
 __global__ void __launch_bounds__(kK2Warps * 32)
     k2_gateup(LayerArgs L, int B, int n_items, int sh_items, char *__restrict__ ws,
               DecodeLayout lay) {
   extern __shared__ __align__(128) unsigned char sm[];  // stages | x fragment (compact)
-  uint4 *frag = reinterpret_cast<uint4 *>(sm + kK2Stages * kItemBytes);
+  constexpr int kIB = item_bytes<kAff>();
+  uint4 *frag = reinterpret_cast<uint4 *>(sm + kK2Stages * kIB);
   __shared__ __align__(8) uint64_t bar[kK2Stages];
   __shared__ __align__(8) uint64_t fbar;
   __shared__ float s_acc[kK2Warps][32][4];
@@ -516,6 +586,7 @@ __global__ void __launch_bounds__(kK2Warps * 32)
   __shared__ int s_n;
   __shared__ int s_aslot[kMaxB * kTopK];
   __shared__ float s_aw[kMaxB * kTopK];
+  __shared__ float s_xs[kAff ? 32 : 1][kMaxB];  // affine: block input summed per 64-group
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const int c0 = blockIdx.x, step = gridDim.x;
   uint32_t *ctrl = reinterpret_cast<uint32_t *>(ws + lay.ctrl);
@@ -528,8 +599,8 @@ __global__ void __launch_bounds__(kK2Warps * 32)
     for (int i = 0; i < kK2Stages; ++i) mbar_init(&bar[i], 1);
     mbar_init(&fbar, 1);
     if (c0 < sh_items) {
-      mbar_add_tx(&bar[0], kItemBytes);
-      issue_item(shared_item(L, c0), sm, &bar[0]);
+      mbar_add_tx(&bar[0], kIB);
+      issue_item<kAff>(shared_item<kAff>(L, c0), sm, &bar[0]);
     }
   }
   pdl_wait();  // K1 is complete: routing and the block input fragment are final
@@ -563,11 +634,11 @@ __global__ void __launch_bounds__(kK2Warps * 32)
         if (j == 0 && it < sh_items) {
           mbar_arrive(&bar[0]);  // fetched before the wait
         } else {
-          mbar_add_tx(&bar[j], kItemBytes);
-          issue_item(it < sh_items ? shared_item(L, it)
-                                       : routed_item(L, (int)slot_expert(s_word[j]),
+          mbar_add_tx(&bar[j], kIB);
+          issue_item<kAff>(it < sh_items ? shared_item<kAff>(L, it)
+                                       : routed_item<kAff>(L, (int)slot_expert(s_word[j]),
                                                      8 * ((it - sh_items) & 63)),
-                     sm + j * kItemBytes, &bar[j]);
+                     sm + j * kIB, &bar[j]);
           mbar_arrive(&bar[j]);
         }
       }
@@ -577,6 +648,25 @@ __global__ void __launch_bounds__(kK2Warps * 32)
   const int n = s_n;
   const bool fok = dwait(&fbar, 0);
   bool ok = fok;
+  if (kAff && fok) {
+    // sum of the block input over 64-group gg of row b, from the fragment:
+    // lanes tt = 2 (gg % 2), +1 of 128-group gg / 2 hold its 64 elements;
+    // read by the items after the barrier that opens each of them
+    for (int task = tid; task < 32 * B; task += kK2Warps * 32) {
+      const int gg = task / B, b = task % B, G = gg >> 1;
+      float sx = 0.f;
+      for (int tt = 2 * (gg & 1); tt < 2 * (gg & 1) + 2; ++tt)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 v = frag[(size_t)(G * 4 * B + b * 4 + tt) * 4 + q];
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            sx += __uint_as_float(w[i] << 16) + __uint_as_float(w[i] & 0xffff0000u);
+        }
+      s_xs[gg][b] = sx;
+    }
+  }
   if (n == 0) {
     if (!fok) {
       if (tid == 0) set_status(ctrl + 1, kStatusTimeout);
@@ -588,7 +678,7 @@ __global__ void __launch_bounds__(kK2Warps * 32)
     const int st = j % kK2Stages;
     const int it = c0 + j * step;
     const uint32_t word = s_word[j];
-    unsigned char *buf = sm + st * kItemBytes;
+    unsigned char *buf = sm + st * kIB;
     ok = dwait(&bar[st], (uint32_t)((j / kK2Stages) & 1)) && ok;
     trace_point(2, 2);
     if (__syncthreads_or(!ok)) {
@@ -600,7 +690,10 @@ __global__ void __launch_bounds__(kK2Warps * 32)
       return;
     }
     float acc[4];
-    item_part(buf, frag, B, warp, lane, acc);
+    if (kAff)
+      item_part_aff(buf, frag, &s_xs[0][0], B, warp, lane, acc);
+    else
+      item_part(buf, frag, B, warp, lane, acc);
     trace_point(2, 4);
 #pragma unroll
     for (int i = 0; i < 4; ++i) s_acc[warp][lane][i] = acc[i];
@@ -608,9 +701,9 @@ __global__ void __launch_bounds__(kK2Warps * 32)
     trace_point(2, 5);
     if (tid == 0 && j + kK2Stages < n) {
       const int jn = j + kK2Stages, itn = c0 + jn * step;
-      mbar_add_tx(&bar[st], kItemBytes);
-      issue_item(itn < sh_items ? shared_item(L, itn)
-                                    : routed_item(L, (int)slot_expert(s_word[jn]),
+      mbar_add_tx(&bar[st], kIB);
+      issue_item<kAff>(itn < sh_items ? shared_item<kAff>(L, itn)
+                                    : routed_item<kAff>(L, (int)slot_expert(s_word[jn]),
                                                   8 * ((itn - sh_items) & 63)),
                  buf, &bar[st]);
       mbar_arrive(&bar[st]);
@@ -661,16 +754,21 @@ __global__ void __launch_bounds__(kK2Warps * 32)
 
 // ============================================================== K3: down + combine
 // Shared-memory plan (bytes): weights [umax][16 rows][256] | scales
-// [umax][16][4] bf16 | shared down [16][512] | shared scales [16][8] |
-// intermediates (kStage) routed [B][6][2][512] bf16, shared [B][2][1024] |
-// per-row partial results [8 rows][16 parts][16 columns] fp32.
+// [umax][16][4] bf16 (affine: [umax] of fp16 scales [16][8] then offsets
+// [16][8]) | shared down [16][512] | shared scales [16][8] (affine: fp16
+// scales [16][16] then offsets [16][16]) | intermediates (kStage) routed
+// [B][6][2][512] bf16, shared [B][2][1024] | per-row partial results
+// [8 rows][16 parts][16 columns] fp32.
 struct K3Smem {
   int umax, B;
+  bool aff;
+  __host__ __device__ int slot_sb() const { return aff ? 512 : 128; }
+  __host__ __device__ int sh_sb() const { return aff ? 1024 : 256; }
   __host__ __device__ size_t w() const { return 0; }
   __host__ __device__ size_t s() const { return (size_t)umax * 4096; }
-  __host__ __device__ size_t shw() const { return s() + (size_t)umax * 128; }
+  __host__ __device__ size_t shw() const { return s() + (size_t)umax * slot_sb(); }
   __host__ __device__ size_t shs() const { return shw() + 8192; }
-  __host__ __device__ size_t hr() const { return shs() + 256; }
+  __host__ __device__ size_t hr() const { return shs() + sh_sb(); }
   __host__ __device__ size_t hs() const { return hr() + (size_t)B * kTopK * 2 * kI * 2; }
   __host__ __device__ size_t ysel(bool stage) const {
     return stage ? hs() + (size_t)B * 2 * kIs * 2 : hr();
@@ -678,13 +776,13 @@ struct K3Smem {
   __host__ __device__ size_t total(bool stage) const { return ysel(stage) + 8 * 16 * 16 * 4; }
 };
 
-template <bool kResidual, bool kStage>
+template <bool kResidual, bool kStage, bool kAff>
 __global__ void __launch_bounds__(kK3Threads)
     k3_down_combine(LayerArgs L, int B, uint16_t *__restrict__ out, float *__restrict__ h,
                     float *__restrict__ pout, int with_shared, char *__restrict__ ws,
                     DecodeLayout lay, int umax) {
   extern __shared__ __align__(128) unsigned char sm[];
-  const K3Smem P{umax, B};
+  const K3Smem P{umax, B, kAff};
   unsigned char *wsm = sm + P.w();
   unsigned char *ssm = sm + P.s();
   unsigned char *shm = sm + P.shw();
@@ -699,6 +797,10 @@ __global__ void __launch_bounds__(kK3Threads)
   // slot u's i-th row (ascending) b and the slot's place j among that row's
   // experts (ascending), as b | j << 4
   __shared__ uint8_t s_rbj[kMaxB * kTopK][kMaxB];
+  // affine: each intermediate image pair (hi + lo) summed over its 64-groups:
+  // row b's j-th routed expert at b * 6 + j (8 groups), its shared one at
+  // 48 + b (16 groups)
+  __shared__ float s_hs[kAff ? kMaxB * kTopK + kMaxB : 1][16];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const int n0 = blockIdx.x * 16;
@@ -722,15 +824,29 @@ __global__ void __launch_bounds__(kK3Threads)
     if (word != kSlotInvalid && tid < umax) {
       const size_t e = slot_expert(word);
       s_rows[tid] = slot_mask(word) & ((1u << B) - 1u);
-      mbar_add_tx(&bar, 4096 + 128);
-      bulk_g2s(wsm + tid * 4096, L.w2_q + (e * kH + n0) * (kI / 2), 4096, &bar);
-      bulk_g2s(ssm + tid * 128, L.w2_s + (e * kH + n0) * (kI / kG), 128, &bar);
+      if (kAff) {  // fp16 scales then offsets, 8 per row
+        mbar_add_tx(&bar, 4096 + 512);
+        bulk_g2s(wsm + tid * 4096, L.w2_q + (e * kH + n0) * (kI / 2), 4096, &bar);
+        bulk_g2s(ssm + tid * 512, L.w2_s + (e * kH + n0) * (kI / 64), 256, &bar);
+        bulk_g2s(ssm + tid * 512 + 256, L.w2_m + (e * kH + n0) * (kI / 64), 256, &bar);
+      } else {
+        mbar_add_tx(&bar, 4096 + 128);
+        bulk_g2s(wsm + tid * 4096, L.w2_q + (e * kH + n0) * (kI / 2), 4096, &bar);
+        bulk_g2s(ssm + tid * 128, L.w2_s + (e * kH + n0) * (kI / kG), 128, &bar);
+      }
       if (tid == 0) s_ns = min(slot_count(word), umax);
     }
   } else if (tid == kE && with_shared) {
-    mbar_add_tx(&bar, 8192 + 256);
-    bulk_g2s(shm, L.sh2_q + (size_t)n0 * (kIs / 2), 8192, &bar);
-    bulk_g2s(shs, L.sh2_s + (size_t)n0 * (kIs / kG), 256, &bar);
+    if (kAff) {  // fp16 scales then offsets, 16 per row
+      mbar_add_tx(&bar, 8192 + 1024);
+      bulk_g2s(shm, L.sh2_q + (size_t)n0 * (kIs / 2), 8192, &bar);
+      bulk_g2s(shs, L.sh2_s + (size_t)n0 * (kIs / 64), 512, &bar);
+      bulk_g2s(shs + 512, L.sh2_m + (size_t)n0 * (kIs / 64), 512, &bar);
+    } else {
+      mbar_add_tx(&bar, 8192 + 256);
+      bulk_g2s(shm, L.sh2_q + (size_t)n0 * (kIs / 2), 8192, &bar);
+      bulk_g2s(shs, L.sh2_s + (size_t)n0 * (kIs / kG), 256, &bar);
+    }
   } else if (tid >= kE + 32 && tid < kE + 32 + B * kTopK) {
     const int i = tid - kE - 32;
     s_asc[i] = (int)ld_cg_u32(reinterpret_cast<const uint32_t *>(ws + lay.asc_slot) + i);
@@ -775,6 +891,32 @@ __global__ void __launch_bounds__(kK3Threads)
 
   const uint16_t *gr = kStage ? himg_r : reinterpret_cast<const uint16_t *>(ws + lay.hfr);
   const uint16_t *gs = kStage ? himg_s : reinterpret_cast<const uint16_t *>(ws + lay.hfs);
+  if (kAff) {
+    // an image's 64-group gg (of its 128-group gg / 2, lanes 2 (gg % 2) and
+    // +1) is 64 contiguous bf16 in the fragment order; hi then lo per element
+    for (int task = tid; task < B * (kTopK * 8 + 16); task += kK3Threads) {
+      const bool shr = task >= B * kTopK * 8;
+      const int tk = shr ? task - B * kTopK * 8 : task;
+      const int gg = shr ? tk & 15 : tk & 7, row = shr ? tk >> 4 : tk >> 3;  // row: b*6+j or b
+      const size_t len = shr ? kIs : kI;
+      const uint16_t *hi = shr ? gs + (size_t)(2 * row) * kIs : gr + (size_t)(2 * row) * kI;
+      const size_t off = (size_t)(gg >> 1) * 128 + (size_t)(gg & 1) * 64;
+      float sx = 0.f;
+      for (int e8 = 0; e8 < 8; ++e8) {
+        const uint4 a = kStage ? *reinterpret_cast<const uint4 *>(hi + off + 8 * e8)
+                               : ld_cg_v4(hi + off + 8 * e8);
+        const uint4 c = kStage ? *reinterpret_cast<const uint4 *>(hi + len + off + 8 * e8)
+                               : ld_cg_v4(hi + len + off + 8 * e8);
+        const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wc[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          sx += (__uint_as_float(wa[i] << 16) + __uint_as_float(wc[i] << 16)) +
+                (__uint_as_float(wa[i] & 0xffff0000u) + __uint_as_float(wc[i] & 0xffff0000u));
+      }
+      s_hs[shr ? kMaxB * kTopK + row : row][gg] = sx;
+    }
+    __syncthreads();
+  }
   // tasks: two k-parts (2 groups each) of routed slots 0..ns-1, then four
   // k-parts of the shared expert; partial sums land in ysel[b][m] with
   // m = 2j + part for the row's j-th expert (ascending), 12 + part shared.
@@ -787,13 +929,16 @@ __global__ void __launch_bounds__(kK3Threads)
     const int part = sh ? task - 2 * ns : task & 1;
     const int rowbytes = sh ? kIs / 2 : kI / 2;
     const unsigned char *wbase = sh ? shm : wsm + slot * 4096;
-    const uint16_t *sc = reinterpret_cast<const uint16_t *>(sh ? shs : ssm + slot * 128);
-    const int spr = sh ? kIs / kG : kI / kG;
+    const uint16_t *sc =
+        reinterpret_cast<const uint16_t *>(sh ? shs : ssm + slot * (kAff ? 512 : 128));
+    // scale groups per row (affine: per 64, the offsets after the scales)
+    const int spr = kAff ? (sh ? kIs / 64 : kI / 64) : (sh ? kIs / kG : kI / kG);
+    const uint16_t *mo = sc + 16 * spr;
     const uint32_t mask = sh ? ((1u << B) - 1u) : s_rows[slot];
     const int nr = __popc(mask);
     // this lane's column (g) in each pass, and its output row (t)
     const uint16_t *img[2] = {nullptr, nullptr};
-    int orow[2] = {-1, -1}, om[2] = {0, 0};
+    int orow[2] = {-1, -1}, om[2] = {0, 0}, hrow[2] = {0, 0};
 #pragma unroll
     for (int p = 0; p < 2; ++p) {
       const int ic = 4 * p + (g >> 1), io = 4 * p + t;
@@ -810,10 +955,12 @@ __global__ void __launch_bounds__(kK3Threads)
         if (sh) {
           orow[p] = io;
           om[p] = 12 + part;
+          hrow[p] = kMaxB * kTopK + io;
         } else {
           const int bj = s_rbj[slot][io];
           orow[p] = bj & 15;
           om[p] = 2 * (bj >> 4) + part;
+          hrow[p] = (bj & 15) * kTopK + (bj >> 4);
         }
       }
     }
@@ -825,10 +972,15 @@ __global__ void __launch_bounds__(kK3Threads)
       const uint4 w1 =
           *reinterpret_cast<const uint4 *>(wbase + (g + 8) * rowbytes + 64 * G + 16 * t);
       uint32_t ra[16], rb[16];
-      int4x32_to_bf16x2(w0, ra);
-      int4x32_to_bf16x2(w1, rb);
-      const float s0 = bf16_bits_to_f32(sc[g * spr + G]);
-      const float s1 = bf16_bits_to_f32(sc[(g + 8) * spr + G]);
+      if (kAff) {
+        uint4x32_to_bf16x2(w0, ra);
+        uint4x32_to_bf16x2(w1, rb);
+      } else {
+        int4x32_to_bf16x2(w0, ra);
+        int4x32_to_bf16x2(w1, rb);
+      }
+      const float s0 = kAff ? 0.f : bf16_bits_to_f32(sc[g * spr + G]);
+      const float s1 = kAff ? 0.f : bf16_bits_to_f32(sc[(g + 8) * spr + G]);
 #pragma unroll
       for (int p = 0; p < 2; ++p) {
         if (4 * p < nr) {  // the same for the whole warp
@@ -845,10 +997,31 @@ __global__ void __launch_bounds__(kK3Threads)
 #pragma unroll
             for (int i = 0; i < 16; ++i) xb[i] = 0u;
           }
-          float d[4] = {0.f, 0.f, 0.f, 0.f};
-          group_mma_acc(ra, rb, xb, d);
-          acc[p][0] = fmaf(d[0] + d[1], s0, acc[p][0]);
-          acc[p][1] = fmaf(d[2] + d[3], s1, acc[p][1]);
+          if (kAff) {
+            // lanes t < 2 hold 64-group 2G of the 128-group, t >= 2 group
+            // 2G + 1: one MMA per group with the other's columns zeroed
+            const uint32_t mA = t < 2 ? 0xffffffffu : 0u, mB = ~mA;
+            uint32_t xa[16], xo[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) xa[i] = xb[i] & mA, xo[i] = xb[i] & mB;
+            float dA[4] = {0.f, 0.f, 0.f, 0.f}, dB[4] = {0.f, 0.f, 0.f, 0.f};
+            group_mma_acc(ra, rb, xa, dA);
+            group_mma_acc(ra, rb, xo, dB);
+            const int gA = 2 * G, gB = 2 * G + 1;
+            auto h2f = [](uint16_t v) { return __half2float(__ushort_as_half(v)); };
+            const float hA = s_hs[hrow[p]][gA], hB = s_hs[hrow[p]][gB];
+            acc[p][0] += fmaf(h2f(sc[g * spr + gA]), dA[0] + dA[1], h2f(mo[g * spr + gA]) * hA) +
+                         fmaf(h2f(sc[g * spr + gB]), dB[0] + dB[1], h2f(mo[g * spr + gB]) * hB);
+            acc[p][1] += fmaf(h2f(sc[(g + 8) * spr + gA]), dA[2] + dA[3],
+                              h2f(mo[(g + 8) * spr + gA]) * hA) +
+                         fmaf(h2f(sc[(g + 8) * spr + gB]), dB[2] + dB[3],
+                              h2f(mo[(g + 8) * spr + gB]) * hB);
+          } else {
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            group_mma_acc(ra, rb, xb, d);
+            acc[p][0] = fmaf(d[0] + d[1], s0, acc[p][0]);
+            acc[p][1] = fmaf(d[2] + d[3], s1, acc[p][1]);
+          }
         }
       }
     }
@@ -905,22 +1078,30 @@ static int current_device() {
 }
 
 // dynamic shared memory cap: the 227 KB opt-in limit minus K3's static arrays
-constexpr size_t kK3MaxSmem = 224 * 1024;
+// (1.6 KB; 5.2 KB with the affine format's intermediate group sums)
+constexpr size_t kK3MaxSmem = 224 * 1024, kK3MaxSmemAff = 220 * 1024;
 constexpr int kK1Smem = 16 * kRouterRowStride + kXFragBytes;
-constexpr int kK2Smem = kK2Stages * kItemBytes + kXFragBytes;  // ring + fragment for B <= 8
-static size_t k2_smem(int B) { return (size_t)kK2Stages * kItemBytes + (size_t)4096 * B; }
+constexpr int kK2Smem = kK2Stages * kItemBytesAff + kXFragBytes;  // ring + fragment, B <= 8
+static size_t k2_smem(int B, bool aff) {
+  return (size_t)kK2Stages * (aff ? kItemBytesAff : kItemBytes) + (size_t)4096 * B;
+}
 
 // K2 grid: as many CTAs as fit on the device at once (at most one per item),
 // but never so few that a CTA would own more than kK2MaxItems items.
-static int k2_grid(int dev, int B, int n_items) {
-  static int cache[64][kMaxB + 1];  // 0 = not computed
-  int per_sm = dev < 64 ? cache[dev][B] : 0;
+static int k2_grid(int dev, int B, int n_items, bool aff) {
+  static int cache[64][2][kMaxB + 1];  // 0 = not computed
+  int per_sm = dev < 64 ? cache[dev][aff][B] : 0;
   if (per_sm == 0) {
     int sms = 0, occ = 0;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k2_gateup, kK2Warps * 32, k2_smem(B));
+    if (aff)
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k2_gateup<true>, kK2Warps * 32,
+                                                    k2_smem(B, true));
+    else
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k2_gateup<false>, kK2Warps * 32,
+                                                    k2_smem(B, false));
     per_sm = sms * (occ > 0 ? occ : 1);
-    if (dev < 64) cache[dev][B] = per_sm;
+    if (dev < 64) cache[dev][aff][B] = per_sm;
   }
   int grid = per_sm < n_items ? per_sm : n_items;
   const int floor_grid = (n_items + kK2MaxItems - 1) / kK2MaxItems;
@@ -935,17 +1116,22 @@ static cudaError_t set_attrs(int dev) {
   cudaError_t e = cudaFuncSetAttribute(k1_router<kResidual>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kK1Smem);
   if (e == cudaSuccess)
-    e = noted(cudaFuncSetAttribute(k2_gateup,
+    e = noted(cudaFuncSetAttribute(k2_gateup<false>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kK2Smem),
               "k2_gateup smem attribute");
   if (e == cudaSuccess)
-    e = noted(cudaFuncSetAttribute(k3_down_combine<kResidual, true>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kK3MaxSmem),
-              "k3 smem attribute");
-  if (e == cudaSuccess)
-    e = noted(cudaFuncSetAttribute(k3_down_combine<kResidual, false>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kK3MaxSmem),
-              "k3 (unstaged) smem attribute");
+    e = noted(cudaFuncSetAttribute(k2_gateup<true>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kK2Smem),
+              "k2_gateup (affine) smem attribute");
+  auto k3_attr = [&](const void *f, size_t cap) {
+    if (e == cudaSuccess)
+      e = noted(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cap),
+                "k3 smem attribute");
+  };
+  k3_attr(reinterpret_cast<const void *>(k3_down_combine<kResidual, true, false>), kK3MaxSmem);
+  k3_attr(reinterpret_cast<const void *>(k3_down_combine<kResidual, false, false>), kK3MaxSmem);
+  k3_attr(reinterpret_cast<const void *>(k3_down_combine<kResidual, true, true>), kK3MaxSmemAff);
+  k3_attr(reinterpret_cast<const void *>(k3_down_combine<kResidual, false, true>), kK3MaxSmemAff);
   if (e == cudaSuccess && dev < 64) done |= uint64_t(1) << dev;
   return e;
 }
@@ -965,18 +1151,28 @@ static cudaError_t launch_decode_t(const LayerArgs &L, const uint16_t *x, float 
   const int umax = kTopK * B < span ? kTopK * B : span;
   const int sh_items = sh.with_shared ? kSharedItems : 0;
   const int n_items = sh_items + 64 * umax;
+  const bool aff = L.fmt == FLINT_FMT_AFFINE_INT4;
   note_step("k2_gateup launch");
-  err = launch_pdl(k2_gateup, k2_grid(current_device(), B, n_items > 0 ? n_items : 1),
-                   kK2Warps * 32, k2_smem(B), st, L, B, n_items, sh_items, ws, lay);
+  const int g2 = k2_grid(current_device(), B, n_items > 0 ? n_items : 1, aff);
+  err = aff ? launch_pdl(k2_gateup<true>, g2, kK2Warps * 32, k2_smem(B, true), st, L, B, n_items,
+                         sh_items, ws, lay)
+            : launch_pdl(k2_gateup<false>, g2, kK2Warps * 32, k2_smem(B, false), st, L, B,
+                         n_items, sh_items, ws, lay);
   if (err != cudaSuccess) return err;
-  const K3Smem P{umax, B};
+  const K3Smem P{umax, B, aff};
   const int wsh = sh.with_shared ? 1 : 0;
   note_step("k3_down_combine launch");
-  if (P.total(true) <= kK3MaxSmem)
-    return launch_pdl(k3_down_combine<kResidual, true>, kH / 16, kK3Threads, P.total(true), st,
-                      L, B, out, h, sh.partial, wsh, ws, lay, umax);
-  return launch_pdl(k3_down_combine<kResidual, false>, kH / 16, kK3Threads, P.total(false), st, L,
-                    B, out, h, sh.partial, wsh, ws, lay, umax);
+  const bool stage = P.total(true) <= (aff ? kK3MaxSmemAff : kK3MaxSmem);
+  const size_t smem = P.total(stage);
+  if (aff)
+    return stage ? launch_pdl(k3_down_combine<kResidual, true, true>, kH / 16, kK3Threads, smem,
+                              st, L, B, out, h, sh.partial, wsh, ws, lay, umax)
+                 : launch_pdl(k3_down_combine<kResidual, false, true>, kH / 16, kK3Threads, smem,
+                              st, L, B, out, h, sh.partial, wsh, ws, lay, umax);
+  return stage ? launch_pdl(k3_down_combine<kResidual, true, false>, kH / 16, kK3Threads, smem, st,
+                            L, B, out, h, sh.partial, wsh, ws, lay, umax)
+               : launch_pdl(k3_down_combine<kResidual, false, false>, kH / 16, kK3Threads, smem,
+                            st, L, B, out, h, sh.partial, wsh, ws, lay, umax);
 }
 
 cudaError_t decode_set_wait_polls(uint32_t polls) {

@@ -116,12 +116,21 @@ struct LayerArgs {
   const uint8_t *sh2_q;
   const uint16_t *sh2_s;
   float interm_div;  // routed up projections stored divided by this (a power of two, >= 1)
+  int fmt;           // FLINT_FMT_SYM_INT4 or FLINT_FMT_AFFINE_INT4 (experts)
+  const uint16_t *w13_m;  // affine offsets (fmt 1)
+  const uint16_t *w2_m;
+  const uint16_t *sh13_m;
+  const uint16_t *sh2_m;
 };
 
 inline LayerArgs layer_args(const flint_moe_layer *l) {
   const int d = l->expert_interm_div > 1 ? l->expert_interm_div : 1;
+  const bool aff = l->format == FLINT_FMT_AFFINE_INT4;
   return LayerArgs{l->router_w, l->router_b, l->w13_q,  l->w13_s, l->w2_q,
-                   l->w2_s,     l->sh13_q,   l->sh13_s, l->sh2_q, l->sh2_s, (float)d};
+                   l->w2_s,     l->sh13_q,   l->sh13_s, l->sh2_q, l->sh2_s, (float)d,
+                   aff ? FLINT_FMT_AFFINE_INT4 : FLINT_FMT_SYM_INT4,
+                   aff ? l->w13_m : nullptr, aff ? l->w2_m : nullptr,
+                   aff ? l->sh13_m : nullptr, aff ? l->sh2_m : nullptr};
 }
 
 // Where the calling thread's last failing CUDA call was made (for
