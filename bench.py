@@ -44,6 +44,9 @@ DECODE_TRAFFIC_RATIO = 110.687744 / 109.891584
 TIMING_REPEATS = 20
 HEAD_COPIES = 3  # copies of the head the head timing rotates over (3 x 158.6 MB > L2)
 EXPERT_BYTES = 1024 * (1024 + 32) + 2048 * (256 + 8)
+# group-64 affine experts: fp16 scale and offset per 64 codes
+AFF_EXPERT_BYTES = 1024 * (1024 + 128) + 2048 * (256 + 32)
+AFF_LAYER_FIXED_BYTES = 256 * 2048 * 2 + 256 * 4 + 2048 * (1024 + 128) + 2048 * (512 + 64)
 HEAD_BYTES = synth.VOCAB * (1024 + 32)
 METRIC = "us per MoE-layer decode (B=4), fraction of HBM roofline"
 
@@ -59,6 +62,7 @@ def parse():
     p.add_argument("--no-head", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
     p.add_argument("--no-prefill", action="store_true")
+    p.add_argument("--no-affine", action="store_true")
     p.add_argument("--prefill-t", type=int, nargs="+", default=[2048, 4096, 32768],
                    help="prefill token counts timed as extra lines")
     return p.parse_args()
@@ -430,6 +434,37 @@ def main():
                            "roofline_frac": b1_bytes / (us1 * 1e-6) / 1e9 / hbm,
                            "bytes_per_layer": b1_bytes}
         del g1, gw1
+
+    # ---- the same stack with group-64 affine int4 experts (MLX int4 / Q4_1
+    # layout): 8 layers of synthetic affine weights (3.7 GB, larger than L2)
+    if not args.no_affine:
+        naff = 8
+        aff_structs = [F.make_layer(synth.affine_layer_device(l, dev)) for l in range(naff)]
+        aff_arr = F.layer_array(aff_structs)
+        for ab in sorted({1, min(B, F.FLINT_MAX_DECODE_B_AFFINE)}):
+            ha = torch.empty((ab, H), dtype=torch.float32, device=dev)
+            nba = F.flint_workspace_bytes(F.FLINT_OP_DECODE, ab)
+            wsa = torch.zeros(nba, dtype=torch.uint8, device=dev)
+            F.flint_workspace_init(wsa, nba)
+
+            def aff_step(s, st, ha=ha, ab=ab, wsa=wsa, nba=nba):
+                ha.copy_(h_dev[s, :ab], non_blocking=True)
+                F.flint_moe_decode_stack(aff_arr, naff, ha, ab, None, None, None, wsa, nba,
+                                         stream=st)
+
+            ga, gwa = capture(aff_step)
+            repsa = timed(ga)
+            usa = statistics.median(repsa) * 1e3 / (args.steps * naff)
+            rec = {"layers": naff, "us_per_layer": usa,
+                   "us_per_layer_min": min(repsa) * 1e3 / (args.steps * naff),
+                   "us_per_layer_max": max(repsa) * 1e3 / (args.steps * naff)}
+            if ab == 1:  # six distinct experts: the bytes are known without the routing
+                ab_bytes = AFF_LAYER_FIXED_BYTES + 6 * AFF_EXPERT_BYTES + 2 * H * 4
+                rec.update({"bytes_per_layer": ab_bytes,
+                            "roofline_frac": ab_bytes / (usa * 1e-6) / 1e9 / hbm})
+            extra[f"decode_affine_b{ab}"] = rec
+            del ga, gwa
+        del aff_structs, aff_arr
 
     # ---- e2e through the C ABI with host buffers: H2D of the step's rows,
     # the stack call, D2H of the result rows, every step

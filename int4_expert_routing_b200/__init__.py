@@ -43,6 +43,7 @@ _WEIGHTS = ("router_w", "router_b", "w13_q", "w13_s", "w2_q", "w2_s",
 _OFFSETS = ("w13_m", "w2_m", "sh13_m", "sh2_m")
 FLINT_FMT_SYM_INT4 = 0
 FLINT_FMT_AFFINE_INT4 = 1
+FLINT_MAX_DECODE_B_AFFINE = 7  # decode batch limit of affine layers (flint.h)
 
 
 class flint_moe_layer(C.Structure):
