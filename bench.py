@@ -464,7 +464,10 @@ def main():
                             "roofline_frac": ab_bytes / (usa * 1e-6) / 1e9 / hbm})
             extra[f"decode_affine_b{ab}"] = rec
             del ga, gwa
+        aff_pf = aff_structs[:3]  # prefill on affine experts rotates over three of them
         del aff_structs, aff_arr
+    else:
+        aff_pf = []
 
     # ---- e2e through the C ABI with host buffers: H2D of the step's rows,
     # the stack call, D2H of the result rows, every step
@@ -578,6 +581,14 @@ def main():
                                       "gemm1_TFLOPs": g1_tf, "gemm1_frac": g1_tf / peak_tf,
                                       "gemm2_TFLOPs": g2_tf, "gemm2_frac": g2_tf / peak_tf,
                                       "grouped_gemms_frac": gg_tf / peak_tf}
+            if aff_pf:  # the same call on group-64 affine experts
+                us_a = rotating_us([lambda l=l: F.flint_moe_prefill(l, xt, T, out_t, wsp, nbp,
+                                                                    stream=stream)
+                                    for l in aff_pf], iters=8, skip=2, spin_cycles=2_000_000)
+                tf_a = T * PREFILL_FLOP_PER_TOKEN / (us_a * 1e-6) / 1e12
+                extra[f"prefill_affine_T{T}"] = {"us": us_a, "tokens_per_s": T / (us_a * 1e-6),
+                                                 "TFLOPs": tf_a, "tensor_frac": tf_a / peak_tf,
+                                                 "peak_kind": peak_kind_tf}
             del wsp, out_t, xt
     sampler.stop()
 

@@ -112,9 +112,8 @@ typedef struct {
    * offsets, one per 64 elements along K: w13_s / w13_m [E][2I][H/64],
    * w2_s / w2_m [E][H][I/64], sh13_s / sh13_m [2Is][H/64], sh2_s / sh2_m
    * [H][Is/64]; weight = code * scale + offset.  The *_m pointers are read
-   * only for format 1 (16-byte aligned there).  Decode, route and the stack
-   * and expert-parallel calls take both formats; prefill takes format 0
-   * only (FLINT_EINVAL otherwise). */
+   * only for format 1 (16-byte aligned there).  Every call takes both
+   * formats (decode of format 1 up to FLINT_MAX_DECODE_B_AFFINE rows). */
   int format;
   const uint16_t *w13_m;
   const uint16_t *w2_m;
@@ -279,6 +278,9 @@ FLINT_API int flint_moe_decode_stack(const flint_moe_layer *layers, int L, float
  * power-of-two shift per weight matrix; token rows with one per token) in one
  * fp32 accumulation per output; the SwiGLU intermediate is rounded once, to
  * fp16 after a per-token power-of-two shift from a bound it cannot exceed.
+ * Group-64 affine experts (format 1): each weight code x scale + offset
+ * (times the matrix's power of two) is rounded once to fp16, a relative
+ * error of at most 2^-11 per weight; the rest is as above.
  *   x bf16 [T][2048];  out bf16 [T][2048] (may not alias x);  1 <= T <= 2^20
  *   ws workspace of flint_workspace_bytes(FLINT_OP_PREFILL, T) (about 67 KB
  *      per token, 70 KB up to T = 4,608 where the router keeps two fp64

@@ -346,6 +346,97 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// Group-64 affine experts (unsigned codes n in 0..15, one fp16 scale s and
+// offset m per 64 elements; "How to Run Flint Locally", section "Every build
+// and its size"): a weight n s + m lies between m and 15 s + m, so
+// W = max(|m|, |15 s + m|) bounds the group.  The shift S of a matrix puts its
+// largest W in [2^-7, 2^-6): then |s| 2^-S <= 2 W 2^-S / 15 < 2^-8.9, so the
+// dequant multipliers s 2^(24-S) stay below fp16's largest value, and every
+// weight x 2^-S is at most 2^-6.  A row's norm is at most sqrt(64 sum_g W_g^2).
+FLINT_DEV float affine_bound(uint32_t sbits, uint32_t mbits) {
+  const float s = __half2float(__ushort_as_half((unsigned short)sbits));
+  const float m = __half2float(__ushort_as_half((unsigned short)mbits));
+  return fmaxf(fabsf(m), fabsf(fmaf(15.f, s, m)));
+}
+
+__global__ void __launch_bounds__(256)
+    k_pf_wstats_aff(const uint16_t *__restrict__ w13_s, const uint16_t *__restrict__ w13_m,
+                    const uint16_t *__restrict__ w2_s, const uint16_t *__restrict__ w2_m,
+                    const uint16_t *__restrict__ sh13_s, const uint16_t *__restrict__ sh13_m,
+                    const uint16_t *__restrict__ sh2_s, const uint16_t *__restrict__ sh2_m,
+                    float up_mul, float4 *__restrict__ wst, float *__restrict__ wbound) {
+  pdl_trigger();  // weights only before the wait, as in k_pf_wstats
+  __shared__ float red[4][8];
+  const int e = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool sh = e == kE;
+  constexpr int g13 = kH / 64;  // groups per gate/up row: 4 uint4 of scales, 4 of offsets
+  const int r13 = sh ? 2 * kIs : 2 * kI;
+  const uint16_t *s13 = sh ? sh13_s : w13_s + (size_t)e * r13 * g13;
+  const uint16_t *m13 = sh ? sh13_m : w13_m + (size_t)e * r13 * g13;
+  const int g2 = (sh ? kIs : kI) / 64;
+  const uint16_t *s2 = sh ? sh2_s : w2_s + (size_t)e * kH * g2;
+  const uint16_t *m2 = sh ? sh2_m : w2_m + (size_t)e * kH * g2;
+  float mx1 = 0.f, mx2 = 0.f, bg = 0.f, bu = 0.f;
+#pragma unroll 2
+  for (int r = tid; r < r13; r += 256) {
+    const uint4 *ps = reinterpret_cast<const uint4 *>(s13 + (size_t)r * g13);
+    const uint4 *pm = reinterpret_cast<const uint4 *>(m13 + (size_t)r * g13);
+    uint4 sv[4], mv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sv[i] = __ldg(ps + i), mv[i] = __ldg(pm + i);
+    const float um = (!sh && r >= r13 / 2) ? up_mul : 1.f;  // both s and m were divided
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t a[4] = {sv[i].x, sv[i].y, sv[i].z, sv[i].w};
+      const uint32_t b[4] = {mv[i].x, mv[i].y, mv[i].z, mv[i].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float W = affine_bound(a[q] >> (16 * h), b[q] >> (16 * h)) * um;
+          mx1 = fmaxf(mx1, W);
+          ss = fmaf(W, W, ss);
+        }
+    }
+    const float rb = 8.f * sqrtf(ss);
+    if (r < r13 / 2) bg = fmaxf(bg, rb);
+    else bu = fmaxf(bu, rb);
+  }
+  {  // down: uint4 words of 8 groups (routed 2,048 words, shared 4,096)
+    const int nw = kH * g2 / 8;
+    const uint4 *ps = reinterpret_cast<const uint4 *>(s2), *pm = reinterpret_cast<const uint4 *>(m2);
+#pragma unroll 4
+    for (int k = tid; k < nw; k += 256) {
+      const uint4 sv = __ldg(ps + k), mv = __ldg(pm + k);
+      const uint32_t a[4] = {sv.x, sv.y, sv.z, sv.w}, b[4] = {mv.x, mv.y, mv.z, mv.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        mx2 = fmaxf(mx2, fmaxf(affine_bound(a[q], b[q]), affine_bound(a[q] >> 16, b[q] >> 16)));
+    }
+  }
+  pdl_wait();  // the previous kernel in the stream is complete before any write
+  float v[4] = {mx1, mx2, bg, bu};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v[k] = fmaxf(v[k], __shfl_xor_sync(0xffffffffu, v[k], o));
+    if (lane == 0) red[k][warp] = v[k];
+  }
+  __syncthreads();
+  if (tid == 0) {
+    float m[4];
+    for (int k = 0; k < 4; ++k) {
+      m[k] = red[k][0];
+      for (int w = 1; w < 8; ++w) m[k] = fmaxf(m[k], red[k][w]);
+    }
+    const int S1 = m[0] > 0.f ? clamp_shift(ilogbf(m[0]) + 7) : 0;
+    const int S2 = m[1] > 0.f ? clamp_shift(ilogbf(m[1]) + 7) : 0;
+    wst[e] = make_float4(exp2i(-S1), exp2i(S1), exp2i(-S2), exp2i(S2));
+    wbound[e] = m[2] * m[3];
+  }
+}
+
 // Token rows as the fp16 operand of GEMM 1: rows [0, 6T) are the routed rows
 // in sorted order, rows [6T, 7T) every token for the shared expert.  One warp
 // per token (grid-stride) reads the row once and takes its shifts: F puts
@@ -498,6 +589,8 @@ struct GemmArgs {
   int T;
   const uint16_t *sc_r;  // scales of the routed weight tensor
   const uint16_t *sc_s;  // scales of the shared expert's tensor
+  const uint16_t *mo_r;  // affine: offsets of the routed weight tensor
+  const uint16_t *mo_s;  // affine: offsets of the shared expert's tensor
   const float4 *wst;     // per expert: 2^-S1, 2^S1, 2^-S2, 2^S2
   const uint32_t *rsc;   // per row: F | E << 16 (int16 each): multipliers 2^F, 2^-E
   const float *rm3;      // per row: 2^E x routing weight
@@ -649,12 +742,16 @@ FLINT_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync
 // n 2^-24 (s 2^24) - 8 s (or with s 2^20) forms code x s exactly inside and
 // rounds once, and code x s is itself an fp16, so the result is exact.
 // m24 = s 2^24, m20 = s 2^20 and c8 = -8 s as fp16x2 (both halves equal).
+// Unsigned codes (kSigned false, the affine format) are n itself: with c8 the
+// group's offset m (times 2^-S) the same FMA forms n s + m, rounded once.
+template <bool kSigned = true>
 FLINT_DEV void codes8_f16(uint32_t w, uint32_t m24, uint32_t m20, uint32_t c8, uint32_t *out) {
+  constexpr uint32_t x0 = kSigned ? 0x00080008u : 0u, x1 = kSigned ? 0x00800080u : 0u;
   const uint32_t w8 = w >> 8;
-  const uint32_t t0 = and_xor(w, 0x000F000Fu, 0x00080008u);   // codes 0, 4
-  const uint32_t t1 = and_xor(w, 0x00F000F0u, 0x00800080u);   // codes 1, 5
-  const uint32_t t2 = and_xor(w8, 0x000F000Fu, 0x00080008u);  // codes 2, 6
-  const uint32_t t3 = and_xor(w8, 0x00F000F0u, 0x00800080u);  // codes 3, 7
+  const uint32_t t0 = and_xor(w, 0x000F000Fu, x0);   // codes 0, 4
+  const uint32_t t1 = and_xor(w, 0x00F000F0u, x1);   // codes 1, 5
+  const uint32_t t2 = and_xor(w8, 0x000F000Fu, x0);  // codes 2, 6
+  const uint32_t t3 = and_xor(w8, 0x00F000F0u, x1);  // codes 3, 7
   asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(out[0]) : "r"(t0), "r"(m24), "r"(c8));
   asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(out[1]) : "r"(t1), "r"(m20), "r"(c8));
   asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(out[2]) : "r"(t2), "r"(m24), "r"(c8));
@@ -713,7 +810,7 @@ FLINT_DEV uint2 tile_word(const GemmArgs &args, uint32_t ti, uint32_t ntiles) {
 // carry on across tiles and one tile's epilogue overlaps the next tile's MMAs.
 // Barriers that gather both CTAs (full, afull, accempty) live in the first
 // CTA; the MMA commits arrive on both CTAs' copies of empty, aempty, accfull.
-template <int kMode>
+template <int kMode, bool kAff>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     k_pf_gemm(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
               const __grid_constant__ CUtensorMap tmB_r, const __grid_constant__ CUtensorMap tmB_s,
@@ -890,6 +987,113 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       umma_commit_pair(&mma_done);
       if (!cwait_sleep(&mma_done, 0)) s_fail = 1;
     }  // other lanes and warp 3: idle (register donors)
+  } else if (warp < 8 && kAff) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegDeq));
+    // ---- dequant, group-64 affine weights: as below, but every 64 codes have
+    // their own fp16 scale s and offset m, and a weight is n s + m (times
+    // 2^-S) rounded once to fp16 by the FMA of codes8_f16<false>.  A stage
+    // (two 128-groups) takes four scales and four offsets of the row, one
+    // uint2 apiece: a tile's first stage loaded during the previous tile
+    // (with the tile descriptors two ahead), the others from L1.
+    static_assert(KS == 2, "a stage's four 64-groups are one uint2 of scales and one of offsets");
+    const int i = tid - 128, q = warp - 4;
+    const int raw_row = kMode == 1 ? ((i & 1) ? 64 + (i >> 1) : (i >> 1)) : i;
+    // this thread's row of a tile: its scales and offsets as uint2 (4 groups each)
+    auto row_of = [&](const PfTile &tn, const uint2 *&ps, const uint2 *&pm) {
+      const int wrow = kMode == 1 ? ((i & 1) ? tn.row1 : tn.row0) + (i >> 1) : tn.row0 + i;
+      const size_t g64 = 2 * (size_t)tn.ng;  // 64-groups per row
+      ps = reinterpret_cast<const uint2 *>((tn.sh ? args.sc_s : args.sc_r) + (size_t)wrow * g64);
+      pm = reinterpret_cast<const uint2 *>((tn.sh ? args.mo_s : args.mo_r) + (size_t)wrow * g64);
+    };
+    auto fetch = [&](uint2 w, uint2 &s0, uint2 &m0, float &mul) {  // a tile's first stage
+      PfTile tn;
+      if (!pf_tile<kMode>(args, w, rank, tn)) return;
+      const uint2 *ps, *pm;
+      row_of(tn, ps, pm);
+      s0 = __ldg(ps);
+      m0 = __ldg(pm);
+      const float4 ws = __ldg(args.wst + tn.e);
+      mul = kMode == 1 ? ws.x : ws.z;
+      if (kMode == 1 && (i & 1) && !tn.sh) mul *= args.up_mul;  // routed up rows: undo the divisor
+    };
+    uint2 wa = tile_word(args, pair, ntiles), wb = tile_word(args, pair + npairs, ntiles);
+    uint2 ns = make_uint2(0u, 0u), nm = make_uint2(0u, 0u);
+    float muln = 0.f;
+    fetch(wa, ns, nm, muln);
+    uint32_t it = 0;
+    for (uint32_t ti = pair; ti < ntiles && !s_fail; ti += npairs) {
+      const uint2 w = wa;
+      wa = wb;
+      wb = tile_word(args, ti + 2 * npairs, ntiles);
+      PfTile t;
+      const bool valid = pf_tile<kMode>(args, w, rank, t);
+      uint2 cs = ns, cm = nm;
+      const float smul = muln;
+      fetch(wa, ns, nm, muln);  // the next tile's, in flight during this one
+      if (!valid) continue;
+      const uint2 *ps, *pm;
+      row_of(t, ps, pm);
+      // the row's scales and offsets (t.ng / 2 uint2 each) into L1; a stage's
+      // are read before its wait
+      for (int c = 0; c < t.ng / 2; c += 16) {
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(ps + c));
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(pm + c));
+      }
+      bool ok = true;
+      for (int G0 = 0; G0 < t.ng; G0 += KS, ++it) {
+        if (G0 > 0) cs = __ldg(ps + G0 / 2), cm = __ldg(pm + G0 / 2);
+        const int rr = it % R, a = it % NA;
+        if (!mbar_wait_sleep(&rfull[rr], (it / R) & 1) ||
+            (it >= (uint32_t)NA && !cwait_sleep(&aempty[a], ((it / NA) - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // 64-groups 2 G0 .. 2 G0 + 3 of the row, in memory order
+        const uint32_t sv[4] = {cs.x & 0xffffu, cs.x >> 16, cs.y & 0xffffu, cs.y >> 16};
+        const uint32_t mv[4] = {cm.x & 0xffffu, cm.x >> 16, cm.y & 0xffffu, cm.y >> 16};
+#pragma unroll
+        for (int g = 0; g < KS; ++g) {  // group G0 + g -> TMEM columns 64 g .. of the tile
+          const unsigned char *raw = sm + Cfg::raw_off(rr) + g * kRawBytes + raw_row * 64;
+          const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + Cfg::a_col(a) + 64u * g;
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {  // 64-group 2 (G0 + g) + hf: chunks 2 hf, 2 hf + 1
+            // s 2^(24-S), s 2^(20-S) and m 2^-S as fp16x2: fp16 values times
+            // powers of two, exact while normal (the scale's are, by the
+            // choice of S; an offset far below the group's bound W may round
+            // there, by less than 2^-25 against weights near 2^-7)
+            const float sf = __half2float(__ushort_as_half((unsigned short)sv[2 * g + hf])) * smul;
+            const float mf = __half2float(__ushort_as_half((unsigned short)mv[2 * g + hf])) * smul;
+            const uint32_t h24 = __half_as_ushort(__float2half_rn(sf * 16777216.f));
+            const uint32_t h20 = __half_as_ushort(__float2half_rn(sf * 1048576.f));
+            const uint32_t hm = __half_as_ushort(__float2half_rn(mf));
+            const uint32_t m24 = h24 | (h24 << 16), m20 = h20 | (h20 << 16), mm = hm | (hm << 16);
+            uint32_t v[32];
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+              const int j = 2 * hf + jj;  // the box is 64-byte swizzled, as below
+              const uint4 wv = *reinterpret_cast<const uint4 *>(raw + 16 * (j ^ ((raw_row >> 1) & 3)));
+              codes8_f16<false>(wv.x, m24, m20, mm, v + 16 * jj + 0);
+              codes8_f16<false>(wv.y, m24, m20, mm, v + 16 * jj + 4);
+              codes8_f16<false>(wv.z, m24, m20, mm, v + 16 * jj + 8);
+              codes8_f16<false>(wv.w, m24, m20, mm, v + 16 * jj + 12);
+            }
+            tmem_st32(tbase + 32u * hf, v);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&rempty[rr]);  // the codes are in registers and TMEM
+          mbar_arrive_cluster(afull_cl + 8u * a);
+        }
+      }
+      if (!ok) {
+        s_fail = 1;
+        break;
+      }
+    }
   } else if (warp < 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegDeq));
     // ---- dequant: thread i owns weight row i of every tile, TMEM lane i
@@ -1421,6 +1625,38 @@ cudaError_t prefill_stage_times(float *ms, int n) {
   return e;
 }
 
+// The two grouped GEMMs of a prefill call, for the experts' weight format
+// (symmetric int4 with bf16 scales, or group-64 affine with fp16 scales and
+// offsets): persistent, as many CTA pairs as fit at once (the tile counts are
+// on the device).  Stage event 4 falls between them.
+template <bool kAff>
+cudaError_t launch_gemms(const PrefillLayout &P, const CUtensorMap &mA1r, const CUtensorMap &mA1s,
+                         const CUtensorMap &mB1, const CUtensorMap &mA2r, const CUtensorMap &mA2s,
+                         const CUtensorMap &mB2r, const CUtensorMap &mB2s, const GemmArgs &a1,
+                         const GemmArgs &a2, cudaStream_t st) {
+  cudaError_t e;
+  note_step("prefill GEMM attributes");
+  if ((e = cudaFuncSetAttribute(k_pf_gemm<1, kAff>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)GemmCfg<1>::kSmem)) != cudaSuccess ||
+      (e = cudaFuncSetAttribute(k_pf_gemm<2, kAff>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)GemmCfg<2>::kSmem)) != cudaSuccess)
+    return e;
+  int pairs1 = 0, pairs2 = 0;
+  if ((e = max_pairs(reinterpret_cast<const void *>(k_pf_gemm<1, kAff>), GemmCfg<1>::kSmem,
+                     &pairs1)) ||
+      (e = max_pairs(reinterpret_cast<const void *>(k_pf_gemm<2, kAff>), GemmCfg<2>::kSmem,
+                     &pairs2)))
+    return e;
+  note_step("prefill GEMM 1 launch");
+  e = pf_launch(k_pf_gemm<1, kAff>, 2 * min(P.max_tiles1, pairs1), kGemmThreads, GemmCfg<1>::kSmem,
+                st, mA1r, mA1s, mB1, mB1, a1);
+  if (e != cudaSuccess) return e;
+  stage_mark(4, st);
+  note_step("prefill GEMM 2 launch");
+  return pf_launch(k_pf_gemm<2, kAff>, 2 * min(P.max_tiles2, pairs2), kGemmThreads,
+                   GemmCfg<2>::kSmem, st, mA2r, mA2s, mB2r, mB2s, a2);
+}
+
 cudaError_t launch_route_many(const LayerArgs &L, const uint16_t *x, int T, int32_t *idx, float *w,
                               char *ws, cudaStream_t st) {
   const PrefillLayout P = prefill_layout(T);
@@ -1493,8 +1729,11 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
   stage_mark(2, st);
   // 3. power-of-two shifts of the fp16 operands, and the fp16 token rows
   note_step("prefill operand scaling launches");
-  if ((e = pf_launch(k_pf_wstats, kE + 1, 256, 0, st, L.w13_s, L.w2_s, L.sh13_s, L.sh2_s,
-                     L.interm_div, wst, wbound)))
+  const bool aff = L.fmt == FLINT_FMT_AFFINE_INT4;
+  if ((e = aff ? pf_launch(k_pf_wstats_aff, kE + 1, 256, 0, st, L.w13_s, L.w13_m, L.w2_s, L.w2_m,
+                           L.sh13_s, L.sh13_m, L.sh2_s, L.sh2_m, L.interm_div, wst, wbound)
+               : pf_launch(k_pf_wstats, kE + 1, 256, 0, st, L.w13_s, L.w2_s, L.sh13_s, L.sh2_s,
+                           L.interm_div, wst, wbound)))
     return e;
   {
     int blocks = (T + 7) / 8;  // 8 tokens (warps) per block
@@ -1520,29 +1759,12 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
       (e = make_map(&mB2r, hr, F16, kI, (uint64_t)P.mr, kI * 2, 64, GemmCfg<2>::kBRows, SW)) ||
       (e = make_map(&mB2s, hs, F16, kIs, (uint64_t)T, kIs * 2, 64, GemmCfg<2>::kBRows, SW)))
     return e;
-  note_step("prefill GEMM attributes");
-  if ((e = cudaFuncSetAttribute(k_pf_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)GemmCfg<1>::kSmem)) != cudaSuccess ||
-      (e = cudaFuncSetAttribute(k_pf_gemm<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)GemmCfg<2>::kSmem)) != cudaSuccess)
-    return e;
-  // persistent GEMMs: as many CTA pairs as fit at once (the tile counts are on the device)
-  int pairs1 = 0, pairs2 = 0;
-  if ((e = max_pairs(reinterpret_cast<const void *>(k_pf_gemm<1>), GemmCfg<1>::kSmem, &pairs1)) ||
-      (e = max_pairs(reinterpret_cast<const void *>(k_pf_gemm<2>), GemmCfg<2>::kSmem, &pairs2)))
-    return e;
-  GemmArgs a1{tiles1, ctrl,    3,  ebase, ecount, T,  L.w13_s,   L.sh13_s,
-              wst,    rsc,     rm3, hr,   hs,     ctrl + 1, L.interm_div};
-  note_step("prefill GEMM 1 launch");
-  e = pf_launch(k_pf_gemm<1>, 2 * min(P.max_tiles1, pairs1), kGemmThreads, GemmCfg<1>::kSmem, st,
-                mA1r, mA1s, mB1, mB1, a1);
-  if (e != cudaSuccess) return e;
-  stage_mark(4, st);
-  GemmArgs a2{tiles2, ctrl, 4,  ebase, ecount, T,  L.w2_s,   L.sh2_s,
-              wst,    rsc,  rm3, yw,   ys,     ctrl + 1, 1.f};
-  note_step("prefill GEMM 2 launch");
-  e = pf_launch(k_pf_gemm<2>, 2 * min(P.max_tiles2, pairs2), kGemmThreads, GemmCfg<2>::kSmem, st,
-                mA2r, mA2s, mB2r, mB2s, a2);
+  GemmArgs a1{tiles1, ctrl, 3,   ebase, ecount,   T,   L.w13_s, L.sh13_s, L.w13_m,
+              L.sh13_m, wst, rsc, rm3, hr,     hs, ctrl + 1, L.interm_div};
+  GemmArgs a2{tiles2, ctrl, 4,   ebase, ecount,   T,   L.w2_s, L.sh2_s, L.w2_m,
+              L.sh2_m, wst, rsc, rm3, yw,     ys, ctrl + 1, 1.f};
+  e = aff ? launch_gemms<true>(P, mA1r, mA1s, mB1, mA2r, mA2s, mB2r, mB2s, a1, a2, st)
+          : launch_gemms<false>(P, mA1r, mA1s, mB1, mA2r, mA2s, mB2r, mB2s, a1, a2, st);
   if (e != cudaSuccess) return e;
   stage_mark(5, st);
   // 5. combine

@@ -210,6 +210,23 @@ def divide_routed_up(layer: dict, log2_div: int = 7) -> dict:
     return out
 
 
+def divide_routed_up_affine(layer: dict, log2_div: int = 2) -> dict:
+    """The affine-format counterpart of ``divide_routed_up``: the routed
+    experts' up-projection fp16 scales and offsets (rows I .. 2I-1 of each
+    gate/up block) divided by 2^log2_div by lowering their exponent fields,
+    exact while they stay normal (zeros stay zero)."""
+    out = dict(layer)
+    for name in ("w13_s", "w13_m"):
+        a = layer[name].copy()
+        I = a.shape[1] // 2
+        up = a[:, I:, :].astype(np.int32)
+        nz = (up & 0x7FFF) != 0
+        assert ((up[nz] >> 10) & 0x1F).min() > log2_div, "value would leave the normal range"
+        a[:, I:, :] = np.where(nz, up - (log2_div << 10), up).astype(np.uint16)
+        out[name] = a
+    return out
+
+
 def outlier_channels(hidden: int = HIDDEN, n: int = N_OUTLIERS) -> np.ndarray:
     """The fixed outlier channels: a partial Fisher-Yates shuffle of 0..hidden-1
     drawn from stream (0, T_OUTLIER); the first n entries, in draw order."""

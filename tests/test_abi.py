@@ -74,17 +74,17 @@ def test_bad_arguments_rejected_before_launch(lib):
 
 
 def test_weight_format_rejected_before_launch(lib):
-    """An unknown expert format, an affine layer without its offsets, and an
-    affine layer given to prefill (which reads the symmetric format only) are
-    refused on the host."""
+    """An unknown expert format and an affine layer without its offsets (or
+    with a misaligned one) are refused on the host, by decode and prefill."""
     fake = 1 << 20
     for fmt, offs in ((2, [fake] * 4), (-1, [fake] * 4), (1, [None] * 4), (1, [fake, fake + 2, fake, fake])):
         bad = F.flint_moe_layer(*([fake] * 10), 0, fmt, *offs)
         with pytest.raises(F.FlintError) as e:
             F.flint_moe_decode(bad, fake, 1, fake + 4096, fake, 1 << 20, stream=0)
         assert e.value.code == F.FLINT_EINVAL
-    aff = F.flint_moe_layer(*([fake] * 10), 0, F.FLINT_FMT_AFFINE_INT4, *([fake] * 4))
     nb = F.flint_workspace_bytes(F.FLINT_OP_PREFILL, 16)
-    with pytest.raises(F.FlintError) as e:
-        F.flint_moe_prefill(aff, fake, 16, fake + (1 << 24), fake, nb, stream=0)
-    assert e.value.code == F.FLINT_EINVAL
+    for offs in ([fake, fake, None, fake], [fake, fake, fake, fake + 8]):
+        aff = F.flint_moe_layer(*([fake] * 10), 0, F.FLINT_FMT_AFFINE_INT4, *offs)
+        with pytest.raises(F.FlintError) as e:
+            F.flint_moe_prefill(aff, fake, 16, fake + (1 << 24), fake, nb, stream=0)
+        assert e.value.code == F.FLINT_EINVAL

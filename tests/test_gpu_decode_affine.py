@@ -99,12 +99,3 @@ def test_affine_batch_limit(aff):
                                                          device="cuda"), ws, nb)
     torch().cuda.synchronize()
 
-
-def test_affine_prefill_is_refused(aff):
-    T = 16
-    x = dev_bf16(synth.decode_x(list(range(T))))
-    out = torch().empty((T, 2048), dtype=torch().int16, device="cuda")
-    ws, nb = workspace(F.FLINT_OP_PREFILL, T)
-    with pytest.raises(F.FlintError) as e:
-        F.flint_moe_prefill(aff["L"], x, T, out, ws, nb)
-    assert e.value.code == F.FLINT_EINVAL

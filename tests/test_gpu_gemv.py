@@ -59,7 +59,11 @@ def test_head_batch_invariance(head):
         assert np.array_equal(y4[b], y1[0]) and a4[b] == a1[0]
 
 
-@pytest.mark.parametrize("N,K,B", [(1007, 384, 3), (16, 128, 8), (5, 2048, 1), (4099, 8192, 2)])
+# K = 512, 1,024 and 2,048 take the kernel that holds the activation fragment
+# in registers (with full tiles and a ragged last tile); the others the
+# shared-memory fragment
+@pytest.mark.parametrize("N,K,B", [(1007, 384, 3), (16, 128, 8), (5, 2048, 1), (4099, 8192, 2),
+                                   (1000, 512, 2), (2049, 1024, 5), (3001, 2048, 8)])
 def test_ragged_shapes(N, K, B):
     q = synth.random_bytes(N, 77, N * K // 2).reshape(N, K // 2)
     s = synth.scale_bits(N, 78, N * K // 128).reshape(N, K // 128)
