@@ -69,6 +69,13 @@ enum {
   FLINT_ETIMEOUT = 3, /* a bounded device-side wait gave up (status word) */
   FLINT_EDEVICE = 4   /* a device-side check failed (status word) */
 };
+/* FLINT_EDEVICE comes from the bounds-checked build of this library
+ * (libflint_debug.so, the same sources compiled with FLINT_DEBUG): its kernels
+ * check every index they read back from device memory (slot words, expert
+ * indices, sorted token rows, grouped-GEMM tile descriptors) before it
+ * addresses memory, skip the access when a check fails and record
+ * FLINT_EDEVICE in the call's status word (flint_read_status).  The release
+ * build compiles the checks away.  Both export this same ABI. */
 
 /* Workspace kinds for flint_workspace_bytes. */
 enum { FLINT_OP_ROUTE = 0, FLINT_OP_DECODE = 1, FLINT_OP_PREFILL = 2, FLINT_OP_GEMV = 3 };

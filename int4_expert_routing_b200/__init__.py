@@ -8,11 +8,15 @@ current stream.  A missing or unloadable library raises: there is no fallback.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes as C
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libflint.so")
+# the bounds-checked build (FLINT_DEBUG): same ABI, every index the kernels
+# read back from device memory checked before use (FLINT_EDEVICE on failure)
+DEBUG_LIB_PATH = os.path.join(HERE, "libflint_debug.so")
 
 FLINT_OK, FLINT_EINVAL, FLINT_ECUDA, FLINT_ETIMEOUT, FLINT_EDEVICE = range(5)
 FLINT_OP_ROUTE, FLINT_OP_DECODE, FLINT_OP_PREFILL, FLINT_OP_GEMV = range(4)
@@ -29,6 +33,7 @@ EXPORTS = ("flint_version", "flint_strerror", "flint_last_cuda_error", "flint_wo
            "flint_debug_prefill_stage_ms")
 
 _lib = None
+_loaded = {}  # path -> CDLL with its signatures set
 
 
 class FlintError(RuntimeError):
@@ -52,18 +57,38 @@ class flint_moe_layer(C.Structure):
         (n, C.c_void_p) for n in _OFFSETS]
 
 
-def build(force: bool = False) -> str:
+def build(force: bool = False, debug: bool = False) -> str:
     from . import buildlib
-    return buildlib.build(force=force)
+    return buildlib.build(force=force, debug=debug)
 
 
 def lib() -> C.CDLL:
     """Load libflint.so (raises if it is not built)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"{LIB_PATH} is not built: run int4_expert_routing_b200.build()")
-        L = C.CDLL(LIB_PATH)
+        _lib = _load(LIB_PATH)
+    return _lib
+
+
+@contextlib.contextmanager
+def using_library(path: str):
+    """Route the calls made inside the block to the library at ``path`` (for
+    instance DEBUG_LIB_PATH, built by ``build(debug=True)``); the default
+    library afterwards."""
+    global _lib
+    saved = lib()
+    _lib = _load(path)
+    try:
+        yield _lib
+    finally:
+        _lib = saved
+
+
+def _load(path: str) -> C.CDLL:
+    if path not in _loaded:
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is not built: run int4_expert_routing_b200.build()")
+        L = C.CDLL(path)
         vp, i, sz = C.c_void_p, C.c_int, C.c_size_t
         L.flint_version.restype = i
         L.flint_strerror.restype = C.c_char_p
@@ -93,8 +118,8 @@ def lib() -> C.CDLL:
         L.flint_int4_gemv_noalloc_status.argtypes = [C.POINTER(C.c_int), vp]
         for name in EXPORTS:
             getattr(L, name).restype = getattr(L, name).restype or i
-        _lib = L
-    return _lib
+        _loaded[path] = L
+    return _loaded[path]
 
 
 def strerror(code: int) -> str:

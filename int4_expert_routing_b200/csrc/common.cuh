@@ -41,6 +41,23 @@ constexpr uint32_t kWaitPolls = 1u << 26;
 
 FLINT_DEV void set_status(uint32_t *st, uint32_t code) { atomicCAS(st, 0u, code); }
 
+// The bounds-checked build (FLINT_DEBUG, libflint_debug.so): FLINT_CHECK(ok,
+// status) records a failed check as kStatusDevice in the call's status word
+// (the first error recorded wins) and yields ok, so the caller skips the
+// access it guards.  Every index a kernel reads back from device memory (slot
+// words, expert indices, sorted rows, tile descriptors) passes one before it
+// addresses memory.  In the release build it is the constant true and the
+// check compiles away.
+#ifdef FLINT_DEBUG
+FLINT_DEV bool check_or_flag(bool ok, uint32_t *st) {
+  if (!ok) set_status(st, kStatusDevice);
+  return ok;
+}
+#define FLINT_CHECK(ok, st) ::flint::check_or_flag((ok), (st))
+#else
+#define FLINT_CHECK(ok, st) true
+#endif
+
 // ------------------------------------------------------------------ loads
 // Weights: read once, never written while a kernel runs; keep them out of L1.
 FLINT_DEV uint4 ld_stream(const void *p) {

@@ -618,6 +618,14 @@ __global__ void __launch_bounds__(kK2Warps * 32)
     uint32_t w = kSlotInvalid;
     if (it < sh_items) w = 0u;
     else if (it < n_items) w = ld_cg_u32(slot_word + ((it - sh_items) >> 6));
+    // the bounds-checked build: a routed item's word counts at most 6B slots,
+    // the item's slot among them, and names only rows of this call (a refused
+    // word ends the CTA's list like an invalid one)
+    if (it >= sh_items && w != kSlotInvalid &&
+        !FLINT_CHECK(slot_count(w) <= kTopK * B && ((it - sh_items) >> 6) < slot_count(w) &&
+                         (slot_mask(w) >> B) == 0u,
+                     ctrl + 1))
+      w = kSlotInvalid;
     s_word[tid] = w;
   } else if (tid >= 32 && tid < 32 + B * kTopK) {
     s_aslot[tid - 32] = (int)ld_cg_u32(reinterpret_cast<const uint32_t *>(ws + lay.asc_slot) + tid - 32);
@@ -821,7 +829,12 @@ __global__ void __launch_bounds__(kK3Threads)
     // at most umax slots have room here; a routing left by a failed K1 may
     // hold more, and none of it is used after the status is set
     s_rows[tid] = 0u;  // rows of an invalid slot: none
-    if (word != kSlotInvalid && tid < umax) {
+    // the bounds-checked build: the word counts at most 6B slots, this one
+    // among them, and names only rows of this call
+    if (word != kSlotInvalid && tid < umax &&
+        FLINT_CHECK(slot_count(word) <= kTopK * B && tid < slot_count(word) &&
+                        (slot_mask(word) >> B) == 0u,
+                    ctrl + 1)) {
       const size_t e = slot_expert(word);
       s_rows[tid] = slot_mask(word) & ((1u << B) - 1u);
       if (kAff) {  // fp16 scales then offsets, 8 per row

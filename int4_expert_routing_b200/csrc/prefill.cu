@@ -107,22 +107,27 @@ __global__ void __launch_bounds__(256)
 // ============================================================== stable sort by expert
 // Per chunk of 256 tokens (one per thread), bits[e][w] has bit `lane` set when
 // token 32w + lane of the chunk chose expert e.
-FLINT_DEV void chunk_bits(const int32_t *asc_e, int T, int c, uint32_t (*bits)[8]) {
+FLINT_DEV void chunk_bits(const int32_t *asc_e, int T, int c, uint32_t (*bits)[8],
+                          uint32_t *status) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int i = tid; i < kE * 8; i += 256) bits[i >> 3][i & 7] = 0u;
   __syncthreads();
   const int tok = c * kPfChunk + tid;
   if (tok < T)
-    for (int j = 0; j < kTopK; ++j) atomicOr(&bits[asc_e[(size_t)tok * kTopK + j]][warp], 1u << lane);
+    for (int j = 0; j < kTopK; ++j) {
+      const int e = asc_e[(size_t)tok * kTopK + j];
+      if (FLINT_CHECK((unsigned)e < (unsigned)kE, status)) atomicOr(&bits[e][warp], 1u << lane);
+    }
   __syncthreads();
 }
 
 __global__ void __launch_bounds__(256)
-    k_pf_count(const int32_t *__restrict__ asc_e, int T, int32_t *__restrict__ chunk_cnt) {
+    k_pf_count(const int32_t *__restrict__ asc_e, int T, int32_t *__restrict__ chunk_cnt,
+               uint32_t *__restrict__ status) {
   pdl_wait();  // the previous kernel in the stream is complete (programmatic launch)
   pdl_trigger();
   __shared__ uint32_t bits[kE][8];
-  chunk_bits(asc_e, T, blockIdx.x, bits);
+  chunk_bits(asc_e, T, blockIdx.x, bits, status);
   const int e = threadIdx.x;
   int n = 0;
 #pragma unroll
@@ -213,17 +218,19 @@ __global__ void __launch_bounds__(256)
 // pos[t][j]: the sorted row of token t's j-th expert (ascending expert order)
 __global__ void __launch_bounds__(256)
     k_pf_place(const int32_t *__restrict__ asc_e, int T, const int32_t *__restrict__ chunk_off,
-               const int32_t *__restrict__ ebase, int32_t *__restrict__ pos) {
+               const int32_t *__restrict__ ebase, int32_t *__restrict__ pos,
+               uint32_t *__restrict__ status) {
   pdl_wait();  // the previous kernel in the stream is complete (programmatic launch)
   pdl_trigger();
   __shared__ uint32_t bits[kE][8];
   const int c = blockIdx.x;
-  chunk_bits(asc_e, T, c, bits);
+  chunk_bits(asc_e, T, c, bits, status);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tok = c * kPfChunk + tid;
   if (tok >= T) return;
   for (int j = 0; j < kTopK; ++j) {
     const int e = asc_e[(size_t)tok * kTopK + j];
+    if (!FLINT_CHECK((unsigned)e < (unsigned)kE, status)) continue;  // (flagged in chunk_bits too)
     int rank = __popc(bits[e][warp] & ((1u << lane) - 1u));
     for (int w = 0; w < warp; ++w) rank += __popc(bits[e][w]);
     const int p = ebase[e] + chunk_off[(size_t)c * kE + e] + rank;
@@ -448,7 +455,8 @@ __global__ void __launch_bounds__(256)
 __global__ void __launch_bounds__(256)
     k_pf_gather(const uint16_t *__restrict__ x, int T, const int32_t *__restrict__ pos,
                 const float *__restrict__ asc_w, const float *__restrict__ wbound,
-                uint16_t *__restrict__ xp, uint32_t *__restrict__ rsc, float *__restrict__ rm3) {
+                uint16_t *__restrict__ xp, uint32_t *__restrict__ rsc, float *__restrict__ rm3,
+                uint32_t *__restrict__ status) {
   pdl_wait();  // the previous kernel in the stream is complete (programmatic launch)
   pdl_trigger();
   __shared__ float s_k;
@@ -465,8 +473,12 @@ __global__ void __launch_bounds__(256)
   for (int tok = blockIdx.x * 8 + (threadIdx.x >> 5); tok < T; tok += nwarps) {
     // lanes 0..5: the token's routed rows; lane 6: its shared row
     int myrow = 0;
-    if (lane < kTopK) myrow = __ldg(pos + (size_t)tok * kTopK + lane);
-    else if (lane == kTopK) myrow = 6 * T + tok;
+    if (lane < kTopK) {
+      myrow = __ldg(pos + (size_t)tok * kTopK + lane);
+      if (!FLINT_CHECK((unsigned)myrow < (unsigned)(6 * T), status)) myrow = -1;  // not written
+    } else if (lane == kTopK) {
+      myrow = 6 * T + tok;
+    }
     const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)tok * kH);
     uint4 v[8];
 #pragma unroll
@@ -508,11 +520,12 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int j = 0; j <= kTopK; ++j) {
       const int row = __shfl_sync(0xffffffffu, myrow, j);
+      if (row < 0) continue;  // a row the bounds-checked build refused (the same for the warp)
       uint4 *dst = reinterpret_cast<uint4 *>(xp + (size_t)row * kH);
 #pragma unroll
       for (int c = 0; c < 8; ++c) dst[32 * c + lane] = v[c];
     }
-    if (lane <= kTopK) {
+    if (lane <= kTopK && myrow >= 0) {
       rsc[myrow] = ((uint32_t)F & 0xffffu) | ((uint32_t)E << 16);
       rm3[myrow] = lane < kTopK ? exp2i(E) * __ldg(asc_w + (size_t)tok * kTopK + lane) : exp2i(E);
     }
@@ -786,6 +799,16 @@ FLINT_DEV bool pf_tile(const GemmArgs &args, uint2 w, uint32_t rank, PfTile &t) 
   t.n_valid = (int)(w.y >> 23);
   t.sh = t.e == kE;
   if (t.n_valid <= 0) return false;  // guards against an N = 0 MMA
+  // the bounds-checked build: the descriptor names an expert (or the shared
+  // one), a weight tile inside its matrix and token rows inside the operand
+  // and output arrays; every role of both CTAs refuses the same tiles
+  if (!FLINT_CHECK(t.e <= kE && t.n_valid <= kN &&
+                       t.mt < (kMode == 1 ? (t.sh ? kIs : kI) / 64 : kH / 128) &&
+                       (t.sh ? t.n0 + t.n_valid <= args.T
+                             : t.b_row + t.n_valid <= kTopK * args.T) &&
+                       (!t.sh || t.b_row == kTopK * args.T + t.n0),
+                   args.status))
+    return false;
   t.n_mma = (t.n_valid + 31) & ~31;  // the pair MMA takes N in steps of 32
   t.ng = (kMode == 1 ? kH : (t.sh ? kIs : kI)) / kG;  // 128-wide k-groups
   if (kMode == 1) {  // weight rows: gate (tile rows 2i) / up (2i+1)
@@ -1491,7 +1514,8 @@ __global__ void __launch_bounds__(kRtThreads, 1)
 // ============================================================== combine
 __global__ void __launch_bounds__(256)
     k_pf_combine(const int32_t *__restrict__ pos, const uint16_t *__restrict__ yw,
-                 const uint16_t *__restrict__ ys, int T, uint16_t *__restrict__ out) {
+                 const uint16_t *__restrict__ ys, int T, uint16_t *__restrict__ out,
+                 uint32_t *__restrict__ status) {
   pdl_wait();  // the previous kernel in the stream is complete (programmatic launch)
   pdl_trigger();
   const size_t n = (size_t)T * (kH / 8);
@@ -1499,7 +1523,9 @@ __global__ void __launch_bounds__(256)
     const size_t tok = i / (kH / 8), c = i % (kH / 8);
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int j = 0; j <= kTopK; ++j) {
-      const uint16_t *src = j < kTopK ? yw + (size_t)pos[tok * kTopK + j] * kH : ys + tok * kH;
+      const int p = j < kTopK ? pos[tok * kTopK + j] : 0;
+      if (!FLINT_CHECK(j == kTopK || (unsigned)p < (unsigned)(6 * T), status)) continue;
+      const uint16_t *src = j < kTopK ? yw + (size_t)p * kH : ys + tok * kH;
       const uint4 v = ld_cg_v4(src + 8 * c);
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -1721,10 +1747,10 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
   stage_mark(1, st);
   // 2. stable sort by expert
   note_step("prefill sort launches");
-  if ((e = pf_launch(k_pf_count, P.nchunks, 256, 0, st, asc_e, T, cc)) ||
+  if ((e = pf_launch(k_pf_count, P.nchunks, 256, 0, st, asc_e, T, cc, ctrl + 1)) ||
       (e = pf_launch(k_pf_scan, 1, 256, 0, st, T, P.nchunks, cc, co, ebase, ecount, tiles1, tiles2,
                      ctrl)) ||
-      (e = pf_launch(k_pf_place, P.nchunks, 256, 0, st, asc_e, T, co, ebase, pos)))
+      (e = pf_launch(k_pf_place, P.nchunks, 256, 0, st, asc_e, T, co, ebase, pos, ctrl + 1)))
     return e;
   stage_mark(2, st);
   // 3. power-of-two shifts of the fp16 operands, and the fp16 token rows
@@ -1738,7 +1764,8 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
   {
     int blocks = (T + 7) / 8;  // 8 tokens (warps) per block
     if (blocks > 148 * 8) blocks = 148 * 8;
-    if ((e = pf_launch(k_pf_gather, blocks, 256, 0, st, x, T, pos, asc_w, wbound, xp, rsc, rm3)))
+    if ((e = pf_launch(k_pf_gather, blocks, 256, 0, st, x, T, pos, asc_w, wbound, xp, rsc, rm3,
+                       ctrl + 1)))
       return e;
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1772,7 +1799,8 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
   {
     int blocks = (int)(((size_t)T * (kH / 8) + 255) / 256);
     if (blocks > 148 * 16) blocks = 148 * 16;
-    if ((e = pf_launch(k_pf_combine, blocks, 256, 0, st, pos, yw, ys, T, out))) return e;
+    if ((e = pf_launch(k_pf_combine, blocks, 256, 0, st, pos, yw, ys, T, out, ctrl + 1)))
+      return e;
   }
   stage_mark(6, st);
   return cudaGetLastError();

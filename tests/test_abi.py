@@ -33,6 +33,22 @@ def test_every_declared_symbol_is_exported(lib):
     assert set(names) == set(F.EXPORTS)
 
 
+def test_bounds_checked_build_exports_the_same_symbols():
+    """libflint_debug.so (FLINT_DEBUG) is the same ABI: it builds from the same
+    sources and exports every declared entry point; its argument checks are
+    the release library's."""
+    F.build(debug=True)
+    with F.using_library(F.DEBUG_LIB_PATH) as dbg:
+        for n in declared_entry_points():
+            assert hasattr(dbg, n), n
+        assert F.lib() is dbg and F.version() >= 100
+        with pytest.raises(F.FlintError) as e:
+            F.flint_int4_gemv(1 << 20, 1 << 20, 16, 100, 1 << 20, 1, 1 << 20, None, 1 << 20,
+                              1 << 20, stream=0)
+        assert e.value.code == F.FLINT_EINVAL
+    assert F.lib()._name == F.LIB_PATH  # the default library again
+
+
 def test_version_and_strerror(lib):
     assert F.version() >= 100
     assert "invalid" in F.strerror(F.FLINT_EINVAL)
