@@ -66,7 +66,8 @@ class _LayerC(C.Structure):
         (n, C.c_void_p) for n in ("router_w", "router_b", "w13_q", "w13_s", "w2_q", "w2_s",
                                   "sh13_q", "sh13_s", "sh2_q", "sh2_s")] + [
         ("expert_interm_div", C.c_double), ("format", C.c_int)] + [
-        (n, C.c_void_p) for n in ("w13_m", "w2_m", "sh13_m", "sh2_m")]
+        (n, C.c_void_p) for n in ("w13_m", "w2_m", "sh13_m", "sh2_m",
+                                  "w13_g", "w2_g", "sh13_g", "sh2_g")]
 
 
 _DT = {"router_w": np.uint16, "router_b": np.float32, "w13_q": np.uint8, "w13_s": np.uint16,
@@ -75,25 +76,34 @@ _DT = {"router_w": np.uint16, "router_b": np.float32, "w13_q": np.uint8, "w13_s"
 
 
 _OFFSETS = ("w13_m", "w2_m", "sh13_m", "sh2_m")
+_GLOBALS = ("w13_g", "w2_g", "sh13_g", "sh2_g")
+_SCALES = ("w13_s", "w2_s", "sh13_s", "sh2_s")
 
 
 class Layer:
-    """A MoE layer's host tensors (the dict ``synth.layer_host`` returns, or
+    """A MoE layer's host tensors (the dict ``synth.layer_host`` returns;
     ``synth.affine_layer_host``: with the *_m offset arrays the expert
-    matrices are read as group-64 affine int4)."""
+    matrices are read as group-64 affine int4; ``synth.nvfp4_layer_host``:
+    with the *_g global scales they are NVFP4, the *_s arrays E4M3 bytes)."""
 
     def __init__(self, t: dict, top_k: int = 6, expert_interm_div: float = 0.0):
-        self.t = {k: np.ascontiguousarray(t[k], dtype=_DT[k]) for k in _DT}
         self.affine = "w13_m" in t
+        self.nvfp4 = "w13_g" in t
+        self.t = {k: np.ascontiguousarray(t[k], dtype=np.uint8 if (self.nvfp4 and k in _SCALES)
+                                          else _DT[k]) for k in _DT}
         if self.affine:
             self.t.update({k: np.ascontiguousarray(t[k], dtype=np.uint16) for k in _OFFSETS})
+        if self.nvfp4:
+            self.t.update({k: np.ascontiguousarray(t[k], dtype=np.float32) for k in _GLOBALS})
         E, H = self.t["router_w"].shape
         self.E, self.H, self.k = E, H, top_k
         self.I = self.t["w13_s"].shape[1] // 2
         self.Is = self.t["sh13_s"].shape[0] // 2
         offs = [_p(self.t[n]).value if self.affine else None for n in _OFFSETS]
+        gls = [_p(self.t[n]).value if self.nvfp4 else None for n in _GLOBALS]
+        fmt = 1 if self.affine else (2 if self.nvfp4 else 0)
         self.c = _LayerC(E, top_k, H, self.I, self.Is, *[_p(self.t[n]).value for n in _DT],
-                         float(expert_interm_div), 1 if self.affine else 0, *offs)
+                         float(expert_interm_div), fmt, *offs, *gls)
 
 
 def unpack_int4(q: np.ndarray) -> np.ndarray:

@@ -334,29 +334,45 @@ void oracle_route(const oracle_layer *L, const uint16_t *x, int B, double *z, do
 /* Several matrix-vector products whose output rows are numbered one after
  * the other, so that one par_for covers them all; each output element is the
  * plain left-to-right row_dot. */
+/* A matrix of the set in one of the layer formats: fmt 0 symmetric int4
+ * (s bf16), 1 group-64 affine (s fp16 scales, m fp16 offsets), 2 NVFP4 (s
+ * E4M3 bytes, g the global scale). */
 typedef struct {
   int n;
-  const uint8_t *q[8];
-  const uint16_t *s[8];
-  const uint16_t *m[8]; /* affine offsets, or NULL for the symmetric format */
-  int64_t K[8], rows[8];
-  const double *x[8];
-  double *y[8];
+  const uint8_t *q[16];
+  const void *s[16];
+  const uint16_t *m[16];
+  int fmt[16];
+  double g[16];
+  int64_t K[16], rows[16];
+  const double *x[16];
+  double *y[16];
 } matvec_set;
+
+static double row_dot_nvfp4(const uint8_t *q, const uint8_t *s, double global, int64_t K,
+                            int64_t n, const double *x) {
+  double acc = 0.0;
+  for (int64_t k = 0; k < K; ++k) acc += weight_nvfp4(q, s, global, K, n, k) * x[k];
+  return acc;
+}
 
 static void matvec_set_row(void *p, int64_t i) {
   matvec_set *m = (matvec_set *)p;
   int j = 0;
   while (i >= m->rows[j]) i -= m->rows[j++];
-  m->y[j][i] = m->m[j] ? row_dot_affine(m->q[j], m->s[j], m->m[j], m->K[j], i, m->x[j])
-                       : row_dot(m->q[j], m->s[j], m->K[j], i, m->x[j]);
+  if (m->fmt[j] == 2)
+    m->y[j][i] = row_dot_nvfp4(m->q[j], (const uint8_t *)m->s[j], m->g[j], m->K[j], i, m->x[j]);
+  else if (m->fmt[j] == 1)
+    m->y[j][i] = row_dot_affine(m->q[j], (const uint16_t *)m->s[j], m->m[j], m->K[j], i, m->x[j]);
+  else
+    m->y[j][i] = row_dot(m->q[j], (const uint16_t *)m->s[j], m->K[j], i, m->x[j]);
 }
 
-static void matvec_set_add(matvec_set *m, const uint8_t *q, const uint16_t *s,
-                           const uint16_t *off, int64_t rows, int64_t K, const double *x,
-                           double *y) {
-  m->q[m->n] = q, m->s[m->n] = s, m->m[m->n] = off, m->rows[m->n] = rows, m->K[m->n] = K;
-  m->x[m->n] = x, m->y[m->n] = y;
+static void matvec_set_add(matvec_set *m, int fmt, const uint8_t *q, const void *s,
+                           const uint16_t *off, double global, int64_t rows, int64_t K,
+                           const double *x, double *y) {
+  m->q[m->n] = q, m->s[m->n] = s, m->m[m->n] = off, m->fmt[m->n] = fmt, m->g[m->n] = global;
+  m->rows[m->n] = rows, m->K[m->n] = K, m->x[m->n] = x, m->y[m->n] = y;
   ++m->n;
 }
 
@@ -376,11 +392,11 @@ void oracle_swiglu_expert(const uint8_t *q13, const uint16_t *s13, const uint8_t
   double *g = (double *)malloc(sizeof(double) * 2 * inter);
   double *hmid = (double *)malloc(sizeof(double) * inter);
   matvec_set m = {0};
-  matvec_set_add(&m, q13, s13, NULL, 2 * inter, hidden, x, g);
+  matvec_set_add(&m, 0, q13, s13, NULL, 0.0, 2 * inter, hidden, x, g);
   matvec_set_run(&m);
   swiglu_mid(g, inter, hmid);
   matvec_set m2 = {0};
-  matvec_set_add(&m2, q2, s2, NULL, hidden, inter, hmid, y);
+  matvec_set_add(&m2, 0, q2, s2, NULL, 0.0, hidden, inter, hmid, y);
   matvec_set_run(&m2);
   free(g);
   free(hmid);
@@ -418,19 +434,34 @@ static void moe_row(void *p, int64_t b) {
     const int inter = j < k ? I : Is;
     const size_t go = 2 * (size_t)I * j, ho = (size_t)I * j;
     if (j < k ? (e < c->e_lo || e >= c->e_hi) : !c->with_shared) continue; /* term not summed */
-    /* scales (and affine offsets) per 128 (symmetric) or 64 (affine) elements */
-    const int gs = L->format == 1 ? 64 : 128;
-    const int aff = L->format == 1;
-    if (j < k) {
-      const int64_t g13 = e * (2 * I) * (H / gs), g2 = e * H * (I / gs);
-      matvec_set_add(&m13, L->w13_q + e * (2 * I) * (H / 2), L->w13_s + g13,
-                     aff ? L->w13_m + g13 : NULL, 2 * inter, H, xd, g + go);
-      matvec_set_add(&m2, L->w2_q + e * H * (I / 2), L->w2_s + g2, aff ? L->w2_m + g2 : NULL, H,
-                     inter, hmid + ho, ys + (size_t)H * j);
+    /* scales (and affine offsets) per 128 (symmetric), 64 (affine) or 16
+     * (NVFP4: one E4M3 byte each) elements; NVFP4 adds a global scale */
+    const int fmt = L->format, aff = fmt == 1, nv = fmt == 2;
+    const int gs = aff ? 64 : (nv ? 16 : 128), sb = nv ? 1 : 2; /* scale bytes */
+    const char *s13b = (const char *)L->w13_s, *s2b = (const char *)L->w2_s;
+    const uint8_t *q13 = j < k ? L->w13_q + e * (2 * I) * (H / 2) : L->sh13_q;
+    const int64_t g13 = j < k ? e * (2 * I) * (H / gs) : 0;
+    const char *s13 = (j < k ? s13b : (const char *)L->sh13_s) + sb * g13;
+    if (nv) {
+      /* NVFP4: the gate rows and the up rows have global scales of their own
+       * (w13_g[e][0], w13_g[e][1]; sh13_g[0], sh13_g[1]) */
+      const float *gl = j < k ? L->w13_g + 2 * e : L->sh13_g;
+      matvec_set_add(&m13, fmt, q13, s13, NULL, (double)gl[0], inter, H, xd, g + go);
+      matvec_set_add(&m13, fmt, q13 + (int64_t)inter * (H / 2), s13 + (int64_t)inter * (H / gs),
+                     NULL, (double)gl[1], inter, H, xd, g + go + inter);
     } else {
-      matvec_set_add(&m13, L->sh13_q, L->sh13_s, aff ? L->sh13_m : NULL, 2 * inter, H, xd, g + go);
-      matvec_set_add(&m2, L->sh2_q, L->sh2_s, aff ? L->sh2_m : NULL, H, inter, hmid + ho,
-                     ys + (size_t)H * j);
+      matvec_set_add(&m13, fmt, q13, s13,
+                     aff ? (j < k ? L->w13_m + g13 : L->sh13_m) : NULL, 0.0, 2 * inter, H, xd,
+                     g + go);
+    }
+    if (j < k) {
+      const int64_t g2 = e * H * (I / gs);
+      matvec_set_add(&m2, fmt, L->w2_q + e * H * (I / 2), s2b + sb * g2,
+                     aff ? L->w2_m + g2 : NULL, nv ? (double)L->w2_g[e] : 0.0, H, inter,
+                     hmid + ho, ys + (size_t)H * j);
+    } else {
+      matvec_set_add(&m2, fmt, L->sh2_q, L->sh2_s, aff ? L->sh2_m : NULL,
+                     nv ? (double)L->sh2_g[0] : 0.0, H, inter, hmid + ho, ys + (size_t)H * j);
     }
   }
   matvec_set_run(&m13);

@@ -56,9 +56,16 @@ typedef struct {
    * section "Every build and its size": the MLX int4 build, the Q4_1 GGUF):
    * unsigned codes 0..15 in the same nibble order, the *_s arrays fp16 scales
    * [rows][K/64] and the *_m arrays fp16 offsets [rows][K/64],
-   * weight = code * scale + offset. */
+   * weight = code * scale + offset.  2 NVFP4 weight-only ("How to Run Flint
+   * Locally", section "What vLLM changed": the NVFP4 checkpoint runs with BF16
+   * activations): the *_q arrays FP4 E2M1 codes in the same nibble order, the
+   * *_s arrays (read as bytes) FP8 E4M3 scales [rows][K/16], and one fp32
+   * global scale per expert matrix in the *_g arrays (w13_g [E] for an
+   * expert's gate and up rows, w2_g [E], sh13_g [1], sh2_g [1]);
+   * weight = e2m1(code) * e4m3(scale) * global. */
   int format;
   const uint16_t *w13_m, *w2_m, *sh13_m, *sh2_m;
+  const float *w13_g, *w2_g, *sh13_g, *sh2_g;
 } oracle_layer;
 
 void oracle_set_threads(int n);

@@ -86,6 +86,11 @@ T_AFL_SH13_S = 44
 T_AFL_SH13_M = 45
 T_AFL_SH2_S = 46
 T_AFL_SH2_M = 47
+T_NVL_W13_S = 50
+T_NVL_W2_S = 51
+T_NVL_SH13_S = 52
+T_NVL_SH2_S = 53
+T_NVL_G = 54
 
 N_OUTLIERS = 8
 OUTLIER_GAIN = 20.0
@@ -368,6 +373,40 @@ def affine_layer_host(seed: int, dims: Dims = FLINT, with_codes: bool = True) ->
     return d
 
 
+NVFP4_LAYER_GLOBAL = 2.0 ** -15
+
+
+def _nvfp4_scales(seed: int, tid: int, rows: int, k: int) -> np.ndarray:
+    """E4M3 bytes [rows, k/16] with exponent field 13 or 14 and any mantissa
+    (values 64 .. 240), as the NVFP4 head recipe."""
+    r = random_bytes(seed, tid, rows * (k // 16)).astype(np.uint32)
+    return (((13 + (r & 1)) << 3) | ((r >> 1) & 7)).astype(np.uint8).reshape(rows, k // 16)
+
+
+def nvfp4_layer_host(seed: int, dims: Dims = FLINT, with_codes: bool = True) -> dict:
+    """A MoE layer whose expert matrices are NVFP4 weight-only: the router as
+    in ``layer_host``; the same packed bytes as the symmetric layer of this
+    seed, each nibble read as an FP4 E2M1 code (uniform over the 16 codes);
+    one E4M3 scale per 16 elements along K (values 64 .. 240) as bytes
+    [rows, K/16] per matrix (w13_s [E, 2I, H/16], w2_s [E, H, I/16], sh13_s
+    [2Is, H/16], sh2_s [H, Is/16]); fp32 global scales 2^-15 x U(0.75, 1.25)
+    per expert matrix (w13_g [E, 2]: gate, up; w2_g [E]; sh13_g [2]; sh2_g
+    [1]).  Weights span about [-0.055, 0.055], rms about 0.011."""
+    dims.check()
+    E, H, I, Is = dims.n_experts, dims.hidden, dims.expert_i, dims.shared_i
+    d = layer_host(seed, dims, with_codes=with_codes)
+    d["w13_s"] = _nvfp4_scales(seed, T_NVL_W13_S, E * 2 * I, H).reshape(E, 2 * I, H // 16)
+    d["w2_s"] = _nvfp4_scales(seed, T_NVL_W2_S, E * H, I).reshape(E, H, I // 16)
+    d["sh13_s"] = _nvfp4_scales(seed, T_NVL_SH13_S, 2 * Is, H)
+    d["sh2_s"] = _nvfp4_scales(seed, T_NVL_SH2_S, H, Is)
+    g = (NVFP4_LAYER_GLOBAL * (0.75 + 0.5 * uniforms(seed, T_NVL_G, 3 * E + 3))).astype(np.float32)
+    d["w13_g"] = g[:2 * E].reshape(E, 2)
+    d["w2_g"] = g[2 * E:3 * E].copy()
+    d["sh13_g"] = g[3 * E:3 * E + 2].copy()
+    d["sh2_g"] = g[3 * E + 2:].copy()
+    return d
+
+
 def affine_from_symmetric(t: dict) -> dict:
     """The same weights in the affine format, exactly: code c -> c + 8 (each
     nibble XOR 8), each bf16 scale -> two fp16 scales of the same value (one
@@ -455,6 +494,13 @@ def to_device(arrays: dict, device) -> dict:
             a = a.view(np.int16)
         out[k] = torch.from_numpy(a).to(device)
     return out
+
+
+def nvfp4_layer_device(seed: int, device, dims: Dims = FLINT) -> dict:
+    """``nvfp4_layer_host`` on ``device``, the codes drawn on the device."""
+    d = to_device(nvfp4_layer_host(seed, dims, with_codes=False), device)
+    d.update(layer_codes_torch(seed, device, dims))
+    return d
 
 
 def affine_layer_device(seed: int, device, dims: Dims = FLINT) -> dict:

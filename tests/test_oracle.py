@@ -514,6 +514,68 @@ def test_affine_layer_equals_symmetric_layer_exactly():
     assert np.array_equal(got, ref) and np.array_equal(idx, idx2)
 
 
+def test_nvfp4_layer_matches_numpy_definition_random():
+    """The block with NVFP4 experts ("How to Run Flint Locally", section "What
+    vLLM changed": NVFP4 weights with BF16 activations): E2M1 codes, E4M3
+    scales per 16, a global scale per matrix (gate and up rows each their own),
+    against a numpy statement built on the published E2M1 table and torch's
+    E4M3 decoder (nvfp4_dequant_np)."""
+    dims = synth.Dims(hidden=256, n_experts=16, top_k=6, expert_i=128, shared_i=256)
+    t = synth.nvfp4_layer_host(17, dims)
+    x = bf16(np.random.default_rng(11).normal(size=(2, 256)))
+    out, idx, w, gap = oracle.moe_layer(oracle.Layer(t), x)
+
+    def expert(q13, s13, g13, q2, s2, g2, xd):
+        I = q13.shape[0] // 2
+        Wg = nvfp4_dequant_np(q13[:I], s13[:I], g13[0])
+        Wu = nvfp4_dequant_np(q13[I:], s13[I:], g13[1])
+        g, u = Wg @ xd, Wu @ xd
+        return nvfp4_dequant_np(q2, s2, g2) @ (g / (1 + np.exp(-g)) * u)
+
+    for row in range(2):
+        xd = synth.bf16_to_f64(x[row])
+        s = 1 / (1 + np.exp(-(synth.bf16_to_f64(t["router_w"]) @ xd)))
+        sel = np.lexsort((np.arange(16), -(s + t["router_b"].astype(np.float64))))[:6]
+        assert list(sel) == list(idx[row])
+        expect = sum(s[e] / s[sel].sum() * expert(t["w13_q"][e], t["w13_s"][e], t["w13_g"][e],
+                                                  t["w2_q"][e], t["w2_s"][e], t["w2_g"][e], xd)
+                     for e in sel)
+        expect = expect + expert(t["sh13_q"], t["sh13_s"], t["sh13_g"], t["sh2_q"], t["sh2_s"],
+                                 t["sh2_g"][0], xd)
+        np.testing.assert_allclose(out[row], expect, rtol=1e-10, atol=1e-13)
+
+
+def test_nvfp4_layer_equals_symmetric_layer_exactly():
+    """Weights that both formats hold exactly: values in {0, +-1, +-2, +-3,
+    +-4, +-6}, as symmetric int4 codes with every bf16 scale 2^-7, and as E2M1
+    codes with every E4M3 scale 1.0 and every global scale 2^-7.  The two
+    blocks are the same function, so their outputs agree bit for bit."""
+    t, dims = tiny_layer(E=8, H=256, I=128, Is=256, seed=27)
+    rng = np.random.default_rng(28)
+    vals = np.array([0, 1, 2, 3, 4, 6, -1, -2, -3, -4, -6])
+    e2m1 = {0: 0x0, 1: 0x2, 2: 0x4, 3: 0x5, 4: 0x6, 6: 0x7}
+    sym, nv = dict(t), dict(t)
+    for name in ("w13", "w2", "sh13", "sh2"):
+        shape = t[name + "_q"].shape
+        v = rng.choice(vals, size=shape[:-1] + (2 * shape[-1],))
+        sym_nib = (v & 0xF).astype(np.uint8)
+        nv_nib = np.vectorize(lambda a: e2m1[abs(a)] | (0x8 if a < 0 else 0))(v).astype(np.uint8)
+        sym[name + "_q"] = sym_nib[..., 0::2] | (sym_nib[..., 1::2] << 4)
+        nv[name + "_q"] = nv_nib[..., 0::2] | (nv_nib[..., 1::2] << 4)
+        ss = t[name + "_s"].shape
+        sym[name + "_s"] = np.full(ss, bf16(2.0 ** -7), np.uint16)
+        nv[name + "_s"] = np.full(ss[:-1] + (ss[-1] * 8,), 0x38, np.uint8)  # E4M3 1.0 per 16
+    E = dims.n_experts
+    nv["w13_g"] = np.full((E, 2), 2.0 ** -7, np.float32)
+    nv["w2_g"] = np.full(E, 2.0 ** -7, np.float32)
+    nv["sh13_g"] = np.full(2, 2.0 ** -7, np.float32)
+    nv["sh2_g"] = np.full(1, 2.0 ** -7, np.float32)
+    x = bf16(rng.normal(size=(3, 256)))
+    ref, idx, *_ = oracle.moe_layer(oracle.Layer(sym), x)
+    got, idx2, *_ = oracle.moe_layer(oracle.Layer(nv), x)
+    assert np.array_equal(got, ref) and np.array_equal(idx, idx2)
+
+
 # ------------------------------------------------------------------ stack
 def test_interm_div_layer_equals_undivided_layer_exactly():
     """Routed up projections stored / 128 with the routing weights multiplied

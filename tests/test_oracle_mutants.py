@@ -24,9 +24,18 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
 # name -> [(text in oracle.c, replacement)]; every text occurs exactly once,
 # and every mutant keeps its indexes inside the arrays it reads
 MUTANTS = {
-    "affine layer read as symmetric": [("m->m[j] ? row_dot_affine(", "0 ? row_dot_affine(")],
-    "affine layer with 128-groups": [("const int gs = L->format == 1 ? 64 : 128;",
-                                      "const int gs = 128;")],
+    "affine layer read as symmetric": [("else if (m->fmt[j] == 1)", "else if (0)")],
+    "affine layer with 128-groups": [("const int gs = aff ? 64 : (nv ? 16 : 128)",
+                                      "const int gs = aff ? 128 : (nv ? 16 : 128)")],
+    "nvfp4 layer read as symmetric": [("if (m->fmt[j] == 2)", "if (0)")],
+    "nvfp4 down global from gate/up": [("nv ? (double)L->w2_g[e] : 0.0",
+                                        "nv ? (double)L->w13_g[e] : 0.0")],
+    "nvfp4 up rows with the gate's global scale": [
+        ("NULL, (double)gl[1], inter, H, xd, g + go + inter);",
+         "NULL, (double)gl[0], inter, H, xd, g + go + inter);")],
+    "nvfp4 gate/up global scales of the wrong expert": [
+        ("const float *gl = j < k ? L->w13_g + 2 * e : L->sh13_g;",
+         "const float *gl = j < k ? L->w13_g + e : L->sh13_g;")],
     "affine down offsets from gate/up": [("aff ? L->w2_m + g2 : NULL", "aff ? L->w13_m + g2 : NULL")],
     "nibble as offset binary": [("return nib >= 8 ? nib - 16 : nib;", "return nib - 8;")],
     "nibble order swapped": [("int nib = (k % 2 == 0) ? (byte & 0x0F) : (byte >> 4);",
