@@ -436,38 +436,43 @@ def main():
         del g1, gw1
 
     # ---- the same stack with group-64 affine int4 experts (MLX int4 / Q4_1
-    # layout): 8 layers of synthetic affine weights (3.7 GB, larger than L2)
+    # layout) and with NVFP4 experts (weight-only, BF16 activations): 8 layers
+    # of synthetic weights each (3.7 GB, larger than L2)
+    aff_pf = []
     if not args.no_affine:
         naff = 8
-        aff_structs = [F.make_layer(synth.affine_layer_device(l, dev)) for l in range(naff)]
-        aff_arr = F.layer_array(aff_structs)
-        for ab in sorted({1, min(B, F.FLINT_MAX_DECODE_B_AFFINE)}):
-            ha = torch.empty((ab, H), dtype=torch.float32, device=dev)
-            nba = F.flint_workspace_bytes(F.FLINT_OP_DECODE, ab)
-            wsa = torch.zeros(nba, dtype=torch.uint8, device=dev)
-            F.flint_workspace_init(wsa, nba)
+        for fmt_name, make in (("affine", synth.affine_layer_device),
+                               ("nvfp4", synth.nvfp4_layer_device)):
+            fmt_structs = [F.make_layer(make(l, dev)) for l in range(naff)]
+            fmt_arr = F.layer_array(fmt_structs)
+            for ab in sorted({1, min(B, F.FLINT_MAX_DECODE_B_AFFINE)}):
+                ha = torch.empty((ab, H), dtype=torch.float32, device=dev)
+                nba = F.flint_workspace_bytes(F.FLINT_OP_DECODE, ab)
+                wsa = torch.zeros(nba, dtype=torch.uint8, device=dev)
+                F.flint_workspace_init(wsa, nba)
 
-            def aff_step(s, st, ha=ha, ab=ab, wsa=wsa, nba=nba):
-                ha.copy_(h_dev[s, :ab], non_blocking=True)
-                F.flint_moe_decode_stack(aff_arr, naff, ha, ab, None, None, None, wsa, nba,
-                                         stream=st)
+                def fmt_step(s, st, ha=ha, ab=ab, wsa=wsa, nba=nba, arr=fmt_arr):
+                    ha.copy_(h_dev[s, :ab], non_blocking=True)
+                    F.flint_moe_decode_stack(arr, naff, ha, ab, None, None, None, wsa, nba,
+                                             stream=st)
 
-            ga, gwa = capture(aff_step)
-            repsa = timed(ga)
-            usa = statistics.median(repsa) * 1e3 / (args.steps * naff)
-            rec = {"layers": naff, "us_per_layer": usa,
-                   "us_per_layer_min": min(repsa) * 1e3 / (args.steps * naff),
-                   "us_per_layer_max": max(repsa) * 1e3 / (args.steps * naff)}
-            if ab == 1:  # six distinct experts: the bytes are known without the routing
-                ab_bytes = AFF_LAYER_FIXED_BYTES + 6 * AFF_EXPERT_BYTES + 2 * H * 4
-                rec.update({"bytes_per_layer": ab_bytes,
-                            "roofline_frac": ab_bytes / (usa * 1e-6) / 1e9 / hbm})
-            extra[f"decode_affine_b{ab}"] = rec
-            del ga, gwa
-        aff_pf = aff_structs[:3]  # prefill on affine experts rotates over three of them
-        del aff_structs, aff_arr
-    else:
-        aff_pf = []
+                ga, gwa = capture(fmt_step)
+                repsa = timed(ga)
+                usa = statistics.median(repsa) * 1e3 / (args.steps * naff)
+                rec = {"layers": naff, "us_per_layer": usa,
+                       "us_per_layer_min": min(repsa) * 1e3 / (args.steps * naff),
+                       "us_per_layer_max": max(repsa) * 1e3 / (args.steps * naff)}
+                if ab == 1:  # six distinct experts: the bytes are known without the routing
+                    # (the same for both formats: 4.5 bits per weight; NVFP4 adds
+                    # 12 bytes of global scales per expert)
+                    ab_bytes = AFF_LAYER_FIXED_BYTES + 6 * AFF_EXPERT_BYTES + 2 * H * 4
+                    rec.update({"bytes_per_layer": ab_bytes,
+                                "roofline_frac": ab_bytes / (usa * 1e-6) / 1e9 / hbm})
+                extra[f"decode_{fmt_name}_b{ab}"] = rec
+                del ga, gwa
+            if fmt_name == "affine":
+                aff_pf = fmt_structs[:3]  # prefill on affine experts rotates over three of them
+            del fmt_structs, fmt_arr
 
     # ---- e2e through the C ABI with host buffers: H2D of the step's rows,
     # the stack call, D2H of the result rows, every step

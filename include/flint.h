@@ -53,10 +53,10 @@ extern "C" {
 #define FLINT_SHARED_I 1024
 #define FLINT_GROUP 128
 #define FLINT_MAX_DECODE_B 8
-/* The decode calls on a layer in the group-64 affine format take B <= 7:
- * each of the 128 down-projection CTAs holds up to 6B experts' rows with
- * their fp16 scales and offsets, and 48 of them do not fit its shared
- * memory.  (flint_moe_route takes B <= 8 in both formats.) */
+/* The decode calls on a layer in the group-64 affine or the NVFP4 format
+ * take B <= 7: each of the 128 down-projection CTAs holds up to 6B experts'
+ * rows with their scales (and offsets), and 48 of them do not fit its shared
+ * memory.  (flint_moe_route takes B <= 8 in every format.) */
 #define FLINT_MAX_DECODE_B_AFFINE 7
 #define FLINT_MAX_PREFILL_T (1 << 20)
 #define FLINT_MAX_STACK_LAYERS 256
@@ -119,17 +119,34 @@ typedef struct {
    * offsets, one per 64 elements along K: w13_s / w13_m [E][2I][H/64],
    * w2_s / w2_m [E][H][I/64], sh13_s / sh13_m [2Is][H/64], sh2_s / sh2_m
    * [H][Is/64]; weight = code * scale + offset.  The *_m pointers are read
-   * only for format 1 (16-byte aligned there).  Every call takes both
-   * formats (decode of format 1 up to FLINT_MAX_DECODE_B_AFFINE rows). */
+   * only for format 1 (16-byte aligned there).
+   * FLINT_FMT_NVFP4 (2): NVFP4 weight-only ("How to Run Flint Locally",
+   * section "What vLLM changed": the NVFP4 checkpoint runs with BF16
+   * activations): the *_q arrays FP4 E2M1 codes in the same nibble order
+   * (the lower nibble is the even element); the *_s arrays FP8 E4M3 scales,
+   * one byte per 16 elements along K (w13_s [E][2I][H/16], w2_s [E][H][I/16],
+   * sh13_s [2Is][H/16], sh2_s [H][Is/16]); and fp32 global scales in the *_g
+   * arrays: w13_g [E][2] (an expert's gate rows, then its up rows), w2_g [E],
+   * sh13_g [2] (gate, up), sh2_g [1]; weight = e2m1(code) * e4m3(scale) *
+   * global.  The *_g pointers are read only for format 2 (4-byte aligned
+   * there).
+   * Decode, route, the stack and expert-parallel calls take every format
+   * (formats 1 and 2 decode up to FLINT_MAX_DECODE_B_AFFINE rows); prefill
+   * takes formats 0 and 1 (FLINT_EINVAL for format 2). */
   int format;
   const uint16_t *w13_m;
   const uint16_t *w2_m;
   const uint16_t *sh13_m;
   const uint16_t *sh2_m;
+  const float *w13_g;
+  const float *w2_g;
+  const float *sh13_g;
+  const float *sh2_g;
 } flint_moe_layer;
 
 #define FLINT_FMT_SYM_INT4 0
 #define FLINT_FMT_AFFINE_INT4 1
+#define FLINT_FMT_NVFP4 2
 
 /* Library version (major*10000 + minor*100 + patch). */
 FLINT_API int flint_version(void);

@@ -46,15 +46,17 @@ class FlintError(RuntimeError):
 _WEIGHTS = ("router_w", "router_b", "w13_q", "w13_s", "w2_q", "w2_s",
             "sh13_q", "sh13_s", "sh2_q", "sh2_s")
 _OFFSETS = ("w13_m", "w2_m", "sh13_m", "sh2_m")
+_GLOBALS = ("w13_g", "w2_g", "sh13_g", "sh2_g")
 FLINT_FMT_SYM_INT4 = 0
 FLINT_FMT_AFFINE_INT4 = 1
-FLINT_MAX_DECODE_B_AFFINE = 7  # decode batch limit of affine layers (flint.h)
+FLINT_FMT_NVFP4 = 2
+FLINT_MAX_DECODE_B_AFFINE = 7  # decode batch limit of affine and NVFP4 layers (flint.h)
 
 
 class flint_moe_layer(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in _WEIGHTS] + [
         ("expert_interm_div", C.c_int), ("format", C.c_int)] + [
-        (n, C.c_void_p) for n in _OFFSETS]
+        (n, C.c_void_p) for n in _OFFSETS + _GLOBALS]
 
 
 def build(force: bool = False, debug: bool = False) -> str:
@@ -155,12 +157,14 @@ def make_layer(t: dict, expert_interm_div: int = 0) -> flint_moe_layer:
     """The C layer struct from a dict of device tensors (keys as in flint.h)
     and the divisor of the routed up projections (0: not divided).  With the
     *_m offset tensors the experts are group-64 affine int4
-    (FLINT_FMT_AFFINE_INT4).  The struct keeps a reference to the tensors, so
-    their memory stays allocated while the struct is alive."""
-    affine = "w13_m" in t
-    layer = flint_moe_layer(*[_ptr(t[n]) for n in _WEIGHTS], int(expert_interm_div),
-                            FLINT_FMT_AFFINE_INT4 if affine else FLINT_FMT_SYM_INT4,
-                            *[_ptr(t[n]) if affine else None for n in _OFFSETS])
+    (FLINT_FMT_AFFINE_INT4); with the *_g global-scale tensors they are NVFP4
+    (FLINT_FMT_NVFP4).  The struct keeps a reference to the tensors, so their
+    memory stays allocated while the struct is alive."""
+    affine, nvfp4 = "w13_m" in t, "w13_g" in t
+    fmt = FLINT_FMT_AFFINE_INT4 if affine else (FLINT_FMT_NVFP4 if nvfp4 else FLINT_FMT_SYM_INT4)
+    layer = flint_moe_layer(*[_ptr(t[n]) for n in _WEIGHTS], int(expert_interm_div), fmt,
+                            *[_ptr(t[n]) if affine else None for n in _OFFSETS],
+                            *[_ptr(t[n]) if nvfp4 else None for n in _GLOBALS])
     layer._tensors = t
     return layer
 

@@ -12,14 +12,22 @@ using namespace flint;
 namespace {
 
 bool aligned16(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// the NVFP4 global-scale arrays are read one float at a time (and an expert
+// shard may offset them by its first expert)
+bool aligned4(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 // 0 or 1 (not divided), or a power of two from 2 to 2^16
 bool div_ok(int d) { return d == 0 || (d > 0 && d <= 65536 && (d & (d - 1)) == 0); }
 
 bool layer_ok(const flint_moe_layer *l) {
-  if (!l || (l->format != FLINT_FMT_SYM_INT4 && l->format != FLINT_FMT_AFFINE_INT4)) return false;
+  if (!l || (l->format != FLINT_FMT_SYM_INT4 && l->format != FLINT_FMT_AFFINE_INT4 &&
+             l->format != FLINT_FMT_NVFP4))
+    return false;
   if (l->format == FLINT_FMT_AFFINE_INT4 &&
       !(aligned16(l->w13_m) && aligned16(l->w2_m) && aligned16(l->sh13_m) && aligned16(l->sh2_m)))
+    return false;
+  if (l->format == FLINT_FMT_NVFP4 &&
+      !(aligned4(l->w13_g) && aligned4(l->w2_g) && aligned4(l->sh13_g) && aligned4(l->sh2_g)))
     return false;
   return div_ok(l->expert_interm_div) && aligned16(l->router_w) && aligned16(l->router_b) &&
          aligned16(l->w13_q) &&
@@ -29,10 +37,11 @@ bool layer_ok(const flint_moe_layer *l) {
 
 // the decode calls' batch limit for a layer: K3 stages up to 6B experts'
 // down rows of its 16 output rows; the affine format's fp16 scales and
-// offsets (4.5 KB a slot instead of 4.1 KB) fit 42 slots, not 48
+// offsets, and the NVFP4 format's E4M3 scales per 16 (4.5 KB a slot instead
+// of 4.1 KB), fit 42 slots, not 48
 bool decode_batch_ok(const flint_moe_layer *l, int B) {
-  return B >= 1 && B <= (l->format == FLINT_FMT_AFFINE_INT4 ? FLINT_MAX_DECODE_B_AFFINE
-                                                            : FLINT_MAX_DECODE_B);
+  return B >= 1 && B <= (l->format != FLINT_FMT_SYM_INT4 ? FLINT_MAX_DECODE_B_AFFINE
+                                                         : FLINT_MAX_DECODE_B);
 }
 
 thread_local cudaError_t g_last_cuda = cudaSuccess;
@@ -251,7 +260,7 @@ int flint_int4_gemv_nvfp4(const uint8_t *q, const uint8_t *s, float global_scale
 
 int flint_moe_prefill(const flint_moe_layer *layer, const uint16_t *x, int T, uint16_t *out,
                       void *ws, size_t ws_bytes, void *stream) {
-  if (!layer_ok(layer) || !aligned16(x) ||
+  if (!layer_ok(layer) || layer->format == FLINT_FMT_NVFP4 || !aligned16(x) ||
       !aligned16(out) || T < 1 || T > FLINT_MAX_PREFILL_T || !aligned16(ws) ||
       ws_bytes < flint_workspace_bytes(FLINT_OP_PREFILL, T) ||
       static_cast<const void *>(x) == static_cast<const void *>(out))

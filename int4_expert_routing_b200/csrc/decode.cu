@@ -444,10 +444,13 @@ constexpr int kK2Groups = 16 / kK2Warps;  // k-groups per warp
 static_assert(kK2Warps * kK2Groups == 16, "the warps split the 16 k-groups evenly");
 constexpr int kItemBytes = 16384 + 512;      // codes, bf16 scales per 128
 constexpr int kItemBytesAff = 16384 + 2048;  // codes, fp16 scales and offsets per 64
+                                             // (NVFP4: E4M3 scales per 16, the same size)
 constexpr int kSharedItems = kIs / 8;
-template <bool kAff>
+// expert formats (FLINT_FMT_*): symmetric int4, group-64 affine int4, NVFP4
+constexpr int kFmtSym = 0, kFmtAff = 1, kFmtNv = 2;
+template <int kFmt>
 constexpr int item_bytes() {
-  return kAff ? kItemBytesAff : kItemBytes;
+  return kFmt == kFmtSym ? kItemBytes : kItemBytesAff;
 }
 
 struct ItemSrc {
@@ -459,24 +462,27 @@ struct ItemSrc {
   const uint16_t *up_m;
 };
 
-// scale (and offset) groups per gate/up row: 16 of 128 or 32 of 64
-template <bool kAff>
+// scale (and offset) words of 16 bits per gate/up row: 16 scales of 128, 32
+// of 64, or (NVFP4) the 128 E4M3 bytes of the blocks of 16 as 64 words
+template <int kFmt>
 constexpr int item_groups() {
-  return kAff ? kH / 64 : kH / kG;
+  return kFmt == kFmtAff ? kH / 64 : (kFmt == kFmtNv ? kH / 32 : kH / kG);
 }
-template <bool kAff>
+template <int kFmt>
 FLINT_DEV ItemSrc shared_item(const LayerArgs &L, int it) {
+  constexpr bool kAff = kFmt == kFmtAff;
   const int r = 8 * it;
-  constexpr int gpr = item_groups<kAff>();
+  constexpr int gpr = item_groups<kFmt>();
   return ItemSrc{L.sh13_q + (size_t)r * (kH / 2), L.sh13_q + (size_t)(kIs + r) * (kH / 2),
                  L.sh13_s + (size_t)r * gpr, L.sh13_s + (size_t)(kIs + r) * gpr,
                  kAff ? L.sh13_m + (size_t)r * gpr : nullptr,
                  kAff ? L.sh13_m + (size_t)(kIs + r) * gpr : nullptr};
 }
-template <bool kAff>
+template <int kFmt>
 FLINT_DEV ItemSrc routed_item(const LayerArgs &L, int e, int r0) {
+  constexpr bool kAff = kFmt == kFmtAff;
   const size_t row = (size_t)e * (2 * kI) + r0;
-  constexpr int gpr = item_groups<kAff>();
+  constexpr int gpr = item_groups<kFmt>();
   return ItemSrc{L.w13_q + row * (kH / 2), L.w13_q + (row + kI) * (kH / 2),
                  L.w13_s + row * gpr, L.w13_s + (row + kI) * gpr,
                  kAff ? L.w13_m + row * gpr : nullptr, kAff ? L.w13_m + (row + kI) * gpr : nullptr};
@@ -484,14 +490,14 @@ FLINT_DEV ItemSrc routed_item(const LayerArgs &L, int e, int r0) {
 // one thread; the caller accounts the bytes on the barrier (mbar_add_tx).
 // Item layout: gate codes, up codes (8 rows x 1 KB each), then the gate and
 // up rows' scales (8 rows x groups) and, affine, their offsets.
-template <bool kAff>
+template <int kFmt>
 FLINT_DEV void issue_item(const ItemSrc &src, unsigned char *buf, uint64_t *bar) {
-  constexpr uint32_t sb = 8 * item_groups<kAff>() * 2;  // 256 or 512 bytes
+  constexpr uint32_t sb = 8 * item_groups<kFmt>() * 2;  // 256, 512 or 1,024 bytes
   bulk_g2s(buf, src.gate, 8192, bar);
   bulk_g2s(buf + 8192, src.up, 8192, bar);
   bulk_g2s(buf + 16384, src.gate_s, sb, bar);
   bulk_g2s(buf + 16384 + sb, src.up_s, sb, bar);
-  if (kAff) {
+  if (kFmt == kFmtAff) {
     bulk_g2s(buf + 16384 + 2 * sb, src.gate_m, sb, bar);
     bulk_g2s(buf + 16384 + 3 * sb, src.up_m, sb, bar);
   }
@@ -565,6 +571,80 @@ FLINT_DEV void item_part_aff(const unsigned char *buf, const uint4 *frag, const 
   }
 }
 
+// 32 NVFP4 codes (one 16-byte load; E2M1, the lower nibble the even element)
+// -> 16 bf16 pairs {w(8q+p), w(8q+p+4)} at register 4q+p (the order of
+// int4x32_to_bf16x2), each weight its code times its 16-element block's E4M3
+// scale: elements 0..15 take the low byte of sw, 16..31 the high byte.  An
+// E2M1 value times an E4M3 scale has at most 6 significant bits and lies in
+// [2^-10, 2,688], so every weight is exact in bf16.  Per pair: the two codes
+// as one byte, the hardware conversion to an fp16 pair (exact), the fp16 bits
+// read as bf16 times 2^-112 (exponent and fraction moved three bits right:
+// exact, zero stays zero), one bf16 multiply by the scale times 2^112 (exact).
+FLINT_DEV uint32_t nv_scale_bf16x2(uint32_t e4m3) {  // the scale x 2^112, both halves
+  uint32_t h;
+  asm("{ .reg .b16 t; cvt.u16.u32 t, %1; cvt.rn.f16x2.e4m3x2 %0, t; }" : "=r"(h) : "r"(e4m3));
+  const float f = __half2float(__ushort_as_half((unsigned short)(h & 0xffffu))) * 0x1p112f;
+  const uint32_t b = __float_as_uint(f) >> 16;  // exact: 4 significant bits
+  return b | (b << 16);
+}
+FLINT_DEV void nvfp4x32_to_bf16x2(const uint4 w, uint32_t sw, uint32_t (&r)[16]) {
+  const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+  const uint32_t sA = nv_scale_bf16x2(sw & 0xffu), sB = nv_scale_bf16x2(sw >> 8);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    // nibbles n0..n7 of the word: lo bytes (n0, n2, n4, n6), hi bytes (n1,
+    // n3, n5, n7); x | x >> 12 puts (n0 | n4 << 4, n2 | n6 << 4) in bytes 0-1
+    const uint32_t lo = words[q] & 0x0F0F0F0Fu, hi = (words[q] >> 4) & 0x0F0F0F0Fu;
+    const uint32_t X = lo | (lo >> 12), Y = hi | (hi >> 12);
+    uint32_t h[4];  // pairs p = 0, 1, 2, 3 as fp16
+    asm("{ .reg .b8 x0, x1, x2, x3, y0, y1, y2, y3;\n"
+        "mov.b32 {x0, x1, x2, x3}, %4;\n"
+        "mov.b32 {y0, y1, y2, y3}, %5;\n"
+        "cvt.rn.f16x2.e2m1x2 %0, x0;\n"
+        "cvt.rn.f16x2.e2m1x2 %1, y0;\n"
+        "cvt.rn.f16x2.e2m1x2 %2, x1;\n"
+        "cvt.rn.f16x2.e2m1x2 %3, y1; }"
+        : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+        : "r"(X), "r"(Y));
+    const uint32_t s2 = q < 2 ? sA : sB;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const uint32_t b = and_or(h[p] >> 3, 0x0FFF0FFFu, h[p] & 0x80008000u);
+      uint32_t c;
+      asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(c) : "r"(b), "r"(s2));
+      r[4 * q + p] = c;
+    }
+  }
+}
+
+// The NVFP4 item: rows g (gate) and g + 8 (up) of the lane's 32 elements as
+// exact bf16 weights, each with its two block scales; the block scales are
+// inside the weights, so the k-groups' sums add up directly.  The expert's
+// global scales are applied by the caller after the warps' sums.
+FLINT_DEV void item_part_nv(const unsigned char *buf, const uint4 *frag, int B, int warp, int lane,
+                            float (&acc)[4]) {
+  const int g = lane >> 2, t = lane & 3;
+  acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+  const unsigned char *sg = buf + 16384 + g * 128, *su = buf + 16384 + 1024 + g * 128;
+#pragma unroll
+  for (int k = 0; k < kK2Groups; ++k) {
+    const int G = kK2Groups * warp + k;
+    const uint4 wg = *reinterpret_cast<const uint4 *>(buf + g * 1024 + 64 * G + 16 * t);
+    const uint4 wu = *reinterpret_cast<const uint4 *>(buf + 8192 + g * 1024 + 64 * G + 16 * t);
+    // blocks 8G + 2t and 8G + 2t + 1 of each row: one 16-bit load
+    const uint32_t sgw = *reinterpret_cast<const uint16_t *>(sg + 8 * G + 2 * t);
+    const uint32_t suw = *reinterpret_cast<const uint16_t *>(su + 8 * G + 2 * t);
+    uint32_t ra[16], rb[16], xb[16];
+    nvfp4x32_to_bf16x2(wg, sgw, ra);
+    nvfp4x32_to_bf16x2(wu, suw, rb);
+    load_frag_compact(frag, G, B, lane, xb);
+    float d[4];
+    group_mma(ra, rb, xb, d);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i] += d[i];
+  }
+}
+
 constexpr int kK2Stages = 2;     // items in flight per CTA
 constexpr int kK2MaxItems = 16;  // items per CTA (the host sizes the grid to keep within it)
 
@@ -572,12 +652,13 @@ constexpr int kK2MaxItems = 16;  // items per CTA (the host sizes the grid to ke
 // shared expert is left to another call), then 64 items per routed slot.
 // CTA c takes items c, c + grid, c + 2 grid, ...; a CTA's first item is
 // fetched before the wait when it is a shared one.
-template <bool kAff>
+template <int kFmt>
 __global__ void __launch_bounds__(kK2Warps * 32)
     k2_gateup(LayerArgs L, int B, int n_items, int sh_items, char *__restrict__ ws,
               DecodeLayout lay) {
   extern __shared__ __align__(128) unsigned char sm[];  // stages | x fragment (compact)
-  constexpr int kIB = item_bytes<kAff>();
+  constexpr bool kAff = kFmt == kFmtAff, kNv = kFmt == kFmtNv;
+  constexpr int kIB = item_bytes<kFmt>();
   uint4 *frag = reinterpret_cast<uint4 *>(sm + kK2Stages * kIB);
   __shared__ __align__(8) uint64_t bar[kK2Stages];
   __shared__ __align__(8) uint64_t fbar;
@@ -600,7 +681,7 @@ __global__ void __launch_bounds__(kK2Warps * 32)
     mbar_init(&fbar, 1);
     if (c0 < sh_items) {
       mbar_add_tx(&bar[0], kIB);
-      issue_item<kAff>(shared_item<kAff>(L, c0), sm, &bar[0]);
+      issue_item<kFmt>(shared_item<kFmt>(L, c0), sm, &bar[0]);
     }
   }
   pdl_wait();  // K1 is complete: routing and the block input fragment are final
@@ -643,8 +724,8 @@ __global__ void __launch_bounds__(kK2Warps * 32)
           mbar_arrive(&bar[0]);  // fetched before the wait
         } else {
           mbar_add_tx(&bar[j], kIB);
-          issue_item<kAff>(it < sh_items ? shared_item<kAff>(L, it)
-                                       : routed_item<kAff>(L, (int)slot_expert(s_word[j]),
+          issue_item<kFmt>(it < sh_items ? shared_item<kFmt>(L, it)
+                                       : routed_item<kFmt>(L, (int)slot_expert(s_word[j]),
                                                      8 * ((it - sh_items) & 63)),
                      sm + j * kIB, &bar[j]);
           mbar_arrive(&bar[j]);
@@ -700,6 +781,8 @@ __global__ void __launch_bounds__(kK2Warps * 32)
     float acc[4];
     if (kAff)
       item_part_aff(buf, frag, &s_xs[0][0], B, warp, lane, acc);
+    else if (kNv)
+      item_part_nv(buf, frag, B, warp, lane, acc);
     else
       item_part(buf, frag, B, warp, lane, acc);
     trace_point(2, 4);
@@ -710,8 +793,8 @@ __global__ void __launch_bounds__(kK2Warps * 32)
     if (tid == 0 && j + kK2Stages < n) {
       const int jn = j + kK2Stages, itn = c0 + jn * step;
       mbar_add_tx(&bar[st], kIB);
-      issue_item<kAff>(itn < sh_items ? shared_item<kAff>(L, itn)
-                                    : routed_item<kAff>(L, (int)slot_expert(s_word[jn]),
+      issue_item<kFmt>(itn < sh_items ? shared_item<kFmt>(L, itn)
+                                    : routed_item<kFmt>(L, (int)slot_expert(s_word[jn]),
                                                   8 * ((itn - sh_items) & 63)),
                  buf, &bar[st]);
       mbar_arrive(&bar[st]);
@@ -723,6 +806,11 @@ __global__ void __launch_bounds__(kK2Warps * 32)
 #pragma unroll
         for (int w = 1; w < kK2Warps; ++w) a += s_acc[w][lane][i];
         acc[i] = a;
+      }
+      if (kNv) {  // the expert's global scales: gate rows, then up rows
+        const float *gp = it < sh_items ? L.sh13_g : L.w13_g + 2 * (size_t)slot_expert(word);
+        const float gg = __ldg(gp), gu = __ldg(gp + 1);
+        acc[0] *= gg, acc[1] *= gg, acc[2] *= gu, acc[3] *= gu;
       }
       if (it < sh_items) {
         uint16_t *hfs = reinterpret_cast<uint16_t *>(ws + lay.hfs);
@@ -763,15 +851,16 @@ __global__ void __launch_bounds__(kK2Warps * 32)
 // ============================================================== K3: down + combine
 // Shared-memory plan (bytes): weights [umax][16 rows][256] | scales
 // [umax][16][4] bf16 (affine: [umax] of fp16 scales [16][8] then offsets
-// [16][8]) | shared down [16][512] | shared scales [16][8] (affine: fp16
-// scales [16][16] then offsets [16][16]) | intermediates (kStage) routed
-// [B][6][2][512] bf16, shared [B][2][1024] | per-row partial results
-// [8 rows][16 parts][16 columns] fp32.
+// [16][8]; NVFP4: [umax] of E4M3 scales [16][32]) | shared down [16][512] |
+// shared scales [16][8] (affine: fp16 scales [16][16] then offsets [16][16];
+// NVFP4: E4M3 [16][64]) | intermediates (kStage) routed [B][6][2][512] bf16,
+// shared [B][2][1024] | per-row partial results [8 rows][16 parts][16
+// columns] fp32.  `wide`: the affine and NVFP4 formats (512-byte slot scales).
 struct K3Smem {
   int umax, B;
-  bool aff;
-  __host__ __device__ int slot_sb() const { return aff ? 512 : 128; }
-  __host__ __device__ int sh_sb() const { return aff ? 1024 : 256; }
+  bool wide;
+  __host__ __device__ int slot_sb() const { return wide ? 512 : 128; }
+  __host__ __device__ int sh_sb() const { return wide ? 1024 : 256; }
   __host__ __device__ size_t w() const { return 0; }
   __host__ __device__ size_t s() const { return (size_t)umax * 4096; }
   __host__ __device__ size_t shw() const { return s() + (size_t)umax * slot_sb(); }
@@ -784,13 +873,14 @@ struct K3Smem {
   __host__ __device__ size_t total(bool stage) const { return ysel(stage) + 8 * 16 * 16 * 4; }
 };
 
-template <bool kResidual, bool kStage, bool kAff>
+template <bool kResidual, bool kStage, int kFmt>
 __global__ void __launch_bounds__(kK3Threads)
     k3_down_combine(LayerArgs L, int B, uint16_t *__restrict__ out, float *__restrict__ h,
                     float *__restrict__ pout, int with_shared, char *__restrict__ ws,
                     DecodeLayout lay, int umax) {
   extern __shared__ __align__(128) unsigned char sm[];
-  const K3Smem P{umax, B, kAff};
+  constexpr bool kAff = kFmt == kFmtAff, kNv = kFmt == kFmtNv;
+  const K3Smem P{umax, B, kFmt != kFmtSym};
   unsigned char *wsm = sm + P.w();
   unsigned char *ssm = sm + P.s();
   unsigned char *shm = sm + P.shw();
@@ -809,6 +899,8 @@ __global__ void __launch_bounds__(kK3Threads)
   // row b's j-th routed expert at b * 6 + j (8 groups), its shared one at
   // 48 + b (16 groups)
   __shared__ float s_hs[kAff ? kMaxB * kTopK + kMaxB : 1][16];
+  // NVFP4: each slot's global scale of its down projection
+  __shared__ float s_gd[kNv ? kMaxB * kTopK : 1];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const int n0 = blockIdx.x * 16;
@@ -842,6 +934,13 @@ __global__ void __launch_bounds__(kK3Threads)
         bulk_g2s(wsm + tid * 4096, L.w2_q + (e * kH + n0) * (kI / 2), 4096, &bar);
         bulk_g2s(ssm + tid * 512, L.w2_s + (e * kH + n0) * (kI / 64), 256, &bar);
         bulk_g2s(ssm + tid * 512 + 256, L.w2_m + (e * kH + n0) * (kI / 64), 256, &bar);
+      } else if (kNv) {  // E4M3 scales, 32 bytes per row; the global scale
+        mbar_add_tx(&bar, 4096 + 512);
+        bulk_g2s(wsm + tid * 4096, L.w2_q + (e * kH + n0) * (kI / 2), 4096, &bar);
+        bulk_g2s(ssm + tid * 512,
+                 reinterpret_cast<const unsigned char *>(L.w2_s) + (e * kH + n0) * (kI / 16), 512,
+                 &bar);
+        s_gd[tid] = __ldg(L.w2_g + e);
       } else {
         mbar_add_tx(&bar, 4096 + 128);
         bulk_g2s(wsm + tid * 4096, L.w2_q + (e * kH + n0) * (kI / 2), 4096, &bar);
@@ -855,6 +954,11 @@ __global__ void __launch_bounds__(kK3Threads)
       bulk_g2s(shm, L.sh2_q + (size_t)n0 * (kIs / 2), 8192, &bar);
       bulk_g2s(shs, L.sh2_s + (size_t)n0 * (kIs / 64), 512, &bar);
       bulk_g2s(shs + 512, L.sh2_m + (size_t)n0 * (kIs / 64), 512, &bar);
+    } else if (kNv) {  // E4M3 scales, 64 bytes per row
+      mbar_add_tx(&bar, 8192 + 1024);
+      bulk_g2s(shm, L.sh2_q + (size_t)n0 * (kIs / 2), 8192, &bar);
+      bulk_g2s(shs, reinterpret_cast<const unsigned char *>(L.sh2_s) + (size_t)n0 * (kIs / 16),
+               1024, &bar);
     } else {
       mbar_add_tx(&bar, 8192 + 256);
       bulk_g2s(shm, L.sh2_q + (size_t)n0 * (kIs / 2), 8192, &bar);
@@ -943,7 +1047,8 @@ __global__ void __launch_bounds__(kK3Threads)
     const int rowbytes = sh ? kIs / 2 : kI / 2;
     const unsigned char *wbase = sh ? shm : wsm + slot * 4096;
     const uint16_t *sc =
-        reinterpret_cast<const uint16_t *>(sh ? shs : ssm + slot * (kAff ? 512 : 128));
+        reinterpret_cast<const uint16_t *>(sh ? shs : ssm + slot * (kFmt != kFmtSym ? 512 : 128));
+    const int nvr = sh ? kIs / 16 : kI / 16;  // NVFP4: scale bytes per row
     // scale groups per row (affine: per 64, the offsets after the scales)
     const int spr = kAff ? (sh ? kIs / 64 : kI / 64) : (sh ? kIs / kG : kI / kG);
     const uint16_t *mo = sc + 16 * spr;
@@ -988,12 +1093,18 @@ __global__ void __launch_bounds__(kK3Threads)
       if (kAff) {
         uint4x32_to_bf16x2(w0, ra);
         uint4x32_to_bf16x2(w1, rb);
+      } else if (kNv) {  // rows g, g + 8: E4M3 bytes of blocks 8G + 2t, 8G + 2t + 1
+        const unsigned char *sb = reinterpret_cast<const unsigned char *>(sc);
+        nvfp4x32_to_bf16x2(w0, *reinterpret_cast<const uint16_t *>(sb + g * nvr + 8 * G + 2 * t),
+                           ra);
+        nvfp4x32_to_bf16x2(
+            w1, *reinterpret_cast<const uint16_t *>(sb + (g + 8) * nvr + 8 * G + 2 * t), rb);
       } else {
         int4x32_to_bf16x2(w0, ra);
         int4x32_to_bf16x2(w1, rb);
       }
-      const float s0 = kAff ? 0.f : bf16_bits_to_f32(sc[g * spr + G]);
-      const float s1 = kAff ? 0.f : bf16_bits_to_f32(sc[(g + 8) * spr + G]);
+      const float s0 = kFmt != kFmtSym ? 0.f : bf16_bits_to_f32(sc[g * spr + G]);
+      const float s1 = kFmt != kFmtSym ? 0.f : bf16_bits_to_f32(sc[(g + 8) * spr + G]);
 #pragma unroll
       for (int p = 0; p < 2; ++p) {
         if (4 * p < nr) {  // the same for the whole warp
@@ -1029,6 +1140,11 @@ __global__ void __launch_bounds__(kK3Threads)
                               h2f(mo[(g + 8) * spr + gA]) * hA) +
                          fmaf(h2f(sc[(g + 8) * spr + gB]), dB[2] + dB[3],
                               h2f(mo[(g + 8) * spr + gB]) * hB);
+          } else if (kNv) {  // the block scales are inside the weights
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            group_mma_acc(ra, rb, xb, d);
+            acc[p][0] += d[0] + d[1];
+            acc[p][1] += d[2] + d[3];
           } else {
             float d[4] = {0.f, 0.f, 0.f, 0.f};
             group_mma_acc(ra, rb, xb, d);
@@ -1038,11 +1154,13 @@ __global__ void __launch_bounds__(kK3Threads)
         }
       }
     }
+    // NVFP4: the down projection's global scale, once per part
+    const float gd = kNv ? (sh ? __ldg(L.sh2_g) : s_gd[slot]) : 1.f;
 #pragma unroll
     for (int p = 0; p < 2; ++p) {
       if (orow[p] >= 0) {
-        ysel[(orow[p] * 16 + om[p]) * 16 + g] = acc[p][0];
-        ysel[(orow[p] * 16 + om[p]) * 16 + g + 8] = acc[p][1];
+        ysel[(orow[p] * 16 + om[p]) * 16 + g] = kNv ? acc[p][0] * gd : acc[p][0];
+        ysel[(orow[p] * 16 + om[p]) * 16 + g + 8] = kNv ? acc[p][1] * gd : acc[p][1];
       }
     }
   }
@@ -1091,30 +1209,37 @@ static int current_device() {
 }
 
 // dynamic shared memory cap: the 227 KB opt-in limit minus K3's static arrays
-// (1.6 KB; 5.2 KB with the affine format's intermediate group sums)
+// (1.6 KB; 5.2 KB with the affine format's intermediate group sums; the NVFP4
+// format's slot global scales are 192 B)
 constexpr size_t kK3MaxSmem = 224 * 1024, kK3MaxSmemAff = 220 * 1024;
 constexpr int kK1Smem = 16 * kRouterRowStride + kXFragBytes;
 constexpr int kK2Smem = kK2Stages * kItemBytesAff + kXFragBytes;  // ring + fragment, B <= 8
-static size_t k2_smem(int B, bool aff) {
-  return (size_t)kK2Stages * (aff ? kItemBytesAff : kItemBytes) + (size_t)4096 * B;
+static size_t k2_smem(int B, int fmt) {
+  return (size_t)kK2Stages * (fmt == kFmtSym ? kItemBytes : kItemBytesAff) + (size_t)4096 * B;
+}
+static size_t k3_cap(int fmt) { return fmt == kFmtSym ? kK3MaxSmem : kK3MaxSmemAff; }
+
+template <int kFmt>
+static int k2_occupancy(int B) {
+  int occ = 0;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k2_gateup<kFmt>, kK2Warps * 32,
+                                                k2_smem(B, kFmt));
+  return occ;
 }
 
 // K2 grid: as many CTAs as fit on the device at once (at most one per item),
 // but never so few that a CTA would own more than kK2MaxItems items.
-static int k2_grid(int dev, int B, int n_items, bool aff) {
-  static int cache[64][2][kMaxB + 1];  // 0 = not computed
-  int per_sm = dev < 64 ? cache[dev][aff][B] : 0;
+static int k2_grid(int dev, int B, int n_items, int fmt) {
+  static int cache[64][3][kMaxB + 1];  // 0 = not computed
+  int per_sm = dev < 64 ? cache[dev][fmt][B] : 0;
   if (per_sm == 0) {
-    int sms = 0, occ = 0;
+    int sms = 0;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (aff)
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k2_gateup<true>, kK2Warps * 32,
-                                                    k2_smem(B, true));
-    else
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k2_gateup<false>, kK2Warps * 32,
-                                                    k2_smem(B, false));
+    const int occ = fmt == kFmtAff  ? k2_occupancy<kFmtAff>(B)
+                    : fmt == kFmtNv ? k2_occupancy<kFmtNv>(B)
+                                    : k2_occupancy<kFmtSym>(B);
     per_sm = sms * (occ > 0 ? occ : 1);
-    if (dev < 64) cache[dev][aff][B] = per_sm;
+    if (dev < 64) cache[dev][fmt][B] = per_sm;
   }
   int grid = per_sm < n_items ? per_sm : n_items;
   const int floor_grid = (n_items + kK2MaxItems - 1) / kK2MaxItems;
@@ -1128,25 +1253,51 @@ static cudaError_t set_attrs(int dev) {
   note_step("k1_router smem attribute");
   cudaError_t e = cudaFuncSetAttribute(k1_router<kResidual>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kK1Smem);
-  if (e == cudaSuccess)
-    e = noted(cudaFuncSetAttribute(k2_gateup<false>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kK2Smem),
-              "k2_gateup smem attribute");
-  if (e == cudaSuccess)
-    e = noted(cudaFuncSetAttribute(k2_gateup<true>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kK2Smem),
-              "k2_gateup (affine) smem attribute");
-  auto k3_attr = [&](const void *f, size_t cap) {
+  auto attr = [&](const void *f, size_t bytes, const char *what) {
     if (e == cudaSuccess)
-      e = noted(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cap),
-                "k3 smem attribute");
+      e = noted(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes),
+                what);
   };
-  k3_attr(reinterpret_cast<const void *>(k3_down_combine<kResidual, true, false>), kK3MaxSmem);
-  k3_attr(reinterpret_cast<const void *>(k3_down_combine<kResidual, false, false>), kK3MaxSmem);
-  k3_attr(reinterpret_cast<const void *>(k3_down_combine<kResidual, true, true>), kK3MaxSmemAff);
-  k3_attr(reinterpret_cast<const void *>(k3_down_combine<kResidual, false, true>), kK3MaxSmemAff);
+  attr(reinterpret_cast<const void *>(k2_gateup<kFmtSym>), kK2Smem, "k2_gateup smem attribute");
+  attr(reinterpret_cast<const void *>(k2_gateup<kFmtAff>), kK2Smem,
+       "k2_gateup (affine) smem attribute");
+  attr(reinterpret_cast<const void *>(k2_gateup<kFmtNv>), kK2Smem,
+       "k2_gateup (NVFP4) smem attribute");
+  attr(reinterpret_cast<const void *>(k3_down_combine<kResidual, true, kFmtSym>), kK3MaxSmem,
+       "k3 smem attribute");
+  attr(reinterpret_cast<const void *>(k3_down_combine<kResidual, false, kFmtSym>), kK3MaxSmem,
+       "k3 smem attribute");
+  attr(reinterpret_cast<const void *>(k3_down_combine<kResidual, true, kFmtAff>), kK3MaxSmemAff,
+       "k3 (affine) smem attribute");
+  attr(reinterpret_cast<const void *>(k3_down_combine<kResidual, false, kFmtAff>), kK3MaxSmemAff,
+       "k3 (affine) smem attribute");
+  attr(reinterpret_cast<const void *>(k3_down_combine<kResidual, true, kFmtNv>), kK3MaxSmemAff,
+       "k3 (NVFP4) smem attribute");
+  attr(reinterpret_cast<const void *>(k3_down_combine<kResidual, false, kFmtNv>), kK3MaxSmemAff,
+       "k3 (NVFP4) smem attribute");
   if (e == cudaSuccess && dev < 64) done |= uint64_t(1) << dev;
   return e;
+}
+
+// K2 and K3 of one decode call for the experts' format
+template <bool kResidual, int kFmt>
+static cudaError_t launch_k2_k3(const LayerArgs &L, int B, uint16_t *out, float *h, char *ws,
+                                const DecodeLayout &lay, cudaStream_t st, const DecodeShard &sh,
+                                int umax, int n_items, int sh_items) {
+  note_step("k2_gateup launch");
+  const int g2 = k2_grid(current_device(), B, n_items > 0 ? n_items : 1, kFmt);
+  cudaError_t err = launch_pdl(k2_gateup<kFmt>, g2, kK2Warps * 32, k2_smem(B, kFmt), st, L, B,
+                               n_items, sh_items, ws, lay);
+  if (err != cudaSuccess) return err;
+  const K3Smem P{umax, B, kFmt != kFmtSym};
+  const int wsh = sh.with_shared ? 1 : 0;
+  note_step("k3_down_combine launch");
+  const bool stage = P.total(true) <= k3_cap(kFmt);
+  const size_t smem = P.total(stage);
+  return stage ? launch_pdl(k3_down_combine<kResidual, true, kFmt>, kH / 16, kK3Threads, smem, st,
+                            L, B, out, h, sh.partial, wsh, ws, lay, umax)
+               : launch_pdl(k3_down_combine<kResidual, false, kFmt>, kH / 16, kK3Threads, smem,
+                            st, L, B, out, h, sh.partial, wsh, ws, lay, umax);
 }
 
 template <bool kResidual>
@@ -1164,28 +1315,11 @@ static cudaError_t launch_decode_t(const LayerArgs &L, const uint16_t *x, float 
   const int umax = kTopK * B < span ? kTopK * B : span;
   const int sh_items = sh.with_shared ? kSharedItems : 0;
   const int n_items = sh_items + 64 * umax;
-  const bool aff = L.fmt == FLINT_FMT_AFFINE_INT4;
-  note_step("k2_gateup launch");
-  const int g2 = k2_grid(current_device(), B, n_items > 0 ? n_items : 1, aff);
-  err = aff ? launch_pdl(k2_gateup<true>, g2, kK2Warps * 32, k2_smem(B, true), st, L, B, n_items,
-                         sh_items, ws, lay)
-            : launch_pdl(k2_gateup<false>, g2, kK2Warps * 32, k2_smem(B, false), st, L, B,
-                         n_items, sh_items, ws, lay);
-  if (err != cudaSuccess) return err;
-  const K3Smem P{umax, B, aff};
-  const int wsh = sh.with_shared ? 1 : 0;
-  note_step("k3_down_combine launch");
-  const bool stage = P.total(true) <= (aff ? kK3MaxSmemAff : kK3MaxSmem);
-  const size_t smem = P.total(stage);
-  if (aff)
-    return stage ? launch_pdl(k3_down_combine<kResidual, true, true>, kH / 16, kK3Threads, smem,
-                              st, L, B, out, h, sh.partial, wsh, ws, lay, umax)
-                 : launch_pdl(k3_down_combine<kResidual, false, true>, kH / 16, kK3Threads, smem,
-                              st, L, B, out, h, sh.partial, wsh, ws, lay, umax);
-  return stage ? launch_pdl(k3_down_combine<kResidual, true, false>, kH / 16, kK3Threads, smem, st,
-                            L, B, out, h, sh.partial, wsh, ws, lay, umax)
-               : launch_pdl(k3_down_combine<kResidual, false, false>, kH / 16, kK3Threads, smem,
-                            st, L, B, out, h, sh.partial, wsh, ws, lay, umax);
+  if (L.fmt == kFmtAff)
+    return launch_k2_k3<kResidual, kFmtAff>(L, B, out, h, ws, lay, st, sh, umax, n_items, sh_items);
+  if (L.fmt == kFmtNv)
+    return launch_k2_k3<kResidual, kFmtNv>(L, B, out, h, ws, lay, st, sh, umax, n_items, sh_items);
+  return launch_k2_k3<kResidual, kFmtSym>(L, B, out, h, ws, lay, st, sh, umax, n_items, sh_items);
 }
 
 cudaError_t decode_set_wait_polls(uint32_t polls) {

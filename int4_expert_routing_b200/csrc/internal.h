@@ -116,21 +116,27 @@ struct LayerArgs {
   const uint8_t *sh2_q;
   const uint16_t *sh2_s;
   float interm_div;  // routed up projections stored divided by this (a power of two, >= 1)
-  int fmt;           // FLINT_FMT_SYM_INT4 or FLINT_FMT_AFFINE_INT4 (experts)
+  int fmt;           // FLINT_FMT_SYM_INT4, _AFFINE_INT4 or _NVFP4 (experts)
   const uint16_t *w13_m;  // affine offsets (fmt 1)
   const uint16_t *w2_m;
   const uint16_t *sh13_m;
   const uint16_t *sh2_m;
+  const float *w13_g;  // NVFP4 global scales (fmt 2): [E][2], [E], [2], [1]
+  const float *w2_g;
+  const float *sh13_g;
+  const float *sh2_g;
 };
 
 inline LayerArgs layer_args(const flint_moe_layer *l) {
   const int d = l->expert_interm_div > 1 ? l->expert_interm_div : 1;
-  const bool aff = l->format == FLINT_FMT_AFFINE_INT4;
+  const bool aff = l->format == FLINT_FMT_AFFINE_INT4, nv = l->format == FLINT_FMT_NVFP4;
   return LayerArgs{l->router_w, l->router_b, l->w13_q,  l->w13_s, l->w2_q,
                    l->w2_s,     l->sh13_q,   l->sh13_s, l->sh2_q, l->sh2_s, (float)d,
-                   aff ? FLINT_FMT_AFFINE_INT4 : FLINT_FMT_SYM_INT4,
+                   l->format,
                    aff ? l->w13_m : nullptr, aff ? l->w2_m : nullptr,
-                   aff ? l->sh13_m : nullptr, aff ? l->sh2_m : nullptr};
+                   aff ? l->sh13_m : nullptr, aff ? l->sh2_m : nullptr,
+                   nv ? l->w13_g : nullptr, nv ? l->w2_g : nullptr,
+                   nv ? l->sh13_g : nullptr, nv ? l->sh2_g : nullptr};
 }
 
 // Where the calling thread's last failing CUDA call was made (for

@@ -90,17 +90,22 @@ def test_bad_arguments_rejected_before_launch(lib):
 
 
 def test_weight_format_rejected_before_launch(lib):
-    """An unknown expert format and an affine layer without its offsets (or
-    with a misaligned one) are refused on the host, by decode and prefill."""
+    """An unknown expert format, an affine layer without its offsets (or
+    with a misaligned one) and an NVFP4 layer without its global scales (or
+    with a misaligned one) are refused on the host, by decode and prefill; an
+    NVFP4 layer is refused by prefill."""
     fake = 1 << 20
-    for fmt, offs in ((2, [fake] * 4), (-1, [fake] * 4), (1, [None] * 4), (1, [fake, fake + 2, fake, fake])):
+    for fmt, offs in ((3, [fake] * 8), (-1, [fake] * 8), (1, [None] * 8),
+                      (1, [fake, fake + 2, fake, fake] + [None] * 4),
+                      (2, [fake] * 4 + [None] * 4), (2, [None] * 4 + [fake, fake + 2, fake, fake])):
         bad = F.flint_moe_layer(*([fake] * 10), 0, fmt, *offs)
         with pytest.raises(F.FlintError) as e:
             F.flint_moe_decode(bad, fake, 1, fake + 4096, fake, 1 << 20, stream=0)
         assert e.value.code == F.FLINT_EINVAL
     nb = F.flint_workspace_bytes(F.FLINT_OP_PREFILL, 16)
-    for offs in ([fake, fake, None, fake], [fake, fake, fake, fake + 8]):
-        aff = F.flint_moe_layer(*([fake] * 10), 0, F.FLINT_FMT_AFFINE_INT4, *offs)
+    for fmt, offs in ((1, [fake, fake, None, fake]), (1, [fake, fake, fake, fake + 8]),
+                      (2, [None] * 4 + [fake] * 4)):
+        bad = F.flint_moe_layer(*([fake] * 10), 0, fmt, *offs)
         with pytest.raises(F.FlintError) as e:
-            F.flint_moe_prefill(aff, fake, 16, fake + (1 << 24), fake, nb, stream=0)
+            F.flint_moe_prefill(bad, fake, 16, fake + (1 << 24), fake, nb, stream=0)
         assert e.value.code == F.FLINT_EINVAL

@@ -6,9 +6,9 @@ memory, a failed check reported as FLINT_EDEVICE in the call's status word.
 On valid inputs the checks must neither fire nor change a result: every call
 here runs through both libraries on the same inputs and workspaces, and the
 debug library's outputs must equal the release library's bit for bit with the
-status word clear.  Decode (batch 1, 4 and the residual form), an expert
-shard, routing and prefill at 5, 300 and 2,048 tokens, both weight formats,
-and the head GEMV."""
+status word clear.  Decode (batch 1, 4 and the residual form; all three
+expert formats), an expert shard, routing and prefill at 5, 300 and 2,048
+tokens (symmetric and affine), and the head GEMV."""
 import numpy as np
 import pytest
 
@@ -25,7 +25,9 @@ def env():
     F.build(debug=True)
     sym = synth.layer_device(0, "cuda", host=synth.layer_host(0))
     aff = synth.to_device(synth.affine_layer_host(0), "cuda")
-    return {"sym": F.make_layer(sym), "aff": F.make_layer(aff), "keep": (sym, aff)}
+    nv = synth.nvfp4_layer_device(0, "cuda")
+    return {"sym": F.make_layer(sym), "aff": F.make_layer(aff), "nv": F.make_layer(nv),
+            "keep": (sym, aff, nv)}
 
 
 def both(run):
@@ -50,7 +52,7 @@ def decode(L, xbits):
     return host_bf16(out), idx.cpu().numpy()
 
 
-@pytest.mark.parametrize("fmt", ["sym", "aff"])
+@pytest.mark.parametrize("fmt", ["sym", "aff", "nv"])
 @pytest.mark.parametrize("seeds", [[0], [1, 2, 3, 4]])
 def test_debug_decode_bitwise(env, fmt, seeds):
     x = synth.decode_x(seeds)
