@@ -438,7 +438,7 @@ def main():
     # ---- the same stack with group-64 affine int4 experts (MLX int4 / Q4_1
     # layout) and with NVFP4 experts (weight-only, BF16 activations): 8 layers
     # of synthetic weights each (3.7 GB, larger than L2)
-    aff_pf = []
+    aff_pf, nv_pf = [], []
     if not args.no_affine:
         naff = 8
         for fmt_name, make in (("affine", synth.affine_layer_device),
@@ -472,6 +472,8 @@ def main():
                 del ga, gwa
             if fmt_name == "affine":
                 aff_pf = fmt_structs[:3]  # prefill on affine experts rotates over three of them
+            else:
+                nv_pf = fmt_structs[:3]
             del fmt_structs, fmt_arr
 
     # ---- e2e through the C ABI with host buffers: H2D of the step's rows,
@@ -586,14 +588,16 @@ def main():
                                       "gemm1_TFLOPs": g1_tf, "gemm1_frac": g1_tf / peak_tf,
                                       "gemm2_TFLOPs": g2_tf, "gemm2_frac": g2_tf / peak_tf,
                                       "grouped_gemms_frac": gg_tf / peak_tf}
-            if aff_pf:  # the same call on group-64 affine experts
+            for fmt_name, fmt_layers in (("affine", aff_pf), ("nvfp4", nv_pf)):
+                if not fmt_layers:  # the same call on group-64 affine / NVFP4 experts
+                    continue
                 us_a = rotating_us([lambda l=l: F.flint_moe_prefill(l, xt, T, out_t, wsp, nbp,
                                                                     stream=stream)
-                                    for l in aff_pf], iters=8, skip=2, spin_cycles=2_000_000)
+                                    for l in fmt_layers], iters=8, skip=2, spin_cycles=2_000_000)
                 tf_a = T * PREFILL_FLOP_PER_TOKEN / (us_a * 1e-6) / 1e12
-                extra[f"prefill_affine_T{T}"] = {"us": us_a, "tokens_per_s": T / (us_a * 1e-6),
-                                                 "TFLOPs": tf_a, "tensor_frac": tf_a / peak_tf,
-                                                 "peak_kind": peak_kind_tf}
+                extra[f"prefill_{fmt_name}_T{T}"] = {"us": us_a, "tokens_per_s": T / (us_a * 1e-6),
+                                                     "TFLOPs": tf_a, "tensor_frac": tf_a / peak_tf,
+                                                     "peak_kind": peak_kind_tf}
             del wsp, out_t, xt
     sampler.stop()
 

@@ -130,9 +130,8 @@ typedef struct {
    * sh13_g [2] (gate, up), sh2_g [1]; weight = e2m1(code) * e4m3(scale) *
    * global.  The *_g pointers are read only for format 2 (4-byte aligned
    * there).
-   * Decode, route, the stack and expert-parallel calls take every format
-   * (formats 1 and 2 decode up to FLINT_MAX_DECODE_B_AFFINE rows); prefill
-   * takes formats 0 and 1 (FLINT_EINVAL for format 2). */
+   * Every call takes every format (formats 1 and 2 decode up to
+   * FLINT_MAX_DECODE_B_AFFINE rows). */
   int format;
   const uint16_t *w13_m;
   const uint16_t *w2_m;
@@ -304,7 +303,9 @@ FLINT_API int flint_moe_decode_stack(const flint_moe_layer *layers, int L, float
  * fp16 after a per-token power-of-two shift from a bound it cannot exceed.
  * Group-64 affine experts (format 1): each weight code x scale + offset
  * (times the matrix's power of two) is rounded once to fp16, a relative
- * error of at most 2^-11 per weight; the rest is as above.
+ * error of at most 2^-11 per weight; the rest is as above.  NVFP4 experts
+ * (format 2): each E2M1 value times its E4M3 block scale is an exact fp16
+ * weight (no shift); the global scales multiply the GEMMs' read-out.
  *   x bf16 [T][2048];  out bf16 [T][2048] (may not alias x);  1 <= T <= 2^20
  *   ws workspace of flint_workspace_bytes(FLINT_OP_PREFILL, T) (about 67 KB
  *      per token, 70 KB up to T = 4,608 where the router keeps two fp64

@@ -260,7 +260,7 @@ int flint_int4_gemv_nvfp4(const uint8_t *q, const uint8_t *s, float global_scale
 
 int flint_moe_prefill(const flint_moe_layer *layer, const uint16_t *x, int T, uint16_t *out,
                       void *ws, size_t ws_bytes, void *stream) {
-  if (!layer_ok(layer) || layer->format == FLINT_FMT_NVFP4 || !aligned16(x) ||
+  if (!layer_ok(layer) || !aligned16(x) ||
       !aligned16(out) || T < 1 || T > FLINT_MAX_PREFILL_T || !aligned16(ws) ||
       ws_bytes < flint_workspace_bytes(FLINT_OP_PREFILL, T) ||
       static_cast<const void *>(x) == static_cast<const void *>(out))

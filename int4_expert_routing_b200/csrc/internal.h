@@ -51,7 +51,7 @@ constexpr int kPfN2 = 256;
 constexpr int kPfChunk = 256;
 struct PrefillLayout {
   size_t ctrl, z, sel_idx, sel_w, asc_e, asc_w, route_total;
-  size_t pos, chunk_cnt, chunk_off, ebase, ecount, tiles1, tiles2, wst, wbound,
+  size_t pos, chunk_cnt, chunk_off, ebase, ecount, tiles1, tiles2, wst, wsg, wbound,
       rsc, rm3, xp, hr, hs, yw, ys, total;
   int mr, max_tiles1, max_tiles2, nchunks;
 };
@@ -92,6 +92,7 @@ inline PrefillLayout prefill_layout(int T) {
   L.tiles1 = take(sizeof(uint32_t) * 2 * (size_t)L.max_tiles1);  // tile descriptors (2 words)
   L.tiles2 = take(sizeof(uint32_t) * 2 * (size_t)L.max_tiles2);
   L.wst = take(sizeof(float) * 4 * 257);   // per expert matrix pair: power-of-two shifts
+  L.wsg = take(sizeof(float) * 4 * 257);   // per expert: NVFP4 global scales gate, up, down
   L.wbound = take(sizeof(float) * 257);    // per expert: bound factor of the SwiGLU output
   L.rsc = take(sizeof(uint32_t) * (size_t)7 * T);    // per row: F | E << 16
   L.rm3 = take(sizeof(float) * (size_t)7 * T);       // per row: 2^E x routing weight

@@ -444,6 +444,79 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// NVFP4 experts (E2M1 codes, an E4M3 scale per 16 elements, fp32 global
+// scales; "How to Run Flint Locally", section "What vLLM changed"): an E2M1
+// value times an E4M3 scale is an fp16 value (at most 6 significant bits, in
+// [2^-10, 2,688]), so the GEMMs take the weights unshifted (S = 0) and the
+// global scales multiply the epilogues' read-out: wsg[e] = (gate, up times
+// the stored divisor of a routed expert's up rows, down).  A row's norm is at
+// most 6 |g| sqrt(16 sum_b s_b^2) over its blocks b.
+FLINT_DEV float e4m3_to_f32(uint32_t b) {
+  uint32_t h;
+  asm("{ .reg .b16 t; cvt.u16.u32 t, %1; cvt.rn.f16x2.e4m3x2 %0, t; }" : "=r"(h) : "r"(b));
+  return __half2float(__ushort_as_half((unsigned short)(h & 0xffffu)));
+}
+
+__global__ void __launch_bounds__(256)
+    k_pf_wstats_nv(const uint8_t *__restrict__ w13_s, const float *__restrict__ w13_g,
+                   const float *__restrict__ w2_g, const uint8_t *__restrict__ sh13_s,
+                   const float *__restrict__ sh13_g, const float *__restrict__ sh2_g,
+                   float up_mul, float4 *__restrict__ wst, float4 *__restrict__ wsg,
+                   float *__restrict__ wbound) {
+  pdl_trigger();  // weights only before the wait, as in k_pf_wstats
+  __shared__ float red[2][8];
+  const int e = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool sh = e == kE;
+  constexpr int rb = kH / 16;  // scale bytes per gate/up row: 8 uint4
+  const int r13 = sh ? 2 * kIs : 2 * kI;
+  const uint8_t *s13 = sh ? sh13_s : w13_s + (size_t)e * r13 * rb;
+  float bg = 0.f, bu = 0.f;
+#pragma unroll 2
+  for (int r = tid; r < r13; r += 256) {
+    const uint4 *ps = reinterpret_cast<const uint4 *>(s13 + (size_t)r * rb);
+    uint4 sv[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) sv[i] = __ldg(ps + i);
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t a[4] = {sv[i].x, sv[i].y, sv[i].z, sv[i].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float v = e4m3_to_f32((a[q] >> (8 * k)) & 0xffu);
+          ss = fmaf(v, v, ss);
+        }
+    }
+    const float rn = 24.f * sqrtf(ss);  // 6 sqrt(16 ss), times |g| below
+    if (r < r13 / 2) bg = fmaxf(bg, rn);
+    else bu = fmaxf(bu, rn);
+  }
+  pdl_wait();  // the previous kernel in the stream is complete before any write
+  float v[2] = {bg, bu};
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v[k] = fmaxf(v[k], __shfl_xor_sync(0xffffffffu, v[k], o));
+    if (lane == 0) red[k][warp] = v[k];
+  }
+  __syncthreads();
+  if (tid == 0) {
+    float m[2];
+    for (int k = 0; k < 2; ++k) {
+      m[k] = red[k][0];
+      for (int w = 1; w < 8; ++w) m[k] = fmaxf(m[k], red[k][w]);
+    }
+    const float gg = sh ? __ldg(sh13_g) : __ldg(w13_g + 2 * e);
+    const float gu = (sh ? __ldg(sh13_g + 1) : __ldg(w13_g + 2 * e + 1)) * (sh ? 1.f : up_mul);
+    const float gd = sh ? __ldg(sh2_g) : __ldg(w2_g + e);
+    wst[e] = make_float4(1.f, 1.f, 1.f, 1.f);
+    wsg[e] = make_float4(gg, gu, gd, 0.f);
+    wbound[e] = (m[0] * fabsf(gg)) * (m[1] * fabsf(gu)) * (1.f + 1.f / 1024);
+  }
+}
+
 // Token rows as the fp16 operand of GEMM 1: rows [0, 6T) are the routed rows
 // in sorted order, rows [6T, 7T) every token for the shared expert.  One warp
 // per token (grid-stride) reads the row once and takes its shifts: F puts
@@ -605,6 +678,7 @@ struct GemmArgs {
   const uint16_t *mo_r;  // affine: offsets of the routed weight tensor
   const uint16_t *mo_s;  // affine: offsets of the shared expert's tensor
   const float4 *wst;     // per expert: 2^-S1, 2^S1, 2^-S2, 2^S2
+  const float4 *wsg;     // per expert, NVFP4: global scales of gate, up, down
   const uint32_t *rsc;   // per row: F | E << 16 (int16 each): multipliers 2^F, 2^-E
   const float *rm3;      // per row: 2^E x routing weight
   uint16_t *out_r;       // GEMM 1: Hr fp16 [6T][512]; GEMM 2: Yw bf16 [6T][2048]
@@ -771,6 +845,37 @@ FLINT_DEV void codes8_f16(uint32_t w, uint32_t m24, uint32_t m20, uint32_t c8, u
   asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(out[3]) : "r"(t3), "r"(m20), "r"(c8));
 }
 
+// One E4M3 byte -> fp16 pair (both halves the value; exact: E4M3 has 4
+// significant bits and lies in [2^-9, 448]).
+FLINT_DEV uint32_t e4m3x2_dup(uint32_t b) {
+  uint32_t h;
+  asm("{ .reg .b16 t; cvt.u16.u32 t, %1; cvt.rn.f16x2.e4m3x2 %0, t; }" : "=r"(h) : "r"(b | (b << 8)));
+  return h;
+}
+// 8 E2M1 codes (one word, code k in bits 4k..4k+3, the lower nibble the even
+// element) times a block scale s (fp16 pair): fp16 pairs (k, k+4) for k =
+// 0..3 (the order of codes8_f16), exact.  Masks and a shift-or put the pairs'
+// nibbles into bytes: (n0 | n4 << 4, n2 | n6 << 4) and (n1 | n5 << 4, n3 |
+// n7 << 4); the hardware converts each byte to an fp16 pair.
+FLINT_DEV void e2m1x8_f16_scaled(uint32_t w, uint32_t s, uint32_t *out) {
+  const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+  const uint32_t X = lo | (lo >> 12), Y = hi | (hi >> 12);
+  uint32_t h0, h1, h2, h3;
+  asm("{ .reg .b8 x0, x1, x2, x3, y0, y1, y2, y3;\n"
+      "mov.b32 {x0, x1, x2, x3}, %4;\n"
+      "mov.b32 {y0, y1, y2, y3}, %5;\n"
+      "cvt.rn.f16x2.e2m1x2 %0, x0;\n"
+      "cvt.rn.f16x2.e2m1x2 %1, y0;\n"
+      "cvt.rn.f16x2.e2m1x2 %2, x1;\n"
+      "cvt.rn.f16x2.e2m1x2 %3, y1; }"
+      : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
+      : "r"(X), "r"(Y));
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(out[0]) : "r"(h0), "r"(s));
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(out[1]) : "r"(h1), "r"(s));
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(out[2]) : "r"(h2), "r"(s));
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(out[3]) : "r"(h3), "r"(s));
+}
+
 // 16-bit global store, skipped when `pred` is false (no branch)
 FLINT_DEV void st_u16_if(uint16_t *p, uint32_t v, bool pred) {
   asm volatile("{ .reg .pred q; setp.ne.b32 q, %2, 0; @q st.global.b16 [%0], %1; }" ::"l"(p),
@@ -833,13 +938,14 @@ FLINT_DEV uint2 tile_word(const GemmArgs &args, uint32_t ti, uint32_t ntiles) {
 // carry on across tiles and one tile's epilogue overlaps the next tile's MMAs.
 // Barriers that gather both CTAs (full, afull, accempty) live in the first
 // CTA; the MMA commits arrive on both CTAs' copies of empty, aempty, accfull.
-template <int kMode, bool kAff>
+template <int kMode, int kFmt>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     k_pf_gemm(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
               const __grid_constant__ CUtensorMap tmB_r, const __grid_constant__ CUtensorMap tmB_s,
               GemmArgs args) {
   pdl_wait();  // the previous kernel in the stream is complete (programmatic launch)
   pdl_trigger();
+  constexpr bool kAff = kFmt == 1, kNv = kFmt == 2;  // FLINT_FMT_*
   using Cfg = GemmCfg<kMode>;
   constexpr int S = Cfg::kS, R = Cfg::kR, NA = Cfg::kNA, NACC = Cfg::kAcc, kN = Cfg::kN;
   constexpr int KS = Cfg::kKS;
@@ -1010,6 +1116,89 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       umma_commit_pair(&mma_done);
       if (!cwait_sleep(&mma_done, 0)) s_fail = 1;
     }  // other lanes and warp 3: idle (register donors)
+  } else if (warp < 8 && kNv) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegDeq));
+    // ---- dequant, NVFP4 weights: each code pair's byte through the hardware
+    // E2M1 conversion (an exact fp16 pair) times its 16-element block's E4M3
+    // scale (an exact fp16 product: at most 6 significant bits, in [2^-10,
+    // 2,688]); no shift (S = 0), the global scales in the epilogue.  A stage
+    // (two 128-groups, 16 blocks) takes 16 scale bytes of the row, one uint4:
+    // a tile's first stage loaded during the previous tile, the others from L1.
+    static_assert(KS == 2, "a stage's 16 blocks are one uint4 of E4M3 scales");
+    const int i = tid - 128, q = warp - 4;
+    const int raw_row = kMode == 1 ? ((i & 1) ? 64 + (i >> 1) : (i >> 1)) : i;
+    auto row_of = [&](const PfTile &tn) {  // this thread's row of scale bytes, as uint4
+      const int wrow = kMode == 1 ? ((i & 1) ? tn.row1 : tn.row0) + (i >> 1) : tn.row0 + i;
+      return reinterpret_cast<const uint4 *>(
+          reinterpret_cast<const uint8_t *>(tn.sh ? args.sc_s : args.sc_r) +
+          (size_t)wrow * (8 * (size_t)tn.ng));  // 8 blocks of 16 per 128-group
+    };
+    auto fetch = [&](uint2 w, uint4 &s0) {  // a tile's first stage
+      PfTile tn;
+      if (!pf_tile<kMode>(args, w, rank, tn)) return;
+      s0 = __ldg(row_of(tn));
+    };
+    uint2 wa = tile_word(args, pair, ntiles), wb = tile_word(args, pair + npairs, ntiles);
+    uint4 ns = make_uint4(0u, 0u, 0u, 0u);
+    fetch(wa, ns);
+    uint32_t it = 0;
+    for (uint32_t ti = pair; ti < ntiles && !s_fail; ti += npairs) {
+      const uint2 w = wa;
+      wa = wb;
+      wb = tile_word(args, ti + 2 * npairs, ntiles);
+      PfTile t;
+      const bool valid = pf_tile<kMode>(args, w, rank, t);
+      uint4 cs = ns;
+      fetch(wa, ns);  // the next tile's, in flight during this one
+      if (!valid) continue;
+      const uint4 *ps = row_of(t);
+      for (int c = 0; c < t.ng / 2; c += 8) asm volatile("prefetch.global.L1 [%0];" ::"l"(ps + c));
+      bool ok = true;
+      for (int G0 = 0; G0 < t.ng; G0 += KS, ++it) {
+        if (G0 > 0) cs = __ldg(ps + G0 / 2);
+        const int rr = it % R, a = it % NA;
+        if (!mbar_wait_sleep(&rfull[rr], (it / R) & 1) ||
+            (it >= (uint32_t)NA && !cwait_sleep(&aempty[a], ((it / NA) - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sw[4] = {cs.x, cs.y, cs.z, cs.w};  // blocks 0..15 of the stage, a byte each
+#pragma unroll
+        for (int g = 0; g < KS; ++g) {  // group G0 + g -> TMEM columns 64 g .. of the tile
+          const unsigned char *raw = sm + Cfg::raw_off(rr) + g * kRawBytes + raw_row * 64;
+          const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + Cfg::a_col(a) + 64u * g;
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {  // columns 32 hf ..: chunks 2 hf, 2 hf + 1
+            uint32_t v[32];
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+              const int j = 2 * hf + jj;  // chunk j: blocks 8 g + 2 j, 8 g + 2 j + 1
+              const uint4 wv = *reinterpret_cast<const uint4 *>(raw + 16 * (j ^ ((raw_row >> 1) & 3)));
+              const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
+              const int b0 = 8 * g + 2 * j;
+              const uint32_t sA = e4m3x2_dup((sw[b0 >> 2] >> (8 * (b0 & 3))) & 0xffu);
+              const uint32_t sB = e4m3x2_dup((sw[(b0 + 1) >> 2] >> (8 * ((b0 + 1) & 3))) & 0xffu);
+#pragma unroll
+              for (int wi = 0; wi < 4; ++wi)
+                e2m1x8_f16_scaled(words[wi], wi < 2 ? sA : sB, v + 16 * jj + 4 * wi);
+            }
+            tmem_st32(tbase + 32u * hf, v);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&rempty[rr]);  // the codes are in registers and TMEM
+          mbar_arrive_cluster(afull_cl + 8u * a);
+        }
+      }
+      if (!ok) {
+        s_fail = 1;
+        break;
+      }
+    }
   } else if (warp < 8 && kAff) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegDeq));
     // ---- dequant, group-64 affine weights: as below, but every 64 codes have
@@ -1230,6 +1419,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       if (!pf_tile<kMode>(args, w, rank, t)) continue;
       const int b = tc % NACC;
       const float4 ws = __ldg(args.wst + t.e);
+      const float4 gsc = kNv ? __ldg(args.wsg + t.e) : make_float4(1.f, 1.f, 1.f, 1.f);
       uint32_t pre = 0u;
       if (et < t.n_valid)
         pre = kMode == 1 ? __ldg(args.rsc + t.b_row + et)
@@ -1283,7 +1473,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 __shfl_xor_sync(0xffffffffu, __uint_as_float(up_lane ? acc[jj] : acc[kQ + jj]), 1);
             const uint32_t fe = s_mul[c_lo + j0 + jj];  // F | E << 16
             const float m = mw * exp2i((int)(int16_t)(fe & 0xffffu));
-            const float g = (up_lane ? theirs : mine) * m, uu = (up_lane ? mine : theirs) * m;
+            // (NVFP4: times the gate's and the up rows' global scales)
+            const float g = (up_lane ? theirs : mine) * (kNv ? m * gsc.x : m);
+            const float uu = (up_lane ? mine : theirs) * (kNv ? m * gsc.y : m);
             const float h = __fdividef(g, 1.f + __expf(-g)) * uu *
                             exp2i(-(int)(int16_t)(fe >> 16));  // silu(gate) * up / 2^E
             const uint32_t hv = __half_as_ushort(__float2half_rn(h));
@@ -1302,7 +1494,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                             : args.out_r + (size_t)t.b_row * kH + col;
 #pragma unroll
         for (int j = 0; j < kHalf; ++j) {
-          const float m = mw * __uint_as_float(s_mul[c_lo + j]);
+          const float m = mw * __uint_as_float(s_mul[c_lo + j]) * (kNv ? gsc.z : 1.f);
           st_u16_if(yb + (size_t)(c_lo + j) * kH, f32_to_bf16_bits(__uint_as_float(acc[j]) * m), j < nv);
         }
       }
@@ -1652,34 +1844,34 @@ cudaError_t prefill_stage_times(float *ms, int n) {
 }
 
 // The two grouped GEMMs of a prefill call, for the experts' weight format
-// (symmetric int4 with bf16 scales, or group-64 affine with fp16 scales and
-// offsets): persistent, as many CTA pairs as fit at once (the tile counts are
+// (FLINT_FMT_*: symmetric int4 with bf16 scales, group-64 affine with fp16
+// scales and offsets, or NVFP4): persistent, as many CTA pairs as fit at once (the tile counts are
 // on the device).  Stage event 4 falls between them.
-template <bool kAff>
+template <int kFmt>
 cudaError_t launch_gemms(const PrefillLayout &P, const CUtensorMap &mA1r, const CUtensorMap &mA1s,
                          const CUtensorMap &mB1, const CUtensorMap &mA2r, const CUtensorMap &mA2s,
                          const CUtensorMap &mB2r, const CUtensorMap &mB2s, const GemmArgs &a1,
                          const GemmArgs &a2, cudaStream_t st) {
   cudaError_t e;
   note_step("prefill GEMM attributes");
-  if ((e = cudaFuncSetAttribute(k_pf_gemm<1, kAff>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if ((e = cudaFuncSetAttribute(k_pf_gemm<1, kFmt>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)GemmCfg<1>::kSmem)) != cudaSuccess ||
-      (e = cudaFuncSetAttribute(k_pf_gemm<2, kAff>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      (e = cudaFuncSetAttribute(k_pf_gemm<2, kFmt>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)GemmCfg<2>::kSmem)) != cudaSuccess)
     return e;
   int pairs1 = 0, pairs2 = 0;
-  if ((e = max_pairs(reinterpret_cast<const void *>(k_pf_gemm<1, kAff>), GemmCfg<1>::kSmem,
+  if ((e = max_pairs(reinterpret_cast<const void *>(k_pf_gemm<1, kFmt>), GemmCfg<1>::kSmem,
                      &pairs1)) ||
-      (e = max_pairs(reinterpret_cast<const void *>(k_pf_gemm<2, kAff>), GemmCfg<2>::kSmem,
+      (e = max_pairs(reinterpret_cast<const void *>(k_pf_gemm<2, kFmt>), GemmCfg<2>::kSmem,
                      &pairs2)))
     return e;
   note_step("prefill GEMM 1 launch");
-  e = pf_launch(k_pf_gemm<1, kAff>, 2 * min(P.max_tiles1, pairs1), kGemmThreads, GemmCfg<1>::kSmem,
+  e = pf_launch(k_pf_gemm<1, kFmt>, 2 * min(P.max_tiles1, pairs1), kGemmThreads, GemmCfg<1>::kSmem,
                 st, mA1r, mA1s, mB1, mB1, a1);
   if (e != cudaSuccess) return e;
   stage_mark(4, st);
   note_step("prefill GEMM 2 launch");
-  return pf_launch(k_pf_gemm<2, kAff>, 2 * min(P.max_tiles2, pairs2), kGemmThreads,
+  return pf_launch(k_pf_gemm<2, kFmt>, 2 * min(P.max_tiles2, pairs2), kGemmThreads,
                    GemmCfg<2>::kSmem, st, mA2r, mA2s, mB2r, mB2s, a2);
 }
 
@@ -1755,12 +1947,19 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
   stage_mark(2, st);
   // 3. power-of-two shifts of the fp16 operands, and the fp16 token rows
   note_step("prefill operand scaling launches");
-  const bool aff = L.fmt == FLINT_FMT_AFFINE_INT4;
-  if ((e = aff ? pf_launch(k_pf_wstats_aff, kE + 1, 256, 0, st, L.w13_s, L.w13_m, L.w2_s, L.w2_m,
-                           L.sh13_s, L.sh13_m, L.sh2_s, L.sh2_m, L.interm_div, wst, wbound)
-               : pf_launch(k_pf_wstats, kE + 1, 256, 0, st, L.w13_s, L.w2_s, L.sh13_s, L.sh2_s,
-                           L.interm_div, wst, wbound)))
-    return e;
+  const int fmt = L.fmt;
+  float4 *wsg = reinterpret_cast<float4 *>(ws + P.wsg);
+  if (fmt == FLINT_FMT_AFFINE_INT4)
+    e = pf_launch(k_pf_wstats_aff, kE + 1, 256, 0, st, L.w13_s, L.w13_m, L.w2_s, L.w2_m, L.sh13_s,
+                  L.sh13_m, L.sh2_s, L.sh2_m, L.interm_div, wst, wbound);
+  else if (fmt == FLINT_FMT_NVFP4)
+    e = pf_launch(k_pf_wstats_nv, kE + 1, 256, 0, st, reinterpret_cast<const uint8_t *>(L.w13_s),
+                  L.w13_g, L.w2_g, reinterpret_cast<const uint8_t *>(L.sh13_s), L.sh13_g, L.sh2_g,
+                  L.interm_div, wst, wsg, wbound);
+  else
+    e = pf_launch(k_pf_wstats, kE + 1, 256, 0, st, L.w13_s, L.w2_s, L.sh13_s, L.sh2_s,
+                  L.interm_div, wst, wbound);
+  if (e) return e;
   {
     int blocks = (T + 7) / 8;  // 8 tokens (warps) per block
     if (blocks > 148 * 8) blocks = 148 * 8;
@@ -1786,12 +1985,18 @@ cudaError_t launch_prefill(const LayerArgs &L, const uint16_t *x, int T, uint16_
       (e = make_map(&mB2r, hr, F16, kI, (uint64_t)P.mr, kI * 2, 64, GemmCfg<2>::kBRows, SW)) ||
       (e = make_map(&mB2s, hs, F16, kIs, (uint64_t)T, kIs * 2, 64, GemmCfg<2>::kBRows, SW)))
     return e;
+  // (NVFP4: the routed up rows' divisor is in the up global scale, not the weights)
+  const float up_mul = fmt == FLINT_FMT_NVFP4 ? 1.f : L.interm_div;
   GemmArgs a1{tiles1, ctrl, 3,   ebase, ecount,   T,   L.w13_s, L.sh13_s, L.w13_m,
-              L.sh13_m, wst, rsc, rm3, hr,     hs, ctrl + 1, L.interm_div};
+              L.sh13_m, wst, wsg, rsc, rm3, hr,     hs, ctrl + 1, up_mul};
   GemmArgs a2{tiles2, ctrl, 4,   ebase, ecount,   T,   L.w2_s, L.sh2_s, L.w2_m,
-              L.sh2_m, wst, rsc, rm3, yw,     ys, ctrl + 1, 1.f};
-  e = aff ? launch_gemms<true>(P, mA1r, mA1s, mB1, mA2r, mA2s, mB2r, mB2s, a1, a2, st)
-          : launch_gemms<false>(P, mA1r, mA1s, mB1, mA2r, mA2s, mB2r, mB2s, a1, a2, st);
+              L.sh2_m, wst, wsg, rsc, rm3, yw,     ys, ctrl + 1, 1.f};
+  if (fmt == FLINT_FMT_AFFINE_INT4)
+    e = launch_gemms<FLINT_FMT_AFFINE_INT4>(P, mA1r, mA1s, mB1, mA2r, mA2s, mB2r, mB2s, a1, a2, st);
+  else if (fmt == FLINT_FMT_NVFP4)
+    e = launch_gemms<FLINT_FMT_NVFP4>(P, mA1r, mA1s, mB1, mA2r, mA2s, mB2r, mB2s, a1, a2, st);
+  else
+    e = launch_gemms<FLINT_FMT_SYM_INT4>(P, mA1r, mA1s, mB1, mA2r, mA2s, mB2r, mB2s, a1, a2, st);
   if (e != cudaSuccess) return e;
   stage_mark(5, st);
   // 5. combine

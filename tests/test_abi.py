@@ -92,8 +92,7 @@ def test_bad_arguments_rejected_before_launch(lib):
 def test_weight_format_rejected_before_launch(lib):
     """An unknown expert format, an affine layer without its offsets (or
     with a misaligned one) and an NVFP4 layer without its global scales (or
-    with a misaligned one) are refused on the host, by decode and prefill; an
-    NVFP4 layer is refused by prefill."""
+    with a misaligned one) are refused on the host, by decode and prefill."""
     fake = 1 << 20
     for fmt, offs in ((3, [fake] * 8), (-1, [fake] * 8), (1, [None] * 8),
                       (1, [fake, fake + 2, fake, fake] + [None] * 4),
@@ -104,7 +103,8 @@ def test_weight_format_rejected_before_launch(lib):
         assert e.value.code == F.FLINT_EINVAL
     nb = F.flint_workspace_bytes(F.FLINT_OP_PREFILL, 16)
     for fmt, offs in ((1, [fake, fake, None, fake]), (1, [fake, fake, fake, fake + 8]),
-                      (2, [None] * 4 + [fake] * 4)):
+                      (2, [None] * 4 + [fake, None, fake, fake]),
+                      (2, [None] * 4 + [fake, fake, fake + 1, fake])):
         bad = F.flint_moe_layer(*([fake] * 10), 0, fmt, *offs)
         with pytest.raises(F.FlintError) as e:
             F.flint_moe_prefill(bad, fake, 16, fake + (1 << 24), fake, nb, stream=0)

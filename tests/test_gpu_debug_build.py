@@ -6,9 +6,9 @@ memory, a failed check reported as FLINT_EDEVICE in the call's status word.
 On valid inputs the checks must neither fire nor change a result: every call
 here runs through both libraries on the same inputs and workspaces, and the
 debug library's outputs must equal the release library's bit for bit with the
-status word clear.  Decode (batch 1, 4 and the residual form; all three
-expert formats), an expert shard, routing and prefill at 5, 300 and 2,048
-tokens (symmetric and affine), and the head GEMV."""
+status word clear.  Decode (batch 1, 4 and the residual form) and prefill
+(5, 300 and 2,048 tokens) in the three expert formats, an expert shard,
+routing, and the head GEMV."""
 import numpy as np
 import pytest
 
@@ -93,7 +93,8 @@ def prefill(L, xbits):
     return host_bf16(out), idx.cpu().numpy()
 
 
-@pytest.mark.parametrize("fmt,T", [("sym", 5), ("sym", 300), ("sym", 2048), ("aff", 300)])
+@pytest.mark.parametrize("fmt,T", [("sym", 5), ("sym", 300), ("sym", 2048), ("aff", 300),
+                                   ("nv", 300)])
 def test_debug_prefill_bitwise(env, fmt, T):
     x = synth.prefill_x(T, T)
     (o1, i1), (o2, i2) = both(lambda: prefill(env[fmt], x))

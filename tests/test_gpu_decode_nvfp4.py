@@ -136,19 +136,12 @@ def test_nvfp4_form_of_exactly_shared_weights_decodes_bitwise():
     assert np.array_equal(ia, ib) and np.array_equal(a, b)
 
 
-def test_nvfp4_batch_limit_and_prefill_refused(nv):
-    """NVFP4 layers decode up to FLINT_MAX_DECODE_B_AFFINE = 7 rows (8 is
-    refused before any launch); prefill reads formats 0 and 1 only."""
+def test_nvfp4_batch_limit(nv):
+    """NVFP4 layers decode up to FLINT_MAX_DECODE_B_AFFINE = 7 rows; 8 is
+    refused before any launch."""
     x = dev_bf16(synth.decode_x(list(range(8))))
     out = torch().empty((8, 2048), dtype=torch().int16, device="cuda")
     ws, nb = workspace(F.FLINT_OP_DECODE, 8)
     with pytest.raises(F.FlintError) as e:
         F.flint_moe_decode(nv["L"], x, 8, out, ws, nb)
-    assert e.value.code == F.FLINT_EINVAL
-    T = 16
-    xt = dev_bf16(synth.prefill_x(T, T))
-    outp = torch().empty((T, 2048), dtype=torch().int16, device="cuda")
-    wsp, nbp = workspace(F.FLINT_OP_PREFILL, T)
-    with pytest.raises(F.FlintError) as e:
-        F.flint_moe_prefill(nv["L"], xt, T, outp, wsp, nbp)
     assert e.value.code == F.FLINT_EINVAL
