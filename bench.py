@@ -35,12 +35,12 @@ N_LAYERS = synth.N_MOE_LAYERS
 H = synth.HIDDEN
 LAYER_FIXED_BYTES = 256 * 2048 * 2 + 256 * 4 + 2048 * (1024 + 32) + 2048 * (512 + 16)
 # DRAM bytes per decode layer over algorithmic bytes, from one ncu capture of
-# four stacked layers of this workload at batch 4 (110.69 MB read against
+# four stacked layers of this workload at batch 4 (110.67 MB read against
 # 109.89 MB algorithmic, caches flushed before every launch).  Traffic grows
 # with the expert count the same way, so a full layer's traffic is reported as
 # this ratio times its algorithmic bytes: a figure scaled from that capture,
 # not measured in this run.
-DECODE_TRAFFIC_RATIO = 110.687744 / 109.891584
+DECODE_TRAFFIC_RATIO = 110.672128 / 109.891584
 TIMING_REPEATS = 20
 HEAD_COPIES = 3  # copies of the head the head timing rotates over (3 x 158.6 MB > L2)
 EXPERT_BYTES = 1024 * (1024 + 32) + 2048 * (256 + 8)
