@@ -391,7 +391,8 @@ def nvfp4_layer_host(seed: int, dims: Dims = FLINT, with_codes: bool = True) -> 
     [rows, K/16] per matrix (w13_s [E, 2I, H/16], w2_s [E, H, I/16], sh13_s
     [2Is, H/16], sh2_s [H, Is/16]); fp32 global scales 2^-15 x U(0.75, 1.25)
     per expert matrix (w13_g [E, 2]: gate, up; w2_g [E]; sh13_g [2]; sh2_g
-    [1]).  Weights span about [-0.055, 0.055], rms about 0.011."""
+    [1]).  Weights span about [-0.055, 0.055], rms about 0.013 (E2M1 rms 2.93 x
+    E4M3 rms 148 x 2^-15)."""
     dims.check()
     E, H, I, Is = dims.n_experts, dims.hidden, dims.expert_i, dims.shared_i
     d = layer_host(seed, dims, with_codes=with_codes)

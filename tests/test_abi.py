@@ -49,6 +49,17 @@ def test_bounds_checked_build_exports_the_same_symbols():
     assert F.lib()._name == F.LIB_PATH  # the default library again
 
 
+def test_using_library_restores_the_default_after_an_error():
+    """An error raised inside the block still leaves the default library
+    selected afterwards."""
+    F.build(debug=True)
+    with pytest.raises(F.FlintError):
+        with F.using_library(F.DEBUG_LIB_PATH):
+            F.flint_moe_route(F.flint_moe_layer(), 1 << 20, 1, None, None, 1 << 20, 1 << 20,
+                              stream=0)
+    assert F.lib()._name == F.LIB_PATH
+
+
 def test_version_and_strerror(lib):
     assert F.version() >= 100
     assert "invalid" in F.strerror(F.FLINT_EINVAL)

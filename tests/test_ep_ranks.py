@@ -22,7 +22,7 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _rank_main(rank, world, port, out):
+def _rank_main(rank, world, port, out, fmt="sym"):
     import datetime
 
     import torch
@@ -36,7 +36,9 @@ def _rank_main(rank, world, port, out):
                             timeout=datetime.timedelta(seconds=60))
     try:
         dims = synth.Dims(hidden=128, n_experts=256, top_k=6, expert_i=128, shared_i=128)
-        L = oracle.Layer(synth.layer_host(3, dims))
+        make = {"sym": synth.layer_host, "affine": synth.affine_layer_host,
+                "nvfp4": synth.nvfp4_layer_host}[fmt]
+        L = oracle.Layer(make(3, dims))
         x = synth.bf16_bits(np.random.default_rng(4).normal(size=(3, 128)))
         lo, hi = ep.shard_range(rank, world)
         part = torch.from_numpy(oracle.moe_layer_partial(L, x, lo, hi, rank == 0))
@@ -48,12 +50,15 @@ def _rank_main(rank, world, port, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 4])
-def test_ranks_sum_their_shards_to_the_block(world):
+@pytest.mark.parametrize("world,fmt", [(2, "sym"), (4, "sym"), (2, "affine"), (3, "nvfp4")])
+def test_ranks_sum_their_shards_to_the_block(world, fmt):
+    """Each weight format: the shards' partials, all-reduced over gloo ranks,
+    are the block output."""
     port = _free_port()
     ctx = mp.get_context("spawn")
     out = ctx.Queue()
-    procs = [ctx.Process(target=_rank_main, args=(r, world, port, out)) for r in range(world)]
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, out, fmt))
+             for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:

@@ -63,3 +63,38 @@ def test_expert_slice_equals_full_array_slice():
     t = synth.layer_host(2, d)
     w13, w2 = synth.expert_codes_host(2, 1, d)
     assert np.array_equal(w13, t["w13_q"][1]) and np.array_equal(w2, t["w2_q"][1])
+
+
+def _e2m1(nib):
+    table = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6, 0, -0.5, -1, -1.5, -2, -3, -4, -6])
+    return table[nib]
+
+
+def test_affine_and_nvfp4_recipe_value_ranges():
+    """The other two formats' synthetic layers hold what their recipes state:
+    affine groups roughly centred on zero within the symmetric recipe's
+    largest weight (offset -7.5 scale x U(0.9, 1.1)),
+    NVFP4 weights within about +-0.055 with an rms near 0.013 (E4M3 block
+    scales 64 .. 240, global scales 2^-15 x U(0.75, 1.25))."""
+    d = synth.Dims(n_experts=4)
+    a = synth.affine_layer_host(1, d)
+    s = a["w13_s"].view(np.float16).astype(np.float64)
+    m = a["w13_m"].view(np.float16).astype(np.float64)
+    assert s.min() > 0.02 * 0.5 / 7.5 * 0.999 and s.max() < 0.02 * 1.5 / 7.5 * 1.001
+    assert np.all(m < 0) and np.all(-m / s > 7.5 * 0.9 * 0.999) and np.all(-m / s < 7.5 * 1.1 * 1.001)
+    lo, hi = m, m + 15 * s                      # a group's weights lie between these
+    mid = np.abs(0.5 * (lo + hi)).max()         # groups roughly centred on zero
+    sym_max = 8 * 0.02 * 1.5 / 7                # the symmetric recipe's largest |weight|
+    assert np.abs(lo).max() < sym_max and np.abs(hi).max() < sym_max and mid < 0.005
+    n = synth.nvfp4_layer_host(1, d)
+    sc = n["w13_s"].astype(np.int64)
+    assert set(np.unique(sc >> 3).tolist()) <= {13, 14}    # exponent fields, sign 0
+    g = n["w13_g"].astype(np.float64)
+    assert g.min() >= 2.0 ** -15 * 0.75 and g.max() <= 2.0 ** -15 * 1.25
+    q = n["w13_q"][0].astype(np.int64)
+    codes = np.stack([q & 15, q >> 4], axis=-1).reshape(q.shape[0], -1)
+    sv = torch.from_numpy(np.ascontiguousarray(n["w13_s"][0])).view(torch.float8_e4m3fn)
+    W = _e2m1(codes) * np.repeat(sv.to(torch.float64).numpy(), 16, axis=1)
+    W[:512] *= g[0, 0]
+    W[512:] *= g[0, 1]
+    assert np.abs(W).max() < 0.056 and 0.012 < np.sqrt((W ** 2).mean()) < 0.015
