@@ -15,7 +15,10 @@
  *  - The quantization format (symmetric int4, codes in [-8, 7], one bf16 scale
  *    per 128 consecutive elements along K) and the stack recipe (RMSNorm with
  *    eps 1e-6 and unit weight, residual add in fp32) are the workload's own
- *    definitions; the pages ship other 4-bit formats.
+ *    definitions; the pages ship other 4-bit formats, which the layer's
+ *    `format` also states: group-64 affine int4 ("How to Run Flint Locally",
+ *    section "Every build and its size") and NVFP4 weight-only (section "What
+ *    vLLM changed").
  *
  * Readings where the pages are silent: the bias is added to sigmoid(z) and is
  * used for selection only; the combine weights are the unbiased sigmoid
