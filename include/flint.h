@@ -213,7 +213,8 @@ FLINT_API int flint_moe_route(const flint_moe_layer *layer, const uint16_t *x, i
                     float *w, void *ws, size_t ws_bytes, void *stream);
 
 /*
- * Decode step of the MoE block for B in [1, 8] rows:
+ * Decode step of the MoE block for B in [1, 8] rows (B in [1, 7] for a layer in
+ * the affine or NVFP4 format, FLINT_MAX_DECODE_B_AFFINE):
  *   out[r] = sum_j w[r][j] * W2_e (silu(W1_e x) * (W3_e x))  (j over the 6
  *            chosen experts e, in ascending expert order)
  *          + W2_sh (silu(W1_sh x) * (W3_sh x))               (shared expert)
@@ -229,7 +230,8 @@ FLINT_API int flint_moe_decode(const flint_moe_layer *layer, const uint16_t *x, 
                      void *ws, size_t ws_bytes, void *stream);
 
 /*
- * One stacked decode layer on an fp32 residual stream h [B][2048], B in [1, 8]:
+ * One stacked decode layer on an fp32 residual stream h [B][2048], B in [1, 8]
+ * (B in [1, 7] for the affine and NVFP4 formats):
  *   x = bf16(h / sqrt(mean(h^2) + 1e-6))   (RMSNorm, unit weight, fp64 inside)
  *   h = h + bf16(moe(x))                   (residual add in fp32, in place)
  * Optional outputs (NULL to skip): idx int32 [B][6], w fp32 [B][6] in
