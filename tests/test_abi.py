@@ -49,6 +49,27 @@ def test_bounds_checked_build_exports_the_same_symbols():
     assert F.lib()._name == F.LIB_PATH  # the default library again
 
 
+def test_decode_batch_limit_per_format_before_launch(lib):
+    """B = 8 is refused for affine and NVFP4 layers (their down slots do not
+    fit 48 in K3's shared memory) by every decode call, before any launch;
+    the symmetric format's limit is 8, and B = 9 is refused for all."""
+    fake = 1 << 20
+    nb = F.flint_workspace_bytes(F.FLINT_OP_DECODE, 8)
+    for fmt in (F.FLINT_FMT_AFFINE_INT4, F.FLINT_FMT_NVFP4):
+        L = F.flint_moe_layer(*([fake] * 10), 0, fmt, *([fake] * 8))
+        for call in (lambda: F.flint_moe_decode(L, fake, 8, fake + 65536, fake, nb, stream=0),
+                     lambda: F.flint_moe_decode_residual(L, fake, 8, None, None, fake, nb,
+                                                         stream=0)):
+            with pytest.raises(F.FlintError) as e:
+                call()
+            assert e.value.code == F.FLINT_EINVAL
+    for fmt in (F.FLINT_FMT_SYM_INT4, F.FLINT_FMT_AFFINE_INT4, F.FLINT_FMT_NVFP4):
+        L = F.flint_moe_layer(*([fake] * 10), 0, fmt, *([fake] * 8))
+        with pytest.raises(F.FlintError) as e:
+            F.flint_moe_decode(L, fake, 9, fake + 65536, fake, 1 << 24, stream=0)
+        assert e.value.code == F.FLINT_EINVAL
+
+
 def test_using_library_restores_the_default_after_an_error():
     """An error raised inside the block still leaves the default library
     selected afterwards."""
