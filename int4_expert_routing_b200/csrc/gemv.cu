@@ -336,7 +336,7 @@ FLINT_DEV uint32_t hmul2(uint32_t a, uint32_t b) {
 // NVFP4 rows ra, rb: codes at row stride K/2 bytes, E4M3 block scales at row
 // stride K/16 bytes.  Lane t's 32 elements of a 128-block are two 16-element
 // scale blocks (2t, 2t+1); every code times its block scale is exact in fp16
-// (at most 5 significant bits, magnitudes 2^-10 .. 2,688), so the f16 MMAs
+// (at most 6 significant bits, magnitudes 2^-10 .. 2,688), so the f16 MMAs
 // accumulate the exact products of the weights and the f16 activations in
 // fp32, block after block, with no per-block step (the fragment holds x in
 // natural order: pair j = elements 2j, 2j+1 of the lane's slice).
